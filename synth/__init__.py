@@ -1,0 +1,94 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module only draws random numbers and lays them out in the canonical storage formats
+(GGUF Q8_0 / Q4_0 blocks, NVFP4 code and scale planes); it holds none of the layer's arithmetic.
+Rounding of drawn reals to fp16 / bf16 / E4M3 storage uses torch's own conversions
+(round-to-nearest-even).
+
+Canonical layouts (the public conventions; the pages name the formats but not their bytes):
+  Q8_0  one row = K/32 blocks of 34 bytes: fp16 scale d (little endian), then 32 int8 codes
+  Q4_0  one row = K/32 blocks of 18 bytes: fp16 scale d, then 16 bytes; byte j holds element j
+        in its low nibble and element j+16 in its high nibble
+  NVFP4 codes [N][K/2] (byte i = element 2i low nibble, 2i+1 high nibble), E4M3 scales [N][K/16],
+        one fp32 per-tensor scale
+
+Workload recipes (seeded; shapes from the synthetic layer stacks the bench and tests use):
+  Q8_0:  codes uniform over [-127, 127], scale uniform real in [1e-3, 1e-2] rounded to fp16
+  Q4_0:  4-bit codes uniform over 0..15 (value = code - 8), scale uniform real in [1e-3, 2e-2]
+  NVFP4: codes uniform over all 16, E4M3 scales uniform real in [0.5, 448] rounded to E4M3,
+         per-tensor scale fp32(1/448)
+  activations N(0, 1) (fp32, or fp32 draws rounded to bf16); router logits N(0, 1)
+"""
+from __future__ import annotations
+
+import torch
+
+Q8_0, Q4_0, NVFP4 = 1, 2, 3
+FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4"}
+NVFP4_G = float(torch.tensor(1.0 / 448.0, dtype=torch.float32))
+
+
+def gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def seed_for(config: int, layer: int = 0, tensor: int = 0) -> int:
+    """Per-tensor seed: config id * 1000 + layer * 10 + tensor index."""
+    return config * 1000 + layer * 10 + tensor
+
+
+def _fp16_bytes(vals: torch.Tensor) -> torch.Tensor:
+    return vals.to(torch.float16).contiguous().view(torch.uint8).reshape(*vals.shape, 2)
+
+
+def q8_0(N, K, g, device="cpu", d_range=(1e-3, 1e-2), q_range=(-127, 127)):
+    """Canonical Q8_0 tensor, uint8 [N, K/32*34]."""
+    assert K % 32 == 0
+    nb = K // 32
+    d = torch.empty(N, nb, dtype=torch.float32, device=device).uniform_(*d_range, generator=g)
+    q = torch.randint(q_range[0], q_range[1] + 1, (N, nb, 32), generator=g, device=device,
+                      dtype=torch.int16).to(torch.int8).view(torch.uint8)
+    return torch.cat([_fp16_bytes(d), q], dim=2).reshape(N, nb * 34).contiguous()
+
+
+def q4_0(N, K, g, device="cpu", d_range=(1e-3, 2e-2)):
+    """Canonical Q4_0 tensor, uint8 [N, K/32*18]."""
+    assert K % 32 == 0
+    nb = K // 32
+    d = torch.empty(N, nb, dtype=torch.float32, device=device).uniform_(*d_range, generator=g)
+    qs = torch.randint(0, 256, (N, nb, 16), generator=g, device=device,
+                       dtype=torch.int16).to(torch.uint8)
+    return torch.cat([_fp16_bytes(d), qs], dim=2).reshape(N, nb * 18).contiguous()
+
+
+def nvfp4(N, K, g, device="cpu", s_range=(0.5, 448.0)):
+    """Canonical NVFP4 tensor: (codes uint8 [N, K/2], scales uint8 [N, K/16], fp32 tensor scale)."""
+    assert K % 16 == 0
+    codes = torch.randint(0, 256, (N, K // 2), generator=g, device=device,
+                          dtype=torch.int16).to(torch.uint8)
+    s = torch.empty(N, K // 16, dtype=torch.float32, device=device).uniform_(*s_range, generator=g)
+    scales = s.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    return codes.contiguous(), scales, NVFP4_G
+
+
+def weights(fmt, N, K, g, device="cpu"):
+    """Canonical tensor of the given format: (blocks, scales or None, per-tensor scale)."""
+    if fmt == Q8_0:
+        return q8_0(N, K, g, device), None, 1.0
+    if fmt == Q4_0:
+        return q4_0(N, K, g, device), None, 1.0
+    if fmt == NVFP4:
+        return nvfp4(N, K, g, device)
+    raise ValueError(fmt)
+
+
+def activations(M, K, g, dtype=torch.float32, device="cpu"):
+    """N(0,1) activations; bf16 rows are fp32 draws rounded to bf16."""
+    x = torch.randn(M, K, generator=g, dtype=torch.float32, device=device)
+    return x.to(dtype).contiguous()
+
+
+def router_logits(M, E, g, device="cpu"):
+    return torch.randn(M, E, generator=g, dtype=torch.float32, device=device)

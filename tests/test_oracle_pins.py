@@ -1,0 +1,335 @@
+"""Pins of the fp64 oracle against what the formats and the mathematics fix (CPU only).
+
+Each check is chosen so that a plausible mistake in the oracle (a swapped nibble, a wrong
+exponent bias, a dropped term, a transposed operand, a wrong tie rule) fails one of them.  None of
+them re-derives a value through the oracle's own code path: the references are golden fixtures
+worked by hand from the format definitions, library routines (numpy float16, torch float8,
+torch silu, numpy argsort), exact rational arithmetic, and closed forms.
+"""
+import math
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from conftest import read_golden
+
+
+def f32_bits(v):
+    return struct.unpack("<I", struct.pack("<f", v))[0]
+
+
+# ----------------------------------------------------------------------------- scalar decoders
+def test_fp16_all_codes_match_numpy():
+    ref = np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.float16).astype(np.float64)
+    got = np.array([oracle.fp16(b) for b in range(65536)])
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert np.array_equal(np.signbit(ref[~nan]), np.signbit(got[~nan]))
+
+
+def test_e4m3_all_codes_match_torch():
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3(b) for b in range(256)])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2  # S.1111.111 only: the "fn" variant has no infinities
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert oracle.e4m3(0x7E) == 448.0 and oracle.e4m3(0x01) == 2.0 ** -9
+
+
+def test_e2m1_all_codes_match_golden():
+    rows = [l.split() for l in read_golden("e2m1_values.txt")]
+    assert len(rows) == 16
+    for code, val in rows:
+        c, v = int(code, 16), float(val)
+        got = oracle.e2m1(c)
+        assert got == v and math.copysign(1, got) == math.copysign(1, v), (c, got, v)
+
+
+# ----------------------------------------------------------------------------- block dequant
+def _golden_blocks(name):
+    lines = read_golden(name)
+    out = []
+    for i in range(0, len(lines), 2):
+        assert lines[i].startswith("bytes:") and lines[i + 1].startswith("values:")
+        b = bytes(int(t, 16) for t in lines[i].split()[1:])
+        v = [float(t) for t in lines[i + 1].split()[1:]]
+        out.append((b, v))
+    return out
+
+
+@pytest.mark.parametrize("fmt,name", [(oracle.Q8_0, "q8_0_block.txt"), (oracle.Q4_0, "q4_0_block.txt")])
+def test_gguf_block_dequant_matches_golden(fmt, name):
+    for b, v in _golden_blocks(name):
+        blocks = np.frombuffer(b, np.uint8)
+        w = oracle.dequant(fmt, 1, 32, blocks)[0]
+        assert list(w) == v
+        w32 = oracle.dequant_f32(fmt, 1, 32, blocks)[0]
+        assert np.array_equal(w32.astype(np.float64), np.array(v))
+
+
+def test_gguf_blocks_stack_along_k_and_rows():
+    # Two golden blocks side by side in one row, and the same row twice: block b of row n covers
+    # k in [32b, 32b+32); rows are independent.
+    (b0, v0), (b1, v1) = _golden_blocks("q4_0_block.txt")[:2]
+    row = np.frombuffer(b0 + b1, np.uint8)
+    W = oracle.dequant(oracle.Q4_0, 2, 64, np.concatenate([row, row[::-1][::-1]]))
+    assert list(W[0]) == v0 + v1 and list(W[1]) == v0 + v1
+
+
+def test_nvfp4_dequant_rounding_golden():
+    for line in read_golden("nvfp4_rounding.txt"):
+        code, sc, gb, wb = (int(t, 16) for t in line.split())
+        g = struct.unpack("<f", struct.pack("<I", gb))[0]
+        codes = np.zeros((1, 8), np.uint8)
+        codes[0, 0] = code  # element 0 is the low nibble of byte 0
+        codes[0, 7] = code << 4  # element 15 is the high nibble of byte 7
+        scales = np.array([[sc]], np.uint8)
+        w32 = oracle.dequant_f32(oracle.NVFP4, 1, 16, codes, scales, g)[0]
+        assert f32_bits(float(w32[0])) == wb, (hex(code), hex(f32_bits(float(w32[0]))), hex(wb))
+        assert f32_bits(float(w32[15])) == wb
+        assert all(f32_bits(float(t)) == 0 for t in w32[1:15])
+
+
+def test_nvfp4_scale_applies_per_16():
+    # Codes all 0x2 (1.0); scales 1.0, 2.0, 0.5 for k in [0,16), [16,32), [32,48).
+    codes = np.full((1, 24), 0x22, np.uint8)
+    scales = np.array([[0x38, 0x40, 0x30]], np.uint8)  # E4M3 1.0, 2.0, 0.5
+    w = oracle.dequant(oracle.NVFP4, 1, 48, codes, scales, 1.0)[0]
+    assert list(w) == [1.0] * 16 + [2.0] * 16 + [0.5] * 16
+
+
+# ----------------------------------------------------------------------------- GEMV
+def _identity_q8(K):
+    blk = np.zeros((K, K // 32, 34), np.uint8)
+    blk[:, :, 0:2] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    for n in range(K):
+        blk[n, n // 32, 2 + n % 32] = 1
+    return blk.reshape(K, -1)
+
+
+def _identity_q4(K):
+    blk = np.zeros((K, K // 32, 18), np.uint8)
+    blk[:, :, 0:2] = np.frombuffer(np.float16(1.0).tobytes(), np.uint8)
+    blk[:, :, 2:] = 0x88  # every nibble 8 -> 0
+    for n in range(K):
+        j = n % 32
+        if j < 16:
+            blk[n, n // 32, 2 + j] = (blk[n, n // 32, 2 + j] & 0xF0) | 9
+        else:
+            blk[n, n // 32, 2 + j - 16] = (blk[n, n // 32, 2 + j - 16] & 0x0F) | (9 << 4)
+    return blk.reshape(K, -1)
+
+
+def _identity_nvfp4(K):
+    codes = np.zeros((K, K // 2), np.uint8)
+    for n in range(K):
+        codes[n, n // 2] = 0x2 << (4 * (n & 1))
+    return codes, np.full((K, K // 16), 0x38, np.uint8)
+
+
+@pytest.mark.parametrize("fmt", [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4])
+def test_gemv_identity_gives_x(fmt):
+    K = 96
+    x = synth.activations(3, K, synth.gen(1)).double().numpy()
+    if fmt == oracle.Q8_0:
+        blocks, scales = _identity_q8(K), None
+    elif fmt == oracle.Q4_0:
+        blocks, scales = _identity_q4(K), None
+    else:
+        blocks, scales = _identity_nvfp4(K)
+    y, A = oracle.gemv(fmt, K, K, blocks, x, scales=scales, g=1.0)
+    assert np.array_equal(y, x)
+    assert np.array_equal(A, np.abs(x))
+
+
+@pytest.mark.parametrize("fmt", [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4])
+def test_gemv_one_hot_selects_a_column(fmt):
+    N, K = 40, 64  # N != K so a transposed operand cannot pass
+    blocks, scales, g = synth.weights(fmt, N, K, synth.gen(2))
+    blocks, scales = blocks.numpy(), None if scales is None else scales.numpy()
+    W = oracle.dequant(fmt, N, K, blocks, scales, g)
+    for k in (0, 17, 31, 32, 63):
+        x = np.zeros((1, K))
+        x[0, k] = 1.0
+        y, _ = oracle.gemv(fmt, N, K, blocks, x, scales=scales, g=g)
+        assert np.array_equal(y[0], W[:, k])
+
+
+@pytest.mark.parametrize("fmt", [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4])
+def test_gemv_matches_exact_rational_sum(fmt):
+    N, K, M = 5, 64, 3
+    blocks, scales, g = synth.weights(fmt, N, K, synth.gen(3))
+    blocks, scales = blocks.numpy(), None if scales is None else scales.numpy()
+    W = oracle.dequant(fmt, N, K, blocks, scales, g)
+    x = synth.activations(M, K, synth.gen(4)).double().numpy()
+    y, A = oracle.gemv(fmt, N, K, blocks, x, scales=scales, g=g)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(W[n, k]) * Fraction(x[m, k]) for k in range(K))
+            absum = sum(abs(Fraction(W[n, k]) * Fraction(x[m, k])) for k in range(K))
+            assert abs(Fraction(y[m, n]) - exact) <= Fraction(K * 2.0 ** -52) * absum
+            assert abs(Fraction(A[m, n]) - absum) <= Fraction(K * 2.0 ** -52) * absum
+
+
+def test_gemv_row_subset_matches_full():
+    N, K = 33, 128
+    blocks, _, _ = synth.weights(oracle.Q4_0, N, K, synth.gen(5))
+    x = synth.activations(2, K, synth.gen(6)).double().numpy()
+    y, A = oracle.gemv(oracle.Q4_0, N, K, blocks.numpy(), x)
+    rows = [32, 0, 7]
+    ys, As = oracle.gemv(oracle.Q4_0, N, K, blocks.numpy(), x, rows=rows)
+    assert np.array_equal(ys, y[:, rows]) and np.array_equal(As, A[:, rows])
+
+
+# ----------------------------------------------------------------------------- SiLU gate
+def test_silu_matches_torch_and_identities():
+    z = np.linspace(-30, 30, 601)
+    ref = torch.nn.functional.silu(torch.tensor(z, dtype=torch.float64)).numpy()
+    got = np.array([oracle.silu(t) for t in z])
+    assert np.allclose(got, ref, rtol=1e-15, atol=1e-300)
+    assert oracle.silu(0.0) == 0.0
+    for t in (0.3, 2.0, 7.5):  # silu(-z) = silu(z) - z
+        assert abs(oracle.silu(-t) - (oracle.silu(t) - t)) < 1e-15 * 10
+
+
+def test_silu_gate_uses_first_half_as_gate():
+    gu = np.array([[1.0, -2.0, 3.0, 5.0]])  # gate = [1, -2], up = [3, 5]
+    h, _ = oracle.silu_gate(gu)
+    sig = lambda t: 1.0 / (1.0 + math.exp(-t))
+    assert np.allclose(h[0], [1.0 * sig(1.0) * 3.0, -2.0 * sig(-2.0) * 5.0], rtol=1e-15)
+
+
+# ----------------------------------------------------------------------------- routing / MoE
+def test_route_matches_stable_sort_and_renormalises():
+    logits = synth.router_logits(8, 32, synth.gen(7)).double().numpy()
+    ids, wts = oracle.route(logits, 4)
+    p = torch.softmax(torch.tensor(logits), dim=1).numpy()
+    for m in range(8):
+        order = np.argsort(-p[m], kind="stable")[:4]
+        assert list(ids[m]) == list(order)
+        assert np.allclose(wts[m], p[m, order] / p[m, order].sum(), rtol=1e-14)
+        assert abs(wts[m].sum() - 1.0) < 1e-15 * 8
+
+
+def test_route_tie_goes_to_lower_expert():
+    ids, wts = oracle.route(np.zeros((1, 6)), 3)
+    assert list(ids[0]) == [0, 1, 2]
+    assert np.allclose(wts[0], 1.0 / 3.0)
+
+
+def _moe_case(fmt, E, H, I, seed):
+    gu = [synth.weights(fmt, 2 * I, H, synth.gen(seed + e)) for e in range(E)]
+    dn = [synth.weights(fmt, H, I, synth.gen(seed + 100 + e)) for e in range(E)]
+    cat = lambda ts, j: None if ts[0][j] is None else np.stack([t[j].numpy() for t in ts])
+    return (cat(gu, 0), cat(gu, 1), np.array([t[2] for t in gu], np.float32),
+            cat(dn, 0), cat(dn, 1), np.array([t[2] for t in dn], np.float32))
+
+
+def _mlp(fmt, H, I, gu_b, gu_s, gu_g, dn_b, dn_s, dn_g, x):
+    gu, _ = oracle.gemv(fmt, 2 * I, H, gu_b, x, scales=gu_s, g=gu_g)
+    h, _ = oracle.silu_gate(gu)
+    y, _ = oracle.gemv(fmt, H, I, dn_b, h, scales=dn_s, g=dn_g)
+    return y
+
+
+@pytest.mark.parametrize("fmt", [oracle.Q4_0, oracle.NVFP4])
+def test_moe_all_experts_uniform_logits_is_mean(fmt):
+    E, H, I = 4, 64, 32
+    gub, gus, gug, dnb, dns, dng = _moe_case(fmt, E, H, I, 10)
+    x = synth.activations(2, H, synth.gen(11)).double().numpy()
+    r = oracle.moe(fmt, E, H, I, E, gub, dnb, np.zeros((2, E)), x, gus, dns, gug, dng)
+    mean = sum(_mlp(fmt, H, I, gub[e], None if gus is None else gus[e], gug[e], dnb[e],
+                    None if dns is None else dns[e], dng[e], x) for e in range(E)) / E
+    assert np.allclose(r["y"], mean, rtol=1e-12, atol=1e-12)
+    assert np.allclose(r["wts"], 1.0 / E)
+
+
+def test_moe_top1_is_dense_mlp_of_argmax():
+    fmt, E, H, I = oracle.Q4_0, 5, 64, 32
+    gub, gus, gug, dnb, dns, dng = _moe_case(fmt, E, H, I, 20)
+    logits = synth.router_logits(3, E, synth.gen(21)).double().numpy()
+    x = synth.activations(3, H, synth.gen(22)).double().numpy()
+    r = oracle.moe(fmt, E, H, I, 1, gub, dnb, logits, x, gus, dns, gug, dng)
+    for m in range(3):
+        e = int(np.argmax(logits[m]))
+        ref = _mlp(fmt, H, I, gub[e], None, 1.0, dnb[e], None, 1.0, x[m:m + 1])
+        assert r["ids"][m, 0] == e and r["wts"][m, 0] == 1.0
+        assert np.array_equal(r["y"][m], ref[0])
+
+
+def test_moe_identical_experts_is_dense_and_permutation_invariant():
+    fmt, E, H, I = oracle.Q4_0, 6, 64, 32
+    gub, gus, gug, dnb, dns, dng = _moe_case(fmt, E, H, I, 30)
+    logits = synth.router_logits(2, E, synth.gen(31)).double().numpy()
+    x = synth.activations(2, H, synth.gen(32)).double().numpy()
+    same = oracle.moe(fmt, E, H, I, 3, np.stack([gub[0]] * E), np.stack([dnb[0]] * E), logits, x)
+    dense = _mlp(fmt, H, I, gub[0], None, 1.0, dnb[0], None, 1.0, x)
+    assert np.allclose(same["y"], dense, rtol=1e-12, atol=1e-12)
+    perm = np.array([3, 5, 0, 1, 4, 2])
+    a = oracle.moe(fmt, E, H, I, 3, gub, dnb, logits, x)
+    b = oracle.moe(fmt, E, H, I, 3, gub[perm], dnb[perm], logits[:, perm], x)
+    # the softmax denominator is summed in a different order, so equal up to fp64 rounding
+    assert np.allclose(a["y"], b["y"], rtol=1e-13, atol=1e-16)
+    assert np.array_equal(perm[b["ids"]], a["ids"])
+
+
+# ----------------------------------------------------------------------------- NVFP4 act quant
+def test_round_e2m1_golden_ties_and_nearest():
+    for line in read_golden("e2m1_ties.txt"):
+        v, c = line.split()
+        assert oracle.round_e2m1(float(v)) == int(c, 16), (v, c)
+    grid = [oracle.e2m1(c) for c in range(8)]
+    rng = np.random.default_rng(0)
+    for v in rng.uniform(-8, 8, 2000).astype(np.float32):
+        c = oracle.round_e2m1(float(v))
+        got = oracle.e2m1(c)
+        if abs(v) < 6:
+            assert all(abs(abs(v) - abs(got)) <= abs(abs(v) - t) for t in grid)
+        assert (c >> 3) == (1 if v < 0 else 0)
+    for c in range(16):  # every grid value round-trips
+        assert oracle.round_e2m1(oracle.e2m1(c)) == c
+
+
+def test_round_e4m3_matches_torch():
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([rng.uniform(0, 448, 3000), np.exp(rng.uniform(-12, 6, 3000))])
+    vals = vals[vals <= 448].astype(np.float32)
+    # midpoints between consecutive codes: exact ties
+    pos = [oracle.e4m3(c) for c in range(0x7F)]
+    mids = np.array([(a + b) / 2 for a, b in zip(pos[:-1], pos[1:])], np.float32)
+    allv = np.concatenate([vals, mids])
+    ref = torch.tensor(allv).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.round_e4m3(float(v)) for v in allv], np.uint8)
+    assert np.array_equal(got, ref)
+    assert oracle.round_e4m3(1000.0) == 0x7E and oracle.round_e4m3(0.0) == 0
+
+
+def test_act_quant_grid_values_are_exact():
+    grid = [0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -6.0, -0.5, 0.0, 1.0, -1.5, 2.0, -3.0, 4.0, 6.0]
+    X = np.array([grid], np.float32)
+    codes, scales, ag = oracle.act_quant(X)
+    assert scales[0, 0] == 0x7E  # amax_b / (6 a_g) = 448 exactly after rounding
+    dec = [oracle.e2m1((codes[0, j // 2] >> (4 * (j & 1))) & 0xF) for j in range(16)]
+    assert dec == grid
+    assert ag == np.float32(np.float32(6.0) / np.float32(6.0 * 448.0))
+
+
+def test_act_quant_error_bound_and_zero_tensor():
+    X = synth.activations(3, 64, synth.gen(40), dtype=torch.bfloat16).float().numpy()
+    codes, scales, ag = oracle.act_quant(X)
+    Aq = oracle.dequant(oracle.NVFP4, 3, 64, codes, scales, ag)
+    for m in range(3):
+        for b in range(4):
+            s = oracle.e4m3(int(scales[m, b])) * ag
+            blk = X[m, 16 * b:16 * b + 16].astype(np.float64)
+            # inside the E2M1 range the error is at most half of the largest grid step (1.0)
+            assert np.all(np.abs(blk - Aq[m, 16 * b:16 * b + 16]) <= 1.0 * s * (1 + 1e-6))
+    z_codes, z_scales, z_ag = oracle.act_quant(np.zeros((2, 32), np.float32))
+    assert z_ag == 0.0 and not z_codes.any() and not z_scales.any()

@@ -191,7 +191,10 @@ void qo_silu_gate(int M, int64_t I, const double* gu, const double* Agu, double*
 /* ---------------------------------------------------------------- MoE routing */
 
 /* Router for one token: p = softmax(logits) in fp64; the top_k experts by descending p (a tie
- * goes to the lower expert index); weights renormalised over the selected experts. */
+ * goes to the lower expert index); weights renormalised over the selected experts.
+ * softmax is strictly increasing in each logit, so ranking by p is ranking by the logits
+ * themselves: the selection compares the given logits (exact comparisons of the inputs, the same
+ * decision in any precision), and p is used only for the weights. */
 void qo_route(int E, int top_k, const double* logits, int32_t* ids, double* wts) {
     double mx = -INFINITY, z = 0.0;
     double* p = (double*)malloc(sizeof(double) * E);
@@ -203,7 +206,7 @@ void qo_route(int E, int top_k, const double* logits, int32_t* ids, double* wts)
     for (int s = 0; s < top_k; ++s) {
         int best = -1;
         for (int e = 0; e < E; ++e)
-            if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+            if (!taken[e] && (best < 0 || logits[e] > logits[best])) best = e;
         taken[best] = 1;
         ids[s] = best;
         wts[s] = p[best];

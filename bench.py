@@ -1,0 +1,385 @@
+#!/usr/bin/env python3
+"""Benchmark of the quantized decode-step linear layer on B200.
+
+Default workload: a synthetic Q4_0 dense decode layer stack shaped like a 4B model at M = 1:
+36 layers of hidden 2560, each with the projections q/k/v (2560 -> 4096/1024/1024, packed and
+launched as one fused 6144-row GEMV), o (4096 -> 2560), gate_up (2560 -> 2 x 9728, fused SiLU gate)
+and down (9728 -> 2560).  One step = one decode token through all 36 layers = 144 GEMV launches,
+captured once in a CUDA graph (with programmatic dependent launch between the kernels) and
+replayed.  Attention, norms, embeddings and the LM head are not part of the path and are not run.
+
+Metric: quantized GEMV weight-stream GB/s (algorithmic bytes: packed codes + scales + activations
++ outputs, each once) and the equivalent decode tokens/s; JSON line on stdout (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qlin|reference] [--config NAME]
+
+--impl reference times the fp64 CPU oracle (the test reference) on a bounded sample of the same
+workload; the oracle is used nowhere else in this file except the cpu_baseline leg.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "quantized GEMV weight-stream GB/s (% of B200 HBM peak); synthetic decode tok/s"
+HIDDEN, LAYERS = 2560, 36
+# (name, N, K, epilogue) per layer; q/k/v share their input and are packed as one 6144-row matrix
+STACK = [("qkv", 4096 + 1024 + 1024, 2560, 0), ("o", 2560, 4096, 0),
+         ("gate_up", 2 * 9728, 2560, 1), ("down", 2560, 9728, 0)]
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.lines = index, None, []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [t.strip() for t in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workloads
+class DenseStack:
+    """The packed layer stack on one GPU, with its inputs and outputs resident in HBM.
+
+    All per-layer activations live in one device buffer (xbuf) and all per-layer outputs that
+    leave the step (qkv, o, down) in another (ybuf), so the end-to-end leg moves them with one
+    host->device and one device->host copy per step."""
+
+    def __init__(self, fmt, layers, M=1, device="cuda"):
+        import gemm_dequant_gemv_q8_b200 as q
+        self.q, self.fmt, self.M, self.layers = q, fmt, M, layers
+        self.packed, self.ws = [], []
+        self.weight_bytes = 0
+        xs = [(l, pi, K) for l in range(layers) for pi, (n_, N, K, e) in enumerate(STACK) if n_ != "down"]
+        ys = [(l, pi, N) for l in range(layers) for pi, (n_, N, K, e) in enumerate(STACK) if n_ != "gate_up"]
+        self.xbuf = torch.empty(M, sum(k for _, _, k in xs), device=device)
+        self.ybuf = torch.empty(M, sum(n for _, _, n in ys), device=device)
+        self.hbuf = torch.empty(layers, M, STACK[2][1] // 2, device=device)
+        self.x, self.y = {}, {}
+        off = 0
+        for l, pi, K in xs:
+            self.x[(l, pi)] = self.xbuf[:, off:off + K]
+            off += K
+        off = 0
+        for l, pi, N in ys:
+            self.y[(l, pi)] = self.ybuf[:, off:off + N]
+            off += N
+        for l in range(layers):
+            self.x[(l, 3)] = self.hbuf[l]
+            self.y[(l, 2)] = self.hbuf[l]
+            lp, lw = [], []
+            for pi, (name, N, K, epi) in enumerate(STACK):
+                g = synth.gen(synth.seed_for(2, l, pi), device=device)
+                blocks, scales, gs = synth.weights(fmt, N, K, g, device=device)
+                pf = q.QLIN_PACK_GATE_UP if epi else q.QLIN_PACK_DEFAULT
+                lp.append(q.qlin_pack_weights(fmt, N, K, blocks, scales, gs, pf))
+                del blocks, scales
+                self.weight_bytes += q.qlin_packed_bytes(fmt, N, K, pf) - 256
+                lw.append(q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, N, K), device))
+                if name != "down":
+                    self.x[(l, pi)].copy_(synth.activations(
+                        M, K, synth.gen(synth.seed_for(2, l, 5 + pi), device=device), device=device))
+            self.packed.append(lp)
+            self.ws.append(lw)
+        torch.cuda.synchronize()
+        # algorithmic bytes per step: weights once + every activation read + every output written
+        act = 0
+        for (name, N, K, epi) in STACK:
+            act += 4 * M * K + 4 * M * (N // 2 if epi else N)
+        self.act_bytes = act * layers
+        self.step_bytes = self.weight_bytes + self.act_bytes
+        self.launches_per_step = len(STACK) * layers
+
+    def step(self, pdl=True):
+        q = self.q
+        fl = q.QLIN_FLAG_PDL if pdl else 0
+        for l in range(self.layers):
+            P, W = self.packed[l], self.ws[l]
+            for pi, (name, N, K, epi) in enumerate(STACK):
+                q.qlin_gemv(self.fmt, P[pi], N, K, self.x[(l, pi)], y=self.y[(l, pi)], ws=W[pi],
+                            flags=fl | (q.QLIN_EPI_SILU_GATE if epi else 0))
+
+    def capture(self, pdl=True, host_io=None):
+        """CUDA graph of one step; with host_io=(pinned_x, pinned_y) the graph also copies the
+        step's inputs in and its outputs out."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step(pdl)  # warm (attributes, module load)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if host_io:
+                self.xbuf.copy_(host_io[0], non_blocking=True)
+            self.step(pdl)
+            if host_io:
+                host_io[1].copy_(self.ybuf, non_blocking=True)
+        torch.cuda.synchronize()
+        return g
+
+
+def time_graph(graph, steps, warmup):
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        graph.replay()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def time_dominant_kernel(stack, reps=3):
+    """Average duration of the gate_up + SiLU GEMV launch (the largest per-launch share),
+    timed with CUDA events on the launching stream, rotating over the layers' matrices
+    (1 GB of weights at 36 layers, so every launch streams from HBM)."""
+    q = stack.q
+    name, N, K, epi = STACK[2]
+    st = torch.cuda.current_stream()
+
+    def run():
+        for l in range(stack.layers):
+            q.qlin_gemv(stack.fmt, stack.packed[l][2], N, K, stack.x[(l, 2)], y=stack.y[(l, 2)],
+                        ws=stack.ws[l][2], flags=q.QLIN_EPI_SILU_GATE)
+
+    run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(reps):
+        run()
+    b.record(st)
+    b.synchronize()
+    ms = a.elapsed_time(b) / (reps * stack.layers)
+    bytes_ = (q.qlin_packed_bytes(stack.fmt, N, K, q.QLIN_PACK_GATE_UP) - 256) + 4 * stack.M * (K + N // 2)
+    return ms, bytes_
+
+
+def e2e_stack(stack, steps, warmup, pdl=True):
+    """Same metric through the public API with host buffers: every step copies its inputs from
+    pinned host memory, runs the stack, and reads its outputs back, all inside the timed region
+    (one graph: H2D copy, 144 GEMV launches, D2H copy)."""
+    hx = stack.xbuf.cpu().pin_memory()
+    hy = torch.empty(stack.ybuf.shape, dtype=torch.float32).pin_memory()
+    g = stack.capture(pdl, host_io=(hx, hy))
+    ms = time_graph(g, steps, warmup)
+    del g
+    return ms, hx.numel() * 4, hy.numel() * 4
+
+
+def cpu_baseline_stack(fmt, budget_s=12.0, seed=7):
+    """The fp64 oracle on a bounded sample of the stack: rows of every projection shape, timed
+    on the host; scaled to GB/s of weights processed.  Returns (GB/s, cores, description)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    per_shape = []
+    for (name, N, K, epi) in STACK:
+        b, s, gs = synth.weights(fmt, 64, K, synth.gen(seed + N))
+        x = synth.activations(1, K, synth.gen(seed + K)).double().numpy()
+        per_shape.append((N, K, b.numpy(), None if s is None else s.numpy(), gs, x))
+    # probe, then size the sample to the budget
+    done_bytes, t_used, rows = 0, 0.0, 0
+    t0 = time.perf_counter()
+    while t_used < budget_s:
+        for (N, K, b, s, gs, x) in per_shape:
+            r = rng.integers(0, 64, 16)
+            oracle.gemv(fmt, 64, K, b, x, scales=s, g=gs, rows=r)
+            rowb = oracle.row_bytes(fmt, K)
+            done_bytes += 16 * rowb
+            rows += 16
+        t_used = time.perf_counter() - t0
+    gbs = done_bytes / t_used / 1e9
+    desc = (f"{rows} weight rows of the four stack projection shapes (K = 2560/4096/2560/9728), "
+            f"single-threaded fp64 oracle, {t_used:.1f} s")
+    return gbs, 1, desc
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="qlin", choices=["qlin", "reference"])
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    fmt = synth.Q4_0
+    workload = (f"Q4_0 dense decode layer stack shaped like a 4B model, M=1: {args.layers} layers of "
+                "hidden 2560; qkv 2560->6144 (q/k/v fused), o 4096->2560, gate_up 2560->2x9728 + SiLU, "
+                "down 9728->2560")
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        gbs, cores, desc = cpu_baseline_stack(fmt, budget_s=max(5.0, 2.0 * args.steps))
+        stack_w = sum((N * K * 9 // 16) for (_, N, K, _) in STACK) * args.layers
+        tok_s = gbs * 1e9 / stack_w
+        line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 / tok_s, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference", "decode_tok_s": tok_s,
+                "config": {"workload": workload, "format": "q4_0", "M": 1, "layers": args.layers},
+                "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
+                "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+
+    stack = DenseStack(fmt, args.layers)
+    graph = stack.capture(pdl=not args.no_pdl)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        graph.replay()
+    barrier()
+    with ClockSampler(local) as clk:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            graph.replay()
+        b.record()
+        b.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+    barrier()
+    ms_t = torch.tensor([ms], device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    dom_ms, dom_bytes = time_dominant_kernel(stack)
+    e2e_ms, h2d, d2h = e2e_stack(stack, args.steps, args.warmup, pdl=not args.no_pdl)
+    e2e_t = torch.tensor([e2e_ms], device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+    del graph
+
+    if rank == 0:
+        peak, peak_src = peaks()
+        gbs = world * stack.step_bytes / (ms_max * 1e-3) / 1e9
+        dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+        traffic = None
+        try:
+            with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+                traffic = json.load(f).get("gate_up_q4_0_m1_bytes_per_launch")
+        except Exception:
+            pass
+        line = {
+            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "decode_tok_s": world * 1e3 / ms_max,
+            "hbm_frac": gbs / world / peak,
+            "config": {"workload": workload, "format": "q4_0", "M": 1, "layers": args.layers,
+                       "weight_bytes_per_step": stack.weight_bytes, "algorithmic_bytes_per_step": stack.step_bytes,
+                       "launches_per_step": stack.launches_per_step, "cuda_graph": True, "pdl": not args.no_pdl,
+                       "l2": "inputs larger than L2: 2.04 GB of packed weights streamed per step (L2 126 MB)",
+                       "parallelism": f"replicas{world}"},
+            "roofline": {"bound": "hbm", "kernel": "gemv_kernel<Q4_0, M=1, SiLU-gate> (gate_up 2560->19456)",
+                         "achieved": dom_gbs, "peak": peak, "peak_source": f"{peak_src} hbm_gbs (copy)",
+                         "unit": "GB/s", "frac": dom_gbs / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": dom_ms * 1e3},
+            "e2e": {"value": world * stack.step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": stack.launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            cg, cores, desc = cpu_baseline_stack(fmt)
+            line["cpu_baseline"] = {"value": cg, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,163 @@
+// api.cu -- the C ABI of libqlin: host-side validation, status codes, launches on the caller's
+// stream.  Declarations and the contract of every entry point are in include/qlin.h.
+#include <stdio.h>
+
+#include "qlin_common.cuh"
+
+extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void* scales, int64_t N,
+                                        int64_t K, int pack_flags, float gs, void* packed,
+                                        cudaStream_t s);
+extern "C" cudaError_t qlin_launch_unpack(int fmt, const void* packed, int64_t N, int64_t K,
+                                          int pack_flags, float* w, cudaStream_t s);
+extern "C" size_t qlin_gemv_ws_bytes(int fmt, int M, int64_t N, int64_t K, int pack_flags);
+extern "C" size_t qlin_moe_ws_bytes(int fmt, int M, int64_t H, int64_t I, int E, int top_k);
+extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, int E, int64_t H, int64_t I,
+                                       int top_k, const float* logits, int32_t* ids, float* wts, const void* x,
+                                       int xdt, int M, float* y, float* h, int flags, void* ws, cudaStream_t s);
+extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, int64_t K,
+                                        const void* x, int xdt, int M, int64_t ldx, float* y,
+                                        int64_t ldy, int flags, void* ws, cudaStream_t s);
+
+namespace {
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+bool valid_fmt(int f) { return f == QLIN_Q8_0 || f == QLIN_Q4_0 || f == QLIN_NVFP4; }
+
+bool valid_shape(int fmt, int64_t N, int64_t K) {
+    if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return false;
+    return fmt == QLIN_NVFP4 ? (K % 16 == 0) : (K % 32 == 0);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+qlin_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags) {
+    if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
+    if (pack_flags & ~QLIN_PACK_GATE_UP) return 0;
+    if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return 0;
+    qlin::Geometry g = qlin::geometry(fmt, N, K, pack_flags);
+    return (size_t)qlin::kHdrBytes + (size_t)g.U * (size_t)qlin::unit_bytes(fmt);
+}
+
+qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const void* blocks,
+                                const void* scales, float global_scale, int pack_flags,
+                                void* packed, size_t packed_bytes, qlin_stream_t stream) {
+    if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
+    if (!valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
+    if (pack_flags & ~QLIN_PACK_GATE_UP) return QLIN_ERR_INVALID_ARG;
+    if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
+    if (!blocks || !packed) return QLIN_ERR_INVALID_ARG;
+    if (fmt == QLIN_NVFP4 && !scales) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(packed, 256)) return QLIN_ERR_ALIGNMENT;
+    if (packed_bytes < qlin_packed_bytes(fmt, N, K, pack_flags)) return QLIN_ERR_INVALID_ARG;
+    const float gs = fmt == QLIN_NVFP4 ? global_scale : 1.0f;
+    return cuda_status(qlin_launch_pack(fmt, blocks, scales, N, K, pack_flags, gs, packed,
+                                        (cudaStream_t)stream));
+}
+
+size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t K, int E, int top_k) {
+    (void)E;
+    (void)top_k;
+    if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
+    if (op == QLIN_OP_MOE) {  /* N = H, K = I */
+        if (M < 1 || M > 8 || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return 0;
+        if (!valid_shape(fmt, 2 * K, N) || !valid_shape(fmt, N, K)) return 0;
+        return qlin_moe_ws_bytes(fmt, M, N, K, E, top_k);
+    }
+    if (op == QLIN_OP_GEMV) {
+        if (M < 1 || M > 8) return 0;
+        size_t a = qlin_gemv_ws_bytes(fmt, M, N, K, 0);
+        size_t b = (N % 2 == 0) ? qlin_gemv_ws_bytes(fmt, M, N, K, QLIN_PACK_GATE_UP) : 0;
+        return a > b ? a : b;
+    }
+    return 0;
+}
+
+qlin_status_t qlin_gemv(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,
+                        qlin_dtype_t xdt, int M, int64_t ldx, float* y, int64_t ldy, int flags,
+                        void* ws, size_t ws_bytes, qlin_stream_t stream) {
+    if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
+    if (M < 1 || M > 8) return QLIN_ERR_INVALID_ARG;
+    if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
+    const int epi = flags & 0xff;
+    if (epi != QLIN_EPI_NONE && epi != QLIN_EPI_SILU_GATE) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~(0xff | QLIN_FLAG_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (epi == QLIN_EPI_SILU_GATE && (N % 2)) return QLIN_ERR_INVALID_ARG;
+    if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
+    const int64_t ncols = epi == QLIN_EPI_SILU_GATE ? N / 2 : N;
+    if (ldx < K || ldy < ncols) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(packed, 256) || !aligned(x, 16) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
+    if (ldx % (xdt == QLIN_F32 ? 4 : 8)) return QLIN_ERR_ALIGNMENT;
+    const int pack_flags = epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0;
+    const size_t need = qlin_gemv_ws_bytes(fmt, M, N, K, pack_flags);
+    if (!ws || ws_bytes < need) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_gemv(fmt, packed, N, K, x, xdt, M, ldx, y, ldy, flags, ws,
+                                        (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, const void* down_packed,
+                               int E, int64_t H, int64_t I, int top_k, const float* router_logits,
+                               int32_t* topk_ids, float* topk_w, const void* x, qlin_dtype_t xdt, int M,
+                               float* y, float* h, int flags, void* ws, size_t ws_bytes,
+                               qlin_stream_t stream) {
+    if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
+    if (M < 1 || M > 8 || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return QLIN_ERR_INVALID_ARG;
+    if (!valid_shape(fmt, 2 * I, H) || !valid_shape(fmt, H, I)) return QLIN_ERR_INVALID_ARG;
+    if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~QLIN_FLAG_PDL) return QLIN_ERR_INVALID_ARG;
+    if (!gate_up_packed || !down_packed || !topk_ids || !topk_w || !x || !y) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(gate_up_packed, 256) || !aligned(down_packed, 256) || !aligned(x, 16) || !aligned(y, 4) ||
+        !aligned(topk_ids, 4) || !aligned(topk_w, 4) || (router_logits && !aligned(router_logits, 4)) ||
+        (h && !aligned(h, 16)))
+        return QLIN_ERR_ALIGNMENT;
+    const size_t need = qlin_moe_ws_bytes(fmt, M, H, I, E, top_k);
+    if (!ws || ws_bytes < need) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_moe(fmt, gate_up_packed, down_packed, E, H, I, top_k, router_logits, topk_ids,
+                                       topk_w, x, xdt, M, y, h, flags, ws, (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
+                                 int pack_flags, float* w, qlin_stream_t stream) {
+    if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
+    if (pack_flags & ~QLIN_PACK_GATE_UP) return QLIN_ERR_INVALID_ARG;
+    if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
+    if (!packed || !w) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(packed, 256) || !aligned(w, 4)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_unpack(fmt, packed, N, K, pack_flags, w, (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_ws_status(void* ws, qlin_stream_t stream) {
+    if (!ws) return QLIN_ERR_INVALID_ARG;
+    unsigned int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return QLIN_ERR_CUDA;
+    if (word == 0) return QLIN_OK;
+    e = cudaMemsetAsync(ws, 0, sizeof(word), (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return QLIN_ERR_CUDA;
+    return (word & 1u) ? QLIN_ERR_TIMEOUT : QLIN_ERR_INVALID_ARG;  /* bit 1: bad expert id */
+}
+
+const char* qlin_status_string(qlin_status_t s) {
+    switch (s) {
+        case QLIN_OK: return "QLIN_OK";
+        case QLIN_ERR_INVALID_ARG: return "QLIN_ERR_INVALID_ARG";
+        case QLIN_ERR_UNSUPPORTED: return "QLIN_ERR_UNSUPPORTED";
+        case QLIN_ERR_ALIGNMENT: return "QLIN_ERR_ALIGNMENT";
+        case QLIN_ERR_WORKSPACE: return "QLIN_ERR_WORKSPACE";
+        case QLIN_ERR_CUDA: return "QLIN_ERR_CUDA";
+        case QLIN_ERR_TIMEOUT: return "QLIN_ERR_TIMEOUT";
+    }
+    return "QLIN_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+// pack.cu -- canonical GGUF / NVFP4 tensors -> the packed tile layout, and its inverse for tests.
+//
+// The repacker is the offline step that re-lays weights once per tensor (the pages' prior art:
+// Imparo README intro, a "private GateUp layout" built from the canonical GGUF; imp README "Why
+// this exists", an NVFP4 decode cache transformed at init).  It moves bytes only: no rounding.
+#include "qlin_common.cuh"
+
+namespace qlin {
+
+// Source row of packed tile row r, or -1 for padding.
+__device__ __forceinline__ int64_t source_row(int64_t t, int r, int64_t N, int gate_up) {
+    if (gate_up) {
+        int64_t half = N / 2;
+        int64_t i = t * 16 + (r & 15);
+        if (i >= half) return -1;
+        return r < 16 ? i : half + i;
+    }
+    int64_t n = t * kTileRows + r;
+    return n < N ? n : -1;
+}
+
+// One CTA per unit; thread (r, p) = (tid / 8, tid % 8) writes row r, part p.
+template <int FMT>
+__global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ blocks,
+                                                   const uint8_t* __restrict__ scales, int64_t N,
+                                                   int64_t K, int gate_up, uint8_t* __restrict__ packed,
+                                                   int64_t G) {
+    const int64_t unit = blockIdx.x;
+    const int64_t t = unit / G, g = unit % G;
+    const int r = threadIdx.x >> 3, p = threadIdx.x & 7;
+    uint8_t* ub = packed + kHdrBytes + unit * (int64_t)unit_bytes(FMT);
+    const int64_t n = source_row(t, r, N, gate_up);
+    const int64_t k0 = g * kGroupK + p * 32;  // first element of this part
+    const int lane = (r & 3) * 8 + p, slot = r >> 2;
+    uint8_t* sc = ub + code_bytes(FMT) + lane * 16 + slot * 2;
+
+    if (FMT == QLIN_Q4_0) {
+        uint8_t out[16];
+        uint16_t d = 0;
+        if (n >= 0 && k0 < K) {
+            const uint8_t* blk = blocks + n * (K / 32) * 18 + (k0 / 32) * 18;
+            d = (uint16_t)(blk[0] | (blk[1] << 8));
+            uint8_t e[32];
+            for (int j = 0; j < 16; ++j) {
+                e[j] = blk[2 + j] & 0xf;
+                e[j + 16] = blk[2 + j] >> 4;
+            }
+            for (int j = 0; j < 16; ++j) out[j] = (uint8_t)(e[2 * j] | (e[2 * j + 1] << 4));
+        } else {
+            for (int j = 0; j < 16; ++j) out[j] = 0x88;  // code 8 -> value 0, with d = 0
+        }
+        uint4 v;
+        memcpy(&v, out, 16);
+        *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v;
+        sc[0] = (uint8_t)(d & 0xff);
+        sc[1] = (uint8_t)(d >> 8);
+    } else if (FMT == QLIN_Q8_0) {
+        uint8_t out[32];
+        uint16_t d = 0;
+        if (n >= 0 && k0 < K) {
+            const uint8_t* blk = blocks + n * (K / 32) * 34 + (k0 / 32) * 34;
+            d = (uint16_t)(blk[0] | (blk[1] << 8));
+            for (int j = 0; j < 32; ++j) out[j] = (uint8_t)(blk[2 + j] ^ 0x80u);  // q + 128
+        } else {
+            for (int j = 0; j < 32; ++j) out[j] = 0x80;  // q = 0
+        }
+        uint4 v0, v1;
+        memcpy(&v0, out, 16);
+        memcpy(&v1, out + 16, 16);
+        *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v0;
+        *reinterpret_cast<uint4*>(ub + 4096 + (r * 8 + p) * 16) = v1;
+        sc[0] = (uint8_t)(d & 0xff);
+        sc[1] = (uint8_t)(d >> 8);
+    } else {  // NVFP4: codes already two per byte in element order
+        uint8_t out[16];
+        uint8_t s0 = 0, s1 = 0;
+        for (int j = 0; j < 16; ++j) out[j] = 0;
+        if (n >= 0 && k0 < K) {
+            const uint8_t* row = blocks + n * (K / 2);
+            const uint8_t* srow = scales + n * (K / 16);
+            const int64_t valid = (K - k0) >= 32 ? 32 : (K - k0);  // 16 or 32
+            for (int j = 0; j < valid / 2; ++j) out[j] = row[k0 / 2 + j];
+            s0 = srow[k0 / 16];
+            if (valid == 32) s1 = srow[k0 / 16 + 1];
+        }
+        uint4 v;
+        memcpy(&v, out, 16);
+        *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v;
+        sc[0] = s0;
+        sc[1] = s1;
+    }
+}
+
+__global__ void write_header_kernel(uint8_t* packed, uint32_t fmt, int64_t N, int64_t K,
+                                    uint32_t flags, float gs, int32_t T, int32_t G) {
+    PackedHeader* h = reinterpret_cast<PackedHeader*>(packed);
+    if (threadIdx.x == 0) {
+        h->magic = kMagic;
+        h->fmt = fmt;
+        h->N = N;
+        h->K = K;
+        h->flags = flags;
+        h->global_scale = gs;
+        h->T = T;
+        h->G = G;
+        h->unit_bytes = (uint32_t)unit_bytes((int)fmt);
+    }
+    if (threadIdx.x >= 1 && threadIdx.x < 54) h->reserved[threadIdx.x - 1] = 0;
+}
+
+// Inverse for tests: one CTA per unit, thread (r, p) writes the 32 fp32 weights of its part.
+template <int FMT>
+__global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__ packed, int64_t N,
+                                                     int64_t K, int gate_up, int64_t G,
+                                                     float* __restrict__ w) {
+    const int64_t unit = blockIdx.x;
+    const int64_t t = unit / G, g = unit % G;
+    const int r = threadIdx.x >> 3, p = threadIdx.x & 7;
+    const uint8_t* ub = packed + kHdrBytes + unit * (int64_t)unit_bytes(FMT);
+    const int64_t n = source_row(t, r, N, gate_up);
+    const int64_t k0 = g * kGroupK + p * 32;
+    if (n < 0 || k0 >= K) return;
+    const int lane = (r & 3) * 8 + p, slot = r >> 2;
+    const uint8_t* sc = ub + code_bytes(FMT) + lane * 16 + slot * 2;
+    const float gs = reinterpret_cast<const PackedHeader*>(packed)->global_scale;
+    const int64_t valid = (K - k0) >= 32 ? 32 : (K - k0);
+    float* out = w + n * K + k0;
+    const uint8_t* cv = ub + (r * 8 + p) * 16;
+    if (FMT == QLIN_Q4_0) {
+        float d = fp16_bits_to_f32(sc[0] | (sc[1] << 8));
+        for (int e = 0; e < 32; ++e) {
+            int nib = (cv[e / 2] >> (4 * (e & 1))) & 0xf;
+            out[e] = d * (float)(nib - 8);
+        }
+    } else if (FMT == QLIN_Q8_0) {
+        float d = fp16_bits_to_f32(sc[0] | (sc[1] << 8));
+        for (int e = 0; e < 32; ++e) {
+            int b = (e < 16 ? cv[e] : cv[4096 + e - 16]);
+            out[e] = d * (float)(b - 128);
+        }
+    } else {
+        for (int e = 0; e < valid; ++e) {
+            uint32_t h2 = e2m1x2_to_f16x2(cv[e / 2]);
+            float v = __half2float(__ushort_as_half((unsigned short)((e & 1) ? (h2 >> 16) : (h2 & 0xffff))));
+            float s = e4m3_to_f32(sc[e / 16]);
+            out[e] = __fmul_rn(__fmul_rn(v, s), gs);  // v*s is exact; the tensor scale rounds once
+        }
+    }
+}
+
+}  // namespace qlin
+
+using namespace qlin;
+
+extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void* scales, int64_t N,
+                                        int64_t K, int pack_flags, float gs, void* packed,
+                                        cudaStream_t s) {
+    Geometry geo = geometry(fmt, N, K, pack_flags);
+    const int gu = (pack_flags & QLIN_PACK_GATE_UP) ? 1 : 0;
+    write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags,
+                                         gs, (int32_t)geo.T, (int32_t)geo.G);
+    dim3 grid((unsigned)geo.U);
+    if (fmt == QLIN_Q4_0)
+        pack_kernel<QLIN_Q4_0><<<grid, 256, 0, s>>>((const uint8_t*)blocks, nullptr, N, K, gu,
+                                                     (uint8_t*)packed, geo.G);
+    else if (fmt == QLIN_Q8_0)
+        pack_kernel<QLIN_Q8_0><<<grid, 256, 0, s>>>((const uint8_t*)blocks, nullptr, N, K, gu,
+                                                     (uint8_t*)packed, geo.G);
+    else
+        pack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)blocks, (const uint8_t*)scales,
+                                                      N, K, gu, (uint8_t*)packed, geo.G);
+    return cudaGetLastError();
+}
+
+extern "C" cudaError_t qlin_launch_unpack(int fmt, const void* packed, int64_t N, int64_t K,
+                                          int pack_flags, float* w, cudaStream_t s) {
+    Geometry geo = geometry(fmt, N, K, pack_flags);
+    const int gu = (pack_flags & QLIN_PACK_GATE_UP) ? 1 : 0;
+    dim3 grid((unsigned)geo.U);
+    if (fmt == QLIN_Q4_0)
+        unpack_kernel<QLIN_Q4_0><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
+    else if (fmt == QLIN_Q8_0)
+        unpack_kernel<QLIN_Q8_0><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
+    else
+        unpack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
+    return cudaGetLastError();
+}

@@ -1,0 +1,164 @@
+/*
+ * qlin.h -- C ABI of libqlin, a B200 (sm_100a) library for the decode-step linear layer over
+ * block-quantized weights: fused dequantize-and-multiply of GGUF Q8_0 / Q4_0 blocks and NVFP4
+ * tensors against a small batch of activation rows, the routed MoE expert projections, and an
+ * NVFP4 prefill-chunk GEMM on the tcgen05 tensor cores.
+ *
+ * What the operations compute comes from the pages describing the "imp" engine (README
+ * "Features" table, rows "Quantization", "Architectures" and "sm_120a kernels"; README "Why this
+ * exists") and the "Imparo" engine (README intro: Q4_0 MoE decode with CUDA expert routing).  The
+ * pages name the formats but not their byte layout; the layouts below are the public conventions.
+ *
+ * Conventions for every entry point
+ *   - W is N x K (output x input), row-major along K; y[m][n] = sum_k x[m][k] * W[n][k].
+ *   - Every pointer argument is a caller-owned DEVICE pointer unless stated otherwise.  The
+ *     library allocates nothing and keeps no global state (apart from a per-device SM-count
+ *     cache); all work is enqueued asynchronously on `stream` (NULL = the legacy default stream).
+ *   - Arguments are validated on the host before anything is launched; a failed check returns
+ *     its status code and enqueues nothing.  A launch failure returns QLIN_ERR_CUDA.
+ *   - No C++ exception crosses this boundary.
+ *   - Workspaces ("ws") are caller-owned device buffers of at least qlin_workspace_bytes(...)
+ *     bytes, 256-byte aligned, ZERO-FILLED before their first use.  Every call leaves the
+ *     workspace's counters zero again when it completes, so a workspace can be reused by calls
+ *     that run one after another on one stream; calls that overlap on the GPU must not share one.
+ */
+#ifndef QLIN_H
+#define QLIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qlin_stream_t; /* a cudaStream_t */
+
+typedef enum { QLIN_Q8_0 = 1, QLIN_Q4_0 = 2, QLIN_NVFP4 = 3 } qlin_format_t;
+typedef enum { QLIN_F32 = 0, QLIN_BF16 = 1 } qlin_dtype_t;
+typedef enum {
+    QLIN_OK = 0,
+    QLIN_ERR_INVALID_ARG = 1, /* a null pointer, a size out of range, an unknown enum value   */
+    QLIN_ERR_UNSUPPORTED = 2, /* a valid combination this library does not implement          */
+    QLIN_ERR_ALIGNMENT = 3,   /* a pointer or leading dimension breaks the alignment rules    */
+    QLIN_ERR_WORKSPACE = 4,   /* ws is NULL or smaller than qlin_workspace_bytes()            */
+    QLIN_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, attribute query)         */
+    QLIN_ERR_TIMEOUT = 6      /* a bounded device wait gave up (reported by qlin_ws_status)   */
+} qlin_status_t;
+
+/* qlin_gemv flags (OR-able) */
+enum {
+    QLIN_EPI_NONE = 0,      /* y[m][n] for n < N                                                 */
+    QLIN_EPI_SILU_GATE = 1, /* gated MLP epilogue: rows [0, N/2) are the gate g, rows [N/2, N) the
+                               up projection u; y[m][i] = silu(g_i) * u_i for i < N/2, with
+                               silu(z) = z / (1 + exp(-z)).  Requires a QLIN_PACK_GATE_UP buffer. */
+    QLIN_FLAG_PDL = 0x100   /* launch with programmatic dependent launch: the kernel starts
+                               streaming its weights while the previous kernel on the stream is
+                               still running, and waits for it before touching x or y.  Only
+                               valid when the packed weights were written before the previous
+                               kernel on the stream started.                                      */
+};
+
+/* qlin_pack_weights flags */
+enum {
+    QLIN_PACK_DEFAULT = 0,
+    QLIN_PACK_GATE_UP = 1 /* the N rows are [gate ; up] halves (N even): each packed tile pairs
+                             16 gate rows with their 16 up rows so the SiLU-gate epilogue fuses */
+};
+
+/* qlin_workspace_bytes ops */
+enum { QLIN_OP_GEMV = 1, QLIN_OP_MOE = 2, QLIN_OP_CHUNK = 3 };
+
+/* ------------------------------------------------------------------------- weight repacking */
+
+/* Bytes of the packed buffer for an N x K tensor (0 for invalid arguments).
+ * The packed layout is library-private: a 256-byte header (format, sizes, the NVFP4 per-tensor
+ * scale), then tiles of 32 output rows x 256 inputs, each stored as 16-byte code vectors that a
+ * warp reads contiguously, followed by that tile's scales; K is padded to a multiple of 256 and N
+ * to a multiple of 32 (16 per half for QLIN_PACK_GATE_UP) with zero codes and zero scales.
+ * The packed size is the canonical size plus that padding (Q8_0 1.0625 B/weight, Q4_0 and NVFP4
+ * 0.5625 B/weight).  Prior art for a private re-laid-out weight copy: Imparo README intro
+ * ("private GateUp layout"); imp README "Why this exists" (an NVFP4 decode cache built at init). */
+size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags);
+
+/* Re-lay a canonical tensor into the packed layout (one kernel, enqueued on `stream`).
+ *   Q8_0 : blocks = GGUF block_q8_0 rows [N][K/32] x 34 B (fp16 d, int8 q[32]), scales = NULL
+ *   Q4_0 : blocks = GGUF block_q4_0 rows [N][K/32] x 18 B (fp16 d, 16 B of nibbles; byte j holds
+ *          element j low, element j+16 high), scales = NULL
+ *   NVFP4: blocks = E2M1 codes [N][K/2] (byte i: element 2i low nibble, 2i+1 high nibble),
+ *          scales = E4M3 [N][K/16], global_scale = the fp32 per-tensor scale
+ * K % 32 == 0 for Q8_0 / Q4_0, K % 16 == 0 for NVFP4; N >= 1; QLIN_PACK_GATE_UP needs N even.
+ * `packed` must be 256-byte aligned and hold qlin_packed_bytes(...) bytes.  Canonical inputs
+ * have no alignment requirement.  The canonical buffers may be freed once the kernel has run. */
+qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const void* blocks,
+                                const void* scales, float global_scale, int pack_flags,
+                                void* packed, size_t packed_bytes, qlin_stream_t stream);
+
+/* ------------------------------------------------------------------------- dense GEMV (M = 1..8) */
+
+/* Workspace bytes for an op.  QLIN_OP_GEMV: (fmt, M, N, K); QLIN_OP_MOE: (fmt, M, N = H,
+ * K = I, E, top_k); QLIN_OP_CHUNK: (fmt, M, N, K).  0 for invalid arguments. */
+size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t K, int E,
+                            int top_k);
+
+/* y = x * W^T for M activation rows, W packed by qlin_pack_weights with the same fmt, N, K
+ * (QLIN_PACK_GATE_UP with QLIN_EPI_SILU_GATE, QLIN_PACK_DEFAULT otherwise).
+ *   x   : M rows of K values, fp32 or bf16 (xdt), row stride ldx elements; 16-byte aligned with
+ *         ldx a multiple of 4 (fp32) or 8 (bf16)
+ *   y   : fp32, row stride ldy elements; N columns per row, or N/2 with QLIN_EPI_SILU_GATE
+ *   flags: QLIN_EPI_* | QLIN_FLAG_PDL
+ * Weights stream from HBM once; dequantization happens in registers; products and sums are fp32
+ * (activations are never quantized).  Results are deterministic for a given device and shape.
+ * The dequantize-and-multiply of quantized weight blocks against activations is the "NVFP4
+ * block-scaled GEMM/GEMV" and "dp4a Q8_0 decode" of the imp pages (README "Features"; release
+ * notes v0.4.1), re-designed here for sm_100a. */
+qlin_status_t qlin_gemv(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,
+                        qlin_dtype_t xdt, int M, int64_t ldx, float* y, int64_t ldy, int flags,
+                        void* ws, size_t ws_bytes, qlin_stream_t stream);
+
+/* ------------------------------------------------------------------------- routed MoE experts */
+
+/* Top-k routed MoE expert projections for M = 1..8 tokens.  Follows the Imparo README intro (a
+ * Q4_0 MoE decode through "CUDA expert routing", LFM2.5-8B-A1B) and the imp README "Features"
+ * table (MoE top-k grouped GEMM; an ordered, deterministic MoE reduction):
+ *   route  : p = softmax(router_logits[m]); the top_k experts by p (a tie goes to the lower expert
+ *            index); weights renormalised over the selected experts
+ *   experts: h = silu(W_gate[e] x) * (W_up[e] x);  o = W_down[e] h   (fp32, as qlin_gemv)
+ *   output : y[m] = sum over slots in slot order of weight * o
+ * Only the selected experts' weights are read, each once per call for all tokens routed to it.
+ * Arguments:
+ *   gate_up_packed: E consecutive buffers, each qlin_packed_bytes(fmt, 2I, H, QLIN_PACK_GATE_UP)
+ *                   bytes, expert e packed from its [gate ; up] rows (2I x H)
+ *   down_packed   : E consecutive buffers, each qlin_packed_bytes(fmt, H, I, 0) bytes (H x I)
+ *   router_logits : M x E fp32, or NULL -- then topk_ids / topk_w are inputs (ids in [0, E), no
+ *                   repeats within a token; a bad slot is skipped and qlin_ws_status() reports
+ *                   QLIN_ERR_INVALID_ARG)
+ *   topk_ids, topk_w: M x top_k int32 / fp32, written when router_logits is given
+ *   x : M x H rows (fp32 or bf16), contiguous;  y : M x H fp32, contiguous
+ *   h : optional M x top_k x I fp32 output of the SiLU-gated intermediate (NULL: kept in ws)
+ *   flags: 0 or QLIN_FLAG_PDL;  ws: qlin_workspace_bytes(QLIN_OP_MOE, fmt, M, H, I, E, top_k)
+ * E <= 256, top_k <= min(8, E).  Two kernel launches on `stream`, no host synchronisation. */
+qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, const void* down_packed,
+                               int E, int64_t H, int64_t I, int top_k, const float* router_logits,
+                               int32_t* topk_ids, float* topk_w, const void* x, qlin_dtype_t xdt, int M,
+                               float* y, float* h, int flags, void* ws, size_t ws_bytes,
+                               qlin_stream_t stream);
+
+/* Dequantize a packed buffer back to fp32 W[N][K] (row-major, canonical row order, also for
+ * QLIN_PACK_GATE_UP buffers; pass the pack_flags the buffer was packed with).  The value of every
+ * weight is the exact fp32 number d*q (Q8_0), d*(q-8) (Q4_0), or fp32(e2m1*e4m3*g) rounded once
+ * (NVFP4).  A test and inspection aid; not on the hot path.  w must be 4-byte aligned. */
+qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
+                                 int pack_flags, float* w, qlin_stream_t stream);
+
+/* Read and clear the sticky device status word of a workspace (synchronises `stream`).
+ * Returns QLIN_OK, QLIN_ERR_TIMEOUT if a bounded device wait gave up since the last check, or
+ * QLIN_ERR_INVALID_ARG if qlin_moe_experts met an invalid or repeated expert id. */
+qlin_status_t qlin_ws_status(void* ws, qlin_stream_t stream);
+
+const char* qlin_status_string(qlin_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLIN_H */

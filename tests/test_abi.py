@@ -1,0 +1,94 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry point
+declared in include/qlin.h, and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gemm_dequant_gemv_q8_b200 as q
+from gemm_dequant_gemv_q8_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return q.lib()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"\b(qlin_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "qlin_gemv" in names and "qlin_pack_weights" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(q.SIGNATURES) <= set(names)
+
+
+def test_status_strings(lib):
+    for code, name in q.STATUS.items():
+        assert q.qlin_status_string(code) == name
+
+
+def test_packed_bytes_sizes(lib):
+    # Q4_0 / NVFP4: 0.5625 B per weight, Q8_0: 1.0625, plus a 256-byte header; N->32, K->256 pad.
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 4096, 2560) == 256 + 4096 * 2560 * 9 // 16
+    assert q.qlin_packed_bytes(q.QLIN_Q8_0, 1024, 256) == 256 + 1024 * 256 * 17 // 16
+    assert q.qlin_packed_bytes(q.QLIN_NVFP4, 32, 16) == 256 + 4608
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 33, 288) == 256 + 2 * 2 * 4608
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 64, 256, q.QLIN_PACK_GATE_UP) == 256 + 2 * 4608
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 64, 100) == 0  # K % 32
+    assert q.qlin_packed_bytes(q.QLIN_NVFP4, 64, 40) == 0  # K % 16
+    assert q.qlin_packed_bytes(7, 64, 256) == 0
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 63, 256, q.QLIN_PACK_GATE_UP) == 0  # odd N
+
+
+def _gemv(lib, fmt=2, packed=0x100000, N=64, K=256, x=0x200000, xdt=0, M=1, ldx=256, y=0x300000,
+          ldy=64, flags=0, ws=0x400000, ws_bytes=1 << 30):
+    P = ctypes.c_void_p
+    return lib.qlin_gemv(fmt, P(packed), N, K, P(x), xdt, M, ldx, P(y), ldy, flags, P(ws), ws_bytes, None)
+
+
+def test_gemv_argument_checks_return_before_launch(lib):
+    E_ARG, E_ALIGN, E_WS = 1, 3, 4
+    assert _gemv(lib, fmt=9) == E_ARG
+    assert _gemv(lib, M=0) == E_ARG and _gemv(lib, M=9) == E_ARG
+    assert _gemv(lib, K=100) == E_ARG
+    assert _gemv(lib, xdt=5) == E_ARG
+    assert _gemv(lib, flags=7) == E_ARG
+    assert _gemv(lib, flags=q.QLIN_EPI_SILU_GATE, N=63) == E_ARG
+    assert _gemv(lib, packed=0) == E_ARG and _gemv(lib, x=0) == E_ARG and _gemv(lib, y=0) == E_ARG
+    assert _gemv(lib, ldx=128) == E_ARG and _gemv(lib, ldy=10) == E_ARG
+    assert _gemv(lib, x=0x200004) == E_ALIGN
+    assert _gemv(lib, packed=0x100010) == E_ALIGN
+    assert _gemv(lib, ldx=258) == E_ALIGN
+    assert _gemv(lib, ws=0) == E_WS and _gemv(lib, ws_bytes=16) == E_WS
+    assert _gemv(lib, ws=0x400010) == E_ALIGN
+
+
+def test_pack_argument_checks(lib):
+    P = ctypes.c_void_p
+    f = lib.qlin_pack_weights
+    assert f(2, 64, 256, P(0), None, 1.0, 0, P(0x1000), 1 << 30, None) == 1
+    assert f(3, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # NVFP4 needs scales
+    assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10010), 1 << 30, None) == 3
+    assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 10, None) == 1
+    assert f(2, 64, 256, P(0x1000), None, 1.0, 8, P(0x10000), 1 << 30, None) == 1
+
+
+def test_workspace_bytes_cover_partials(lib):
+    b1 = q.qlin_workspace_bytes(q.QLIN_OP_GEMV, q.QLIN_Q4_0, 1, 4096, 2560)
+    b8 = q.qlin_workspace_bytes(q.QLIN_OP_GEMV, q.QLIN_Q4_0, 8, 4096, 2560)
+    assert 0 < b1 < b8
+    assert q.qlin_workspace_bytes(q.QLIN_OP_GEMV, q.QLIN_Q4_0, 0, 4096, 2560) == 0

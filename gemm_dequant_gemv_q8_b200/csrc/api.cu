@@ -95,6 +95,7 @@ qlin_status_t qlin_gemv(qlin_format_t fmt, const void* packed, int64_t N, int64_
     if (!aligned(packed, 256) || !aligned(x, 16) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
     if (ldx % (xdt == QLIN_F32 ? 4 : 8)) return QLIN_ERR_ALIGNMENT;
     const int pack_flags = epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0;
+    if (qlin::geometry(fmt, N, K, pack_flags).U >= ((int64_t)1 << 31)) return QLIN_ERR_UNSUPPORTED;
     const size_t need = qlin_gemv_ws_bytes(fmt, M, N, K, pack_flags);
     if (!ws || ws_bytes < need) return QLIN_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;

@@ -107,10 +107,15 @@ __device__ __forceinline__ void flush_tile(const GemvArgs& a, int64_t t, int64_t
 }
 
 // ------------------------------------------------------------------ the kernel
+// Rows of x handled per pass is MP (1 or 2).  With MAXM <= 2 every row fits one pass: each lane
+// keeps its 8 row-part accumulators across all units of a tile (one FMA per block) and the
+// 8-lane reduce-scatter runs once per tile; x of the next unit is loaded while this one computes.
+// With MAXM > 2 the unit is processed in passes of two rows, each pass reduced at once.
 template <int FMT, int MAXM, bool XBF16, int EPI>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a) {
     using C = RingCfg<FMT>;
-    constexpr int MP = MAXM >= 2 ? 2 : 1;  // activation rows per pass
+    constexpr int MP = MAXM >= 2 ? 2 : 1;
+    constexpr bool kOnePass = MAXM <= 2;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* ring = smem + warp * C::D * C::UB;
@@ -121,9 +126,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
     // The per-tensor scale lives in the packed header (immutable, like the weights).
     const float gs = FMT == QLIN_NVFP4 ? reinterpret_cast<const PackedHeader*>(a.packed)->global_scale : 1.0f;
 
-    const int64_t gw = (int64_t)blockIdx.x * kGemvWarps + warp;
-    const int64_t ub = gw * a.U / a.Wt, ue = (gw + 1) * a.U / a.Wt;
-    const int64_t n = ue - ub;
+    const int U = (int)a.U, Wt = (int)a.Wt, G = (int)a.G;
+    const int gw = blockIdx.x * kGemvWarps + warp;
+    const int ub = (int)((int64_t)gw * U / Wt), ue = (int)((int64_t)(gw + 1) * U / Wt);
+    const int n = ue - ub;
     if (n <= 0) return;
 
     if (lane == 0) {
@@ -133,74 +139,114 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
         // Weight prefetch: independent of the previous kernel in the stream.
         for (int s = 0; s < C::D && s < n; ++s) {
             mbar_arrive_expect_tx(&bars[s], C::UB);
-            bulk_g2s(ring + s * C::UB, units + (ub + s) * C::UB, C::UB, &bars[s]);
+            bulk_g2s(ring + s * C::UB, units + (int64_t)(ub + s) * C::UB, C::UB, &bars[s]);
         }
     }
     __syncwarp();
     griddep_wait();  // x, y and the workspace may belong to the previous kernel
 
+    const int part = lane & 7;
+    int t = ub / G, g = ub - t * G;
     float acc[MAXM];
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
-    int64_t cur_t = ub / a.G;
-    bool failed = false;
-    int64_t j = 0;
-    for (; j < n; ++j) {
-        const int64_t u = ub + j;
-        const int64_t t = u / a.G, g = u - t * a.G;
-        if (t != cur_t) {
-            flush_tile<MAXM>(a, cur_t, gw, ub, ue, lane, acc, EPI, gs);
+    float acc8[8][MP];
+    float2 xv[MP][16];
+    const void* rows0[MP];
 #pragma unroll
-            for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
-            cur_t = t;
+    for (int mm = 0; mm < MP; ++mm)
+        rows0[mm] = (mm < a.M) ? (XBF16 ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.x) + mm * a.ldx)
+                                        : (const void*)(reinterpret_cast<const float*>(a.x) + mm * a.ldx))
+                               : nullptr;
+    if (kOnePass) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
+        load_x_rows<XBF16, MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xv);
+    }
+    bool failed = false;
+    int j = 0;
+    for (; j < n; ++j) {
+        int tn = t, gn = g + 1;
+        if (gn == G) {
+            gn = 0;
+            ++tn;
         }
-        const int slot = (int)(j % C::D);
+        float2 xn[MP][16];
+        if (kOnePass && j + 1 < n) load_x_rows<XBF16, MP>(rows0, (int64_t)gn * kGroupK + part * 32, a.K, xn);
+        const int slot = j % C::D;
         if (!mbar_wait_bounded(&bars[slot], (uint32_t)((j / C::D) & 1))) {
             failed = true;
             break;
         }
         const uint8_t* ubuf = ring + slot * C::UB;
-        const int64_t k0 = g * kGroupK + (lane & 7) * 32;
+        if (kOnePass) {
+            unit_dot<FMT, MP, true>(ubuf, lane, xv, acc8);
+        } else {
+            const int64_t k0 = (int64_t)g * kGroupK + part * 32;
 #pragma unroll 1
-        for (int m0 = 0; m0 < a.M; m0 += MP) {  // passes over pairs of activation rows
-            float2 xv[MP][16];
-            const void* rows[MP];
-#pragma unroll
-            for (int mm = 0; mm < MP; ++mm)
-                rows[mm] = (m0 + mm < a.M)
-                               ? (XBF16 ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.x) + (m0 + mm) * a.ldx)
-                                        : (const void*)(reinterpret_cast<const float*>(a.x) + (m0 + mm) * a.ldx))
-                               : nullptr;
-            load_x_rows<XBF16, MP>(rows, k0, a.K, xv);
-            float res[8][MP];
-            unit_dot<FMT, MP>(ubuf, lane, xv, res);
-            float r[MP];
-            reduce_scatter8<MP>(res, lane, r);
-#pragma unroll
-            for (int q = 0; q < MAXM; ++q)  // static register indexing of acc[m0 + mm]
+            for (int m0 = 0; m0 < a.M; m0 += MP) {  // passes over pairs of activation rows
+                float2 xp[MP][16];
+                const void* rows[MP];
 #pragma unroll
                 for (int mm = 0; mm < MP; ++mm)
-                    if (q == m0 + mm) acc[q] += r[mm];
+                    rows[mm] = (m0 + mm < a.M)
+                                   ? (XBF16 ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.x) + (m0 + mm) * a.ldx)
+                                            : (const void*)(reinterpret_cast<const float*>(a.x) + (m0 + mm) * a.ldx))
+                                   : nullptr;
+                load_x_rows<XBF16, MP>(rows, k0, a.K, xp);
+                float res[8][MP];
+                unit_dot<FMT, MP>(ubuf, lane, xp, res);
+                float r[MP];
+                reduce_scatter8<MP>(res, lane, r);
+#pragma unroll
+                for (int q = 0; q < MAXM; ++q)  // static register indexing of acc[m0 + mm]
+#pragma unroll
+                    for (int mm = 0; mm < MP; ++mm)
+                        if (q == m0 + mm) acc[q] += r[mm];
+            }
         }
         __syncwarp();
         if (lane == 0 && j + C::D < n) {
             fence_proxy_async_smem();
             mbar_arrive_expect_tx(&bars[slot], C::UB);
-            bulk_g2s(ring + slot * C::UB, units + (u + C::D) * C::UB, C::UB, &bars[slot]);
+            bulk_g2s(ring + slot * C::UB, units + (int64_t)(ub + j + C::D) * C::UB, C::UB, &bars[slot]);
+        }
+        if (tn != t || j + 1 == n) {  // last unit of tile t in this warp's range
+            if (kOnePass) {
+                float r[MP];
+                reduce_scatter8<MP>(acc8, lane, r);
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) acc[mm] = r[mm];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
+            }
+            flush_tile<MAXM>(a, t, gw, ub, ue, lane, acc, EPI, gs);
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
+        }
+        t = tn;
+        g = gn;
+        if (kOnePass) {
+#pragma unroll
+            for (int mm = 0; mm < MP; ++mm)
+#pragma unroll
+                for (int q = 0; q < 16; ++q) xv[mm][q] = xn[mm][q];
         }
     }
     if (failed) {
         // Report, then wait (bounded) for this warp's copies still in flight before exiting.
         if (lane == 0) {
             atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
-            const int64_t issued = (j + C::D < n) ? j + C::D : n;
-            for (int64_t q = j; q < issued; ++q)
+            const int issued = (j + C::D < n) ? j + C::D : n;
+            for (int q = j; q < issued; ++q)
                 mbar_wait_bounded(&bars[q % C::D], (uint32_t)((q / C::D) & 1), 100000000ull);
         }
         __syncwarp();
-        return;
     }
-    flush_tile<MAXM>(a, cur_t, gw, ub, ue, lane, acc, EPI, gs);
 }
 
 // ------------------------------------------------------------------ host side
@@ -222,15 +268,14 @@ struct GemvPlan {
     size_t ws_bytes;
 };
 
-constexpr int kGemvCtasPerSm = 2;
-
 static GemvPlan plan_gemv(int fmt, int M, int64_t N, int64_t K, int pack_flags) {
     GemvPlan p;
     Geometry geo = geometry(fmt, N, K, pack_flags);
     p.T = geo.T;
     p.G = geo.G;
     p.U = geo.U;
-    const int64_t wmax = (int64_t)sm_count_cached() * kGemvCtasPerSm * kGemvWarps;
+    const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
+    const int64_t wmax = (int64_t)sm_count_cached() * cps * kGemvWarps;
     int64_t wt = p.U < wmax ? p.U : wmax;
     p.grid = (int)((wt + kGemvWarps - 1) / kGemvWarps);
     p.Wt = wt;

@@ -10,9 +10,10 @@ constexpr int kGemvWarps = 4;  // warps per CTA
 
 template <int FMT>
 struct RingCfg {
-    static constexpr int D = (FMT == QLIN_Q8_0) ? 2 : 3;  // ring depth (units) per warp
+    static constexpr int D = 2;  // ring depth (units) per warp
     static constexpr int UB = unit_bytes(FMT);
     static constexpr int kSmem = kGemvWarps * D * (UB + 8);
+    static constexpr int kCtasPerSm = (FMT == QLIN_Q8_0) ? 3 : 4;  // 12-16 warps per SM
 };
 
 
@@ -91,8 +92,9 @@ __device__ __forceinline__ void load_x_rows(const void* const (&rows)[MP], int64
 }
 
 // ------------------------------------------------------------------ one unit, rows of one m-pass
-// res[i][mm] = contribution of (row (lane/8) + 4i, part lane%8) for activation row m0 + mm.
-template <int FMT, int MP>
+// res[i][mm] = contribution of (row (lane/8) + 4i, part lane%8) for activation row m0 + mm;
+// with ACC the contribution is added to res instead (one fused multiply-add per block).
+template <int FMT, int MP, bool ACC = false>
 __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const float2 (&xv)[MP][16],
                                          float (&res)[8][MP]) {
     const uint4 sv = lds128(ub + code_bytes(FMT) + lane * 16);
@@ -120,7 +122,10 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
             }
             const float d = fp16_bits_to_f32(sc & 0xffffu);
 #pragma unroll
-            for (int mm = 0; mm < MP; ++mm) res[i][mm] = d * ((s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y));
+            for (int mm = 0; mm < MP; ++mm) {
+                const float bsum = (s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y);
+                res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
+            }
         } else if (FMT == QLIN_Q8_0) {
             const uint4 c0 = lds128(ub + (lane + 32 * i) * 16);
             const uint4 c1 = lds128(ub + 4096 + (lane + 32 * i) * 16);
@@ -140,7 +145,10 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
             }
             const float d = fp16_bits_to_f32(sc & 0xffffu);
 #pragma unroll
-            for (int mm = 0; mm < MP; ++mm) res[i][mm] = d * ((s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y));
+            for (int mm = 0; mm < MP; ++mm) {
+                const float bsum = (s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y);
+                res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
+            }
         } else {  // NVFP4: two 16-element blocks per part, one E4M3 scale each
             const uint4 c = lds128(ub + (lane + 32 * i) * 16);
             const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
@@ -168,7 +176,8 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
             }
             const float e0 = e4m3_to_f32(sc & 0xffu), e1 = e4m3_to_f32((sc >> 8) & 0xffu);
 #pragma unroll
-            for (int mm = 0; mm < MP; ++mm) res[i][mm] = e0 * bs[0][mm] + e1 * bs[1][mm];
+            for (int mm = 0; mm < MP; ++mm)
+                res[i][mm] = ACC ? fmaf(e1, bs[1][mm], fmaf(e0, bs[0][mm], res[i][mm])) : e0 * bs[0][mm] + e1 * bs[1][mm];
         }
     }
 }

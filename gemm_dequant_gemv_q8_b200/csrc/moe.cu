@@ -19,7 +19,6 @@
 namespace qlin {
 
 constexpr int kMoeMaxTopK = 8;
-constexpr int kMoeMaxE = 256;
 constexpr int kMoeMaxM = 8;
 constexpr int kMoeMaxAct = kMoeMaxM * kMoeMaxTopK;
 
@@ -368,7 +367,8 @@ static MoePlan plan_moe(int fmt, int M, int64_t H, int64_t I, int E, int top_k, 
     p.nmax = (int64_t)M * top_k < E ? (int64_t)M * top_k : E;
     p.T0 = g0.T; p.G0 = g0.G; p.Ue0 = g0.U;
     p.T1 = g1.T; p.G1 = g1.G; p.Ue1 = g1.U;
-    p.Wt = (int64_t)moe_sm_count() * 2 * kGemvWarps;
+    const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
+    p.Wt = (int64_t)moe_sm_count() * cps * kGemvWarps;
     p.grid = (int)(p.Wt / kGemvWarps);
     auto smax_for = [&](int64_t Ue, int64_t G) {
         int64_t per = Ue / p.Wt;  // smallest per-warp share: one active expert

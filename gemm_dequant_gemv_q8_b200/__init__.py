@@ -37,6 +37,7 @@ SIGNATURES = {
     "qlin_pack_weights": (_I, [_I, _I64, _I64, _P, _P, _F, _I, _P, _SZ, _P]),
     "qlin_workspace_bytes": (_SZ, [_I, _I, _I, _I64, _I64, _I, _I]),
     "qlin_gemv": (_I, [_I, _P, _I64, _I64, _P, _I, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
+    "qlin_gemv_noalloc": (_I, [_I, _P, _I64, _I64, _P, _I, _I, _I64, _P, _I64, _I, _P]),
     "qlin_moe_experts": (_I, [_I, _P, _P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P, _I, _P, _SZ, _P]),
     "qlin_dequant_debug": (_I, [_I, _P, _I64, _I64, _I, _P, _P]),
     "qlin_ws_status": (_I, [_P, _P]),

@@ -361,3 +361,67 @@ extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, 
     if (fmt == QLIN_Q8_0) return launch_fmt<QLIN_Q8_0>(a, bf16, epi, p.grid, s, pdl);
     return launch_fmt<QLIN_NVFP4>(a, bf16, epi, p.grid, s, pdl);
 }
+
+// ------------------------------------------------------------------ allocation-free variant
+// qlin_gemv_noalloc: the same GEMV for callers that cannot allocate device memory themselves.
+// Its workspace is a fixed array in the library's own device memory (held by every GPU that
+// loads the library, until the process exits) instead of a caller-provided buffer.
+#include <mutex>
+
+namespace qlin {
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+static void* g_noalloc_addr[64] = {nullptr};  // device address of the array, per device
+static std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (looked up once per device; in host
+// code the array's name is only a stand-in, never a device address).
+static cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+}  // namespace qlin
+
+extern "C" qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
+                                           const void* x, qlin_dtype_t xdt, int M, int64_t ldx, float* y,
+                                           int64_t ldy, int flags, qlin_stream_t stream) {
+    if (fmt != QLIN_Q8_0 && fmt != QLIN_Q4_0 && fmt != QLIN_NVFP4) return QLIN_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || N > ((int64_t)1 << 31) || K > ((int64_t)1 << 31)) return QLIN_ERR_INVALID_ARG;
+    if (fmt == QLIN_NVFP4 ? (K % 16) : (K % 32)) return QLIN_ERR_INVALID_ARG;
+    if (M < 1 || M > 8) return QLIN_ERR_INVALID_ARG;
+    if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
+    const int epi = flags & 0xff;
+    if (epi != QLIN_EPI_NONE && epi != QLIN_EPI_SILU_GATE) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~(0xff | QLIN_FLAG_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (epi == QLIN_EPI_SILU_GATE && (N % 2)) return QLIN_ERR_INVALID_ARG;
+    if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
+    const int64_t ncols = epi == QLIN_EPI_SILU_GATE ? N / 2 : N;
+    if (ldx < K || ldy < ncols) return QLIN_ERR_INVALID_ARG;
+    if ((uintptr_t)packed % 256 || (uintptr_t)x % 16 || (uintptr_t)y % 4) return QLIN_ERR_ALIGNMENT;
+    if (ldx % (xdt == QLIN_F32 ? 4 : 8)) return QLIN_ERR_ALIGNMENT;
+    const int pack_flags = epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0;
+    if (geometry(fmt, N, K, pack_flags).U >= ((int64_t)1 << 31)) return QLIN_ERR_UNSUPPORTED;
+    const GemvPlan p = plan_gemv(fmt, M, N, K, pack_flags);
+    if (p.ws_bytes > kNoAllocScratchBytes) return QLIN_ERR_WORKSPACE;  // beyond the fixed maximum
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return QLIN_ERR_CUDA;
+    // The array keeps the previous call's contents: the status word and the tile tickets must
+    // start at zero (the partial sums are always written before they are read).
+    if (cudaMemsetAsync(scratch, 0, (size_t)ws_partials_off(p.T), (cudaStream_t)stream) != cudaSuccess)
+        return QLIN_ERR_CUDA;
+    return qlin_launch_gemv(fmt, packed, N, K, x, xdt, M, ldx, y, ldy, flags, scratch, (cudaStream_t)stream) ==
+                   cudaSuccess
+               ? QLIN_OK
+               : QLIN_ERR_CUDA;
+}

@@ -116,6 +116,25 @@ qlin_status_t qlin_gemv(qlin_format_t fmt, const void* packed, int64_t N, int64_
                         qlin_dtype_t xdt, int M, int64_t ldx, float* y, int64_t ldy, int flags,
                         void* ws, size_t ws_bytes, qlin_stream_t stream);
 
+/* Allocation-free variant of qlin_gemv.  The pages have no counterpart: this entry point exists
+ * for callers that cannot allocate device memory for a workspace -- for example a plugin inside
+ * a host application that owns every device allocation and hands out only the tensors it
+ * manages, or a latency-critical decode loop that must not call cudaMalloc (which can
+ * synchronise the device) once it is running.  Same arguments, semantics and results as
+ * qlin_gemv, minus the workspace: the split-tile partial sums and tickets live in a fixed 8 MiB
+ * array of the library's own device memory, which every GPU that loads the library holds until
+ * the process exits.  It calls no cudaMalloc / cudaFree and no allocating library routine.
+ *   - A shape whose workspace (qlin_workspace_bytes(QLIN_OP_GEMV, ...)) exceeds 8 MiB is rejected
+ *     with QLIN_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call clears the array's status word and tickets on `stream` (cudaMemsetAsync), then
+ *     launches the kernel.  All calls share the one array: calls that can overlap on the GPU
+ *     (different streams without ordering between them) race and must not be issued. */
+qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
+                                const void* x, qlin_dtype_t xdt, int M, int64_t ldx, float* y,
+                                int64_t ldy, int flags, qlin_stream_t stream);
+
 /* ------------------------------------------------------------------------- routed MoE experts */
 
 /* Top-k routed MoE expert projections for M = 1..8 tokens.  Follows the Imparo README intro (a

@@ -264,6 +264,113 @@ def cpu_baseline_stack(fmt, budget_s=12.0, seed=7):
     return gbs, 1, desc
 
 
+
+# ----------------------------------------------------------------------------- other configs
+def _time_graph_of(fn, steps, warmup):
+    """Capture fn() (a sequence of launches) in one CUDA graph and time replays with events."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    ms = time_graph(g, steps, warmup)
+    del g
+    return ms
+
+
+def run_config(name, args):
+    """Measure one of the non-default workloads; one JSON line per (config, M)."""
+    import gemm_dequant_gemv_q8_b200 as q
+    torch.cuda.set_device(0)
+    peak, peak_src = peaks()
+    lines = []
+    if name == "q8_small":
+        fmt, N, K, M, copies = q.QLIN_Q8_0, 256, 1024, 1, 1000  # 278 MB of rotating copies > 2x L2
+        packs = []
+        for c in range(copies):
+            b, s_, g = synth.weights(fmt, N, K, synth.gen(1000 + c, device="cuda"), device="cuda")
+            packs.append(q.qlin_pack_weights(fmt, N, K, b, s_, g))
+        x = synth.activations(M, K, synth.gen(1, device="cuda"), device="cuda")
+        y = torch.empty(M, N, device="cuda")
+        ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, N, K)) for _ in range(copies)]
+        fn = lambda: [q.qlin_gemv(fmt, packs[c], N, K, x, y=y, ws=ws[c], flags=q.QLIN_FLAG_PDL) for c in range(copies)]
+        ms = _time_graph_of(fn, max(3, args.steps // 4), args.warmup) / copies
+        wb = q.qlin_packed_bytes(fmt, N, K) - 256
+        bytes_ = wb + 4 * M * (K + N)
+        lines.append(dict(workload="Q8_0 GEMV M=1 K=1024 N=256 (launch-latency bound; graph of 1000 "
+                          "launches over distinct weight copies, PDL)", M=M, us_per_launch=ms * 1e3,
+                          gbs=bytes_ / (ms * 1e-3) / 1e9))
+    elif name == "nvfp4_mlp":
+        fmt, H, I = q.QLIN_NVFP4, 5120, 17408
+        for M in (1, 4):
+            L = 2
+            gu, dn, wsg, wsd = [], [], [], []
+            for l in range(L):
+                b, s_, g = synth.weights(fmt, 2 * I, H, synth.gen(3000 + l, device="cuda"), device="cuda")
+                gu.append(q.qlin_pack_weights(fmt, 2 * I, H, b, s_, g, q.QLIN_PACK_GATE_UP))
+                b, s_, g = synth.weights(fmt, H, I, synth.gen(3100 + l, device="cuda"), device="cuda")
+                dn.append(q.qlin_pack_weights(fmt, H, I, b, s_, g))
+                wsg.append(q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, 2 * I, H)))
+                wsd.append(q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, H, I)))
+            x = synth.activations(M, H, synth.gen(3200, device="cuda"), dtype=torch.bfloat16, device="cuda")
+            h = torch.empty(M, I, device="cuda")
+            y = torch.empty(M, H, device="cuda")
+
+            def fn():
+                for l in range(L):
+                    q.qlin_gemv(fmt, gu[l], 2 * I, H, x, y=h, ws=wsg[l], flags=q.QLIN_EPI_SILU_GATE | q.QLIN_FLAG_PDL)
+                    q.qlin_gemv(fmt, dn[l], H, I, h, y=y, ws=wsd[l], flags=q.QLIN_FLAG_PDL)
+            ms = _time_graph_of(fn, args.steps, args.warmup) / L
+            wb = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
+            bytes_ = wb + M * (2 * H + 4 * I + 4 * I + 4 * H)
+            lines.append(dict(workload="NVFP4 MLP shaped like a 27B model: gate_up 5120->2x17408 + SiLU, "
+                              "down 17408->5120, bf16 activations", M=M, us_per_layer=ms * 1e3,
+                              gbs=bytes_ / (ms * 1e-3) / 1e9, tokens_per_s=M / (ms * 1e-3)))
+            del gu, dn
+    elif name == "moe":
+        fmt, E, H, I, k = q.QLIN_Q4_0, 32, 2048, 1792, 4
+        L = 2
+        canon_gu = [[synth.weights(fmt, 2 * I, H, synth.gen(4000 + 100 * l + e, device="cuda"), device="cuda")
+                     for e in range(E)] for l in range(L)]
+        gu = [q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_GATE_UP) for c in canon_gu]
+        del canon_gu
+        canon_dn = [[synth.weights(fmt, H, I, synth.gen(5000 + 100 * l + e, device="cuda"), device="cuda")
+                     for e in range(E)] for l in range(L)]
+        dn = [q.pack_experts(fmt, E, H, I, c) for c in canon_dn]
+        del canon_dn
+        per_expert = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
+        for M in (1, 8):
+            logits = [synth.router_logits(M, E, synth.gen(6000 + l, device="cuda"), device="cuda") for l in range(L)]
+            x = synth.activations(M, H, synth.gen(6100, device="cuda"), device="cuda")
+            ids = torch.empty(M, k, dtype=torch.int32, device="cuda")
+            w = torch.empty(M, k, device="cuda")
+            y = torch.empty(M, H, device="cuda")
+            ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE, fmt, M, H, I, E, k)) for _ in range(L)]
+            distinct = []
+
+            def fn():
+                for l in range(L):
+                    q.qlin_moe_experts(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
+                                       topk_w=w, y=y, ws=ws[l], flags=q.QLIN_FLAG_PDL)
+            ms = _time_graph_of(fn, args.steps, args.warmup) / L
+            for l in range(L):  # actual distinct experts per layer for these seeds
+                q.qlin_moe_experts(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
+                                   topk_w=w, y=y, ws=ws[l])
+                distinct.append(len(set(ids.cpu().flatten().tolist())))
+            nd = sum(distinct) / L
+            bytes_ = nd * per_expert + M * (4 * H + 4 * H + 4 * E)
+            lines.append(dict(workload="Q4_0 MoE expert layer shaped like an 8B-A1B model: hidden 2048, 32 experts "
+                              "gate_up 2048->2x1792, down 1792->2048, top-4", M=M, distinct_experts=nd,
+                              us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9))
+    for ln in lines:
+        ln.update(metric=METRIC, unit="GB/s", value=ln["gbs"], hbm_frac=ln["gbs"] / peak,
+                  peak=peak, peak_source=peak_src, config=name, impl="qlin", n_gpus=1)
+        print(json.dumps(ln), flush=True)
+
 # ----------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -274,7 +381,12 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "moe"],
+                    help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
+    if args.config != "stack":
+        run_config(args.config, args)
+        return
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -29,7 +29,7 @@ struct GemvArgs {
     float* y;
     int64_t ldy;
     uint8_t* ws;
-    int64_t Wt;   // total warps sharing the units
+    int64_t Wt;   // number of CTAs sharing the units
     int smax;     // partial slots per tile
 };
 
@@ -66,23 +66,19 @@ __device__ __forceinline__ void write_tile(const GemvArgs& a, int64_t t, int lan
 __host__ __device__ inline int64_t ws_counters_off() { return 256; }
 __host__ __device__ inline int64_t ws_partials_off(int64_t T) { return 256 + ((4 * T + 255) / 256) * 256; }
 
+// Global split-tile fixup between CTAs: store this CTA's partial of tile t, take a ticket; the
+// CTA that arrives last sums every partial in CTA order (deterministic) and writes the tile.
 template <int MAXM>
-__device__ __forceinline__ void flush_tile(const GemvArgs& a, int64_t t, int64_t gw, int64_t ub,
-                                           int64_t ue, int lane, float (&acc)[MAXM], int epi,
-                                           float gs) {
+__device__ __forceinline__ void global_fixup(const GemvArgs& a, int64_t t, int64_t c, int lane,
+                                             float (&acc)[MAXM], int epi, float gs) {
     const int64_t f = t * a.G, l = f + a.G - 1;
-    if (f >= ub && l < ue) {  // whole tile inside this warp's range
-        write_tile<MAXM>(a, t, lane, acc, epi, gs);
-        return;
-    }
-    const int64_t c_first = ((f + 1) * a.Wt - 1) / a.U;
-    const int64_t c_last = ((l + 1) * a.Wt - 1) / a.U;
+    const int64_t C = a.Wt;  // number of CTAs sharing the units
+    const int64_t c_first = ((f + 1) * C - 1) / a.U, c_last = ((l + 1) * C - 1) / a.U;
     const int n_t = (int)(c_last - c_first + 1);
-    const int slot = (int)(gw - c_first);
-    const int row = (lane >> 3) + 4 * (lane & 7);
+    const int slot = (int)(c - c_first);
     float* part = reinterpret_cast<float*>(a.ws + ws_partials_off(a.T));
     int* cnt = reinterpret_cast<int*>(a.ws + ws_counters_off());
-    float* mine = part + ((t * a.smax + slot) * 32 + row) * a.M;
+    float* mine = part + ((t * a.smax + slot) * 32 + lane) * a.M;
 #pragma unroll
     for (int m = 0; m < MAXM; ++m)
         if (m < a.M) __stcg(mine + m, acc[m]);
@@ -97,7 +93,7 @@ __device__ __forceinline__ void flush_tile(const GemvArgs& a, int64_t t, int64_t
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) sum[m] = 0.f;
     for (int s = 0; s < n_t; ++s) {
-        const float* src = part + ((t * a.smax + s) * 32 + row) * a.M;
+        const float* src = part + ((t * a.smax + s) * 32 + lane) * a.M;
 #pragma unroll
         for (int m = 0; m < MAXM; ++m)
             if (m < a.M) sum[m] += __ldcg(src + m);
@@ -107,16 +103,21 @@ __device__ __forceinline__ void flush_tile(const GemvArgs& a, int64_t t, int64_t
 }
 
 // ------------------------------------------------------------------ the kernel
-// Rows of x handled per pass is MP (1 or 2).  With MAXM <= 2 every row fits one pass: each lane
-// keeps its 8 row-part accumulators across all units of a tile (one FMA per block) and the
-// 8-lane reduce-scatter runs once per tile; x of the next unit is loaded while this one computes.
-// With MAXM > 2 the unit is processed in passes of two rows, each pass reduced at once.
+// Work split: CTA c owns the contiguous units [c U / C, (c+1) U / C); its warp w owns the w-th
+// quarter of that range.  A tile wholly inside one warp's range is written by that warp.  A tile
+// shared by warps of one CTA is combined in shared memory, in warp order, after one barrier; only
+// tiles at the CTA's two ends can be shared with other CTAs and go through the global fixup.
+// Rows of x per pass is MP (1 or 2).  With MAXM <= 2 all rows fit one pass: each lane keeps its 8
+// row-part accumulators across the units of a tile (one FMA per block) and reduces once per tile;
+// x of the next unit loads while this one computes.  With MAXM > 2 each pass reduces at once.
 template <int FMT, int MAXM, bool XBF16, int EPI>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a) {
     using C = RingCfg<FMT>;
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     constexpr bool kOnePass = MAXM <= 2;
+    constexpr bool kH = (FMT == QLIN_NVFP4) && XBF16;  // f16-product path (see load_x_fp4h)
     extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ float slots[kGemvWarps][2][32][MAXM];  // warp-boundary tile partials
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t* ring = smem + warp * C::D * C::UB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemvWarps * C::D * C::UB) + warp * C::D;
@@ -126,13 +127,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
     // The per-tensor scale lives in the packed header (immutable, like the weights).
     const float gs = FMT == QLIN_NVFP4 ? reinterpret_cast<const PackedHeader*>(a.packed)->global_scale : 1.0f;
 
-    const int U = (int)a.U, Wt = (int)a.Wt, G = (int)a.G;
-    const int gw = blockIdx.x * kGemvWarps + warp;
-    const int ub = (int)((int64_t)gw * U / Wt), ue = (int)((int64_t)(gw + 1) * U / Wt);
+    const int U = (int)a.U, nC = (int)a.Wt, G = (int)a.G;
+    const int cu0 = (int)((int64_t)blockIdx.x * U / nC), cu1 = (int)((int64_t)(blockIdx.x + 1) * U / nC);
+    const int ub = cu0 + (int)((int64_t)warp * (cu1 - cu0) / kGemvWarps);
+    const int ue = cu0 + (int)((int64_t)(warp + 1) * (cu1 - cu0) / kGemvWarps);
     const int n = ue - ub;
-    if (n <= 0) return;
 
-    if (lane == 0) {
+    if (lane == 0 && n > 0) {
 #pragma unroll
         for (int s = 0; s < C::D; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
@@ -146,12 +147,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
     griddep_wait();  // x, y and the workspace may belong to the previous kernel
 
     const int part = lane & 7;
-    int t = ub / G, g = ub - t * G;
+    int t = n > 0 ? ub / G : 0, g = n > 0 ? ub - t * G : 0;
+    const int t_first = t, t_last = n > 0 ? (ue - 1) / G : -1;
     float acc[MAXM];
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
     float acc8[8][MP];
     float2 xv[MP][16];
+    uint32_t xh[MP][16];
+    float xsc[MP][2];
     const void* rows0[MP];
 #pragma unroll
     for (int mm = 0; mm < MP; ++mm)
@@ -163,7 +167,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
         for (int i = 0; i < 8; ++i)
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
-        load_x_rows<XBF16, MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xv);
+        if (n > 0) {
+            if constexpr (kH) {
+                load_x_fp4h<MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xh, xsc);
+            } else {
+                load_x_rows<XBF16, MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xv);
+                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xv);
+            }
+        }
     }
     bool failed = false;
     int j = 0;
@@ -174,7 +185,16 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
             ++tn;
         }
         float2 xn[MP][16];
-        if (kOnePass && j + 1 < n) load_x_rows<XBF16, MP>(rows0, (int64_t)gn * kGroupK + part * 32, a.K, xn);
+        uint32_t xhn[MP][16];
+        float xscn[MP][2];
+        if (kOnePass && j + 1 < n) {
+            if constexpr (kH) {
+                load_x_fp4h<MP>(rows0, (int64_t)gn * kGroupK + part * 32, a.K, xhn, xscn);
+            } else {
+                load_x_rows<XBF16, MP>(rows0, (int64_t)gn * kGroupK + part * 32, a.K, xn);
+                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xn);
+            }
+        }
         const int slot = j % C::D;
         if (!mbar_wait_bounded(&bars[slot], (uint32_t)((j / C::D) & 1))) {
             failed = true;
@@ -182,7 +202,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
         }
         const uint8_t* ubuf = ring + slot * C::UB;
         if (kOnePass) {
-            unit_dot<FMT, MP, true>(ubuf, lane, xv, acc8);
+            if constexpr (kH) unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+            else unit_dot<FMT, MP, true>(ubuf, lane, xv, acc8);
         } else {
             const int64_t k0 = (int64_t)g * kGroupK + part * 32;
 #pragma unroll 1
@@ -195,9 +216,17 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
                                    ? (XBF16 ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.x) + (m0 + mm) * a.ldx)
                                             : (const void*)(reinterpret_cast<const float*>(a.x) + (m0 + mm) * a.ldx))
                                    : nullptr;
-                load_x_rows<XBF16, MP>(rows, k0, a.K, xp);
                 float res[8][MP];
-                unit_dot<FMT, MP>(ubuf, lane, xp, res);
+                if constexpr (kH) {
+                    uint32_t xph[MP][16];
+                    float xps[MP][2];
+                    load_x_fp4h<MP>(rows, k0, a.K, xph, xps);
+                    unit_dot_fp4h<MP>(ubuf, lane, xph, xps, res);
+                } else {
+                    load_x_rows<XBF16, MP>(rows, k0, a.K, xp);
+                    if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xp);
+                    unit_dot<FMT, MP>(ubuf, lane, xp, res);
+                }
                 float r[MP];
                 reduce_scatter8<MP>(res, lane, r);
 #pragma unroll
@@ -224,7 +253,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
 #pragma unroll
                     for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
             }
-            flush_tile<MAXM>(a, t, gw, ub, ue, lane, acc, EPI, gs);
+            if ((int64_t)t * G >= ub && (int64_t)t * G + G <= ue) {
+                write_tile<MAXM>(a, t, lane, acc, EPI, gs);  // whole tile inside this warp
+            } else {
+                const int k = (t == t_first) ? 0 : 1;  // shared tiles are a warp's first or last
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m) slots[warp][k][lane][m] = acc[m];
+            }
 #pragma unroll
             for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
         }
@@ -232,20 +267,50 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
         g = gn;
         if (kOnePass) {
 #pragma unroll
-            for (int mm = 0; mm < MP; ++mm)
+            for (int mm = 0; mm < MP; ++mm) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) xv[mm][q] = xn[mm][q];
+                for (int q = 0; q < 16; ++q) {
+                    if constexpr (kH) xh[mm][q] = xhn[mm][q];
+                    else xv[mm][q] = xn[mm][q];
+                }
+                if constexpr (kH) { xsc[mm][0] = xscn[mm][0]; xsc[mm][1] = xscn[mm][1]; }
+            }
         }
     }
-    if (failed) {
-        // Report, then wait (bounded) for this warp's copies still in flight before exiting.
-        if (lane == 0) {
-            atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
-            const int issued = (j + C::D < n) ? j + C::D : n;
-            for (int q = j; q < issued; ++q)
-                mbar_wait_bounded(&bars[q % C::D], (uint32_t)((q / C::D) & 1), 100000000ull);
+    if (failed && lane == 0) {
+        // Report, then wait (bounded) for this warp's copies still in flight.
+        atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
+        const int issued = (j + C::D < n) ? j + C::D : n;
+        for (int q = j; q < issued; ++q)
+            mbar_wait_bounded(&bars[q % C::D], (uint32_t)((q / C::D) & 1), 100000000ull);
+    }
+    __syncthreads();  // every warp reaches this, with or without units
+    if (failed || n <= 0) return;
+    // Combine the tiles this warp is the lowest-index toucher of and that it does not own whole.
+    const int range_len = cu1 - cu0;
+#pragma unroll 1
+    for (int k = 0; k < 2; ++k) {
+        const int tt = k == 0 ? t_first : t_last;
+        if (k == 1 && t_last == t_first) break;
+        const int64_t f = (int64_t)tt * G;
+        if (f >= ub && f + G <= ue) continue;  // owned whole by this warp, already written
+        // The nearest lower warp with units ends exactly at ub, so a lower warp of this CTA touches
+        // the tile iff f < ub and some lower warp has units (ub > cu0).  Then it combines instead.
+        if (f < ub && ub > cu0) continue;
+        float sum[MAXM];
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) sum[m] = 0.f;
+        for (int w2 = warp; w2 < kGemvWarps; ++w2) {
+            const int b2 = cu0 + (int)((int64_t)w2 * range_len / kGemvWarps);
+            const int e2 = cu0 + (int)((int64_t)(w2 + 1) * range_len / kGemvWarps);
+            if (e2 <= b2) continue;
+            if (b2 >= f + G) break;                      // past the tile
+            const int k2 = (b2 / G == tt) ? 0 : 1;        // tt is w2's first or last tile
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) sum[m] += slots[w2][k2][lane][m];
         }
-        __syncwarp();
+        if (f >= cu0 && f + G <= cu1) write_tile<MAXM>(a, tt, lane, sum, EPI, gs);
+        else global_fixup<MAXM>(a, tt, blockIdx.x, lane, sum, EPI, gs);
     }
 }
 
@@ -275,13 +340,15 @@ static GemvPlan plan_gemv(int fmt, int M, int64_t N, int64_t K, int pack_flags) 
     p.G = geo.G;
     p.U = geo.U;
     const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
-    const int64_t wmax = (int64_t)sm_count_cached() * cps * kGemvWarps;
-    int64_t wt = p.U < wmax ? p.U : wmax;
-    p.grid = (int)((wt + kGemvWarps - 1) / kGemvWarps);
-    p.Wt = wt;
-    const int64_t per = p.U / p.Wt;  // >= 1
+    const int64_t cmax = (int64_t)sm_count_cached() * cps;
+    int64_t c = (p.U + kGemvWarps - 1) / kGemvWarps;  // at least one unit per warp
+    if (c > cmax) c = cmax;
+    if (c < 1) c = 1;
+    p.grid = (int)c;
+    p.Wt = c;  // the kernel splits units between CTAs, then between a CTA's warps
+    const int64_t per = p.U / c;  // >= 1 unit per CTA
     int64_t smax = (p.G + per - 1) / per + 1;
-    if (smax > p.Wt) smax = p.Wt;
+    if (smax > c) smax = c;
     p.smax = (int)smax;
     p.ws_bytes = (size_t)ws_partials_off(p.T) + (size_t)p.T * p.smax * 32 * (M > 0 ? M : 1) * 4;
     return p;

@@ -308,11 +308,19 @@ __global__ void __launch_bounds__(kGemvWarps * 32) moe_kernel(const MoeArgs a) {
                     rows[mm] = a.h + ((int64_t)r.row_m[act][q] * a.top_k + r.row_s[act][q]) * a.I;
                 }
             }
-            float2 xv[MP][16];
             constexpr bool kXB = (PHASE == 0) && XBF16;
-            load_x_rows<kXB, MP>(rows, k0, a.Kin, xv);
             float res[8][MP];
-            unit_dot<FMT, MP>(ubuf, lane, xv, res);
+            if constexpr (kXB && FMT == QLIN_NVFP4) {
+                uint32_t xh[MP][16];
+                float xsc[MP][2];
+                load_x_fp4h<MP>(rows, k0, a.Kin, xh, xsc);
+                unit_dot_fp4h<MP>(ubuf, lane, xh, xsc, res);
+            } else {
+                float2 xv[MP][16];
+                load_x_rows<kXB, MP>(rows, k0, a.Kin, xv);
+                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xv);
+                unit_dot<FMT, MP>(ubuf, lane, xv, res);
+            }
             float rr[MP];
             reduce_scatter8<MP>(res, lane, rr);
 #pragma unroll

@@ -19,7 +19,7 @@ import torch
 QLIN_Q8_0, QLIN_Q4_0, QLIN_NVFP4 = 1, 2, 3
 QLIN_F32, QLIN_BF16 = 0, 1
 QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_FLAG_PDL = 0, 1, 0x100
-QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP = 0, 1
+QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA = 0, 1, 2
 QLIN_OP_GEMV, QLIN_OP_MOE, QLIN_OP_CHUNK = 1, 2, 3
 STATUS = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED",
           3: "QLIN_ERR_ALIGNMENT", 4: "QLIN_ERR_WORKSPACE", 5: "QLIN_ERR_CUDA",
@@ -39,6 +39,8 @@ SIGNATURES = {
     "qlin_gemv": (_I, [_I, _P, _I64, _I64, _P, _I, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "qlin_gemv_noalloc": (_I, [_I, _P, _I64, _I64, _P, _I, _I, _I64, _P, _I64, _I, _P]),
     "qlin_moe_experts": (_I, [_I, _P, _P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P, _I, _P, _SZ, _P]),
+    "qlin_gemm_chunk": (_I, [_I, _P, _I64, _I64, _P, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
+    "qlin_act_quant_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "qlin_dequant_debug": (_I, [_I, _P, _I64, _I64, _I, _P, _P]),
     "qlin_ws_status": (_I, [_P, _P]),
     "qlin_status_string": (ctypes.c_char_p, [_I]),
@@ -181,6 +183,36 @@ def pack_experts(fmt, E, N, K, canon, pack_flags=QLIN_PACK_DEFAULT, stream=None)
     for e, (b, s, g) in enumerate(canon):
         qlin_pack_weights(fmt, N, K, b, s, g, pack_flags, packed=buf[e * stride:(e + 1) * stride], stream=stream)
     return buf
+
+
+def qlin_gemm_chunk(fmt, packed, N, K, x, y=None, flags=0, ws=None, stream=None):
+    """NVFP4 prefill-chunk GEMM: y (M, N) fp32 = quantized x (M, K) bf16 times W^T."""
+    if x.dtype != torch.bfloat16 or x.stride(1) != 1:
+        raise TypeError("x must be bfloat16 with contiguous rows")
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(qlin_workspace_bytes(QLIN_OP_CHUNK, fmt, M, N, K), x.device)
+    st = lib().qlin_gemm_chunk(fmt, _dev(packed, "packed"), N, K, _dev(x, "x"), M, x.stride(0),
+                               _dev(y, "y", torch.float32), y.stride(0), flags, _dev(ws, "ws"),
+                               ws.numel() * ws.element_size(), _stream(stream))
+    _check("qlin_gemm_chunk", st)
+    return y
+
+
+def qlin_act_quant_debug(x, ws=None, stream=None):
+    """Quantized activations of the chunk path in the canonical layout: (codes, scales, a_g)."""
+    M, K = x.shape
+    codes = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(M, K // 16, dtype=torch.uint8, device=x.device)
+    ag = torch.empty(1, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(qlin_workspace_bytes(QLIN_OP_CHUNK, QLIN_NVFP4, M, 256, K), x.device)
+    st = lib().qlin_act_quant_debug(_dev(x, "x"), M, K, x.stride(0), _dev(codes, "codes"), _dev(scales, "scales"),
+                                    _dev(ag, "a_g"), _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    _check("qlin_act_quant_debug", st)
+    return codes, scales, ag
 
 
 def qlin_dequant_debug(fmt, packed, N, K, pack_flags=QLIN_PACK_DEFAULT, stream=None):

@@ -14,6 +14,11 @@ extern "C" size_t qlin_moe_ws_bytes(int fmt, int M, int64_t H, int64_t I, int E,
 extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, int E, int64_t H, int64_t I,
                                        int top_k, const float* logits, int32_t* ids, float* wts, const void* x,
                                        int xdt, int M, float* y, float* h, int flags, void* ws, cudaStream_t s);
+extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K);
+extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
+                                         float* y, int64_t ldy, void* ws, int flags, cudaStream_t s);
+extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* ws,
+                                                   void* codes, void* scales, float* ag, cudaStream_t s);
 extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, int64_t K,
                                         const void* x, int xdt, int M, int64_t ldx, float* y,
                                         int64_t ldy, int flags, void* ws, cudaStream_t s);
@@ -39,6 +44,10 @@ extern "C" {
 
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags) {
     if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
+    if (pack_flags == QLIN_PACK_MMA) {
+        if (fmt != QLIN_NVFP4) return 0;
+        return (size_t)qlin::kHdrBytes + (size_t)((N + 255) / 256) * (size_t)((K + 255) / 256) * 36864u;
+    }
     if (pack_flags & ~QLIN_PACK_GATE_UP) return 0;
     if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return 0;
     qlin::Geometry g = qlin::geometry(fmt, N, K, pack_flags);
@@ -50,7 +59,8 @@ qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const v
                                 void* packed, size_t packed_bytes, qlin_stream_t stream) {
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
-    if (pack_flags & ~QLIN_PACK_GATE_UP) return QLIN_ERR_INVALID_ARG;
+    if (pack_flags == QLIN_PACK_MMA && fmt != QLIN_NVFP4) return QLIN_ERR_UNSUPPORTED;
+    if (pack_flags != QLIN_PACK_MMA && (pack_flags & ~QLIN_PACK_GATE_UP)) return QLIN_ERR_INVALID_ARG;
     if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
     if (!blocks || !packed) return QLIN_ERR_INVALID_ARG;
     if (fmt == QLIN_NVFP4 && !scales) return QLIN_ERR_INVALID_ARG;
@@ -69,6 +79,10 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
         if (M < 1 || M > 8 || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return 0;
         if (!valid_shape(fmt, 2 * K, N) || !valid_shape(fmt, N, K)) return 0;
         return qlin_moe_ws_bytes(fmt, M, N, K, E, top_k);
+    }
+    if (op == QLIN_OP_CHUNK) {
+        if (fmt != QLIN_NVFP4 || M < 1 || M > (1 << 20)) return 0;
+        return qlin_chunk_ws_bytes(M, N, K);
     }
     if (op == QLIN_OP_GEMV) {
         if (M < 1 || M > 8) return 0;
@@ -123,6 +137,29 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
     if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
     return cuda_status(qlin_launch_moe(fmt, gate_up_packed, down_packed, E, H, I, top_k, router_logits, topk_ids,
                                        topk_w, x, xdt, M, y, h, flags, ws, (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,
+                              int M, int64_t ldx, float* y, int64_t ldy, int flags, void* ws,
+                              size_t ws_bytes, qlin_stream_t stream) {
+    if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
+    if (fmt != QLIN_NVFP4) return QLIN_ERR_UNSUPPORTED;
+    if (!valid_shape(fmt, N, K) || M < 1 || M > (1 << 20)) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~QLIN_FLAG_PDL) return QLIN_ERR_INVALID_ARG;
+    if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
+    if (ldx < K || ldy < N) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(packed, 256) || !aligned(x, 2) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
+    if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, N, K)) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_chunk(packed, N, K, x, M, ldx, y, ldy, ws, flags, (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* codes, void* scales,
+                                   float* a_g, void* ws, size_t ws_bytes, qlin_stream_t stream) {
+    if (!x || !codes || !scales || !a_g || M < 1 || K < 16 || K % 16 || ldx < K) return QLIN_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, 256, K)) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256) || !aligned(codes, 8) || !aligned(a_g, 4)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_act_quant_debug(x, M, K, ldx, ws, codes, scales, a_g, (cudaStream_t)stream));
 }
 
 qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,

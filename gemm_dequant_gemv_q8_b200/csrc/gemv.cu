@@ -108,8 +108,8 @@ __device__ __forceinline__ void global_fixup(const GemvArgs& a, int64_t t, int64
 // shared by warps of one CTA is combined in shared memory, in warp order, after one barrier; only
 // tiles at the CTA's two ends can be shared with other CTAs and go through the global fixup.
 // Rows of x per pass is MP (1 or 2).  With MAXM <= 2 all rows fit one pass: each lane keeps its 8
-// row-part accumulators across the units of a tile (one FMA per block) and reduces once per tile;
-// x of the next unit loads while this one computes.  With MAXM > 2 each pass reduces at once.
+// row-part accumulators across the units of a tile (one FMA per block) and reduces once per tile.
+// With MAXM > 2 each pass reduces at once.
 template <int FMT, int MAXM, bool XBF16, int EPI>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a) {
     using C = RingCfg<FMT>;
@@ -184,23 +184,20 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
             gn = 0;
             ++tn;
         }
-        float2 xn[MP][16];
-        uint32_t xhn[MP][16];
-        float xscn[MP][2];
-        if (kOnePass && j + 1 < n) {
-            if constexpr (kH) {
-                load_x_fp4h<MP>(rows0, (int64_t)gn * kGroupK + part * 32, a.K, xhn, xscn);
-            } else {
-                load_x_rows<XBF16, MP>(rows0, (int64_t)gn * kGroupK + part * 32, a.K, xn);
-                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xn);
-            }
-        }
         const int slot = j % C::D;
         if (!mbar_wait_bounded(&bars[slot], (uint32_t)((j / C::D) & 1))) {
             failed = true;
             break;
         }
         const uint8_t* ubuf = ring + slot * C::UB;
+        if (kOnePass && j > 0) {  // activations of this unit (the first unit's were loaded above)
+            if constexpr (kH) {
+                load_x_fp4h<MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xh, xsc);
+            } else {
+                load_x_rows<XBF16, MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xv);
+                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xv);
+            }
+        }
         if (kOnePass) {
             if constexpr (kH) unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
             else unit_dot<FMT, MP, true>(ubuf, lane, xv, acc8);
@@ -265,17 +262,6 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
         }
         t = tn;
         g = gn;
-        if (kOnePass) {
-#pragma unroll
-            for (int mm = 0; mm < MP; ++mm) {
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    if constexpr (kH) xh[mm][q] = xhn[mm][q];
-                    else xv[mm][q] = xn[mm][q];
-                }
-                if constexpr (kH) { xsc[mm][0] = xscn[mm][0]; xsc[mm][1] = xscn[mm][1]; }
-            }
-        }
     }
     if (failed && lane == 0) {
         // Report, then wait (bounded) for this warp's copies still in flight.

@@ -95,7 +95,7 @@ __global__ void write_header_kernel(uint8_t* packed, uint32_t fmt, int64_t N, in
                                     uint32_t flags, float gs, int32_t T, int32_t G) {
     PackedHeader* h = reinterpret_cast<PackedHeader*>(packed);
     if (threadIdx.x == 0) {
-        h->magic = kMagic;
+        h->magic = kMagic;  // unit_bytes below is the GEMV unit; QLIN_PACK_MMA units are 36864 B
         h->fmt = fmt;
         h->N = N;
         h->K = K;
@@ -152,9 +152,17 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
 
 using namespace qlin;
 
+extern "C" cudaError_t qlin_launch_pack_mma(const void* codes, const void* scales, int64_t N, int64_t K, float gs,
+                                            void* packed, cudaStream_t s);
+
 extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void* scales, int64_t N,
                                         int64_t K, int pack_flags, float gs, void* packed,
                                         cudaStream_t s) {
+    if (pack_flags == QLIN_PACK_MMA) {
+        write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags, gs,
+                                             (int32_t)((N + 255) / 256), (int32_t)((K + 255) / 256));
+        return qlin_launch_pack_mma(blocks, scales, N, K, gs, packed, s);
+    }
     Geometry geo = geometry(fmt, N, K, pack_flags);
     const int gu = (pack_flags & QLIN_PACK_GATE_UP) ? 1 : 0;
     write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags,

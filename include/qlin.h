@@ -62,8 +62,11 @@ enum {
 /* qlin_pack_weights flags */
 enum {
     QLIN_PACK_DEFAULT = 0,
-    QLIN_PACK_GATE_UP = 1 /* the N rows are [gate ; up] halves (N even): each packed tile pairs
+    QLIN_PACK_GATE_UP = 1, /* the N rows are [gate ; up] halves (N even): each packed tile pairs
                              16 gate rows with their 16 up rows so the SiLU-gate epilogue fuses */
+    QLIN_PACK_MMA = 2      /* NVFP4 only: the tensor-core operand layout of qlin_gemm_chunk (tiles of
+                             256 rows x 256 values, 128-byte-swizzled K-major codes, scale factors
+                             in 512-byte atoms); 0.5625 B/weight plus padding to 256 x 256 */
 };
 
 /* qlin_workspace_bytes ops */
@@ -162,6 +165,32 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
                                int32_t* topk_ids, float* topk_w, const void* x, qlin_dtype_t xdt, int M,
                                float* y, float* h, int flags, void* ws, size_t ws_bytes,
                                qlin_stream_t stream);
+
+/* ------------------------------------------------------------------------- prefill-chunk GEMM */
+
+/* NVFP4 GEMM for prefill chunks (M rows of bf16 activations, M >= 1; built for M >= 64) on the
+ * tcgen05 tensor cores.  The counterpart on the pages is imp's NVFP4 block-scaled GEMM for
+ * prefill (README "Features", row "sm_120a kernels": block-scaled mxf4nvf4 MMA, there with
+ * mma.sync for sm_120a).  Two steps, three launches on `stream`:
+ *   1. quantize x to NVFP4 (the A operand), all in fp32 with round-to-nearest-even:
+ *        a_g = amax|x| / (6 * 448);  s_b = E4M3_rne_satfinite(amax_b / (6 * a_g)) per 16 values;
+ *        code = E2M1_rne_satfinite(x / (e4m3(s_b) * a_g)), 0 where that divisor is 0
+ *   2. y[m][n] = (a_g * g_w) * sum_k A_q[m][k] * W_q[n][k], block scales applied inside the MMA
+ *      (kind::mxf4nvf4 block16), fp32 accumulation in tensor memory.
+ *   packed: qlin_pack_weights(QLIN_NVFP4, N, K, ..., QLIN_PACK_MMA);  x: bf16 M x K, row stride ldx;
+ *   y: fp32, row stride ldy;  flags: 0 or QLIN_FLAG_PDL;
+ *   ws: qlin_workspace_bytes(QLIN_OP_CHUNK, QLIN_NVFP4, M, N, K, 0, 0) bytes.
+ * Other formats return QLIN_ERR_UNSUPPORTED.  Bounded device waits: a timeout sets the workspace
+ * status word (qlin_ws_status). */
+qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,
+                              int M, int64_t ldx, float* y, int64_t ldy, int flags, void* ws,
+                              size_t ws_bytes, qlin_stream_t stream);
+
+/* Test and inspection aid: run step 1 of qlin_gemm_chunk alone and also write the quantized
+ * activations in the canonical NVFP4 layout: codes [M][K/2] (element 2i in the low nibble), E4M3
+ * scales [M][K/16], and a_g (one float, device memory).  ws as for qlin_gemm_chunk. */
+qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* codes, void* scales,
+                                   float* a_g, void* ws, size_t ws_bytes, qlin_stream_t stream);
 
 /* Dequantize a packed buffer back to fp32 W[N][K] (row-major, canonical row order, also for
  * QLIN_PACK_GATE_UP buffers; pass the pack_flags the buffer was packed with).  The value of every

@@ -366,6 +366,31 @@ def run_config(name, args):
             lines.append(dict(workload="Q4_0 MoE expert layer shaped like an 8B-A1B model: hidden 2048, 32 experts "
                               "gate_up 2048->2x1792, down 1792->2048, top-4", M=M, distinct_experts=nd,
                               us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9))
+    if name == "chunk":
+        fmt, N, K = q.QLIN_NVFP4, 17408, 5120
+        b, s_, g = synth.weights(fmt, N, K, synth.gen(7000, device="cuda"), device="cuda")
+        packs = [q.qlin_pack_weights(fmt, N, K, b, s_, g, q.QLIN_PACK_MMA)]
+        b2, s2, g2 = synth.weights(fmt, N, K, synth.gen(7001, device="cuda"), device="cuda")
+        packs.append(q.qlin_pack_weights(fmt, N, K, b2, s2, g2, q.QLIN_PACK_MMA))  # 2 copies > L2 with y
+        del b, s_, b2, s2
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                bf16 = float(json.load(f)["bf16_tflops"])
+            fp4_peak, fp4_src = 4 * bf16, "measured bf16 burst x 4 (nominal fp4/bf16 ratio)"
+        except Exception:
+            fp4_peak, fp4_src = 4 * 1590.0, "fallback bf16 x 4"
+        for M in (512, 64, 16, 8, 4, 2, 1):
+            x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
+            y = torch.empty(M, N, device="cuda")
+            ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+            fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL) for c in range(2)]
+            ms = _time_graph_of(fn, args.steps, args.warmup) / 2
+            flop = 2.0 * M * N * K
+            bytes_ = (q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA) - 256) + 2 * M * K + 4 * M * N
+            lines.append(dict(workload=f"NVFP4 prefill-chunk GEMM M={M} K=5120 N=17408 (activation quantization "
+                              "+ tcgen05 block-scaled GEMM, 3 launches)", M=M, us_per_call=ms * 1e3,
+                              tflops=flop / (ms * 1e-3) / 1e12, fp4_peak_tflops=fp4_peak, fp4_peak_source=fp4_src,
+                              fp4_frac=flop / (ms * 1e-3) / 1e12 / fp4_peak, gbs=bytes_ / (ms * 1e-3) / 1e9))
     for ln in lines:
         ln.update(metric=METRIC, unit="GB/s", value=ln["gbs"], hbm_frac=ln["gbs"] / peak,
                   peak=peak, peak_source=peak_src, config=name, impl="qlin", n_gpus=1)
@@ -381,7 +406,7 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "moe"],
+    ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "moe", "chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
     if args.config != "stack":

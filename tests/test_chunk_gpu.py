@@ -3,10 +3,11 @@
 The quantized activations must equal the oracle's bit for bit (codes, scales, a_g: the rule is
 stated in fp32 and both sides take each rounding in fp32).  The GEMM output must match the fp64
 product of the same quantized operands within 2e-6 * sum|a_q * w| (fp32 accumulation).  Against
-the fp64 product of the unquantized bf16 activations the bound is 1e-2 * sum|x * w| (the
-bf16-operand tolerance of the chunk path) at the configured K = 5120: the activation quantization
-error relative to sum|x * w| shrinks like 1/sqrt(K) (about 0.15% rms at K = 5120, about 0.6% at
-K = 256, where single outputs exceed 1%), so that check is made at K = 5120 only.
+the fp64 product of the unquantized bf16 activations two checks hold at the configured K = 5120:
+per output, the triangle-inequality bound 2e-6 * sum|a_q * w| + sum|w| * |x - a_q| (always true if
+the kernel multiplies the quantized operands it was given), and over all sampled outputs an rms of
+|y - y_exact| / sum|x * w| below 5e-3 (the activation quantization alone gives about 2.5e-3 for
+N(0,1) activations; single outputs reach 1e-2, so a per-output 1e-2 bound is not a valid check).
 """
 import numpy as np
 import pytest
@@ -49,15 +50,17 @@ def _chunk(M, N, K, seed, rows=None):
     ac, asc, ag = oracle.act_quant(x.float().numpy())
     if rows is None:
         rows = np.arange(N)
-    yq, Aq = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), oracle.dequant(q.QLIN_NVFP4, M, K, ac, asc, ag),
-                         scales=scales.numpy(), g=g, rows=rows)
-    ye, Ae = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), x.double().numpy(), scales=scales.numpy(), g=g, rows=rows)
-    return y.cpu().double().numpy()[:, rows], yq, Aq, ye, Ae
+    xq = oracle.dequant(q.QLIN_NVFP4, M, K, ac, asc, ag)
+    yq, Aq = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xq, scales=scales.numpy(), g=g, rows=rows)
+    xd = x.double().numpy()
+    ye, Ae = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xd, scales=scales.numpy(), g=g, rows=rows)
+    _, Ed = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xd - xq, scales=scales.numpy(), g=g, rows=rows)
+    return y.cpu().double().numpy()[:, rows], yq, Aq, ye, Ae, Ed
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (70, 300, 272), (200, 512, 1024)])
 def test_chunk_gemm_small(M, N, K):
-    y, yq, Aq, ye, Ae = _chunk(M, N, K, 10 * M + N)
+    y, yq, Aq, _, _, _ = _chunk(M, N, K, 10 * M + N)
     err = np.abs(y - yq)
     assert (err <= 2e-6 * Aq).all(), float(np.max(err / np.maximum(Aq, 1e-300)))
 
@@ -66,9 +69,11 @@ def test_chunk_gemm_small(M, N, K):
 def test_chunk_gemm_27b_shape_sampled(M):
     N, K = 17408, 5120
     rows = np.unique(np.concatenate([[0, 255, 256, N - 1], np.random.default_rng(M).integers(0, N, 60)]))
-    y, yq, Aq, ye, Ae = _chunk(M, N, K, 77, rows)
+    y, yq, Aq, ye, Ae, Ed = _chunk(M, N, K, 77, rows)
     assert (np.abs(y - yq) <= 2e-6 * Aq).all(), float(np.max(np.abs(y - yq) / np.maximum(Aq, 1e-300)))
-    assert (np.abs(y - ye) <= 1e-2 * Ae).all()
+    assert (np.abs(y - ye) <= 2e-6 * Aq + Ed + 1e-12 * Ae).all()
+    rel = np.abs(y - ye) / Ae
+    assert float(np.sqrt(np.mean(rel * rel))) < 5e-3, float(np.sqrt(np.mean(rel * rel)))
 
 
 def test_chunk_gemm_status_clean_and_deterministic():

@@ -111,7 +111,7 @@ __device__ __forceinline__ void global_fixup(const GemvArgs& a, int64_t t, int64
 // row-part accumulators across the units of a tile (one FMA per block) and reduces once per tile.
 // With MAXM > 2 each pass reduces at once.
 template <int FMT, int MAXM, bool XBF16, int EPI>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) gemv_kernel(const GemvArgs a) {
     using C = RingCfg<FMT>;
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     constexpr bool kOnePass = MAXM <= 2;
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
 
     griddep_launch_dependents();
     // The per-tensor scale lives in the packed header (immutable, like the weights).
-    const float gs = FMT == QLIN_NVFP4 ? reinterpret_cast<const PackedHeader*>(a.packed)->global_scale : 1.0f;
+    const float gs = format_out_scale<FMT>(a.packed);
 
     const int U = (int)a.U, nC = (int)a.Wt, G = (int)a.G;
     const int cu0 = (int)((int64_t)blockIdx.x * U / nC), cu1 = (int)((int64_t)(blockIdx.x + 1) * U / nC);
@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
     for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
     float acc8[8][MP];
     float2 xv[MP][16];
+    float xb[MP];
     uint32_t xh[MP][16];
     float xsc[MP][2];
     const void* rows0[MP];
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
                 load_x_fp4h<MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xh, xsc);
             } else {
                 load_x_rows<XBF16, MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xv);
-                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xv);
+                prep_x<FMT, MP>(xv, xb);
             }
         }
     }
@@ -195,12 +196,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
                 load_x_fp4h<MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xh, xsc);
             } else {
                 load_x_rows<XBF16, MP>(rows0, (int64_t)g * kGroupK + part * 32, a.K, xv);
-                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xv);
+                prep_x<FMT, MP>(xv, xb);
             }
         }
         if (kOnePass) {
             if constexpr (kH) unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
-            else unit_dot<FMT, MP, true>(ubuf, lane, xv, acc8);
+            else unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
         } else {
             const int64_t k0 = (int64_t)g * kGroupK + part * 32;
 #pragma unroll 1
@@ -220,9 +221,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
                     load_x_fp4h<MP>(rows, k0, a.K, xph, xps);
                     unit_dot_fp4h<MP>(ubuf, lane, xph, xps, res);
                 } else {
+                    float xpb[MP];
                     load_x_rows<XBF16, MP>(rows, k0, a.K, xp);
-                    if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xp);
-                    unit_dot<FMT, MP>(ubuf, lane, xp, res);
+                    prep_x<FMT, MP>(xp, xpb);
+                    unit_dot<FMT, MP>(ubuf, lane, xp, xpb, res);
                 }
                 float r[MP];
                 reduce_scatter8<MP>(res, lane, r);

@@ -18,45 +18,101 @@ struct RingCfg {
 
 
 // ------------------------------------------------------------------ code decoders
-// Magic-exponent construction: OR-ing a nibble/byte into the mantissa of 2^E, placed so that its
-// unit bit is the float's unit-in-last-place, gives exactly 2^E + code; subtracting (2^E + bias)
-// leaves the signed code exactly.  Different nibble positions use different E, so no shifts.
-__device__ __forceinline__ float magic(uint32_t w, uint32_t mask, uint32_t expbits) {
-    return __uint_as_float((w & mask) | expbits);
+// Q4_0 / Q8_0 codes as denormal floats.  A 32-bit pattern P < 2^24 read as an fp32 number is
+// exactly P * 2^-149 (patterns below 2^23 are denormals, 2^23 .. 2^24-1 continue seamlessly as
+// the first binade).  So a nibble or byte masked in place at bit 4j (8j), with nothing else set,
+// IS the float n * 2^(4j) * 2^-149: one AND per weight, no shift, no subtraction.  Codes are
+// unsigned (Q4_0 nibble n = q + 8, Q8_0 byte = q + 128); the offset is removed once per block
+// from a sum of the activations taken in the same order (see prep_x_q4 / prep_x_q8).
+// Activations are pre-scaled by 2^(kXExp - 4j) (2^(kXExp - 8j) for Q8_0), so every product is
+// the exact n * x * 2^(kXExp - 149) computed inside an fp32 FMA; block sums carry 2^(kXExp - 149)
+// and the tile output multiplies by kDenormUnscale = 2^(149 - kXExp).  Products stay normal and
+// exact for 2^-40 <= |x| < 2^65; smaller activations lose relative precision (each product is
+// then exact to 2^-63 in absolute terms), larger ones overflow.
+constexpr int kXExp = 63;
+constexpr float kDenormUnscale = 0x1p86f;  // 2^(149 - kXExp)
+
+// Output scale of a format's block sums: the NVFP4 per-tensor scale, or 2^86 for Q4_0 / Q8_0.
+template <int FMT>
+__device__ __forceinline__ float format_out_scale(const uint8_t* packed) {
+    if (FMT == QLIN_NVFP4) return reinterpret_cast<const PackedHeader*>(packed)->global_scale;
+    return kDenormUnscale;
 }
 
-// Q4_0 word: elements 8k..8k+7 (nibble i = element i).  One shared exponent 2^23 for every
-// nibble position: the nibble at bits 4j (j = i mod 4, taken from w or w >> 16) gives the exact
-// float 2^23 + code * 16^j, and subtracting 2^23 + 8 * 16^j leaves (code - 8) * 16^j exactly.
-// The matching activations are pre-scaled by 16^-j (exact), see prescale_x_q4.  Returns four
-// pairs for elements (0,1), (2,3), (4,5), (6,7).
+// Q4_0 word: elements 8k..8k+7, element i at bits 4i.  Elements 0..5 are masked in place
+// (position j = i); elements 6 and 7 are taken from w >> 8 at positions 4 and 5.  Pairs:
+// (0,1) (2,3) (4,5) (6,7).
 __device__ __forceinline__ void dec_q4(uint32_t w, float2 (&p)[4]) {
-    const uint32_t e23 = 0x4b000000u;
-    const float2 c01 = make_float2(-(8388608.0f + 8.0f), -(8388608.0f + 128.0f));
-    const float2 c23 = make_float2(-(8388608.0f + 2048.0f), -(8388608.0f + 32768.0f));
-    const uint32_t h = w >> 16;
-    p[0] = __fadd2_rn(make_float2(__uint_as_float((w & 0xfu) | e23), __uint_as_float((w & 0xf0u) | e23)), c01);
-    p[1] = __fadd2_rn(make_float2(__uint_as_float((w & 0xf00u) | e23), __uint_as_float((w & 0xf000u) | e23)), c23);
-    p[2] = __fadd2_rn(make_float2(__uint_as_float((h & 0xfu) | e23), __uint_as_float((h & 0xf0u) | e23)), c01);
-    p[3] = __fadd2_rn(make_float2(__uint_as_float((h & 0xf00u) | e23), __uint_as_float((h & 0xf000u) | e23)), c23);
+    const uint32_t h = w >> 8;
+    p[0] = make_float2(__uint_as_float(w & 0xfu), __uint_as_float(w & 0xf0u));
+    p[1] = make_float2(__uint_as_float(w & 0xf00u), __uint_as_float(w & 0xf000u));
+    p[2] = make_float2(__uint_as_float(w & 0xf0000u), __uint_as_float(w & 0xf00000u));
+    p[3] = make_float2(__uint_as_float(h & 0xf0000u), __uint_as_float(h & 0xf00000u));
 }
 
-// Pre-scale a lane's 32 activations for dec_q4: element e (pair e/2) times 16^-(e mod 4).
-template <int MP>
-__device__ __forceinline__ void prescale_x_q4(float2 (&xv)[MP][16]) {
-    const float2 s01 = make_float2(1.0f, 0.0625f), s23 = make_float2(0.00390625f, 0.000244140625f);
-#pragma unroll
-    for (int mm = 0; mm < MP; ++mm)
-#pragma unroll
-        for (int q = 0; q < 16; ++q) xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 1) ? s23 : s01);
-}
-
-// Q8_0 word: 4 elements stored as q + 128 -> two pairs of q.
+// Q8_0 word: elements 4k..4k+3 stored as q + 128 in bytes 0..3.  Bytes 0..2 are masked in
+// place (positions 0, 1, 2); byte 3 is w >> 24 (position 0).  Pairs: (0,1) (2,3).
 __device__ __forceinline__ void dec_q8(uint32_t w, float2 (&p)[2]) {
-    const float2 c = make_float2(-(8388608.0f + 128.0f), -(32768.0f + 128.0f));
-    const uint32_t h = w >> 16;
-    p[0] = __fadd2_rn(make_float2(magic(w, 0xffu, 0x4b000000u), magic(w, 0xff00u, 0x47000000u)), c);
-    p[1] = __fadd2_rn(make_float2(magic(h, 0xffu, 0x4b000000u), magic(h, 0xff00u, 0x47000000u)), c);
+    p[0] = make_float2(__uint_as_float(w & 0xffu), __uint_as_float(w & 0xff00u));
+    p[1] = make_float2(__uint_as_float(w & 0xff0000u), __uint_as_float(w >> 24));
+}
+
+// Offset sum of one lane's part: the products of code == offset (8 for Q4_0, 128 for Q8_0) are
+// offset * x * 2^(kXExp - 149), a power of two times x, and a power-of-two factor commutes with
+// fp32 rounding.  So adding the raw activations in exactly the order unit_dot adds its products
+// (two interleaved pair chains, then the pairs combined lane-wise, then the two halves), times
+// offset * 2^(kXExp - 149), reproduces bit for bit what a block of offset codes sums to: a block
+// of zero weights gives exactly 0.  Both decoders feed even pairs to chain 0 and odd pairs to
+// chain 1, in increasing pair order.
+__device__ __forceinline__ float offset_sum(const float2 (&x)[16]) {
+    float2 t0 = x[0], t1 = x[1];
+#pragma unroll
+    for (int q = 2; q < 16; q += 2) {
+        t0 = __fadd2_rn(t0, x[q]);
+        t1 = __fadd2_rn(t1, x[q + 1]);
+    }
+    const float2 u = __fadd2_rn(t0, t1);
+    return u.x + u.y;
+}
+
+// Prepare a lane's 32 activations for the Q4_0 decoder: the offset term 8 * sum (scaled), then
+// element e (pair e/2) times 2^(kXExp - 4 j) with j the decoder's position of element e mod 8.
+template <int MP>
+__device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float (&xb)[MP]) {
+    constexpr float c = 0x1p-83f;  // 8 * 2^(kXExp - 149)
+    const float2 s0 = make_float2(0x1p63f, 0x1p59f), s1 = make_float2(0x1p55f, 0x1p51f);
+    const float2 s2 = make_float2(0x1p47f, 0x1p43f);
+#pragma unroll
+    for (int mm = 0; mm < MP; ++mm) {
+        xb[mm] = c * offset_sum(xv[mm]);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 3) == 0 ? s0 : (q & 3) == 1 ? s1 : s2);
+    }
+}
+
+// Prepare a lane's 32 activations for the Q8_0 decoder: offset 128 * sum (scaled), pairs
+// (4k, 4k+1) times (2^63, 2^55) and (4k+2, 4k+3) times (2^47, 2^63).
+template <int MP>
+__device__ __forceinline__ void prep_x_q8(float2 (&xv)[MP][16], float (&xb)[MP]) {
+    constexpr float c = 0x1p-79f;  // 128 * 2^(kXExp - 149)
+    const float2 s0 = make_float2(0x1p63f, 0x1p55f), s1 = make_float2(0x1p47f, 0x1p63f);
+#pragma unroll
+    for (int mm = 0; mm < MP; ++mm) {
+        xb[mm] = c * offset_sum(xv[mm]);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 1) ? s1 : s0);
+    }
+}
+
+// Prepare a lane's activations for unit_dot<FMT> (NVFP4 needs no preparation; xb is unused).
+template <int FMT, int MP>
+__device__ __forceinline__ void prep_x(float2 (&xv)[MP][16], float (&xb)[MP]) {
+    if (FMT == QLIN_Q4_0) prep_x_q4<MP>(xv, xb);
+    else if (FMT == QLIN_Q8_0) prep_x_q8<MP>(xv, xb);
+    else {
+#pragma unroll
+        for (int mm = 0; mm < MP; ++mm) xb[mm] = 0.f;
+    }
 }
 
 // NVFP4 word: elements 8k..8k+7, byte j = elements 2j (low nibble), 2j+1 -> four pairs of e2m1.
@@ -69,9 +125,16 @@ __device__ __forceinline__ void dec_fp4(uint32_t w, float2 (&p)[4]) {
 }
 
 // ------------------------------------------------------------------ activations
+// 16-byte activation load; CG = through L2 only (activations written earlier by the same grid).
+template <bool CG, typename V>
+__device__ __forceinline__ V ldx16(const V* p) {
+    if constexpr (CG) return __ldcg(p);
+    else return *p;
+}
+
 // Lane's 32 activations of one part (elements k0 .. k0+31) for MP rows given by pointers (NULL
 // row = zeros); elements at or beyond K read as 0 (NVFP4 K may end in the middle of a part).
-template <bool XBF16, int MP>
+template <bool XBF16, int MP, bool CG = false>
 __device__ __forceinline__ void load_x_rows(const void* const (&rows)[MP], int64_t k0, int64_t K,
                                             float2 (&xv)[MP][16]) {
     const int64_t left = K - k0;
@@ -86,7 +149,7 @@ __device__ __forceinline__ void load_x_rows(const void* const (&rows)[MP], int64
                     reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(rows[mm]) + k0 + 16 * h);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    uint4 v = ok ? src[q] : make_uint4(0, 0, 0, 0);
+                    uint4 v = ok ? ldx16<CG>(src + q) : make_uint4(0, 0, 0, 0);
                     uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
@@ -97,7 +160,7 @@ __device__ __forceinline__ void load_x_rows(const void* const (&rows)[MP], int64
                 const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rows[mm]) + k0 + 16 * h);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    float4 v = ok ? src[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float4 v = ok ? ldx16<CG>(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
                     xv[mm][8 * h + 2 * q] = make_float2(v.x, v.y);
                     xv[mm][8 * h + 2 * q + 1] = make_float2(v.z, v.w);
                 }
@@ -114,7 +177,7 @@ __device__ __forceinline__ void load_x_rows(const void* const (&rows)[MP], int64
 // f16 (exact except for elements more than 2^38 below the block maximum, whose contribution is
 // far below fp32 rounding), and 2^s is folded into the block's E4M3 scale.  Products then go
 // through fma.rn.f32.f16: exact products, fp32 sums.
-template <int MP>
+template <int MP, bool CG = false>
 __device__ __forceinline__ void load_x_fp4h(const void* const (&rows)[MP], int64_t k0, int64_t K,
                                             uint32_t (&xh)[MP][16], float (&xsc)[MP][2]) {
     const int64_t left = K - k0;
@@ -127,8 +190,8 @@ __device__ __forceinline__ void load_x_fp4h(const void* const (&rows)[MP], int64
                 reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(rows[mm]) + k0 + 16 * b);
             uint32_t u[8];
             {
-                uint4 v0 = ok ? src[0] : make_uint4(0, 0, 0, 0);
-                uint4 v1 = ok ? src[1] : make_uint4(0, 0, 0, 0);
+                uint4 v0 = ok ? ldx16<CG>(src) : make_uint4(0, 0, 0, 0);
+                uint4 v1 = ok ? ldx16<CG>(src + 1) : make_uint4(0, 0, 0, 0);
                 u[0] = v0.x; u[1] = v0.y; u[2] = v0.z; u[3] = v0.w;
                 u[4] = v1.x; u[5] = v1.y; u[6] = v1.z; u[7] = v1.w;
             }
@@ -212,7 +275,7 @@ __device__ __forceinline__ void unit_dot_fp4h(const uint8_t* ub, int lane, const
 // with ACC the contribution is added to res instead (one fused multiply-add per block).
 template <int FMT, int MP, bool ACC = false>
 __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const float2 (&xv)[MP][16],
-                                         float (&res)[8][MP]) {
+                                         const float (&xb)[MP], float (&res)[8][MP]) {
     const uint4 sv = lds128(ub + code_bytes(FMT) + lane * 16);
     const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
@@ -239,7 +302,8 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
             const float d = fp16_bits_to_f32(sc & 0xffffu);
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) {
-                const float bsum = (s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y);
+                const float2 u = __fadd2_rn(s0[mm], s1[mm]);
+                const float bsum = (u.x + u.y) - xb[mm];
                 res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
             }
         } else if (FMT == QLIN_Q8_0) {
@@ -262,7 +326,8 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
             const float d = fp16_bits_to_f32(sc & 0xffffu);
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) {
-                const float bsum = (s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y);
+                const float2 u = __fadd2_rn(s0[mm], s1[mm]);
+                const float bsum = (u.x + u.y) - xb[mm];
                 res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
             }
         } else {  // NVFP4: two 16-element blocks per part, one E4M3 scale each

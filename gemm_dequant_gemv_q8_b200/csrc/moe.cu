@@ -227,7 +227,7 @@ __device__ __forceinline__ void moe_flush(const MoeArgs& a, const RouteSmem& r, 
 }
 
 template <int FMT, int MAXM, bool XBF16, int PHASE>
-__global__ void __launch_bounds__(kGemvWarps * 32) moe_kernel(const MoeArgs a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe_kernel(const MoeArgs a) {
     using C = RingCfg<FMT>;
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -267,9 +267,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) moe_kernel(const MoeArgs a) {
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
     int64_t cur_key = ub / a.G;  // key = act * T + t  (units of one expert are contiguous)
-    float gs = 1.0f;
-    if (FMT == QLIN_NVFP4)
-        gs = reinterpret_cast<const PackedHeader*>(a.packed + (int64_t)r.expert[cur_key / a.T] * a.stride)->global_scale;
+    float gs = format_out_scale<FMT>(a.packed + (int64_t)r.expert[cur_key / a.T] * a.stride);
     bool failed = false;
     int64_t j = 0;
     for (; j < n; ++j) {
@@ -317,9 +315,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) moe_kernel(const MoeArgs a) {
                 unit_dot_fp4h<MP>(ubuf, lane, xh, xsc, res);
             } else {
                 float2 xv[MP][16];
+                float xb[MP];
                 load_x_rows<kXB, MP>(rows, k0, a.Kin, xv);
-                if (FMT == QLIN_Q4_0) prescale_x_q4<MP>(xv);
-                unit_dot<FMT, MP>(ubuf, lane, xv, res);
+                prep_x<FMT, MP>(xv, xb);
+                unit_dot<FMT, MP>(ubuf, lane, xv, xb, res);
             }
             float rr[MP];
             reduce_scatter8<MP>(res, lane, rr);

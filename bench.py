@@ -53,7 +53,8 @@ def peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    """SM clock and clock-event (throttle) reasons sampled every ~2 ms through NVML (read-only
+    queries) while the timed region runs; nvidia-smi is the fallback when NVML is unavailable."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -61,14 +62,51 @@ class ClockSampler:
 
     def __init__(self, index):
         self.index, self.proc, self.lines = index, None, []
+        self.stop = threading.Event()
+        self.t = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            p = torch.cuda.get_device_properties(self.index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            idx = int(vis.split(",")[self.index]) if vis and vis.split(",")[0].isdigit() else self.index
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _poll_nvml(self, nv, h):
+        bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                flags = ["Active" if r & b else "Not Active" for b in bits]
+                self.lines.append(f"{self.index}, {sm}, {mx}, {pw}, {r:#x}, " + ", ".join(flags))
+            except Exception:
+                break
+            time.sleep(0.002)
 
     def __enter__(self):
         try:
+            nv, h = self._nvml_handle()
+            self.t = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.t.start()
+            return self
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            time.sleep(1.0)  # nvidia-smi's first sample
         except Exception:
             self.proc = None
         return self
@@ -78,12 +116,15 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        elif self.t is not None:
+            self.t.join(timeout=1.0)
 
     def summary(self):
         sm, mx, reasons = [], None, set()
@@ -112,9 +153,15 @@ class DenseStack:
     leave the step (qkv, o, down) in another (ybuf), so the end-to-end leg moves them with one
     host->device and one device->host copy per step."""
 
-    def __init__(self, fmt, layers, M=1, device="cuda"):
+    MODES = ("chain", "layer_chain", "launches")
+
+    def __init__(self, fmt, layers, M=1, device="cuda", mode="chain"):
+        """mode: "chain" = the whole step as qlin_gemv_chain launches of up to 256 ops (one for
+        36 layers); "layer_chain" = one chain of four ops per layer; "launches" = one qlin_gemv
+        per projection.  In the chains, down waits for its layer's gate_up (it reads h)."""
         import gemm_dequant_gemv_q8_b200 as q
-        self.q, self.fmt, self.M, self.layers = q, fmt, M, layers
+        assert mode in self.MODES
+        self.q, self.fmt, self.M, self.layers, self.mode = q, fmt, M, layers, mode
         self.packed, self.ws = [], []
         self.weight_bytes = 0
         xs = [(l, pi, K) for l in range(layers) for pi, (n_, N, K, e) in enumerate(STACK) if n_ != "down"]
@@ -155,11 +202,35 @@ class DenseStack:
             act += 4 * M * K + 4 * M * (N // 2 if epi else N)
         self.act_bytes = act * layers
         self.step_bytes = self.weight_bytes + self.act_bytes
-        self.launches_per_step = len(STACK) * layers
+        self.chains = []  # (ops, workspace) per launch
+        if mode != "launches":
+            ops = []
+            for l in range(layers):
+                for pi, (name, N, K, epi) in enumerate(STACK):
+                    if mode == "layer_chain" and pi == 0:
+                        ops = []
+                    elif mode == "chain" and len(ops) + len(STACK) > q.qlin_chain_max_ops() and pi == 0:
+                        self.chains.append(ops)
+                        ops = []
+                    wait = len(ops) - 1 if name == "down" else -1
+                    ops.append(q.gemv_op(self.packed[l][pi], N, K, self.x[(l, pi)], self.y[(l, pi)],
+                                         q.QLIN_EPI_SILU_GATE if epi else q.QLIN_EPI_NONE, wait))
+                    if mode == "layer_chain" and pi == len(STACK) - 1:
+                        self.chains.append(ops)
+            if mode == "chain":
+                self.chains.append(ops)
+            self.chains = [(o, q.workspace(q.qlin_chain_workspace_bytes(fmt, M, o), device)) for o in self.chains]
+            self.launches_per_step = len(self.chains)
+        else:
+            self.launches_per_step = len(STACK) * layers
 
     def step(self, pdl=True):
         q = self.q
         fl = q.QLIN_FLAG_PDL if pdl else 0
+        if self.chains:
+            for ops, ws in self.chains:
+                q.qlin_gemv_chain(self.fmt, q.QLIN_F32, self.M, ops, flags=fl, ws=ws)
+            return
         for l in range(self.layers):
             P, W = self.packed[l], self.ws[l]
             for pi, (name, N, K, epi) in enumerate(STACK):
@@ -197,6 +268,28 @@ def time_graph(graph, steps, warmup):
     b.record()
     b.synchronize()
     return a.elapsed_time(b) / steps
+
+
+def time_chain_kernel(stack, reps=3):
+    """Average duration of one chain launch, timed with CUDA events on the launching stream
+    (eager launches, no graph); algorithmic bytes of the ops that launch covers."""
+    q = stack.q
+    st = torch.cuda.current_stream()
+
+    def run():
+        for ops, ws in stack.chains:
+            q.qlin_gemv_chain(stack.fmt, q.QLIN_F32, stack.M, ops, ws=ws)
+
+    run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(reps):
+        run()
+    b.record(st)
+    b.synchronize()
+    ms = a.elapsed_time(b) / (reps * len(stack.chains))
+    return ms, stack.step_bytes / len(stack.chains)
 
 
 def time_dominant_kernel(stack, reps=3):
@@ -406,6 +499,8 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="chain", choices=list(DenseStack.MODES),
+                    help="how the stack step is launched (default: one persistent GEMV chain)")
     ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "moe", "chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
@@ -446,7 +541,7 @@ def main():
     else:
         torch.cuda.set_device(0)
 
-    stack = DenseStack(fmt, args.layers)
+    stack = DenseStack(fmt, args.layers, mode=args.mode)
     graph = stack.capture(pdl=not args.no_pdl)
 
     def barrier():
@@ -471,7 +566,13 @@ def main():
         torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
     ms_max = float(ms_t.item())
 
-    dom_ms, dom_bytes = time_dominant_kernel(stack)
+    if stack.chains:
+        dom_ms, dom_bytes = time_chain_kernel(stack)
+        dom_name = (f"chain_kernel<Q4_0, M=1> ({len(stack.chains[0][0])} GEMVs per launch, "
+                    f"{len(stack.chains)} launches per step)")
+    else:
+        dom_ms, dom_bytes = time_dominant_kernel(stack)
+        dom_name = "gemv_kernel<Q4_0, M=1, SiLU-gate> (gate_up 2560->19456)"
     e2e_ms, h2d, d2h = e2e_stack(stack, args.steps, args.warmup, pdl=not args.no_pdl)
     e2e_t = torch.tensor([e2e_ms], device="cuda")
     if world > 1:
@@ -486,7 +587,8 @@ def main():
         traffic = None
         try:
             with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-                traffic = json.load(f).get("gate_up_q4_0_m1_bytes_per_launch")
+                key = f"{args.mode}_q4_0_m1_bytes_per_launch" if stack.chains else "gate_up_q4_0_m1_bytes_per_launch"
+                traffic = json.load(f).get(key)
         except Exception:
             pass
         line = {
@@ -497,10 +599,11 @@ def main():
             "hbm_frac": gbs / world / peak,
             "config": {"workload": workload, "format": "q4_0", "M": 1, "layers": args.layers,
                        "weight_bytes_per_step": stack.weight_bytes, "algorithmic_bytes_per_step": stack.step_bytes,
-                       "launches_per_step": stack.launches_per_step, "cuda_graph": True, "pdl": not args.no_pdl,
+                       "launches_per_step": stack.launches_per_step, "mode": args.mode,
+                       "cuda_graph": True, "pdl": not args.no_pdl,
                        "l2": "inputs larger than L2: 2.04 GB of packed weights streamed per step (L2 126 MB)",
                        "parallelism": f"replicas{world}"},
-            "roofline": {"bound": "hbm", "kernel": "gemv_kernel<Q4_0, M=1, SiLU-gate> (gate_up 2560->19456)",
+            "roofline": {"bound": "hbm", "kernel": dom_name,
                          "achieved": dom_gbs, "peak": peak, "peak_source": f"{peak_src} hbm_gbs (copy)",
                          "unit": "GB/s", "frac": dom_gbs / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": dom_ms * 1e3},

@@ -42,9 +42,18 @@ SIGNATURES = {
     "qlin_gemm_chunk": (_I, [_I, _P, _I64, _I64, _P, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "qlin_act_quant_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "qlin_dequant_debug": (_I, [_I, _P, _I64, _I64, _I, _P, _P]),
+    "qlin_chain_max_ops": (_I, []),
+    "qlin_chain_workspace_bytes": (_SZ, [_I, _I, _P, _I]),
+    "qlin_gemv_chain": (_I, [_I, _I, _I, _P, _I, _I, _P, _SZ, _P]),
     "qlin_ws_status": (_I, [_P, _P]),
     "qlin_status_string": (ctypes.c_char_p, [_I]),
 }
+
+
+class GemvOp(ctypes.Structure):
+    """struct qlin_gemv_op of include/qlin.h (64 bytes)."""
+    _fields_ = [("packed", _P), ("N", _I64), ("K", _I64), ("x", _P), ("ldx", _I64), ("y", _P),
+                ("ldy", _I64), ("epilogue", ctypes.c_int32), ("wait_for", ctypes.c_int32)]
 
 
 class QlinError(RuntimeError):
@@ -230,3 +239,41 @@ def qlin_ws_status(ws, stream=None):
 
 def qlin_status_string(status):
     return lib().qlin_status_string(status).decode()
+
+
+def gemv_op(packed, N, K, x, y, epilogue=QLIN_EPI_NONE, wait_for=-1):
+    """One op of a chain: the qlin_gemv arguments for one matrix (x, y CUDA tensors with
+    contiguous rows) and the index of an earlier op whose y this op's x reads (or -1)."""
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if y.dim() == 1:
+        y = y.unsqueeze(0)
+    if x.stride(1) != 1 or y.stride(1) != 1:
+        raise ValueError("x and y rows must be contiguous")
+    return GemvOp(_dev(packed, "packed").value, N, K, _dev(x, "x").value, x.stride(0),
+                  _dev(y, "y", torch.float32).value, y.stride(0), epilogue, wait_for)
+
+
+def _op_array(ops):
+    arr = (GemvOp * len(ops))(*ops)
+    return arr, ctypes.cast(arr, ctypes.c_void_p)
+
+
+def qlin_chain_max_ops():
+    return lib().qlin_chain_max_ops()
+
+
+def qlin_chain_workspace_bytes(fmt, M, ops):
+    arr, ptr = _op_array(ops)
+    return lib().qlin_chain_workspace_bytes(fmt, M, ptr, len(ops))
+
+
+def qlin_gemv_chain(fmt, xdt, M, ops, flags=0, ws=None, stream=None):
+    """Run the GEMVs `ops` (a list of gemv_op(...)) in one persistent launch; returns ws."""
+    arr, ptr = _op_array(ops)
+    if ws is None:
+        ws = workspace(lib().qlin_chain_workspace_bytes(fmt, M, ptr, len(ops)))
+    st = lib().qlin_gemv_chain(fmt, xdt, M, ptr, len(ops), flags, _dev(ws, "ws"),
+                               ws.numel() * ws.element_size(), _stream(stream))
+    _check("qlin_gemv_chain", st)
+    return ws

@@ -23,6 +23,11 @@ extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, 
                                         const void* x, int xdt, int M, int64_t ldx, float* y,
                                         int64_t ldy, int flags, void* ws, cudaStream_t s);
 
+extern "C" int qlin_chain_max_ops();
+extern "C" size_t qlin_chain_ws_bytes(int fmt, int M, const qlin_gemv_op* ops, int n_ops);
+extern "C" cudaError_t qlin_launch_chain(int fmt, int xdt, int M, const qlin_gemv_op* ops, int n_ops, int flags,
+                                         void* ws, cudaStream_t s);
+
 namespace {
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
@@ -38,9 +43,52 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 qlin_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA; }
 
+// One chain op against the qlin_gemv rules (op j of the chain).
+qlin_status_t check_chain_op(int fmt, int xdt, const qlin_gemv_op& o, int j) {
+    if (!valid_shape(fmt, o.N, o.K)) return QLIN_ERR_INVALID_ARG;
+    const int epi = o.epilogue;
+    if (epi != QLIN_EPI_NONE && epi != QLIN_EPI_SILU_GATE) return QLIN_ERR_INVALID_ARG;
+    if (epi == QLIN_EPI_SILU_GATE && (o.N % 2)) return QLIN_ERR_INVALID_ARG;
+    if (!o.packed || !o.x || !o.y) return QLIN_ERR_INVALID_ARG;
+    const int64_t ncols = epi == QLIN_EPI_SILU_GATE ? o.N / 2 : o.N;
+    if (o.ldx < o.K || o.ldy < ncols || o.ldx >= kMaxDim || o.ldy >= kMaxDim) return QLIN_ERR_INVALID_ARG;
+    if (o.wait_for < -1 || o.wait_for >= j) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(o.packed, 256) || !aligned(o.x, 16) || !aligned(o.y, 4)) return QLIN_ERR_ALIGNMENT;
+    if (o.ldx % (xdt == QLIN_F32 ? 4 : 8)) return QLIN_ERR_ALIGNMENT;
+    const int pack_flags = epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0;
+    if (qlin::geometry(fmt, o.N, o.K, pack_flags).U >= ((int64_t)1 << 30)) return QLIN_ERR_UNSUPPORTED;
+    return QLIN_OK;
+}
+
+qlin_status_t check_chain(int fmt, int xdt, int M, const qlin_gemv_op* ops, int n_ops) {
+    if (!valid_fmt(fmt) || (xdt != QLIN_F32 && xdt != QLIN_BF16) || M < 1 || M > 8) return QLIN_ERR_INVALID_ARG;
+    if (!ops || n_ops < 1 || n_ops > qlin_chain_max_ops()) return QLIN_ERR_INVALID_ARG;
+    for (int j = 0; j < n_ops; ++j) {
+        const qlin_status_t st = check_chain_op(fmt, xdt, ops[j], j);
+        if (st != QLIN_OK) return st;
+    }
+    return QLIN_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t qlin_chain_workspace_bytes(qlin_format_t fmt, int M, const qlin_gemv_op* ops, int n_ops) {
+    if (check_chain(fmt, QLIN_F32, M, ops, n_ops) != QLIN_OK && check_chain(fmt, QLIN_BF16, M, ops, n_ops) != QLIN_OK)
+        return 0;
+    return qlin_chain_ws_bytes(fmt, M, ops, n_ops);
+}
+
+qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const qlin_gemv_op* ops, int n_ops,
+                              int flags, void* ws, size_t ws_bytes, qlin_stream_t stream) {
+    const qlin_status_t st = check_chain(fmt, xdt, M, ops, n_ops);
+    if (st != QLIN_OK) return st;
+    if (flags & ~QLIN_FLAG_PDL) return QLIN_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < qlin_chain_ws_bytes(fmt, M, ops, n_ops)) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_chain(fmt, xdt, M, ops, n_ops, flags, ws, (cudaStream_t)stream));
+}
 
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags) {
     if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;

@@ -112,6 +112,8 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
  *   flags: QLIN_EPI_* | QLIN_FLAG_PDL
  * Weights stream from HBM once; dequantization happens in registers; products and sums are fp32
  * (activations are never quantized).  Results are deterministic for a given device and shape.
+ * Q8_0 / Q4_0 products are exact in fp32 for activations with 2^-40 <= |x| < 2^65; below that
+ * range a product is exact to 2^-63 in absolute terms, at or above it the result overflows.
  * The dequantize-and-multiply of quantized weight blocks against activations is the "NVFP4
  * block-scaled GEMM/GEMV" and "dp4a Q8_0 decode" of the imp pages (README "Features"; release
  * notes v0.4.1), re-designed here for sm_100a. */
@@ -137,6 +139,48 @@ qlin_status_t qlin_gemv(qlin_format_t fmt, const void* packed, int64_t N, int64_
 qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
                                 const void* x, qlin_dtype_t xdt, int M, int64_t ldx, float* y,
                                 int64_t ldy, int flags, qlin_stream_t stream);
+
+/* ------------------------------------------------------------------------- GEMV chains */
+
+/* One GEMV of a chain: the arguments of qlin_gemv for one weight matrix, plus a dependency. */
+typedef struct qlin_gemv_op {
+    const void* packed; /* qlin_pack_weights output for (fmt, N, K); QLIN_PACK_GATE_UP iff SiLU gate */
+    int64_t N, K;       /* packed rows and inputs, as for qlin_gemv (N, K < 2^31)                    */
+    const void* x;      /* M x K activations in the chain's xdt, row stride ldx (qlin_gemv rules)    */
+    int64_t ldx;
+    float* y;           /* M x N (N/2 with QLIN_EPI_SILU_GATE) fp32, row stride ldy                  */
+    int64_t ldy;
+    int32_t epilogue;   /* QLIN_EPI_NONE or QLIN_EPI_SILU_GATE                                       */
+    int32_t wait_for;   /* -1, or the index of an EARLIER op of the same chain whose y this op's x
+                           reads: the op then reads x only after every tile of that op is written */
+} qlin_gemv_op;
+
+/* Most ops in one chain. */
+int qlin_chain_max_ops(void);
+
+/* Workspace bytes of qlin_gemv_chain for these ops on the current device (0 if invalid). */
+size_t qlin_chain_workspace_bytes(qlin_format_t fmt, int M, const qlin_gemv_op* ops, int n_ops);
+
+/* Run n_ops GEMVs (all with format fmt, activation dtype xdt and M rows) in ONE persistent
+ * launch.  Each op computes what qlin_gemv computes for its arguments, to the same tolerance (the
+ * split of the K sums between warps differs, so the last bits can differ from qlin_gemv's;
+ * repeated runs of one chain on one device agree bit for bit).  The weights of all ops stream back to back: the ramp-up and tail of
+ * the HBM pipeline are paid once per chain instead of once per matrix, which is what a decode step
+ * of many 2-30 MB projections needs (the pages capture their decode steps in CUDA graphs for the
+ * per-launch overhead: imp release notes v0.4).  Ops run in order as far as their inputs allow:
+ * an op with wait_for = i reads its x only after op i has written all of its y (a bounded
+ * device-side wait; a wait that gives up after ~2 s sets the workspace status word, reported by
+ * qlin_ws_status as QLIN_ERR_TIMEOUT).  An op without wait_for must read nothing that an op of
+ * the same chain writes.  The grid holds a fixed number of CTAs per SM; the dependency waits
+ * assume nothing else keeps SMs busy for seconds while the chain runs.
+ *   ops   : host array of n_ops descriptors (1 <= n_ops <= qlin_chain_max_ops()), read during the
+ *           call only
+ *   flags : 0 or QLIN_FLAG_PDL
+ *   ws    : qlin_chain_workspace_bytes(fmt, M, ops, n_ops) bytes, zero-filled before first use
+ * Errors: as qlin_gemv, per op; QLIN_ERR_INVALID_ARG also for n_ops out of range or a wait_for
+ * that does not name an earlier op. */
+qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const qlin_gemv_op* ops, int n_ops,
+                              int flags, void* ws, size_t ws_bytes, qlin_stream_t stream);
 
 /* ------------------------------------------------------------------------- routed MoE experts */
 

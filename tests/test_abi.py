@@ -92,3 +92,40 @@ def test_workspace_bytes_cover_partials(lib):
     b8 = q.qlin_workspace_bytes(q.QLIN_OP_GEMV, q.QLIN_Q4_0, 8, 4096, 2560)
     assert 0 < b1 < b8
     assert q.qlin_workspace_bytes(q.QLIN_OP_GEMV, q.QLIN_Q4_0, 0, 4096, 2560) == 0
+
+
+def _chain_op(packed=0x100000, N=64, K=256, x=0x200000, ldx=256, y=0x300000, ldy=64, epi=0, wait_for=-1):
+    return q.GemvOp(packed, N, K, x, ldx, y, ldy, epi, wait_for)
+
+
+def test_chain_argument_checks_return_before_launch(lib):
+    E_ARG, E_ALIGN, E_WS = 1, 3, 4
+    P = ctypes.c_void_p
+
+    def call(ops, n=None, fmt=2, xdt=0, M=1, flags=0, ws=0x400000, ws_bytes=1 << 30):
+        arr = (q.GemvOp * max(len(ops), 1))(*ops)
+        return lib.qlin_gemv_chain(fmt, xdt, M, ctypes.cast(arr, P), len(ops) if n is None else n, flags,
+                                   P(ws), ws_bytes, None)
+
+    ok = _chain_op()
+    assert call([ok], n=0) == E_ARG and call([ok], n=lib.qlin_chain_max_ops() + 1) == E_ARG
+    assert call([ok], M=9) == E_ARG and call([ok], fmt=7) == E_ARG and call([ok], xdt=3) == E_ARG
+    assert call([ok], flags=1) == E_ARG
+    assert call([ok, _chain_op(wait_for=1)]) == E_ARG   # must name an EARLIER op
+    assert call([ok, _chain_op(wait_for=-2)]) == E_ARG
+    assert call([ok, _chain_op(K=100)]) == E_ARG
+    assert call([ok, _chain_op(epi=1, N=63)]) == E_ARG
+    assert call([ok, _chain_op(ldy=10)]) == E_ARG
+    assert call([ok, _chain_op(packed=0x100010)]) == E_ALIGN
+    assert call([ok, _chain_op(x=0x200008)]) == E_ALIGN
+    assert call([ok], ws=0) == E_WS and call([ok], ws_bytes=64) == E_WS
+    assert call([ok], ws=0x400010) == E_ALIGN
+
+
+def test_chain_workspace_bytes(lib):
+    ops = [_chain_op(), _chain_op(N=2 * 9728, K=2560, epi=1, ldy=9728, ldx=2560),
+           _chain_op(N=2560, K=9728, ldx=9728, ldy=2560, wait_for=1)]
+    b1 = q.qlin_chain_workspace_bytes(q.QLIN_Q4_0, 1, ops)
+    b8 = q.qlin_chain_workspace_bytes(q.QLIN_Q4_0, 8, ops)
+    assert 256 < b1 < b8 and b1 % 256 == 0
+    assert q.qlin_chain_workspace_bytes(q.QLIN_Q4_0, 1, [_chain_op(wait_for=0)]) == 0

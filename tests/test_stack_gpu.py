@@ -1,5 +1,6 @@
-"""The bench's workload at full size, in the launch configuration bench.py times (graph-captured,
-PDL between kernels): sampled outputs of every projection checked one by one against the oracle."""
+"""The bench's workload at full size, in the launch configurations bench.py times (graph-captured;
+one persistent GEMV chain per step, one chain per layer, or one launch per projection with PDL
+between kernels): sampled outputs of every projection checked one by one against the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -11,10 +12,11 @@ import synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("pdl", [True, False])
-def test_stack_sampled_outputs_match_oracle(pdl):
+@pytest.mark.parametrize("mode,pdl", [("chain", True), ("chain", False), ("layer_chain", True),
+                                      ("launches", True), ("launches", False)])
+def test_stack_sampled_outputs_match_oracle(mode, pdl):
     fmt, layers = synth.Q4_0, 2
-    st = bench.DenseStack(fmt, layers)
+    st = bench.DenseStack(fmt, layers, mode=mode)
     g = st.capture(pdl=pdl)
     for _ in range(3):
         g.replay()

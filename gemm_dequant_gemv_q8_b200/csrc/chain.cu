@@ -4,56 +4,83 @@
 // gate_up + SiLU, down).  Launched one by one, each GEMV pays the HBM pipeline's ramp-up at its
 // start and its slowest warp at its end; for the 2-30 MB matrices of a decode step that fixed cost
 // is as large as the streaming itself.  Weights never depend on activations, so this kernel
-// streams the weights of the whole sequence back to back through every warp's copy ring, and
-// only the activations wait: an op whose input is the output of an earlier op of the same launch
-// waits (bounded) until that op's tiles are all written, while its weights are already arriving.
-// (The pages' engines capture the decode step in CUDA graphs for the same reason: imp release
-// notes v0.4, "CUDA graphs"; the per-launch overhead is what a persistent launch removes.)
+// streams the weights of the whole sequence back to back through every warp's copy ring, and only
+// the activations wait.  (The pages' engines capture the decode step in CUDA graphs for the
+// per-launch overhead: imp release notes v0.4, "CUDA graphs".)
 //
-// Work split.  Every op is split across ALL warps of the grid into contiguous unit ranges of q or
-// q+1 units; the warps receiving the extra units rotate from op to op, so that over a chain each
-// warp streams the same number of units to within one.  A tile split between warps is finished
-// by the last-arriving contributor (atomic ticket), which sums the partials in range order:
-// results are deterministic and independent of timing.
+// Segments.  The ops are grouped by dependency level: level 0 = ops that wait for nothing, level
+// d+1 = ops waiting for an op of level d.  One level is one segment; its ops' units, concatenated
+// in the given op order, are split into one contiguous range per warp (equal to within one unit,
+// the warps receiving the extra unit rotating from segment to segment).  So a warp's range ends in
+// at most one tile shared with the next warp, whatever the number of ops in the segment, and a
+// segment never waits for itself: an op of segment d+1 waits (bounded) for the op of segment d
+// it reads, normally already finished.  A chain of independent projections is one segment; a
+// fully sequential chain is one segment per op.
+//
+// Split tiles.  A tile crossing a range boundary is computed in pieces by consecutive warps.
+// Every piece is published as 64-bit words {fp32 partial, launch tag} (single-copy atomic stores;
+// no fence, no read-modify-write), and the warp owning the tile's first unit -- its piece ends that
+// warp's range -- finishes the tile when it moves on to the next segment (or before it waits, or
+// at the end): it reads the pieces in range order, re-reading (bounded) any word whose tag is not
+// this launch's, adds them in that order and writes the tile.  Results are deterministic and
+// independent of timing; no warp waits for work another warp has not started.
 #include <algorithm>
+#include <vector>
 
 #include "gemv_core.cuh"
 
 namespace qlin {
 
-constexpr int kMaxChainOps = 256;
+constexpr int kMaxChainOps = 192;
 
 struct ChainOp {
     const uint8_t* packed;
     const void* x;
     float* y;
-    int64_t ws_off;     // byte offset of this op's tile tickets in the workspace
+    int64_t ws_off;     // byte offset of this op's partial words in the workspace
     int32_t ldx, ldy;
     int32_t N, K;       // packed rows (gate + up rows for SiLU-gate ops) and inputs
     int32_t T, G;       // tiles, k-groups
     int32_t U;          // units = T * G
-    int32_t q, r;       // split: range v has q + (v < r) units
-    int32_t rot;        // warp w has range v = (w - rot) mod W
+    int32_t base;       // first unit of this op in its segment's concatenated units
     int32_t smax;       // partial slots per tile
-    int32_t wait_for;   // earlier op whose y this op reads, or -1
+    int32_t wait_for;   // op (execution index) whose y this op reads, or -1
     int32_t epi;        // QLIN_EPI_*; bit 8: a later op waits for this one
-    int32_t part_rel;   // partials start at ws_off + part_rel
+    int32_t seg;        // segment index
+};
+
+struct ChainSeg {
+    int32_t first, end;  // ops [first, end)
+    int32_t U;           // units
+    int32_t q, r;        // range v has q + (v < r) units
+    int32_t rot;         // warp w has range v = (w - rot) mod W
 };
 
 struct ChainArgs {
     ChainOp op[kMaxChainOps];
+    ChainSeg seg[kMaxChainOps];
     uint8_t* ws;
-    int32_t n_ops;
+    int32_t n_ops, n_seg;
     int32_t M;
     int32_t W;  // warps in the grid
-    int32_t pad;
 };
 
 constexpr int kChainSignal = 0x100;
-// Workspace: [0,4) status word; [64,68) exit counter; [256, 256 + 4 n_ops) per-op count of
-// written tiles; then per op: T tickets (rounded to 256 B) and T x smax x 32 x M fp32 partials.
+// Workspace: [0,4) status word; [64,68) exit counter; [128,132) launch counter; [256, 256 +
+// 4 n_ops) per-op count of written tiles; then per op T x smax x 32 x M partial words (8 B).
 constexpr int64_t kChainExitOff = 64;
+constexpr int64_t kChainEpochOff = 128;
 constexpr int64_t kChainDoneOff = 256;
+
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const unsigned int* p) {
     uint32_t v;
@@ -65,50 +92,60 @@ __device__ __forceinline__ void red_release_add(unsigned int* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Unit range [b, e) of warp gw in op o.
-__device__ __forceinline__ void chain_range(const ChainOp& o, int gw, int W, int& b, int& e) {
-    int v = gw - o.rot;
+// Range [b, e) (segment units) of warp gw in segment s.
+__device__ __forceinline__ void seg_range(const ChainSeg& s, int gw, int W, int& b, int& e) {
+    int v = gw - s.rot;
     if (v < 0) v += W;
-    b = v * o.q + min(v, o.r);
-    e = b + o.q + (v < o.r ? 1 : 0);
+    b = v * s.q + min(v, s.r);
+    e = b + s.q + (v < s.r ? 1 : 0);
 }
 
-// Range index (v) of the warp that owns unit u of op o.
-__device__ __forceinline__ int chain_owner(const ChainOp& o, int u) {
-    const int big = o.r * (o.q + 1);
-    if (u < big) return u / (o.q + 1);
-    return o.r + (u - big) / o.q;  // q >= 1 here: u < U = W q + r
+// Range index of the warp owning segment unit u.
+__device__ __forceinline__ int seg_owner(const ChainSeg& s, int u) {
+    const int big = s.r * (s.q + 1);
+    if (u < big) return u / (s.q + 1);
+    return s.r + (u - big) / s.q;  // q >= 1 here: u < U = W q + r
 }
 
-// A warp's position in its sequence of units: op j, unit u of that op, end of its range in op j.
+// A warp's position: segment s, op j, segment unit u; its range in s ends at e.
 struct ChainCursor {
-    int j, u, e;
+    int s, j, u, e;
 };
 
-__device__ __forceinline__ void chain_seek(const ChainArgs& a, int gw, ChainCursor& c, int j) {
-    for (; j < a.n_ops; ++j) {
+// First unit of the first non-empty range of this warp in segments >= s.
+__device__ __forceinline__ void chain_seek(const ChainArgs& a, int gw, ChainCursor& c, int s) {
+    for (; s < a.n_seg; ++s) {
         int b, e;
-        chain_range(a.op[j], gw, a.W, b, e);
+        seg_range(a.seg[s], gw, a.W, b, e);
         if (e > b) {
+            int j = a.seg[s].first;
+            while (b >= a.op[j].base + a.op[j].U) ++j;
+            c.s = s;
             c.j = j;
             c.u = b;
             c.e = e;
             return;
         }
     }
+    c.s = a.n_seg;
     c.j = a.n_ops;
     c.u = c.e = 0;
 }
 
 __device__ __forceinline__ void chain_step(const ChainArgs& a, int gw, ChainCursor& c) {
-    if (++c.u >= c.e) chain_seek(a, gw, c, c.j + 1);
+    if (++c.u >= c.e) {
+        chain_seek(a, gw, c, c.s + 1);
+        return;
+    }
+    if (c.u >= a.op[c.j].base + a.op[c.j].U) ++c.j;  // ops of a segment are contiguous
 }
 
 template <int FMT>
 __device__ __forceinline__ void chain_issue(const ChainArgs& a, const ChainCursor& p, uint8_t* dst, uint64_t* bar) {
     constexpr int UB = RingCfg<FMT>::UB;
+    const ChainOp& o = a.op[p.j];
     mbar_arrive_expect_tx(bar, UB);
-    bulk_g2s(dst, a.op[p.j].packed + kHdrBytes + (int64_t)p.u * UB, UB, bar);
+    bulk_g2s(dst, o.packed + kHdrBytes + (int64_t)(p.u - o.base) * UB, UB, bar);
 }
 
 // Write tile t of op o from the reduced values (lane holds tile row (lane/8) + 4 (lane%8)).
@@ -138,54 +175,89 @@ __device__ __forceinline__ void chain_write_tile(const ChainOp& o, int M, int t,
     }
 }
 
-// Finish tile t of op j held by this warp: write it if the warp's range covers it, else store the
-// partial and take a ticket; the last contributor sums all partials in range order and writes.
-// Whoever writes the tile counts it for ops that a later op waits for.
+// Write tile t of op j (values already summed) and count it if a later op waits for op j.
 template <int MAXM>
-__device__ __forceinline__ void chain_finish_tile(const ChainArgs& a, int j, int t, int b, int e, int lane,
-                                                  float (&acc)[MAXM], float gs) {
+__device__ __forceinline__ void chain_emit(const ChainArgs& a, int j, int t, int lane, float (&v)[MAXM], float gs) {
     const ChainOp& o = a.op[j];
-    const int f = t * o.G, l = f + o.G - 1;
-    bool wrote = false;
-    if (f >= b && l < e) {
-        chain_write_tile<MAXM>(o, a.M, t, lane, acc, gs);
-        wrote = true;
-    } else {
-        const int v_first = chain_owner(o, f), v_last = chain_owner(o, l);
-        const int n_t = v_last - v_first + 1;
-        const int slot = chain_owner(o, b > f ? b : f) - v_first;
-        float* part = reinterpret_cast<float*>(a.ws + o.ws_off + o.part_rel);
-        int* cnt = reinterpret_cast<int*>(a.ws + o.ws_off);
-        float* mine = part + (((int64_t)t * o.smax + slot) * 32 + lane) * a.M;
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m)
-            if (m < a.M) __stcg(mine + m, acc[m]);
-        __threadfence();
-        __syncwarp();
-        int ticket = 0;
-        if (lane == 0) ticket = atomicAdd(cnt + t, 1);
-        ticket = __shfl_sync(0xffffffffu, ticket, 0);
-        if (ticket == n_t - 1) {
-            __threadfence();
-            float sum[MAXM];
-#pragma unroll
-            for (int m = 0; m < MAXM; ++m) sum[m] = 0.f;
-            for (int s = 0; s < n_t; ++s) {
-                const float* src = part + (((int64_t)t * o.smax + s) * 32 + lane) * a.M;
-#pragma unroll
-                for (int m = 0; m < MAXM; ++m)
-                    if (m < a.M) sum[m] += __ldcg(src + m);
-            }
-            chain_write_tile<MAXM>(o, a.M, t, lane, sum, gs);
-            if (lane == 0) cnt[t] = 0;  // leave the workspace reusable
-            wrote = true;
-        }
-    }
-    if (wrote && (o.epi & kChainSignal)) {
+    chain_write_tile<MAXM>(o, a.M, t, lane, v, gs);
+    if (o.epi & kChainSignal) {
         __threadfence();
         __syncwarp();
         if (lane == 0) red_release_add(reinterpret_cast<unsigned int*>(a.ws + kChainDoneOff) + j, 1u);
     }
+}
+
+// Split-tile geometry of tile t of op j: range index of its first piece and number of pieces.
+__device__ __forceinline__ void chain_pieces(const ChainArgs& a, int j, int t, int& v_first, int& n_t) {
+    const ChainOp& o = a.op[j];
+    const ChainSeg& s = a.seg[o.seg];
+    const int f = o.base + t * o.G;
+    v_first = seg_owner(s, f);
+    n_t = seg_owner(s, f + o.G - 1) - v_first + 1;
+}
+
+// Publish this warp's piece (slot = its place in range order) of split tile t of op j.
+template <int MAXM>
+__device__ __forceinline__ void chain_publish(const ChainArgs& a, int j, int t, int slot, int lane,
+                                              const float (&acc)[MAXM], uint32_t tag) {
+    const ChainOp& o = a.op[j];
+    uint64_t* w = reinterpret_cast<uint64_t*>(a.ws + o.ws_off) + (((int64_t)t * o.smax + slot) * 32 + lane) * a.M;
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m)
+        if (m < a.M) st_relaxed_u64(w + m, ((uint64_t)tag << 32) | __float_as_uint(acc[m]));
+}
+
+// Finish split tile t of op j: add its n_t published pieces in range order (re-reading, bounded,
+// any word not yet tagged with this launch), then write it.  False if a piece never arrived (~2 s).
+template <int MAXM>
+__device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int lane, float gs, uint32_t tag) {
+    const ChainOp& o = a.op[j];
+    int v_first, n_t;
+    chain_pieces(a, j, t, v_first, n_t);
+    const uint64_t* part = reinterpret_cast<const uint64_t*>(a.ws + o.ws_off) + ((int64_t)t * o.smax * 32 + lane) * a.M;
+    const int64_t sstride = 32 * (int64_t)a.M;  // words per slot
+    constexpr int CH = MAXM >= 16 ? 1 : 16 / MAXM;
+    float sum[MAXM];
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) sum[m] = 0.f;
+    for (int s0 = 0; s0 < n_t; s0 += CH) {
+        uint64_t w[CH][MAXM];
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m)
+                w[c][m] = (s0 + c < n_t && m < a.M) ? ld_relaxed_u64(part + (s0 + c) * sstride + m)
+                                                    : ((uint64_t)tag << 32);
+        bool ready = true;
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) ready &= (uint32_t)(w[c][m] >> 32) == tag;
+        if (!__all_sync(0xffffffffu, ready)) {  // a piece is not visible yet: re-read (bounded)
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t it = 1;; ++it) {
+                __nanosleep(100);
+                ready = true;
+#pragma unroll
+                for (int c = 0; c < CH; ++c)
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m)
+                        if (s0 + c < n_t && m < a.M && (uint32_t)(w[c][m] >> 32) != tag) {
+                            w[c][m] = ld_relaxed_u64(part + (s0 + c) * sstride + m);
+                            ready &= (uint32_t)(w[c][m] >> 32) == tag;
+                        }
+                if (__all_sync(0xffffffffu, ready)) break;
+                if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m)
+                if (s0 + c < n_t) sum[m] += __uint_as_float((uint32_t)w[c][m]);
+    }
+    chain_emit<MAXM>(a, j, t, lane, sum, gs);
+    return true;
 }
 
 // Bounded wait until every tile of op j is written (2 s); false on timeout.
@@ -222,16 +294,18 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
 #pragma unroll
         for (int s = 0; s < C::D; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
-        for (int s = 0; s < C::D && p.j < a.n_ops; ++s) {  // weights: independent of earlier kernels
+        for (int s = 0; s < C::D && p.s < a.n_seg; ++s) {  // weights: independent of earlier kernels
             chain_issue<FMT>(a, p, ring + s * C::UB, &bars[s]);
             chain_step(a, gw, p);
         }
     }
+    p.s = __shfl_sync(0xffffffffu, p.s, 0);
     p.j = __shfl_sync(0xffffffffu, p.j, 0);
     p.u = __shfl_sync(0xffffffffu, p.u, 0);
     p.e = __shfl_sync(0xffffffffu, p.e, 0);
     __syncwarp();
     griddep_wait();  // activations, outputs and the workspace may belong to the previous kernel
+    const uint32_t tag = __ldcg(reinterpret_cast<const unsigned int*>(a.ws + kChainEpochOff)) + 1u;
 
     const int part = lane & 7;
     float acc[MAXM];
@@ -244,15 +318,27 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
         for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
 
     bool failed = false;
-    int seq = 0;        // units consumed
-    int cur_op = -1;    // op of the previous unit
-    int b = 0, e = 0;   // this warp's range in cur_op
+    int pend_j = -1, pend_t = 0;  // split tile this warp finishes on leaving the segment
+    float pend_gs = 1.f;
+    int seq = 0;                  // units consumed
+    int cur_seg = -1, cur_op = -1;
+    int b = 0, e = 0;             // this warp's range in cur_seg
     float gs = 1.f;
-    while (c.j < a.n_ops) {
+    while (c.s < a.n_seg) {
         const ChainOp& o = a.op[c.j];
+        if (c.s != cur_seg) {
+            cur_seg = c.s;
+            seg_range(a.seg[c.s], gw, a.W, b, e);
+            if (pend_j >= 0) {
+                if (!chain_flush<MAXM>(a, pend_j, pend_t, lane, pend_gs, tag)) {
+                    failed = true;
+                    break;
+                }
+                pend_j = -1;
+            }
+        }
         if (c.j != cur_op) {
             cur_op = c.j;
-            chain_range(o, gw, a.W, b, e);
             gs = format_out_scale<FMT>(o.packed);
             if (o.wait_for >= 0 && !chain_wait_op(a, o.wait_for)) {
                 failed = true;
@@ -265,7 +351,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
             break;
         }
         const uint8_t* ubuf = ring + slot * C::UB;
-        const int t = c.u / o.G, g = c.u - t * o.G;
+        const int uo = c.u - o.base;
+        const int t = uo / o.G, g = uo - t * o.G;
         const int64_t k0 = (int64_t)g * kGroupK + part * 32;
         if (kOnePass) {
             const void* rows[MP];
@@ -320,15 +407,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
         }
         __syncwarp();
         // Refill this slot with the producer's next unit (the ring runs C::D units ahead).
-        if (lane == 0 && p.j < a.n_ops) {
+        if (lane == 0 && p.s < a.n_seg) {
             fence_proxy_async_smem();
             chain_issue<FMT>(a, p, ring + slot * C::UB, &bars[slot]);
         }
-        if (p.j < a.n_ops) chain_step(a, gw, p);
+        if (p.s < a.n_seg) chain_step(a, gw, p);
         ++seq;
-        const int j_now = c.j;
+        const int s_now = c.s, j_now = c.j;
         chain_step(a, gw, c);
-        if (c.j != j_now || c.u / o.G != t) {  // tile t of op j_now ends in this warp
+        if (c.s != s_now || c.j != j_now || (c.u - o.base) / o.G != t) {  // tile t of op j_now ends here
             if (kOnePass) {
                 float r[MP];
                 reduce_scatter8<MP>(acc8, lane, r);
@@ -339,21 +426,34 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
 #pragma unroll
                     for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
             }
-            chain_finish_tile<MAXM>(a, j_now, t, b, e, lane, acc, gs);
+            const int f = o.base + t * o.G;  // the tile in segment units: [f, f + G)
+            if (f >= b && f + o.G <= e) {
+                chain_emit<MAXM>(a, j_now, t, lane, acc, gs);  // the whole tile is this warp's
+            } else {
+                const ChainSeg& sg = a.seg[s_now];
+                const int sl = seg_owner(sg, b > f ? b : f) - seg_owner(sg, f);
+                chain_publish<MAXM>(a, j_now, t, sl, lane, acc, tag);
+                if (sl == 0) {  // first piece: this warp's range ends in the tile; finish it later
+                    pend_j = j_now;
+                    pend_t = t;
+                    pend_gs = gs;
+                }
+            }
 #pragma unroll
             for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
         }
     }
+    if (!failed && pend_j >= 0 && !chain_flush<MAXM>(a, pend_j, pend_t, lane, pend_gs, tag)) failed = true;
     if (failed && lane == 0) {
         atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
-        // Wait (bounded) for this warp's copies still in flight: the C::D units after seq.
+        // Wait (bounded) for this warp's copies still in flight: the C::D units from seq on.
         ChainCursor q = c;
-        for (int s = 0; s < C::D && q.j < a.n_ops; ++s) {
+        for (int s = 0; s < C::D && q.s < a.n_seg; ++s) {
             mbar_wait_bounded(&bars[(seq + s) % C::D], (uint32_t)(((seq + s) / C::D) & 1), 100000000ull);
             chain_step(a, gw, q);
         }
     }
-    // The last CTA to leave resets the per-op tile counts for the next launch.
+    // The last CTA to leave resets the per-op tile counts and advances the launch counter.
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -362,6 +462,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
             __threadfence();
             unsigned int* done = reinterpret_cast<unsigned int*>(a.ws + kChainDoneOff);
             for (int j = 0; j < a.n_ops; ++j) done[j] = 0u;
+            *reinterpret_cast<unsigned int*>(a.ws + kChainEpochOff) = tag;  // next launch tags with tag + 1
             *ex = 0u;
         }
     }
@@ -388,15 +489,34 @@ static int chain_grid(int fmt) {
 
 static int64_t al256(int64_t v) { return (v + 255) / 256 * 256; }
 
-// Fill the device descriptors; returns the workspace bytes the chain needs.
+// Execution order: by dependency level (0 = waits for nothing, d + 1 = waits for an op of level
+// d), then by the given order.  Each level becomes one segment.
+static std::vector<int> chain_levels(const qlin_gemv_op* ops, int n, std::vector<int>& level) {
+    level.assign(n, 0);
+    for (int j = 0; j < n; ++j) level[j] = ops[j].wait_for >= 0 ? level[ops[j].wait_for] + 1 : 0;
+    std::vector<int> order(n);
+    for (int j = 0; j < n; ++j) order[j] = j;
+    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return level[x] < level[y]; });
+    return order;
+}
+
+// Fill the device descriptors (if a is not null); returns the workspace bytes the chain needs.
 static int64_t chain_plan(int fmt, int M, const qlin_gemv_op* ops, int n, int W, ChainArgs* a) {
+    std::vector<int> level;
+    const std::vector<int> order = chain_levels(ops, n, level);
+    std::vector<int> pos(n);
+    for (int i = 0; i < n; ++i) pos[order[i]] = i;
+    std::vector<ChainOp> op(n);
+    std::vector<ChainSeg> seg;
     int64_t off = kChainDoneOff + al256(4 * (int64_t)n);
-    int64_t before = 0;  // units of the ops before this one
-    for (int j = 0; j < n; ++j) {
+    for (int i = 0; i < n; ++i) {
+        const int j = order[i];
         const qlin_gemv_op& u = ops[j];
+        if (i == 0 || level[j] != level[order[i - 1]]) seg.push_back(ChainSeg{i, i, 0, 0, 0, 0});
+        ChainSeg& sg = seg.back();
         const int epi = u.epilogue & 0xff;
         const Geometry geo = geometry(fmt, u.N, u.K, epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0);
-        ChainOp o = {};
+        ChainOp& o = op[i];
         o.packed = (const uint8_t*)u.packed;
         o.x = u.x;
         o.y = u.y;
@@ -407,19 +527,34 @@ static int64_t chain_plan(int fmt, int M, const qlin_gemv_op* ops, int n, int W,
         o.T = (int32_t)geo.T;
         o.G = (int32_t)geo.G;
         o.U = (int32_t)geo.U;
-        o.q = (int32_t)(geo.U / W);
-        o.r = (int32_t)(geo.U % W);
-        o.rot = (int32_t)(before % W);
-        o.smax = (int32_t)(o.q == 0 ? o.G : std::min<int64_t>(o.G, (o.G + o.q - 1) / o.q + 1));
-        o.wait_for = u.wait_for;
+        o.base = sg.U;
+        o.seg = (int32_t)seg.size() - 1;
+        o.wait_for = u.wait_for >= 0 ? pos[u.wait_for] : -1;
         o.epi = epi;
         for (int k = j + 1; k < n; ++k)
             if (ops[k].wait_for == j) o.epi |= kChainSignal;
+        sg.U += o.U;
+        sg.end = i + 1;
+    }
+    int64_t rot = 0;
+    for (ChainSeg& sg : seg) {
+        sg.q = sg.U / W;
+        sg.r = sg.U % W;
+        sg.rot = (int32_t)rot;
+        rot = (rot + sg.r) % W;  // the next segment's extra units go to the warps after these
+    }
+    for (int i = 0; i < n; ++i) {
+        ChainOp& o = op[i];
+        const int q = seg[o.seg].q;
+        o.smax = (int32_t)(q == 0 ? o.G : std::min<int64_t>(o.G, (o.G + q - 1) / q + 1));
         o.ws_off = off;
-        o.part_rel = (int32_t)al256(4 * (int64_t)o.T);
-        off += o.part_rel + al256((int64_t)o.T * o.smax * 32 * M * 4);
-        before += geo.U;
-        if (a) a->op[j] = o;
+        off += al256((int64_t)o.T * o.smax * 32 * M * 8);
+    }
+    if (a) {
+        for (int i = 0; i < n; ++i) a->op[i] = op[i];
+        for (size_t s = 0; s < seg.size(); ++s) a->seg[s] = seg[s];
+        a->n_ops = n;
+        a->n_seg = (int32_t)seg.size();
     }
     return off;
 }
@@ -478,7 +613,6 @@ extern "C" cudaError_t qlin_launch_chain(int fmt, int xdt, int M, const qlin_gem
     ChainArgs* a = new ChainArgs();  // ~20 KB: not on the caller's stack
     chain_plan(fmt, M, ops, n_ops, grid * kGemvWarps, a);
     a->ws = (uint8_t*)ws;
-    a->n_ops = n_ops;
     a->M = M;
     a->W = grid * kGemvWarps;
     const bool pdl = (flags & QLIN_FLAG_PDL) != 0, bf16 = xdt == QLIN_BF16;

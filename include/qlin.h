@@ -167,11 +167,12 @@ size_t qlin_chain_workspace_bytes(qlin_format_t fmt, int M, const qlin_gemv_op* 
  * repeated runs of one chain on one device agree bit for bit).  The weights of all ops stream back to back: the ramp-up and tail of
  * the HBM pipeline are paid once per chain instead of once per matrix, which is what a decode step
  * of many 2-30 MB projections needs (the pages capture their decode steps in CUDA graphs for the
- * per-launch overhead: imp release notes v0.4).  Ops run in order as far as their inputs allow:
- * an op with wait_for = i reads its x only after op i has written all of its y (a bounded
- * device-side wait; a wait that gives up after ~2 s sets the workspace status word, reported by
- * qlin_ws_status as QLIN_ERR_TIMEOUT).  An op without wait_for must read nothing that an op of
- * the same chain writes.  The grid holds a fixed number of CTAs per SM; the dependency waits
+ * per-launch overhead: imp release notes v0.4).  Ops run concurrently, in any order that respects
+ * wait_for: an op with wait_for = i reads its x only after op i has written all of its y (a
+ * bounded device-side wait; a wait that gives up after ~2 s sets the workspace status word,
+ * reported by qlin_ws_status as QLIN_ERR_TIMEOUT), and the library may issue such an op a few
+ * places later than given, after ops that do not wait.  No op may write memory that another op of
+ * the chain reads or writes, except the y that a waiting op reads as its x.  The grid holds a fixed number of CTAs per SM; the dependency waits
  * assume nothing else keeps SMs busy for seconds while the chain runs.
  *   ops   : host array of n_ops descriptors (1 <= n_ops <= qlin_chain_max_ops()), read during the
  *           call only

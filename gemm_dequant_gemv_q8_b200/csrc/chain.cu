@@ -175,16 +175,20 @@ __device__ __forceinline__ void chain_write_tile(const ChainOp& o, int M, int t,
     }
 }
 
-// Write tile t of op j (values already summed) and count it if a later op waits for op j.
+// Count n written tiles of op j for the ops waiting for it (one release per batch of tiles).
+__device__ __forceinline__ void chain_signal(const ChainArgs& a, int j, uint32_t n, int lane) {
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) red_release_add(reinterpret_cast<unsigned int*>(a.ws + kChainDoneOff) + j, n);
+}
+
+// Write tile t of op j (values already summed); with `signal`, count it at once.
 template <int MAXM>
-__device__ __forceinline__ void chain_emit(const ChainArgs& a, int j, int t, int lane, float (&v)[MAXM], float gs) {
+__device__ __forceinline__ void chain_emit(const ChainArgs& a, int j, int t, int lane, float (&v)[MAXM], float gs,
+                                           bool signal) {
     const ChainOp& o = a.op[j];
     chain_write_tile<MAXM>(o, a.M, t, lane, v, gs);
-    if (o.epi & kChainSignal) {
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) red_release_add(reinterpret_cast<unsigned int*>(a.ws + kChainDoneOff) + j, 1u);
-    }
+    if (signal && (o.epi & kChainSignal)) chain_signal(a, j, 1u, lane);
 }
 
 // Split-tile geometry of tile t of op j: range index of its first piece and number of pieces.
@@ -256,7 +260,7 @@ __device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int l
             for (int m = 0; m < MAXM; ++m)
                 if (s0 + c < n_t) sum[m] += __uint_as_float((uint32_t)w[c][m]);
     }
-    chain_emit<MAXM>(a, j, t, lane, sum, gs);
+    chain_emit<MAXM>(a, j, t, lane, sum, gs, true);
     return true;
 }
 
@@ -272,6 +276,17 @@ __device__ __forceinline__ bool chain_wait_op(const ChainArgs& a, int j) {
         if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
     }
 }
+
+// Shared memory of the chain kernel: the per-warp weight rings and their barriers, then (for
+// M <= 2, except Q8_0 whose ring leaves no room) two activation stages per warp.
+template <int FMT, int MAXM, bool XBF16>
+struct ChainSmem {
+    static constexpr int MP = MAXM >= 2 ? 2 : 1;
+    static constexpr bool kStaged = MAXM <= 2 && FMT != QLIN_Q8_0;
+    static constexpr int kStageBytes = MP * XStage<XBF16>::kRowBytes;  // one stage of one warp
+    static constexpr int kXOff = (RingCfg<FMT>::kSmem + 127) / 128 * 128;
+    static constexpr int kBytes = kStaged ? kXOff + kGemvWarps * 2 * kStageBytes : RingCfg<FMT>::kSmem;
+};
 
 template <int FMT, int MAXM, bool XBF16>
 __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
@@ -307,6 +322,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
     griddep_wait();  // activations, outputs and the workspace may belong to the previous kernel
     const uint32_t tag = __ldcg(reinterpret_cast<const unsigned int*>(a.ws + kChainEpochOff)) + 1u;
 
+    using XS = ChainSmem<FMT, MAXM, XBF16>;
+    uint8_t* xst = smem + XS::kXOff + warp * 2 * XS::kStageBytes;  // used only if XS::kStaged
+    bool xready = false;  // the current unit's activations were staged by the previous iteration
+    int sig_j = -1;       // written tiles of op sig_j not yet counted
+    uint32_t sig_n = 0;
     const int part = lane & 7;
     float acc[MAXM];
 #pragma unroll
@@ -340,6 +360,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
         if (c.j != cur_op) {
             cur_op = c.j;
             gs = format_out_scale<FMT>(o.packed);
+            if (sig_n) {
+                chain_signal(a, sig_j, sig_n, lane);
+                sig_n = 0;
+            }
             if (o.wait_for >= 0 && !chain_wait_op(a, o.wait_for)) {
                 failed = true;
                 break;
@@ -354,7 +378,34 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
         const int uo = c.u - o.base;
         const int t = uo / o.G, g = uo - t * o.G;
         const int64_t k0 = (int64_t)g * kGroupK + part * 32;
-        if (kOnePass) {
+        ChainCursor cn = c;  // the next unit of this warp
+        chain_step(a, gw, cn);
+        if constexpr (XS::kStaged) {
+            uint8_t* xcur = xst + (seq & 1) * XS::kStageBytes;
+            if (!xready) stage_x<XBF16, MP>(o.x, o.ldx, a.M, o.K, g, xcur, lane);
+            cp_async_wait_all();
+            __syncwarp();
+            // Stage the next unit's slice now, unless its op must first wait for another op.
+            xready = false;
+            if (cn.s < a.n_seg && (cn.j == c.j || a.op[cn.j].wait_for < 0)) {
+                const ChainOp& on = a.op[cn.j];
+                stage_x<XBF16, MP>(on.x, on.ldx, a.M, on.K, (cn.u - on.base) % on.G,
+                                   xst + ((seq + 1) & 1) * XS::kStageBytes, lane);
+                xready = true;
+            }
+            if constexpr (kH) {
+                uint32_t xh[MP][16];
+                float xsc[MP][2];
+                load_x_fp4h_staged<MP>(xcur, part, xh, xsc);
+                unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+            } else {
+                float2 xv[MP][16];
+                float xb[MP];
+                load_x_staged<XBF16, MP>(xcur, part, xv);
+                prep_x<FMT, MP>(xv, xb);
+                unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
+            }
+        } else if (kOnePass) {
             const void* rows[MP];
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm)
@@ -414,7 +465,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
         if (p.s < a.n_seg) chain_step(a, gw, p);
         ++seq;
         const int s_now = c.s, j_now = c.j;
-        chain_step(a, gw, c);
+        c = cn;
         if (c.s != s_now || c.j != j_now || (c.u - o.base) / o.G != t) {  // tile t of op j_now ends here
             if (kOnePass) {
                 float r[MP];
@@ -427,8 +478,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                     for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
             }
             const int f = o.base + t * o.G;  // the tile in segment units: [f, f + G)
-            if (f >= b && f + o.G <= e) {
-                chain_emit<MAXM>(a, j_now, t, lane, acc, gs);  // the whole tile is this warp's
+            if (f >= b && f + o.G <= e) {  // the whole tile is this warp's
+                chain_emit<MAXM>(a, j_now, t, lane, acc, gs, false);
+                if (o.epi & kChainSignal) {
+                    if (sig_n && sig_j != j_now) chain_signal(a, sig_j, sig_n, lane), sig_n = 0;
+                    sig_j = j_now;
+                    ++sig_n;
+                }
             } else {
                 const ChainSeg& sg = a.seg[s_now];
                 const int sl = seg_owner(sg, b > f ? b : f) - seg_owner(sg, f);
@@ -443,7 +499,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
             for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
         }
     }
+    if (sig_n) chain_signal(a, sig_j, sig_n, lane);
     if (!failed && pend_j >= 0 && !chain_flush<MAXM>(a, pend_j, pend_t, lane, pend_gs, tag)) failed = true;
+    if constexpr (XS::kStaged) cp_async_wait_all();  // no copy into this CTA's memory outlives it
     if (failed && lane == 0) {
         atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
         // Wait (bounded) for this warp's copies still in flight: the C::D units from seq on.
@@ -563,13 +621,14 @@ template <int FMT, int MAXM, bool XBF16>
 static cudaError_t chain_launch(const ChainArgs* a, int grid, cudaStream_t s, bool pdl) {
     using C = RingCfg<FMT>;
     auto kern = chain_kernel<FMT, MAXM, XBF16>;
+    constexpr int kSmem = ChainSmem<FMT, MAXM, XBF16>::kBytes;
     static bool attr_set = false;  // per instantiation; idempotent
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         // The dependency waits need every CTA of the grid resident at once.
         int occ = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvWarps * 32, C::kSmem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvWarps * 32, kSmem);
         if (e != cudaSuccess) return e;
         if (occ < C::kCtasPerSm) return cudaErrorLaunchOutOfResources;
         attr_set = true;
@@ -577,7 +636,7 @@ static cudaError_t chain_launch(const ChainArgs* a, int grid, cudaStream_t s, bo
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kGemvWarps * 32);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

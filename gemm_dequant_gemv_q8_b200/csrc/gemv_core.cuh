@@ -177,6 +177,28 @@ __device__ __forceinline__ void load_x_rows(const void* const (&rows)[MP], int64
 // f16 (exact except for elements more than 2^38 below the block maximum, whose contribution is
 // far below fp32 rounding), and 2^s is folded into the block's E4M3 scale.  Products then go
 // through fma.rn.f32.f16: exact products, fp32 sums.
+// One 16-element block of bf16 activations (8 words, two elements each) -> eight f16x2 words
+// scaled by 2^-s, and 2^s.
+__device__ __forceinline__ void fp4h_block(const uint32_t (&u)[8], uint32_t* xh, float& xsc) {
+    uint32_t mx = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) mx = __vmaxu2(mx, u[q] & 0x7fff7fffu);
+    const uint32_t mb = max(mx & 0xffffu, mx >> 16);
+    int s = (int)(mb >> 7) - 141;  // block max exponent - 127 - 14
+    s = s < -110 ? -110 : s;
+    const float down = __uint_as_float((uint32_t)(127 - s) << 23);  // 2^-s
+    xsc = __uint_as_float((uint32_t)(127 + s) << 23);               // 2^s
+    const float2 dd = make_float2(down, down);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float2 f = make_float2(__uint_as_float(u[q] << 16), __uint_as_float(u[q] & 0xffff0000u));
+        f = __fmul2_rn(f, dd);
+        uint32_t h;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(f.y), "f"(f.x));  // low half = even element
+        xh[q] = h;
+    }
+}
+
 template <int MP, bool CG = false>
 __device__ __forceinline__ void load_x_fp4h(const void* const (&rows)[MP], int64_t k0, int64_t K,
                                             uint32_t (&xh)[MP][16], float (&xsc)[MP][2]) {
@@ -195,23 +217,93 @@ __device__ __forceinline__ void load_x_fp4h(const void* const (&rows)[MP], int64
                 u[0] = v0.x; u[1] = v0.y; u[2] = v0.z; u[3] = v0.w;
                 u[4] = v1.x; u[5] = v1.y; u[6] = v1.z; u[7] = v1.w;
             }
-            uint32_t mx = 0;
+            fp4h_block(u, &xh[mm][8 * b], xsc[mm][b]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ activations staged in smem
+// A unit's activation slice (256 values per row) staged in shared memory by per-lane 16-byte
+// cp.async copies, one unit ahead of its use, so the L2 latency of the activations overlaps the
+// previous unit's arithmetic.  Part p (32 values) of row m sits at m * 8 * pitch + p * pitch:
+// the 16-byte pad per part puts the eight parts that a quarter-warp reads at once on disjoint
+// banks.  Values at or beyond K are zero-filled by the copy (K is a multiple of 16).
+template <bool XBF16>
+struct XStage {
+    static constexpr int kPitch = XBF16 ? 80 : 144;   // bytes per part (64 or 128 + 16)
+    static constexpr int kVecPerPart = XBF16 ? 4 : 8;  // 16-byte vectors per part
+    static constexpr int kRowBytes = 8 * kPitch;
+};
+
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Issue the copies of k-group g of MP rows (row m at x + m * ldx; rows >= M zero-filled).
+template <bool XBF16, int MP>
+__device__ __forceinline__ void stage_x(const void* x, int64_t ldx, int M, int64_t K, int g, uint8_t* buf, int lane) {
+    using S = XStage<XBF16>;
+    constexpr int kEl = XBF16 ? 8 : 4;  // values per vector
+    constexpr int kEs = XBF16 ? 2 : 4;  // bytes per value
 #pragma unroll
-            for (int q = 0; q < 8; ++q) mx = __vmaxu2(mx, u[q] & 0x7fff7fffu);
-            const uint32_t mb = max(mx & 0xffffu, mx >> 16);
-            int s = (int)(mb >> 7) - 141;  // block max exponent - 127 - 14
-            s = s < -110 ? -110 : s;
-            const float down = __uint_as_float((uint32_t)(127 - s) << 23);  // 2^-s
-            xsc[mm][b] = __uint_as_float((uint32_t)(127 + s) << 23);        // 2^s
-            const float2 dd = make_float2(down, down);
+    for (int mm = 0; mm < MP; ++mm) {
+        const uint8_t* row = reinterpret_cast<const uint8_t*>(x) + (int64_t)mm * ldx * kEs;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float2 f = make_float2(__uint_as_float(u[q] << 16), __uint_as_float(u[q] & 0xffff0000u));
-                f = __fmul2_rn(f, dd);
-                uint32_t h;
-                asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(f.y), "f"(f.x));  // low half = even element
-                xh[mm][8 * b + q] = h;
+        for (int i = 0; i < (8 * S::kVecPerPart) / 32; ++i) {
+            const int vi = lane + 32 * i, p = vi / S::kVecPerPart, q = vi % S::kVecPerPart;
+            const int64_t el = (int64_t)g * kGroupK + (int64_t)vi * kEl;
+            const bool ok = mm < M && el < K;
+            cp_async16_zfill(buf + mm * S::kRowBytes + p * S::kPitch + q * 16,
+                             ok ? (const void*)(row + el * kEs) : x, ok ? 16u : 0u);
+        }
+    }
+    cp_async_commit();
+}
+
+// A lane's 32 activations of its part from the staged slice (same result as load_x_rows).
+template <bool XBF16, int MP>
+__device__ __forceinline__ void load_x_staged(const uint8_t* buf, int part, float2 (&xv)[MP][16]) {
+    using S = XStage<XBF16>;
+#pragma unroll
+    for (int mm = 0; mm < MP; ++mm) {
+        const uint8_t* b = buf + mm * S::kRowBytes + part * S::kPitch;
+        if (XBF16) {
+#pragma unroll
+            for (int vq = 0; vq < 4; ++vq) {
+                const uint4 v = lds128(b + 16 * vq);
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    xv[mm][4 * vq + j] = make_float2(__uint_as_float(u[j] << 16), __uint_as_float(u[j] & 0xffff0000u));
             }
+        } else {
+#pragma unroll
+            for (int vq = 0; vq < 8; ++vq) {
+                const uint4 v = lds128(b + 16 * vq);
+                xv[mm][2 * vq] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+                xv[mm][2 * vq + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+            }
+        }
+    }
+}
+
+// The NVFP4 f16-product activations (see load_x_fp4h) from a staged bf16 slice.
+template <int MP>
+__device__ __forceinline__ void load_x_fp4h_staged(const uint8_t* buf, int part, uint32_t (&xh)[MP][16],
+                                                   float (&xsc)[MP][2]) {
+    using S = XStage<true>;
+#pragma unroll
+    for (int mm = 0; mm < MP; ++mm) {
+        const uint8_t* bp = buf + mm * S::kRowBytes + part * S::kPitch;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const uint4 v0 = lds128(bp + 32 * b), v1 = lds128(bp + 32 * b + 16);
+            const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            fp4h_block(u, &xh[mm][8 * b], xsc[mm][b]);
         }
     }
 }

@@ -90,13 +90,17 @@ class ClockSampler:
                 self.lines.append(f"{self.index}, {sm}, {mx}, {pw}, {r:#x}, " + ", ".join(flags))
             except Exception:
                 break
-            time.sleep(0.002)
+            time.sleep(0.001)
 
     def __enter__(self):
         try:
             nv, h = self._nvml_handle()
             self.t = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
             self.t.start()
+            t0 = time.perf_counter()
+            while not self.lines and time.perf_counter() - t0 < 2.0:  # sampling is running
+                time.sleep(0.001)
+            self.lines.clear()  # keep only samples taken inside the timed region
             return self
         except Exception:
             pass
@@ -155,20 +159,31 @@ class DenseStack:
 
     MODES = ("chain", "layer_chain", "launches")
 
-    def __init__(self, fmt, layers, M=1, device="cuda", mode="chain"):
-        """mode: "chain" = the whole step as qlin_gemv_chain launches of up to 256 ops (one for
-        36 layers); "layer_chain" = one chain of four ops per layer; "launches" = one qlin_gemv
-        per projection.  In the chains, down waits for its layer's gate_up (it reads h)."""
+    DATAFLOWS = ("stated", "serial")
+
+    def __init__(self, fmt, layers, M=1, device="cuda", mode="chain", dataflow="stated", share=None):
+        """mode: "chain" = the whole step as qlin_gemv_chain launches of up to
+        qlin_chain_max_ops() ops (one for 36 layers); "layer_chain" = one chain of four ops per
+        layer; "launches" = one qlin_gemv per projection.
+        dataflow: "stated" = every projection reads its own N(0,1) activations except down, which
+        reads its layer's h; "serial" = every projection reads the previous one's output, as in a
+        decode step (o reads the first 4096 of the 6144 qkv outputs, qkv of layer l+1 reads down
+        of layer l), so each op waits for the one before it.
+        share: another DenseStack whose packed weights and buffers this one reuses."""
         import gemm_dequant_gemv_q8_b200 as q
-        assert mode in self.MODES
+        assert mode in self.MODES and dataflow in self.DATAFLOWS
         self.q, self.fmt, self.M, self.layers, self.mode = q, fmt, M, layers, mode
+        self.dataflow = dataflow
         self.packed, self.ws = [], []
         self.weight_bytes = 0
         xs = [(l, pi, K) for l in range(layers) for pi, (n_, N, K, e) in enumerate(STACK) if n_ != "down"]
         ys = [(l, pi, N) for l in range(layers) for pi, (n_, N, K, e) in enumerate(STACK) if n_ != "gate_up"]
-        self.xbuf = torch.empty(M, sum(k for _, _, k in xs), device=device)
-        self.ybuf = torch.empty(M, sum(n for _, _, n in ys), device=device)
-        self.hbuf = torch.empty(layers, M, STACK[2][1] // 2, device=device)
+        if share is not None:
+            self.xbuf, self.ybuf, self.hbuf = share.xbuf, share.ybuf, share.hbuf
+        else:
+            self.xbuf = torch.empty(M, sum(k for _, _, k in xs), device=device)
+            self.ybuf = torch.empty(M, sum(n for _, _, n in ys), device=device)
+            self.hbuf = torch.empty(layers, M, STACK[2][1] // 2, device=device)
         self.x, self.y = {}, {}
         off = 0
         for l, pi, K in xs:
@@ -181,6 +196,8 @@ class DenseStack:
         for l in range(layers):
             self.x[(l, 3)] = self.hbuf[l]
             self.y[(l, 2)] = self.hbuf[l]
+            if share is not None:
+                continue
             lp, lw = [], []
             for pi, (name, N, K, epi) in enumerate(STACK):
                 g = synth.gen(synth.seed_for(2, l, pi), device=device)
@@ -195,6 +212,8 @@ class DenseStack:
                         M, K, synth.gen(synth.seed_for(2, l, 5 + pi), device=device), device=device))
             self.packed.append(lp)
             self.ws.append(lw)
+        if share is not None:
+            self.packed, self.ws, self.weight_bytes = share.packed, share.ws, share.weight_bytes
         torch.cuda.synchronize()
         # algorithmic bytes per step: weights once + every activation read + every output written
         act = 0
@@ -202,23 +221,30 @@ class DenseStack:
             act += 4 * M * K + 4 * M * (N // 2 if epi else N)
         self.act_bytes = act * layers
         self.step_bytes = self.weight_bytes + self.act_bytes
+        deps = {}  # (l, pi) -> the projection whose output it reads
+        for l in range(layers):
+            deps[(l, 3)] = (l, 2)
+            if dataflow == "serial":
+                if l > 0:
+                    self.x[(l, 0)] = self.y[(l - 1, 3)]
+                    deps[(l, 0)] = (l - 1, 3)
+                self.x[(l, 1)] = self.y[(l, 0)][:, :STACK[1][2]]
+                self.x[(l, 2)] = self.y[(l, 1)]
+                deps[(l, 1)], deps[(l, 2)] = (l, 0), (l, 1)
         self.chains = []  # (ops, workspace) per launch
         if mode != "launches":
-            ops = []
+            ops, index = [], {}
             for l in range(layers):
                 for pi, (name, N, K, epi) in enumerate(STACK):
-                    if mode == "layer_chain" and pi == 0:
-                        ops = []
-                    elif mode == "chain" and len(ops) + len(STACK) > q.qlin_chain_max_ops() and pi == 0:
+                    if pi == 0 and ops and (mode == "layer_chain" or
+                                            len(ops) + len(STACK) > q.qlin_chain_max_ops()):
                         self.chains.append(ops)
-                        ops = []
-                    wait = len(ops) - 1 if name == "down" else -1
+                        ops, index = [], {}
+                    wait = index.get(deps.get((l, pi)), -1)  # an op of an earlier launch is done
+                    index[(l, pi)] = len(ops)
                     ops.append(q.gemv_op(self.packed[l][pi], N, K, self.x[(l, pi)], self.y[(l, pi)],
                                          q.QLIN_EPI_SILU_GATE if epi else q.QLIN_EPI_NONE, wait))
-                    if mode == "layer_chain" and pi == len(STACK) - 1:
-                        self.chains.append(ops)
-            if mode == "chain":
-                self.chains.append(ops)
+            self.chains.append(ops)
             self.chains = [(o, q.workspace(q.qlin_chain_workspace_bytes(fmt, M, o), device)) for o in self.chains]
             self.launches_per_step = len(self.chains)
         else:
@@ -501,6 +527,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="chain", choices=list(DenseStack.MODES),
                     help="how the stack step is launched (default: one persistent GEMV chain)")
+    ap.add_argument("--dataflow", default="stated", choices=list(DenseStack.DATAFLOWS),
+                    help="stated: independent inputs, down reads h; serial: every projection reads the "
+                         "previous one's output (reported as an extra field either way)")
     ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "moe", "chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
@@ -541,7 +570,7 @@ def main():
     else:
         torch.cuda.set_device(0)
 
-    stack = DenseStack(fmt, args.layers, mode=args.mode)
+    stack = DenseStack(fmt, args.layers, mode=args.mode, dataflow=args.dataflow)
     graph = stack.capture(pdl=not args.no_pdl)
 
     def barrier():
@@ -565,6 +594,17 @@ def main():
     if world > 1:
         torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
     ms_max = float(ms_t.item())
+
+    # The other dataflow on the same weights (device-timed, same launch mode).
+    other_df = "serial" if args.dataflow == "stated" else "stated"
+    other = DenseStack(fmt, args.layers, mode=args.mode, dataflow=other_df, share=stack)
+    g2 = other.capture(pdl=not args.no_pdl)
+    other_ms = time_graph(g2, args.steps, args.warmup)
+    del g2
+    ot = torch.tensor([other_ms], device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(ot, op=torch.distributed.ReduceOp.MAX)
+    other_ms = float(ot.item())
 
     if stack.chains:
         dom_ms, dom_bytes = time_chain_kernel(stack)
@@ -598,6 +638,7 @@ def main():
             "decode_tok_s": world * 1e3 / ms_max,
             "hbm_frac": gbs / world / peak,
             "config": {"workload": workload, "format": "q4_0", "M": 1, "layers": args.layers,
+                       "dataflow": args.dataflow,
                        "weight_bytes_per_step": stack.weight_bytes, "algorithmic_bytes_per_step": stack.step_bytes,
                        "launches_per_step": stack.launches_per_step, "mode": args.mode,
                        "cuda_graph": True, "pdl": not args.no_pdl,
@@ -609,6 +650,9 @@ def main():
                          "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": dom_ms * 1e3},
             "e2e": {"value": world * stack.step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            f"{other_df}_dataflow": {"value": world * other.step_bytes / (other_ms * 1e-3) / 1e9, "unit": "GB/s",
+                                     "ms_per_step": other_ms, "mode": args.mode,
+                                     "launches_per_step": other.launches_per_step},
             "gpu_launches": stack.launches_per_step * args.steps,
             "clocks": clk.summary(),
         }

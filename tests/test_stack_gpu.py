@@ -12,11 +12,13 @@ import synth
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("mode,pdl", [("chain", True), ("chain", False), ("layer_chain", True),
-                                      ("launches", True), ("launches", False)])
-def test_stack_sampled_outputs_match_oracle(mode, pdl):
+@pytest.mark.parametrize("mode,pdl,dataflow", [("chain", True, "stated"), ("chain", False, "stated"),
+                                               ("chain", True, "serial"), ("layer_chain", True, "stated"),
+                                               ("layer_chain", True, "serial"), ("launches", True, "stated"),
+                                               ("launches", False, "serial")])
+def test_stack_sampled_outputs_match_oracle(mode, pdl, dataflow):
     fmt, layers = synth.Q4_0, 2
-    st = bench.DenseStack(fmt, layers, mode=mode)
+    st = bench.DenseStack(fmt, layers, mode=mode, dataflow=dataflow)
     g = st.capture(pdl=pdl)
     for _ in range(3):
         g.replay()

@@ -107,9 +107,10 @@ __device__ __forceinline__ int seg_owner(const ChainSeg& s, int u) {
     return s.r + (u - big) / s.q;  // q >= 1 here: u < U = W q + r
 }
 
-// A warp's position: segment s, op j, segment unit u; its range in s ends at e.
+// A warp's position: segment s, op j, segment unit u (tile t, k-group g of op j); its range in s
+// ends at e.  t and g advance incrementally: no division per unit.
 struct ChainCursor {
-    int s, j, u, e;
+    int s, j, u, e, t, g;
 };
 
 // First unit of the first non-empty range of this warp in segments >= s.
@@ -124,12 +125,14 @@ __device__ __forceinline__ void chain_seek(const ChainArgs& a, int gw, ChainCurs
             c.j = j;
             c.u = b;
             c.e = e;
+            c.t = (b - a.op[j].base) / a.op[j].G;
+            c.g = b - a.op[j].base - c.t * a.op[j].G;
             return;
         }
     }
     c.s = a.n_seg;
     c.j = a.n_ops;
-    c.u = c.e = 0;
+    c.u = c.e = c.t = c.g = 0;
 }
 
 __device__ __forceinline__ void chain_step(const ChainArgs& a, int gw, ChainCursor& c) {
@@ -137,7 +140,13 @@ __device__ __forceinline__ void chain_step(const ChainArgs& a, int gw, ChainCurs
         chain_seek(a, gw, c, c.s + 1);
         return;
     }
-    if (c.u >= a.op[c.j].base + a.op[c.j].U) ++c.j;  // ops of a segment are contiguous
+    if (c.u >= a.op[c.j].base + a.op[c.j].U) {  // ops of a segment are contiguous
+        ++c.j;
+        c.t = c.g = 0;
+    } else if (++c.g == a.op[c.j].G) {
+        c.g = 0;
+        ++c.t;
+    }
 }
 
 template <int FMT>
@@ -318,6 +327,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
     p.j = __shfl_sync(0xffffffffu, p.j, 0);
     p.u = __shfl_sync(0xffffffffu, p.u, 0);
     p.e = __shfl_sync(0xffffffffu, p.e, 0);
+    p.t = __shfl_sync(0xffffffffu, p.t, 0);
+    p.g = __shfl_sync(0xffffffffu, p.g, 0);
     __syncwarp();
     griddep_wait();  // activations, outputs and the workspace may belong to the previous kernel
     const uint32_t tag = __ldcg(reinterpret_cast<const unsigned int*>(a.ws + kChainEpochOff)) + 1u;
@@ -375,8 +386,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
             break;
         }
         const uint8_t* ubuf = ring + slot * C::UB;
-        const int uo = c.u - o.base;
-        const int t = uo / o.G, g = uo - t * o.G;
+        const int t = c.t, g = c.g;
         const int64_t k0 = (int64_t)g * kGroupK + part * 32;
         ChainCursor cn = c;  // the next unit of this warp
         chain_step(a, gw, cn);
@@ -389,7 +399,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
             xready = false;
             if (cn.s < a.n_seg && (cn.j == c.j || a.op[cn.j].wait_for < 0)) {
                 const ChainOp& on = a.op[cn.j];
-                stage_x<XBF16, MP>(on.x, on.ldx, a.M, on.K, (cn.u - on.base) % on.G,
+                stage_x<XBF16, MP>(on.x, on.ldx, a.M, on.K, cn.g,
                                    xst + ((seq + 1) & 1) * XS::kStageBytes, lane);
                 xready = true;
             }
@@ -466,7 +476,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
         ++seq;
         const int s_now = c.s, j_now = c.j;
         c = cn;
-        if (c.s != s_now || c.j != j_now || (c.u - o.base) / o.G != t) {  // tile t of op j_now ends here
+        if (c.s != s_now || c.j != j_now || c.t != t) {  // tile t of op j_now ends here
             if (kOnePass) {
                 float r[MP];
                 reduce_scatter8<MP>(acc8, lane, r);

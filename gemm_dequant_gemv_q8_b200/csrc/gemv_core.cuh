@@ -39,15 +39,21 @@ __device__ __forceinline__ float format_out_scale(const uint8_t* packed) {
     return kDenormUnscale;
 }
 
-// Q4_0 word: elements 8k..8k+7, element i at bits 4i.  Elements 0..5 are masked in place
-// (position j = i); elements 6 and 7 are taken from w >> 8 at positions 4 and 5.  Pairs:
-// (0,1) (2,3) (4,5) (6,7).
-__device__ __forceinline__ void dec_q4(uint32_t w, float2 (&p)[4]) {
-    const uint32_t h = w >> 8;
-    p[0] = make_float2(__uint_as_float(w & 0xfu), __uint_as_float(w & 0xf0u));
-    p[1] = make_float2(__uint_as_float(w & 0xf00u), __uint_as_float(w & 0xf000u));
-    p[2] = make_float2(__uint_as_float(w & 0xf0000u), __uint_as_float(w & 0xf00000u));
-    p[3] = make_float2(__uint_as_float(h & 0xf0000u), __uint_as_float(h & 0xf00000u));
+// Q4_0 words w0, w1 (elements 8k..8k+7 and 8k+8..8k+15, element i of a word at bits 4i).
+// Elements 0..5 of each word are masked in place (position j = i).  The top bytes of the two
+// words (elements 6 and 7 of each) are gathered by one byte permute into bits 0..15 of a third
+// word, where they sit at positions 0, 1 (word w0) and 2, 3 (word w1).  Pairs per word: (0,1)
+// (2,3) (4,5) (6,7).
+__device__ __forceinline__ void dec_q4_pair(uint32_t w0, uint32_t w1, float2 (&p0)[4], float2 (&p1)[4]) {
+    const uint32_t top = __byte_perm(w0, w1, 0x0073u);  // byte 0 = w0 byte 3, byte 1 = w1 byte 3
+    p0[0] = make_float2(__uint_as_float(w0 & 0xfu), __uint_as_float(w0 & 0xf0u));
+    p0[1] = make_float2(__uint_as_float(w0 & 0xf00u), __uint_as_float(w0 & 0xf000u));
+    p0[2] = make_float2(__uint_as_float(w0 & 0xf0000u), __uint_as_float(w0 & 0xf00000u));
+    p0[3] = make_float2(__uint_as_float(top & 0xfu), __uint_as_float(top & 0xf0u));
+    p1[0] = make_float2(__uint_as_float(w1 & 0xfu), __uint_as_float(w1 & 0xf0u));
+    p1[1] = make_float2(__uint_as_float(w1 & 0xf00u), __uint_as_float(w1 & 0xf000u));
+    p1[2] = make_float2(__uint_as_float(w1 & 0xf0000u), __uint_as_float(w1 & 0xf00000u));
+    p1[3] = make_float2(__uint_as_float(top & 0xf00u), __uint_as_float(top & 0xf000u));
 }
 
 // Q8_0 word: elements 4k..4k+3 stored as q + 128 in bytes 0..3.  Bytes 0..2 are masked in
@@ -86,7 +92,8 @@ __device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float (&xb)[MP])
     for (int mm = 0; mm < MP; ++mm) {
         xb[mm] = c * offset_sum(xv[mm]);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 3) == 0 ? s0 : (q & 3) == 1 ? s1 : s2);
+        for (int q = 0; q < 16; ++q)  // pair q = 4k + (q & 3); pair 4k+3 sits at positions 0,1 (k even) or 2,3
+            xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 3) == 0 ? s0 : (q & 3) == 1 ? s1 : (q & 3) == 2 ? s2 : ((q >> 2) & 1) ? s1 : s0);
     }
 }
 
@@ -380,15 +387,19 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) s0[mm] = s1[mm] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float2 p[4];
-                dec_q4(cw[k], p);
+            for (int kp = 0; kp < 2; ++kp) {
+                float2 p[2][4];
+                dec_q4_pair(cw[2 * kp], cw[2 * kp + 1], p[0], p[1]);
 #pragma unroll
-                for (int mm = 0; mm < MP; ++mm) {
-                    s0[mm] = __ffma2_rn(p[0], xv[mm][4 * k + 0], s0[mm]);
-                    s1[mm] = __ffma2_rn(p[1], xv[mm][4 * k + 1], s1[mm]);
-                    s0[mm] = __ffma2_rn(p[2], xv[mm][4 * k + 2], s0[mm]);
-                    s1[mm] = __ffma2_rn(p[3], xv[mm][4 * k + 3], s1[mm]);
+                for (int h = 0; h < 2; ++h) {
+                    const int k = 2 * kp + h;
+#pragma unroll
+                    for (int mm = 0; mm < MP; ++mm) {
+                        s0[mm] = __ffma2_rn(p[h][0], xv[mm][4 * k + 0], s0[mm]);
+                        s1[mm] = __ffma2_rn(p[h][1], xv[mm][4 * k + 1], s1[mm]);
+                        s0[mm] = __ffma2_rn(p[h][2], xv[mm][4 * k + 2], s0[mm]);
+                        s1[mm] = __ffma2_rn(p[h][3], xv[mm][4 * k + 3], s1[mm]);
+                    }
                 }
             }
             const float d = fp16_bits_to_f32(sc & 0xffffu);

@@ -204,7 +204,10 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
  *   x : M x H rows (fp32 or bf16), contiguous;  y : M x H fp32, contiguous
  *   h : optional M x top_k x I fp32 output of the SiLU-gated intermediate (NULL: kept in ws)
  *   flags: 0 or QLIN_FLAG_PDL;  ws: qlin_workspace_bytes(QLIN_OP_MOE, fmt, M, H, I, E, top_k)
- * E <= 256, top_k <= min(8, E).  Two kernel launches on `stream`, no host synchronisation. */
+ * E <= 256, top_k <= min(8, E), H <= 32768 (else QLIN_ERR_UNSUPPORTED).  One kernel launch on
+ * `stream` (routing, gate_up of the selected experts, down, weighted sum), no host
+ * synchronisation.  The status word (qlin_ws_status) reports a bad input expert id (the slot is
+ * skipped) or a timed-out device wait. */
 qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, const void* down_packed,
                                int E, int64_t H, int64_t I, int top_k, const float* router_logits,
                                int32_t* topk_ids, float* topk_w, const void* x, qlin_dtype_t xdt, int M,

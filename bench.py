@@ -447,8 +447,22 @@ def run_config(name, args):
             wb = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
             bytes_ = wb + M * (2 * H + 4 * I + 4 * I + 4 * H)
             lines.append(dict(workload="NVFP4 MLP shaped like a 27B model: gate_up 5120->2x17408 + SiLU, "
-                              "down 17408->5120, bf16 activations", M=M, us_per_layer=ms * 1e3,
-                              gbs=bytes_ / (ms * 1e-3) / 1e9, tokens_per_s=M / (ms * 1e-3)))
+                              "down 17408->5120, bf16 activations; one qlin_gemv per projection (fp32 h)",
+                              M=M, us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9,
+                              tokens_per_s=M / (ms * 1e-3)))
+            # The same layers as one GEMV chain per step, h kept in bf16 (QLIN_OUT_BF16).
+            hb = [torch.empty(M, I, device="cuda", dtype=torch.bfloat16) for _ in range(L)]
+            ops = []
+            for l in range(L):
+                ops.append(q.gemv_op(gu[l], 2 * I, H, x, hb[l], q.QLIN_EPI_SILU_GATE | q.QLIN_OUT_BF16))
+                ops.append(q.gemv_op(dn[l], H, I, hb[l], y, q.QLIN_EPI_NONE, len(ops) - 1))
+            cws = q.workspace(q.qlin_chain_workspace_bytes(fmt, M, ops))
+            fn2 = lambda: q.qlin_gemv_chain(fmt, q.QLIN_BF16, M, ops, flags=q.QLIN_FLAG_PDL, ws=cws)
+            ms2 = _time_graph_of(fn2, args.steps, args.warmup) / L
+            bytes2 = wb + M * (2 * H + 2 * I + 2 * I + 4 * H)
+            lines.append(dict(workload="NVFP4 MLP shaped like a 27B model, as above; both layers as one "
+                              "GEMV chain, h in bf16", M=M, us_per_layer=ms2 * 1e3,
+                              gbs=bytes2 / (ms2 * 1e-3) / 1e9, tokens_per_s=M / (ms2 * 1e-3)))
             del gu, dn
     elif name == "moe":
         fmt, E, H, I, k = q.QLIN_Q4_0, 32, 2048, 1792, 4

@@ -18,7 +18,7 @@ import torch
 
 QLIN_Q8_0, QLIN_Q4_0, QLIN_NVFP4 = 1, 2, 3
 QLIN_F32, QLIN_BF16 = 0, 1
-QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_FLAG_PDL = 0, 1, 0x100
+QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_OUT_BF16, QLIN_FLAG_PDL = 0, 1, 0x10, 0x100
 QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA = 0, 1, 2
 QLIN_OP_GEMV, QLIN_OP_MOE, QLIN_OP_CHUNK = 1, 2, 3
 STATUS = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED",
@@ -243,15 +243,17 @@ def qlin_status_string(status):
 
 def gemv_op(packed, N, K, x, y, epilogue=QLIN_EPI_NONE, wait_for=-1):
     """One op of a chain: the qlin_gemv arguments for one matrix (x, y CUDA tensors with
-    contiguous rows) and the index of an earlier op whose y this op's x reads (or -1)."""
+    contiguous rows; y bf16 with QLIN_OUT_BF16 in epilogue) and the index of an earlier op whose
+    y this op's x reads (or -1)."""
     if x.dim() == 1:
         x = x.unsqueeze(0)
     if y.dim() == 1:
         y = y.unsqueeze(0)
     if x.stride(1) != 1 or y.stride(1) != 1:
         raise ValueError("x and y rows must be contiguous")
+    ydt = torch.bfloat16 if epilogue & QLIN_OUT_BF16 else torch.float32
     return GemvOp(_dev(packed, "packed").value, N, K, _dev(x, "x").value, x.stride(0),
-                  _dev(y, "y", torch.float32).value, y.stride(0), epilogue, wait_for)
+                  _dev(y, "y", ydt).value, y.stride(0), epilogue, wait_for)
 
 
 def _op_array(ops):

@@ -46,14 +46,16 @@ qlin_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? QLIN_OK : Q
 // One chain op against the qlin_gemv rules (op j of the chain).
 qlin_status_t check_chain_op(int fmt, int xdt, const qlin_gemv_op& o, int j) {
     if (!valid_shape(fmt, o.N, o.K)) return QLIN_ERR_INVALID_ARG;
-    const int epi = o.epilogue;
+    if (o.epilogue & ~(0xf | QLIN_OUT_BF16)) return QLIN_ERR_INVALID_ARG;
+    const int epi = o.epilogue & 0xf;
     if (epi != QLIN_EPI_NONE && epi != QLIN_EPI_SILU_GATE) return QLIN_ERR_INVALID_ARG;
     if (epi == QLIN_EPI_SILU_GATE && (o.N % 2)) return QLIN_ERR_INVALID_ARG;
     if (!o.packed || !o.x || !o.y) return QLIN_ERR_INVALID_ARG;
     const int64_t ncols = epi == QLIN_EPI_SILU_GATE ? o.N / 2 : o.N;
     if (o.ldx < o.K || o.ldy < ncols || o.ldx >= kMaxDim || o.ldy >= kMaxDim) return QLIN_ERR_INVALID_ARG;
     if (o.wait_for < -1 || o.wait_for >= j) return QLIN_ERR_INVALID_ARG;
-    if (!aligned(o.packed, 256) || !aligned(o.x, 16) || !aligned(o.y, 4)) return QLIN_ERR_ALIGNMENT;
+    if (!aligned(o.packed, 256) || !aligned(o.x, 16) || !aligned(o.y, (o.epilogue & QLIN_OUT_BF16) ? 2 : 4))
+        return QLIN_ERR_ALIGNMENT;
     if (o.ldx % (xdt == QLIN_F32 ? 4 : 8)) return QLIN_ERR_ALIGNMENT;
     const int pack_flags = epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0;
     if (qlin::geometry(fmt, o.N, o.K, pack_flags).U >= ((int64_t)1 << 30)) return QLIN_ERR_UNSUPPORTED;

@@ -45,7 +45,7 @@ struct ChainOp {
     int32_t base;       // first unit of this op in its segment's concatenated units
     int32_t smax;       // partial slots per tile
     int32_t wait_for;   // op (execution index) whose y this op reads, or -1
-    int32_t epi;        // QLIN_EPI_*; bit 8: a later op waits for this one
+    int32_t epi;        // QLIN_EPI_* | QLIN_OUT_BF16; bit 8: a later op waits for this one
     int32_t seg;        // segment index
 };
 
@@ -164,7 +164,12 @@ __device__ __forceinline__ void chain_write_tile(const ChainOp& o, int M, int t,
     const int row = (lane >> 3) + 4 * (lane & 7);
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) v[m] = v[m] * gs;
-    if ((o.epi & 0xff) == QLIN_EPI_SILU_GATE) {
+    const bool bf16 = (o.epi & QLIN_OUT_BF16) != 0;
+    auto store = [&](int64_t idx, float val) {
+        if (bf16) reinterpret_cast<__nv_bfloat16*>(o.y)[idx] = __float2bfloat16_rn(val);
+        else o.y[idx] = val;
+    };
+    if ((o.epi & 0xf) == QLIN_EPI_SILU_GATE) {
         float u[MAXM];
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) u[m] = __shfl_down_sync(0xffffffffu, v[m], 4);
@@ -172,14 +177,14 @@ __device__ __forceinline__ void chain_write_tile(const ChainOp& o, int M, int t,
         if ((lane & 7) < 4 && i < o.N / 2) {
 #pragma unroll
             for (int m = 0; m < MAXM; ++m)
-                if (m < M) o.y[m * (int64_t)o.ldy + i] = silu_f32(v[m]) * u[m];
+                if (m < M) store(m * (int64_t)o.ldy + i, silu_f32(v[m]) * u[m]);
         }
     } else {
         const int64_t n = (int64_t)t * kTileRows + row;
         if (n < o.N) {
 #pragma unroll
             for (int m = 0; m < MAXM; ++m)
-                if (m < M) o.y[m * (int64_t)o.ldy + n] = v[m];
+                if (m < M) store(m * (int64_t)o.ldy + n, v[m]);
         }
     }
 }
@@ -582,8 +587,8 @@ static int64_t chain_plan(int fmt, int M, const qlin_gemv_op* ops, int n, int W,
         const qlin_gemv_op& u = ops[j];
         if (i == 0 || level[j] != level[order[i - 1]]) seg.push_back(ChainSeg{i, i, 0, 0, 0, 0});
         ChainSeg& sg = seg.back();
-        const int epi = u.epilogue & 0xff;
-        const Geometry geo = geometry(fmt, u.N, u.K, epi == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0);
+        const int epi = u.epilogue & (0xf | QLIN_OUT_BF16);
+        const Geometry geo = geometry(fmt, u.N, u.K, (epi & 0xf) == QLIN_EPI_SILU_GATE ? QLIN_PACK_GATE_UP : 0);
         ChainOp& o = op[i];
         o.packed = (const uint8_t*)u.packed;
         o.x = u.x;

@@ -52,6 +52,8 @@ enum {
     QLIN_EPI_SILU_GATE = 1, /* gated MLP epilogue: rows [0, N/2) are the gate g, rows [N/2, N) the
                                up projection u; y[m][i] = silu(g_i) * u_i for i < N/2, with
                                silu(z) = z / (1 + exp(-z)).  Requires a QLIN_PACK_GATE_UP buffer. */
+    QLIN_OUT_BF16 = 0x10,   /* qlin_gemv_chain ops only: y is bf16 (round to nearest even), ldy in
+                               elements -- so that a later op of a bf16 chain can read it as x */
     QLIN_FLAG_PDL = 0x100   /* launch with programmatic dependent launch: the kernel starts
                                streaming its weights while the previous kernel on the stream is
                                still running, and waits for it before touching x or y.  Only
@@ -148,9 +150,10 @@ typedef struct qlin_gemv_op {
     int64_t N, K;       /* packed rows and inputs, as for qlin_gemv (N, K < 2^31)                    */
     const void* x;      /* M x K activations in the chain's xdt, row stride ldx (qlin_gemv rules)    */
     int64_t ldx;
-    float* y;           /* M x N (N/2 with QLIN_EPI_SILU_GATE) fp32, row stride ldy                  */
+    float* y;           /* M x N (N/2 with QLIN_EPI_SILU_GATE) fp32 (bf16 with QLIN_OUT_BF16, passed
+                           through this pointer), row stride ldy elements                           */
     int64_t ldy;
-    int32_t epilogue;   /* QLIN_EPI_NONE or QLIN_EPI_SILU_GATE                                       */
+    int32_t epilogue;   /* QLIN_EPI_NONE or QLIN_EPI_SILU_GATE, optionally | QLIN_OUT_BF16           */
     int32_t wait_for;   /* -1, or the index of an EARLIER op of the same chain whose y this op's x
                            reads: the op then reads x only after every tile of that op is written */
 } qlin_gemv_op;

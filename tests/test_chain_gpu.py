@@ -21,14 +21,15 @@ TOL = 2e-6
 
 class Op:
     def __init__(self, fmt, N, K, M, seed, epi=q.QLIN_EPI_NONE, x=None, wait_for=-1, xdt=torch.float32):
-        pf = q.QLIN_PACK_GATE_UP if epi == q.QLIN_EPI_SILU_GATE else q.QLIN_PACK_DEFAULT
+        pf = q.QLIN_PACK_GATE_UP if (epi & 0xF) == q.QLIN_EPI_SILU_GATE else q.QLIN_PACK_DEFAULT
         blocks, scales, g = synth.weights(fmt, N, K, synth.gen(seed))
         self.packed = q.qlin_pack_weights(fmt, N, K, blocks.cuda(), None if scales is None else scales.cuda(), g, pf)
         self.blocks, self.scales, self.g = blocks.numpy(), None if scales is None else scales.numpy(), g
         self.fmt, self.N, self.K, self.epi, self.wait_for = fmt, N, K, epi, wait_for
         self.x = x if x is not None else synth.activations(M, K, synth.gen(seed + 1), dtype=xdt).cuda()
-        ncols = N // 2 if epi == q.QLIN_EPI_SILU_GATE else N
-        self.y = torch.full((M, ncols), float("nan"), device="cuda")
+        ncols = N // 2 if (epi & 0xF) == q.QLIN_EPI_SILU_GATE else N
+        ydt = torch.bfloat16 if epi & q.QLIN_OUT_BF16 else torch.float32
+        self.y = torch.full((M, ncols), float("nan"), device="cuda", dtype=ydt)
 
     def op(self):
         return q.gemv_op(self.packed, self.N, self.K, self.x, self.y, self.epi, self.wait_for)
@@ -37,12 +38,15 @@ class Op:
         x = self.x.double().cpu().numpy()
         y = self.y.double().cpu().numpy()
         ref, A = oracle.gemv(self.fmt, self.N, self.K, self.blocks, x, scales=self.scales, g=self.g)
-        if self.epi == q.QLIN_EPI_SILU_GATE:
+        if (self.epi & 0xF) == q.QLIN_EPI_SILU_GATE:
             href, Ah = oracle.silu_gate(ref, A)
             tol = TOL * Ah + 8 * 2.0 ** -24 * np.abs(href) + 4 * 2.0 ** -126 * (1 + np.abs(ref[:, self.N // 2:]))
             err = np.abs(y - href)
         else:
             tol, err = TOL * A, np.abs(y - ref)
+            href = ref
+        if self.epi & q.QLIN_OUT_BF16:  # one rounding to bf16 (8 significant bits): half an ulp
+            tol = tol + 2.0 ** -8 * np.abs(href) + 2.0 ** -133
         assert (err <= tol).all(), (self.N, self.K, float(np.max(err / np.maximum(tol, 1e-300))))
 
 
@@ -152,3 +156,19 @@ def test_chain_argument_checks():
     assert lib.qlin_gemv_chain(fmt, q.QLIN_F32, M, ptr, 0, 0, q._dev(ws, "ws"), ws.numel(), q._stream()) == 1
     assert lib.qlin_gemv_chain(fmt, q.QLIN_F32, 9, ptr, 1, 0, q._dev(ws, "ws"), ws.numel(), q._stream()) == 1
     assert lib.qlin_gemv_chain(fmt, q.QLIN_F32, M, ptr, 1, 0, q._dev(ws, "ws"), 16, q._stream()) == 4
+
+
+@pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_Q4_0])
+@pytest.mark.parametrize("M", [1, 4])
+def test_chain_bf16_mlp(fmt, M):
+    """A bf16 chain of gated MLPs: gate_up writes h in bf16 (QLIN_OUT_BF16), down reads it."""
+    ops = []
+    for l in range(2):
+        gu = Op(fmt, 2 * 352, 1024, M, 200 + l, epi=q.QLIN_EPI_SILU_GATE | q.QLIN_OUT_BF16, xdt=torch.bfloat16)
+        dn = Op(fmt, 288, 352, M, 210 + l, x=gu.y, wait_for=len(ops), xdt=torch.bfloat16)
+        ops += [gu, dn]
+    ws = run(fmt, torch.bfloat16, M, ops)
+    torch.cuda.synchronize()
+    assert q.qlin_ws_status(ws) == 0
+    for o in ops:
+        o.check()

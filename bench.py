@@ -283,6 +283,20 @@ class DenseStack:
         return g
 
 
+def max_over_ranks(v, world, device="cuda"):
+    """The largest of every rank's value (every rank calls it, in the same order)."""
+    t = torch.tensor([float(v)], device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(step_bytes, world, ms):
+    """Whole-job throughput: every rank streams step_bytes per step, the job takes the slowest rank's
+    time (replicas: the work per GPU is fixed as the GPU count grows)."""
+    return world * step_bytes / (ms * 1e-3) / 1e9
+
+
 def time_graph(graph, steps, warmup):
     for _ in range(warmup):
         graph.replay()
@@ -604,10 +618,7 @@ def main():
         b.synchronize()
         ms = a.elapsed_time(b) / args.steps
     barrier()
-    ms_t = torch.tensor([ms], device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, world)
 
     # The other dataflow on the same weights (device-timed, same launch mode).
     other_df = "serial" if args.dataflow == "stated" else "stated"
@@ -615,10 +626,7 @@ def main():
     g2 = other.capture(pdl=not args.no_pdl)
     other_ms = time_graph(g2, args.steps, args.warmup)
     del g2
-    ot = torch.tensor([other_ms], device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(ot, op=torch.distributed.ReduceOp.MAX)
-    other_ms = float(ot.item())
+    other_ms = max_over_ranks(other_ms, world)
 
     if stack.chains:
         dom_ms, dom_bytes = time_chain_kernel(stack)
@@ -628,15 +636,12 @@ def main():
         dom_ms, dom_bytes = time_dominant_kernel(stack)
         dom_name = "gemv_kernel<Q4_0, M=1, SiLU-gate> (gate_up 2560->19456)"
     e2e_ms, h2d, d2h = e2e_stack(stack, args.steps, args.warmup, pdl=not args.no_pdl)
-    e2e_t = torch.tensor([e2e_ms], device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(e2e_t, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(e2e_t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world)
     del graph
 
     if rank == 0:
         peak, peak_src = peaks()
-        gbs = world * stack.step_bytes / (ms_max * 1e-3) / 1e9
+        gbs = whole_job_gbs(stack.step_bytes, world, ms_max)
         dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
         traffic = None
         try:
@@ -662,9 +667,9 @@ def main():
                          "achieved": dom_gbs, "peak": peak, "peak_source": f"{peak_src} hbm_gbs (copy)",
                          "unit": "GB/s", "frac": dom_gbs / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": dom_ms * 1e3},
-            "e2e": {"value": world * stack.step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": whole_job_gbs(stack.step_bytes, world, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            f"{other_df}_dataflow": {"value": world * other.step_bytes / (other_ms * 1e-3) / 1e9, "unit": "GB/s",
+            f"{other_df}_dataflow": {"value": whole_job_gbs(other.step_bytes, world, other_ms), "unit": "GB/s",
                                      "ms_per_step": other_ms, "mode": args.mode,
                                      "launches_per_step": other.launches_per_step},
             "gpu_launches": stack.launches_per_step * args.steps,

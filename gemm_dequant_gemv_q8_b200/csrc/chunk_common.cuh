@@ -31,4 +31,128 @@ __host__ __device__ inline int64_t mma_scale_off(int kb, int r, int j, int halve
     return (int64_t)(kb * halves + h) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + j;
 }
 
+// ------------------------------------------------------------------ activation quantization
+// The rule (every step in fp32 with IEEE round-to-nearest-even):
+//   a_g  = amax|X| / (6 * 448)                       per tensor
+//   s_b  = E4M3_rne_satfinite( amax_b / (6 * a_g) )  per 16 consecutive values of a row
+//   code = E2M1_rne_satfinite( x / (e4m3(s_b) * a_g) ), 0 where that divisor is 0
+__device__ __forceinline__ float act_global_scale(float amax) { return __fdiv_rn(amax, __fmul_rn(6.0f, 448.0f)); }
+
+__device__ __forceinline__ uint8_t e4m3_rne_sat(float v) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return (uint8_t)(r & 0xffu);
+}
+
+// two E2M1 codes: low nibble from lo, high nibble from hi
+__device__ __forceinline__ uint32_t e2m1x2_rne_sat(float lo, float hi) {
+    uint32_t r;
+    asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r & 0xffu;
+}
+
+// Max |x| over the M x K bf16 activations, one partial per thread (fmaxf: a NaN input is skipped).
+// `vec`: x is 16-byte aligned and ldx % 8 == 0 (8 values per load).
+__device__ __forceinline__ float act_amax_partial(const __nv_bfloat16* __restrict__ x, int M, int64_t K, int64_t ldx,
+                                                  bool vec, int64_t tid, int64_t nthreads) {
+    float m = 0.f;
+    if (vec) {
+        const int64_t per_row = K / 8;
+        const int64_t total = (int64_t)M * per_row;
+        for (int64_t i = tid; i < total; i += nthreads) {
+            const int64_t r = i / per_row, c = i - r * per_row;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + r * ldx) + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                m = fmaxf(m, fabsf(__uint_as_float(w[j] << 16)));
+                m = fmaxf(m, fabsf(__uint_as_float(w[j] & 0xffff0000u)));
+            }
+        }
+    } else {
+        const int64_t total = (int64_t)M * K;
+        for (int64_t i = tid; i < total; i += nthreads) {
+            const int64_t r = i / K, c = i - r * K;
+            m = fmaxf(m, fabsf(__bfloat162float(x[r * ldx + c])));
+        }
+    }
+    return m;
+}
+
+// The 16 bf16 values of item (row m, 16-value block b) as 8 words (value 2j in the low half of
+// word j); zeros outside the M x K activations.
+__device__ __forceinline__ void act_load_item(const __nv_bfloat16* __restrict__ x, int M, int64_t K, int64_t ldx,
+                                              bool vec, int m, int64_t b, uint32_t (&w)[8]) {
+    const int64_t k = b * 16;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = 0u;
+    if (m >= M || k >= K) return;
+    const __nv_bfloat16* xr = x + (int64_t)m * ldx + k;
+    if (vec) {
+        const uint4 a0 = __ldg(reinterpret_cast<const uint4*>(xr));
+        const uint4 a1 = __ldg(reinterpret_cast<const uint4*>(xr) + 1);
+        w[0] = a0.x, w[1] = a0.y, w[2] = a0.z, w[3] = a0.w, w[4] = a1.x, w[5] = a1.y, w[6] = a1.z, w[7] = a1.w;
+    } else {
+        const unsigned short* xs = reinterpret_cast<const unsigned short*>(xr);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = (uint32_t)xs[2 * j] | ((uint32_t)xs[2 * j + 1] << 16);
+    }
+}
+
+__device__ __forceinline__ float act_item_amax(const uint32_t (&w)[8]) {
+    float bmax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        bmax = fmaxf(bmax, fabsf(__uint_as_float(w[j] << 16)));
+        bmax = fmaxf(bmax, fabsf(__uint_as_float(w[j] & 0xffff0000u)));
+    }
+    return bmax;
+}
+
+// Scale byte and 8 code bytes (element 2j in the low nibble of byte j) of one 16-value block.
+__device__ __forceinline__ uint8_t act_quant_block(const uint32_t (&w)[8], float bmax, float ag, uint32_t (&c8)[2]) {
+    c8[0] = c8[1] = 0u;
+    uint8_t s = 0;
+    if (ag > 0.f) s = e4m3_rne_sat(__fdiv_rn(bmax, __fmul_rn(6.0f, ag)));
+    const float div = __fmul_rn(e4m3_to_f32(s), ag);
+    if (div > 0.f) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            c8[j >> 2] |= e2m1x2_rne_sat(__fdiv_rn(__uint_as_float(w[j] << 16), div),
+                                         __fdiv_rn(__uint_as_float(w[j] & 0xffff0000u), div))
+                          << (8 * (j & 3));
+    }
+    return s;
+}
+
+// Store item (m, b) of the padded operand (TM*128 rows x G*16 blocks) in the MMA unit layout and,
+// optionally, in the canonical layout (codes [M][K/2], scales [M][K/16]).
+__device__ __forceinline__ void act_store_item(int M, int64_t K, int64_t G, int m, int64_t b, uint8_t s,
+                                               const uint32_t (&c8)[2], uint8_t* __restrict__ aq,
+                                               uint8_t* __restrict__ canon_codes, uint8_t* __restrict__ canon_scales) {
+    const int64_t k = b * 16;
+    const int tm = m / kMmaARows, r = m % kMmaARows;
+    const int64_t g = k / kGroupK;
+    const int kin = (int)(k % kGroupK);
+    uint8_t* ub = aq + ((int64_t)tm * G + g) * kMmaAUnit;
+    const int chunk = kin / 32, within = (kin % 32) / 2;  // 8 code bytes at byte 0 or 8 of the chunk
+    *reinterpret_cast<uint2*>(ub + mma_code_off(r, chunk) + within) = make_uint2(c8[0], c8[1]);
+    ub[kMmaARows * 128 + mma_scale_off(kin / 64, r, (kin % 64) / 16, 1)] = s;
+    if (canon_codes && m < M && k < K) {
+        memcpy(canon_codes + (int64_t)m * (K / 2) + k / 2, c8, 8);
+        canon_scales[(int64_t)m * (K / 16) + k / 16] = s;
+    }
+}
+
+// Load, quantize and store item (m, b); rows >= M and values >= K are written as zeros.
+__device__ __forceinline__ void act_quant_item(const __nv_bfloat16* __restrict__ x, int M, int64_t K, int64_t ldx,
+                                               int64_t G, float ag, bool vec, int m, int64_t b,
+                                               uint8_t* __restrict__ aq, uint8_t* __restrict__ canon_codes,
+                                               uint8_t* __restrict__ canon_scales) {
+    uint32_t w[8], c8[2];
+    act_load_item(x, M, K, ldx, vec, m, b, w);
+    const uint8_t s = act_quant_block(w, act_item_amax(w), ag, c8);
+    act_store_item(M, K, G, m, b, s, c8, aq, canon_codes, canon_scales);
+}
+
 }  // namespace qlin

@@ -45,18 +45,15 @@ __global__ void __launch_bounds__(256) pack_mma_kernel(const uint8_t* __restrict
 }
 
 // ------------------------------------------------------------------ activation quantization
+// The standalone form of step 1 of the chunk path, used by the inspection entry point
+// (qlin_act_quant_debug); qlin_gemm_chunk runs the same per-item code inside its persistent kernel.
 // Block-wide max of |x| folded into one word with atomicMax (order-independent, deterministic);
 // the last block to finish turns it into a_g and clears the accumulator for the next call.
 __global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __restrict__ x, int M, int64_t K,
-                                                       int64_t ldx, unsigned* __restrict__ words) {
+                                                       int64_t ldx, bool vec, unsigned* __restrict__ words) {
     // words[0] = amax bits (accumulating), words[1] = ticket, words[2] = a_g (float bits, output)
-    griddep_wait();
-    float m = 0.f;
-    const int64_t total = (int64_t)M * K;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / K, c = i - r * K;
-        m = fmaxf(m, fabsf(__bfloat162float(x[r * ldx + c])));
-    }
+    float m = act_amax_partial(x, M, K, ldx, vec, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
+                               (int64_t)gridDim.x * blockDim.x);
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     __shared__ float wmax[8];
     if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
@@ -70,71 +67,25 @@ __global__ void __launch_bounds__(256) act_amax_kernel(const __nv_bfloat16* __re
         if (ticket == gridDim.x - 1) {
             __threadfence();
             const float amax = __uint_as_float(atomicAdd(&words[0], 0u));
-            const float ag = __fdiv_rn(amax, __fmul_rn(6.0f, 448.0f));
-            words[2] = __float_as_uint(ag);
+            words[2] = __float_as_uint(act_global_scale(amax));
             words[0] = 0u;
             words[1] = 0u;
         }
     }
 }
 
-__device__ __forceinline__ uint8_t e4m3_rne_sat(float v) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-    return (uint8_t)(r & 0xffu);
-}
-
-// two E2M1 codes: low nibble from lo, high nibble from hi
-__device__ __forceinline__ uint8_t e2m1x2_rne_sat(float lo, float hi) {
-    uint32_t r;
-    asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}\n" : "=r"(r) : "f"(hi), "f"(lo));
-    return (uint8_t)(r & 0xffu);
-}
-
-// One thread per (row, 16-value block) of the padded operand.  Writes the MMA layout and,
-// optionally, the canonical layout (codes [M][K/2], scales [M][K/16]) for inspection.
+// One thread per (row, 16-value block) of the padded operand.
 __global__ void __launch_bounds__(256) act_quant_kernel(const __nv_bfloat16* __restrict__ x, int M, int64_t K,
-                                                        int64_t ldx, int64_t G, int TM, const unsigned* __restrict__ words,
-                                                        uint8_t* __restrict__ aq, uint8_t* __restrict__ canon_codes,
+                                                        int64_t ldx, int64_t G, int TM, bool vec,
+                                                        const unsigned* __restrict__ words, uint8_t* __restrict__ aq,
+                                                        uint8_t* __restrict__ canon_codes,
                                                         uint8_t* __restrict__ canon_scales) {
-    griddep_wait();
     const int64_t nblk16 = G * 16;  // 16-value blocks per padded row
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (int64_t)TM * kMmaARows * nblk16) return;
     const int m = (int)(idx / nblk16);
-    const int64_t b = idx - (int64_t)m * nblk16;
-    const int64_t k = b * 16;
-    const float ag = __uint_as_float(words[2]);
-    uint8_t codes[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    uint8_t s = 0;
-    if (m < M && k < K) {
-        float v[16];
-        float bmax = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            v[j] = __bfloat162float(x[(int64_t)m * ldx + k + j]);
-            bmax = fmaxf(bmax, fabsf(v[j]));
-        }
-        if (ag > 0.f) s = e4m3_rne_sat(__fdiv_rn(bmax, __fmul_rn(6.0f, ag)));
-        const float div = __fmul_rn(e4m3_to_f32(s), ag);
-        if (div > 0.f) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) codes[j] = e2m1x2_rne_sat(__fdiv_rn(v[2 * j], div), __fdiv_rn(v[2 * j + 1], div));
-        }
-    }
-    const int tm = m / kMmaARows, r = m % kMmaARows;
-    const int64_t g = k / kGroupK;
-    const int kin = (int)(k % kGroupK);
-    uint8_t* ub = aq + ((int64_t)tm * G + g) * kMmaAUnit;
-    const int chunk = kin / 32, within = (kin % 32) / 2;  // 8 code bytes at byte 0 or 8 of the chunk
-    uint2 cv;
-    memcpy(&cv, codes, 8);
-    *reinterpret_cast<uint2*>(ub + mma_code_off(r, chunk) + within) = cv;
-    ub[kMmaARows * 128 + mma_scale_off(kin / 64, r, (kin % 64) / 16, 1)] = s;
-    if (canon_codes && m < M && k < K) {
-        memcpy(canon_codes + (int64_t)m * (K / 2) + k / 2, codes, 8);
-        canon_scales[(int64_t)m * (K / 16) + k / 16] = s;
-    }
+    act_quant_item(x, M, K, ldx, G, __uint_as_float(words[2]), vec, m, idx - (int64_t)m * nblk16, aq, canon_codes,
+                   canon_scales);
 }
 
 }  // namespace qlin
@@ -151,26 +102,19 @@ extern "C" cudaError_t qlin_launch_pack_mma(const void* codes, const void* scale
 }
 
 extern "C" cudaError_t qlin_launch_act_quant(const void* x, int M, int64_t K, int64_t ldx, void* words, void* aq,
-                                             void* canon_codes, void* canon_scales, cudaStream_t s, bool pdl) {
+                                             void* canon_codes, void* canon_scales, cudaStream_t s) {
     const int64_t G = (K + kGroupK - 1) / kGroupK;
     const int TM = (M + kMmaARows - 1) / kMmaARows;
+    const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && (ldx % 8 == 0);
     int blocks = (int)(((int64_t)M * K + 255) / 256);
     if (blocks > 1184) blocks = 1184;
     if (blocks < 1) blocks = 1;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    cfg.blockDim = dim3(256);
-    cfg.stream = s;
-    cfg.gridDim = dim3((unsigned)blocks);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, act_amax_kernel, (const __nv_bfloat16*)x, M, K, ldx, (unsigned*)words);
+    act_amax_kernel<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)x, M, K, ldx, vec, (unsigned*)words);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t threads = (int64_t)TM * kMmaARows * G * 16;
-    cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
-    cfg.numAttrs = 1;  // depends only on the amax kernel just launched
-    return cudaLaunchKernelEx(&cfg, act_quant_kernel, (const __nv_bfloat16*)x, M, K, ldx, G, TM,
-                              (const unsigned*)words, (uint8_t*)aq, (uint8_t*)canon_codes, (uint8_t*)canon_scales);
+    act_quant_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+        (const __nv_bfloat16*)x, M, K, ldx, G, TM, vec, (const unsigned*)words, (uint8_t*)aq, (uint8_t*)canon_codes,
+        (uint8_t*)canon_scales);
+    return cudaGetLastError();
 }

@@ -86,3 +86,52 @@ def test_chunk_gemm_status_clean_and_deterministic():
     y2 = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x, ws=ws)
     assert torch.equal(y1, y2)
     assert q.qlin_ws_status(ws) == 0
+
+
+@pytest.mark.parametrize("xpad,ypad", [(0, 4), (4, 3), (8, 0)])
+def test_chunk_gemm_strided_operands(xpad, ypad):
+    """Row strides other than K and N: x rows ldx = K + xpad apart (xpad = 4: 8-byte-aligned rows,
+    the quantizer's scalar loads), y rows ldy = N + ypad apart (ypad = 3: rows not 16-byte aligned,
+    the epilogue's plain stores; otherwise the tensor-store epilogue with a pitch)."""
+    M, N, K = 70, 300, 272
+    codes, scales, g = synth.nvfp4(N, K, synth.gen(31))
+    packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA)
+    x = synth.activations(M, K, synth.gen(32), dtype=torch.bfloat16)
+    xbig = torch.zeros(M, K + xpad, dtype=torch.bfloat16)
+    xbig[:, :K] = x
+    ybig = torch.full((M, N + ypad), float("nan"), device="cuda")
+    y = ybig[:, :N]
+    q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, xbig.cuda()[:, :K], y=y)
+    torch.cuda.synchronize()
+    ac, asc, ag = oracle.act_quant(x.float().numpy())
+    xq = oracle.dequant(q.QLIN_NVFP4, M, K, ac, asc, ag)
+    yq, Aq = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xq, scales=scales.numpy(), g=g)
+    yy = y.cpu().double().numpy()
+    assert (np.abs(yy - yq) <= 2e-6 * Aq).all(), float(np.nanmax(np.abs(yy - yq) / np.maximum(Aq, 1e-300)))
+    if ypad:  # the padding columns are untouched
+        assert torch.isnan(ybig[:, N:]).all()
+
+
+@pytest.mark.parametrize("M", [1, 33, 127, 129])
+def test_chunk_gemm_ragged_rows(M):
+    """Row counts that leave part of a 128-row tile, and of a warp's 32 rows, empty."""
+    y, yq, Aq, _, _, _ = _chunk(M, 288, 512, 500 + M)
+    assert (np.abs(y - yq) <= 2e-6 * Aq).all(), float(np.max(np.abs(y - yq) / np.maximum(Aq, 1e-300)))
+
+
+def test_chunk_gemm_alternating_shapes_one_workspace():
+    """The workspace's barrier counters return to zero after every call: calls of different M
+    (different grid sizes) on one workspace all succeed with a clean status."""
+    N, K = 512, 512
+    codes, scales, g = synth.nvfp4(N, K, synth.gen(41))
+    packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA)
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, q.QLIN_NVFP4, 512, N, K))
+    for M in (512, 3, 256, 64, 512):
+        x = synth.activations(M, K, synth.gen(42 + M), dtype=torch.bfloat16)
+        y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda(), ws=ws)
+        torch.cuda.synchronize()
+        assert q.qlin_ws_status(ws) == 0
+        ac, asc, ag = oracle.act_quant(x.float().numpy())
+        xq = oracle.dequant(q.QLIN_NVFP4, M, K, ac, asc, ag)
+        yq, Aq = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xq, scales=scales.numpy(), g=g)
+        assert (np.abs(y.cpu().double().numpy() - yq) <= 2e-6 * Aq).all()

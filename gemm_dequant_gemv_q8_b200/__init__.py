@@ -18,7 +18,7 @@ import torch
 
 QLIN_Q8_0, QLIN_Q4_0, QLIN_NVFP4 = 1, 2, 3
 QLIN_F32, QLIN_BF16 = 0, 1
-QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_OUT_BF16, QLIN_FLAG_PDL = 0, 1, 0x10, 0x100
+QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_OUT_BF16, QLIN_FLAG_PDL, QLIN_FLAG_CTA_PAIRS = 0, 1, 0x10, 0x100, 0x200
 QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA = 0, 1, 2
 QLIN_OP_GEMV, QLIN_OP_MOE, QLIN_OP_CHUNK = 1, 2, 3
 STATUS = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED",

@@ -196,7 +196,7 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
     if (fmt != QLIN_NVFP4) return QLIN_ERR_UNSUPPORTED;
     if (!valid_shape(fmt, N, K) || M < 1 || M > (1 << 20)) return QLIN_ERR_INVALID_ARG;
-    if (flags & ~QLIN_FLAG_PDL) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~(QLIN_FLAG_PDL | QLIN_FLAG_CTA_PAIRS)) return QLIN_ERR_INVALID_ARG;
     if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
     if (ldx < K || ldy < N) return QLIN_ERR_INVALID_ARG;
     if (!aligned(packed, 256) || !aligned(x, 2) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;

@@ -7,41 +7,73 @@
 // "Features", row "sm_120a kernels", written there with mma.sync for sm_120a); this is the
 // datacenter-Blackwell form: TMEM accumulators, smem descriptors, a single thread issuing MMAs.
 //
-// One launch, one persistent CTA per SM:
+// One launch, persistent CTAs (one per SM):
 //   phase Q (all warps of all CTAs): max |x| over the whole tensor (one atomicMax per CTA), a
 //            bounded grid-wide barrier, a_g, then every CTA quantizes its share of the
-//            (row, 16-value block) items into the MMA operand layout; a second grid barrier.
-//   phase G (warp roles), over 128 x 256 output tiles:
+//            (row, 16-value block) items into the MMA operand layout, taken unit by unit, and
+//            counts them into a per-unit ready counter (no second grid barrier: each producer
+//            waits only for the units of its own tiles).
+//   phase G (warp roles), over output tiles of 128 * CG activation rows x 256 weight rows:
 //     warp 0   : producer -- bulk copies of one A unit (128 rows x 256 values + scales, 18 KB) and
-//                one W unit (256 rows x 256 values + scales, 36 KB) per stage, 4-stage ring;
-//     warp 1   : one thread issues the stage's 4 block-scaled MMAs (K = 64 each), commits the
-//                stage back and, after the tile's last stage, the accumulator to the epilogue;
+//                this CTA's part of one W unit (CG = 1: 256 rows, 36 KB; CG = 2: 128 rows' codes
+//                plus all 256 rows' scales, 20 KB) per stage into a shared-memory ring;
+//     warp 1   : (CG = 1, or rank 0 of a pair) one thread issues the stage's 4 block-scaled MMAs
+//                (K = 64 each), commits the stage back to every CTA of the group and, after the
+//                tile's last stage, the accumulator to the epilogues; (rank 1 of a pair) one thread
+//                tells rank 0 when a stage of this CTA is ready (data landed, scales written);
 //     warps 2-5: scale-factor writers -- move the stage's E4M3 scales from shared memory into
-//                tensor memory with tcgen05.st (one TMEM lane quarter each), so that the tensor
-//                pipe spends its time on MMAs only;
+//                tensor memory with tcgen05.st (one TMEM lane quarter each), off the tensor pipe;
 //     warps 6-9: epilogue -- tcgen05.ld of the 128 x 256 fp32 accumulator, 32 columns at a time,
-//                released to the MMAs as soon as it has been read; the scaled values go out
-//                through a small per-warp transpose buffer so that stores are row-contiguous.
+//                released to the MMAs as soon as it has been read; scaled values leave through
+//                shared memory, as TMA tensor stores of 32 x 32 boxes (CG = 2, 16-byte aligned y)
+//                or as row-contiguous plain stores.
 // Every wait is bounded; a timeout sets the status word and the CTA winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "chunk_common.cuh"
 
 namespace qlin {
 
-constexpr int kChunkStages = 4;
-constexpr int kChunkStageBytes = kMmaAUnit + kMmaWUnit;  // 55296, multiple of 1024
-constexpr int kEpiWarps = 4;
-constexpr int kEpiBuf = 32 * 64;                          // one 32 x 16 fp32 transpose buffer per warp
-constexpr int kChunkRingBytes = kChunkStages * kChunkStageBytes;
-constexpr int kChunkEpiBytes = kEpiWarps * kEpiBuf;
-constexpr int kChunkSmem = 1024 + kChunkRingBytes + kChunkEpiBytes + 256;
+constexpr int kAccCols = 256;
+
+// CG = 1: one CTA per 128 x 256 output tile (tcgen05 cta_group::1, M = 128).
+// CG = 2: a cluster of two CTAs per 256 x 256 tile (cta_group::2, M = 256): each CTA holds its
+//         128 activation rows and half of the 256 weight rows; the tensor cores of the pair
+//         exchange the halves, so each SM streams 38 KB per k-group instead of 54 KB.
+template <int CG>
+struct ChunkCfg {
+    static constexpr int kWCodes = 32768 / CG;                      // weight code bytes per CTA per k-group
+    static constexpr int kStageBytes = kMmaAUnit + kWCodes + 4096;  // + all 256 weight rows' scales
+    static constexpr int kStages = CG == 1 ? 4 : 5;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+};
+static_assert(ChunkCfg<1>::kStageBytes % 1024 == 0 && ChunkCfg<2>::kStageBytes % 1024 == 0, "stage alignment");
+// Epilogue warps 6-9, each with a staging box of kBoxRows rows x 32 fp32 columns (128-byte rows,
+// 128B-swizzled) for TMA tensor stores; the same buffer serves as a 32 x 16 transpose buffer
+// when y is not 16-byte aligned.  CG = 1 leaves room for 16-row boxes beside its 4-stage ring.
+template <int CG>
+struct EpiCfg {
+    static constexpr int kWarps = 4;
+    static constexpr int kFirstWarp = 6;
+    static constexpr int kCols = kAccCols;  // accumulator columns per warp
+    static constexpr int kBoxRows = CG == 1 ? 16 : 32;
+    static constexpr int kBuf = kBoxRows * 128;
+    static constexpr int kBytes = kWarps * kBuf;
+};
+template <int CG>
+constexpr int chunk_smem() { return 1024 + ChunkCfg<CG>::kRingBytes + EpiCfg<CG>::kBytes + 256; }
 constexpr int kChunkThreads = 320;
 constexpr int kTmemCols = 512;
-constexpr int kAccCols = 256;
 constexpr int kSfCols = 48;  // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
 constexpr int kQItems = 8;   // activation items held in registers per thread in phase Q
+static_assert(kAccCols + ChunkCfg<1>::kStages * kSfCols <= kTmemCols, "TMEM budget");
+static_assert(kAccCols + ChunkCfg<2>::kStages * kSfCols <= kTmemCols, "TMEM budget");
+static_assert(chunk_smem<1>() <= 232448 && chunk_smem<2>() <= 232448, "shared memory budget");
 
-// workspace words (after the status word): amax accumulator, barrier counters, a_g
-constexpr int kWAmax = 0, kWArrive1 = 1, kWAg = 2, kWArrive2 = 3, kWExit = 4;
+// workspace words (after the status word): amax accumulator, barrier counter, a_g, exit counter
+constexpr int kWAmax = 0, kWArrive1 = 1, kWAg = 2, kWExit = 4;
+constexpr int kUnitItems = kMmaARows * 16;  // (row, 16-value block) items of one 128 x 256 operand unit
 
 struct ChunkArgs {
     const uint8_t* w;   // QLIN_PACK_MMA buffer (header + units)
@@ -49,12 +81,13 @@ struct ChunkArgs {
     int64_t ldx;
     uint8_t* aq;        // quantized activations (units), in the workspace
     unsigned* words;
+    unsigned* ready;    // per activation unit: items quantized so far (kUnitItems when complete)
     float* y;
     int64_t ldy;
     int M;
     int64_t N, K;
-    int T2, G, TM;
-    int xvec;
+    int T2, G, TM;  // TM: 128-row activation units (a multiple of CG)
+    int xvec, tma_store;
     unsigned* status;
 };
 
@@ -65,11 +98,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     d |= (uint64_t)1 << 46;             // descriptor version for sm_100
     d |= (uint64_t)2 << 61;             // 128-byte swizzle
     return d;
-}
-
-// Instruction descriptor: E2M1 x E2M1, E4M3 scales, K-major A and B, M = 128, N = 256, K = 64.
-__host__ __device__ constexpr uint32_t chunk_idesc() {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -116,6 +144,16 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&r)[48])
         : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -123,6 +161,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
@@ -144,14 +188,115 @@ __device__ __forceinline__ bool grid_arrive_wait(unsigned* counter, unsigned tar
     }
 }
 
-__global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const ChunkArgs a) {
+
+// ------------------------------------------------------------------ CTA-pair helpers (CG = 2)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// All threads of both CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
+    asm volatile(
+        "{\n .reg .b32 ra;\n mapa.shared::cluster.u32 ra, %0, %1;\n"
+        " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}\n" ::"r"(smem_u32(bar)),
+        "r"(rank)
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait that also acquires what the other CTA of the pair released before arriving.
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((it & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
+    }
+}
+
+template <int CG>
+__device__ __forceinline__ void tc_mma_cg(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    if constexpr (CG == 1) {
+        tc_mma(d_tmem, adesc, bdesc, idesc, sfa, sfb, accumulate);
+    } else {
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+                d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+    }
+}
+// Commit this thread's MMAs to the mbarrier at `bar` in every CTA of the group.
+template <int CG>
+__device__ __forceinline__ void tc_commit_cg(uint64_t* bar) {
+    if constexpr (CG == 1) {
+        tc_commit(bar);
+    } else {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                smem_u32(bar)),
+            "h"((uint16_t)3)
+            : "memory");
+    }
+}
+// Commit to this CTA's own mbarrier only.
+template <int CG>
+__device__ __forceinline__ void tc_commit_self(uint64_t* bar) {
+    if constexpr (CG == 1)
+        tc_commit(bar);
+    else
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                     : "memory");
+}
+template <int CG>
+__device__ __forceinline__ void tmem_alloc(uint32_t* holder) {
+    if constexpr (CG == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(holder)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    } else {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(holder)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+}
+template <int CG>
+__device__ __forceinline__ void tmem_free(uint32_t tmem) {
+    if constexpr (CG == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    else
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+template <int CG>
+__global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const ChunkArgs a,
+                                                                       const __grid_constant__ CUtensorMap ymap) {
+    using Cfg = ChunkCfg<CG>;
+    using Epi = EpiCfg<CG>;
+    constexpr int S = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* epi = smem + kChunkRingBytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(epi + kChunkEpiBytes);
-    uint64_t* empty = full + kChunkStages;
-    uint64_t* sfready = empty + kChunkStages;
-    uint64_t* acc_full = sfready + kChunkStages;
+    uint8_t* epi = smem + Cfg::kRingBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(epi + Epi::kBytes);
+    uint64_t* empty = full + S;
+    uint64_t* sfready = empty + S;  // this CTA's scale writers are done with the stage
+    uint64_t* pfull = sfready + S;  // CG = 2, rank 0: the other CTA's stage is ready
+    uint64_t* acc_full = pfull + S;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* mma_done = acc_empty + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -160,59 +305,62 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     volatile float* ag_sm = reinterpret_cast<volatile float*>(issued + 1);
     float* red = const_cast<float*>(ag_sm + 1);  // one partial max per warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = CG == 1 ? 0u : cluster_ctarank();  // rank 0 issues the pair's MMAs
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kChunkStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
             mbar_init(&sfready[s], 4);
+            mbar_init(&pfull[s], 1);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kEpiWarps);
+        mbar_init(acc_empty, Epi::kWarps * CG);  // the epilogue warps of every CTA of the group
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         *issued = 0;
         fence_mbar_init();
     }
-    if (warp == 0) {  // the whole warp allocates (and later frees) tensor memory
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                     "r"(kTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
+    if (warp == 0) tmem_alloc<CG>(tmem_holder);  // the whole warp allocates (and later frees) tensor memory
     tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all();  // the pair's barriers exist before either CTA signals the other
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int ntiles = a.T2 * a.TM;
+    const int TMP = a.TM / CG;  // activation tiles of 128 * CG rows
+    const int ntiles = a.T2 * TMP;
+    const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
     griddep_wait();  // x comes from the previous kernels
 
     // ---------------------------------------------------------------- phase Q: quantize x
-    // When every thread has at most kQItems (row, 16-value block) items, the items stay in
-    // registers between the max pass and the quantization (x is read once, all loads in flight
-    // together); otherwise x is read twice.
+    // Items in unit-major order: item i belongs to unit u = i / kUnitItems (u = tm * G + g), row
+    // (i % kUnitItems) / 16 of the unit's 128 and 16-value block i % 16 of its k-group.  When every
+    // thread has at most kQItems items, they stay in registers between the max pass and the
+    // quantization (x is read once, all loads in flight together); otherwise x is read twice.
     {
         const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
         const int64_t gthreads = (int64_t)gridDim.x * blockDim.x;
-        const int64_t nblk16 = (int64_t)a.G * 16;
-        const int64_t items = (int64_t)a.TM * kMmaARows * nblk16;
+        const int64_t items = (int64_t)a.TM * a.G * kUnitItems;
         const bool resident = items <= gthreads * kQItems;
         const bool vec = a.xvec != 0;
+        auto item_mb = [&](int64_t i, int& m, int64_t& b) {
+            const int64_t u = i / kUnitItems;
+            const int within = (int)(i - u * kUnitItems);
+            const int64_t tm = u / a.G;
+            m = (int)(tm * kMmaARows) + (within >> 4);
+            b = (u - tm * a.G) * 16 + (within & 15);
+        };
         uint32_t xw[kQItems][8];
         float bmax[kQItems];
         float m = 0.f;
-        // item i = m * nblk16 + b; thread items i0 + j * gthreads, coordinates advanced without division
-        const int64_t qstep = gthreads / nblk16, rstep = gthreads - qstep * nblk16;
-        const int m_first = (int)(gtid / nblk16);
-        const int64_t b_first = gtid - (int64_t)m_first * nblk16;
         if (resident) {
-            int mj = m_first;
-            int64_t bj = b_first;
 #pragma unroll
             for (int j = 0; j < kQItems; ++j) {
-                act_load_item(a.x, gtid + j * gthreads < items ? a.M : 0, a.K, a.ldx, vec, mj, bj, xw[j]);
-                mj += (int)qstep;
-                bj += rstep;
-                if (bj >= nblk16) bj -= nblk16, ++mj;
+                const int64_t i = gtid + j * gthreads;
+                int mj = 0;
+                int64_t bj = 0;
+                if (i < items) item_mb(i, mj, bj);
+                act_load_item(a.x, i < items ? a.M : 0, a.K, a.ldx, vec, mj, bj, xw[j]);
             }
 #pragma unroll
             for (int j = 0; j < kQItems; ++j) {
@@ -243,35 +391,44 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         if (!*abort_flag) {
             const float ag = *ag_sm;
             if (resident) {
-                int mj = m_first;
-                int64_t bj = b_first;
 #pragma unroll
                 for (int j = 0; j < kQItems; ++j) {
-                    if (gtid + j * gthreads < items) {
+                    const int64_t i = gtid + j * gthreads;
+                    if (i < items) {
+                        int mj;
+                        int64_t bj;
+                        item_mb(i, mj, bj);
                         uint32_t c8[2];
                         const uint8_t sc = act_quant_block(xw[j], bmax[j], ag, c8);
                         act_store_item(a.M, a.K, a.G, mj, bj, sc, c8, a.aq, nullptr, nullptr);
                     }
-                    mj += (int)qstep;
-                    bj += rstep;
-                    if (bj >= nblk16) bj -= nblk16, ++mj;
                 }
             } else {
                 for (int64_t i = gtid; i < items; i += gthreads) {
-                    const int mrow = (int)(i / nblk16);
-                    act_quant_item(a.x, a.M, a.K, a.ldx, a.G, ag, vec, mrow, i - (int64_t)mrow * nblk16, a.aq,
-                                   nullptr, nullptr);
+                    int mi;
+                    int64_t bi;
+                    item_mb(i, mi, bi);
+                    act_quant_item(a.x, a.M, a.K, a.ldx, a.G, ag, vec, mi, bi, a.aq, nullptr, nullptr);
                 }
             }
             fence_proxy_async_global();  // the operand is read back by bulk copies (async proxy)
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            if (!grid_arrive_wait(&a.words[kWArrive2], gridDim.x)) {
-                atomicOr(a.status, 1u);
-                *abort_flag = 1;
+            __syncthreads();
+            // This CTA's items form, per pass j, the range [blockIdx.x * 320 + j * gthreads, +320):
+            // at most two units each.  Count them into the units' ready counters.
+            if (threadIdx.x == 0) __threadfence();
+            __syncthreads();
+            const int64_t first = (int64_t)blockIdx.x * blockDim.x;
+            const int64_t npass = first < items ? (items - first + gthreads - 1) / gthreads : 0;
+            for (int64_t t = threadIdx.x; t < 2 * npass; t += blockDim.x) {
+                const int64_t lo = first + (t >> 1) * gthreads;
+                const int64_t hi = lo + blockDim.x < items ? lo + blockDim.x : items;
+                const int64_t u0 = lo / kUnitItems, split = (u0 + 1) * kUnitItems;
+                if ((t & 1) == 0) {
+                    atomicAdd(&a.ready[u0], (unsigned)((hi < split ? hi : split) - lo));
+                } else if (hi > split) {
+                    atomicAdd(&a.ready[u0 + 1], (unsigned)(hi - split));
+                }
             }
-            fence_proxy_async_global();
         }
         __syncthreads();
     }
@@ -281,30 +438,54 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         if (lane == 0) {
             fence_proxy_async_global();  // this thread's bulk copies read what phase Q wrote
             int it = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
-                const int t2 = tile / a.TM, tm = tile % a.TM;
-                for (int g = 0; g < a.G; ++g, ++it) {
-                    const int s = it % kChunkStages;
-                    if (it >= kChunkStages && !mbar_wait_bounded(&empty[s], ((it / kChunkStages) - 1) & 1)) {
+            for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
+                const int t2 = tile / TMP, tm = (tile % TMP) * CG + (int)rank;
+                {  // every unit of this activation tile quantized (bounded wait)
+                    const unsigned* rd = a.ready + (int64_t)tm * a.G;
+                    const uint64_t t0 = globaltimer_ns();
+                    bool ready = false;
+                    while (!ready) {
+                        ready = true;
+                        for (int g = 0; g < a.G; ++g) ready &= ld_relaxed_gpu(rd + g) >= (unsigned)kUnitItems;
+                        if (!ready) {
+                            if (globaltimer_ns() - t0 > 2000000000ull) break;
+                            __nanosleep(64);
+                        }
+                    }
+                    if (!ready) {
                         atomicOr(a.status, 1u);
                         *abort_flag = 1;
                         break;
                     }
-                    uint8_t* st = smem + s * kChunkStageBytes;
-                    mbar_arrive_expect_tx(&full[s], kChunkStageBytes);
+                    __threadfence();             // acquire what the quantizing CTAs released
+                    fence_proxy_async_global();  // ... for the bulk copies that read it
+                }
+                for (int g = 0; g < a.G; ++g, ++it) {
+                    const int s = it % S;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ((it / S) - 1) & 1)) {
+                        atomicOr(a.status, 1u);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    uint8_t* st = smem + s * Cfg::kStageBytes;
+                    const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g) * kMmaWUnit;
+                    mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
                     bulk_g2s(st, a.aq + ((int64_t)tm * a.G + g) * kMmaAUnit, kMmaAUnit, &full[s]);
-                    bulk_g2s(st + kMmaAUnit, a.w + kHdrBytes + ((int64_t)t2 * a.G + g) * kMmaWUnit, kMmaWUnit, &full[s]);
+                    bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[s]);
+                    bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[s]);
                     *issued = it + 1;
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = chunk_idesc();
+        if (lane == 0 && rank == 0) {
+            // Instruction descriptor: E2M1 x E2M1, E4M3 scales, K-major A and B, M = 128 * CG, N = 256.
+            const uint32_t idesc =
+                (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)((128 * CG) >> 4) << 24);
             int it = 0, tcount = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tcount) {
+            for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep, ++tcount) {
                 if (tcount > 0) {
-                    if (!mbar_wait_bounded(acc_empty, (tcount - 1) & 1)) {
+                    if (!mbar_wait_cluster_bounded(acc_empty, (tcount - 1) & 1)) {
                         atomicOr(a.status, 1u);
                         *abort_flag = 1;
                         break;
@@ -313,56 +494,78 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 }
                 bool ok = true;
                 for (int g = 0; g < a.G; ++g, ++it) {
-                    const int s = it % kChunkStages;
-                    const uint32_t par = (it / kChunkStages) & 1;
-                    if (!mbar_wait_bounded(&full[s], par) || !mbar_wait_bounded(&sfready[s], par)) {
+                    const int s = it % S;
+                    const uint32_t par = (it / S) & 1;
+                    if (!mbar_wait_bounded(&full[s], par) || !mbar_wait_bounded(&sfready[s], par) ||
+                        (CG == 2 && !mbar_wait_cluster_bounded(&pfull[s], par))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + s * kChunkStageBytes);
+                    const uint32_t sa = smem_u32(smem + s * Cfg::kStageBytes);
                     const uint32_t sb = sa + kMmaAUnit;
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
-                        const uint32_t col = kAccCols + (uint32_t)(s * kSfCols + kb * 12);
-                        tc_mma(tmem, sdesc_sw128(sa + kb * 32), sdesc_sw128(sb + kb * 32), idesc, tmem + col,
-                               tmem + col + 4, (g > 0 || kb > 0) ? 1u : 0u);
+                        const uint32_t col = tmem + kAccCols + (uint32_t)(s * kSfCols + kb * 12);  // SFA 4, SFB 8
+                        tc_mma_cg<CG>(tmem, sdesc_sw128(sa + kb * 32), sdesc_sw128(sb + kb * 32), idesc, col, col + 4,
+                                      (g > 0 || kb > 0) ? 1u : 0u);
                     }
-                    tc_commit(&empty[s]);  // frees the stage (smem and its scale columns) once read
+                    tc_commit_cg<CG>(&empty[s]);  // frees the stage (smem and its scale columns) in every CTA
                 }
                 if (!ok) {
                     atomicOr(a.status, 1u);
                     *abort_flag = 1;
                     break;
                 }
-                tc_commit(acc_full);
+                tc_commit_cg<CG>(acc_full);
             }
-            // every tcgen05 operation of this thread has completed before the CTA winds down
-            tc_commit(mma_done);
+            // every tcgen05 operation of this thread has completed before the CTAs wind down
+            tc_commit_self<CG>(mma_done);
             if (!mbar_wait_bounded(mma_done, 0)) atomicOr(a.status, 1u);
+        } else if (CG == 2 && lane == 0) {
+            // rank 1: tell rank 0 when each stage of this CTA is ready (its scale writers waited for
+            // the data before writing the scales)
+            int it = 0;
+            for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
+                bool ok = true;
+                for (int g = 0; g < a.G; ++g, ++it) {
+                    const int s = it % S;
+                    if (!mbar_wait_bounded(&sfready[s], (it / S) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(&pfull[s], 0);
+                }
+                if (!ok) {
+                    atomicOr(a.status, 1u);
+                    *abort_flag = 1;
+                    break;
+                }
+            }
         }
-    } else if (warp < 2 + 4) {  // scale-factor writers: TMEM lane quarter = warp % 4
+    } else if (warp < Epi::kFirstWarp) {  // scale-factor writers: TMEM lane quarter = warp % 4
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         int it = 0;
-        for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
             bool ok = true;
             for (int g = 0; g < a.G; ++g, ++it) {
-                const int s = it % kChunkStages;
-                if (it >= kChunkStages && !mbar_wait_bounded(&empty[s], ((it / kChunkStages) - 1) & 1)) {
+                const int s = it % S;
+                if (it >= S && !mbar_wait_bounded(&empty[s], ((it / S) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                if (!mbar_wait_bounded(&full[s], (it / kChunkStages) & 1)) {
+                if (!mbar_wait_bounded(&full[s], (it / S) & 1)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 // Atom layout (both operands): the 4 scales of row r (0..127 of a 128-row half) are
                 // word r / 32 of 16-byte row r % 32.  Every lane quarter of TMEM gets the whole atom:
-                // lane 32q + i, columns c..c+3 = the atom's 16-byte row i.
-                const uint8_t* st = smem + s * kChunkStageBytes;
+                // lane 32q + i, columns c..c+3 = the atom's 16-byte row i.  Each CTA holds the
+                // scales of its own activation rows and of all 256 weight rows.
+                const uint8_t* st = smem + s * Cfg::kStageBytes;
                 const uint8_t* sfa = st + kMmaARows * 128 + lane * 16;
-                const uint8_t* sfb = st + kMmaAUnit + kMmaWRows * 128 + lane * 16;
+                const uint8_t* sfb = st + kMmaAUnit + Cfg::kWCodes + lane * 16;
                 uint32_t r[48];
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb) {
@@ -388,33 +591,63 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 break;
             }
         }
-    } else {  // epilogue warps 6..9: TMEM lane quarter = warp % 4
+    } else {  // epilogue: TMEM lane quarter = warp % 4
         const int q = warp & 3;
+        const int c_lo = ((warp - Epi::kFirstWarp) >> 2) * Epi::kCols;  // this warp's first column
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float gw_ag = __fmul_rn(reinterpret_cast<const PackedHeader*>(a.w)->global_scale, *ag_sm);
-        // 32 rows x 16 columns, row pitch 64 B, 16-byte chunk j of row r at position j ^ (r % 4)
-        uint8_t* tb = epi + (warp - 6) * kEpiBuf;
-        int tcount = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
+        uint8_t* tb = epi + (warp - Epi::kFirstWarp) * Epi::kBuf;
+        constexpr int R = Epi::kBoxRows;
+        const bool tma = a.tma_store != 0;
+        int tcount = 0, nstore = 0;
+        for (int tile = tile0; tile < ntiles; tile += tstep, ++tcount) {
             if (*abort_flag || !mbar_wait_bounded(acc_full, tcount & 1)) {
                 if (lane == 0) atomicOr(a.status, 1u);
                 *abort_flag = 1;
                 break;
             }
             tc_fence_after();
-            const int t2 = tile / a.TM, tm = tile % a.TM;
+            const int t2 = tile / TMP, tm = (tile % TMP) * CG + (int)rank;
             const int m0 = tm * kMmaARows + q * 32;  // this warp's first row
             const int64_t n0 = (int64_t)t2 * kMmaWRows;
 #pragma unroll 1
-            for (int c = 0; c < kAccCols; c += 32) {
+            for (int c = c_lo; c < c_lo + Epi::kCols; c += 32) {
                 float v[32];
                 tc_ld32(tmem + lane_base + (uint32_t)c, v);
-                if (c == kAccCols - 32) {  // the accumulator has been read: release it to the MMAs
+                if (c == c_lo + Epi::kCols - 32) {  // this warp's columns are read: release them
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(acc_empty);
+                    if (lane == 0) {
+                        if (CG == 1 || rank == 0)
+                            mbar_arrive(acc_empty);
+                        else
+                            mbar_arrive_cluster(acc_empty, 0);
+                    }
                 }
                 if (m0 >= a.M || n0 + c >= a.N) continue;
+                if (tma) {
+                    // rows hh*R .. hh*R+R-1 of the warp's 32 as one R x 32 box; row r's 16-byte chunk j
+                    // at position j ^ (r % 8) (the 128B swizzle of the tensor map)
+#pragma unroll
+                    for (int hh = 0; hh < 32 / R; ++hh) {
+                        if (m0 + hh * R >= a.M) break;
+                        if (lane == 0 && nstore > 0) bulk_wait_read_all();  // the previous store has read the box
+                        __syncwarp();
+                        if (lane / R == hh) {
+                            const int r = lane % R;
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                *reinterpret_cast<float4*>(tb + r * 128 + ((j ^ (r & 7)) << 4)) =
+                                    make_float4(v[4 * j] * gw_ag, v[4 * j + 1] * gw_ag, v[4 * j + 2] * gw_ag,
+                                                v[4 * j + 3] * gw_ag);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) tma_store_2d(&ymap, tb, (int)(n0 + c), m0 + hh * R);
+                        ++nstore;
+                    }
+                    continue;
+                }
                 // Transpose through shared memory so that each store instruction writes 8 rows x
                 // 64 contiguous bytes instead of 32 rows x 16 bytes.
 #pragma unroll
@@ -445,28 +678,38 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 }
             }
         }
+        if (tma && lane == 0) bulk_wait_all();
+        __syncwarp();
     }
     __syncthreads();
+    if (warp == 0 && lane == 0 && *abort_flag) {
+        // wait (bounded) for the last bulk copies issued to land before shared memory is released
+        const int n_it = *issued;
+        for (int j = n_it > S ? n_it - S : 0; j < n_it; ++j)
+            mbar_wait_bounded(&full[j % S], (j / S) & 1, 50000000ull);
+    }
+    // CG = 2: the pair's MMAs read both CTAs' shared memory and write both CTAs' tensor memory;
+    // neither CTA frees either before the issuing CTA has seen them complete (mma_done above).
+    if constexpr (CG == 2) cluster_sync_all();
     if (warp == 0) {
-        if (lane == 0 && *abort_flag) {
-            // wait (bounded) for the last bulk copies issued to land before shared memory is released
-            const int n_it = *issued;
-            for (int j = n_it > kChunkStages ? n_it - kChunkStages : 0; j < n_it; ++j)
-                mbar_wait_bounded(&full[j % kChunkStages], (j / kChunkStages) & 1, 50000000ull);
-        }
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+        tmem_free<CG>(tmem);
     }
-    if (threadIdx.x == 0) {  // the last CTA out clears the counters for the next call
+    // The last CTA out clears the counters for the next call.
+    if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(&a.words[kWExit], 1u) == gridDim.x - 1) {
+        *issued = atomicAdd(&a.words[kWExit], 1u) == gridDim.x - 1 ? -1 : 0;
+    }
+    __syncthreads();
+    if (*issued == -1) {
+        for (int64_t u = threadIdx.x; u < (int64_t)a.TM * a.G; u += blockDim.x) a.ready[u] = 0u;
+        if (threadIdx.x == 0) {
             a.words[kWAmax] = 0u;
             a.words[kWArrive1] = 0u;
-            a.words[kWArrive2] = 0u;
             a.words[kWExit] = 0u;
-            __threadfence();
         }
+        __threadfence();
     }
 }
 
@@ -474,25 +717,126 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
 
 using namespace qlin;
 
+// CTA pairs (cta_group::2) on request (QLIN_FLAG_CTA_PAIRS) when there are more than 128
+// activation rows; single CTAs otherwise.
+static inline int chunk_cg(int M, int flags) { return (flags & QLIN_FLAG_CTA_PAIRS) && M > kMmaARows ? 2 : 1; }
+static inline int64_t chunk_units_m(int M, int flags) {  // 128-row activation units, a multiple of the group size
+    const int cg = chunk_cg(M, flags);
+    const int64_t rows = (int64_t)kMmaARows * cg;
+    return ((M + rows - 1) / rows) * cg;
+}
+
+// Workspace: status word and counters (256 B), quantized activation units, per-unit ready counters.
+// Sized for the larger (CTA-pair) layout, so one workspace serves both.
 extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K) {
     (void)N;
-    const int64_t G = (K + kGroupK - 1) / kGroupK;
-    const int64_t TM = (M + kMmaARows - 1) / kMmaARows;
-    return 256 + (size_t)(TM * G) * kMmaAUnit;
+    const int64_t units = chunk_units_m(M, QLIN_FLAG_CTA_PAIRS) * ((K + kGroupK - 1) / kGroupK);
+    return 256 + (size_t)units * kMmaAUnit + (size_t)((units * 4 + 255) / 256) * 256;
 }
 
 extern "C" cudaError_t qlin_launch_act_quant(const void* x, int M, int64_t K, int64_t ldx, void* words, void* aq,
                                              void* canon_codes, void* canon_scales, cudaStream_t s);
 
-extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
-                                         float* y, int64_t ldy, void* ws, int flags, cudaStream_t s) {
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// y as a 2-D fp32 tensor {N (inner), M} with row pitch ldy * 4 bytes, stored in 32 x 32 boxes with
+// the 128-byte swizzle.  False when y does not meet the tensor-map rules (16-byte aligned base and
+// pitch) or the encoder is unavailable; the kernel then stores y with plain stores.
+static bool make_y_map(CUtensorMap* map, float* y, int M, int64_t N, int64_t ldy, int box_rows) {
+    if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (ldy * 4) % 16 != 0) return false;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldy * 4};
+    const cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int CG>
+static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     static bool attr_set = false;
     cudaError_t e;
     if (!attr_set) {
-        e = cudaFuncSetAttribute(chunk_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChunkSmem);
+        e = cudaFuncSetAttribute(chunk_gemm_kernel<CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk_smem<CG>());
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    // All CTAs must be co-resident (grid-wide barriers): one CTA per SM, and for CG = 2 no more
+    // pairs than the device can hold at once.
+    static int max_units = 0;  // CTAs (CG = 1) or clusters (CG = 2) resident at once, per device
+    static int cached_dev = -1;
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (CG == 2) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.blockDim = dim3(kChunkThreads);
+    cfg.dynamicSmemBytes = chunk_smem<CG>();
+    cfg.stream = s;
+    cfg.attrs = attr;
+    if (cached_dev != dev) {
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gemm_kernel<CG>, kChunkThreads,
+                                                          chunk_smem<CG>());
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        int units = sms;
+        if (CG == 2) {
+            cfg.gridDim = dim3((unsigned)(sms & ~1));
+            cfg.numAttrs = na;
+            int clusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&clusters, chunk_gemm_kernel<CG>, &cfg);
+            if (e != cudaSuccess) return e;
+            if (clusters < 1) return cudaErrorInvalidConfiguration;
+            units = clusters;
+        }
+        max_units = units;
+        cached_dev = dev;
+    }
+    const int ntiles = a.T2 * (a.TM / CG);
+    const int units = ntiles < max_units ? ntiles : max_units;
+    cfg.gridDim = dim3((unsigned)(units * CG));
+    if (flags & QLIN_FLAG_PDL) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.numAttrs = na;
+    CUtensorMap ymap;
+    memset(&ymap, 0, sizeof(ymap));
+    a.tma_store = make_y_map(&ymap, a.y, a.M, a.N, a.ldy, EpiCfg<CG>::kBoxRows) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel<CG>, a, ymap);
+}
+
+extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
+                                         float* y, int64_t ldy, void* ws, int flags, cudaStream_t s) {
     uint8_t* w8 = (uint8_t*)ws;
     ChunkArgs a;
     a.w = (const uint8_t*)packed;
@@ -500,6 +844,7 @@ extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t 
     a.ldx = ldx;
     a.aq = w8 + 256;
     a.words = (unsigned*)(w8 + 64);
+    a.ready = (unsigned*)(w8 + 256 + chunk_units_m(M, QLIN_FLAG_CTA_PAIRS) * ((K + kGroupK - 1) / kGroupK) * kMmaAUnit);
     a.y = y;
     a.ldy = ldy;
     a.M = M;
@@ -507,28 +852,11 @@ extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t 
     a.K = K;
     a.T2 = (int)((N + kMmaWRows - 1) / kMmaWRows);
     a.G = (int)((K + kGroupK - 1) / kGroupK);
-    a.TM = (M + kMmaARows - 1) / kMmaARows;
+    a.TM = (int)chunk_units_m(M, flags);
     a.xvec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && ldx % 8 == 0) ? 1 : 0;
+    a.tma_store = 0;
     a.status = (unsigned*)ws;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // All CTAs must be co-resident (grid-wide barriers): one per SM at most.
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gemm_kernel, kChunkThreads, kChunkSmem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const int ntiles = a.T2 * a.TM;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(ntiles < sms ? ntiles : sms));
-    cfg.blockDim = dim3(kChunkThreads);
-    cfg.dynamicSmemBytes = kChunkSmem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = (flags & QLIN_FLAG_PDL) ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel, a);
+    return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2>(a, flags, s) : launch_chunk_cg<1>(a, flags, s);
 }
 
 extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* ws,

@@ -54,11 +54,15 @@ enum {
                                silu(z) = z / (1 + exp(-z)).  Requires a QLIN_PACK_GATE_UP buffer. */
     QLIN_OUT_BF16 = 0x10,   /* qlin_gemv_chain ops only: y is bf16 (round to nearest even), ldy in
                                elements -- so that a later op of a bf16 chain can read it as x */
-    QLIN_FLAG_PDL = 0x100   /* launch with programmatic dependent launch: the kernel starts
+    QLIN_FLAG_PDL = 0x100,  /* launch with programmatic dependent launch: the kernel starts
                                streaming its weights while the previous kernel on the stream is
                                still running, and waits for it before touching x or y.  Only
                                valid when the packed weights were written before the previous
                                kernel on the stream started.                                      */
+    QLIN_FLAG_CTA_PAIRS = 0x200  /* qlin_gemm_chunk only, M > 128: tile with pairs of CTAs
+                               (tcgen05 cta_group::2, 256 activation rows per tile; each SM streams
+                               half of every weight tile).  Same results; the default single-CTA
+                               tiling is faster on the sizes measured so far. */
 };
 
 /* qlin_pack_weights flags */
@@ -222,14 +226,17 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
 /* NVFP4 GEMM for prefill chunks (M rows of bf16 activations, M >= 1; built for M >= 64) on the
  * tcgen05 tensor cores.  The counterpart on the pages is imp's NVFP4 block-scaled GEMM for
  * prefill (README "Features", row "sm_120a kernels": block-scaled mxf4nvf4 MMA, there with
- * mma.sync for sm_120a).  Two steps, three launches on `stream`:
+ * mma.sync for sm_120a).  One persistent launch on `stream`, two steps:
  *   1. quantize x to NVFP4 (the A operand), all in fp32 with round-to-nearest-even:
  *        a_g = amax|x| / (6 * 448);  s_b = E4M3_rne_satfinite(amax_b / (6 * a_g)) per 16 values;
  *        code = E2M1_rne_satfinite(x / (e4m3(s_b) * a_g)), 0 where that divisor is 0
+ *      (a bounded grid-wide barrier between the max and the quantization; all CTAs of the launch
+ *      are resident at once, one per SM);
  *   2. y[m][n] = (a_g * g_w) * sum_k A_q[m][k] * W_q[n][k], block scales applied inside the MMA
  *      (kind::mxf4nvf4 block16), fp32 accumulation in tensor memory.
  *   packed: qlin_pack_weights(QLIN_NVFP4, N, K, ..., QLIN_PACK_MMA);  x: bf16 M x K, row stride ldx;
- *   y: fp32, row stride ldy;  flags: 0 or QLIN_FLAG_PDL;
+ *   y: fp32, row stride ldy (16-byte aligned y and ldy % 4 == 0 take the TMA-store epilogue);
+ *   flags: QLIN_FLAG_PDL and/or QLIN_FLAG_CTA_PAIRS;
  *   ws: qlin_workspace_bytes(QLIN_OP_CHUNK, QLIN_NVFP4, M, N, K, 0, 0) bytes.
  * Other formats return QLIN_ERR_UNSUPPORTED.  Bounded device waits: a timeout sets the workspace
  * status word (qlin_ws_status). */

@@ -41,11 +41,11 @@ def test_act_quant_zero_and_outlier_rows():
     assert np.array_equal(scales.cpu().numpy(), rs) and np.array_equal(codes.cpu().numpy(), rc)
 
 
-def _chunk(M, N, K, seed, rows=None):
+def _chunk(M, N, K, seed, rows=None, flags=0):
     codes, scales, g = synth.nvfp4(N, K, synth.gen(seed))
     packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA)
     x = synth.activations(M, K, synth.gen(seed + 1), dtype=torch.bfloat16)
-    y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda())
+    y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda(), flags=flags)
     torch.cuda.synchronize()
     ac, asc, ag = oracle.act_quant(x.float().numpy())
     if rows is None:
@@ -58,18 +58,19 @@ def _chunk(M, N, K, seed, rows=None):
     return y.cpu().double().numpy()[:, rows], yq, Aq, ye, Ae, Ed
 
 
+@pytest.mark.parametrize("flags", [0, q.QLIN_FLAG_CTA_PAIRS])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (70, 300, 272), (200, 512, 1024)])
-def test_chunk_gemm_small(M, N, K):
-    y, yq, Aq, _, _, _ = _chunk(M, N, K, 10 * M + N)
+def test_chunk_gemm_small(M, N, K, flags):
+    y, yq, Aq, _, _, _ = _chunk(M, N, K, 10 * M + N, flags=flags)
     err = np.abs(y - yq)
     assert (err <= 2e-6 * Aq).all(), float(np.max(err / np.maximum(Aq, 1e-300)))
 
 
-@pytest.mark.parametrize("M", [64, 512])
-def test_chunk_gemm_27b_shape_sampled(M):
+@pytest.mark.parametrize("M,flags", [(64, 0), (512, 0), (512, q.QLIN_FLAG_CTA_PAIRS)])
+def test_chunk_gemm_27b_shape_sampled(M, flags):
     N, K = 17408, 5120
     rows = np.unique(np.concatenate([[0, 255, 256, N - 1], np.random.default_rng(M).integers(0, N, 60)]))
-    y, yq, Aq, ye, Ae, Ed = _chunk(M, N, K, 77, rows)
+    y, yq, Aq, ye, Ae, Ed = _chunk(M, N, K, 77, rows, flags=flags)
     assert (np.abs(y - yq) <= 2e-6 * Aq).all(), float(np.max(np.abs(y - yq) / np.maximum(Aq, 1e-300)))
     assert (np.abs(y - ye) <= 2e-6 * Aq + Ed + 1e-12 * Ae).all()
     rel = np.abs(y - ye) / Ae
@@ -88,12 +89,13 @@ def test_chunk_gemm_status_clean_and_deterministic():
     assert q.qlin_ws_status(ws) == 0
 
 
+@pytest.mark.parametrize("flags", [0, q.QLIN_FLAG_CTA_PAIRS])
 @pytest.mark.parametrize("xpad,ypad", [(0, 4), (4, 3), (8, 0)])
-def test_chunk_gemm_strided_operands(xpad, ypad):
+def test_chunk_gemm_strided_operands(xpad, ypad, flags):
     """Row strides other than K and N: x rows ldx = K + xpad apart (xpad = 4: 8-byte-aligned rows,
     the quantizer's scalar loads), y rows ldy = N + ypad apart (ypad = 3: rows not 16-byte aligned,
     the epilogue's plain stores; otherwise the tensor-store epilogue with a pitch)."""
-    M, N, K = 70, 300, 272
+    M, N, K = 170, 300, 272
     codes, scales, g = synth.nvfp4(N, K, synth.gen(31))
     packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA)
     x = synth.activations(M, K, synth.gen(32), dtype=torch.bfloat16)
@@ -101,7 +103,7 @@ def test_chunk_gemm_strided_operands(xpad, ypad):
     xbig[:, :K] = x
     ybig = torch.full((M, N + ypad), float("nan"), device="cuda")
     y = ybig[:, :N]
-    q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, xbig.cuda()[:, :K], y=y)
+    q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, xbig.cuda()[:, :K], y=y, flags=flags)
     torch.cuda.synchronize()
     ac, asc, ag = oracle.act_quant(x.float().numpy())
     xq = oracle.dequant(q.QLIN_NVFP4, M, K, ac, asc, ag)
@@ -112,10 +114,12 @@ def test_chunk_gemm_strided_operands(xpad, ypad):
         assert torch.isnan(ybig[:, N:]).all()
 
 
-@pytest.mark.parametrize("M", [1, 33, 127, 129])
-def test_chunk_gemm_ragged_rows(M):
-    """Row counts that leave part of a 128-row tile, and of a warp's 32 rows, empty."""
-    y, yq, Aq, _, _, _ = _chunk(M, 288, 512, 500 + M)
+@pytest.mark.parametrize("flags", [0, q.QLIN_FLAG_CTA_PAIRS])
+@pytest.mark.parametrize("M", [1, 33, 127, 129, 257, 300])
+def test_chunk_gemm_ragged_rows(M, flags):
+    """Row counts that leave part of a 128-row tile (or of a 256-row tile of a CTA pair), and of a
+    warp's 32 rows, empty; M = 300 leaves one CTA of the second pair without any row."""
+    y, yq, Aq, _, _, _ = _chunk(M, 288, 512, 500 + M, flags=flags)
     assert (np.abs(y - yq) <= 2e-6 * Aq).all(), float(np.max(np.abs(y - yq) / np.maximum(Aq, 1e-300)))
 
 
@@ -126,9 +130,9 @@ def test_chunk_gemm_alternating_shapes_one_workspace():
     codes, scales, g = synth.nvfp4(N, K, synth.gen(41))
     packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA)
     ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, q.QLIN_NVFP4, 512, N, K))
-    for M in (512, 3, 256, 64, 512):
+    for M, fl in ((512, 0), (3, 0), (256, q.QLIN_FLAG_CTA_PAIRS), (64, 0), (512, q.QLIN_FLAG_CTA_PAIRS), (300, 0)):
         x = synth.activations(M, K, synth.gen(42 + M), dtype=torch.bfloat16)
-        y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda(), ws=ws)
+        y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda(), ws=ws, flags=fl)
         torch.cuda.synchronize()
         assert q.qlin_ws_status(ws) == 0
         ac, asc, ag = oracle.act_quant(x.float().numpy())

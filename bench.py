@@ -535,7 +535,7 @@ def run_config(name, args):
             flop = 2.0 * M * N * K
             bytes_ = (q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA) - 256) + 2 * M * K + 4 * M * N
             lines.append(dict(workload=f"NVFP4 prefill-chunk GEMM M={M} K=5120 N=17408 (activation quantization "
-                              "+ tcgen05 block-scaled GEMM, 3 launches)", M=M, us_per_call=ms * 1e3,
+                              "+ tcgen05 block-scaled GEMM in one persistent launch)", M=M, us_per_call=ms * 1e3,
                               tflops=flop / (ms * 1e-3) / 1e12, fp4_peak_tflops=fp4_peak, fp4_peak_source=fp4_src,
                               fp4_frac=flop / (ms * 1e-3) / 1e12 / fp4_peak, gbs=bytes_ / (ms * 1e-3) / 1e9))
     for ln in lines:

@@ -251,24 +251,38 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Issue the copies of k-group g of MP rows (row m at x + m * ldx; rows >= M zero-filled).
+// Stage the k-group g slice of MP activation rows (row mm at rows[mm]; NULL rows and values at or
+// beyond K are zero-filled) into buf, 16-byte cp.async copies in the XStage layout.  `any` is a
+// valid global address given to the zero-filling copies (they read nothing from it).
 template <bool XBF16, int MP>
-__device__ __forceinline__ void stage_x(const void* x, int64_t ldx, int M, int64_t K, int g, uint8_t* buf, int lane) {
+__device__ __forceinline__ void stage_x_rows(const void* const (&rows)[MP], int64_t K, int g, uint8_t* buf, int lane,
+                                             const void* any) {
     using S = XStage<XBF16>;
     constexpr int kEl = XBF16 ? 8 : 4;  // values per vector
     constexpr int kEs = XBF16 ? 2 : 4;  // bytes per value
 #pragma unroll
     for (int mm = 0; mm < MP; ++mm) {
-        const uint8_t* row = reinterpret_cast<const uint8_t*>(x) + (int64_t)mm * ldx * kEs;
+        const uint8_t* row = reinterpret_cast<const uint8_t*>(rows[mm]);
 #pragma unroll
         for (int i = 0; i < (8 * S::kVecPerPart) / 32; ++i) {
             const int vi = lane + 32 * i, p = vi / S::kVecPerPart, q = vi % S::kVecPerPart;
             const int64_t el = (int64_t)g * kGroupK + (int64_t)vi * kEl;
-            const bool ok = mm < M && el < K;
+            const bool ok = row != nullptr && el < K;
             cp_async16_zfill(buf + mm * S::kRowBytes + p * S::kPitch + q * 16,
-                             ok ? (const void*)(row + el * kEs) : x, ok ? 16u : 0u);
+                             ok ? (const void*)(row + el * kEs) : any, ok ? 16u : 0u);
         }
     }
     cp_async_commit();
+}
+
+template <bool XBF16, int MP>
+__device__ __forceinline__ void stage_x(const void* x, int64_t ldx, int M, int64_t K, int g, uint8_t* buf, int lane) {
+    constexpr int kEs = XBF16 ? 2 : 4;
+    const void* rows[MP];
+#pragma unroll
+    for (int mm = 0; mm < MP; ++mm)
+        rows[mm] = mm < M ? (const void*)(reinterpret_cast<const uint8_t*>(x) + (int64_t)mm * ldx * kEs) : nullptr;
+    stage_x_rows<XBF16, MP>(rows, K, g, buf, lane, x);
 }
 
 // A lane's 32 activations of its part from the staged slice (same result as load_x_rows).

@@ -82,15 +82,26 @@ __device__ void moe_route(const MoeArgs& a, RouteSmem& r) {
         // One warp per token: each lane holds the logits of experts lane + 32 j; top_k rounds of a
         // warp-wide argmax (largest logit, ties to the lower expert index -- the order a
         // sequential scan with a strict comparison gives).
-        const int warp = tid >> 5, lane = tid & 31;
-        for (int m = warp; m < a.M; m += blockDim.x >> 5) {
-            const float* l = a.logits + (int64_t)m * a.E;
-            float v[kMoeMaxE / 32];
+        const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+        // all of this warp's logits first, so that their loads are in flight together
+        constexpr int kTokPerWarp = (kMoeMaxM + kGemvWarps - 1) / kGemvWarps;
+        float vall[kTokPerWarp][kMoeMaxE / 32];
+#pragma unroll
+        for (int i = 0; i < kTokPerWarp; ++i) {
+            const int m = warp + i * nw;
 #pragma unroll
             for (int j = 0; j < kMoeMaxE / 32; ++j) {
                 const int e = lane + 32 * j;
-                v[j] = e < a.E ? __ldcg(l + e) : -INFINITY;
+                vall[i][j] = (m < a.M && e < a.E) ? __ldcg(a.logits + (int64_t)m * a.E + e) : -INFINITY;
             }
+        }
+#pragma unroll
+        for (int i = 0; i < kTokPerWarp; ++i) {
+            const int m = warp + i * nw;
+            if (m >= a.M) break;
+            float v[kMoeMaxE / 32];
+#pragma unroll
+            for (int j = 0; j < kMoeMaxE / 32; ++j) v[j] = vall[i][j];
             float lsel[kMoeMaxTopK];
             unsigned taken = 0;  // bit j: expert lane + 32 j already selected
             for (int s = 0; s < a.top_k; ++s) {
@@ -335,31 +346,48 @@ __device__ __noinline__ bool moe_flush(const MoeArgs& a, const RouteSmem& r, int
     float sum[MAXM];
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) sum[m] = 0.f;
-    for (int i = 0; i < n_t; ++i) {
-        const uint64_t* w = moe_part(a, s, v + i, i == 0 ? 1 : 0, lane);
-        uint64_t x[MAXM];
+    // pieces fetched together (their loads in flight at once), then added in order; one at a time
+    // with 8 rows, where the wider batch costs more in registers than it saves
+    constexpr int kB = MAXM > 2 ? 1 : 4;
+    for (int i0 = 0; i0 < n_t; i0 += kB) {
+        uint64_t x[kB][MAXM];
 #pragma unroll
-        for (int m = 0; m < MAXM; ++m) x[m] = m < a.M ? moe_ld_relaxed(w + m) : ((uint64_t)tag << 32);
+        for (int b = 0; b < kB; ++b) {
+            const int i = i0 + b;
+            const uint64_t* w = i < n_t ? moe_part(a, s, v + i, i == 0 ? 1 : 0, lane) : nullptr;
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m)
+                x[b][m] = (w != nullptr && m < a.M) ? moe_ld_relaxed(w + m) : ((uint64_t)tag << 32);
+        }
         bool ready = true;
 #pragma unroll
-        for (int m = 0; m < MAXM; ++m) ready &= (uint32_t)(x[m] >> 32) == tag;
+        for (int b = 0; b < kB; ++b)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) ready &= (uint32_t)(x[b][m] >> 32) == tag;
         if (!__all_sync(0xffffffffu, ready)) {
             const uint64_t t0 = globaltimer_ns();
             for (uint32_t it = 1;; ++it) {
                 __nanosleep(100);
                 ready = true;
 #pragma unroll
-                for (int m = 0; m < MAXM; ++m)
-                    if (m < a.M && (uint32_t)(x[m] >> 32) != tag) {
-                        x[m] = moe_ld_relaxed(w + m);
-                        ready &= (uint32_t)(x[m] >> 32) == tag;
-                    }
+                for (int b = 0; b < kB; ++b) {
+                    const int i = i0 + b;
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m)
+                        if (i < n_t && m < a.M && (uint32_t)(x[b][m] >> 32) != tag) {
+                            x[b][m] = moe_ld_relaxed(moe_part(a, s, v + i, i == 0 ? 1 : 0, lane) + m);
+                            ready &= (uint32_t)(x[b][m] >> 32) == tag;
+                        }
+                }
                 if (__all_sync(0xffffffffu, ready)) break;
                 if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
             }
         }
 #pragma unroll
-        for (int m = 0; m < MAXM; ++m) sum[m] += __uint_as_float((uint32_t)x[m]);
+        for (int b = 0; b < kB; ++b)
+            if (i0 + b < n_t)
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m) sum[m] += __uint_as_float((uint32_t)x[b][m]);
     }
     moe_write_tile<MAXM>(a, r, s, act, t, lane, sum, gs);
     return true;
@@ -381,38 +409,53 @@ __device__ __forceinline__ bool moe_wait_count(const unsigned int* p, uint32_t t
     }
 }
 
-// One unit of segment s for the rows of active expert `act`: segment 0 reads the tokens' x
-// (XB: bf16), segment 1 their h rows (fp32).  One-pass (MAXM <= 2) accumulates into acc8 across a
-// tile's units; otherwise each pass is reduced at once into acc.
-template <int FMT, int MAXM, bool XB>
+// Row pointers of the pass starting at row q0 of active expert `act` in segment s (segment 0:
+// the tokens' x rows, XB: bf16; segment 1: their fp32 h rows); NULL past the expert's rows.
+template <int MP, bool XB>
+__device__ __forceinline__ void moe_rows(const MoeArgs& a, const RouteSmem& r, int s, int act, int q0,
+                                         const void* (&rows)[MP]) {
+    const int nr = r.nrows[act];
+#pragma unroll
+    for (int mm = 0; mm < MP; ++mm) {
+        const int q = q0 + mm;
+        if (q >= nr) {
+            rows[mm] = nullptr;
+        } else if (s == 0) {
+            const int64_t off = (int64_t)r.row_m[act][q] * a.H;
+            rows[mm] = XB ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.x) + off)
+                          : (const void*)(reinterpret_cast<const float*>(a.x) + off);
+        } else {
+            rows[mm] = a.h + ((int64_t)r.row_m[act][q] * a.top_k + r.row_s[act][q]) * a.I;
+        }
+    }
+}
+
+// One unit of segment s for the rows of active expert `act`.  One-pass (MAXM <= 2, or an expert
+// with at most 2 rows) accumulates into acc8 across a tile's units; otherwise each pass is
+// reduced at once into acc.  xs: the first pass's rows already staged in shared memory (or
+// NULL); after_first_load() runs once the first pass's activations are in registers.
+template <int FMT, int MAXM, bool XB, typename F>
 __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, int s, int act, int g,
                                          const uint8_t* ubuf, int lane, float (&acc8)[8][MAXM >= 2 ? 2 : 1],
-                                         float (&acc)[MAXM]) {
+                                         float (&acc)[MAXM], const uint8_t* xs, F&& after_first_load) {
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     const int nr = r.nrows[act];
     const bool kOnePass = MAXM <= 2 || nr <= 2;  // an expert with at most 2 rows: accumulate in acc8
     const int64_t Kin = s == 0 ? a.H : a.I;
-    const int64_t k0 = (int64_t)g * kGroupK + (lane & 7) * 32;
+    const int part = lane & 7;
+    const int64_t k0 = (int64_t)g * kGroupK + part * 32;
 #pragma unroll 1
     for (int q0 = 0; q0 < (kOnePass ? 1 : nr); q0 += MP) {
         const void* rows[MP];
-#pragma unroll
-        for (int mm = 0; mm < MP; ++mm) {
-            const int q = q0 + mm;
-            if (q >= nr) {
-                rows[mm] = nullptr;
-            } else if (s == 0) {
-                const int64_t off = (int64_t)r.row_m[act][q] * a.H;
-                rows[mm] = XB ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(a.x) + off)
-                              : (const void*)(reinterpret_cast<const float*>(a.x) + off);
-            } else {
-                rows[mm] = a.h + ((int64_t)r.row_m[act][q] * a.top_k + r.row_s[act][q]) * a.I;
-            }
-        }
+        moe_rows<MP, XB>(a, r, s, act, q0, rows);
         if constexpr (XB && FMT == QLIN_NVFP4) {
             uint32_t xh[MP][16];
             float xsc[MP][2];
-            load_x_fp4h<MP, true>(rows, k0, Kin, xh, xsc);
+            if (q0 == 0 && xs != nullptr)
+                load_x_fp4h_staged<MP>(xs, part, xh, xsc);
+            else
+                load_x_fp4h<MP, true>(rows, k0, Kin, xh, xsc);
+            if (q0 == 0) after_first_load();
             if (kOnePass) {
                 unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
             } else {
@@ -429,7 +472,11 @@ __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, i
         } else {
             float2 xv[MP][16];
             float xb[MP];
-            load_x_rows<XB, MP, true>(rows, k0, Kin, xv);
+            if (q0 == 0 && xs != nullptr)
+                load_x_staged<XB, MP>(xs, part, xv);
+            else
+                load_x_rows<XB, MP, true>(rows, k0, Kin, xv);
+            if (q0 == 0) after_first_load();
             prep_x<FMT, MP>(xv, xb);
             if (kOnePass) {
                 unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
@@ -448,6 +495,18 @@ __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, i
     }
 }
 
+// Shared memory of the MoE kernel: the per-warp weight rings and their barriers, then (for at most
+// 2 rows, except Q8_0 whose ring leaves no room) one activation stage per warp: the next unit's
+// rows, copied while the current unit computes.  (With 8 rows the staging measured slower.)
+template <int FMT, int MAXM>
+struct MoeSmem {
+    static constexpr int MP = MAXM >= 2 ? 2 : 1;
+    static constexpr bool kStaged = FMT != QLIN_Q8_0 && MAXM <= 2;
+    static constexpr int kStageBytes = MP * XStage<false>::kRowBytes;  // fp32 layout; bf16 rows fit
+    static constexpr int kXOff = (RingCfg<FMT>::kSmem + 127) / 128 * 128;
+    static constexpr int kBytes = kStaged ? kXOff + kGemvWarps * kStageBytes : RingCfg<FMT>::kSmem;
+};
+
 template <int FMT>
 __device__ __forceinline__ float moe_scale(const MoeArgs& a, const RouteSmem& r, int s, int act) {
     return format_out_scale<FMT>(s == 0 ? a.gu + (int64_t)r.expert[act] * a.gu_stride
@@ -457,6 +516,7 @@ __device__ __forceinline__ float moe_scale(const MoeArgs& a, const RouteSmem& r,
 template <int FMT, int MAXM, bool XBF16>
 __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe_kernel(const MoeArgs a) {
     using C = RingCfg<FMT>;
+    using MS = MoeSmem<FMT, MAXM>;
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     constexpr bool kOnePass = MAXM <= 2;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -465,6 +525,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
     const int gw = blockIdx.x * kGemvWarps + warp;
     uint8_t* ring = smem + warp * C::D * C::UB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemvWarps * C::D * C::UB) + warp * C::D;
+    uint8_t* xst = smem + MS::kXOff + warp * MS::kStageBytes;  // used only if MS::kStaged
 
     griddep_launch_dependents();
     griddep_wait();  // logits / ids / x come from earlier kernels
@@ -519,6 +580,17 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
     int pend_s = -1, pend_a = 0, pend_t = 0, pend_v = 0, pend_n = 0;  // split tile finished later
     float pend_gs = 1.f;
     int seq = 0, cur_s = -1, cur_a = -1, b = 0, e = 0;
+    bool xready = false;  // the current unit's first-pass rows are already staged
+    auto stage_unit = [&](const MoeCursor& u) {
+        const void* rows[MP];
+        if (u.s == 0) {
+            moe_rows<MP, XBF16>(a, r, 0, u.a, 0, rows);
+            stage_x_rows<XBF16, MP>(rows, a.H, u.g, xst, lane, a.ws);
+        } else {
+            moe_rows<MP, false>(a, r, 1, u.a, 0, rows);
+            stage_x_rows<false, MP>(rows, a.I, u.g, xst, lane, a.ws);
+        }
+    };
     float gs = 1.f;
     while (c.s < 2) {
         if (c.s != cur_s) {  // new segment: finish the pending tile of the previous one
@@ -549,10 +621,29 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
             break;
         }
         const uint8_t* ubuf = ring + slot * C::UB;
+        const uint8_t* xs = nullptr;
+        MoeCursor cn = c;  // the next unit of this warp
+        bool stage_next = false;
+        if constexpr (MS::kStaged) {
+            if (!xready) stage_unit(c);
+            cp_async_wait_all();
+            __syncwarp();
+            xs = xst;
+            moe_step(sg, gw, a.W, cn);
+            // h rows of a down unit may be read only after that expert's wait
+            stage_next = cn.s < 2 && (cn.s == 0 || (c.s == 1 && cn.a == c.a));
+        }
+        auto after_first_load = [&]() {  // the stage is free: copy the next unit's rows into it
+            if constexpr (MS::kStaged) {
+                __syncwarp();
+                if (stage_next) stage_unit(cn);
+            }
+        };
         if (c.s == 0)
-            moe_unit<FMT, MAXM, XBF16>(a, r, 0, c.a, c.g, ubuf, lane, acc8, acc);
+            moe_unit<FMT, MAXM, XBF16>(a, r, 0, c.a, c.g, ubuf, lane, acc8, acc, xs, after_first_load);
         else
-            moe_unit<FMT, MAXM, false>(a, r, 1, c.a, c.g, ubuf, lane, acc8, acc);
+            moe_unit<FMT, MAXM, false>(a, r, 1, c.a, c.g, ubuf, lane, acc8, acc, xs, after_first_load);
+        xready = stage_next;
         __syncwarp();
         if (lane == 0 && p.s < 2) {
             fence_proxy_async_smem();
@@ -600,6 +691,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
     if (!failed && pend_s >= 0 &&
         !moe_flush<MAXM>(a, r, pend_s, pend_a, pend_t, pend_v, pend_n, lane, pend_gs, tag))
         failed = true;
+    if constexpr (MS::kStaged) cp_async_wait_all();  // no copy into this CTA's memory outlives it
     if (failed && lane == 0) {
         atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
         MoeCursor q = c;  // wait (bounded) for this warp's copies still in flight
@@ -661,14 +753,15 @@ static MoePlan plan_moe(int fmt, int M, int64_t H, int64_t I, int top_k, bool ne
 template <int FMT, int MAXM, bool XBF16>
 static cudaError_t moe_launch(const MoeArgs& a, int grid, cudaStream_t s, bool pdl) {
     using C = RingCfg<FMT>;
+    constexpr int kSmem = MoeSmem<FMT, MAXM>::kBytes;
     auto kern = moe_kernel<FMT, MAXM, XBF16>;
     static bool attr_set = false;  // per instantiation; idempotent
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess) return e;
         // The waits between the steps need every CTA of the grid resident at once.
         int occ = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvWarps * 32, C::kSmem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGemvWarps * 32, kSmem);
         if (e != cudaSuccess) return e;
         if (occ < C::kCtasPerSm) return cudaErrorLaunchOutOfResources;
         attr_set = true;
@@ -676,7 +769,7 @@ static cudaError_t moe_launch(const MoeArgs& a, int grid, cudaStream_t s, bool p
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kGemvWarps * 32);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -5,8 +5,9 @@ may import this package.  The product path (``gemm_dequant_gemv_q8_b200``) never
 shares no code with it.  The arithmetic lives in ``oracle.c`` (plain C, fp64, sequential sums);
 this module compiles it with gcc on first use and marshals numpy arrays.
 
-Every function cites what it follows; the format layouts are the public GGUF / NVFP4 conventions
-(the pages name the formats -- imp README, "Features" table -- but do not print their layout).
+Every function cites what it follows; the format layouts are the public GGUF / NVFP4 / OCP MX
+conventions (the pages name the formats -- imp README, "Features" table; imp release notes v0.6,
+"Native MXFP4 GGUF weight format" -- but do not print their layout).
 
 Parity pins for every function here live in ``tests/test_oracle_pins.py``.
 """
@@ -19,7 +20,7 @@ import threading
 
 import numpy as np
 
-Q8_0, Q4_0, NVFP4 = 1, 2, 3
+Q8_0, Q4_0, NVFP4, MXFP4 = 1, 2, 3, 4
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
@@ -46,6 +47,7 @@ def _l():
             lib.qo_fp16.restype = D; lib.qo_fp16.argtypes = [ctypes.c_uint16]
             lib.qo_e4m3.restype = D; lib.qo_e4m3.argtypes = [ctypes.c_uint8]
             lib.qo_e2m1.restype = D; lib.qo_e2m1.argtypes = [ctypes.c_uint8]
+            lib.qo_e8m0.restype = D; lib.qo_e8m0.argtypes = [ctypes.c_uint8]
             lib.qo_silu.restype = D; lib.qo_silu.argtypes = [D]
             lib.qo_row_bytes.restype = I64; lib.qo_row_bytes.argtypes = [I, I64]
             lib.qo_dequant.restype = I; lib.qo_dequant.argtypes = [I, I64, I64, P, P, F, P]
@@ -90,6 +92,11 @@ def e4m3(bits: int) -> float:
 def e2m1(code: int) -> float:
     """OCP FP4 E2M1 decode (bias 1, subnormal m*0.5, max 6)."""
     return _l().qo_e2m1(code)
+
+
+def e8m0(bits: int) -> float:
+    """OCP MX UE8M0 scale decode: 2^(bits - 127), bits 0xFF = NaN."""
+    return _l().qo_e8m0(bits)
 
 
 def silu(z: float) -> float:

@@ -12,6 +12,8 @@
  *     NVFP4 weights, NVFP4 block-scaled GEMM/GEMV, e2m1 / e4m3 decode.
  *   - Imparo README intro: Q4_0 MoE decode with CUDA expert routing (LFM2.5-8B-A1B).
  *   - imp README, "Features" table, row "Server": an ordered (deterministic) MoE reduction.
+ *   - imp release notes, v0.6 "Native MXFP4 GGUF weight format": E2M1 codes with UE8M0 block
+ *     scales, 4.25 bits per weight (one 8-bit scale per 32 values).
  * The pages name the formats but never print their byte layout.  The layouts used here are the
  * public conventions (GGUF block_q8_0 / block_q4_0; NVFP4 = E2M1 codes, one E4M3 scale per 16
  * values, one FP32 per-tensor scale), the plainest reading the pages support.
@@ -24,7 +26,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { QO_Q8_0 = 1, QO_Q4_0 = 2, QO_NVFP4 = 3 };
+enum { QO_Q8_0 = 1, QO_Q4_0 = 2, QO_NVFP4 = 3, QO_MXFP4 = 4 };
 
 /* ---------------------------------------------------------------- scalar decoders */
 
@@ -62,13 +64,19 @@ double qo_e2m1(uint8_t c) {
     return s ? -v : v;
 }
 
+/* OCP MX UE8M0 scale: an 8-bit biased exponent (bias 127), no sign, no mantissa; 0xFF is NaN. */
+double qo_e8m0(uint8_t b) {
+    if (b == 0xff) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
 /* ---------------------------------------------------------------- block dequantization */
 
 /* Bytes of one canonical row of K weights. */
 int64_t qo_row_bytes(int fmt, int64_t K) {
     if (fmt == QO_Q8_0) return (K / 32) * 34;
     if (fmt == QO_Q4_0) return (K / 32) * 18;
-    if (fmt == QO_NVFP4) return K / 2;
+    if (fmt == QO_NVFP4 || fmt == QO_MXFP4) return K / 2;
     return -1;
 }
 
@@ -77,7 +85,8 @@ int64_t qo_row_bytes(int fmt, int64_t K) {
  *   Q4_0 block (18 B): fp16 d, uint8 qs[16];        element j (j<16) is the low nibble of qs[j],
  *                                                   element j+16 its high nibble; w = d * (nib - 8)
  *   NVFP4: codes [N][K/2], byte i = elements 2i (low nibble) and 2i+1 (high nibble);
- *          scales [N][K/16] E4M3; w = e2m1(code) * e4m3(scale of k/16) * g            */
+ *          scales [N][K/16] E4M3; w = e2m1(code) * e4m3(scale of k/16) * g
+ *   MXFP4: codes as NVFP4; scales [N][K/32] UE8M0; w = e2m1(code) * 2^(scale of k/32 - 127) */
 static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t* scales, float g,
                         int64_t n, double* w) {
     if (fmt == QO_Q8_0 || fmt == QO_Q4_0) {
@@ -95,7 +104,7 @@ static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t
                 w[b * 32 + j] = d * q;
             }
         }
-    } else {
+    } else if (fmt == QO_NVFP4) {
         const uint8_t* row = blocks + n * (K / 2);
         const uint8_t* srow = scales + n * (K / 16);
         for (int64_t k = 0; k < K; ++k) {
@@ -103,13 +112,24 @@ static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t
             uint8_t c = (k & 1) ? (byte >> 4) : (byte & 0xf);
             w[k] = qo_e2m1(c) * qo_e4m3(srow[k / 16]) * (double)g;
         }
+    } else {
+        const uint8_t* row = blocks + n * (K / 2);
+        const uint8_t* srow = scales + n * (K / 32);
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = row[k / 2];
+            uint8_t c = (k & 1) ? (byte >> 4) : (byte & 0xf);
+            w[k] = qo_e2m1(c) * qo_e8m0(srow[k / 32]);
+        }
     }
 }
+
+/* Values per block along K (scale granularity): 16 for NVFP4, 32 otherwise. */
+static int64_t qo_block_k(int fmt) { return fmt == QO_NVFP4 ? 16 : 32; }
 
 /* Full-tensor dequantization to fp64.  Returns 0, or -1 on a bad argument. */
 int qo_dequant(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
                float g, double* W) {
-    if (qo_row_bytes(fmt, K) < 0 || K % (fmt == QO_NVFP4 ? 16 : 32)) return -1;
+    if (qo_row_bytes(fmt, K) < 0 || K % qo_block_k(fmt)) return -1;
     for (int64_t n = 0; n < N; ++n) dequant_row(fmt, K, blocks, scales, g, n, W + n * K);
     return 0;
 }
@@ -119,7 +139,7 @@ int qo_dequant(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8
  * scale g is the one rounding: w32 = fp32( (e2m1*e4m3) * g ), rounded once to nearest-even. */
 int qo_dequant_f32(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
                    float g, float* W) {
-    if (qo_row_bytes(fmt, K) < 0 || K % (fmt == QO_NVFP4 ? 16 : 32)) return -1;
+    if (qo_row_bytes(fmt, K) < 0 || K % qo_block_k(fmt)) return -1;
     double* w = (double*)malloc(sizeof(double) * K);
     if (!w) return -1;
     for (int64_t n = 0; n < N; ++n) {
@@ -139,7 +159,7 @@ int qo_dequant_f32(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const u
 int qo_gemv_rows(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
                  float g, int M, const double* x, const int64_t* rows, int64_t nrows, double* y,
                  double* A) {
-    if (qo_row_bytes(fmt, K) < 0 || K % (fmt == QO_NVFP4 ? 16 : 32)) return -1;
+    if (qo_row_bytes(fmt, K) < 0 || K % qo_block_k(fmt)) return -1;
     double* w = (double*)malloc(sizeof(double) * (K ? K : 1));
     if (!w) return -1;
     for (int64_t j = 0; j < nrows; ++j) {
@@ -241,9 +261,10 @@ int qo_moe(int fmt, int E, int64_t H, int64_t I, int top_k, const uint8_t* gu_bl
             int e = ids[(int64_t)m * top_k + s];
             double ws = wts[(int64_t)m * top_k + s];
             const uint8_t* gb = gu_blocks + (int64_t)e * 2 * I * gu_rb;
-            const uint8_t* gsc = fmt == QO_NVFP4 ? gu_scales + (int64_t)e * 2 * I * (H / 16) : NULL;
+            const int fp4 = fmt == QO_NVFP4 || fmt == QO_MXFP4;
+            const uint8_t* gsc = fp4 ? gu_scales + (int64_t)e * 2 * I * (H / qo_block_k(fmt)) : NULL;
             const uint8_t* db = dn_blocks + (int64_t)e * H * dn_rb;
-            const uint8_t* dsc = fmt == QO_NVFP4 ? dn_scales + (int64_t)e * H * (I / 16) : NULL;
+            const uint8_t* dsc = fp4 ? dn_scales + (int64_t)e * H * (I / qo_block_k(fmt)) : NULL;
             qo_gemv(fmt, 2 * I, H, gb, gsc, gu_g ? gu_g[e] : 1.0f, 1, x + (int64_t)m * H, gu, NULL);
             double* hm = h + ((int64_t)m * top_k + s) * I;
             qo_silu_gate(1, I, gu, NULL, hm, NULL);

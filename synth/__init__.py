@@ -1,7 +1,7 @@
 """Seeded synthetic inputs shared by the tests, the smoke check and the bench.
 
 This module only draws random numbers and lays them out in the canonical storage formats
-(GGUF Q8_0 / Q4_0 blocks, NVFP4 code and scale planes); it holds none of the layer's arithmetic.
+(GGUF Q8_0 / Q4_0 blocks, NVFP4 / MXFP4 code and scale planes); it holds none of the layer's arithmetic.
 Rounding of drawn reals to fp16 / bf16 / E4M3 storage uses torch's own conversions
 (round-to-nearest-even).
 
@@ -11,20 +11,22 @@ Canonical layouts (the public conventions; the pages name the formats but not th
         in its low nibble and element j+16 in its high nibble
   NVFP4 codes [N][K/2] (byte i = element 2i low nibble, 2i+1 high nibble), E4M3 scales [N][K/16],
         one fp32 per-tensor scale
+  MXFP4 codes as NVFP4, UE8M0 scale bytes [N][K/32] (one per 32 values), no per-tensor scale
 
 Workload recipes (seeded; shapes from the synthetic layer stacks the bench and tests use):
   Q8_0:  codes uniform over [-127, 127], scale uniform real in [1e-3, 1e-2] rounded to fp16
   Q4_0:  4-bit codes uniform over 0..15 (value = code - 8), scale uniform real in [1e-3, 2e-2]
   NVFP4: codes uniform over all 16, E4M3 scales uniform real in [0.5, 448] rounded to E4M3,
          per-tensor scale fp32(1/448)
+  MXFP4: codes uniform over all 16, scale bytes uniform integers in [118, 130] (2^-9 .. 2^3)
   activations N(0, 1) (fp32, or fp32 draws rounded to bf16); router logits N(0, 1)
 """
 from __future__ import annotations
 
 import torch
 
-Q8_0, Q4_0, NVFP4 = 1, 2, 3
-FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4"}
+Q8_0, Q4_0, NVFP4, MXFP4 = 1, 2, 3, 4
+FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4", MXFP4: "mxfp4"}
 NVFP4_G = float(torch.tensor(1.0 / 448.0, dtype=torch.float32))
 
 
@@ -73,12 +75,25 @@ def nvfp4(N, K, g, device="cpu", s_range=(0.5, 448.0)):
     return codes.contiguous(), scales, NVFP4_G
 
 
+def mxfp4(N, K, g, device="cpu", e_range=(118, 130)):
+    """Canonical MXFP4 tensor: (codes uint8 [N, K/2], UE8M0 scale bytes [N, K/32], 1.0).
+    Codes uniform over all 16; scale bytes uniform integers in e_range (2^-9 .. 2^3)."""
+    assert K % 32 == 0
+    codes = torch.randint(0, 256, (N, K // 2), generator=g, device=device,
+                          dtype=torch.int16).to(torch.uint8)
+    scales = torch.randint(e_range[0], e_range[1] + 1, (N, K // 32), generator=g, device=device,
+                           dtype=torch.int16).to(torch.uint8)
+    return codes.contiguous(), scales.contiguous(), 1.0
+
+
 def weights(fmt, N, K, g, device="cpu"):
     """Canonical tensor of the given format: (blocks, scales or None, per-tensor scale)."""
     if fmt == Q8_0:
         return q8_0(N, K, g, device), None, 1.0
     if fmt == Q4_0:
         return q4_0(N, K, g, device), None, 1.0
+    if fmt == MXFP4:
+        return mxfp4(N, K, g, device=device)
     if fmt == NVFP4:
         return nvfp4(N, K, g, device)
     raise ValueError(fmt)

@@ -52,6 +52,17 @@ def test_e2m1_all_codes_match_golden():
         assert got == v and math.copysign(1, got) == math.copysign(1, v), (c, got, v)
 
 
+def test_e8m0_all_codes_match_fp32_bit_construction():
+    # UE8M0 byte b is the biased exponent of a power of two: the fp32 number with exponent field b
+    # and a zero mantissa for b = 1..254, the fp32 subnormal 0x00400000 (2^-127) for b = 0, NaN
+    # for 0xFF.  Built from bits here, not through the oracle's ldexp.
+    for b in range(1, 255):
+        ref = float(np.array([b << 23], np.uint32).view(np.float32)[0])
+        assert oracle.e8m0(b) == ref, b
+    assert oracle.e8m0(0) == float(np.array([0x00400000], np.uint32).view(np.float32)[0]) == 2.0 ** -127
+    assert math.isnan(oracle.e8m0(255))
+
+
 # ----------------------------------------------------------------------------- block dequant
 def _golden_blocks(name):
     lines = read_golden(name)
@@ -105,6 +116,39 @@ def test_nvfp4_scale_applies_per_16():
     assert list(w) == [1.0] * 16 + [2.0] * 16 + [0.5] * 16
 
 
+def test_mxfp4_dequant_matches_golden():
+    lines = read_golden("mxfp4_block.txt")
+    codes = np.array([[int(t, 16) for t in lines[0].split()[1:]]], np.uint8)
+    scales = np.array([[int(t, 16) for t in lines[1].split()[1:]]], np.uint8)
+    v = [float(t) for t in lines[2].split()[1:]]
+    w = oracle.dequant(oracle.MXFP4, 1, 64, codes, scales)[0]
+    assert list(w) == v and list(np.signbit(w)) == [math.copysign(1, t) < 0 for t in v]
+    w32 = oracle.dequant_f32(oracle.MXFP4, 1, 64, codes, scales)[0]
+    assert np.array_equal(w32.astype(np.float64), np.array(v))
+
+
+def test_mxfp4_equals_nvfp4_with_the_same_power_of_two_scales():
+    # A UE8M0 scale 2^(e-127) with e in [120, 134] is exactly an E4M3 value (2^-7 .. 2^7); giving
+    # both 16-value halves of each 32-value block that E4M3 scale (converted by torch) and the
+    # per-tensor scale 1 must give the same weights through the (separately pinned) NVFP4 decode.
+    N, K = 6, 128
+    codes, _, _ = synth.weights(oracle.MXFP4, N, K, synth.gen(11))
+    e = torch.randint(120, 135, (N, K // 32), generator=synth.gen(12), dtype=torch.int32)
+    pow2 = torch.pow(2.0, (e - 127).to(torch.float64)).to(torch.float32)
+    e4 = pow2.to(torch.float8_e4m3fn)
+    assert torch.equal(e4.to(torch.float32), pow2)
+    nv_scales = e4.view(torch.uint8).repeat_interleave(2, dim=1).numpy()
+    Wmx = oracle.dequant(oracle.MXFP4, N, K, codes.numpy(), e.to(torch.uint8).numpy())
+    Wnv = oracle.dequant(oracle.NVFP4, N, K, codes.numpy(), nv_scales, 1.0)
+    assert np.array_equal(Wmx, Wnv)
+
+
+def test_mxfp4_scale_ff_is_nan_only_in_its_block():
+    codes = np.full((1, 32), 0x22, np.uint8)  # every element 1.0
+    w = oracle.dequant(oracle.MXFP4, 1, 64, codes, np.array([[0xFF, 0x7F]], np.uint8))[0]
+    assert np.isnan(w[:32]).all() and list(w[32:]) == [1.0] * 32
+
+
 # ----------------------------------------------------------------------------- GEMV
 def _identity_q8(K):
     blk = np.zeros((K, K // 32, 34), np.uint8)
@@ -134,7 +178,15 @@ def _identity_nvfp4(K):
     return codes, np.full((K, K // 16), 0x38, np.uint8)
 
 
-@pytest.mark.parametrize("fmt", [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4])
+def _identity_mxfp4(K):
+    codes, _ = _identity_nvfp4(K)
+    return codes, np.full((K, K // 32), 0x7F, np.uint8)  # UE8M0 2^0
+
+
+FMTS_ALL = [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4, oracle.MXFP4]
+
+
+@pytest.mark.parametrize("fmt", FMTS_ALL)
 def test_gemv_identity_gives_x(fmt):
     K = 96
     x = synth.activations(3, K, synth.gen(1)).double().numpy()
@@ -142,14 +194,16 @@ def test_gemv_identity_gives_x(fmt):
         blocks, scales = _identity_q8(K), None
     elif fmt == oracle.Q4_0:
         blocks, scales = _identity_q4(K), None
-    else:
+    elif fmt == oracle.NVFP4:
         blocks, scales = _identity_nvfp4(K)
+    else:
+        blocks, scales = _identity_mxfp4(K)
     y, A = oracle.gemv(fmt, K, K, blocks, x, scales=scales, g=1.0)
     assert np.array_equal(y, x)
     assert np.array_equal(A, np.abs(x))
 
 
-@pytest.mark.parametrize("fmt", [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4])
+@pytest.mark.parametrize("fmt", FMTS_ALL)
 def test_gemv_one_hot_selects_a_column(fmt):
     N, K = 40, 64  # N != K so a transposed operand cannot pass
     blocks, scales, g = synth.weights(fmt, N, K, synth.gen(2))
@@ -162,7 +216,7 @@ def test_gemv_one_hot_selects_a_column(fmt):
         assert np.array_equal(y[0], W[:, k])
 
 
-@pytest.mark.parametrize("fmt", [oracle.Q8_0, oracle.Q4_0, oracle.NVFP4])
+@pytest.mark.parametrize("fmt", FMTS_ALL)
 def test_gemv_matches_exact_rational_sum(fmt):
     N, K, M = 5, 64, 3
     blocks, scales, g = synth.weights(fmt, N, K, synth.gen(3))

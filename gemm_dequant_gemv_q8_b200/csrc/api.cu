@@ -32,7 +32,7 @@ namespace {
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
-bool valid_fmt(int f) { return f == QLIN_Q8_0 || f == QLIN_Q4_0 || f == QLIN_NVFP4; }
+bool valid_fmt(int f) { return f == QLIN_Q8_0 || f == QLIN_Q4_0 || f == QLIN_NVFP4 || f == QLIN_MXFP4; }
 
 bool valid_shape(int fmt, int64_t N, int64_t K) {
     if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return false;
@@ -113,7 +113,7 @@ qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const v
     if (pack_flags != QLIN_PACK_MMA && (pack_flags & ~QLIN_PACK_GATE_UP)) return QLIN_ERR_INVALID_ARG;
     if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
     if (!blocks || !packed) return QLIN_ERR_INVALID_ARG;
-    if (fmt == QLIN_NVFP4 && !scales) return QLIN_ERR_INVALID_ARG;
+    if ((fmt == QLIN_NVFP4 || fmt == QLIN_MXFP4) && !scales) return QLIN_ERR_INVALID_ARG;
     if (!aligned(packed, 256)) return QLIN_ERR_ALIGNMENT;
     if (packed_bytes < qlin_packed_bytes(fmt, N, K, pack_flags)) return QLIN_ERR_INVALID_ARG;
     const float gs = fmt == QLIN_NVFP4 ? global_scale : 1.0f;
@@ -176,6 +176,7 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
     if (M < 1 || M > 8 || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, 2 * I, H) || !valid_shape(fmt, H, I)) return QLIN_ERR_INVALID_ARG;
     if (H > 32768) return QLIN_ERR_UNSUPPORTED;  // down tiles per expert are tracked per token
+    if (fmt == QLIN_MXFP4) return QLIN_ERR_UNSUPPORTED;  // the expert kernel is built for the other formats
     if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
     if (flags & ~QLIN_FLAG_PDL) return QLIN_ERR_INVALID_ARG;
     if (!gate_up_packed || !down_packed || !topk_ids || !topk_w || !x || !y) return QLIN_ERR_INVALID_ARG;

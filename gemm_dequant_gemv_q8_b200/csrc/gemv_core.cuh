@@ -32,10 +32,12 @@ struct RingCfg {
 constexpr int kXExp = 63;
 constexpr float kDenormUnscale = 0x1p86f;  // 2^(149 - kXExp)
 
-// Output scale of a format's block sums: the NVFP4 per-tensor scale, or 2^86 for Q4_0 / Q8_0.
+// Output scale of a format's block sums: the NVFP4 per-tensor scale, 1 for MXFP4 (its block
+// scales are applied in full per block), or 2^86 for Q4_0 / Q8_0.
 template <int FMT>
 __device__ __forceinline__ float format_out_scale(const uint8_t* packed) {
     if (FMT == QLIN_NVFP4) return reinterpret_cast<const PackedHeader*>(packed)->global_scale;
+    if (FMT == QLIN_MXFP4) return 1.0f;
     return kDenormUnscale;
 }
 
@@ -389,11 +391,18 @@ __device__ __forceinline__ void unit_dot_fp4h(const uint8_t* ub, int lane, const
 template <int FMT, int MP, bool ACC = false>
 __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const float2 (&xv)[MP][16],
                                          const float (&xb)[MP], float (&res)[8][MP]) {
-    const uint4 sv = lds128(ub + code_bytes(FMT) + lane * 16);
-    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+    uint32_t sw[4];
+    if (FMT == QLIN_MXFP4) {  // 8 bits of scale per (row, part)
+        const uint2 s2 = *reinterpret_cast<const uint2*>(ub + code_bytes(FMT) + lane * 8);
+        sw[0] = s2.x, sw[1] = s2.y, sw[2] = sw[3] = 0u;
+    } else {
+        const uint4 sv = lds128(ub + code_bytes(FMT) + lane * 16);
+        sw[0] = sv.x, sw[1] = sv.y, sw[2] = sv.z, sw[3] = sv.w;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const uint32_t sc = sw[i >> 1] >> (16 * (i & 1));  // 16 bits of scale for (row, part)
+        // 16 bits of scale for (row, part); MXFP4: 8 bits
+        const uint32_t sc = FMT == QLIN_MXFP4 ? (sw[i >> 2] >> (8 * (i & 3))) : (sw[i >> 1] >> (16 * (i & 1)));
         if (FMT == QLIN_Q4_0) {
             const uint4 c = lds128(ub + (lane + 32 * i) * 16);
             const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
@@ -446,6 +455,30 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
                 const float2 u = __fadd2_rn(s0[mm], s1[mm]);
                 const float bsum = (u.x + u.y) - xb[mm];
                 res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
+            }
+        } else if (FMT == QLIN_MXFP4) {  // one 32-element block per part, one UE8M0 scale
+            const uint4 c = lds128(ub + (lane + 32 * i) * 16);
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+            float2 s0[MP], s1[MP];
+#pragma unroll
+            for (int mm = 0; mm < MP; ++mm) s0[mm] = s1[mm] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 p[4];
+                dec_fp4(cw[k], p);
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) {
+                    s0[mm] = __ffma2_rn(p[0], xv[mm][4 * k + 0], s0[mm]);
+                    s1[mm] = __ffma2_rn(p[1], xv[mm][4 * k + 1], s1[mm]);
+                    s0[mm] = __ffma2_rn(p[2], xv[mm][4 * k + 2], s0[mm]);
+                    s1[mm] = __ffma2_rn(p[3], xv[mm][4 * k + 3], s1[mm]);
+                }
+            }
+            const float e = e8m0_to_f32(sc);
+#pragma unroll
+            for (int mm = 0; mm < MP; ++mm) {
+                const float bsum = (s0[mm].x + s0[mm].y) + (s1[mm].x + s1[mm].y);
+                res[i][mm] = ACC ? fmaf(e, bsum, res[i][mm]) : e * bsum;
             }
         } else {  // NVFP4: two 16-element blocks per part, one E4M3 scale each
             const uint4 c = lds128(ub + (lane + 32 * i) * 16);

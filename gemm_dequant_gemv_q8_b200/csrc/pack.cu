@@ -1,4 +1,4 @@
-// pack.cu -- canonical GGUF / NVFP4 tensors -> the packed tile layout, and its inverse for tests.
+// pack.cu -- canonical GGUF / NVFP4 / MXFP4 tensors -> the packed tile layout, and its inverse for tests.
 //
 // The repacker is the offline step that re-lays weights once per tensor (the pages' prior art:
 // Imparo README intro, a "private GateUp layout" built from the canonical GGUF; imp README "Why
@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ b
     const int64_t n = source_row(t, r, N, gate_up);
     const int64_t k0 = g * kGroupK + p * 32;  // first element of this part
     const int lane = (r & 3) * 8 + p, slot = r >> 2;
-    uint8_t* sc = ub + code_bytes(FMT) + lane * 16 + slot * 2;
+    uint8_t* sc = ub + code_bytes(FMT) + (FMT == QLIN_MXFP4 ? lane * 8 + slot : lane * 16 + slot * 2);
 
     if (FMT == QLIN_Q4_0) {
         uint8_t out[16];
@@ -71,6 +71,19 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ b
         *reinterpret_cast<uint4*>(ub + 4096 + (r * 8 + p) * 16) = v1;
         sc[0] = (uint8_t)(d & 0xff);
         sc[1] = (uint8_t)(d >> 8);
+    } else if (FMT == QLIN_MXFP4) {  // codes as NVFP4, one UE8M0 scale per part
+        uint8_t out[16];
+        uint8_t s = 0;
+        for (int j = 0; j < 16; ++j) out[j] = 0;
+        if (n >= 0 && k0 < K) {
+            const uint8_t* row = blocks + n * (K / 2);
+            for (int j = 0; j < 16; ++j) out[j] = row[k0 / 2 + j];
+            s = scales[n * (K / 32) + k0 / 32];
+        }
+        uint4 v;
+        memcpy(&v, out, 16);
+        *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v;
+        sc[0] = s;
     } else {  // NVFP4: codes already two per byte in element order
         uint8_t out[16];
         uint8_t s0 = 0, s1 = 0;
@@ -121,7 +134,7 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
     const int64_t k0 = g * kGroupK + p * 32;
     if (n < 0 || k0 >= K) return;
     const int lane = (r & 3) * 8 + p, slot = r >> 2;
-    const uint8_t* sc = ub + code_bytes(FMT) + lane * 16 + slot * 2;
+    const uint8_t* sc = ub + code_bytes(FMT) + (FMT == QLIN_MXFP4 ? lane * 8 + slot : lane * 16 + slot * 2);
     const float gs = reinterpret_cast<const PackedHeader*>(packed)->global_scale;
     const int64_t valid = (K - k0) >= 32 ? 32 : (K - k0);
     float* out = w + n * K + k0;
@@ -137,6 +150,13 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
         for (int e = 0; e < 32; ++e) {
             int b = (e < 16 ? cv[e] : cv[4096 + e - 16]);
             out[e] = d * (float)(b - 128);
+        }
+    } else if (FMT == QLIN_MXFP4) {
+        const float s = e8m0_to_f32(sc[0]);
+        for (int e = 0; e < valid; ++e) {
+            uint32_t h2 = e2m1x2_to_f16x2(cv[e / 2]);
+            float v = __half2float(__ushort_as_half((unsigned short)((e & 1) ? (h2 >> 16) : (h2 & 0xffff))));
+            out[e] = __fmul_rn(v, s);  // a power of two times an E2M1 value: exact unless it overflows
         }
     } else {
         for (int e = 0; e < valid; ++e) {
@@ -174,6 +194,9 @@ extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void*
     else if (fmt == QLIN_Q8_0)
         pack_kernel<QLIN_Q8_0><<<grid, 256, 0, s>>>((const uint8_t*)blocks, nullptr, N, K, gu,
                                                      (uint8_t*)packed, geo.G);
+    else if (fmt == QLIN_MXFP4)
+        pack_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>((const uint8_t*)blocks, (const uint8_t*)scales,
+                                                      N, K, gu, (uint8_t*)packed, geo.G);
     else
         pack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)blocks, (const uint8_t*)scales,
                                                       N, K, gu, (uint8_t*)packed, geo.G);
@@ -189,6 +212,8 @@ extern "C" cudaError_t qlin_launch_unpack(int fmt, const void* packed, int64_t N
         unpack_kernel<QLIN_Q4_0><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     else if (fmt == QLIN_Q8_0)
         unpack_kernel<QLIN_Q8_0><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
+    else if (fmt == QLIN_MXFP4)
+        unpack_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     else
         unpack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     return cudaGetLastError();

@@ -19,6 +19,7 @@ namespace qlin {
 //           as two planes [half][row][part]; vector index of (row r, part p) is r * 8 + p.
 //   scales: 32 lanes x 16 B.  Lane l = (r % 4) * 8 + p holds, in slot i = r / 4, the scale(s) of
 //           (row r, part p): one fp16 d (Q8_0 / Q4_0) or two E4M3 bytes (NVFP4, one per 16).
+//           MXFP4: 32 lanes x 8 B, one UE8M0 byte per (row, part) in slot i.
 // A warp reading vector (lane + 32 * i) in step i therefore touches 512 contiguous bytes, and
 // lane l always works on part l % 8 of rows l / 8 + 4 i (i = 0..7).
 // Element order inside a part:
@@ -46,7 +47,7 @@ struct PackedHeader {
 static_assert(sizeof(PackedHeader) == kHdrBytes, "header size");
 
 __host__ __device__ constexpr int code_bytes(int fmt) { return fmt == QLIN_Q8_0 ? 8192 : 4096; }
-__host__ __device__ constexpr int unit_bytes(int fmt) { return code_bytes(fmt) + 512; }
+__host__ __device__ constexpr int unit_bytes(int fmt) { return code_bytes(fmt) + (fmt == QLIN_MXFP4 ? 256 : 512); }
 
 struct Geometry {
     int64_t T, G, U;  // tiles, k-groups, units
@@ -151,6 +152,13 @@ __device__ __forceinline__ float fp16_bits_to_f32(uint32_t h) {
 }
 
 // OCP E4M3 ("fn") byte -> fp32, exact (hardware conversion via the x2 form).
+// OCP MX UE8M0 scale byte: 2^(b - 127) as fp32 (b = 0: the subnormal 2^-127), 0xFF = NaN.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
+    b &= 0xffu;
+    if (b == 0xffu) return __uint_as_float(0x7fc00000u);
+    return __uint_as_float(b == 0u ? 0x00400000u : b << 23);
+}
+
 __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
     uint32_t h2;
     uint16_t in = static_cast<uint16_t>(b & 0xffu);

@@ -1,13 +1,15 @@
 /*
  * qlin.h -- C ABI of libqlin, a B200 (sm_100a) library for the decode-step linear layer over
- * block-quantized weights: fused dequantize-and-multiply of GGUF Q8_0 / Q4_0 blocks and NVFP4
- * tensors against a small batch of activation rows, the routed MoE expert projections, and an
- * NVFP4 prefill-chunk GEMM on the tcgen05 tensor cores.
+ * block-quantized weights: fused dequantize-and-multiply of GGUF Q8_0 / Q4_0 blocks and NVFP4 /
+ * MXFP4 tensors against a small batch of activation rows, the routed MoE expert projections, and
+ * an NVFP4 prefill-chunk GEMM on the tcgen05 tensor cores.
  *
  * What the operations compute comes from the pages describing the "imp" engine (README
  * "Features" table, rows "Quantization", "Architectures" and "sm_120a kernels"; README "Why this
- * exists") and the "Imparo" engine (README intro: Q4_0 MoE decode with CUDA expert routing).  The
- * pages name the formats but not their byte layout; the layouts below are the public conventions.
+ * exists"; release notes v0.6, "Native MXFP4 GGUF weight format") and the "Imparo" engine (README
+ * intro: Q4_0 MoE decode with CUDA expert routing).  The pages name the formats but not their byte
+ * layout; the layouts below are the public conventions (MXFP4: the OCP MX one, with the code byte
+ * order of NVFP4).
  *
  * Conventions for every entry point
  *   - W is N x K (output x input), row-major along K; y[m][n] = sum_k x[m][k] * W[n][k].
@@ -34,7 +36,7 @@ extern "C" {
 
 typedef struct CUstream_st* qlin_stream_t; /* a cudaStream_t */
 
-typedef enum { QLIN_Q8_0 = 1, QLIN_Q4_0 = 2, QLIN_NVFP4 = 3 } qlin_format_t;
+typedef enum { QLIN_Q8_0 = 1, QLIN_Q4_0 = 2, QLIN_NVFP4 = 3, QLIN_MXFP4 = 4 } qlin_format_t;
 typedef enum { QLIN_F32 = 0, QLIN_BF16 = 1 } qlin_dtype_t;
 typedef enum {
     QLIN_OK = 0,
@@ -86,7 +88,7 @@ enum { QLIN_OP_GEMV = 1, QLIN_OP_MOE = 2, QLIN_OP_CHUNK = 3 };
  * warp reads contiguously, followed by that tile's scales; K is padded to a multiple of 256 and N
  * to a multiple of 32 (16 per half for QLIN_PACK_GATE_UP) with zero codes and zero scales.
  * The packed size is the canonical size plus that padding (Q8_0 1.0625 B/weight, Q4_0 and NVFP4
- * 0.5625 B/weight).  Prior art for a private re-laid-out weight copy: Imparo README intro
+ * 0.5625 B/weight, MXFP4 0.53125 B/weight).  Prior art for a private re-laid-out weight copy: Imparo README intro
  * ("private GateUp layout"); imp README "Why this exists" (an NVFP4 decode cache built at init). */
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags);
 
@@ -96,7 +98,11 @@ size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags
  *          element j low, element j+16 high), scales = NULL
  *   NVFP4: blocks = E2M1 codes [N][K/2] (byte i: element 2i low nibble, 2i+1 high nibble),
  *          scales = E4M3 [N][K/16], global_scale = the fp32 per-tensor scale
- * K % 32 == 0 for Q8_0 / Q4_0, K % 16 == 0 for NVFP4; N >= 1; QLIN_PACK_GATE_UP needs N even.
+ *   MXFP4: blocks = E2M1 codes as NVFP4, scales = UE8M0 bytes [N][K/32] (value 2^(byte - 127),
+ *          0xFF = NaN), global_scale ignored (imp release notes v0.6: E2M1 + UE8M0 block scales,
+ *          4.25 bits per weight)
+ * K % 32 == 0 for Q8_0 / Q4_0 / MXFP4, K % 16 == 0 for NVFP4; N >= 1; QLIN_PACK_GATE_UP needs N
+ * even.
  * `packed` must be 256-byte aligned and hold qlin_packed_bytes(...) bytes.  Canonical inputs
  * have no alignment requirement.  The canonical buffers may be freed once the kernel has run. */
 qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const void* blocks,
@@ -211,7 +217,7 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
  *   x : M x H rows (fp32 or bf16), contiguous;  y : M x H fp32, contiguous
  *   h : optional M x top_k x I fp32 output of the SiLU-gated intermediate (NULL: kept in ws)
  *   flags: 0 or QLIN_FLAG_PDL;  ws: qlin_workspace_bytes(QLIN_OP_MOE, fmt, M, H, I, E, top_k)
- * E <= 256, top_k <= min(8, E), H <= 32768 (else QLIN_ERR_UNSUPPORTED).  One kernel launch on
+ * E <= 256, top_k <= min(8, E), H <= 32768, fmt other than QLIN_MXFP4 (else QLIN_ERR_UNSUPPORTED).  One kernel launch on
  * `stream` (routing, gate_up of the selected experts, down, weighted sum), no host
  * synchronisation.  The status word (qlin_ws_status) reports a bad input expert id (the slot is
  * skipped) or a timed-out device wait. */
@@ -252,8 +258,8 @@ qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx,
 
 /* Dequantize a packed buffer back to fp32 W[N][K] (row-major, canonical row order, also for
  * QLIN_PACK_GATE_UP buffers; pass the pack_flags the buffer was packed with).  The value of every
- * weight is the exact fp32 number d*q (Q8_0), d*(q-8) (Q4_0), or fp32(e2m1*e4m3*g) rounded once
- * (NVFP4).  A test and inspection aid; not on the hot path.  w must be 4-byte aligned. */
+ * weight is the exact fp32 number d*q (Q8_0), d*(q-8) (Q4_0), fp32(e2m1*e4m3*g) rounded once
+ * (NVFP4), or e2m1 * 2^(scale - 127) (MXFP4: exact, +-Inf where it overflows fp32).  A test and inspection aid; not on the hot path.  w must be 4-byte aligned. */
 qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
                                  int pack_flags, float* w, qlin_stream_t stream);
 

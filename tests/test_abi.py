@@ -50,6 +50,9 @@ def test_packed_bytes_sizes(lib):
     assert q.qlin_packed_bytes(q.QLIN_Q4_0, 64, 256, q.QLIN_PACK_GATE_UP) == 256 + 2 * 4608
     assert q.qlin_packed_bytes(q.QLIN_Q4_0, 64, 100) == 0  # K % 32
     assert q.qlin_packed_bytes(q.QLIN_NVFP4, 64, 40) == 0  # K % 16
+    # MXFP4: codes as NVFP4, one scale byte per 32 values: 4096 + 256 bytes per 32 x 256 unit
+    assert q.qlin_packed_bytes(q.QLIN_MXFP4, 4096, 2560) == 256 + 4096 * 2560 * 17 // 32
+    assert q.qlin_packed_bytes(q.QLIN_MXFP4, 64, 272) == 0  # K % 32
     assert q.qlin_packed_bytes(7, 64, 256) == 0
     assert q.qlin_packed_bytes(q.QLIN_Q4_0, 63, 256, q.QLIN_PACK_GATE_UP) == 0  # odd N
 
@@ -82,6 +85,8 @@ def test_pack_argument_checks(lib):
     f = lib.qlin_pack_weights
     assert f(2, 64, 256, P(0), None, 1.0, 0, P(0x1000), 1 << 30, None) == 1
     assert f(3, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # NVFP4 needs scales
+    assert f(4, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # MXFP4 needs scales
+    assert f(4, 64, 256, P(0x1000), P(0x2000), 1.0, 2, P(0x10000), 1 << 30, None) == 2  # no MMA layout
     assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10010), 1 << 30, None) == 3
     assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 10, None) == 1
     assert f(2, 64, 256, P(0x1000), None, 1.0, 8, P(0x10000), 1 << 30, None) == 1
@@ -129,3 +134,11 @@ def test_chain_workspace_bytes(lib):
     b8 = q.qlin_chain_workspace_bytes(q.QLIN_Q4_0, 8, ops)
     assert 256 < b1 < b8 and b1 % 256 == 0
     assert q.qlin_chain_workspace_bytes(q.QLIN_Q4_0, 1, [_chain_op(wait_for=0)]) == 0
+
+
+def test_moe_rejects_mxfp4_before_launch(lib):
+    P = ctypes.c_void_p
+    st = lib.qlin_moe_experts(q.QLIN_MXFP4, P(0x100000), P(0x200000), 32, 2048, 1792, 4, P(0x300000),
+                              P(0x400000), P(0x500000), P(0x600000), 1, 1, P(0x700000), None, 0,
+                              P(0x800000), 1 << 30, None)
+    assert st == 2  # QLIN_ERR_UNSUPPORTED

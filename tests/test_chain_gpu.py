@@ -15,7 +15,7 @@ import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
-FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4]
+FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4, q.QLIN_MXFP4]
 TOL = 2e-6
 
 
@@ -158,7 +158,7 @@ def test_chain_argument_checks():
     assert lib.qlin_gemv_chain(fmt, q.QLIN_F32, M, ptr, 1, 0, q._dev(ws, "ws"), 16, q._stream()) == 4
 
 
-@pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_Q4_0])
+@pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_Q4_0, q.QLIN_MXFP4])
 @pytest.mark.parametrize("M", [1, 4])
 def test_chain_bf16_mlp(fmt, M):
     """A bf16 chain of gated MLPs: gate_up writes h in bf16 (QLIN_OUT_BF16), down reads it."""

@@ -13,7 +13,7 @@ import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
-FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4]
+FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4, q.QLIN_MXFP4]
 TOL = 2e-6
 
 
@@ -45,6 +45,23 @@ def test_dequant_bit_exact(fmt, N, K):
     w = q.qlin_dequant_debug(fmt, packed, N, K).cpu().numpy()
     ref = oracle.dequant_f32(fmt, N, K, blocks, scales, g)
     assert np.array_equal(w.view(np.uint32), ref.view(np.uint32))
+
+
+def test_dequant_mxfp4_special_scale_bytes():
+    """UE8M0 bytes at the ends of the range: 0 (2^-127, subnormal products), 1, 126..128, 254
+    (6 * 2^127 overflows fp32 to Inf on both sides) and 255 (NaN).  Non-NaN weights bit-exact,
+    NaN exactly where the oracle has NaN."""
+    N, K = 32, 512
+    codes, _, _ = synth.weights(q.QLIN_MXFP4, N, K, synth.gen(8))
+    special = torch.tensor([0, 1, 126, 127, 128, 254, 255, 130], dtype=torch.uint8)
+    scales = special.repeat(N * K // 32 // 8 + 1)[: N * K // 32].reshape(N, K // 32).contiguous()
+    packed = q.qlin_pack_weights(q.QLIN_MXFP4, N, K, codes.cuda(), scales.cuda())
+    w = q.qlin_dequant_debug(q.QLIN_MXFP4, packed, N, K).cpu().numpy()
+    ref = oracle.dequant_f32(q.QLIN_MXFP4, N, K, codes.numpy(), scales.numpy())
+    nan = np.isnan(ref)
+    assert nan.any() and np.isinf(ref).any()
+    assert np.array_equal(np.isnan(w), nan)
+    assert np.array_equal(w[~nan].view(np.uint32), ref[~nan].view(np.uint32))
 
 
 def test_dequant_nvfp4_k_multiple_of_16_only():

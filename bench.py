@@ -437,8 +437,9 @@ def run_config(name, args):
         lines.append(dict(workload="Q8_0 GEMV M=1 K=1024 N=256 (launch-latency bound; graph of 1000 "
                           "launches over distinct weight copies, PDL)", M=M, us_per_launch=ms * 1e3,
                           gbs=bytes_ / (ms * 1e-3) / 1e9))
-    elif name == "nvfp4_mlp":
-        fmt, H, I = q.QLIN_NVFP4, 5120, 17408
+    elif name in ("nvfp4_mlp", "mxfp4_mlp"):
+        fmt, H, I = (q.QLIN_NVFP4 if name == "nvfp4_mlp" else q.QLIN_MXFP4), 5120, 17408
+        fname = "NVFP4" if fmt == q.QLIN_NVFP4 else "MXFP4"
         for M in (1, 4):
             L = 2
             gu, dn, wsg, wsd = [], [], [], []
@@ -460,7 +461,7 @@ def run_config(name, args):
             ms = _time_graph_of(fn, args.steps, args.warmup) / L
             wb = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
             bytes_ = wb + M * (2 * H + 4 * I + 4 * I + 4 * H)
-            lines.append(dict(workload="NVFP4 MLP shaped like a 27B model: gate_up 5120->2x17408 + SiLU, "
+            lines.append(dict(workload=f"{fname} MLP shaped like a 27B model: gate_up 5120->2x17408 + SiLU, "
                               "down 17408->5120, bf16 activations; one qlin_gemv per projection (fp32 h)",
                               M=M, us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9,
                               tokens_per_s=M / (ms * 1e-3)))
@@ -474,7 +475,7 @@ def run_config(name, args):
             fn2 = lambda: q.qlin_gemv_chain(fmt, q.QLIN_BF16, M, ops, flags=q.QLIN_FLAG_PDL, ws=cws)
             ms2 = _time_graph_of(fn2, args.steps, args.warmup) / L
             bytes2 = wb + M * (2 * H + 2 * I + 2 * I + 4 * H)
-            lines.append(dict(workload="NVFP4 MLP shaped like a 27B model, as above; both layers as one "
+            lines.append(dict(workload=f"{fname} MLP shaped like a 27B model, as above; both layers as one "
                               "GEMV chain, h in bf16", M=M, us_per_layer=ms2 * 1e3,
                               gbs=bytes2 / (ms2 * 1e-3) / 1e9, tokens_per_s=M / (ms2 * 1e-3)))
             del gu, dn
@@ -558,7 +559,7 @@ def main():
     ap.add_argument("--dataflow", default="stated", choices=list(DenseStack.DATAFLOWS),
                     help="stated: independent inputs, down reads h; serial: every projection reads the "
                          "previous one's output (reported as an extra field either way)")
-    ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "moe", "chunk"],
+    ap.add_argument("--config", default="stack", choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
     if args.config != "stack":

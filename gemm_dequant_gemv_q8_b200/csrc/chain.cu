@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
     using C = RingCfg<FMT>;
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     constexpr bool kOnePass = MAXM <= 2;
-    constexpr bool kH = (FMT == QLIN_NVFP4) && XBF16;
+    constexpr bool kH = (FMT == QLIN_NVFP4 || FMT == QLIN_MXFP4) && XBF16;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kGemvWarps + warp;
@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                 uint32_t xh[MP][16];
                 float xsc[MP][2];
                 load_x_fp4h_staged<MP>(xcur, part, xh, xsc);
-                unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+                unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
             } else {
                 float2 xv[MP][16];
                 float xb[MP];
@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                 uint32_t xh[MP][16];
                 float xsc[MP][2];
                 load_x_fp4h<MP, true>(rows, k0, o.K, xh, xsc);
-                unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+                unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
             } else {
                 float2 xv[MP][16];
                 float xb[MP];
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                     uint32_t xh[MP][16];
                     float xsc[MP][2];
                     load_x_fp4h<MP, true>(rows, k0, o.K, xh, xsc);
-                    unit_dot_fp4h<MP>(ubuf, lane, xh, xsc, res);
+                    unit_dot_fp4h<MP, false, FMT>(ubuf, lane, xh, xsc, res);
                 } else {
                     float2 xv[MP][16];
                     float xb[MP];

@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) gem
     using C = RingCfg<FMT>;
     constexpr int MP = MAXM >= 2 ? 2 : 1;
     constexpr bool kOnePass = MAXM <= 2;
-    constexpr bool kH = (FMT == QLIN_NVFP4) && XBF16;  // f16-product path (see load_x_fp4h)
+    constexpr bool kH = (FMT == QLIN_NVFP4 || FMT == QLIN_MXFP4) && XBF16;  // f16-product path (see load_x_fp4h)
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ float slots[kGemvWarps][2][32][MAXM];  // warp-boundary tile partials
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) gem
             }
         }
         if (kOnePass) {
-            if constexpr (kH) unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+            if constexpr (kH) unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
             else unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
         } else {
             const int64_t k0 = (int64_t)g * kGroupK + part * 32;
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) gem
                     uint32_t xph[MP][16];
                     float xps[MP][2];
                     load_x_fp4h<MP>(rows, k0, a.K, xph, xps);
-                    unit_dot_fp4h<MP>(ubuf, lane, xph, xps, res);
+                    unit_dot_fp4h<MP, false, FMT>(ubuf, lane, xph, xps, res);
                 } else {
                     float xpb[MP];
                     load_x_rows<XBF16, MP>(rows, k0, a.K, xp);

@@ -348,16 +348,28 @@ __device__ __forceinline__ void dec_fp4_h(uint32_t w, uint32_t (&h)[4]) {
         : "r"(w));
 }
 
-// NVFP4 unit dot with f16 products (see load_x_fp4h); same contract as unit_dot.
-template <int MP, bool ACC = false>
+// NVFP4 / MXFP4 unit dot with f16 products (see load_x_fp4h); same contract as unit_dot.
+// FMT: QLIN_NVFP4 (two E4M3 scales per part) or QLIN_MXFP4 (one UE8M0 scale for both halves).
+template <int MP, bool ACC = false, int FMT = QLIN_NVFP4>
 __device__ __forceinline__ void unit_dot_fp4h(const uint8_t* ub, int lane, const uint32_t (&xh)[MP][16],
                                               const float (&xsc)[MP][2], float (&res)[8][MP]) {
-    const uint4 sv = lds128(ub + 4096 + lane * 16);
-    const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+    uint32_t sw[4];
+    if (FMT == QLIN_MXFP4) {
+        const uint2 s2 = *reinterpret_cast<const uint2*>(ub + 4096 + lane * 8);
+        sw[0] = s2.x, sw[1] = s2.y, sw[2] = sw[3] = 0u;
+    } else {
+        const uint4 sv = lds128(ub + 4096 + lane * 16);
+        sw[0] = sv.x, sw[1] = sv.y, sw[2] = sv.z, sw[3] = sv.w;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const uint32_t sc = sw[i >> 1] >> (16 * (i & 1));
-        const float e0 = e4m3_to_f32(sc & 0xffu), e1 = e4m3_to_f32((sc >> 8) & 0xffu);
+        float e0, e1;
+        if (FMT == QLIN_MXFP4) {
+            e0 = e1 = e8m0_to_f32(sw[i >> 2] >> (8 * (i & 3)));
+        } else {
+            const uint32_t sc = sw[i >> 1] >> (16 * (i & 1));
+            e0 = e4m3_to_f32(sc & 0xffu), e1 = e4m3_to_f32((sc >> 8) & 0xffu);
+        }
         const uint4 c = lds128(ub + (lane + 32 * i) * 16);
         const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll

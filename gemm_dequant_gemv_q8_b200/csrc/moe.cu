@@ -9,20 +9,22 @@
 // The routing is computed on the device -- no host round trip, so the layer is graph-capturable
 // (the lesson of the imp release notes v0.7.0, where a host round trip of the routing made MoE
 // decode incompatible with CUDA graphs) -- redundantly by every CTA in shared memory (M x E is
-// tiny), which then plans the launch on the device exactly as the GEMV chain plans it on the
-// host (chain.cu): the gate_up units of the selected experts (each expert once, for all tokens
-// routed to it) form segment 0, their down units segment 1, and each segment is split into one
-// contiguous range per warp.  A warp reaching an expert's down units waits (bounded) only for that
-// expert's gate_up tiles.  The last of a token's experts to write a down tile adds the token's
-// slot outputs for that tile in slot order (a ticket per token and tile): deterministic.  Split
-// tiles use the chain's tagged partial words, stored per warp.
+// tiny), which then plans the launch on the device: the work entries (a selected expert with up
+// to two of the tokens routed to it; an expert chosen by more tokens gets more entries) put their
+// gate_up tiles in step 0 and their down tiles in step 1, and each step's tiles are split into
+// one contiguous range per CTA.  A CTA owns its tiles whole: its four warps take the tiles' units
+// (k-groups) in turn, each through its own ring of bulk copies, and add their parts in shared
+// memory.  A CTA reaching an entry's down tiles waits (bounded) only for that entry's gate_up
+// tiles.  The last of a token's experts to write a down tile adds the token's slot outputs for
+// that tile in slot order (a ticket per token and tile): deterministic.
 #include "gemv_core.cuh"
 
 namespace qlin {
 
 constexpr int kMoeMaxTopK = 8;
 constexpr int kMoeMaxM = 8;
-constexpr int kMoeMaxAct = kMoeMaxM * kMoeMaxTopK;
+constexpr int kMoeMaxAct = kMoeMaxM * kMoeMaxTopK;  // work entries (an entry holds >= 1 row)
+constexpr int kMoeEntryRows = 2;                     // rows per work entry
 
 struct MoeArgs {
     const uint8_t* gu;  // E stacked gate_up buffers (QLIN_PACK_GATE_UP, 2I x H)
@@ -39,124 +41,131 @@ struct MoeArgs {
     uint8_t* ws;
     int T0, G0, U0;       // per expert, gate_up: tiles (16 gate + 16 up rows), k-groups over H, units
     int T1, G1, U1;       // per expert, down: tiles of 32 rows of H, k-groups over I, units
-    int W;                // warps in the grid
 };
 
 // Workspace: [0,4) status word (bit 0 timeout, bit 1 bad expert id); [64,68) exit counter;
-// [128,132) launch counter; [256, ...) per-active-expert gate_up tile counts; per-(token, down
-// tile) combine tickets (self-resetting); partial words [segment][warp range][first piece, last
-// piece][32][M].
+// [256, ...) per-work-entry gate_up tile counts; per-(token, down tile) combine tickets (both
+// reset by the last CTA to leave); then the down outputs o and the SiLU-gate outputs h.
 constexpr int64_t kMoeExitOff = 64;
-constexpr int64_t kMoeEpochOff = 128;
 constexpr int64_t kMoeDoneOff = 256;
 constexpr int kMoeMaxT1 = 1024;  // down tiles per expert (H <= 32768)
 __host__ __device__ inline int64_t moe_comb_off() { return kMoeDoneOff + 4 * kMoeMaxAct; }
-__host__ __device__ inline int64_t moe_part_off() { return moe_comb_off() + 4 * (int64_t)kMoeMaxM * kMoeMaxT1; }
+__host__ __device__ inline int64_t moe_head_bytes() { return moe_comb_off() + 4 * (int64_t)kMoeMaxM * kMoeMaxT1; }
 
 // ------------------------------------------------------------------ device-side plan
-// Segment s (0 = gate_up, 1 = down) of the selected experts: per expert Ue units (T tiles x G
-// k-groups), U = n_act Ue in all, warp range v holding q + (v < r) of them, v = (gw - rot) mod W.
+// Segment s (0 = gate_up, 1 = down) of the work entries: Tt = n_act T tiles of G k-group units
+// each.  CTA v = (blockIdx - rot) mod gridDim owns tiles [v q + min(v, r), + q + (v < r)) whole:
+// its four warps take the tiles' units in turn and add their parts in shared memory, so no tile
+// is shared between CTAs and nothing waits for another CTA's piece of a tile.
 struct MoeSeg {
-    int U, q, r, rot, Ue, G, T;
+    int Tt, q, r, rot, G, T;
 };
 
 struct RouteSmem {
     MoeSeg sg[2];  // the device-side plan (identical in every CTA)
+    int tb[2], te[2];  // this CTA's tiles of each step
     int n_act;
     int expert[kMoeMaxAct];
     int nrows[kMoeMaxAct];
-    int8_t row_m[kMoeMaxAct][kMoeMaxM];
-    int8_t row_s[kMoeMaxAct][kMoeMaxM];
+    int8_t row_m[kMoeMaxAct][kMoeEntryRows];
+    int8_t row_s[kMoeMaxAct][kMoeEntryRows];
     int ids[kMoeMaxM][kMoeMaxTopK];
     float w[kMoeMaxM][kMoeMaxTopK];
     int kvalid[kMoeMaxM];  // valid slots of each token
 };
 
-// Routing of all tokens into shared memory (whole CTA participates).  With logits, CTA 0 also
-// writes ids and weights out.  Invalid or repeated input ids skip their slot and set status bit 1.
+// Routing of all tokens into shared memory (whole CTA participates).  With logits, one warp per
+// token: lane l holds the logits of experts l + 32 j, and every expert's slot is its rank in the
+// order "larger logit first, a tie to the lower expert index" (NaN ranks as -inf), counted
+// against all experts at once -- independent comparisons, where top_k argmax rounds would be a
+// chain of dependent shuffles.  The selection is the one a sequential scan with a strict
+// comparison makes.  CTA 0 also writes ids and weights out.  Without logits, invalid or repeated
+// input ids skip their slot and set status bit 1.
 constexpr int kMoeMaxE = 256;
 
-__device__ void moe_route(const MoeArgs& a, RouteSmem& r) {
+__device__ __forceinline__ float moe_key(float v) { return v != v ? -INFINITY : v; }
+
+__device__ __forceinline__ void moe_route(const MoeArgs& a, RouteSmem& r) {
     const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
     if (a.logits) {
-        // One warp per token: each lane holds the logits of experts lane + 32 j; top_k rounds of a
-        // warp-wide argmax (largest logit, ties to the lower expert index -- the order a
-        // sequential scan with a strict comparison gives).
-        const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-        // all of this warp's logits first, so that their loads are in flight together
         constexpr int kTokPerWarp = (kMoeMaxM + kGemvWarps - 1) / kGemvWarps;
-        float vall[kTokPerWarp][kMoeMaxE / 32];
+        constexpr int kJ = kMoeMaxE / 32;
+        const int J = (a.E + 31) >> 5;
+        float vall[kTokPerWarp][kJ];  // all of this warp's logits first: their loads fly together
 #pragma unroll
         for (int i = 0; i < kTokPerWarp; ++i) {
             const int m = warp + i * nw;
 #pragma unroll
-            for (int j = 0; j < kMoeMaxE / 32; ++j) {
+            for (int j = 0; j < kJ; ++j) {
                 const int e = lane + 32 * j;
-                vall[i][j] = (m < a.M && e < a.E) ? __ldcg(a.logits + (int64_t)m * a.E + e) : -INFINITY;
+                vall[i][j] = (m < a.M && e < a.E) ? moe_key(__ldcg(a.logits + (int64_t)m * a.E + e)) : -INFINITY;
             }
         }
 #pragma unroll
         for (int i = 0; i < kTokPerWarp; ++i) {
             const int m = warp + i * nw;
             if (m >= a.M) break;
-            float v[kMoeMaxE / 32];
+            int rank[kJ];
 #pragma unroll
-            for (int j = 0; j < kMoeMaxE / 32; ++j) v[j] = vall[i][j];
-            float lsel[kMoeMaxTopK];
-            unsigned taken = 0;  // bit j: expert lane + 32 j already selected
-            for (int s = 0; s < a.top_k; ++s) {
-                float bv = -INFINITY;
-                int be = 0x7fffffff;
+            for (int j = 0; j < kJ; ++j) rank[j] = 0;
+            if (J == 1) {
+                const float v = vall[i][0];
 #pragma unroll
-                for (int j = 0; j < kMoeMaxE / 32; ++j) {
-                    const int e = lane + 32 * j;
-                    if (e < a.E && !((taken >> j) & 1u) && (be == 0x7fffffff || v[j] > bv || (v[j] == bv && e < be))) {
-                        bv = v[j];
-                        be = e;
+                for (int src = 0; src < 32; ++src) {
+                    const float ov = __shfl_sync(0xffffffffu, v, src);
+                    rank[0] += (src < a.E) & ((ov > v) | ((ov == v) & (src < lane)));
+                }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < kJ; ++jj) {
+                    if (jj >= J) break;
+#pragma unroll 4
+                    for (int src = 0; src < 32; ++src) {
+                        const float ov = __shfl_sync(0xffffffffu, vall[i][jj], src);
+                        const int oe = src + 32 * jj;
+#pragma unroll
+                        for (int j = 0; j < kJ; ++j)
+                            if (j < J)
+                                rank[j] += (oe < a.E) & ((ov > vall[i][j]) | ((ov == vall[i][j]) & (oe < lane + 32 * j)));
                     }
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                    const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-                    if (oe != 0x7fffffff && (be == 0x7fffffff || ov > bv || (ov == bv && oe < be))) {
-                        bv = ov;
-                        be = oe;
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < kMoeMaxE / 32; ++j)  // take it out of later rounds
-                    if (lane + 32 * j == be) taken |= 1u << j;
-                lsel[s] = bv;
-                if (lane == 0) r.ids[m][s] = be;
             }
-            if (lane == 0) {  // renormalised softmax over the selected experts
-                float z = 0.f;
-                for (int s = 0; s < a.top_k; ++s) {
-                    r.w[m][s] = expf(lsel[s] - lsel[0]);
-                    z += r.w[m][s];
+#pragma unroll
+            for (int j = 0; j < kJ; ++j) {
+                const int e = lane + 32 * j;
+                if (e < a.E && rank[j] < a.top_k) {
+                    r.ids[m][rank[j]] = e;
+                    r.w[m][rank[j]] = vall[i][j];
                 }
-                for (int s = 0; s < a.top_k; ++s) r.w[m][s] = r.w[m][s] / z;
-                if (blockIdx.x == 0)
-                    for (int s = 0; s < a.top_k; ++s) {
-                        a.ids[(int64_t)m * a.top_k + s] = r.ids[m][s];
-                        a.wts[(int64_t)m * a.top_k + s] = r.w[m][s];
-                    }
+            }
+            __syncwarp();
+            // weights renormalised over the selected experts: exp(l_s - l_0) / sum
+            const float ex = lane < a.top_k ? expf(r.w[m][lane] - r.w[m][0]) : 0.f;
+            float z = ex;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+            __syncwarp();
+            if (lane < a.top_k) {
+                const float w = ex / z;
+                r.w[m][lane] = w;
+                if (blockIdx.x == 0) {
+                    a.ids[(int64_t)m * a.top_k + lane] = r.ids[m][lane];
+                    a.wts[(int64_t)m * a.top_k + lane] = w;
+                }
             }
         }
     } else if (tid < a.M) {
-        {
-            for (int s = 0; s < a.top_k; ++s) {
-                int e = a.ids[(int64_t)tid * a.top_k + s];
-                bool bad = e < 0 || e >= a.E;
-                for (int q = 0; q < s; ++q) bad |= (r.ids[tid][q] == e);
-                if (bad) {
-                    if (blockIdx.x == 0) atomicOr(reinterpret_cast<unsigned int*>(a.ws), 2u);
-                    e = -1;
-                }
-                r.ids[tid][s] = e;
-                r.w[tid][s] = a.wts[(int64_t)tid * a.top_k + s];
+        for (int s = 0; s < a.top_k; ++s) {
+            int e = a.ids[(int64_t)tid * a.top_k + s];
+            bool bad = e < 0 || e >= a.E;
+            for (int q = 0; q < s; ++q) bad |= (r.ids[tid][q] == e);
+            if (bad) {
+                if (blockIdx.x == 0) atomicOr(reinterpret_cast<unsigned int*>(a.ws), 2u);
+                e = -1;
             }
+            r.ids[tid][s] = e;
+            r.w[tid][s] = a.wts[(int64_t)tid * a.top_k + s];
         }
     }
     __syncthreads();
@@ -167,95 +176,98 @@ __device__ void moe_route(const MoeArgs& a, RouteSmem& r) {
         if (kv == 0 && blockIdx.x == 0)  // no expert: the token's output is zero
             for (int n = 0; n < a.H; ++n) a.y[(int64_t)tid * a.H + n] = 0.f;
     }
-    if (threadIdx.x < 32) {  // warp 0 compacts the active experts in ascending order
-        const int lane = threadIdx.x;
+    if (warp == 0) {
+        // Warp 0 lists the work entries: the selected experts in ascending order, each expert's
+        // rows in (token, slot) order, cut into entries of at most kMoeEntryRows rows (an expert
+        // chosen by more tokens streams its weights once per entry, the later reads mostly from L2).
         int n = 0;
         for (int base = 0; base < a.E; base += 32) {
             const int e = base + lane;
-            int cnt = 0;
-            int8_t rm[kMoeMaxM], rs[kMoeMaxM];
-            if (e < a.E)
-                for (int m = 0; m < a.M; ++m)
-                    for (int s = 0; s < a.top_k; ++s)
-                        if (r.ids[m][s] == e && cnt < kMoeMaxM) {
-                            rm[cnt] = (int8_t)m;
-                            rs[cnt] = (int8_t)s;
-                            ++cnt;
-                        }
-            const unsigned mask = __ballot_sync(0xffffffffu, cnt > 0);
-            if (cnt > 0) {
-                const int idx = n + __popc(mask & ((1u << lane) - 1u));
-                r.expert[idx] = e;
-                r.nrows[idx] = cnt;
-                for (int c = 0; c < cnt; ++c) {
-                    r.row_m[idx][c] = rm[c];
-                    r.row_s[idx][c] = rs[c];
-                }
+            int cnt = 0;  // at most one slot per token: cnt <= M
+            for (int m = 0; m < a.M; ++m)
+                for (int q = 0; q < a.top_k; ++q) cnt += r.ids[m][q] == e;
+            const int ne = (cnt + kMoeEntryRows - 1) / kMoeEntryRows;
+            int incl = ne;  // inclusive prefix sum of the entries over the lanes
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
             }
-            n += __popc(mask);
+            int idx = n + incl - ne, c = 0;
+            for (int m = 0; m < a.M; ++m)
+                for (int q = 0; q < a.top_k; ++q)
+                    if (r.ids[m][q] == e) {
+                        if (c == 0) {
+                            r.expert[idx] = e;
+                            r.nrows[idx] = min(kMoeEntryRows, cnt);
+                        }
+                        r.row_m[idx][c] = (int8_t)m;
+                        r.row_s[idx][c] = (int8_t)q;
+                        if (++c == kMoeEntryRows) {
+                            c = 0;
+                            ++idx;
+                            cnt -= kMoeEntryRows;
+                        }
+                    }
+            n += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0) r.n_act = n;
     }
     __syncthreads();
 }
 
-__device__ __forceinline__ void moe_range(const MoeSeg& s, int gw, int W, int& b, int& e) {
-    int v = gw - s.rot;
-    if (v < 0) v += W;
-    b = v * s.q + min(v, s.r);
-    e = b + s.q + (v < s.r ? 1 : 0);
-}
-
-__device__ __forceinline__ int moe_owner(const MoeSeg& s, int u) {
-    const int big = s.r * (s.q + 1);
-    if (u < big) return u / (s.q + 1);
-    return s.r + (u - big) / s.q;
-}
-
-// Position: segment s (2 = done), active expert a, unit uo of it (tile t, k-group g), segment
-// unit u; the warp's range in s ends at e.  Advanced incrementally (no division per unit).
+// A warp's position in its CTA's units of segment s (tile-major, k-group minor): list index i
+// (this warp takes i = warp, warp + 4, ...), local tile jl and k-group g, work entry act and its
+// tile t; n = units of the CTA in the segment.  Advanced incrementally (no division per unit).
 struct MoeCursor {
-    int s, a, uo, t, g, u, e;
+    int s, i, jl, g, act, t, n;
 };
 
-__device__ __forceinline__ void moe_seek(const MoeSeg (&sg)[2], int gw, int W, MoeCursor& c, int s) {
+__device__ __forceinline__ void moe_seek(const MoeSeg (&sg)[2], const int (&tb)[2], const int (&te)[2], int warp,
+                                         MoeCursor& c, int s) {
     for (; s < 2; ++s) {
-        int b, e;
-        moe_range(sg[s], gw, W, b, e);
-        if (e > b) {
+        const int n = (te[s] - tb[s]) * sg[s].G;
+        if (warp < n) {
             c.s = s;
-            c.a = b / sg[s].Ue;
-            c.uo = b - c.a * sg[s].Ue;
-            c.t = c.uo / sg[s].G;
-            c.g = c.uo - c.t * sg[s].G;
-            c.u = b;
-            c.e = e;
+            c.i = warp;
+            c.jl = warp / sg[s].G;
+            c.g = warp - c.jl * sg[s].G;
+            const int T = tb[s] + c.jl;
+            c.act = T / sg[s].T;
+            c.t = T - c.act * sg[s].T;
+            c.n = n;
             return;
         }
     }
     c.s = 2;
-    c.a = c.uo = c.t = c.g = c.u = c.e = 0;
+    c.i = c.jl = c.g = c.act = c.t = c.n = 0;
 }
 
-__device__ __forceinline__ void moe_step(const MoeSeg (&sg)[2], int gw, int W, MoeCursor& c) {
-    if (++c.u >= c.e) {
-        moe_seek(sg, gw, W, c, c.s + 1);
+__device__ __forceinline__ void moe_step(const MoeSeg (&sg)[2], const int (&tb)[2], const int (&te)[2], int warp,
+                                         MoeCursor& c) {
+    c.i += kGemvWarps;
+    if (c.i >= c.n) {
+        moe_seek(sg, tb, te, warp, c, c.s + 1);
         return;
     }
-    if (++c.uo == sg[c.s].Ue) {
-        ++c.a;
-        c.uo = c.t = c.g = 0;
-    } else if (++c.g == sg[c.s].G) {
-        c.g = 0;
-        ++c.t;
+    const MoeSeg& S = sg[c.s];
+    c.g += kGemvWarps;
+    while (c.g >= S.G) {
+        c.g -= S.G;
+        ++c.jl;
+        if (++c.t == S.T) {
+            c.t = 0;
+            ++c.act;
+        }
     }
 }
 
 template <int FMT>
-__device__ __forceinline__ const uint8_t* moe_unit_src(const MoeArgs& a, const RouteSmem& r, const MoeCursor& c) {
-    const uint8_t* base = c.s == 0 ? a.gu + (int64_t)r.expert[c.a] * a.gu_stride
-                                   : a.dn + (int64_t)r.expert[c.a] * a.dn_stride;
-    return base + kHdrBytes + (int64_t)c.uo * RingCfg<FMT>::UB;
+__device__ __forceinline__ const uint8_t* moe_unit_src(const MoeArgs& a, const RouteSmem& r, const MoeSeg (&sg)[2],
+                                                       const MoeCursor& c) {
+    const uint8_t* base = c.s == 0 ? a.gu + (int64_t)r.expert[c.act] * a.gu_stride
+                                   : a.dn + (int64_t)r.expert[c.act] * a.dn_stride;
+    return base + kHdrBytes + ((int64_t)c.t * sg[c.s].G + c.g) * RingCfg<FMT>::UB;
 }
 
 // Write tile t of active expert `act` in segment s: h rows with the SiLU gate (s = 0) or the
@@ -277,7 +289,8 @@ __device__ __forceinline__ void moe_write_tile(const MoeArgs& a, const RouteSmem
             for (int q = 0; q < MAXM; ++q)
                 if (q < nr) a.h[((int64_t)r.row_m[act][q] * a.top_k + r.row_s[act][q]) * a.I + i] = silu_f32(v[q]) * u[q];
         }
-        __threadfence();  // count the tile for the down units of this expert
+        // Count the tile for the down units of this expert: the warp barrier orders every lane's
+        // stores before lane 0's release (which is cumulative over them).
         __syncwarp();
         if (lane == 0) {
             unsigned int* done = reinterpret_cast<unsigned int*>(a.ws + kMoeDoneOff);
@@ -285,24 +298,29 @@ __device__ __forceinline__ void moe_write_tile(const MoeArgs& a, const RouteSmem
         }
         return;
     }
-    // Down tile: store the slot outputs, then take a ticket per token; the last of a token's
-    // experts for this tile adds the token's slot outputs in slot order into y.
+    // Down tile: store the slot outputs, then take a ticket per token (lane q for the expert's row
+    // q, all at once); the last of a token's experts for this tile adds the token's slot outputs
+    // in slot order into y.  The warp barriers carry the lanes' stores into the tickets' release
+    // and the tickets' acquire into every lane's loads.
     const int n = t * kTileRows + row;
     if (n < a.H) {
 #pragma unroll
         for (int q = 0; q < MAXM; ++q)
             if (q < nr) __stcg(a.o + ((int64_t)r.row_m[act][q] * a.top_k + r.row_s[act][q]) * a.H + n, v[q]);
     }
-    __threadfence();
     __syncwarp();
     unsigned int* comb = reinterpret_cast<unsigned int*>(a.ws + moe_comb_off());
+    unsigned int tk = 0;
+    if (lane < nr)
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(tk)
+                     : "l"(comb + r.row_m[act][lane] * a.T1 + t)
+                     : "memory");
+    __syncwarp();
     for (int q = 0; q < nr; ++q) {
         const int m = r.row_m[act][q];
-        unsigned int ticket = 0;
-        if (lane == 0) ticket = atomicAdd(comb + m * a.T1 + t, 1u);
-        ticket = __shfl_sync(0xffffffffu, ticket, 0);
+        const unsigned int ticket = __shfl_sync(0xffffffffu, tk, q);
         if (ticket == (unsigned)r.kvalid[m] - 1u) {
-            __threadfence();
             if (n < a.H) {
                 float sum = 0.f;
                 for (int k = 0; k < a.top_k; ++k)
@@ -312,85 +330,6 @@ __device__ __forceinline__ void moe_write_tile(const MoeArgs& a, const RouteSmem
             if (lane == 0) comb[m * a.T1 + t] = 0u;  // leave the workspace reusable
         }
     }
-}
-
-// Partial words of range index v, piece kind k (0: the first piece of its range, 1: the last).
-__device__ __forceinline__ uint64_t* moe_part(const MoeArgs& a, int s, int v, int k, int lane) {
-    return reinterpret_cast<uint64_t*>(a.ws + moe_part_off()) + ((((int64_t)s * a.W + v) * 2 + k) * 32 + lane) * a.M;
-}
-
-template <int MAXM>
-__device__ __forceinline__ void moe_publish(const MoeArgs& a, int s, int v, int k, int lane, const float (&acc)[MAXM],
-                                            uint32_t tag) {
-    uint64_t* w = moe_part(a, s, v, k, lane);
-#pragma unroll
-    for (int m = 0; m < MAXM; ++m)
-        if (m < a.M)
-            asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(w + m),
-                         "l"(((uint64_t)tag << 32) | __float_as_uint(acc[m]))
-                         : "memory");
-}
-
-__device__ __forceinline__ uint64_t moe_ld_relaxed(const uint64_t* p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Finish split tile t of expert `act` in segment s, whose first piece is range v's last piece and
-// whose other n_t - 1 pieces are the first pieces of ranges v+1 ..: add them in range order
-// (re-reading, bounded, words not yet tagged with this launch) and write the tile.
-template <int MAXM>
-__device__ __noinline__ bool moe_flush(const MoeArgs& a, const RouteSmem& r, int s, int act, int t, int v, int n_t,
-                                       int lane, float gs, uint32_t tag) {
-    float sum[MAXM];
-#pragma unroll
-    for (int m = 0; m < MAXM; ++m) sum[m] = 0.f;
-    // pieces fetched together (their loads in flight at once), then added in order; one at a time
-    // with 8 rows, where the wider batch costs more in registers than it saves
-    constexpr int kB = MAXM > 2 ? 1 : 4;
-    for (int i0 = 0; i0 < n_t; i0 += kB) {
-        uint64_t x[kB][MAXM];
-#pragma unroll
-        for (int b = 0; b < kB; ++b) {
-            const int i = i0 + b;
-            const uint64_t* w = i < n_t ? moe_part(a, s, v + i, i == 0 ? 1 : 0, lane) : nullptr;
-#pragma unroll
-            for (int m = 0; m < MAXM; ++m)
-                x[b][m] = (w != nullptr && m < a.M) ? moe_ld_relaxed(w + m) : ((uint64_t)tag << 32);
-        }
-        bool ready = true;
-#pragma unroll
-        for (int b = 0; b < kB; ++b)
-#pragma unroll
-            for (int m = 0; m < MAXM; ++m) ready &= (uint32_t)(x[b][m] >> 32) == tag;
-        if (!__all_sync(0xffffffffu, ready)) {
-            const uint64_t t0 = globaltimer_ns();
-            for (uint32_t it = 1;; ++it) {
-                __nanosleep(100);
-                ready = true;
-#pragma unroll
-                for (int b = 0; b < kB; ++b) {
-                    const int i = i0 + b;
-#pragma unroll
-                    for (int m = 0; m < MAXM; ++m)
-                        if (i < n_t && m < a.M && (uint32_t)(x[b][m] >> 32) != tag) {
-                            x[b][m] = moe_ld_relaxed(moe_part(a, s, v + i, i == 0 ? 1 : 0, lane) + m);
-                            ready &= (uint32_t)(x[b][m] >> 32) == tag;
-                        }
-                }
-                if (__all_sync(0xffffffffu, ready)) break;
-                if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
-            }
-        }
-#pragma unroll
-        for (int b = 0; b < kB; ++b)
-            if (i0 + b < n_t)
-#pragma unroll
-                for (int m = 0; m < MAXM; ++m) sum[m] += __uint_as_float((uint32_t)x[b][m]);
-    }
-    moe_write_tile<MAXM>(a, r, s, act, t, lane, sum, gs);
-    return true;
 }
 
 // Bounded wait until *p >= target (2 s); false on timeout.
@@ -430,78 +369,48 @@ __device__ __forceinline__ void moe_rows(const MoeArgs& a, const RouteSmem& r, i
     }
 }
 
-// One unit of segment s for the rows of active expert `act`.  One-pass (MAXM <= 2, or an expert
-// with at most 2 rows) accumulates into acc8 across a tile's units; otherwise each pass is
-// reduced at once into acc.  xs: the first pass's rows already staged in shared memory (or
-// NULL); after_first_load() runs once the first pass's activations are in registers.
+// One unit of segment s for the rows of work entry `act` (at most kMoeEntryRows = MAXM rows),
+// accumulated into acc8 across a tile's units.  xs: the rows already staged in shared memory (or
+// NULL); after_first_load() runs once the activations are in registers.
 template <int FMT, int MAXM, bool XB, typename F>
 __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, int s, int act, int g,
-                                         const uint8_t* ubuf, int lane, float (&acc8)[8][MAXM >= 2 ? 2 : 1],
-                                         float (&acc)[MAXM], const uint8_t* xs, F&& after_first_load) {
-    constexpr int MP = MAXM >= 2 ? 2 : 1;
-    const int nr = r.nrows[act];
-    const bool kOnePass = MAXM <= 2 || nr <= 2;  // an expert with at most 2 rows: accumulate in acc8
+                                         const uint8_t* ubuf, int lane, float (&acc8)[8][MAXM],
+                                         const uint8_t* xs, F&& after_first_load) {
+    constexpr int MP = MAXM;
     const int64_t Kin = s == 0 ? a.H : a.I;
     const int part = lane & 7;
     const int64_t k0 = (int64_t)g * kGroupK + part * 32;
-#pragma unroll 1
-    for (int q0 = 0; q0 < (kOnePass ? 1 : nr); q0 += MP) {
-        const void* rows[MP];
-        moe_rows<MP, XB>(a, r, s, act, q0, rows);
-        if constexpr (XB && FMT == QLIN_NVFP4) {
-            uint32_t xh[MP][16];
-            float xsc[MP][2];
-            if (q0 == 0 && xs != nullptr)
-                load_x_fp4h_staged<MP>(xs, part, xh, xsc);
-            else
-                load_x_fp4h<MP, true>(rows, k0, Kin, xh, xsc);
-            if (q0 == 0) after_first_load();
-            if (kOnePass) {
-                unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
-            } else {
-                float res[8][MP];
-                unit_dot_fp4h<MP>(ubuf, lane, xh, xsc, res);
-                float rr[MP];
-                reduce_scatter8<MP>(res, lane, rr);
-#pragma unroll
-                for (int qq = 0; qq < MAXM; ++qq)
-#pragma unroll
-                    for (int mm = 0; mm < MP; ++mm)
-                        if (qq == q0 + mm) acc[qq] += rr[mm];
-            }
-        } else {
-            float2 xv[MP][16];
-            float xb[MP];
-            if (q0 == 0 && xs != nullptr)
-                load_x_staged<XB, MP>(xs, part, xv);
-            else
-                load_x_rows<XB, MP, true>(rows, k0, Kin, xv);
-            if (q0 == 0) after_first_load();
-            prep_x<FMT, MP>(xv, xb);
-            if (kOnePass) {
-                unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
-            } else {
-                float res[8][MP];
-                unit_dot<FMT, MP>(ubuf, lane, xv, xb, res);
-                float rr[MP];
-                reduce_scatter8<MP>(res, lane, rr);
-#pragma unroll
-                for (int qq = 0; qq < MAXM; ++qq)
-#pragma unroll
-                    for (int mm = 0; mm < MP; ++mm)
-                        if (qq == q0 + mm) acc[qq] += rr[mm];
-            }
-        }
+    const void* rows[MP];
+    moe_rows<MP, XB>(a, r, s, act, 0, rows);
+    if constexpr (XB && FMT == QLIN_NVFP4) {
+        uint32_t xh[MP][16];
+        float xsc[MP][2];
+        if (xs != nullptr)
+            load_x_fp4h_staged<MP>(xs, part, xh, xsc);
+        else
+            load_x_fp4h<MP, true>(rows, k0, Kin, xh, xsc);
+        after_first_load();
+        unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+    } else {
+        float2 xv[MP][16];
+        float xb[MP];
+        if (xs != nullptr)
+            load_x_staged<XB, MP>(xs, part, xv);
+        else
+            load_x_rows<XB, MP, true>(rows, k0, Kin, xv);
+        after_first_load();
+        prep_x<FMT, MP>(xv, xb);
+        unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
     }
 }
 
-// Shared memory of the MoE kernel: the per-warp weight rings and their barriers, then (for at most
-// 2 rows, except Q8_0 whose ring leaves no room) one activation stage per warp: the next unit's
-// rows, copied while the current unit computes.  (With 8 rows the staging measured slower.)
+// Shared memory of the MoE kernel: the per-warp weight rings and their barriers, then (except
+// Q8_0, whose ring leaves no room) one activation stage per warp: the next unit's rows, copied
+// while the current unit computes.
 template <int FMT, int MAXM>
 struct MoeSmem {
-    static constexpr int MP = MAXM >= 2 ? 2 : 1;
-    static constexpr bool kStaged = FMT != QLIN_Q8_0 && MAXM <= 2;
+    static constexpr int MP = MAXM;
+    static constexpr bool kStaged = FMT != QLIN_Q8_0;
     static constexpr int kStageBytes = MP * XStage<false>::kRowBytes;  // fp32 layout; bf16 rows fit
     static constexpr int kXOff = (RingCfg<FMT>::kSmem + 127) / 128 * 128;
     static constexpr int kBytes = kStaged ? kXOff + kGemvWarps * kStageBytes : RingCfg<FMT>::kSmem;
@@ -514,15 +423,15 @@ __device__ __forceinline__ float moe_scale(const MoeArgs& a, const RouteSmem& r,
 }
 
 template <int FMT, int MAXM, bool XBF16>
-__global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe_kernel(const MoeArgs a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe_kernel(const __grid_constant__ MoeArgs a) {
     using C = RingCfg<FMT>;
     using MS = MoeSmem<FMT, MAXM>;
-    constexpr int MP = MAXM >= 2 ? 2 : 1;
-    constexpr bool kOnePass = MAXM <= 2;
+    constexpr int MP = MAXM;
+    static_assert(MAXM >= 1 && MAXM <= kMoeEntryRows, "rows per work entry");
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ RouteSmem r;
+    __shared__ float red[2][kGemvWarps][32][MP];  // the warps' parts of a tile (by tile parity)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * kGemvWarps + warp;
     uint8_t* ring = smem + warp * C::D * C::UB;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemvWarps * C::D * C::UB) + warp * C::D;
     uint8_t* xst = smem + MS::kXOff + warp * MS::kStageBytes;  // used only if MS::kStaged
@@ -530,187 +439,164 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
     griddep_launch_dependents();
     griddep_wait();  // logits / ids / x come from earlier kernels
     moe_route(a, r);
-    const uint32_t tag = __ldcg(reinterpret_cast<const unsigned int*>(a.ws + kMoeEpochOff)) + 1u;
     if (threadIdx.x == 0) {
         MoeSeg* sp = r.sg;
-        sp[0].Ue = a.U0; sp[0].G = a.G0; sp[0].T = a.T0;
-        sp[1].Ue = a.U1; sp[1].G = a.G1; sp[1].T = a.T1;
+        sp[0].G = a.G0; sp[0].T = a.T0;
+        sp[1].G = a.G1; sp[1].T = a.T1;
         for (int s = 0; s < 2; ++s) {
-            sp[s].U = r.n_act * sp[s].Ue;
-            sp[s].q = sp[s].U / a.W;
-            sp[s].r = sp[s].U % a.W;
+            sp[s].Tt = r.n_act * sp[s].T;
+            sp[s].q = sp[s].Tt / (int)gridDim.x;
+            sp[s].r = sp[s].Tt % (int)gridDim.x;
         }
         sp[0].rot = 0;
-        sp[1].rot = sp[0].r;  // the second step's extra units go to the warps after the first's
+        sp[1].rot = sp[0].r;  // the second step's extra tiles go to the CTAs after the first's
+        for (int s = 0; s < 2; ++s) {
+            int v = (int)blockIdx.x - sp[s].rot;
+            if (v < 0) v += gridDim.x;
+            r.tb[s] = v * sp[s].q + min(v, sp[s].r);
+            r.te[s] = r.tb[s] + sp[s].q + (v < sp[s].r ? 1 : 0);
+        }
     }
     __syncthreads();
     const MoeSeg (&sg)[2] = r.sg;
+    const int (&tb)[2] = r.tb;
+    const int (&te)[2] = r.te;
 
     MoeCursor c;
-    moe_seek(sg, gw, a.W, c, 0);
-    MoeCursor p = c;
+    moe_seek(sg, tb, te, warp, c, 0);
+    MoeCursor p = c;  // producer cursor, C::D units ahead once primed
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < C::D; ++s) mbar_init(&bars[s], 1);
         fence_mbar_init();
         for (int s = 0; s < C::D && p.s < 2; ++s) {
             mbar_arrive_expect_tx(&bars[s], C::UB);
-            bulk_g2s(ring + s * C::UB, moe_unit_src<FMT>(a, r, p), C::UB, &bars[s]);
-            moe_step(sg, gw, a.W, p);
+            bulk_g2s(ring + s * C::UB, moe_unit_src<FMT>(a, r, sg, p), C::UB, &bars[s]);
+            moe_step(sg, tb, te, warp, p);
         }
     }
     __syncwarp();
     p.s = __shfl_sync(0xffffffffu, p.s, 0);
-    p.a = __shfl_sync(0xffffffffu, p.a, 0);
-    p.uo = __shfl_sync(0xffffffffu, p.uo, 0);
-    p.t = __shfl_sync(0xffffffffu, p.t, 0);
+    p.i = __shfl_sync(0xffffffffu, p.i, 0);
+    p.jl = __shfl_sync(0xffffffffu, p.jl, 0);
     p.g = __shfl_sync(0xffffffffu, p.g, 0);
-    p.u = __shfl_sync(0xffffffffu, p.u, 0);
-    p.e = __shfl_sync(0xffffffffu, p.e, 0);
+    p.act = __shfl_sync(0xffffffffu, p.act, 0);
+    p.t = __shfl_sync(0xffffffffu, p.t, 0);
+    p.n = __shfl_sync(0xffffffffu, p.n, 0);
 
-    float acc[MAXM];
-#pragma unroll
-    for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
     float acc8[8][MP];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
     bool failed = false;
-    int pend_s = -1, pend_a = 0, pend_t = 0, pend_v = 0, pend_n = 0;  // split tile finished later
-    float pend_gs = 1.f;
-    int seq = 0, cur_s = -1, cur_a = -1, b = 0, e = 0;
-    bool xready = false;  // the current unit's first-pass rows are already staged
+    int seq = 0, waited = -1, tc = 0;
+    bool xready = false;  // the current unit's rows are already staged
     auto stage_unit = [&](const MoeCursor& u) {
         const void* rows[MP];
         if (u.s == 0) {
-            moe_rows<MP, XBF16>(a, r, 0, u.a, 0, rows);
+            moe_rows<MP, XBF16>(a, r, 0, u.act, 0, rows);
             stage_x_rows<XBF16, MP>(rows, a.H, u.g, xst, lane, a.ws);
         } else {
-            moe_rows<MP, false>(a, r, 1, u.a, 0, rows);
+            moe_rows<MP, false>(a, r, 1, u.act, 0, rows);
             stage_x_rows<false, MP>(rows, a.I, u.g, xst, lane, a.ws);
         }
     };
-    float gs = 1.f;
-    while (c.s < 2) {
-        if (c.s != cur_s) {  // new segment: finish the pending tile of the previous one
-            cur_s = c.s;
-            cur_a = -1;
-            moe_range(sg[c.s], gw, a.W, b, e);
-            if (pend_s >= 0) {
-                if (!moe_flush<MAXM>(a, r, pend_s, pend_a, pend_t, pend_v, pend_n, lane, pend_gs, tag)) {
+    const unsigned int* done = reinterpret_cast<const unsigned int*>(a.ws + kMoeDoneOff);
+    for (int s = 0; s < 2; ++s) {
+        const int T = sg[s].T;
+        int act = tb[s] / T, t = tb[s] - act * T;  // the CTA's current tile
+        float gs = act < r.n_act ? moe_scale<FMT>(a, r, s, act) : 1.f;
+        for (int jl = 0; jl < te[s] - tb[s]; ++jl, ++tc) {
+            // down units read h: wait (bounded) for this entry's gate_up tiles
+            if (s == 1 && act != waited && !failed) {
+                waited = act;
+                if (!moe_wait_count(done + act, (uint32_t)a.T0)) failed = true;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
+            while (!failed && c.s == s && c.jl == jl) {
+                const int slot = seq % C::D;
+                if (!mbar_wait_bounded(&bars[slot], (uint32_t)((seq / C::D) & 1))) {
                     failed = true;
                     break;
                 }
-                pend_s = -1;
-            }
-        }
-        if (c.a != cur_a) {
-            cur_a = c.a;
-            gs = moe_scale<FMT>(a, r, c.s, c.a);
-            // down units read h: wait for this expert's gate_up tiles
-            if (c.s == 1 && !moe_wait_count(reinterpret_cast<const unsigned int*>(a.ws + kMoeDoneOff) + c.a,
-                                            (uint32_t)a.T0)) {
-                failed = true;
-                break;
-            }
-        }
-        const int slot = seq % C::D;
-        if (!mbar_wait_bounded(&bars[slot], (uint32_t)((seq / C::D) & 1))) {
-            failed = true;
-            break;
-        }
-        const uint8_t* ubuf = ring + slot * C::UB;
-        const uint8_t* xs = nullptr;
-        MoeCursor cn = c;  // the next unit of this warp
-        bool stage_next = false;
-        if constexpr (MS::kStaged) {
-            if (!xready) stage_unit(c);
-            cp_async_wait_all();
-            __syncwarp();
-            xs = xst;
-            moe_step(sg, gw, a.W, cn);
-            // h rows of a down unit may be read only after that expert's wait
-            stage_next = cn.s < 2 && (cn.s == 0 || (c.s == 1 && cn.a == c.a));
-        }
-        auto after_first_load = [&]() {  // the stage is free: copy the next unit's rows into it
-            if constexpr (MS::kStaged) {
-                __syncwarp();
-                if (stage_next) stage_unit(cn);
-            }
-        };
-        if (c.s == 0)
-            moe_unit<FMT, MAXM, XBF16>(a, r, 0, c.a, c.g, ubuf, lane, acc8, acc, xs, after_first_load);
-        else
-            moe_unit<FMT, MAXM, false>(a, r, 1, c.a, c.g, ubuf, lane, acc8, acc, xs, after_first_load);
-        xready = stage_next;
-        __syncwarp();
-        if (lane == 0 && p.s < 2) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&bars[slot], C::UB);
-            bulk_g2s(ring + slot * C::UB, moe_unit_src<FMT>(a, r, p), C::UB, &bars[slot]);
-        }
-        if (p.s < 2) moe_step(sg, gw, a.W, p);
-        ++seq;
-        const int s_now = c.s, a_now = c.a, t = c.t;
-        moe_step(sg, gw, a.W, c);
-        if (c.s != s_now || c.a != a_now || c.t != t) {  // tile t of expert a_now ends here
-            if (kOnePass || r.nrows[a_now] <= 2) {  // the tile was accumulated in acc8
-                float rr[MP];
-                reduce_scatter8<MP>(acc8, lane, rr);
-#pragma unroll
-                for (int mm = 0; mm < MP; ++mm) acc[mm] = rr[mm];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int mm = 0; mm < MP; ++mm) acc8[i][mm] = 0.f;
-            }
-            const MoeSeg& S = sg[s_now];
-            const int f = a_now * S.Ue + t * S.G;  // the tile in segment units
-            if (f >= b && f + S.G <= e) {
-                moe_write_tile<MAXM>(a, r, s_now, a_now, t, lane, acc, gs);
-            } else {
-                const int v_first = moe_owner(S, f);
-                const int v = moe_owner(S, b > f ? b : f);
-                if (v > v_first) {
-                    moe_publish<MAXM>(a, s_now, v, 0, lane, acc, tag);  // first piece of range v
-                } else {  // range v ends in the tile and owns its first unit: finish it later
-                    moe_publish<MAXM>(a, s_now, v, 1, lane, acc, tag);
-                    pend_s = s_now;
-                    pend_a = a_now;
-                    pend_t = t;
-                    pend_v = v;
-                    pend_n = moe_owner(S, f + S.G - 1) - v_first + 1;
-                    pend_gs = gs;
+                const uint8_t* ubuf = ring + slot * C::UB;
+                const uint8_t* xs = nullptr;
+                MoeCursor cn = c;  // the next unit of this warp
+                bool stage_next = false;
+                if constexpr (MS::kStaged) {
+                    if (!xready) stage_unit(c);
+                    cp_async_wait_all();
+                    __syncwarp();
+                    xs = xst;
+                    moe_step(sg, tb, te, warp, cn);
+                    // h rows of a down unit may be read only after that entry's wait
+                    stage_next = cn.s < 2 && (cn.s == 0 || (c.s == 1 && cn.act == c.act));
                 }
+                auto after_first_load = [&]() {  // the stage is free: copy the next unit's rows into it
+                    if constexpr (MS::kStaged) {
+                        __syncwarp();
+                        if (stage_next) stage_unit(cn);
+                    }
+                };
+                if (s == 0)
+                    moe_unit<FMT, MAXM, XBF16>(a, r, 0, c.act, c.g, ubuf, lane, acc8, xs, after_first_load);
+                else
+                    moe_unit<FMT, MAXM, false>(a, r, 1, c.act, c.g, ubuf, lane, acc8, xs, after_first_load);
+                xready = stage_next;
+                __syncwarp();
+                // Refill this slot with the producer's next unit (the ring runs C::D units ahead).
+                if (lane == 0 && p.s < 2) {
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(&bars[slot], C::UB);
+                    bulk_g2s(ring + slot * C::UB, moe_unit_src<FMT>(a, r, sg, p), C::UB, &bars[slot]);
+                }
+                if (p.s < 2) moe_step(sg, tb, te, warp, p);
+                ++seq;
+                moe_step(sg, tb, te, warp, c);
             }
+            // The tile's parts: each warp's (zero if it had no unit of the tile), added in warp
+            // order by one warp (rotating) -- deterministic.
+            float rr[MP];
+            reduce_scatter8<MP>(acc8, lane, rr);
 #pragma unroll
-            for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
+            for (int mm = 0; mm < MP; ++mm) red[tc & 1][warp][lane][mm] = rr[mm];
+            __syncthreads();
+            if (warp == tc % kGemvWarps) {
+                float v[MP];
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) v[mm] = 0.f;
+#pragma unroll
+                for (int w = 0; w < kGemvWarps; ++w)
+#pragma unroll
+                    for (int mm = 0; mm < MP; ++mm) v[mm] += red[tc & 1][w][lane][mm];
+                moe_write_tile<MAXM>(a, r, s, act, t, lane, v, gs);
+            }
+            if (++t == T && jl + 1 < te[s] - tb[s]) {
+                t = 0;
+                ++act;
+                gs = moe_scale<FMT>(a, r, s, act);
+            }
         }
     }
-    if (!failed && pend_s >= 0 &&
-        !moe_flush<MAXM>(a, r, pend_s, pend_a, pend_t, pend_v, pend_n, lane, pend_gs, tag))
-        failed = true;
     if constexpr (MS::kStaged) cp_async_wait_all();  // no copy into this CTA's memory outlives it
     if (failed && lane == 0) {
         atomicOr(reinterpret_cast<unsigned int*>(a.ws), 1u);
         MoeCursor q = c;  // wait (bounded) for this warp's copies still in flight
         for (int s = 0; s < C::D && q.s < 2; ++s) {
             mbar_wait_bounded(&bars[(seq + s) % C::D], (uint32_t)(((seq + s) / C::D) & 1), 100000000ull);
-            moe_step(sg, gw, a.W, q);
+            moe_step(sg, tb, te, warp, q);
         }
     }
     __syncwarp();
-    // The last CTA to leave resets the tile counts and advances the launch counter.
+    // The last CTA to leave resets the tile counts.
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
         unsigned int* ex = reinterpret_cast<unsigned int*>(a.ws + kMoeExitOff);
         if (atomicAdd(ex, 1u) == gridDim.x - 1) {
             __threadfence();
-            unsigned int* done = reinterpret_cast<unsigned int*>(a.ws + kMoeDoneOff);
-            for (int j = 0; j < kMoeMaxAct; ++j) done[j] = 0u;
-            *reinterpret_cast<unsigned int*>(a.ws + kMoeEpochOff) = tag;
+            unsigned int* dn = reinterpret_cast<unsigned int*>(a.ws + kMoeDoneOff);
+            for (int j = 0; j < kMoeMaxAct; ++j) dn[j] = 0u;
             *ex = 0u;
         }
     }
@@ -731,7 +617,7 @@ static int moe_sm_count() {
 static int64_t al256(int64_t b) { return (b + 255) / 256 * 256; }
 
 struct MoePlan {
-    int grid, W;
+    int grid;
     int64_t o_off, h_off;
     size_t bytes;
 };
@@ -740,8 +626,7 @@ static MoePlan plan_moe(int fmt, int M, int64_t H, int64_t I, int top_k, bool ne
     MoePlan p;
     const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
     p.grid = moe_sm_count() * cps;
-    p.W = p.grid * kGemvWarps;
-    int64_t off = moe_part_off() + al256((int64_t)2 * p.W * 2 * 32 * M * 8);
+    int64_t off = al256(moe_head_bytes());
     p.o_off = off;
     off += al256(4 * (int64_t)M * top_k * H);
     p.h_off = off;
@@ -779,11 +664,11 @@ static cudaError_t moe_launch(const MoeArgs& a, int grid, cudaStream_t s, bool p
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+// Work entries hold at most kMoeEntryRows rows whatever M is.
 template <int FMT, bool XBF16>
 static cudaError_t moe_launch_m(const MoeArgs& a, int grid, cudaStream_t s, bool pdl) {
     if (a.M == 1) return moe_launch<FMT, 1, XBF16>(a, grid, s, pdl);
-    if (a.M == 2) return moe_launch<FMT, 2, XBF16>(a, grid, s, pdl);
-    return moe_launch<FMT, 8, XBF16>(a, grid, s, pdl);
+    return moe_launch<FMT, kMoeEntryRows, XBF16>(a, grid, s, pdl);
 }
 
 }  // namespace qlin
@@ -826,7 +711,6 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
     a.T1 = (int)g1.T;
     a.G1 = (int)g1.G;
     a.U1 = (int)g1.U;
-    a.W = p.W;
     const bool pdl = (flags & QLIN_FLAG_PDL) != 0, bf16 = xdt == QLIN_BF16;
     if (fmt == QLIN_Q4_0) return bf16 ? moe_launch_m<QLIN_Q4_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q4_0, false>(a, p.grid, s, pdl);
     if (fmt == QLIN_Q8_0) return bf16 ? moe_launch_m<QLIN_Q8_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q8_0, false>(a, p.grid, s, pdl);

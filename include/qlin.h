@@ -202,10 +202,11 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
  * Q4_0 MoE decode through "CUDA expert routing", LFM2.5-8B-A1B) and the imp README "Features"
  * table (MoE top-k grouped GEMM; an ordered, deterministic MoE reduction):
  *   route  : p = softmax(router_logits[m]); the top_k experts by p (a tie goes to the lower expert
- *            index); weights renormalised over the selected experts
+ *            index; a NaN logit ranks as -inf); weights renormalised over the selected experts
  *   experts: h = silu(W_gate[e] x) * (W_up[e] x);  o = W_down[e] h   (fp32, as qlin_gemv)
  *   output : y[m] = sum over slots in slot order of weight * o
- * Only the selected experts' weights are read, each once per call for all tokens routed to it.
+ * Only the selected experts' weights are read: once per call for every two tokens routed to the
+ * expert (an expert chosen by 3..8 tokens is streamed 2..4 times, the repeats mostly from L2).
  * Arguments:
  *   gate_up_packed: E consecutive buffers, each qlin_packed_bytes(fmt, 2I, H, QLIN_PACK_GATE_UP)
  *                   bytes, expert e packed from its [gate ; up] rows (2I x H)

@@ -93,8 +93,11 @@ def test_moe_formats_small(fmt, xdt, M):
     run_and_check(ex, M, 2, logits, x)
 
 
-def test_moe_all_experts_uniform_is_mean():
-    fmt, E, H, I, M = q.QLIN_Q4_0, 4, 256, 64, 2
+@pytest.mark.parametrize("M", [2, 8])
+def test_moe_all_experts_uniform_is_mean(M):
+    # equal logits: ties go to the lower expert index; with M = 8 every expert serves all 8
+    # tokens, four work entries of two rows each
+    fmt, E, H, I = q.QLIN_Q4_0, 4, 256, 64
     ex = Experts(fmt, E, H, I, 6000)
     x = synth.activations(M, H, synth.gen(6001))
     ids, w, y = run_and_check(ex, M, E, torch.zeros(M, E), x)

@@ -481,7 +481,7 @@ def run_config(name, args):
             del gu, dn
     elif name == "moe":
         fmt, E, H, I, k = q.QLIN_Q4_0, 32, 2048, 1792, 4
-        L = 2
+        L = 8  # 8 layers (1.6 GB): one replay's selected experts (>= 8 x 25 MB) exceed L2
         canon_gu = [[synth.weights(fmt, 2 * I, H, synth.gen(4000 + 100 * l + e, device="cuda"), device="cuda")
                      for e in range(E)] for l in range(L)]
         gu = [q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_GATE_UP) for c in canon_gu]
@@ -512,7 +512,8 @@ def run_config(name, args):
             nd = sum(distinct) / L
             bytes_ = nd * per_expert + M * (4 * H + 4 * H + 4 * E)
             lines.append(dict(workload="Q4_0 MoE expert layer shaped like an 8B-A1B model: hidden 2048, 32 experts "
-                              "gate_up 2048->2x1792, down 1792->2048, top-4", M=M, distinct_experts=nd,
+                              "gate_up 2048->2x1792, down 1792->2048, top-4; a graph of 8 layers' launches "
+                              "(distinct weights)", M=M, distinct_experts=nd,
                               us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9))
     if name == "chunk":
         fmt, N, K = q.QLIN_NVFP4, 17408, 5120

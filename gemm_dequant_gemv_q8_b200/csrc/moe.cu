@@ -490,12 +490,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
     bool xready = false;  // the current unit's rows are already staged
     auto stage_unit = [&](const MoeCursor& u) {
         const void* rows[MP];
-        if (u.s == 0) {
-            moe_rows<MP, XBF16>(a, r, 0, u.act, 0, rows);
-            stage_x_rows<XBF16, MP>(rows, a.H, u.g, xst, lane, a.ws);
+        if (!XBF16 || u.s == 1) {  // fp32 rows: x (step 0) or h (step 1)
+            moe_rows<MP, false>(a, r, u.s, u.act, 0, rows);
+            stage_x_rows<false, MP>(rows, u.s == 0 ? a.H : a.I, u.g, xst, lane, a.ws);
         } else {
-            moe_rows<MP, false>(a, r, 1, u.act, 0, rows);
-            stage_x_rows<false, MP>(rows, a.I, u.g, xst, lane, a.ws);
+            moe_rows<MP, true>(a, r, 0, u.act, 0, rows);
+            stage_x_rows<true, MP>(rows, a.H, u.g, xst, lane, a.ws);
         }
     };
     const unsigned int* done = reinterpret_cast<const unsigned int*>(a.ws + kMoeDoneOff);
@@ -538,8 +538,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
                         if (stage_next) stage_unit(cn);
                     }
                 };
-                if (s == 0)
-                    moe_unit<FMT, MAXM, XBF16>(a, r, 0, c.act, c.g, ubuf, lane, acc8, xs, after_first_load);
+                if constexpr (!XBF16)  // one copy of the unit code for both steps (instruction cache)
+                    moe_unit<FMT, MAXM, false>(a, r, s, c.act, c.g, ubuf, lane, acc8, xs, after_first_load);
+                else if (s == 0)
+                    moe_unit<FMT, MAXM, true>(a, r, 0, c.act, c.g, ubuf, lane, acc8, xs, after_first_load);
                 else
                     moe_unit<FMT, MAXM, false>(a, r, 1, c.act, c.g, ubuf, lane, acc8, xs, after_first_load);
                 xready = stage_next;

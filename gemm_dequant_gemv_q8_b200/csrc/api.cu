@@ -176,7 +176,6 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
     if (M < 1 || M > 8 || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, 2 * I, H) || !valid_shape(fmt, H, I)) return QLIN_ERR_INVALID_ARG;
     if (H > 32768) return QLIN_ERR_UNSUPPORTED;  // down tiles per expert are tracked per token
-    if (fmt == QLIN_MXFP4) return QLIN_ERR_UNSUPPORTED;  // the expert kernel is built for the other formats
     if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
     if (flags & ~QLIN_FLAG_PDL) return QLIN_ERR_INVALID_ARG;
     if (!gate_up_packed || !down_packed || !topk_ids || !topk_w || !x || !y) return QLIN_ERR_INVALID_ARG;

@@ -382,7 +382,7 @@ __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, i
     const int64_t k0 = (int64_t)g * kGroupK + part * 32;
     const void* rows[MP];
     moe_rows<MP, XB>(a, r, s, act, 0, rows);
-    if constexpr (XB && FMT == QLIN_NVFP4) {
+    if constexpr (XB && (FMT == QLIN_NVFP4 || FMT == QLIN_MXFP4)) {
         uint32_t xh[MP][16];
         float xsc[MP][2];
         if (xs != nullptr)
@@ -390,7 +390,7 @@ __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, i
         else
             load_x_fp4h<MP, true>(rows, k0, Kin, xh, xsc);
         after_first_load();
-        unit_dot_fp4h<MP, true>(ubuf, lane, xh, xsc, acc8);
+        unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
     } else {
         float2 xv[MP][16];
         float xb[MP];
@@ -716,5 +716,6 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
     const bool pdl = (flags & QLIN_FLAG_PDL) != 0, bf16 = xdt == QLIN_BF16;
     if (fmt == QLIN_Q4_0) return bf16 ? moe_launch_m<QLIN_Q4_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q4_0, false>(a, p.grid, s, pdl);
     if (fmt == QLIN_Q8_0) return bf16 ? moe_launch_m<QLIN_Q8_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q8_0, false>(a, p.grid, s, pdl);
+    if (fmt == QLIN_MXFP4) return bf16 ? moe_launch_m<QLIN_MXFP4, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_MXFP4, false>(a, p.grid, s, pdl);
     return bf16 ? moe_launch_m<QLIN_NVFP4, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_NVFP4, false>(a, p.grid, s, pdl);
 }

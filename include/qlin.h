@@ -218,7 +218,7 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
  *   x : M x H rows (fp32 or bf16), contiguous;  y : M x H fp32, contiguous
  *   h : optional M x top_k x I fp32 output of the SiLU-gated intermediate (NULL: kept in ws)
  *   flags: 0 or QLIN_FLAG_PDL;  ws: qlin_workspace_bytes(QLIN_OP_MOE, fmt, M, H, I, E, top_k)
- * E <= 256, top_k <= min(8, E), H <= 32768, fmt other than QLIN_MXFP4 (else QLIN_ERR_UNSUPPORTED).  One kernel launch on
+ * E <= 256, top_k <= min(8, E), H <= 32768 (else QLIN_ERR_UNSUPPORTED), any format.  One kernel launch on
  * `stream` (routing, gate_up of the selected experts, down, weighted sum), no host
  * synchronisation.  The status word (qlin_ws_status) reports a bad input expert id (the slot is
  * skipped) or a timed-out device wait. */

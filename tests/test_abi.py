@@ -136,9 +136,9 @@ def test_chain_workspace_bytes(lib):
     assert q.qlin_chain_workspace_bytes(q.QLIN_Q4_0, 1, [_chain_op(wait_for=0)]) == 0
 
 
-def test_moe_rejects_mxfp4_before_launch(lib):
+def test_moe_rejects_oversized_hidden_before_launch(lib):
     P = ctypes.c_void_p
-    st = lib.qlin_moe_experts(q.QLIN_MXFP4, P(0x100000), P(0x200000), 32, 2048, 1792, 4, P(0x300000),
+    st = lib.qlin_moe_experts(q.QLIN_MXFP4, P(0x100000), P(0x200000), 32, 32768 + 256, 1792, 4, P(0x300000),
                               P(0x400000), P(0x500000), P(0x600000), 1, 1, P(0x700000), None, 0,
                               P(0x800000), 1 << 30, None)
-    assert st == 2  # QLIN_ERR_UNSUPPORTED
+    assert st == 2  # QLIN_ERR_UNSUPPORTED: down tiles per expert are tracked for H <= 32768

@@ -84,7 +84,8 @@ def test_moe_q4_0_lfm2_shape(M):
 
 
 @pytest.mark.parametrize("fmt,xdt", [(q.QLIN_Q8_0, torch.float32), (q.QLIN_NVFP4, torch.bfloat16),
-                                     (q.QLIN_Q4_0, torch.bfloat16)])
+                                     (q.QLIN_Q4_0, torch.bfloat16), (q.QLIN_MXFP4, torch.bfloat16),
+                                     (q.QLIN_MXFP4, torch.float32)])
 @pytest.mark.parametrize("M", [1, 3, 8])
 def test_moe_formats_small(fmt, xdt, M):
     ex = Experts(fmt, 6, 256, 96, 5000 + fmt)

@@ -6,8 +6,8 @@ shares no code with it.  The arithmetic lives in ``oracle.c`` (plain C, fp64, se
 this module compiles it with gcc on first use and marshals numpy arrays.
 
 Every function cites what it follows; the format layouts are the public GGUF / NVFP4 / OCP MX
-conventions (the pages name the formats -- imp README, "Features" table; imp release notes v0.6,
-"Native MXFP4 GGUF weight format" -- but do not print their layout).
+conventions (the pages name the formats -- imp README, "Features" table, row "Quantization";
+imp release notes v0.6, "Native MXFP4 GGUF weight format" -- but do not print their layout).
 
 Parity pins for every function here live in ``tests/test_oracle_pins.py``.
 """
@@ -20,7 +20,7 @@ import threading
 
 import numpy as np
 
-Q8_0, Q4_0, NVFP4, MXFP4 = 1, 2, 3, 4
+Q8_0, Q4_0, NVFP4, MXFP4, Q4_K = 1, 2, 3, 4, 5
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")

@@ -14,6 +14,8 @@
  *   - imp README, "Features" table, row "Server": an ordered (deterministic) MoE reduction.
  *   - imp release notes, v0.6 "Native MXFP4 GGUF weight format": E2M1 codes with UE8M0 block
  *     scales, 4.25 bits per weight (one 8-bit scale per 32 values).
+ *   - imp README, "Features" table, row "Quantization": GGUF K-quants (Q4_K_M and others) among
+ *     the weight formats.
  * The pages name the formats but never print their byte layout.  The layouts used here are the
  * public conventions (GGUF block_q8_0 / block_q4_0; NVFP4 = E2M1 codes, one E4M3 scale per 16
  * values, one FP32 per-tensor scale), the plainest reading the pages support.
@@ -26,7 +28,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { QO_Q8_0 = 1, QO_Q4_0 = 2, QO_NVFP4 = 3, QO_MXFP4 = 4 };
+enum { QO_Q8_0 = 1, QO_Q4_0 = 2, QO_NVFP4 = 3, QO_MXFP4 = 4, QO_Q4_K = 5 };
 
 /* ---------------------------------------------------------------- scalar decoders */
 
@@ -77,7 +79,23 @@ int64_t qo_row_bytes(int fmt, int64_t K) {
     if (fmt == QO_Q8_0) return (K / 32) * 34;
     if (fmt == QO_Q4_0) return (K / 32) * 18;
     if (fmt == QO_NVFP4 || fmt == QO_MXFP4) return K / 2;
+    if (fmt == QO_Q4_K) return (K / 256) * 144;
     return -1;
+}
+
+/* GGUF Q4_K super-block (256 values, 144 bytes): fp16 d, fp16 dmin, 12 bytes holding eight 6-bit
+ * scales and eight 6-bit mins (one pair per 32-value sub-block), 128 bytes of 4-bit codes.
+ * Sub-blocks 0..3 keep their scale and min in the low 6 bits of bytes 0..3 and 4..7; sub-blocks
+ * 4..7 keep the low 4 bits of each in byte 8..11 (scale low nibble, min high nibble) and the top
+ * 2 bits in the spare high bits of bytes 0..3 (scale) and 4..7 (min) of sub-block j - 4. */
+void qo_q4k_scale_min(const uint8_t* sc12, int j, int* sc, int* m) {
+    if (j < 4) {
+        *sc = sc12[j] & 63;
+        *m = sc12[j + 4] & 63;
+    } else {
+        *sc = (sc12[j + 4] & 0xf) | ((sc12[j - 4] >> 6) << 4);
+        *m = (sc12[j + 4] >> 4) | ((sc12[j] >> 6) << 4);
+    }
 }
 
 /* Dequantize row n of a canonical tensor into w[0..K) (fp64, exact real value).
@@ -86,7 +104,11 @@ int64_t qo_row_bytes(int fmt, int64_t K) {
  *                                                   element j+16 its high nibble; w = d * (nib - 8)
  *   NVFP4: codes [N][K/2], byte i = elements 2i (low nibble) and 2i+1 (high nibble);
  *          scales [N][K/16] E4M3; w = e2m1(code) * e4m3(scale of k/16) * g
- *   MXFP4: codes as NVFP4; scales [N][K/32] UE8M0; w = e2m1(code) * 2^(scale of k/32 - 127) */
+ *   MXFP4: codes as NVFP4; scales [N][K/32] UE8M0; w = e2m1(code) * 2^(scale of k/32 - 127)
+ *   Q4_K super-block (144 B per 256 values, see qo_q4k_scale_min): the codes of the 64 values
+ *          64c .. 64c+63 are bytes 32c .. 32c+31 of the code area, values 64c + l in the low
+ *          nibble of byte l, 64c + 32 + l in its high nibble; value k of sub-block j = k / 32:
+ *          w = d * scale_j * code - dmin * min_j */
 static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t* scales, float g,
                         int64_t n, double* w) {
     if (fmt == QO_Q8_0 || fmt == QO_Q4_0) {
@@ -112,6 +134,22 @@ static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t
             uint8_t c = (k & 1) ? (byte >> 4) : (byte & 0xf);
             w[k] = qo_e2m1(c) * qo_e4m3(srow[k / 16]) * (double)g;
         }
+    } else if (fmt == QO_Q4_K) {
+        const uint8_t* row = blocks + n * (K / 256) * 144;
+        for (int64_t b = 0; b < K / 256; ++b) {
+            const uint8_t* blk = row + b * 144;
+            double d = qo_fp16((uint16_t)(blk[0] | (blk[1] << 8)));
+            double dmin = qo_fp16((uint16_t)(blk[2] | (blk[3] << 8)));
+            const uint8_t* sc12 = blk + 4;
+            const uint8_t* qs = blk + 16;
+            for (int k = 0; k < 256; ++k) {
+                int sc, m;
+                qo_q4k_scale_min(sc12, k / 32, &sc, &m);
+                int c = k / 64, l = k % 32;
+                int code = (k % 64) < 32 ? (qs[32 * c + l] & 0xf) : (qs[32 * c + l] >> 4);
+                w[b * 256 + k] = d * sc * code - dmin * m;
+            }
+        }
     } else {
         const uint8_t* row = blocks + n * (K / 2);
         const uint8_t* srow = scales + n * (K / 32);
@@ -123,8 +161,9 @@ static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t
     }
 }
 
-/* Values per block along K (scale granularity): 16 for NVFP4, 32 otherwise. */
-static int64_t qo_block_k(int fmt) { return fmt == QO_NVFP4 ? 16 : 32; }
+/* Values per block along K (the granularity K must respect): 16 for NVFP4, 256 for Q4_K's
+ * super-blocks, 32 otherwise. */
+static int64_t qo_block_k(int fmt) { return fmt == QO_NVFP4 ? 16 : fmt == QO_Q4_K ? 256 : 32; }
 
 /* Full-tensor dequantization to fp64.  Returns 0, or -1 on a bad argument. */
 int qo_dequant(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
@@ -136,7 +175,8 @@ int qo_dequant(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8
 
 /* The fp32 value of each weight ("bit-exact dequant").  For Q8_0 / Q4_0 and for the NVFP4
  * product e2m1*e4m3 the fp64 value is exactly representable in fp32; the NVFP4 per-tensor
- * scale g is the one rounding: w32 = fp32( (e2m1*e4m3) * g ), rounded once to nearest-even. */
+ * scale g is the one rounding: w32 = fp32( (e2m1*e4m3) * g ), rounded once to nearest-even.
+ * Q4_K: both products d*scale*code and dmin*min are exact; their difference is rounded once. */
 int qo_dequant_f32(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
                    float g, float* W) {
     if (qo_row_bytes(fmt, K) < 0 || K % qo_block_k(fmt)) return -1;

@@ -12,6 +12,8 @@ Canonical layouts (the public conventions; the pages name the formats but not th
   NVFP4 codes [N][K/2] (byte i = element 2i low nibble, 2i+1 high nibble), E4M3 scales [N][K/16],
         one fp32 per-tensor scale
   MXFP4 codes as NVFP4, UE8M0 scale bytes [N][K/32] (one per 32 values), no per-tensor scale
+  Q4_K  one row = K/256 super-blocks of 144 bytes: fp16 d, fp16 dmin, 12 bytes of packed 6-bit
+        sub-block scales and mins, 128 bytes of 4-bit codes (GGUF block_q4_K)
 
 Workload recipes (seeded; shapes from the synthetic layer stacks the bench and tests use):
   Q8_0:  codes uniform over [-127, 127], scale uniform real in [1e-3, 1e-2] rounded to fp16
@@ -19,14 +21,17 @@ Workload recipes (seeded; shapes from the synthetic layer stacks the bench and t
   NVFP4: codes uniform over all 16, E4M3 scales uniform real in [0.5, 448] rounded to E4M3,
          per-tensor scale fp32(1/448)
   MXFP4: codes uniform over all 16, scale bytes uniform integers in [118, 130] (2^-9 .. 2^3)
+  Q4_K:  d and dmin uniform real in [2e-4, 2e-3] rounded to fp16; the 12 scale bytes and the
+         128 code bytes uniform over 0..255 (every byte pattern is a valid encoding: sub-block
+         scales and mins uniform over 0..63, codes uniform over 0..15)
   activations N(0, 1) (fp32, or fp32 draws rounded to bf16); router logits N(0, 1)
 """
 from __future__ import annotations
 
 import torch
 
-Q8_0, Q4_0, NVFP4, MXFP4 = 1, 2, 3, 4
-FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4", MXFP4: "mxfp4"}
+Q8_0, Q4_0, NVFP4, MXFP4, Q4_K = 1, 2, 3, 4, 5
+FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4", MXFP4: "mxfp4", Q4_K: "q4_k"}
 NVFP4_G = float(torch.tensor(1.0 / 448.0, dtype=torch.float32))
 
 
@@ -65,6 +70,15 @@ def q4_0(N, K, g, device="cpu", d_range=(1e-3, 2e-2)):
     return torch.cat([_fp16_bytes(d), qs], dim=2).reshape(N, nb * 18).contiguous()
 
 
+def q4_k(N, K, g, device="cpu", d_range=(2e-4, 2e-3)):
+    """Canonical Q4_K tensor, uint8 [N, K/256*144]."""
+    assert K % 256 == 0
+    nb = K // 256
+    d = torch.empty(N, nb, 2, dtype=torch.float32, device=device).uniform_(*d_range, generator=g)
+    rest = torch.randint(0, 256, (N, nb, 140), generator=g, device=device, dtype=torch.int16).to(torch.uint8)
+    return torch.cat([_fp16_bytes(d).reshape(N, nb, 4), rest], dim=2).reshape(N, nb * 144).contiguous()
+
+
 def nvfp4(N, K, g, device="cpu", s_range=(0.5, 448.0)):
     """Canonical NVFP4 tensor: (codes uint8 [N, K/2], scales uint8 [N, K/16], fp32 tensor scale)."""
     assert K % 16 == 0
@@ -96,6 +110,8 @@ def weights(fmt, N, K, g, device="cpu"):
         return mxfp4(N, K, g, device=device)
     if fmt == NVFP4:
         return nvfp4(N, K, g, device)
+    if fmt == Q4_K:
+        return q4_k(N, K, g, device), None, 1.0
     raise ValueError(fmt)
 
 

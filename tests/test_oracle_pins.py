@@ -178,6 +178,104 @@ def _identity_nvfp4(K):
     return codes, np.full((K, K // 16), 0x38, np.uint8)
 
 
+# ----------------------------------------------------------------------------- Q4_K
+def _q4k_block(d_bits, dmin_bits, sc, m, codes):
+    """One GGUF Q4_K super-block packed from its fields, written here from the block_q4_K
+    definition in the packing direction (the oracle only unpacks): 6-bit scales and mins of
+    sub-blocks 0..3 in the low bits of bytes 0..3 / 4..7, the low 4 bits of those of sub-blocks
+    4..7 in the nibbles of bytes 8..11, their top 2 bits in bits 6..7 of bytes 0..3 / 4..7; code k
+    (c = k / 64, l = k % 32) in the low nibble of qs[32c + l] for k % 64 < 32, else the high one."""
+    head = bytearray(struct.pack("<HH", d_bits, dmin_bits))
+    s12 = bytearray(12)
+    for j in range(8):
+        if j < 4:
+            s12[j] |= sc[j]
+            s12[j + 4] |= m[j]
+        else:
+            s12[j + 4] |= (sc[j] & 15) | ((m[j] & 15) << 4)
+            s12[j - 4] |= (sc[j] >> 4) << 6
+            s12[j] |= (m[j] >> 4) << 6
+    qs = bytearray(128)
+    for k in range(256):
+        c, l = k // 64, k % 32
+        qs[32 * c + l] |= codes[k] if k % 64 < 32 else codes[k] << 4
+    return bytes(head + s12 + qs)
+
+
+def test_q4k_dequant_matches_golden():
+    lines = read_golden("q4k_block.txt")
+    blk = bytearray(int(t, 16) for t in lines[0].split()[1:])
+    qs = bytearray(128)
+    for t in lines[1].split()[1:]:
+        i, v = t.split(":")
+        qs[int(i)] = int(v, 16)
+    w = oracle.dequant(oracle.Q4_K, 1, 256, np.frombuffer(bytes(blk + qs), np.uint8)[None, :])[0]
+    for t in lines[2].split()[1:]:
+        k, v = t.split(":")
+        assert w[int(k)] == float(v), (k, w[int(k)], v)
+
+
+def test_q4k_packed_fields_decode_exactly():
+    # Every 6-bit scale and min value in every sub-block position, random codes, fp16 d / dmin
+    # drawn by numpy: the oracle must return d * sc * code - dmin * m exactly (fp64 holds it).
+    rng = np.random.default_rng(7)
+    for rep in range(64):
+        sc = [int(v) for v in (np.arange(8) * 8 + rep) % 64]
+        m = [int(v) for v in (63 - np.arange(8) * 8 - rep) % 64]
+        codes = [int(v) for v in rng.integers(0, 16, 256)]
+        d16, dm16 = np.float16(rng.uniform(1e-3, 2.0)), np.float16(rng.uniform(1e-3, 2.0))
+        blk = _q4k_block(int(d16.view(np.uint16)), int(dm16.view(np.uint16)), sc, m, codes)
+        w = oracle.dequant(oracle.Q4_K, 1, 256, np.frombuffer(blk, np.uint8)[None, :])[0]
+        ref = [Fraction(float(d16)) * sc[k // 32] * codes[k] - Fraction(float(dm16)) * m[k // 32] for k in range(256)]
+        assert all(Fraction(w[k]) == ref[k] for k in range(256)), rep
+
+
+def test_q4k_rows_of_several_superblocks_and_identity():
+    # Identity through Q4_K: d = 1, dmin = 0, every sub-block scale 1 and min 0, code 1 at k = n.
+    K = 512
+    rows = []
+    for n in range(K):
+        codes = [0] * K
+        codes[n] = 1
+        rows.append(b"".join(_q4k_block(0x3C00, 0, [1] * 8, [0] * 8, codes[256 * b:256 * (b + 1)])
+                             for b in range(K // 256)))
+    blocks = np.frombuffer(b"".join(rows), np.uint8).reshape(K, -1)
+    assert blocks.shape[1] == oracle.row_bytes(oracle.Q4_K, K) == 288
+    x = synth.activations(2, K, synth.gen(21)).double().numpy()
+    y, A = oracle.gemv(oracle.Q4_K, K, K, blocks, x)
+    assert np.array_equal(y, x) and np.array_equal(A, np.abs(x))
+
+
+def test_q4k_gemv_matches_exact_rational_sum_and_one_hot():
+    N, K, M = 6, 512, 2
+    blocks, _, _ = synth.weights(oracle.Q4_K, N, K, synth.gen(22))
+    blocks = blocks.numpy()
+    W = oracle.dequant(oracle.Q4_K, N, K, blocks)
+    x = synth.activations(M, K, synth.gen(23)).double().numpy()
+    y, A = oracle.gemv(oracle.Q4_K, N, K, blocks, x)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(W[n, k]) * Fraction(x[m, k]) for k in range(K))
+            absum = sum(abs(Fraction(W[n, k]) * Fraction(x[m, k])) for k in range(K))
+            assert abs(Fraction(y[m, n]) - exact) <= Fraction(K * 2.0 ** -52) * absum
+    for k in (0, 31, 32, 255, 256, 300, 511):
+        e = np.zeros((1, K))
+        e[0, k] = 1.0
+        assert np.array_equal(oracle.gemv(oracle.Q4_K, N, K, blocks, e)[0][0], W[:, k])
+
+
+def test_q4k_f32_value_is_one_rounding_of_the_exact_difference():
+    # d = 1, scale 63, code 15: 945; dmin = 2^-24 (fp16 0x0001), min 1: w = 945 - 2^-24, which fp32
+    # rounds (to nearest even) to 945; a min of 0 leaves 945 exactly.
+    codes = [15] * 256
+    blk = _q4k_block(0x3C00, 0x0001, [63] * 8, [1] * 8, codes)
+    a = np.frombuffer(blk, np.uint8)[None, :]
+    w = oracle.dequant(oracle.Q4_K, 1, 256, a)[0]
+    assert Fraction(w[0]) == 945 - Fraction(1, 2 ** 24)
+    w32 = oracle.dequant_f32(oracle.Q4_K, 1, 256, a)[0]
+    assert w32[0] == np.float32(945.0) and np.float32(945.0 - 2.0 ** -24) == np.float32(945.0)
+
+
 def _identity_mxfp4(K):
     codes, _ = _identity_nvfp4(K)
     return codes, np.full((K, K // 32), 0x7F, np.uint8)  # UE8M0 2^0

@@ -694,6 +694,7 @@ extern "C" cudaError_t qlin_launch_chain(int fmt, int xdt, int M, const qlin_gem
     if (fmt == QLIN_Q4_0) e = bf16 ? chain_launch_m<QLIN_Q4_0, true>(a, grid, s, pdl) : chain_launch_m<QLIN_Q4_0, false>(a, grid, s, pdl);
     else if (fmt == QLIN_Q8_0) e = bf16 ? chain_launch_m<QLIN_Q8_0, true>(a, grid, s, pdl) : chain_launch_m<QLIN_Q8_0, false>(a, grid, s, pdl);
     else if (fmt == QLIN_MXFP4) e = bf16 ? chain_launch_m<QLIN_MXFP4, true>(a, grid, s, pdl) : chain_launch_m<QLIN_MXFP4, false>(a, grid, s, pdl);
+    else if (fmt == QLIN_Q4_K) e = bf16 ? chain_launch_m<QLIN_Q4_K, true>(a, grid, s, pdl) : chain_launch_m<QLIN_Q4_K, false>(a, grid, s, pdl);
     else e = bf16 ? chain_launch_m<QLIN_NVFP4, true>(a, grid, s, pdl) : chain_launch_m<QLIN_NVFP4, false>(a, grid, s, pdl);
     delete a;
     return e;

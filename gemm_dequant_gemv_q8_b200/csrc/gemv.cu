@@ -415,6 +415,7 @@ extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, 
     if (fmt == QLIN_Q4_0) return launch_fmt<QLIN_Q4_0>(a, bf16, epi, p.grid, s, pdl);
     if (fmt == QLIN_Q8_0) return launch_fmt<QLIN_Q8_0>(a, bf16, epi, p.grid, s, pdl);
     if (fmt == QLIN_MXFP4) return launch_fmt<QLIN_MXFP4>(a, bf16, epi, p.grid, s, pdl);
+    if (fmt == QLIN_Q4_K) return launch_fmt<QLIN_Q4_K>(a, bf16, epi, p.grid, s, pdl);
     return launch_fmt<QLIN_NVFP4>(a, bf16, epi, p.grid, s, pdl);
 }
 
@@ -452,9 +453,10 @@ static cudaError_t noalloc_scratch(void** out) {
 extern "C" qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
                                            const void* x, qlin_dtype_t xdt, int M, int64_t ldx, float* y,
                                            int64_t ldy, int flags, qlin_stream_t stream) {
-    if (fmt != QLIN_Q8_0 && fmt != QLIN_Q4_0 && fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4) return QLIN_ERR_INVALID_ARG;
+    if (fmt != QLIN_Q8_0 && fmt != QLIN_Q4_0 && fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4 && fmt != QLIN_Q4_K)
+        return QLIN_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || N > ((int64_t)1 << 31) || K > ((int64_t)1 << 31)) return QLIN_ERR_INVALID_ARG;
-    if (fmt == QLIN_NVFP4 ? (K % 16) : (K % 32)) return QLIN_ERR_INVALID_ARG;
+    if (fmt == QLIN_NVFP4 ? (K % 16) : fmt == QLIN_Q4_K ? (K % 256) : (K % 32)) return QLIN_ERR_INVALID_ARG;
     if (M < 1 || M > 8) return QLIN_ERR_INVALID_ARG;
     if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
     const int epi = flags & 0xff;

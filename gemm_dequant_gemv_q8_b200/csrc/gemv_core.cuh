@@ -23,7 +23,9 @@ struct RingCfg {
 // the first binade).  So a nibble or byte masked in place at bit 4j (8j), with nothing else set,
 // IS the float n * 2^(4j) * 2^-149: one AND per weight, no shift, no subtraction.  Codes are
 // unsigned (Q4_0 nibble n = q + 8, Q8_0 byte = q + 128); the offset is removed once per block
-// from a sum of the activations taken in the same order (see prep_x_q4 / prep_x_q8).
+// from a sum of the activations taken in the same order (see prep_x_q4 / prep_x_q8).  Q4_K
+// codes (0..15, placed as Q4_0's) go through the same decoder; their sub-block min multiplies
+// that activation sum instead of an offset.
 // Activations are pre-scaled by 2^(kXExp - 4j) (2^(kXExp - 8j) for Q8_0), so every product is
 // the exact n * x * 2^(kXExp - 149) computed inside an fp32 FMA; block sums carry 2^(kXExp - 149)
 // and the tile output multiplies by kDenormUnscale = 2^(149 - kXExp).  Products stay normal and
@@ -33,7 +35,7 @@ constexpr int kXExp = 63;
 constexpr float kDenormUnscale = 0x1p86f;  // 2^(149 - kXExp)
 
 // Output scale of a format's block sums: the NVFP4 per-tensor scale, 1 for MXFP4 (its block
-// scales are applied in full per block), or 2^86 for Q4_0 / Q8_0.
+// scales are applied in full per block), or 2^86 for Q4_0 / Q8_0 / Q4_K.
 template <int FMT>
 __device__ __forceinline__ float format_out_scale(const uint8_t* packed) {
     if (FMT == QLIN_NVFP4) return reinterpret_cast<const PackedHeader*>(packed)->global_scale;
@@ -85,9 +87,10 @@ __device__ __forceinline__ float offset_sum(const float2 (&x)[16]) {
 
 // Prepare a lane's 32 activations for the Q4_0 decoder: the offset term 8 * sum (scaled), then
 // element e (pair e/2) times 2^(kXExp - 4 j) with j the decoder's position of element e mod 8.
-template <int MP>
+// Q4_K (same code positions, no offset): xb = sum * 2^(kXExp - 149), the min term's factor.
+template <int MP, bool K4 = false>
 __device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float (&xb)[MP]) {
-    constexpr float c = 0x1p-83f;  // 8 * 2^(kXExp - 149)
+    constexpr float c = K4 ? 0x1p-86f : 0x1p-83f;  // (1 or 8) * 2^(kXExp - 149)
     const float2 s0 = make_float2(0x1p63f, 0x1p59f), s1 = make_float2(0x1p55f, 0x1p51f);
     const float2 s2 = make_float2(0x1p47f, 0x1p43f);
 #pragma unroll
@@ -117,6 +120,7 @@ __device__ __forceinline__ void prep_x_q8(float2 (&xv)[MP][16], float (&xb)[MP])
 template <int FMT, int MP>
 __device__ __forceinline__ void prep_x(float2 (&xv)[MP][16], float (&xb)[MP]) {
     if (FMT == QLIN_Q4_0) prep_x_q4<MP>(xv, xb);
+    else if (FMT == QLIN_Q4_K) prep_x_q4<MP, true>(xv, xb);
     else if (FMT == QLIN_Q8_0) prep_x_q8<MP>(xv, xb);
     else {
 #pragma unroll
@@ -411,11 +415,18 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
         const uint4 sv = lds128(ub + code_bytes(FMT) + lane * 16);
         sw[0] = sv.x, sw[1] = sv.y, sw[2] = sv.z, sw[3] = sv.w;
     }
+    uint32_t dmw[FMT == QLIN_Q4_K ? 8 : 1];  // Q4_K: {d, dmin} of the lane's 8 rows
+    if (FMT == QLIN_Q4_K) {
+        const uint4 d0 = lds128(ub + kQ4kDmOff + (lane >> 3) * 32), d1 = lds128(ub + kQ4kDmOff + (lane >> 3) * 32 + 16);
+        const uint32_t t[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+        for (int i = 0; i < (FMT == QLIN_Q4_K ? 8 : 1); ++i) dmw[i] = t[i];
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         // 16 bits of scale for (row, part); MXFP4: 8 bits
         const uint32_t sc = FMT == QLIN_MXFP4 ? (sw[i >> 2] >> (8 * (i & 3))) : (sw[i >> 1] >> (16 * (i & 1)));
-        if (FMT == QLIN_Q4_0) {
+        if (FMT == QLIN_Q4_0 || FMT == QLIN_Q4_K) {
             const uint4 c = lds128(ub + (lane + 32 * i) * 16);
             const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
             float2 s0[MP], s1[MP];
@@ -437,12 +448,23 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
                     }
                 }
             }
-            const float d = fp16_bits_to_f32(sc & 0xffffu);
+            if (FMT == QLIN_Q4_K) {  // d * scale * sum(code x) - dmin * min * sum(x), both factors exact
+                const float2 dd = __half22float2(*reinterpret_cast<const __half2*>(&dmw[FMT == QLIN_Q4_K ? i : 0]));
+                const float ka = dd.x * (float)(sc & 63u), kb = dd.y * (float)((sc >> 6) & 63u);
 #pragma unroll
-            for (int mm = 0; mm < MP; ++mm) {
-                const float2 u = __fadd2_rn(s0[mm], s1[mm]);
-                const float bsum = (u.x + u.y) - xb[mm];
-                res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
+                for (int mm = 0; mm < MP; ++mm) {
+                    const float2 u = __fadd2_rn(s0[mm], s1[mm]);
+                    const float base = ACC ? fmaf(-kb, xb[mm], res[i][mm]) : -kb * xb[mm];
+                    res[i][mm] = fmaf(ka, u.x + u.y, base);
+                }
+            } else {
+                const float d = fp16_bits_to_f32(sc & 0xffffu);
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) {
+                    const float2 u = __fadd2_rn(s0[mm], s1[mm]);
+                    const float bsum = (u.x + u.y) - xb[mm];
+                    res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
+                }
             }
         } else if (FMT == QLIN_Q8_0) {
             const uint4 c0 = lds128(ub + (lane + 32 * i) * 16);

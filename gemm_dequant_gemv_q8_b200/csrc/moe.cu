@@ -717,5 +717,6 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
     if (fmt == QLIN_Q4_0) return bf16 ? moe_launch_m<QLIN_Q4_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q4_0, false>(a, p.grid, s, pdl);
     if (fmt == QLIN_Q8_0) return bf16 ? moe_launch_m<QLIN_Q8_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q8_0, false>(a, p.grid, s, pdl);
     if (fmt == QLIN_MXFP4) return bf16 ? moe_launch_m<QLIN_MXFP4, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_MXFP4, false>(a, p.grid, s, pdl);
+    if (fmt == QLIN_Q4_K) return bf16 ? moe_launch_m<QLIN_Q4_K, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q4_K, false>(a, p.grid, s, pdl);
     return bf16 ? moe_launch_m<QLIN_NVFP4, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_NVFP4, false>(a, p.grid, s, pdl);
 }

@@ -71,6 +71,41 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ b
         *reinterpret_cast<uint4*>(ub + 4096 + (r * 8 + p) * 16) = v1;
         sc[0] = (uint8_t)(d & 0xff);
         sc[1] = (uint8_t)(d >> 8);
+    } else if (FMT == QLIN_Q4_K) {
+        // GGUF Q4_K super-block (144 B per 256 values = one k-group): fp16 d, fp16 dmin, 12 bytes
+        // of packed 6-bit sub-block scales and mins, 128 bytes of codes (values 64c + l in the
+        // low nibble of byte 32c + l, values 64c + 32 + l in its high nibble).  Part p is
+        // sub-block p; its codes move to the 4-bit part order, its scale and min to the slot.
+        uint8_t out[16];
+        uint16_t scm = 0;
+        uint32_t dm = 0;
+        for (int j = 0; j < 16; ++j) out[j] = 0;
+        if (n >= 0) {
+            const uint8_t* blk = blocks + n * (K / 256) * 144 + g * 144;
+            const uint8_t* s12 = blk + 4;
+            const uint8_t* qs = blk + 16 + 32 * (p >> 1);
+            for (int j = 0; j < 16; ++j) {
+                const uint8_t lo = (p & 1) ? (qs[2 * j] >> 4) : (qs[2 * j] & 0xf);
+                const uint8_t hi = (p & 1) ? (qs[2 * j + 1] >> 4) : (qs[2 * j + 1] & 0xf);
+                out[j] = (uint8_t)(lo | (hi << 4));
+            }
+            int scv, mv;
+            if (p < 4) {
+                scv = s12[p] & 63;
+                mv = s12[p + 4] & 63;
+            } else {
+                scv = (s12[p + 4] & 0xf) | ((s12[p - 4] >> 6) << 4);
+                mv = (s12[p + 4] >> 4) | ((s12[p] >> 6) << 4);
+            }
+            scm = (uint16_t)(scv | (mv << 6));
+            dm = (uint32_t)blk[0] | ((uint32_t)blk[1] << 8) | ((uint32_t)blk[2] << 16) | ((uint32_t)blk[3] << 24);
+        }
+        uint4 v;
+        memcpy(&v, out, 16);
+        *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v;
+        sc[0] = (uint8_t)(scm & 0xff);
+        sc[1] = (uint8_t)(scm >> 8);
+        if (p == 0) *reinterpret_cast<uint32_t*>(ub + kQ4kDmOff + ((r & 3) * 8 + (r >> 2)) * 4) = dm;
     } else if (FMT == QLIN_MXFP4) {  // codes as NVFP4, one UE8M0 scale per part
         uint8_t out[16];
         uint8_t s = 0;
@@ -151,6 +186,16 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
             int b = (e < 16 ? cv[e] : cv[4096 + e - 16]);
             out[e] = d * (float)(b - 128);
         }
+    } else if (FMT == QLIN_Q4_K) {
+        // w = d * scale * code - dmin * min: both products exact in fp32, one rounding
+        const uint32_t dm = *reinterpret_cast<const uint32_t*>(ub + kQ4kDmOff + ((r & 3) * 8 + (r >> 2)) * 4);
+        const int scm = sc[0] | (sc[1] << 8);
+        const float a = fp16_bits_to_f32(dm & 0xffffu) * (float)(scm & 63);
+        const float b = fp16_bits_to_f32(dm >> 16) * (float)((scm >> 6) & 63);
+        for (int e = 0; e < 32; ++e) {
+            const int nib = (cv[e / 2] >> (4 * (e & 1))) & 0xf;
+            out[e] = __fmaf_rn(a, (float)nib, -b);
+        }
     } else if (FMT == QLIN_MXFP4) {
         const float s = e8m0_to_f32(sc[0]);
         for (int e = 0; e < valid; ++e) {
@@ -197,6 +242,9 @@ extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void*
     else if (fmt == QLIN_MXFP4)
         pack_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>((const uint8_t*)blocks, (const uint8_t*)scales,
                                                       N, K, gu, (uint8_t*)packed, geo.G);
+    else if (fmt == QLIN_Q4_K)
+        pack_kernel<QLIN_Q4_K><<<grid, 256, 0, s>>>((const uint8_t*)blocks, nullptr, N, K, gu,
+                                                     (uint8_t*)packed, geo.G);
     else
         pack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)blocks, (const uint8_t*)scales,
                                                       N, K, gu, (uint8_t*)packed, geo.G);
@@ -214,6 +262,8 @@ extern "C" cudaError_t qlin_launch_unpack(int fmt, const void* packed, int64_t N
         unpack_kernel<QLIN_Q8_0><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     else if (fmt == QLIN_MXFP4)
         unpack_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
+    else if (fmt == QLIN_Q4_K)
+        unpack_kernel<QLIN_Q4_K><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     else
         unpack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     return cudaGetLastError();

@@ -20,10 +20,15 @@ namespace qlin {
 //   scales: 32 lanes x 16 B.  Lane l = (r % 4) * 8 + p holds, in slot i = r / 4, the scale(s) of
 //           (row r, part p): one fp16 d (Q8_0 / Q4_0) or two E4M3 bytes (NVFP4, one per 16).
 //           MXFP4: 32 lanes x 8 B, one UE8M0 byte per (row, part) in slot i.
+//           Q4_K: as Q4_0, the 16-bit slot holding (row r, part p)'s 6-bit sub-block scale in
+//           bits 0..5 and 6-bit min in bits 6..11; then 32 x 4 B of per-row super-block scales
+//           {fp16 d, fp16 dmin}, row r at entry (r % 4) * 8 + r / 4, so lane l reads the 8 rows
+//           it works on as 32 contiguous bytes at entry (l / 8) * 8.
 // A warp reading vector (lane + 32 * i) in step i therefore touches 512 contiguous bytes, and
 // lane l always works on part l % 8 of rows l / 8 + 4 i (i = 0..7).
 // Element order inside a part:
-//   4-bit: element e in byte e / 2, low nibble for even e (word k holds elements 8k .. 8k+7)
+//   4-bit: element e in byte e / 2, low nibble for even e (word k holds elements 8k .. 8k+7);
+//          Q4_0 and Q4_K codes are stored as they are (0..15)
 //   Q8_0 : element e in byte e of the 32-byte part (plane e / 16), stored as q + 128
 // QLIN_PACK_GATE_UP tiles: rows 0..15 = gate rows 16 t + r, rows 16..31 = up rows N/2 + 16 t + r.
 constexpr int kHdrBytes = 256;
@@ -47,7 +52,10 @@ struct PackedHeader {
 static_assert(sizeof(PackedHeader) == kHdrBytes, "header size");
 
 __host__ __device__ constexpr int code_bytes(int fmt) { return fmt == QLIN_Q8_0 ? 8192 : 4096; }
-__host__ __device__ constexpr int unit_bytes(int fmt) { return code_bytes(fmt) + (fmt == QLIN_MXFP4 ? 256 : 512); }
+__host__ __device__ constexpr int unit_bytes(int fmt) {
+    return code_bytes(fmt) + (fmt == QLIN_MXFP4 ? 256 : fmt == QLIN_Q4_K ? 640 : 512);
+}
+constexpr int kQ4kDmOff = 4096 + 512;  // Q4_K: per-row {d, dmin} after the sub-block slots
 
 struct Geometry {
     int64_t T, G, U;  // tiles, k-groups, units

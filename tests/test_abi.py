@@ -53,6 +53,10 @@ def test_packed_bytes_sizes(lib):
     # MXFP4: codes as NVFP4, one scale byte per 32 values: 4096 + 256 bytes per 32 x 256 unit
     assert q.qlin_packed_bytes(q.QLIN_MXFP4, 4096, 2560) == 256 + 4096 * 2560 * 17 // 32
     assert q.qlin_packed_bytes(q.QLIN_MXFP4, 64, 272) == 0  # K % 32
+    # Q4_K: 4096 B of codes + 512 B of sub-block scale/min slots + 128 B of per-row d/dmin per unit
+    assert q.qlin_packed_bytes(q.QLIN_Q4_K, 4096, 2560) == 256 + (4096 // 32) * (2560 // 256) * 4736
+    assert q.qlin_packed_bytes(q.QLIN_Q4_K, 33, 512) == 256 + 2 * 2 * 4736
+    assert q.qlin_packed_bytes(q.QLIN_Q4_K, 64, 288) == 0  # K % 256
     assert q.qlin_packed_bytes(7, 64, 256) == 0
     assert q.qlin_packed_bytes(q.QLIN_Q4_0, 63, 256, q.QLIN_PACK_GATE_UP) == 0  # odd N
 

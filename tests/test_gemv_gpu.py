@@ -13,8 +13,14 @@ import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
-FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4, q.QLIN_MXFP4]
+FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4, q.QLIN_MXFP4, q.QLIN_Q4_K]
 TOL = 2e-6
+
+
+def k_ok(fmt, K):
+    """Q4_K rows are whole 256-value super-blocks: skip shapes it cannot hold."""
+    if fmt == q.QLIN_Q4_K and K % 256:
+        pytest.skip("Q4_K needs K % 256 == 0")
 
 
 def make(fmt, N, K, seed, pack_flags=q.QLIN_PACK_DEFAULT):
@@ -41,6 +47,7 @@ def check_y(y, yref, A, tol=TOL):
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("N,K", [(32, 256), (100, 288), (257, 2560), (64, 1024)])
 def test_dequant_bit_exact(fmt, N, K):
+    k_ok(fmt, K)
     blocks, scales, g, packed = make(fmt, N, K, 100 + N)
     w = q.qlin_dequant_debug(fmt, packed, N, K).cpu().numpy()
     ref = oracle.dequant_f32(fmt, N, K, blocks, scales, g)
@@ -87,6 +94,7 @@ def test_gemv_parity(fmt, M, xdt):
 @pytest.mark.parametrize("N,K,M", [(1, 32, 1), (31, 96, 2), (33, 544, 5), (4096, 2560, 1), (1024, 9728, 1),
                                    (2560, 17408, 4)])
 def test_gemv_shapes(fmt, N, K, M):
+    k_ok(fmt, K)
     blocks, scales, g, packed = make(fmt, N, K, N + K)
     xdt = torch.bfloat16 if fmt == q.QLIN_NVFP4 else torch.float32
     x = synth.activations(M, K, synth.gen(K), dtype=xdt)
@@ -117,6 +125,28 @@ def test_one_hot_x_gives_dequantized_column(fmt):
     y = q.qlin_gemv(fmt, packed, N, K, x.cuda()).cpu().numpy()
     for i, k in enumerate(ks):
         assert np.array_equal(y[i], W[:, k]), k  # by value: -0 and +0 compare equal
+
+
+def test_dequant_q4k_extreme_fields():
+    """Q4_K super-blocks with the largest and smallest fields: 6-bit scales and mins of 0 and 63,
+    d / dmin of 0, the fp16 maximum 65504 and the smallest subnormal 2^-24, every code; fp32 of
+    d*scale*code - dmin*min rounded once, bit for bit (both products are exact in fp32)."""
+    N, K = 48, 512
+    blocks, _, _ = synth.weights(q.QLIN_Q4_K, N, K, synth.gen(9))
+    b = blocks.clone().view(N, K // 256, 144)
+    fp16 = torch.tensor([0.0, 65504.0, 2.0 ** -24, 1.0], dtype=torch.float16).view(torch.uint8).view(4, 2)
+    for n in range(N):
+        b[n, :, 0:2] = fp16[n % 4]
+        b[n, :, 2:4] = fp16[(n // 4) % 4]
+        if n % 3 == 0:
+            b[n, :, 4:16] = 0xFF  # every scale and min 63
+        elif n % 3 == 1:
+            b[n, :, 4:16] = 0
+    blocks = b.reshape(N, -1).contiguous()
+    packed = q.qlin_pack_weights(q.QLIN_Q4_K, N, K, blocks.cuda())
+    w = q.qlin_dequant_debug(q.QLIN_Q4_K, packed, N, K).cpu().numpy()
+    ref = oracle.dequant_f32(q.QLIN_Q4_K, N, K, blocks.numpy())
+    assert np.array_equal(w.view(np.uint32), ref.view(np.uint32))
 
 
 def test_strided_x_and_y():

@@ -94,6 +94,15 @@ def test_moe_formats_small(fmt, xdt, M):
     run_and_check(ex, M, 2, logits, x)
 
 
+@pytest.mark.parametrize("M", [1, 8])
+def test_moe_q4k_experts(M):
+    # Q4_K experts (K a multiple of 256 for both projections): H = 512, I = 256, top-2 of 6
+    ex = Experts(q.QLIN_Q4_K, 6, 512, 256, 5500)
+    logits = synth.router_logits(M, 6, synth.gen(5600 + M))
+    x = synth.activations(M, 512, synth.gen(5700 + M))
+    run_and_check(ex, M, 2, logits, x)
+
+
 @pytest.mark.parametrize("M", [2, 8])
 def test_moe_all_experts_uniform_is_mean(M):
     # equal logits: ties go to the lower expert index; with M = 8 every expert serves all 8

@@ -20,7 +20,7 @@ import threading
 
 import numpy as np
 
-Q8_0, Q4_0, NVFP4, MXFP4, Q4_K = 1, 2, 3, 4, 5
+Q8_0, Q4_0, NVFP4, MXFP4, Q4_K, Q6_K = 1, 2, 3, 4, 5, 6
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")

@@ -28,7 +28,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { QO_Q8_0 = 1, QO_Q4_0 = 2, QO_NVFP4 = 3, QO_MXFP4 = 4, QO_Q4_K = 5 };
+enum { QO_Q8_0 = 1, QO_Q4_0 = 2, QO_NVFP4 = 3, QO_MXFP4 = 4, QO_Q4_K = 5, QO_Q6_K = 6 };
 
 /* ---------------------------------------------------------------- scalar decoders */
 
@@ -80,6 +80,7 @@ int64_t qo_row_bytes(int fmt, int64_t K) {
     if (fmt == QO_Q4_0) return (K / 32) * 18;
     if (fmt == QO_NVFP4 || fmt == QO_MXFP4) return K / 2;
     if (fmt == QO_Q4_K) return (K / 256) * 144;
+    if (fmt == QO_Q6_K) return (K / 256) * 210;
     return -1;
 }
 
@@ -108,7 +109,13 @@ void qo_q4k_scale_min(const uint8_t* sc12, int j, int* sc, int* m) {
  *   Q4_K super-block (144 B per 256 values, see qo_q4k_scale_min): the codes of the 64 values
  *          64c .. 64c+63 are bytes 32c .. 32c+31 of the code area, values 64c + l in the low
  *          nibble of byte l, 64c + 32 + l in its high nibble; value k of sub-block j = k / 32:
- *          w = d * scale_j * code - dmin * min_j */
+ *          w = d * scale_j * code - dmin * min_j
+ *   Q6_K super-block (210 B per 256 values): ql[128] (low 4 bits of the codes), qh[64] (high 2
+ *          bits), int8 scales[16] (one per 16 values), fp16 d.  In half h (values 128h .. 128h+127,
+ *          bytes ql[64h ..], qh[32h ..], scales[8h ..]) value 128h + 32s + l (s = 0..3, l = 0..31)
+ *          takes its low 4 bits from the low nibble of ql[64h + l] (s = 0), of ql[64h + 32 + l]
+ *          (s = 1), or the high nibbles of those bytes (s = 2, 3), its high 2 bits from bits
+ *          2s, 2s+1 of qh[32h + l], and scale scales[8h + 2s + l / 16]:  w = d * scale * (code - 32) */
 static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t* scales, float g,
                         int64_t n, double* w) {
     if (fmt == QO_Q8_0 || fmt == QO_Q4_0) {
@@ -150,6 +157,23 @@ static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t
                 w[b * 256 + k] = d * sc * code - dmin * m;
             }
         }
+    } else if (fmt == QO_Q6_K) {
+        const uint8_t* row = blocks + n * (K / 256) * 210;
+        for (int64_t b = 0; b < K / 256; ++b) {
+            const uint8_t* blk = row + b * 210;
+            const uint8_t* ql = blk;
+            const uint8_t* qh = blk + 128;
+            const int8_t* sc = (const int8_t*)(blk + 192);
+            double d = qo_fp16((uint16_t)(blk[208] | (blk[209] << 8)));
+            for (int v = 0; v < 256; ++v) {
+                int h = v / 128, s = (v % 128) / 32, l = v % 32;
+                uint8_t lb = ql[64 * h + 32 * (s & 1) + l];
+                int lo = (s < 2) ? (lb & 0xf) : (lb >> 4);
+                int hi = (qh[32 * h + l] >> (2 * s)) & 3;
+                int code = lo | (hi << 4);
+                w[b * 256 + v] = d * sc[8 * h + 2 * s + l / 16] * (code - 32);
+            }
+        }
     } else {
         const uint8_t* row = blocks + n * (K / 2);
         const uint8_t* srow = scales + n * (K / 32);
@@ -161,9 +185,9 @@ static void dequant_row(int fmt, int64_t K, const uint8_t* blocks, const uint8_t
     }
 }
 
-/* Values per block along K (the granularity K must respect): 16 for NVFP4, 256 for Q4_K's
- * super-blocks, 32 otherwise. */
-static int64_t qo_block_k(int fmt) { return fmt == QO_NVFP4 ? 16 : fmt == QO_Q4_K ? 256 : 32; }
+/* Values per block along K (the granularity K must respect): 16 for NVFP4, 256 for the K-quant
+ * super-blocks (Q4_K, Q6_K), 32 otherwise. */
+static int64_t qo_block_k(int fmt) { return fmt == QO_NVFP4 ? 16 : (fmt == QO_Q4_K || fmt == QO_Q6_K) ? 256 : 32; }
 
 /* Full-tensor dequantization to fp64.  Returns 0, or -1 on a bad argument. */
 int qo_dequant(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
@@ -176,7 +200,8 @@ int qo_dequant(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8
 /* The fp32 value of each weight ("bit-exact dequant").  For Q8_0 / Q4_0 and for the NVFP4
  * product e2m1*e4m3 the fp64 value is exactly representable in fp32; the NVFP4 per-tensor
  * scale g is the one rounding: w32 = fp32( (e2m1*e4m3) * g ), rounded once to nearest-even.
- * Q4_K: both products d*scale*code and dmin*min are exact; their difference is rounded once. */
+ * Q4_K: both products d*scale*code and dmin*min are exact; their difference is rounded once.
+ * Q6_K: d*scale*(code - 32) has at most 11 + 7 + 5 significant bits: exact in fp32. */
 int qo_dequant_f32(int fmt, int64_t N, int64_t K, const uint8_t* blocks, const uint8_t* scales,
                    float g, float* W) {
     if (qo_row_bytes(fmt, K) < 0 || K % qo_block_k(fmt)) return -1;

@@ -14,6 +14,8 @@ Canonical layouts (the public conventions; the pages name the formats but not th
   MXFP4 codes as NVFP4, UE8M0 scale bytes [N][K/32] (one per 32 values), no per-tensor scale
   Q4_K  one row = K/256 super-blocks of 144 bytes: fp16 d, fp16 dmin, 12 bytes of packed 6-bit
         sub-block scales and mins, 128 bytes of 4-bit codes (GGUF block_q4_K)
+  Q6_K  one row = K/256 super-blocks of 210 bytes: ql[128] (low code bits), qh[64] (high 2 bits),
+        int8 scales[16] (one per 16 values), fp16 d (GGUF block_q6_K)
 
 Workload recipes (seeded; shapes from the synthetic layer stacks the bench and tests use):
   Q8_0:  codes uniform over [-127, 127], scale uniform real in [1e-3, 1e-2] rounded to fp16
@@ -24,14 +26,16 @@ Workload recipes (seeded; shapes from the synthetic layer stacks the bench and t
   Q4_K:  d and dmin uniform real in [2e-4, 2e-3] rounded to fp16; the 12 scale bytes and the
          128 code bytes uniform over 0..255 (every byte pattern is a valid encoding: sub-block
          scales and mins uniform over 0..63, codes uniform over 0..15)
+  Q6_K:  code bytes (ql, qh) and int8 scales uniform over all byte values (6-bit codes uniform
+         over 0..63), d uniform real in [2e-5, 2e-4] rounded to fp16
   activations N(0, 1) (fp32, or fp32 draws rounded to bf16); router logits N(0, 1)
 """
 from __future__ import annotations
 
 import torch
 
-Q8_0, Q4_0, NVFP4, MXFP4, Q4_K = 1, 2, 3, 4, 5
-FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4", MXFP4: "mxfp4", Q4_K: "q4_k"}
+Q8_0, Q4_0, NVFP4, MXFP4, Q4_K, Q6_K = 1, 2, 3, 4, 5, 6
+FMT_NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", NVFP4: "nvfp4", MXFP4: "mxfp4", Q4_K: "q4_k", Q6_K: "q6_k"}
 NVFP4_G = float(torch.tensor(1.0 / 448.0, dtype=torch.float32))
 
 
@@ -79,6 +83,15 @@ def q4_k(N, K, g, device="cpu", d_range=(2e-4, 2e-3)):
     return torch.cat([_fp16_bytes(d).reshape(N, nb, 4), rest], dim=2).reshape(N, nb * 144).contiguous()
 
 
+def q6_k(N, K, g, device="cpu", d_range=(2e-5, 2e-4)):
+    """Canonical Q6_K tensor, uint8 [N, K/256*210]."""
+    assert K % 256 == 0
+    nb = K // 256
+    rest = torch.randint(0, 256, (N, nb, 208), generator=g, device=device, dtype=torch.int16).to(torch.uint8)
+    d = torch.empty(N, nb, dtype=torch.float32, device=device).uniform_(*d_range, generator=g)
+    return torch.cat([rest, _fp16_bytes(d)], dim=2).reshape(N, nb * 210).contiguous()
+
+
 def nvfp4(N, K, g, device="cpu", s_range=(0.5, 448.0)):
     """Canonical NVFP4 tensor: (codes uint8 [N, K/2], scales uint8 [N, K/16], fp32 tensor scale)."""
     assert K % 16 == 0
@@ -112,6 +125,8 @@ def weights(fmt, N, K, g, device="cpu"):
         return nvfp4(N, K, g, device)
     if fmt == Q4_K:
         return q4_k(N, K, g, device), None, 1.0
+    if fmt == Q6_K:
+        return q6_k(N, K, g, device), None, 1.0
     raise ValueError(fmt)
 
 

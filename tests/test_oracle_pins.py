@@ -276,6 +276,83 @@ def test_q4k_f32_value_is_one_rounding_of_the_exact_difference():
     assert w32[0] == np.float32(945.0) and np.float32(945.0 - 2.0 ** -24) == np.float32(945.0)
 
 
+# ----------------------------------------------------------------------------- Q6_K
+def _q6k_block(d_bits, scales, codes):
+    """One GGUF Q6_K super-block packed from its fields (packing direction, written here from the
+    block_q6_K definition): value v = 128h + 32s + l puts its low 4 bits in the low (s < 2) or high
+    (s >= 2) nibble of ql[64h + 32 (s & 1) + l] and its high 2 bits at bits 2s of qh[32h + l]."""
+    ql, qh = bytearray(128), bytearray(64)
+    for v in range(256):
+        h, s, l = v // 128, (v % 128) // 32, v % 32
+        i = 64 * h + 32 * (s & 1) + l
+        ql[i] |= (codes[v] & 15) << (4 if s >= 2 else 0)
+        qh[32 * h + l] |= (codes[v] >> 4) << (2 * s)
+    return bytes(ql + qh + bytes(int(t) & 0xFF for t in scales) + struct.pack("<H", d_bits))
+
+
+def test_q6k_dequant_matches_golden():
+    lines = read_golden("q6k_block.txt")
+    blk = bytearray(210)
+    blk[192:208] = bytes(int(t, 16) for t in lines[0].split()[1:])
+    blk[208:210] = struct.pack("<H", 0x3C00)
+    for t in lines[1].split()[1:]:
+        i, v = t.split(":")
+        blk[int(i)] = int(v, 16)
+    for t in lines[2].split()[1:]:
+        i, v = t.split(":")
+        blk[128 + int(i)] = int(v, 16)
+    w = oracle.dequant(oracle.Q6_K, 1, 256, np.frombuffer(bytes(blk), np.uint8)[None, :])[0]
+    for t in lines[3].split()[1:]:
+        k, v = t.split(":")
+        assert w[int(k)] == float(v), (k, w[int(k)], v)
+
+
+def test_q6k_packed_fields_decode_exactly():
+    # every 6-bit code and every int8 scale value at every position, fp16 d from numpy: the oracle
+    # returns d * scale * (code - 32) exactly, and that value is exact in fp32 too
+    rng = np.random.default_rng(9)
+    for rep in range(32):
+        codes = [int(v) for v in (np.arange(256) * 7 + rep) % 64]
+        scales = [int(v) for v in ((np.arange(16) * 17 + 8 * rep) % 256) - 128]
+        d16 = np.float16(rng.uniform(1e-3, 4.0))
+        blk = np.frombuffer(_q6k_block(int(d16.view(np.uint16)), scales, codes), np.uint8)[None, :]
+        w = oracle.dequant(oracle.Q6_K, 1, 256, blk)[0]
+        for v in range(256):
+            h, s, l = v // 128, (v % 128) // 32, v % 32
+            ref = Fraction(float(d16)) * scales[8 * h + 2 * s + l // 16] * (codes[v] - 32)
+            assert Fraction(w[v]) == ref, (rep, v)
+        assert np.array_equal(oracle.dequant_f32(oracle.Q6_K, 1, 256, blk)[0].astype(np.float64), w)
+
+
+def test_q6k_identity_exact_sum_and_one_hot():
+    K = 512
+    rows = []
+    for n in range(K):
+        codes = [32] * K
+        codes[n] = 33
+        rows.append(b"".join(_q6k_block(0x3C00, [1] * 16, codes[256 * b:256 * (b + 1)]) for b in range(2)))
+    blocks = np.frombuffer(b"".join(rows), np.uint8).reshape(K, -1)
+    assert blocks.shape[1] == oracle.row_bytes(oracle.Q6_K, K) == 420
+    x = synth.activations(2, K, synth.gen(31)).double().numpy()
+    y, A = oracle.gemv(oracle.Q6_K, K, K, blocks, x)
+    assert np.array_equal(y, x) and np.array_equal(A, np.abs(x))
+    N, M = 5, 2
+    blocks, _, _ = synth.weights(oracle.Q6_K, N, K, synth.gen(32))
+    blocks = blocks.numpy()
+    W = oracle.dequant(oracle.Q6_K, N, K, blocks)
+    x = synth.activations(M, K, synth.gen(33)).double().numpy()
+    y, _ = oracle.gemv(oracle.Q6_K, N, K, blocks, x)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(W[n, k]) * Fraction(x[m, k]) for k in range(K))
+            absum = sum(abs(Fraction(W[n, k]) * Fraction(x[m, k])) for k in range(K))
+            assert abs(Fraction(y[m, n]) - exact) <= Fraction(K * 2.0 ** -52) * absum
+    for k in (0, 15, 16, 127, 128, 300, 511):
+        e = np.zeros((1, K))
+        e[0, k] = 1.0
+        assert np.array_equal(oracle.gemv(oracle.Q6_K, N, K, blocks, e)[0][0], W[:, k])
+
+
 def _identity_mxfp4(K):
     codes, _ = _identity_nvfp4(K)
     return codes, np.full((K, K // 32), 0x7F, np.uint8)  # UE8M0 2^0

@@ -16,7 +16,7 @@ import threading
 
 import torch
 
-QLIN_Q8_0, QLIN_Q4_0, QLIN_NVFP4, QLIN_MXFP4, QLIN_Q4_K = 1, 2, 3, 4, 5
+QLIN_Q8_0, QLIN_Q4_0, QLIN_NVFP4, QLIN_MXFP4, QLIN_Q4_K, QLIN_Q6_K = 1, 2, 3, 4, 5, 6
 QLIN_F32, QLIN_BF16 = 0, 1
 QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_OUT_BF16, QLIN_FLAG_PDL, QLIN_FLAG_CTA_PAIRS = 0, 1, 0x10, 0x100, 0x200
 QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA = 0, 1, 2

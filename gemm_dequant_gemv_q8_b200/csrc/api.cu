@@ -33,12 +33,12 @@ namespace {
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
 bool valid_fmt(int f) {
-    return f == QLIN_Q8_0 || f == QLIN_Q4_0 || f == QLIN_NVFP4 || f == QLIN_MXFP4 || f == QLIN_Q4_K;
+    return f == QLIN_Q8_0 || f == QLIN_Q4_0 || f == QLIN_NVFP4 || f == QLIN_MXFP4 || f == QLIN_Q4_K || f == QLIN_Q6_K;
 }
 
 bool valid_shape(int fmt, int64_t N, int64_t K) {
     if (N < 1 || K < 1 || N > kMaxDim || K > kMaxDim) return false;
-    return fmt == QLIN_NVFP4 ? (K % 16 == 0) : fmt == QLIN_Q4_K ? (K % 256 == 0) : (K % 32 == 0);
+    return fmt == QLIN_NVFP4 ? (K % 16 == 0) : (fmt == QLIN_Q4_K || fmt == QLIN_Q6_K) ? (K % 256 == 0) : (K % 32 == 0);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

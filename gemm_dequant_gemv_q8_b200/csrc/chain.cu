@@ -292,11 +292,11 @@ __device__ __forceinline__ bool chain_wait_op(const ChainArgs& a, int j) {
 }
 
 // Shared memory of the chain kernel: the per-warp weight rings and their barriers, then (for
-// M <= 2, except Q8_0 whose ring leaves no room) two activation stages per warp.
+// M <= 2, except Q8_0 / Q6_K whose rings leave no room) two activation stages per warp.
 template <int FMT, int MAXM, bool XBF16>
 struct ChainSmem {
     static constexpr int MP = MAXM >= 2 ? 2 : 1;
-    static constexpr bool kStaged = MAXM <= 2 && FMT != QLIN_Q8_0;
+    static constexpr bool kStaged = MAXM <= 2 && FMT != QLIN_Q8_0 && FMT != QLIN_Q6_K;
     static constexpr int kStageBytes = MP * XStage<XBF16>::kRowBytes;  // one stage of one warp
     static constexpr int kXOff = (RingCfg<FMT>::kSmem + 127) / 128 * 128;
     static constexpr int kBytes = kStaged ? kXOff + kGemvWarps * 2 * kStageBytes : RingCfg<FMT>::kSmem;
@@ -415,7 +415,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                 unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
             } else {
                 float2 xv[MP][16];
-                float xb[MP];
+                float2 xb[MP];
                 load_x_staged<XBF16, MP>(xcur, part, xv);
                 prep_x<FMT, MP>(xv, xb);
                 unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                 unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
             } else {
                 float2 xv[MP][16];
-                float xb[MP];
+                float2 xb[MP];
                 load_x_rows<XBF16, MP, true>(rows, k0, o.K, xv);
                 prep_x<FMT, MP>(xv, xb);
                 unit_dot<FMT, MP, true>(ubuf, lane, xv, xb, acc8);
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
                     unit_dot_fp4h<MP, false, FMT>(ubuf, lane, xh, xsc, res);
                 } else {
                     float2 xv[MP][16];
-                    float xb[MP];
+                    float2 xb[MP];
                     load_x_rows<XBF16, MP, true>(rows, k0, o.K, xv);
                     prep_x<FMT, MP>(xv, xb);
                     unit_dot<FMT, MP>(ubuf, lane, xv, xb, res);
@@ -556,7 +556,7 @@ static int chain_sm_count() {
 // CTAs of the persistent grid: every SM holds RingCfg<FMT>::kCtasPerSm of them (the register
 // and shared-memory budget of the kernel is sized for exactly that).
 static int chain_grid(int fmt) {
-    const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
+    const int cps = ring_ctas_per_sm(fmt);
     return chain_sm_count() * cps;
 }
 
@@ -695,6 +695,7 @@ extern "C" cudaError_t qlin_launch_chain(int fmt, int xdt, int M, const qlin_gem
     else if (fmt == QLIN_Q8_0) e = bf16 ? chain_launch_m<QLIN_Q8_0, true>(a, grid, s, pdl) : chain_launch_m<QLIN_Q8_0, false>(a, grid, s, pdl);
     else if (fmt == QLIN_MXFP4) e = bf16 ? chain_launch_m<QLIN_MXFP4, true>(a, grid, s, pdl) : chain_launch_m<QLIN_MXFP4, false>(a, grid, s, pdl);
     else if (fmt == QLIN_Q4_K) e = bf16 ? chain_launch_m<QLIN_Q4_K, true>(a, grid, s, pdl) : chain_launch_m<QLIN_Q4_K, false>(a, grid, s, pdl);
+    else if (fmt == QLIN_Q6_K) e = bf16 ? chain_launch_m<QLIN_Q6_K, true>(a, grid, s, pdl) : chain_launch_m<QLIN_Q6_K, false>(a, grid, s, pdl);
     else e = bf16 ? chain_launch_m<QLIN_NVFP4, true>(a, grid, s, pdl) : chain_launch_m<QLIN_NVFP4, false>(a, grid, s, pdl);
     delete a;
     return e;

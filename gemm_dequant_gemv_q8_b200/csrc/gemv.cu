@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) gem
     for (int m = 0; m < MAXM; ++m) acc[m] = 0.f;
     float acc8[8][MP];
     float2 xv[MP][16];
-    float xb[MP];
+    float2 xb[MP];
     uint32_t xh[MP][16];
     float xsc[MP][2];
     const void* rows0[MP];
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) gem
                     load_x_fp4h<MP>(rows, k0, a.K, xph, xps);
                     unit_dot_fp4h<MP, false, FMT>(ubuf, lane, xph, xps, res);
                 } else {
-                    float xpb[MP];
+                    float2 xpb[MP];
                     load_x_rows<XBF16, MP>(rows, k0, a.K, xp);
                     prep_x<FMT, MP>(xp, xpb);
                     unit_dot<FMT, MP>(ubuf, lane, xp, xpb, res);
@@ -327,7 +327,7 @@ static GemvPlan plan_gemv(int fmt, int M, int64_t N, int64_t K, int pack_flags) 
     p.T = geo.T;
     p.G = geo.G;
     p.U = geo.U;
-    const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
+    const int cps = ring_ctas_per_sm(fmt);
     const int64_t cmax = (int64_t)sm_count_cached() * cps;
     int64_t c = (p.U + kGemvWarps - 1) / kGemvWarps;  // at least one unit per warp
     if (c > cmax) c = cmax;
@@ -416,6 +416,7 @@ extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, 
     if (fmt == QLIN_Q8_0) return launch_fmt<QLIN_Q8_0>(a, bf16, epi, p.grid, s, pdl);
     if (fmt == QLIN_MXFP4) return launch_fmt<QLIN_MXFP4>(a, bf16, epi, p.grid, s, pdl);
     if (fmt == QLIN_Q4_K) return launch_fmt<QLIN_Q4_K>(a, bf16, epi, p.grid, s, pdl);
+    if (fmt == QLIN_Q6_K) return launch_fmt<QLIN_Q6_K>(a, bf16, epi, p.grid, s, pdl);
     return launch_fmt<QLIN_NVFP4>(a, bf16, epi, p.grid, s, pdl);
 }
 
@@ -453,10 +454,12 @@ static cudaError_t noalloc_scratch(void** out) {
 extern "C" qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
                                            const void* x, qlin_dtype_t xdt, int M, int64_t ldx, float* y,
                                            int64_t ldy, int flags, qlin_stream_t stream) {
-    if (fmt != QLIN_Q8_0 && fmt != QLIN_Q4_0 && fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4 && fmt != QLIN_Q4_K)
+    if (fmt != QLIN_Q8_0 && fmt != QLIN_Q4_0 && fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4 && fmt != QLIN_Q4_K &&
+        fmt != QLIN_Q6_K)
         return QLIN_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || N > ((int64_t)1 << 31) || K > ((int64_t)1 << 31)) return QLIN_ERR_INVALID_ARG;
-    if (fmt == QLIN_NVFP4 ? (K % 16) : fmt == QLIN_Q4_K ? (K % 256) : (K % 32)) return QLIN_ERR_INVALID_ARG;
+    if (fmt == QLIN_NVFP4 ? (K % 16) : (fmt == QLIN_Q4_K || fmt == QLIN_Q6_K) ? (K % 256) : (K % 32))
+        return QLIN_ERR_INVALID_ARG;
     if (M < 1 || M > 8) return QLIN_ERR_INVALID_ARG;
     if (xdt != QLIN_F32 && xdt != QLIN_BF16) return QLIN_ERR_INVALID_ARG;
     const int epi = flags & 0xff;

@@ -13,8 +13,10 @@ struct RingCfg {
     static constexpr int D = 2;  // ring depth (units) per warp
     static constexpr int UB = unit_bytes(FMT);
     static constexpr int kSmem = kGemvWarps * D * (UB + 8);
-    static constexpr int kCtasPerSm = (FMT == QLIN_Q8_0) ? 3 : 4;  // 12-16 warps per SM
+    static constexpr int kCtasPerSm = (FMT == QLIN_Q8_0 || FMT == QLIN_Q6_K) ? 3 : 4;  // 12-16 warps per SM
 };
+// CTAs per SM of the persistent grids (the ring's shared memory allows 3 for the byte-code formats).
+inline int ring_ctas_per_sm(int fmt) { return (fmt == QLIN_Q8_0 || fmt == QLIN_Q6_K) ? 3 : 4; }
 
 
 // ------------------------------------------------------------------ code decoders
@@ -89,13 +91,13 @@ __device__ __forceinline__ float offset_sum(const float2 (&x)[16]) {
 // element e (pair e/2) times 2^(kXExp - 4 j) with j the decoder's position of element e mod 8.
 // Q4_K (same code positions, no offset): xb = sum * 2^(kXExp - 149), the min term's factor.
 template <int MP, bool K4 = false>
-__device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float (&xb)[MP]) {
+__device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float2 (&xb)[MP]) {
     constexpr float c = K4 ? 0x1p-86f : 0x1p-83f;  // (1 or 8) * 2^(kXExp - 149)
     const float2 s0 = make_float2(0x1p63f, 0x1p59f), s1 = make_float2(0x1p55f, 0x1p51f);
     const float2 s2 = make_float2(0x1p47f, 0x1p43f);
 #pragma unroll
     for (int mm = 0; mm < MP; ++mm) {
-        xb[mm] = c * offset_sum(xv[mm]);
+        xb[mm].x = c * offset_sum(xv[mm]);
 #pragma unroll
         for (int q = 0; q < 16; ++q)  // pair q = 4k + (q & 3); pair 4k+3 sits at positions 0,1 (k even) or 2,3
             xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 3) == 0 ? s0 : (q & 3) == 1 ? s1 : (q & 3) == 2 ? s2 : ((q >> 2) & 1) ? s1 : s0);
@@ -104,13 +106,30 @@ __device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float (&xb)[MP])
 
 // Prepare a lane's 32 activations for the Q8_0 decoder: offset 128 * sum (scaled), pairs
 // (4k, 4k+1) times (2^63, 2^55) and (4k+2, 4k+3) times (2^47, 2^63).
-template <int MP>
-__device__ __forceinline__ void prep_x_q8(float2 (&xv)[MP][16], float (&xb)[MP]) {
-    constexpr float c = 0x1p-79f;  // 128 * 2^(kXExp - 149)
+// Q6_K (codes 0..63 in the same byte positions, offset 32, a scale per 16 values): the offset
+// sums of elements 0..15 and 16..31 separately, each times 32 * 2^(kXExp - 149).
+template <int MP, bool K6 = false>
+__device__ __forceinline__ void prep_x_q8(float2 (&xv)[MP][16], float2 (&xb)[MP]) {
+    constexpr float c = K6 ? 0x1p-81f : 0x1p-79f;  // (32 or 128) * 2^(kXExp - 149)
     const float2 s0 = make_float2(0x1p63f, 0x1p55f), s1 = make_float2(0x1p47f, 0x1p63f);
 #pragma unroll
     for (int mm = 0; mm < MP; ++mm) {
-        xb[mm] = c * offset_sum(xv[mm]);
+        if (K6) {
+            float2 h[2];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {  // pairs 8b .. 8b+7: words 4b .. 4b+3 of the decoder
+                float2 t0 = xv[mm][8 * b], t1 = xv[mm][8 * b + 1];
+#pragma unroll
+                for (int q = 2; q < 8; q += 2) {
+                    t0 = __fadd2_rn(t0, xv[mm][8 * b + q]);
+                    t1 = __fadd2_rn(t1, xv[mm][8 * b + q + 1]);
+                }
+                h[b] = __fadd2_rn(t0, t1);
+            }
+            xb[mm] = make_float2(c * (h[0].x + h[0].y), c * (h[1].x + h[1].y));
+        } else {
+            xb[mm].x = c * offset_sum(xv[mm]);
+        }
 #pragma unroll
         for (int q = 0; q < 16; ++q) xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 1) ? s1 : s0);
     }
@@ -118,13 +137,14 @@ __device__ __forceinline__ void prep_x_q8(float2 (&xv)[MP][16], float (&xb)[MP])
 
 // Prepare a lane's activations for unit_dot<FMT> (NVFP4 needs no preparation; xb is unused).
 template <int FMT, int MP>
-__device__ __forceinline__ void prep_x(float2 (&xv)[MP][16], float (&xb)[MP]) {
+__device__ __forceinline__ void prep_x(float2 (&xv)[MP][16], float2 (&xb)[MP]) {
     if (FMT == QLIN_Q4_0) prep_x_q4<MP>(xv, xb);
     else if (FMT == QLIN_Q4_K) prep_x_q4<MP, true>(xv, xb);
     else if (FMT == QLIN_Q8_0) prep_x_q8<MP>(xv, xb);
+    else if (FMT == QLIN_Q6_K) prep_x_q8<MP, true>(xv, xb);
     else {
 #pragma unroll
-        for (int mm = 0; mm < MP; ++mm) xb[mm] = 0.f;
+        for (int mm = 0; mm < MP; ++mm) xb[mm] = make_float2(0.f, 0.f);
     }
 }
 
@@ -406,7 +426,7 @@ __device__ __forceinline__ void unit_dot_fp4h(const uint8_t* ub, int lane, const
 // with ACC the contribution is added to res instead (one fused multiply-add per block).
 template <int FMT, int MP, bool ACC = false>
 __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const float2 (&xv)[MP][16],
-                                         const float (&xb)[MP], float (&res)[8][MP]) {
+                                         const float2 (&xb)[MP], float (&res)[8][MP]) {
     uint32_t sw[4];
     if (FMT == QLIN_MXFP4) {  // 8 bits of scale per (row, part)
         const uint2 s2 = *reinterpret_cast<const uint2*>(ub + code_bytes(FMT) + lane * 8);
@@ -415,12 +435,14 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
         const uint4 sv = lds128(ub + code_bytes(FMT) + lane * 16);
         sw[0] = sv.x, sw[1] = sv.y, sw[2] = sv.z, sw[3] = sv.w;
     }
-    uint32_t dmw[FMT == QLIN_Q4_K ? 8 : 1];  // Q4_K: {d, dmin} of the lane's 8 rows
-    if (FMT == QLIN_Q4_K) {
-        const uint4 d0 = lds128(ub + kQ4kDmOff + (lane >> 3) * 32), d1 = lds128(ub + kQ4kDmOff + (lane >> 3) * 32 + 16);
+    constexpr bool kRowD = FMT == QLIN_Q4_K || FMT == QLIN_Q6_K;
+    uint32_t dmw[kRowD ? 8 : 1];  // K-quants: {d, dmin} (Q6_K: {d, 0}) of the lane's 8 rows
+    if (kRowD) {
+        const uint8_t* dp = ub + row_d_off(FMT) + (lane >> 3) * 32;
+        const uint4 d0 = lds128(dp), d1 = lds128(dp + 16);
         const uint32_t t[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
 #pragma unroll
-        for (int i = 0; i < (FMT == QLIN_Q4_K ? 8 : 1); ++i) dmw[i] = t[i];
+        for (int i = 0; i < (kRowD ? 8 : 1); ++i) dmw[i] = t[i];
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -449,12 +471,12 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
                 }
             }
             if (FMT == QLIN_Q4_K) {  // d * scale * sum(code x) - dmin * min * sum(x), both factors exact
-                const float2 dd = __half22float2(*reinterpret_cast<const __half2*>(&dmw[FMT == QLIN_Q4_K ? i : 0]));
+                const float2 dd = __half22float2(*reinterpret_cast<const __half2*>(&dmw[kRowD ? i : 0]));
                 const float ka = dd.x * (float)(sc & 63u), kb = dd.y * (float)((sc >> 6) & 63u);
 #pragma unroll
                 for (int mm = 0; mm < MP; ++mm) {
                     const float2 u = __fadd2_rn(s0[mm], s1[mm]);
-                    const float base = ACC ? fmaf(-kb, xb[mm], res[i][mm]) : -kb * xb[mm];
+                    const float base = ACC ? fmaf(-kb, xb[mm].x, res[i][mm]) : -kb * xb[mm].x;
                     res[i][mm] = fmaf(ka, u.x + u.y, base);
                 }
             } else {
@@ -462,7 +484,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
                 for (int mm = 0; mm < MP; ++mm) {
                     const float2 u = __fadd2_rn(s0[mm], s1[mm]);
-                    const float bsum = (u.x + u.y) - xb[mm];
+                    const float bsum = (u.x + u.y) - xb[mm].x;
                     res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
                 }
             }
@@ -487,8 +509,35 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) {
                 const float2 u = __fadd2_rn(s0[mm], s1[mm]);
-                const float bsum = (u.x + u.y) - xb[mm];
+                const float bsum = (u.x + u.y) - xb[mm].x;
                 res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
+            }
+        } else if (FMT == QLIN_Q6_K) {  // Q8_0's byte planes holding 6-bit codes; a scale per 16 values
+            const uint4 c0 = lds128(ub + (lane + 32 * i) * 16);
+            const uint4 c1 = lds128(ub + 4096 + (lane + 32 * i) * 16);
+            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            float2 s0[2][MP], s1[2][MP];  // [16-value block][row]
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) s0[b][mm] = s1[b][mm] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float2 p[2];
+                dec_q8(cw[k], p);
+#pragma unroll
+                for (int mm = 0; mm < MP; ++mm) {
+                    s0[k >> 2][mm] = __ffma2_rn(p[0], xv[mm][2 * k + 0], s0[k >> 2][mm]);
+                    s1[k >> 2][mm] = __ffma2_rn(p[1], xv[mm][2 * k + 1], s1[k >> 2][mm]);
+                }
+            }
+            const float d = __half2float(__ushort_as_half((unsigned short)(dmw[kRowD ? i : 0] & 0xffffu)));
+            const float e0 = d * (float)(int8_t)(sc & 0xffu), e1 = d * (float)(int8_t)((sc >> 8) & 0xffu);  // exact
+#pragma unroll
+            for (int mm = 0; mm < MP; ++mm) {
+                const float2 u0 = __fadd2_rn(s0[0][mm], s1[0][mm]), u1 = __fadd2_rn(s0[1][mm], s1[1][mm]);
+                const float b0 = (u0.x + u0.y) - xb[mm].x, b1 = (u1.x + u1.y) - xb[mm].y;
+                res[i][mm] = fmaf(e1, b1, ACC ? fmaf(e0, b0, res[i][mm]) : e0 * b0);
             }
         } else if (FMT == QLIN_MXFP4) {  // one 32-element block per part, one UE8M0 scale
             const uint4 c = lds128(ub + (lane + 32 * i) * 16);

@@ -393,7 +393,7 @@ __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, i
         unit_dot_fp4h<MP, true, FMT>(ubuf, lane, xh, xsc, acc8);
     } else {
         float2 xv[MP][16];
-        float xb[MP];
+        float2 xb[MP];
         if (xs != nullptr)
             load_x_staged<XB, MP>(xs, part, xv);
         else
@@ -405,12 +405,12 @@ __device__ __forceinline__ void moe_unit(const MoeArgs& a, const RouteSmem& r, i
 }
 
 // Shared memory of the MoE kernel: the per-warp weight rings and their barriers, then (except
-// Q8_0, whose ring leaves no room) one activation stage per warp: the next unit's rows, copied
+// Q8_0 and Q6_K, whose rings leave no room) one activation stage per warp: the next unit's rows, copied
 // while the current unit computes.
 template <int FMT, int MAXM>
 struct MoeSmem {
     static constexpr int MP = MAXM;
-    static constexpr bool kStaged = FMT != QLIN_Q8_0;
+    static constexpr bool kStaged = FMT != QLIN_Q8_0 && FMT != QLIN_Q6_K;
     static constexpr int kStageBytes = MP * XStage<false>::kRowBytes;  // fp32 layout; bf16 rows fit
     static constexpr int kXOff = (RingCfg<FMT>::kSmem + 127) / 128 * 128;
     static constexpr int kBytes = kStaged ? kXOff + kGemvWarps * kStageBytes : RingCfg<FMT>::kSmem;
@@ -626,7 +626,7 @@ struct MoePlan {
 
 static MoePlan plan_moe(int fmt, int M, int64_t H, int64_t I, int top_k, bool need_h) {
     MoePlan p;
-    const int cps = fmt == QLIN_Q8_0 ? RingCfg<QLIN_Q8_0>::kCtasPerSm : RingCfg<QLIN_Q4_0>::kCtasPerSm;
+    const int cps = ring_ctas_per_sm(fmt);
     p.grid = moe_sm_count() * cps;
     int64_t off = al256(moe_head_bytes());
     p.o_off = off;
@@ -718,5 +718,6 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
     if (fmt == QLIN_Q8_0) return bf16 ? moe_launch_m<QLIN_Q8_0, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q8_0, false>(a, p.grid, s, pdl);
     if (fmt == QLIN_MXFP4) return bf16 ? moe_launch_m<QLIN_MXFP4, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_MXFP4, false>(a, p.grid, s, pdl);
     if (fmt == QLIN_Q4_K) return bf16 ? moe_launch_m<QLIN_Q4_K, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q4_K, false>(a, p.grid, s, pdl);
+    if (fmt == QLIN_Q6_K) return bf16 ? moe_launch_m<QLIN_Q6_K, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_Q6_K, false>(a, p.grid, s, pdl);
     return bf16 ? moe_launch_m<QLIN_NVFP4, true>(a, p.grid, s, pdl) : moe_launch_m<QLIN_NVFP4, false>(a, p.grid, s, pdl);
 }

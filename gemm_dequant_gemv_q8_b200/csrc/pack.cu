@@ -105,7 +105,36 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ b
         *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v;
         sc[0] = (uint8_t)(scm & 0xff);
         sc[1] = (uint8_t)(scm >> 8);
-        if (p == 0) *reinterpret_cast<uint32_t*>(ub + kQ4kDmOff + ((r & 3) * 8 + (r >> 2)) * 4) = dm;
+        if (p == 0) *reinterpret_cast<uint32_t*>(ub + row_d_off(FMT) + ((r & 3) * 8 + (r >> 2)) * 4) = dm;
+    } else if (FMT == QLIN_Q6_K) {
+        // GGUF Q6_K super-block (210 B per 256 values = one k-group): ql[128], qh[64], int8
+        // scales[16], fp16 d.  Part p holds values 32p .. 32p+31 = half h = p / 4, quarter s = p % 4
+        // of the super-block; each 6-bit code is assembled into a byte of the Q8_0 planes.
+        uint8_t out[32];
+        uint16_t scs = 0;
+        uint32_t dm = 0;
+        for (int j = 0; j < 32; ++j) out[j] = 32;  // padding: code 32 (value 0), scale 0
+        if (n >= 0) {
+            const uint8_t* blk = blocks + n * (K / 256) * 210 + g * 210;
+            const int h = p >> 2, q = p & 3;
+            const uint8_t* ql = blk + 64 * h + 32 * (q & 1);
+            const uint8_t* qh = blk + 128 + 32 * h;
+            for (int e = 0; e < 32; ++e) {
+                const int lo = (q < 2) ? (ql[e] & 0xf) : (ql[e] >> 4);
+                const int hi = (qh[e] >> (2 * q)) & 3;
+                out[e] = (uint8_t)(lo | (hi << 4));
+            }
+            scs = (uint16_t)(blk[192 + 8 * h + 2 * q] | (blk[192 + 8 * h + 2 * q + 1] << 8));
+            dm = (uint32_t)blk[208] | ((uint32_t)blk[209] << 8);
+        }
+        uint4 v0, v1;
+        memcpy(&v0, out, 16);
+        memcpy(&v1, out + 16, 16);
+        *reinterpret_cast<uint4*>(ub + (r * 8 + p) * 16) = v0;
+        *reinterpret_cast<uint4*>(ub + 4096 + (r * 8 + p) * 16) = v1;
+        sc[0] = (uint8_t)(scs & 0xff);
+        sc[1] = (uint8_t)(scs >> 8);
+        if (p == 0) *reinterpret_cast<uint32_t*>(ub + row_d_off(FMT) + ((r & 3) * 8 + (r >> 2)) * 4) = dm;
     } else if (FMT == QLIN_MXFP4) {  // codes as NVFP4, one UE8M0 scale per part
         uint8_t out[16];
         uint8_t s = 0;
@@ -188,13 +217,22 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
         }
     } else if (FMT == QLIN_Q4_K) {
         // w = d * scale * code - dmin * min: both products exact in fp32, one rounding
-        const uint32_t dm = *reinterpret_cast<const uint32_t*>(ub + kQ4kDmOff + ((r & 3) * 8 + (r >> 2)) * 4);
+        const uint32_t dm = *reinterpret_cast<const uint32_t*>(ub + row_d_off(FMT) + ((r & 3) * 8 + (r >> 2)) * 4);
         const int scm = sc[0] | (sc[1] << 8);
         const float a = fp16_bits_to_f32(dm & 0xffffu) * (float)(scm & 63);
         const float b = fp16_bits_to_f32(dm >> 16) * (float)((scm >> 6) & 63);
         for (int e = 0; e < 32; ++e) {
             const int nib = (cv[e / 2] >> (4 * (e & 1))) & 0xf;
             out[e] = __fmaf_rn(a, (float)nib, -b);
+        }
+    } else if (FMT == QLIN_Q6_K) {
+        // w = d * scale * (code - 32): d * scale and the product are exact in fp32 (<= 23 bits)
+        const uint32_t dm = *reinterpret_cast<const uint32_t*>(ub + row_d_off(FMT) + ((r & 3) * 8 + (r >> 2)) * 4);
+        const float d = fp16_bits_to_f32(dm & 0xffffu);
+        const float e0 = d * (float)(int8_t)sc[0], e1 = d * (float)(int8_t)sc[1];
+        for (int e = 0; e < 32; ++e) {
+            const int b = e < 16 ? cv[e] : cv[4096 + e - 16];
+            out[e] = __fmul_rn(e < 16 ? e0 : e1, (float)(b - 32));
         }
     } else if (FMT == QLIN_MXFP4) {
         const float s = e8m0_to_f32(sc[0]);
@@ -245,6 +283,9 @@ extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void*
     else if (fmt == QLIN_Q4_K)
         pack_kernel<QLIN_Q4_K><<<grid, 256, 0, s>>>((const uint8_t*)blocks, nullptr, N, K, gu,
                                                      (uint8_t*)packed, geo.G);
+    else if (fmt == QLIN_Q6_K)
+        pack_kernel<QLIN_Q6_K><<<grid, 256, 0, s>>>((const uint8_t*)blocks, nullptr, N, K, gu,
+                                                     (uint8_t*)packed, geo.G);
     else
         pack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)blocks, (const uint8_t*)scales,
                                                       N, K, gu, (uint8_t*)packed, geo.G);
@@ -264,6 +305,8 @@ extern "C" cudaError_t qlin_launch_unpack(int fmt, const void* packed, int64_t N
         unpack_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     else if (fmt == QLIN_Q4_K)
         unpack_kernel<QLIN_Q4_K><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
+    else if (fmt == QLIN_Q6_K)
+        unpack_kernel<QLIN_Q6_K><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     else
         unpack_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>((const uint8_t*)packed, N, K, gu, geo.G, w);
     return cudaGetLastError();

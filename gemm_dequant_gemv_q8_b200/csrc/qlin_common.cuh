@@ -24,6 +24,9 @@ namespace qlin {
 //           bits 0..5 and 6-bit min in bits 6..11; then 32 x 4 B of per-row super-block scales
 //           {fp16 d, fp16 dmin}, row r at entry (r % 4) * 8 + r / 4, so lane l reads the 8 rows
 //           it works on as 32 contiguous bytes at entry (l / 8) * 8.
+//           Q6_K: codes as Q8_0's two planes (byte = 6-bit code, 0..63); the 16-bit slot holds the
+//           int8 scales of elements 0..15 (low byte) and 16..31 (high byte); then per-row {fp16 d, 0}
+//           entries as Q4_K.
 // A warp reading vector (lane + 32 * i) in step i therefore touches 512 contiguous bytes, and
 // lane l always works on part l % 8 of rows l / 8 + 4 i (i = 0..7).
 // Element order inside a part:
@@ -51,11 +54,13 @@ struct PackedHeader {
 };
 static_assert(sizeof(PackedHeader) == kHdrBytes, "header size");
 
-__host__ __device__ constexpr int code_bytes(int fmt) { return fmt == QLIN_Q8_0 ? 8192 : 4096; }
+__host__ __device__ constexpr int code_bytes(int fmt) { return (fmt == QLIN_Q8_0 || fmt == QLIN_Q6_K) ? 8192 : 4096; }
 __host__ __device__ constexpr int unit_bytes(int fmt) {
-    return code_bytes(fmt) + (fmt == QLIN_MXFP4 ? 256 : fmt == QLIN_Q4_K ? 640 : 512);
+    return code_bytes(fmt) + (fmt == QLIN_MXFP4 ? 256 : (fmt == QLIN_Q4_K || fmt == QLIN_Q6_K) ? 640 : 512);
 }
-constexpr int kQ4kDmOff = 4096 + 512;  // Q4_K: per-row {d, dmin} after the sub-block slots
+// K-quants: 32 per-row 4-byte entries after the (row, part) slots -- Q4_K {fp16 d, fp16 dmin},
+// Q6_K {fp16 d, 0} -- row r at entry (r % 4) * 8 + r / 4.
+__host__ __device__ constexpr int row_d_off(int fmt) { return code_bytes(fmt) + 512; }
 
 struct Geometry {
     int64_t T, G, U;  // tiles, k-groups, units

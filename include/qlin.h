@@ -1,6 +1,6 @@
 /*
  * qlin.h -- C ABI of libqlin, a B200 (sm_100a) library for the decode-step linear layer over
- * block-quantized weights: fused dequantize-and-multiply of GGUF Q8_0 / Q4_0 / Q4_K blocks and
+ * block-quantized weights: fused dequantize-and-multiply of GGUF Q8_0 / Q4_0 / Q4_K / Q6_K blocks and
  * NVFP4 / MXFP4 tensors against a small batch of activation rows, the routed MoE expert projections, and
  * an NVFP4 prefill-chunk GEMM on the tcgen05 tensor cores.
  *
@@ -9,7 +9,8 @@
  * exists"; release notes v0.6, "Native MXFP4 GGUF weight format") and the "Imparo" engine (README
  * intro: Q4_0 MoE decode with CUDA expert routing).  The pages name the formats but not their byte
  * layout; the layouts below are the public conventions (MXFP4: the OCP MX one, with the code byte
- * order of NVFP4; Q4_K: GGUF's block_q4_K, a K-quant the "Quantization" row lists).
+ * order of NVFP4; Q4_K / Q6_K: GGUF's block_q4_K / block_q6_K, the K-quants of the "Quantization"
+ * row's GGUF files).
  *
  * Conventions for every entry point
  *   - W is N x K (output x input), row-major along K; y[m][n] = sum_k x[m][k] * W[n][k].
@@ -36,7 +37,7 @@ extern "C" {
 
 typedef struct CUstream_st* qlin_stream_t; /* a cudaStream_t */
 
-typedef enum { QLIN_Q8_0 = 1, QLIN_Q4_0 = 2, QLIN_NVFP4 = 3, QLIN_MXFP4 = 4, QLIN_Q4_K = 5 } qlin_format_t;
+typedef enum { QLIN_Q8_0 = 1, QLIN_Q4_0 = 2, QLIN_NVFP4 = 3, QLIN_MXFP4 = 4, QLIN_Q4_K = 5, QLIN_Q6_K = 6 } qlin_format_t;
 typedef enum { QLIN_F32 = 0, QLIN_BF16 = 1 } qlin_dtype_t;
 typedef enum {
     QLIN_OK = 0,
@@ -88,8 +89,9 @@ enum { QLIN_OP_GEMV = 1, QLIN_OP_MOE = 2, QLIN_OP_CHUNK = 3 };
  * warp reads contiguously, followed by that tile's scales; K is padded to a multiple of 256 and N
  * to a multiple of 32 (16 per half for QLIN_PACK_GATE_UP) with zero codes and zero scales.
  * The packed size is the canonical size plus that padding (Q8_0 1.0625 B/weight, Q4_0 and NVFP4
- * 0.5625 B/weight, MXFP4 0.53125 B/weight), except Q4_K: 0.578125 B/weight against the canonical
- * 0.5625 (each sub-block's 6-bit scale and min take a 16-bit slot).  Prior art for a private re-laid-out weight copy: Imparo README intro
+ * 0.5625 B/weight, MXFP4 0.53125 B/weight), except the K-quants: Q4_K 0.578125 B/weight against the
+ * canonical 0.5625 (each sub-block's 6-bit scale and min take a 16-bit slot), Q6_K 1.078 B/weight
+ * against 0.8203 (each 6-bit code takes a byte, decoded like Q8_0).  Prior art for a private re-laid-out weight copy: Imparo README intro
  * ("private GateUp layout"); imp README "Why this exists" (an NVFP4 decode cache built at init). */
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags);
 
@@ -108,7 +110,11 @@ size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags
  *          2 bits in bits 6..7 of bytes 0..3 / 4..7), 128 bytes of codes (values 64c + l in the low
  *          nibble of byte 32c + l, values 64c + 32 + l in its high nibble); value k of sub-block
  *          j = k / 32 is d * scale_j * code - dmin * min_j; scales = NULL
- * K % 32 == 0 for Q8_0 / Q4_0 / MXFP4, K % 16 == 0 for NVFP4, K % 256 == 0 for Q4_K; N >= 1;
+ *   Q6_K : blocks = GGUF block_q6_K rows [N][K/256] x 210 B: ql[128] (low 4 code bits), qh[64]
+ *          (high 2 bits), int8 scales[16] (one per 16 values), fp16 d; value 128h + 32s + l takes
+ *          the low (s < 2) or high nibble of ql[64h + 32 (s & 1) + l], bits 2s..2s+1 of
+ *          qh[32h + l] and scales[8h + 2s + l / 16]: w = d * scale * (code - 32); scales = NULL
+ * K % 32 == 0 for Q8_0 / Q4_0 / MXFP4, K % 16 == 0 for NVFP4, K % 256 == 0 for Q4_K / Q6_K; N >= 1;
  * QLIN_PACK_GATE_UP needs N even.
  * `packed` must be 256-byte aligned and hold qlin_packed_bytes(...) bytes.  Canonical inputs
  * have no alignment requirement.  The canonical buffers may be freed once the kernel has run. */
@@ -131,7 +137,7 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
  *   flags: QLIN_EPI_* | QLIN_FLAG_PDL
  * Weights stream from HBM once; dequantization happens in registers; products and sums are fp32
  * (activations are never quantized).  Results are deterministic for a given device and shape.
- * Q8_0 / Q4_0 / Q4_K products are exact in fp32 for activations with 2^-40 <= |x| < 2^65; below that
+ * Q8_0 / Q4_0 / Q4_K / Q6_K products are exact in fp32 for activations with 2^-40 <= |x| < 2^65; below that
  * range a product is exact to 2^-63 in absolute terms, at or above it the result overflows.
  * The dequantize-and-multiply of quantized weight blocks against activations is the "NVFP4
  * block-scaled GEMM/GEMV" and "dp4a Q8_0 decode" of the imp pages (README "Features"; release
@@ -268,7 +274,8 @@ qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx,
  * QLIN_PACK_GATE_UP buffers; pass the pack_flags the buffer was packed with).  The value of every
  * weight is the exact fp32 number d*q (Q8_0), d*(q-8) (Q4_0), fp32(e2m1*e4m3*g) rounded once
  * (NVFP4), e2m1 * 2^(scale - 127) (MXFP4: exact, +-Inf where it overflows fp32), or
- * fp32(d*scale*code - dmin*min) rounded once (Q4_K: both products are exact in fp32).  A test and inspection aid; not on the hot path.  w must be 4-byte aligned. */
+ * fp32(d*scale*code - dmin*min) rounded once (Q4_K: both products are exact in fp32), or the
+ * exact d*scale*(code - 32) (Q6_K).  A test and inspection aid; not on the hot path.  w must be 4-byte aligned. */
 qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
                                  int pack_flags, float* w, qlin_stream_t stream);
 

@@ -57,6 +57,9 @@ def test_packed_bytes_sizes(lib):
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 4096, 2560) == 256 + (4096 // 32) * (2560 // 256) * 4736
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 33, 512) == 256 + 2 * 2 * 4736
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 64, 288) == 0  # K % 256
+    # Q6_K: two 4096 B byte planes of 6-bit codes + 512 B of int8 scale pairs + 128 B of per-row d
+    assert q.qlin_packed_bytes(q.QLIN_Q6_K, 4096, 2560) == 256 + (4096 // 32) * (2560 // 256) * 8832
+    assert q.qlin_packed_bytes(q.QLIN_Q6_K, 64, 288) == 0  # K % 256
     assert q.qlin_packed_bytes(7, 64, 256) == 0
     assert q.qlin_packed_bytes(q.QLIN_Q4_0, 63, 256, q.QLIN_PACK_GATE_UP) == 0  # odd N
 

@@ -83,13 +83,13 @@ def test_chain_bf16_activations(fmt, M):
         o.check()
 
 
+@pytest.mark.parametrize("fmt", [q.QLIN_Q4_K, q.QLIN_Q6_K])
 @pytest.mark.parametrize("M", [1, 2, 4, 8])
 @pytest.mark.parametrize("xdt", [torch.float32, torch.bfloat16])
-def test_chain_q4k_mlp_with_dependencies(M, xdt):
-    """Q4_K (K a multiple of 256): two gated MLP layers plus an independent projection; down
+def test_chain_kquant_mlp_with_dependencies(fmt, M, xdt):
+    """K-quants (K a multiple of 256): two gated MLP layers plus an independent projection; down
     reads its layer's SiLU output, the second layer's gate_up reads the first layer's down.  With
     bf16 activations every op writes bf16 (the next op's input)."""
-    fmt = q.QLIN_Q4_K
     ob = q.QLIN_OUT_BF16 if xdt == torch.bfloat16 else 0
     ops = []
     x = synth.activations(M, 1024, synth.gen(300), dtype=xdt).cuda()
@@ -183,13 +183,13 @@ def test_chain_argument_checks():
     assert lib.qlin_gemv_chain(fmt, q.QLIN_F32, M, ptr, 1, 0, q._dev(ws, "ws"), 16, q._stream()) == 4
 
 
-@pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_Q4_0, q.QLIN_MXFP4, q.QLIN_Q4_K])
+@pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_Q4_0, q.QLIN_MXFP4, q.QLIN_Q4_K, q.QLIN_Q6_K])
 @pytest.mark.parametrize("M", [1, 4])
 def test_chain_bf16_mlp(fmt, M):
     """A bf16 chain of gated MLPs: gate_up writes h in bf16 (QLIN_OUT_BF16), down reads it."""
     ops = []
     for l in range(2):
-        I = 512 if fmt == q.QLIN_Q4_K else 352  # Q4_K: K a multiple of 256
+        I = 512 if fmt in (q.QLIN_Q4_K, q.QLIN_Q6_K) else 352  # K-quants: K a multiple of 256
         gu = Op(fmt, 2 * I, 1024, M, 200 + l, epi=q.QLIN_EPI_SILU_GATE | q.QLIN_OUT_BF16, xdt=torch.bfloat16)
         dn = Op(fmt, 288, I, M, 210 + l, x=gu.y, wait_for=len(ops), xdt=torch.bfloat16)
         ops += [gu, dn]

@@ -13,14 +13,14 @@ import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
-FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4, q.QLIN_MXFP4, q.QLIN_Q4_K]
+FMTS = [q.QLIN_Q8_0, q.QLIN_Q4_0, q.QLIN_NVFP4, q.QLIN_MXFP4, q.QLIN_Q4_K, q.QLIN_Q6_K]
 TOL = 2e-6
 
 
 def k_ok(fmt, K):
-    """Q4_K rows are whole 256-value super-blocks: skip shapes it cannot hold."""
-    if fmt == q.QLIN_Q4_K and K % 256:
-        pytest.skip("Q4_K needs K % 256 == 0")
+    """K-quant rows are whole 256-value super-blocks: skip shapes they cannot hold."""
+    if fmt in (q.QLIN_Q4_K, q.QLIN_Q6_K) and K % 256:
+        pytest.skip("K-quants need K % 256 == 0")
 
 
 def make(fmt, N, K, seed, pack_flags=q.QLIN_PACK_DEFAULT):
@@ -146,6 +146,28 @@ def test_dequant_q4k_extreme_fields():
     packed = q.qlin_pack_weights(q.QLIN_Q4_K, N, K, blocks.cuda())
     w = q.qlin_dequant_debug(q.QLIN_Q4_K, packed, N, K).cpu().numpy()
     ref = oracle.dequant_f32(q.QLIN_Q4_K, N, K, blocks.numpy())
+    assert np.array_equal(w.view(np.uint32), ref.view(np.uint32))
+
+
+def test_dequant_q6k_extreme_fields():
+    """Q6_K super-blocks with every code 0 or 63 and int8 scales -128 / 127 / 0, d of 0, the fp16
+    maximum and the smallest subnormal: d*scale*(code-32) is exact in fp32, bit for bit."""
+    N, K = 48, 512
+    blocks, _, _ = synth.weights(q.QLIN_Q6_K, N, K, synth.gen(10))
+    b = blocks.clone().view(N, K // 256, 210)
+    fp16 = torch.tensor([0.0, 65504.0, 2.0 ** -24, 1.0], dtype=torch.float16).view(torch.uint8).view(4, 2)
+    for n in range(N):
+        b[n, :, 208:210] = fp16[n % 4]
+        if n % 3 == 0:
+            b[n, :, 0:192] = 0xFF  # every code 63
+            b[n, :, 192:208] = 0x80  # scale -128
+        elif n % 3 == 1:
+            b[n, :, 0:192] = 0  # every code 0
+            b[n, :, 192:208] = 0x7F  # scale 127
+    blocks = b.reshape(N, -1).contiguous()
+    packed = q.qlin_pack_weights(q.QLIN_Q6_K, N, K, blocks.cuda())
+    w = q.qlin_dequant_debug(q.QLIN_Q6_K, packed, N, K).cpu().numpy()
+    ref = oracle.dequant_f32(q.QLIN_Q6_K, N, K, blocks.numpy())
     assert np.array_equal(w.view(np.uint32), ref.view(np.uint32))
 
 

@@ -94,10 +94,11 @@ def test_moe_formats_small(fmt, xdt, M):
     run_and_check(ex, M, 2, logits, x)
 
 
+@pytest.mark.parametrize("fmt", [q.QLIN_Q4_K, q.QLIN_Q6_K])
 @pytest.mark.parametrize("M", [1, 8])
-def test_moe_q4k_experts(M):
-    # Q4_K experts (K a multiple of 256 for both projections): H = 512, I = 256, top-2 of 6
-    ex = Experts(q.QLIN_Q4_K, 6, 512, 256, 5500)
+def test_moe_kquant_experts(fmt, M):
+    # K-quant experts (K a multiple of 256 for both projections): H = 512, I = 256, top-2 of 6
+    ex = Experts(fmt, 6, 512, 256, 5500)
     logits = synth.router_logits(M, 6, synth.gen(5600 + M))
     x = synth.activations(M, 512, synth.gen(5700 + M))
     run_and_check(ex, M, 2, logits, x)

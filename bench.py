@@ -421,15 +421,15 @@ def run_config(name, args):
     torch.cuda.set_device(0)
     peak, peak_src = peaks()
     lines = []
-    if name == "q4_k_stack":
-        # the default stack's shapes (every K a multiple of 256) in GGUF Q4_K, one chain per step
-        fmt = q.QLIN_Q4_K
+    if name in ("q4_k_stack", "q6_k_stack"):
+        # the default stack's shapes (every K a multiple of 256) in a GGUF K-quant, one chain per step
+        fmt, fname, per256 = (q.QLIN_Q4_K, "Q4_K", 144) if name == "q4_k_stack" else (q.QLIN_Q6_K, "Q6_K", 210)
         stack = DenseStack(fmt, args.layers, mode="chain")
         graph = stack.capture(pdl=True)
         ms = time_graph(graph, args.steps, max(args.warmup, 3))
         del graph
-        canon = sum(N * K * 9 // 16 for (_, N, K, _) in STACK) * args.layers  # 144 B per 256 weights
-        lines.append(dict(workload=f"Q4_K dense decode layer stack, the Q4_0 stack's shapes ({args.layers} layers "
+        canon = sum(N * K * per256 // 256 for (_, N, K, _) in STACK) * args.layers
+        lines.append(dict(workload=f"{fname} dense decode layer stack, the Q4_0 stack's shapes ({args.layers} layers "
                           "of hidden 2560: qkv 2560->6144, o 4096->2560, gate_up 2560->2x9728 + SiLU, "
                           "down 9728->2560), one GEMV chain per step", M=1, ms_per_step=ms,
                           packed_weight_bytes=stack.weight_bytes, canonical_weight_bytes=canon,
@@ -575,7 +575,8 @@ def main():
                     help="stated: independent inputs, down reads h; serial: every projection reads the "
                          "previous one's output (reported as an extra field either way)")
     ap.add_argument("--config", default="stack",
-                    choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "chunk", "q4_k_stack"],
+                    choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "chunk", "q4_k_stack",
+                             "q6_k_stack"],
                     help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
     if args.config != "stack":

@@ -661,11 +661,12 @@ def main():
         peak, peak_src = peaks()
         gbs = whole_job_gbs(stack.step_bytes, world, ms_max)
         dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
-        traffic = None
+        traffic = None  # the committed capture's estimate holds for the default 36-layer launch only
         try:
-            with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-                key = f"{args.mode}_q4_0_m1_bytes_per_launch" if stack.chains else "gate_up_q4_0_m1_bytes_per_launch"
-                traffic = json.load(f).get(key)
+            if args.layers == LAYERS:
+                with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+                    key = f"{args.mode}_q4_0_m1_bytes_per_launch" if stack.chains else "gate_up_q4_0_m1_bytes_per_launch"
+                    traffic = json.load(f).get(key)
         except Exception:
             pass
         line = {
@@ -679,7 +680,8 @@ def main():
                        "weight_bytes_per_step": stack.weight_bytes, "algorithmic_bytes_per_step": stack.step_bytes,
                        "launches_per_step": stack.launches_per_step, "mode": args.mode,
                        "cuda_graph": True, "pdl": not args.no_pdl,
-                       "l2": "inputs larger than L2: 2.04 GB of packed weights streamed per step (L2 126 MB)",
+                       "l2": "inputs larger than L2: %.2f GB of packed weights streamed per step (L2 126 MB)"
+                             % (stack.weight_bytes / 1e9),
                        "parallelism": f"replicas{world}"},
             "roofline": {"bound": "hbm", "kernel": dom_name,
                          "achieved": dom_gbs, "peak": peak, "peak_source": f"{peak_src} hbm_gbs (copy)",

@@ -15,6 +15,10 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
                                        int top_k, const float* logits, int32_t* ids, float* wts, const void* x,
                                        int xdt, int M, float* y, float* h, int flags, void* ws, cudaStream_t s);
 extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K);
+extern "C" int64_t qlin_bf16_cache_cols(int64_t K);
+extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
+                                              int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
+                                              cudaStream_t s);
 extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
                                          float* y, int64_t ldy, void* ws, int flags, cudaStream_t s);
 extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* ws,
@@ -97,7 +101,8 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags) {
     if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
     if (pack_flags == QLIN_PACK_MMA) {
-        if (fmt != QLIN_NVFP4) return 0;
+        if (fmt != QLIN_NVFP4)  // the bf16 copy of the dequantized weights, rows of K rounded up to 64
+            return (size_t)qlin::kHdrBytes + (size_t)N * (size_t)qlin_bf16_cache_cols(K) * 2u;
         return (size_t)qlin::kHdrBytes + (size_t)((N + 255) / 256) * (size_t)((K + 255) / 256) * 36864u;
     }
     if (pack_flags & ~QLIN_PACK_GATE_UP) return 0;
@@ -111,7 +116,6 @@ qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const v
                                 void* packed, size_t packed_bytes, qlin_stream_t stream) {
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
-    if (pack_flags == QLIN_PACK_MMA && fmt != QLIN_NVFP4) return QLIN_ERR_UNSUPPORTED;
     if (pack_flags != QLIN_PACK_MMA && (pack_flags & ~QLIN_PACK_GATE_UP)) return QLIN_ERR_INVALID_ARG;
     if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
     if (!blocks || !packed) return QLIN_ERR_INVALID_ARG;
@@ -133,8 +137,8 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
         return qlin_moe_ws_bytes(fmt, M, N, K, E, top_k);
     }
     if (op == QLIN_OP_CHUNK) {
-        if (fmt != QLIN_NVFP4 || M < 1 || M > (1 << 20)) return 0;
-        return qlin_chunk_ws_bytes(M, N, K);
+        if (M < 1 || M > (1 << 20)) return 0;
+        return fmt == QLIN_NVFP4 ? qlin_chunk_ws_bytes(M, N, K) : 256;  // bf16 path: the status word
     }
     if (op == QLIN_OP_GEMV) {
         if (M < 1 || M > 8) return 0;
@@ -196,12 +200,19 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
                               int M, int64_t ldx, float* y, int64_t ldy, int flags, void* ws,
                               size_t ws_bytes, qlin_stream_t stream) {
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
-    if (fmt != QLIN_NVFP4) return QLIN_ERR_UNSUPPORTED;
     if (!valid_shape(fmt, N, K) || M < 1 || M > (1 << 20)) return QLIN_ERR_INVALID_ARG;
     if (flags & ~(QLIN_FLAG_PDL | QLIN_FLAG_CTA_PAIRS)) return QLIN_ERR_INVALID_ARG;
     if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
     if (ldx < K || ldy < N) return QLIN_ERR_INVALID_ARG;
     if (!aligned(packed, 256) || !aligned(x, 2) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
+    if (fmt != QLIN_NVFP4) {  // bf16 path: x is read by tensor-map loads (16-byte aligned rows)
+        if (flags & QLIN_FLAG_CTA_PAIRS) return QLIN_ERR_INVALID_ARG;
+        if (!aligned(x, 16) || ldx % 8) return QLIN_ERR_ALIGNMENT;
+        if (!ws || ws_bytes < 256) return QLIN_ERR_WORKSPACE;
+        if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+        return cuda_status(qlin_launch_chunk_bf16((const uint8_t*)packed + qlin::kHdrBytes, N, K, x, M, ldx, y, ldy,
+                                                  ws, flags, (cudaStream_t)stream));
+    }
     if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, N, K)) return QLIN_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
     return cuda_status(qlin_launch_chunk(packed, N, K, x, M, ldx, y, ldy, ws, flags, (cudaStream_t)stream));

@@ -251,9 +251,80 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
     }
 }
 
+// QLIN_PACK_MMA for the formats other than NVFP4: the dequantized weights as bf16 rows of Kc
+// values (K rounded up to 64, the tail zero), each the fp32 value qlin_dequant_debug gives rounded
+// to nearest-even bf16 -- the operand of the bf16 prefill-chunk GEMM.  Thread = (row, 32 values).
+template <int FMT>
+__global__ void __launch_bounds__(256) pack_bf16_kernel(const uint8_t* __restrict__ blocks,
+                                                        const uint8_t* __restrict__ scales, int64_t N, int64_t K,
+                                                        int64_t Kc, __nv_bfloat16* __restrict__ out) {
+    const int64_t nb = Kc / 32;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= N * nb) return;
+    const int64_t n = idx / nb, b = idx - n * nb, k0 = b * 32;
+    float w[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) w[j] = 0.f;
+    if (k0 < K) {
+        if (FMT == QLIN_Q8_0 || FMT == QLIN_Q4_0) {
+            const int bsz = FMT == QLIN_Q8_0 ? 34 : 18;
+            const uint8_t* blk = blocks + n * (K / 32) * bsz + b * bsz;
+            const float d = fp16_bits_to_f32(blk[0] | (blk[1] << 8));
+            for (int j = 0; j < 32; ++j) {
+                const int q = FMT == QLIN_Q8_0 ? (int)(int8_t)blk[2 + j]
+                                               : (j < 16 ? (blk[2 + j] & 0xf) : (blk[2 + j - 16] >> 4)) - 8;
+                w[j] = d * (float)q;  // exact
+            }
+        } else if (FMT == QLIN_MXFP4) {
+            const uint8_t* row = blocks + n * (K / 2) + k0 / 2;
+            const float sc = e8m0_to_f32(scales[n * (K / 32) + b]);
+            for (int j = 0; j < 32; ++j) {
+                const uint32_t h2 = e2m1x2_to_f16x2(row[j / 2]);
+                const float v = __half2float(__ushort_as_half((unsigned short)((j & 1) ? (h2 >> 16) : (h2 & 0xffff))));
+                w[j] = __fmul_rn(v, sc);  // exact unless it overflows
+            }
+        } else if (FMT == QLIN_Q4_K) {
+            const uint8_t* blk = blocks + n * (K / 256) * 144 + (k0 / 256) * 144;
+            const int p = (int)((k0 % 256) / 32);
+            const uint8_t* s12 = blk + 4;
+            const int scv = p < 4 ? (s12[p] & 63) : ((s12[p + 4] & 0xf) | ((s12[p - 4] >> 6) << 4));
+            const int mv = p < 4 ? (s12[p + 4] & 63) : ((s12[p + 4] >> 4) | ((s12[p] >> 6) << 4));
+            const float ka = fp16_bits_to_f32(blk[0] | (blk[1] << 8)) * (float)scv;  // exact
+            const float kb = fp16_bits_to_f32(blk[2] | (blk[3] << 8)) * (float)mv;   // exact
+            const uint8_t* qs = blk + 16 + 32 * (p >> 1);
+            for (int j = 0; j < 32; ++j) {
+                const int code = (p & 1) ? (qs[j] >> 4) : (qs[j] & 0xf);
+                w[j] = __fmaf_rn(ka, (float)code, -kb);  // one rounding
+            }
+        } else if (FMT == QLIN_Q6_K) {
+            const uint8_t* blk = blocks + n * (K / 256) * 210 + (k0 / 256) * 210;
+            const int p = (int)((k0 % 256) / 32), h = p >> 2, q = p & 3;
+            const uint8_t* ql = blk + 64 * h + 32 * (q & 1);
+            const uint8_t* qh = blk + 128 + 32 * h;
+            const float d = fp16_bits_to_f32(blk[208] | (blk[209] << 8));
+            const float e0 = d * (float)(int8_t)blk[192 + 8 * h + 2 * q], e1 = d * (float)(int8_t)blk[192 + 8 * h + 2 * q + 1];
+            for (int j = 0; j < 32; ++j) {
+                const int code = ((q < 2) ? (ql[j] & 0xf) : (ql[j] >> 4)) | (((qh[j] >> (2 * q)) & 3) << 4);
+                w[j] = __fmul_rn(j < 16 ? e0 : e1, (float)(code - 32));  // exact
+            }
+        }
+    }
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(w[2 * j], w[2 * j + 1]);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + n * Kc + k0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+}
+
 }  // namespace qlin
 
 using namespace qlin;
+
+extern "C" int64_t qlin_bf16_cache_cols(int64_t K);
 
 extern "C" cudaError_t qlin_launch_pack_mma(const void* codes, const void* scales, int64_t N, int64_t K, float gs,
                                             void* packed, cudaStream_t s);
@@ -264,7 +335,19 @@ extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void*
     if (pack_flags == QLIN_PACK_MMA) {
         write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags, gs,
                                              (int32_t)((N + 255) / 256), (int32_t)((K + 255) / 256));
-        return qlin_launch_pack_mma(blocks, scales, N, K, gs, packed, s);
+        if (fmt == QLIN_NVFP4) return qlin_launch_pack_mma(blocks, scales, N, K, gs, packed, s);
+        const int64_t Kc = qlin_bf16_cache_cols(K);
+        const int64_t threads = N * (Kc / 32);
+        const dim3 grid((unsigned)((threads + 255) / 256));
+        const uint8_t* bl = (const uint8_t*)blocks;
+        const uint8_t* sc = (const uint8_t*)scales;
+        __nv_bfloat16* out = (__nv_bfloat16*)((uint8_t*)packed + kHdrBytes);
+        if (fmt == QLIN_Q8_0) pack_bf16_kernel<QLIN_Q8_0><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        else if (fmt == QLIN_Q4_0) pack_bf16_kernel<QLIN_Q4_0><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        else if (fmt == QLIN_MXFP4) pack_bf16_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        else if (fmt == QLIN_Q4_K) pack_bf16_kernel<QLIN_Q4_K><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        else pack_bf16_kernel<QLIN_Q6_K><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        return cudaGetLastError();
     }
     Geometry geo = geometry(fmt, N, K, pack_flags);
     const int gu = (pack_flags & QLIN_PACK_GATE_UP) ? 1 : 0;

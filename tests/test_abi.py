@@ -53,6 +53,9 @@ def test_packed_bytes_sizes(lib):
     # MXFP4: codes as NVFP4, one scale byte per 32 values: 4096 + 256 bytes per 32 x 256 unit
     assert q.qlin_packed_bytes(q.QLIN_MXFP4, 4096, 2560) == 256 + 4096 * 2560 * 17 // 32
     assert q.qlin_packed_bytes(q.QLIN_MXFP4, 64, 272) == 0  # K % 32
+    # QLIN_PACK_MMA for the GGUF / MXFP4 formats: the bf16 copy, rows of K rounded up to 64
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 100, 96, q.QLIN_PACK_MMA) == 256 + 100 * 128 * 2
+    assert q.qlin_packed_bytes(q.QLIN_Q6_K, 64, 512, q.QLIN_PACK_MMA) == 256 + 64 * 512 * 2
     # Q4_K: 4096 B of codes + 512 B of sub-block scale/min slots + 128 B of per-row d/dmin per unit
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 4096, 2560) == 256 + (4096 // 32) * (2560 // 256) * 4736
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 33, 512) == 256 + 2 * 2 * 4736
@@ -93,7 +96,8 @@ def test_pack_argument_checks(lib):
     assert f(2, 64, 256, P(0), None, 1.0, 0, P(0x1000), 1 << 30, None) == 1
     assert f(3, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # NVFP4 needs scales
     assert f(4, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # MXFP4 needs scales
-    assert f(4, 64, 256, P(0x1000), P(0x2000), 1.0, 2, P(0x10000), 1 << 30, None) == 2  # no MMA layout
+    assert f(4, 64, 256, P(0x1000), P(0x2000), 1.0, 3, P(0x10000), 1 << 30, None) == 1  # no gate_up MMA form
+    assert f(2, 64, 256, P(0x1000), None, 1.0, 2, P(0x10000), 256 + 64 * 256, None) == 1  # bf16 copy needs 2 B/w
     assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10010), 1 << 30, None) == 3
     assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 10, None) == 1
     assert f(2, 64, 256, P(0x1000), None, 1.0, 8, P(0x10000), 1 << 30, None) == 1

@@ -1,0 +1,125 @@
+"""GPU parity of the prefill-chunk GEMM for the GGUF and MXFP4 formats (the bf16 path).
+
+qlin_pack_weights(QLIN_PACK_MMA) builds a bf16 copy of the dequantized weights: every weight is the
+fp32 value the oracle's dequant gives, rounded to nearest-even bf16 (torch's conversion is the
+reference rounding) -- checked bit for bit, tail columns zero.  qlin_gemm_chunk then multiplies bf16
+x by that copy on the tensor cores with fp32 accumulation: checked against the fp64 product with
+the same bf16 weights (|y - ref| <= 2 K 2^-24 sum|x w_bf16|: the fp32 summation bound, with one ulp
+per addition allowed for the tensor core's order and rounding) and against the
+unrounded weights within the chunk path's 1e-2 sum|x w| bound.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gemm_dequant_gemv_q8_b200 as q
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [q.QLIN_Q4_0, q.QLIN_Q8_0, q.QLIN_MXFP4, q.QLIN_Q4_K, q.QLIN_Q6_K]
+
+
+def kquant(fmt):
+    return fmt in (q.QLIN_Q4_K, q.QLIN_Q6_K)
+
+
+def make(fmt, N, K, seed):
+    blocks, scales, g = synth.weights(fmt, N, K, synth.gen(seed))
+    packed = q.qlin_pack_weights(fmt, N, K, blocks.cuda(), None if scales is None else scales.cuda(), g,
+                                 q.QLIN_PACK_MMA)
+    w32 = oracle.dequant_f32(fmt, N, K, blocks.numpy(), None if scales is None else scales.numpy(), g)
+    return packed, w32
+
+
+def cache(packed, N, K):
+    kc = (K + 63) // 64 * 64
+    return packed[256:256 + N * kc * 2].view(torch.bfloat16).view(N, kc), kc
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K", [(40, 256), (33, 96), (300, 2560)])
+def test_bf16_cache_bit_exact(fmt, N, K):
+    if kquant(fmt) and K % 256:
+        pytest.skip("K-quants need K % 256 == 0")
+    packed, w32 = make(fmt, N, K, 900 + N)
+    assert packed.numel() == q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA)
+    wb, kc = cache(packed, N, K)
+    ref = torch.from_numpy(w32).to(torch.bfloat16)
+    got = wb[:, :K].cpu()
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
+    assert (wb[:, K:].cpu().float() == 0).all()
+
+
+def check(y, x, w32, tol_exact=1e-2):
+    xd = x.double().cpu().numpy()
+    wb = torch.from_numpy(w32).to(torch.bfloat16).double().numpy()
+    ref = xd @ wb.T
+    A = np.abs(xd) @ np.abs(wb).T
+    K = xd.shape[1]
+    err = np.abs(y.double().cpu().numpy() - ref)
+    bound = 2 * K * 2.0 ** -24 * A + 1e-30
+    assert (err <= bound).all(), float(np.max(err / bound))
+    exact = xd @ w32.astype(np.float64).T
+    A0 = np.abs(xd) @ np.abs(w32.astype(np.float64)).T
+    assert (np.abs(y.double().cpu().numpy() - exact) <= tol_exact * A0 + 1e-30).all()
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (64, 300, 512), (200, 520, 2560), (513, 1000, 1024),
+                                   (37, 70, 96)])
+def test_chunk_bf16_parity(fmt, M, N, K):
+    if kquant(fmt) and K % 256:
+        pytest.skip("K-quants need K % 256 == 0")
+    packed, w32 = make(fmt, N, K, 1000 + M)
+    x = synth.activations(M, K, synth.gen(1100 + M), dtype=torch.bfloat16).cuda()
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+    y = q.qlin_gemm_chunk(fmt, packed, N, K, x, ws=ws)
+    torch.cuda.synchronize()
+    assert q.qlin_ws_status(ws) == 0
+    check(y, x, w32)
+
+
+def test_chunk_bf16_strided_operands_and_reuse():
+    fmt, M, N, K = q.QLIN_Q4_0, 150, 264, 768
+    packed, w32 = make(fmt, N, K, 77)
+    xb = synth.activations(M, K + 40, synth.gen(78), dtype=torch.bfloat16).cuda()  # ldx = K + 40 (8-aligned)
+    x = xb[:, :K]
+    y = torch.full((M, N + 5), float("nan"), device="cuda")
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+    for _ in range(2):
+        q.qlin_gemm_chunk(fmt, packed, N, K, x, y=y[:, :N], ws=ws)
+    torch.cuda.synchronize()
+    assert q.qlin_ws_status(ws) == 0
+    check(y[:, :N], x, w32)
+    assert torch.isnan(y[:, N:]).all()
+
+
+def test_chunk_bf16_full_size_sampled():
+    # a prefill chunk of the Q4_0 4B stack's gate_up: M = 512, K = 2560, N = 2 x 9728; sampled rows
+    fmt, M, N, K = q.QLIN_Q4_0, 512, 19456, 2560
+    blocks, _, _ = synth.weights(fmt, N, K, synth.gen(4242))
+    packed = q.qlin_pack_weights(fmt, N, K, blocks.cuda(), pack_flags=q.QLIN_PACK_MMA)
+    x = synth.activations(M, K, synth.gen(4243), dtype=torch.bfloat16).cuda()
+    y = q.qlin_gemm_chunk(fmt, packed, N, K, x)
+    torch.cuda.synchronize()
+    rows = np.unique(np.linspace(0, N - 1, 61).astype(np.int64))
+    w32 = oracle.dequant_f32(fmt, N, K, blocks.numpy())[rows]
+    check(y[:, rows], x, w32)
+
+
+def test_chunk_bf16_argument_checks():
+    fmt, M, N, K = q.QLIN_Q8_0, 8, 64, 256
+    packed, _ = make(fmt, N, K, 5)
+    lib = q.lib()
+    ws = q.workspace(256)
+    xb = torch.zeros(M, K + 4, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(M, N, device="cuda")
+    # ldx not a multiple of 8: the tensor-map rows would not be 16-byte aligned
+    st = lib.qlin_gemm_chunk(fmt, q._dev(packed, "p"), N, K, q._dev(xb, "x"), M, K + 4, q._dev(y, "y"), N, 0,
+                             q._dev(ws, "ws"), 256, q._stream(None))
+    assert st == 3  # QLIN_ERR_ALIGNMENT
+    st = lib.qlin_gemm_chunk(fmt, q._dev(packed, "p"), N, K, q._dev(xb, "x"), M, K + 4, q._dev(y, "y"), N,
+                             q.QLIN_FLAG_CTA_PAIRS, q._dev(ws, "ws"), 256, q._stream(None))
+    assert st == 1  # QLIN_ERR_INVALID_ARG: CTA pairs are an NVFP4-path option

@@ -529,6 +529,32 @@ def run_config(name, args):
                               "gate_up 2048->2x1792, down 1792->2048, top-4; a graph of 8 layers' launches "
                               "(distinct weights)", M=M, distinct_experts=nd,
                               us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9))
+    if name == "gguf_chunk":
+        # GGUF prefill chunk: the bf16 copy of dequantized Q4_0 weights (QLIN_PACK_MMA) times bf16 x on
+        # the tensor cores (kind::f16), at the NVFP4 chunk workload's shape
+        fmt, N, K = q.QLIN_Q4_0, 17408, 5120
+        packs = []
+        for c in range(2):  # two copies (2 x 178 MB) so consecutive calls do not find the weights in L2
+            b, _, _ = synth.weights(fmt, N, K, synth.gen(7100 + c, device="cuda"), device="cuda")
+            packs.append(q.qlin_pack_weights(fmt, N, K, b, None, 1.0, q.QLIN_PACK_MMA))
+            del b
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                bf16_peak, bf16_src = float(json.load(f)["bf16_tflops"]), "measured bf16 burst (cuBLAS)"
+        except Exception:
+            bf16_peak, bf16_src = 1590.0, "fallback bf16"
+        for M in (512, 64):
+            x = synth.activations(M, K, synth.gen(7200 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
+            y = torch.empty(M, N, device="cuda")
+            ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+            fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL) for c in range(2)]
+            ms = _time_graph_of(fn, args.steps, args.warmup) / 2
+            flop = 2.0 * M * N * K
+            bytes_ = N * K * 2 + 2 * M * K + 4 * M * N
+            lines.append(dict(workload=f"Q4_0 prefill-chunk GEMM M={M} K=5120 N=17408 (bf16 copy of the dequantized "
+                              "weights x bf16 activations, tcgen05 kind::f16, one launch)", M=M, us_per_call=ms * 1e3,
+                              tflops=flop / (ms * 1e-3) / 1e12, bf16_peak_tflops=bf16_peak, bf16_peak_source=bf16_src,
+                              bf16_frac=flop / (ms * 1e-3) / 1e12 / bf16_peak, gbs=bytes_ / (ms * 1e-3) / 1e9))
     if name == "chunk":
         fmt, N, K = q.QLIN_NVFP4, 17408, 5120
         b, s_, g = synth.weights(fmt, N, K, synth.gen(7000, device="cuda"), device="cuda")
@@ -576,7 +602,7 @@ def main():
                          "previous one's output (reported as an extra field either way)")
     ap.add_argument("--config", default="stack",
                     choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "chunk", "q4_k_stack",
-                             "q6_k_stack"],
+                             "q6_k_stack", "gguf_chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
     args = ap.parse_args()
     if args.config != "stack":

@@ -73,9 +73,14 @@ enum {
     QLIN_PACK_DEFAULT = 0,
     QLIN_PACK_GATE_UP = 1, /* the N rows are [gate ; up] halves (N even): each packed tile pairs
                              16 gate rows with their 16 up rows so the SiLU-gate epilogue fuses */
-    QLIN_PACK_MMA = 2      /* NVFP4 only: the tensor-core operand layout of qlin_gemm_chunk (tiles of
-                             256 rows x 256 values, 128-byte-swizzled K-major codes, scale factors
-                             in 512-byte atoms); 0.5625 B/weight plus padding to 256 x 256 */
+    QLIN_PACK_MMA = 2      /* the weight operand of qlin_gemm_chunk.  NVFP4: the tensor-core layout
+                             (tiles of 256 rows x 256 values, 128-byte-swizzled K-major codes, scale
+                             factors in 512-byte atoms), 0.5625 B/weight plus padding to 256 x 256.
+                             Q8_0 / Q4_0 / MXFP4 / Q4_K / Q6_K: a bf16 copy of the dequantized
+                             weights, row-major N x roundup(K, 64) after the 256-byte header, each
+                             weight the fp32 value of qlin_dequant_debug rounded to nearest-even
+                             bf16, the tail columns zero (2 B/weight: the full-precision prefill
+                             copy; imp README "Why this exists": prefill via source dequant) */
 };
 
 /* qlin_workspace_bytes ops */
@@ -243,8 +248,9 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
 
 /* ------------------------------------------------------------------------- prefill-chunk GEMM */
 
-/* NVFP4 GEMM for prefill chunks (M rows of bf16 activations, M >= 1; built for M >= 64) on the
- * tcgen05 tensor cores.  The counterpart on the pages is imp's NVFP4 block-scaled GEMM for
+/* GEMM for prefill chunks (M rows of bf16 activations, M >= 1; built for M >= 64) on the tcgen05
+ * tensor cores.  NVFP4 weights take the block-scaled FP4 path described here; the other formats
+ * the bf16 path described after it.  The counterpart on the pages is imp's NVFP4 block-scaled GEMM for
  * prefill (README "Features", row "sm_120a kernels": block-scaled mxf4nvf4 MMA, there with
  * mma.sync for sm_120a).  One persistent launch on `stream`, two steps:
  *   1. quantize x to NVFP4 (the A operand), all in fp32 with round-to-nearest-even:
@@ -258,8 +264,12 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
  *   y: fp32, row stride ldy (16-byte aligned y and ldy % 4 == 0 take the TMA-store epilogue);
  *   flags: QLIN_FLAG_PDL and/or QLIN_FLAG_CTA_PAIRS;
  *   ws: qlin_workspace_bytes(QLIN_OP_CHUNK, QLIN_NVFP4, M, N, K, 0, 0) bytes.
- * Other formats return QLIN_ERR_UNSUPPORTED.  Bounded device waits: a timeout sets the workspace
- * status word (qlin_ws_status). */
+ * bf16 path (Q8_0, Q4_0, MXFP4, Q4_K, Q6_K): y[m][n] = sum_k x[m][k] * Wb[n][k] with Wb the bf16
+ * copy written by qlin_pack_weights(fmt, N, K, ..., QLIN_PACK_MMA), tcgen05.mma kind::f16 (bf16
+ * operands loaded by tensor-map copies, fp32 accumulation in tensor memory); x must be 16-byte
+ * aligned with ldx % 8 == 0 (else QLIN_ERR_ALIGNMENT); QLIN_FLAG_CTA_PAIRS is not accepted;
+ * ws: qlin_workspace_bytes(QLIN_OP_CHUNK, fmt, M, N, K, 0, 0) bytes (256: the status word).
+ * Bounded device waits: a timeout sets the workspace status word (qlin_ws_status). */
 qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,
                               int M, int64_t ldx, float* y, int64_t ldy, int flags, void* ws,
                               size_t ws_bytes, qlin_stream_t stream);

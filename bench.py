@@ -543,16 +543,19 @@ def run_config(name, args):
                 bf16_peak, bf16_src = float(json.load(f)["bf16_tflops"]), "measured bf16 burst (cuBLAS)"
         except Exception:
             bf16_peak, bf16_src = 1590.0, "fallback bf16"
-        for M in (512, 64):
+        for M, pairs in ((512, True), (512, False), (64, False)):
             x = synth.activations(M, K, synth.gen(7200 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
             y = torch.empty(M, N, device="cuda")
             ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
-            fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL) for c in range(2)]
+            fl = q.QLIN_FLAG_PDL | (q.QLIN_FLAG_CTA_PAIRS if pairs else 0)
+            fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=fl) for c in range(2)]
             ms = _time_graph_of(fn, args.steps, args.warmup) / 2
             flop = 2.0 * M * N * K
             bytes_ = N * K * 2 + 2 * M * K + 4 * M * N
+            tiling = "256 x 256 tiles on CTA pairs" if pairs else "128 x 256 tiles on single CTAs"
             lines.append(dict(workload=f"Q4_0 prefill-chunk GEMM M={M} K=5120 N=17408 (bf16 copy of the dequantized "
-                              "weights x bf16 activations, tcgen05 kind::f16, one launch)", M=M, us_per_call=ms * 1e3,
+                              f"weights x bf16 activations, tcgen05 kind::f16, one launch, {tiling})", M=M,
+                              cta_pairs=pairs, us_per_call=ms * 1e3,
                               tflops=flop / (ms * 1e-3) / 1e12, bf16_peak_tflops=bf16_peak, bf16_peak_source=bf16_src,
                               bf16_frac=flop / (ms * 1e-3) / 1e12 / bf16_peak, gbs=bytes_ / (ms * 1e-3) / 1e9))
     if name == "chunk":

@@ -206,7 +206,6 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
     if (ldx < K || ldy < N) return QLIN_ERR_INVALID_ARG;
     if (!aligned(packed, 256) || !aligned(x, 2) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
     if (fmt != QLIN_NVFP4) {  // bf16 path: x is read by tensor-map loads (16-byte aligned rows)
-        if (flags & QLIN_FLAG_CTA_PAIRS) return QLIN_ERR_INVALID_ARG;
         if (!aligned(x, 16) || ldx % 8) return QLIN_ERR_ALIGNMENT;
         if (!ws || ws_bytes < 256) return QLIN_ERR_WORKSPACE;
         if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;

@@ -7,14 +7,21 @@
 // (README "Why this exists") and runs its prefill GEMMs on the tensor cores; here the dequantized
 // copy is bf16 and the GEMM is tcgen05.mma kind::f16 with TMEM accumulators.
 //
-// One launch, persistent CTAs (at most one per SM), 128 x 256 output tiles, K in stages of 64:
-//   warp 0   : producer -- two TMA tensor loads per stage (x: 128 rows x 64 values, the bf16
-//              weights: 256 rows x 64 values, both 128-byte swizzled by the tensor maps) into a
-//              4-stage ring; rows and columns outside the tensors read as zero;
-//   warp 1   : one thread issues the stage's four M128 N256 K16 MMAs, commits the stage back to the
-//              producer and, after the tile's last stage, the accumulator to the epilogue;
-//   warps 2-5: epilogue -- tcgen05.ld of the 128 x 256 fp32 accumulator (one TMEM lane quarter
-//              each), released to the MMAs once read, stored to y through a transpose buffer.
+// One launch, persistent CTAs (at most one per SM), K in stages of 64, tiles of 128 x 256 (CG = 1)
+// or 256 x 256 per pair of CTAs (CG = 2, cta_group::2: each CTA stages its 128 activation rows and
+// half of the 256 weight rows, so each SM writes and the MMA reads 32 KB of shared memory per
+// stage instead of 48 KB):
+//   warp 0   : producer -- two TMA tensor loads per stage (x rows and weight rows, 64 values each,
+//              128-byte swizzled by the tensor maps) into the ring; rows and columns outside the
+//              tensors read as zero.  With CG = 2 both CTAs' loads complete on the first CTA's
+//              stage barrier (the .cta_group::2 form), which alone tracks a stage's bytes;
+//   warp 1   : one thread (of the first CTA) issues the stage's four M128/M256 N256 K16 MMAs,
+//              commits the stage back to the producers (both CTAs) and, after the tile's last
+//              stage, the accumulator to the epilogues;
+//   warps 2-5: epilogue -- tcgen05.ld of this CTA's 128 x 256 fp32 accumulator rows (one TMEM lane
+//              quarter each), released to the MMAs once read, stored to y through a transpose buffer.
+// Tensor memory holds two accumulators, used by alternate tiles, so a tile's drain overlaps the next
+// tile's MMAs.
 // Every wait is bounded; a timeout sets the status word and the CTA winds down.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -25,19 +32,23 @@ namespace qlin {
 
 namespace cb {
 
-constexpr int kRows = 128;          // activation rows per tile (MMA M)
+constexpr int kRows = 128;          // activation rows per CTA (MMA M per CTA)
 constexpr int kCols = 256;          // weight rows per tile (MMA N)
 constexpr int kKStage = 64;         // K per stage: one 128-byte swizzle span of bf16
 constexpr int kABytes = kRows * 128;
-constexpr int kBBytes = kCols * 128;
-constexpr int kStageBytes = kABytes + kBBytes;  // 48 KB
-constexpr int kStages = 4;
 constexpr int kEpiWarps = 4, kFirstEpi = 2;
 constexpr int kThreads = (kFirstEpi + kEpiWarps) * 32;
 constexpr int kEpiBuf = 32 * 64;  // one warp's 32 x 16 fp32 transpose buffer
-constexpr int kTmemCols = 256;
-constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiWarps * kEpiBuf + 256;
-static_assert(kSmem <= 232448, "shared memory budget");
+constexpr int kTmemCols = 512;  // two 256-column accumulators: the next tile's MMAs run while one drains
+template <int CG>
+struct Cfg {
+    static constexpr int kBRows = kCols / CG;                 // weight rows staged by this CTA
+    static constexpr int kBBytes = kBRows * 128;
+    static constexpr int kStageBytes = kABytes + kBBytes;    // 48 KB (CG = 1) or 32 KB (CG = 2)
+    static constexpr int kStages = CG == 1 ? 4 : 6;
+    static constexpr int kSmem = 1024 + kStages * kStageBytes + kEpiWarps * kEpiBuf + 256;
+};
+static_assert(Cfg<1>::kSmem <= 232448 && Cfg<2>::kSmem <= 232448, "shared memory budget");
 
 struct Args {
     float* y;
@@ -64,19 +75,73 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
+// CTA pairs: the load lands in this CTA's shared memory and completes on the barrier at the same
+// offset in the pair's first CTA (no multicast: each CTA loads its own rows).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        "{\n .reg .b32 rb;\n mapa.shared::cluster.u32 rb, %4, 0;\n"
+        " cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [rb];\n}\n" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
 
+__device__ __forceinline__ uint32_t cta_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on the mbarrier at the same offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
+    asm volatile(
+        "{\n .reg .b32 ra;\n mapa.shared::cluster.u32 ra, %0, %1;\n"
+        " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}\n" ::"r"(smem_u32(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+template <int CG>
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    if constexpr (CG == 1)
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+
+// Commit this thread's MMAs to the barrier at `bar` (CG = 2: in both CTAs of the pair).
+template <int CG>
 __device__ __forceinline__ void commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
+    if constexpr (CG == 1)
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                     : "memory");
+    else
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                smem_u32(bar)),
+            "h"((uint16_t)3)
+            : "memory");
+}
+// Commit to this CTA's own barrier only.
+template <int CG>
+__device__ __forceinline__ void commit_self(uint64_t* bar) {
+    if constexpr (CG == 1)
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                     : "memory");
+    else
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                     : "memory");
 }
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -103,53 +168,69 @@ __device__ __forceinline__ void mbar_arrive_local(uint64_t* bar) {
 
 }  // namespace cb
 
+template <int CG>
 __global__ void __launch_bounds__(cb::kThreads, 1)
     chunk_bf16_kernel(const cb::Args a, const __grid_constant__ CUtensorMap xmap,
                       const __grid_constant__ CUtensorMap wmap) {
     using namespace cb;
-    constexpr int S = kStages;
+    using C = Cfg<CG>;
+    constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* epi = smem + S * kStageBytes;
+    uint8_t* epi = smem + S * C::kStageBytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(epi + kEpiWarps * kEpiBuf);
     uint64_t* empty = full + S;
-    uint64_t* acc_full = empty + S;
-    uint64_t* acc_empty = acc_full + 1;
-    uint64_t* mma_done = acc_empty + 1;
+    uint64_t* acc_full = empty + S;     // [2]: accumulator b holds a finished tile
+    uint64_t* acc_empty = acc_full + 2;  // [2]: accumulator b has been read
+    uint64_t* mma_done = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     volatile int* issued = abort_flag + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = CG == 1 ? 0u : cta_rank();  // rank 0 issues the pair's MMAs
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1);  // CG = 2: rank 0's counts the bytes of both CTAs
             mbar_init(&empty[s], 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], kEpiWarps * CG);  // the epilogue warps of every CTA of the group
+        }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         *issued = 0;
         fence_mbar_init();
     }
     if (warp == 0) {  // the whole warp allocates (and later frees) the accumulator columns
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                     "r"(kTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        if constexpr (CG == 1) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_holder)),
+                         "r"(kTmemCols));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_holder)),
+                         "r"(kTmemCols));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+        }
     }
     fence_before();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync();  // the pair's barriers exist before either CTA signals the other
     fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int ntiles = a.TM * a.TN;
+    const int ntiles = a.TM * a.TN;  // TM: tiles of 128 * CG activation rows
+    const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
     griddep_wait();  // x comes from the previous kernels
 
     if (warp == 0) {
         if (lane == 0) {
             int it = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
-                const int tn = tile / a.TM, tm = tile % a.TM;  // CTAs at work together share weight tiles
+            for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
+                const int tn = tile / a.TM, tm = tile % a.TM;  // groups at work together share weight tiles
+                const int xrow = (tm * CG + (int)rank) * kRows, wrow = tn * kCols + (int)rank * C::kBRows;
                 for (int ks = 0; ks < a.KS; ++ks, ++it) {
                     const int s = it % S;
                     if (it >= S && !mbar_wait_bounded(&empty[s], ((it / S) - 1) & 1)) {
@@ -157,29 +238,37 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
                         *abort_flag = 1;
                         break;
                     }
-                    uint8_t* st = smem + s * kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], kStageBytes);
-                    tma_load_2d(st, &xmap, ks * kKStage, tm * kRows, &full[s]);
-                    tma_load_2d(st + kABytes, &wmap, ks * kKStage, tn * kCols, &full[s]);
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    if constexpr (CG == 1) {
+                        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                        tma_load_2d(st, &xmap, ks * kKStage, xrow, &full[s]);
+                        tma_load_2d(st + kABytes, &wmap, ks * kKStage, wrow, &full[s]);
+                    } else {
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+                        tma_load_2d_pair(st, &xmap, ks * kKStage, xrow, &full[s]);
+                        tma_load_2d_pair(st + kABytes, &wmap, ks * kKStage, wrow, &full[s]);
+                    }
                     *issued = it + 1;
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // bf16 x bf16 -> fp32, both operands K-major, M = 128, N = 256
+        if (lane == 0 && rank == 0) {
+            // bf16 x bf16 -> fp32, both operands K-major, M = 128 * CG, N = 256
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kCols >> 3) << 17) |
-                                   ((uint32_t)(kRows >> 4) << 24);
+                                   ((uint32_t)((kRows * CG) >> 4) << 24);
             int it = 0, tcount = 0;
-            for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++tcount) {
-                if (tcount > 0) {
-                    if (!mbar_wait_bounded(acc_empty, (tcount - 1) & 1)) {
+            for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep, ++tcount) {
+                const int ab = tcount & 1;  // accumulator of this tile
+                if (tcount >= 2) {          // its previous tile (tcount - 2) has been read out
+                    if (!mbar_wait_bounded(&acc_empty[ab], ((tcount - 2) >> 1) & 1)) {
                         atomicOr(a.status, 1u);
                         *abort_flag = 1;
                         break;
                     }
                     fence_after();
                 }
+                const uint32_t dacc = tmem + (uint32_t)(ab * kCols);
                 bool ok = true;
                 for (int ks = 0; ks < a.KS; ++ks, ++it) {
                     const int s = it % S;
@@ -188,46 +277,52 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
                         break;
                     }
                     fence_after();
-                    const uint32_t sa = smem_u32(smem + s * kStageBytes), sb = sa + kABytes;
+                    const uint32_t sa = smem_u32(smem + s * C::kStageBytes), sb = sa + kABytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // K = 16 per MMA: 32 bytes along the swizzled row
-                        mma_bf16(tmem, sdesc_sw128(sa + kk * 32), sdesc_sw128(sb + kk * 32), idesc,
-                                 (ks > 0 || kk > 0) ? 1u : 0u);
-                    commit(&empty[s]);
+                        mma_bf16<CG>(dacc, sdesc_sw128(sa + kk * 32), sdesc_sw128(sb + kk * 32), idesc,
+                                     (ks > 0 || kk > 0) ? 1u : 0u);
+                    commit<CG>(&empty[s]);  // frees the stage in every CTA of the group
                 }
                 if (!ok) {
                     atomicOr(a.status, 1u);
                     *abort_flag = 1;
                     break;
                 }
-                commit(acc_full);
+                commit<CG>(&acc_full[ab]);
             }
-            commit(mma_done);  // every tcgen05 operation of this thread completes before teardown
+            commit_self<CG>(mma_done);  // every tcgen05 operation of this thread completes before teardown
             if (!mbar_wait_bounded(mma_done, 0)) atomicOr(a.status, 1u);
         }
-    } else {  // epilogue: TMEM lane quarter = warp % 4, all 256 columns
+    } else {  // epilogue: TMEM lane quarter = warp % 4, all 256 columns of this CTA's 128 rows
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         uint8_t* tb = epi + (warp - kFirstEpi) * kEpiBuf;
         int tcount = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
-            if (*abort_flag || !mbar_wait_bounded(acc_full, tcount & 1)) {
+        for (int tile = tile0; tile < ntiles; tile += tstep, ++tcount) {
+            const int ab = tcount & 1;
+            if (*abort_flag || !mbar_wait_bounded(&acc_full[ab], (tcount >> 1) & 1)) {
                 if (lane == 0) atomicOr(a.status, 1u);
                 *abort_flag = 1;
                 break;
             }
             fence_after();
             const int tn = tile / a.TM, tm = tile % a.TM;
-            const int m0 = tm * kRows + q * 32;  // this warp's first row
+            const int m0 = (tm * CG + (int)rank) * kRows + q * 32;  // this warp's first row
             const int64_t n0 = (int64_t)tn * kCols;
 #pragma unroll 1
             for (int c = 0; c < kCols; c += 32) {
                 float v[32];
-                ld32(tmem + lane_base + (uint32_t)c, v);
+                ld32(tmem + lane_base + (uint32_t)(ab * kCols + c), v);
                 if (c == kCols - 32) {  // this warp's columns are read: release the accumulator
                     fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_local(acc_empty);
+                    if (lane == 0) {
+                        if (CG == 1 || rank == 0)
+                            mbar_arrive_local(&acc_empty[ab]);
+                        else
+                            mbar_arrive_remote(&acc_empty[ab], 0);
+                    }
                 }
                 if (m0 >= a.M || n0 + c >= a.N) continue;
                 // Transpose through shared memory so that each store instruction writes 8 rows x
@@ -264,13 +359,27 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
     __syncthreads();
     if (warp == 0 && lane == 0 && *abort_flag) {
         // wait (bounded) for the last tensor loads issued to land before shared memory is released
+        // (CG = 2: they complete on rank 0's barriers; rank 1 waits out the same bound instead)
         const int n_it = *issued;
-        for (int j = n_it > S ? n_it - S : 0; j < n_it; ++j) mbar_wait_bounded(&full[j % S], (j / S) & 1, 50000000ull);
+        for (int j = n_it > S ? n_it - S : 0; j < n_it; ++j) {
+            if (CG == 1 || rank == 0)
+                mbar_wait_bounded(&full[j % S], (j / S) & 1, 50000000ull);
+        }
+        if (CG == 2 && rank != 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < 50000000ull) __nanosleep(1000);
+        }
     }
+    // CG = 2: the pair's MMAs read both CTAs' shared memory and write both CTAs' tensor memory;
+    // neither CTA frees either before the issuing CTA has seen them complete (mma_done above).
+    if constexpr (CG == 2) cluster_sync();
     if (warp == 0) {
         __syncwarp();
         fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+        if constexpr (CG == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+        else
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
 
@@ -311,28 +420,74 @@ static bool make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int6
 // Columns of the bf16 weight copy: K rounded up to whole 64-value stages (zero-filled).
 extern "C" int64_t qlin_bf16_cache_cols(int64_t K) { return (K + cb::kKStage - 1) / cb::kKStage * cb::kKStage; }
 
-// wb: the bf16 weights [N][qlin_bf16_cache_cols(K)] (after the 256-byte header of the packed buffer);
-// x: bf16 [M][K] with row pitch ldx (16-byte aligned base, ldx % 8 == 0, checked by the caller).
-extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
-                                              int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
-                                              cudaStream_t s) {
+template <int CG>
+static cudaError_t launch_bf16_cg(const cb::Args& a, const CUtensorMap& xmap, const CUtensorMap& wmap, int flags,
+                                  cudaStream_t s) {
+    using C = cb::Cfg<CG>;
     static bool attr_set = false;
+    static int max_units = 0, cached_dev = -1;  // CTAs (CG = 1) or pairs (CG = 2) resident at once
     cudaError_t e;
     if (!attr_set) {
-        e = cudaFuncSetAttribute(chunk_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cb::kSmem);
+        e = cudaFuncSetAttribute(chunk_bf16_kernel<CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    int dev = 0, sms = 0;
+    int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (CG == 2) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.blockDim = dim3(cb::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    if (cached_dev != dev) {
+        int sms = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        int units = sms;
+        if (CG == 2) {
+            cfg.gridDim = dim3((unsigned)(sms & ~1));
+            cfg.numAttrs = na;
+            int clusters = 0;
+            if ((e = cudaOccupancyMaxActiveClusters(&clusters, chunk_bf16_kernel<CG>, &cfg)) != cudaSuccess) return e;
+            if (clusters < 1) return cudaErrorInvalidConfiguration;
+            units = clusters;
+        }
+        max_units = units;
+        cached_dev = dev;
+    }
+    const int ntiles = a.TM * a.TN;
+    cfg.gridDim = dim3((unsigned)((ntiles < max_units ? ntiles : max_units) * CG));
+    if (flags & QLIN_FLAG_PDL) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, chunk_bf16_kernel<CG>, a, xmap, wmap);
+}
+
+// wb: the bf16 weights [N][qlin_bf16_cache_cols(K)] (after the 256-byte header of the packed buffer);
+// x: bf16 [M][K] with row pitch ldx (16-byte aligned base, ldx % 8 == 0, checked by the caller).
+// QLIN_FLAG_CTA_PAIRS with M > 128: 256 x 256 tiles on pairs of CTAs.
+extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
+                                              int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
+                                              cudaStream_t s) {
+    const int cg = (flags & QLIN_FLAG_CTA_PAIRS) && M > cb::kRows ? 2 : 1;
     cb::Args a;
     a.y = y;
     a.ldy = ldy;
     a.M = M;
     a.N = N;
     a.K = K;
-    a.TM = (M + cb::kRows - 1) / cb::kRows;
+    a.TM = (M + cb::kRows * cg - 1) / (cb::kRows * cg);
     a.TN = (int)((N + cb::kCols - 1) / cb::kCols);
     a.KS = (int)(qlin_bf16_cache_cols(K) / cb::kKStage);
     a.status = (unsigned*)ws;
@@ -340,21 +495,7 @@ extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t
     memset(&xmap, 0, sizeof(xmap));
     memset(&wmap, 0, sizeof(wmap));
     if (!make_bf16_map(&xmap, x, M, K, ldx, cb::kRows)) return cudaErrorInvalidValue;
-    if (!make_bf16_map(&wmap, wb, N, qlin_bf16_cache_cols(K), qlin_bf16_cache_cols(K), cb::kCols))
+    if (!make_bf16_map(&wmap, wb, N, qlin_bf16_cache_cols(K), qlin_bf16_cache_cols(K), cb::kCols / cg))
         return cudaErrorInvalidValue;
-    const int ntiles = a.TM * a.TN;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    cfg.gridDim = dim3((unsigned)(ntiles < sms ? ntiles : sms));
-    cfg.blockDim = dim3(cb::kThreads);
-    cfg.dynamicSmemBytes = cb::kSmem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 0;
-    if (flags & QLIN_FLAG_PDL) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.numAttrs = 1;
-    }
-    return cudaLaunchKernelEx(&cfg, chunk_bf16_kernel, a, xmap, wmap);
+    return cg == 2 ? launch_bf16_cg<2>(a, xmap, wmap, flags, s) : launch_bf16_cg<1>(a, xmap, wmap, flags, s);
 }

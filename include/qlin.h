@@ -267,7 +267,8 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
  * bf16 path (Q8_0, Q4_0, MXFP4, Q4_K, Q6_K): y[m][n] = sum_k x[m][k] * Wb[n][k] with Wb the bf16
  * copy written by qlin_pack_weights(fmt, N, K, ..., QLIN_PACK_MMA), tcgen05.mma kind::f16 (bf16
  * operands loaded by tensor-map copies, fp32 accumulation in tensor memory); x must be 16-byte
- * aligned with ldx % 8 == 0 (else QLIN_ERR_ALIGNMENT); QLIN_FLAG_CTA_PAIRS is not accepted;
+ * aligned with ldx % 8 == 0 (else QLIN_ERR_ALIGNMENT); QLIN_FLAG_CTA_PAIRS (M > 128): 256 x 256
+ * tiles on pairs of CTAs (cta_group::2), each staging its 128 activation rows and 128 weight rows;
  * ws: qlin_workspace_bytes(QLIN_OP_CHUNK, fmt, M, N, K, 0, 0) bytes (256: the status word).
  * Bounded device waits: a timeout sets the workspace status word (qlin_ws_status). */
 qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,

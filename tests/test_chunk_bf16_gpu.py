@@ -66,16 +66,18 @@ def check(y, x, w32, tol_exact=1e-2):
     assert (np.abs(y.double().cpu().numpy() - exact) <= tol_exact * A0 + 1e-30).all()
 
 
+@pytest.mark.parametrize("flags", [0, q.QLIN_FLAG_CTA_PAIRS])
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (64, 300, 512), (200, 520, 2560), (513, 1000, 1024),
-                                   (37, 70, 96)])
-def test_chunk_bf16_parity(fmt, M, N, K):
+                                   (37, 70, 96), (300, 264, 768)])
+def test_chunk_bf16_parity(fmt, M, N, K, flags):
+    # QLIN_FLAG_CTA_PAIRS: 256-row tiles on pairs of CTAs when M > 128 (single CTAs otherwise)
     if kquant(fmt) and K % 256:
         pytest.skip("K-quants need K % 256 == 0")
     packed, w32 = make(fmt, N, K, 1000 + M)
     x = synth.activations(M, K, synth.gen(1100 + M), dtype=torch.bfloat16).cuda()
     ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
-    y = q.qlin_gemm_chunk(fmt, packed, N, K, x, ws=ws)
+    y = q.qlin_gemm_chunk(fmt, packed, N, K, x, ws=ws, flags=flags)
     torch.cuda.synchronize()
     assert q.qlin_ws_status(ws) == 0
     check(y, x, w32)
@@ -96,14 +98,17 @@ def test_chunk_bf16_strided_operands_and_reuse():
     assert torch.isnan(y[:, N:]).all()
 
 
-def test_chunk_bf16_full_size_sampled():
+@pytest.mark.parametrize("flags", [0, q.QLIN_FLAG_CTA_PAIRS])
+def test_chunk_bf16_full_size_sampled(flags):
     # a prefill chunk of the Q4_0 4B stack's gate_up: M = 512, K = 2560, N = 2 x 9728; sampled rows
     fmt, M, N, K = q.QLIN_Q4_0, 512, 19456, 2560
     blocks, _, _ = synth.weights(fmt, N, K, synth.gen(4242))
     packed = q.qlin_pack_weights(fmt, N, K, blocks.cuda(), pack_flags=q.QLIN_PACK_MMA)
     x = synth.activations(M, K, synth.gen(4243), dtype=torch.bfloat16).cuda()
-    y = q.qlin_gemm_chunk(fmt, packed, N, K, x)
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+    y = q.qlin_gemm_chunk(fmt, packed, N, K, x, ws=ws, flags=flags)
     torch.cuda.synchronize()
+    assert q.qlin_ws_status(ws) == 0
     rows = np.unique(np.linspace(0, N - 1, 61).astype(np.int64))
     w32 = oracle.dequant_f32(fmt, N, K, blocks.numpy())[rows]
     check(y[:, rows], x, w32)
@@ -120,6 +125,6 @@ def test_chunk_bf16_argument_checks():
     st = lib.qlin_gemm_chunk(fmt, q._dev(packed, "p"), N, K, q._dev(xb, "x"), M, K + 4, q._dev(y, "y"), N, 0,
                              q._dev(ws, "ws"), 256, q._stream(None))
     assert st == 3  # QLIN_ERR_ALIGNMENT
-    st = lib.qlin_gemm_chunk(fmt, q._dev(packed, "p"), N, K, q._dev(xb, "x"), M, K + 4, q._dev(y, "y"), N,
-                             q.QLIN_FLAG_CTA_PAIRS, q._dev(ws, "ws"), 256, q._stream(None))
-    assert st == 1  # QLIN_ERR_INVALID_ARG: CTA pairs are an NVFP4-path option
+    st = lib.qlin_gemm_chunk(fmt, q._dev(packed, "p"), N, K, q._dev(xb, "x"), M, K, q._dev(y, "y"), N, 0,
+                             q._dev(ws, "ws"), 255, q._stream(None))
+    assert st == 4  # QLIN_ERR_WORKSPACE

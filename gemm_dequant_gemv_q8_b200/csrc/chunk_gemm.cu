@@ -330,6 +330,22 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     const int TMP = a.TM / CG;  // activation tiles of 128 * CG rows
     const int ntiles = a.T2 * TMP;
     const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
+    // The weights do not depend on x: the producer starts the first stages' weight copies now, so
+    // they land during phase Q (the stage barriers also expect the activation bytes, copied once
+    // quantized).
+    int npre = 0;  // stages of the first tile whose weight part is already in flight (thread 0)
+    if (threadIdx.x == 0 && tile0 < ntiles) {
+        const int t2 = tile0 / TMP;
+        npre = a.G < S ? a.G : S;
+        for (int it = 0; it < npre; ++it) {
+            uint8_t* st = smem + it * Cfg::kStageBytes;
+            const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + it) * kMmaWUnit;
+            mbar_arrive_expect_tx(&full[it], Cfg::kStageBytes);
+            bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[it]);
+            bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[it]);
+        }
+        *issued = npre;  // in flight (the abort path waits for them, bounded)
+    }
     griddep_wait();  // x comes from the previous kernels
 
     // ---------------------------------------------------------------- phase Q: quantize x
@@ -469,11 +485,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     }
                     uint8_t* st = smem + s * Cfg::kStageBytes;
                     const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g) * kMmaWUnit;
-                    mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+                    if (it >= npre) {  // (the first stages' weights were started before phase Q)
+                        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+                        bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[s]);
+                        bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[s]);
+                    }
                     bulk_g2s(st, a.aq + ((int64_t)tm * a.G + g) * kMmaAUnit, kMmaAUnit, &full[s]);
-                    bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[s]);
-                    bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[s]);
-                    *issued = it + 1;
+                    *issued = it + 1 > npre ? it + 1 : npre;
                 }
             }
         }

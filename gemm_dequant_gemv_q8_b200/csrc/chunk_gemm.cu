@@ -87,7 +87,8 @@ struct ChunkArgs {
     int M;
     int64_t N, K;
     int T2, G, TM;  // TM: 128-row activation units (a multiple of CG)
-    int xvec, tma_store;
+    int KS, GS;     // k-splits per output tile (1 or 2) and k-groups per split
+    int xvec, yvec, tma_store;  // yvec: y 16-byte aligned with a row pitch of a multiple of 4 floats
     unsigned* status;
 };
 
@@ -146,6 +147,14 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&r)[48])
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The same box added element-wise into global memory (f32 add, the tensor map's type).
+__device__ __forceinline__ void tma_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
                  "r"(x), "r"(y), "r"(smem_u32(src))
                  : "memory");
@@ -328,18 +337,29 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const int TMP = a.TM / CG;  // activation tiles of 128 * CG rows
-    const int ntiles = a.T2 * TMP;
+    const int ntiles = a.T2 * TMP * a.KS;
     const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
+    // Work item `tile`: weight tile t2, activation tile tm (this CTA's 128 rows of it) and the
+    // k-groups [g0, g1) of split tile % KS.  With KS = 2 the two halves of an output tile add into
+    // y, which phase Q zeroes: two addends onto zero give the same sum in either order.
+    auto tile_of = [&](int tile, int& t2, int& tm, int& g0, int& g1) {
+        const int ks = tile % a.KS, rest = tile / a.KS;
+        t2 = rest / TMP;
+        tm = (rest % TMP) * CG + (int)rank;
+        g0 = ks * a.GS;
+        g1 = g0 + a.GS < a.G ? g0 + a.GS : a.G;
+    };
     // The weights do not depend on x: the producer starts the first stages' weight copies now, so
     // they land during phase Q (the stage barriers also expect the activation bytes, copied once
     // quantized).
     int npre = 0;  // stages of the first tile whose weight part is already in flight (thread 0)
     if (threadIdx.x == 0 && tile0 < ntiles) {
-        const int t2 = tile0 / TMP;
-        npre = a.G < S ? a.G : S;
+        int t2, tm, g0, g1;
+        tile_of(tile0, t2, tm, g0, g1);
+        npre = g1 - g0 < S ? g1 - g0 : S;
         for (int it = 0; it < npre; ++it) {
             uint8_t* st = smem + it * Cfg::kStageBytes;
-            const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + it) * kMmaWUnit;
+            const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g0 + it) * kMmaWUnit;
             mbar_arrive_expect_tx(&full[it], Cfg::kStageBytes);
             bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[it]);
             bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[it]);
@@ -385,6 +405,17 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             }
         } else {
             m = act_amax_partial(a.x, a.M, a.K, a.ldx, vec, gtid, gthreads);
+        }
+        if (a.KS > 1) {  // the k-split halves add into y: zero it (ordered before them by the barrier)
+            const int64_t nq = (a.N + 3) / 4;
+            for (int64_t i = gtid; i < (int64_t)a.M * nq; i += gthreads) {
+                const int64_t row = i / nq, c = (i - row * nq) * 4;
+                float* dst = a.y + row * a.ldy + c;
+                if (a.yvec && c + 4 <= a.N)
+                    *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+                else
+                    for (int u = 0; u < 4 && c + u < a.N; ++u) dst[u] = 0.f;
+            }
         }
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) red[warp] = m;
@@ -455,14 +486,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             fence_proxy_async_global();  // this thread's bulk copies read what phase Q wrote
             int it = 0;
             for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
-                const int t2 = tile / TMP, tm = (tile % TMP) * CG + (int)rank;
-                {  // every unit of this activation tile quantized (bounded wait)
+                int t2, tm, g0, g1;
+                tile_of(tile, t2, tm, g0, g1);
+                {  // every unit of this tile's activation rows and k-groups quantized (bounded wait)
                     const unsigned* rd = a.ready + (int64_t)tm * a.G;
                     const uint64_t t0 = globaltimer_ns();
                     bool ready = false;
                     while (!ready) {
                         ready = true;
-                        for (int g = 0; g < a.G; ++g) ready &= ld_relaxed_gpu(rd + g) >= (unsigned)kUnitItems;
+                        for (int g = g0; g < g1; ++g) ready &= ld_relaxed_gpu(rd + g) >= (unsigned)kUnitItems;
                         if (!ready) {
                             if (globaltimer_ns() - t0 > 2000000000ull) break;
                             __nanosleep(64);
@@ -476,7 +508,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     __threadfence();             // acquire what the quantizing CTAs released
                     fence_proxy_async_global();  // ... for the bulk copies that read it
                 }
-                for (int g = 0; g < a.G; ++g, ++it) {
+                for (int g = g0; g < g1; ++g, ++it) {
                     const int s = it % S;
                     if (it >= S && !mbar_wait_bounded(&empty[s], ((it / S) - 1) & 1)) {
                         atomicOr(a.status, 1u);
@@ -510,8 +542,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     }
                     tc_fence_after();
                 }
+                int t2, tm, g0, g1;
+                tile_of(tile, t2, tm, g0, g1);
                 bool ok = true;
-                for (int g = 0; g < a.G; ++g, ++it) {
+                for (int g = 0; g < g1 - g0; ++g, ++it) {
                     const int s = it % S;
                     const uint32_t par = (it / S) & 1;
                     if (!mbar_wait_bounded(&full[s], par) || !mbar_wait_bounded(&sfready[s], par) ||
@@ -545,8 +579,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             // the data before writing the scales)
             int it = 0;
             for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
+                int t2, tm, g0, g1;
+                tile_of(tile, t2, tm, g0, g1);
                 bool ok = true;
-                for (int g = 0; g < a.G; ++g, ++it) {
+                for (int g = g0; g < g1; ++g, ++it) {
                     const int s = it % S;
                     if (!mbar_wait_bounded(&sfready[s], (it / S) & 1)) {
                         ok = false;
@@ -565,8 +601,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         int it = 0;
         for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
+            int t2, tm, g0, g1;
+            tile_of(tile, t2, tm, g0, g1);
             bool ok = true;
-            for (int g = 0; g < a.G; ++g, ++it) {
+            for (int g = g0; g < g1; ++g, ++it) {
                 const int s = it % S;
                 if (it >= S && !mbar_wait_bounded(&empty[s], ((it / S) - 1) & 1)) {
                     ok = false;
@@ -617,6 +655,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         uint8_t* tb = epi + (warp - Epi::kFirstWarp) * Epi::kBuf;
         constexpr int R = Epi::kBoxRows;
         const bool tma = a.tma_store != 0;
+        const bool add = a.KS > 1;  // k-split: add this half into y (zeroed in phase Q)
+        if (add && lane == 0) fence_proxy_async_global();  // the zeroing stores before the TMA adds
         int tcount = 0, nstore = 0;
         for (int tile = tile0; tile < ntiles; tile += tstep, ++tcount) {
             if (*abort_flag || !mbar_wait_bounded(acc_full, tcount & 1)) {
@@ -625,7 +665,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 break;
             }
             tc_fence_after();
-            const int t2 = tile / TMP, tm = (tile % TMP) * CG + (int)rank;
+            int t2, tm, g0, g1;
+            tile_of(tile, t2, tm, g0, g1);
             const int m0 = tm * kMmaARows + q * 32;  // this warp's first row
             const int64_t n0 = (int64_t)t2 * kMmaWRows;
 #pragma unroll 1
@@ -661,7 +702,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                         }
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) tma_store_2d(&ymap, tb, (int)(n0 + c), m0 + hh * R);
+                        if (lane == 0) {
+                            if (add)
+                                tma_add_2d(&ymap, tb, (int)(n0 + c), m0 + hh * R);
+                            else
+                                tma_store_2d(&ymap, tb, (int)(n0 + c), m0 + hh * R);
+                        }
                         ++nstore;
                     }
                     continue;
@@ -684,7 +730,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                         const int64_t ncol = n0 + c + 16 * h + 4 * ch;
                         if (mrow < a.M && ncol < a.N) {
                             float* dst = a.y + (int64_t)mrow * a.ldy + ncol;
-                            if (ncol + 4 <= a.N && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+                            if (add) {
+                                const float e[4] = {val.x, val.y, val.z, val.w};
+                                for (int u = 0; u < 4 && ncol + u < a.N; ++u) atomicAdd(dst + u, e[u]);
+                            } else if (ncol + 4 <= a.N && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
                                 *reinterpret_cast<float4*>(dst) = val;
                             } else {
                                 const float e[4] = {val.x, val.y, val.z, val.w};
@@ -838,7 +887,11 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
         max_units = units;
         cached_dev = dev;
     }
-    const int ntiles = a.T2 * (a.TM / CG);
+    // Too few output tiles to give every CTA one: split each tile's k-groups in two halves.
+    const int base_tiles = a.T2 * (a.TM / CG);
+    a.KS = (CG == 1 && a.G >= 2 && 2 * base_tiles <= max_units) ? 2 : 1;
+    a.GS = (a.G + a.KS - 1) / a.KS;
+    const int ntiles = base_tiles * a.KS;
     const int units = ntiles < max_units ? ntiles : max_units;
     cfg.gridDim = dim3((unsigned)(units * CG));
     if (flags & QLIN_FLAG_PDL) {
@@ -873,6 +926,9 @@ extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t 
     a.TM = (int)chunk_units_m(M, flags);
     a.xvec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && ldx % 8 == 0) ? 1 : 0;
     a.tma_store = 0;
+    a.yvec = ((reinterpret_cast<uintptr_t>(y) & 15) == 0 && ldy % 4 == 0) ? 1 : 0;
+    a.KS = 1;
+    a.GS = a.G;
     a.status = (unsigned*)ws;
     return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2>(a, flags, s) : launch_chunk_cg<1>(a, flags, s);
 }

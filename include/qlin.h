@@ -259,7 +259,10 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
  *      (a bounded grid-wide barrier between the max and the quantization; all CTAs of the launch
  *      are resident at once, one per SM);
  *   2. y[m][n] = (a_g * g_w) * sum_k A_q[m][k] * W_q[n][k], block scales applied inside the MMA
- *      (kind::mxf4nvf4 block16), fp32 accumulation in tensor memory.
+ *      (kind::mxf4nvf4 block16), fp32 accumulation in tensor memory.  When the 128 x 256 output
+ *      tiles number at most half the CTAs (M <= 128 with N <= 37 * 256 on 148 SMs, ...), each tile
+ *      runs as two halves of its k-groups that add into y, which step 1 zeroes; two addends onto
+ *      zero give the same sum in either order, so y stays deterministic.
  *   packed: qlin_pack_weights(QLIN_NVFP4, N, K, ..., QLIN_PACK_MMA);  x: bf16 M x K, row stride ldx;
  *   y: fp32, row stride ldy (16-byte aligned y and ldy % 4 == 0 take the TMA-store epilogue);
  *   flags: QLIN_FLAG_PDL and/or QLIN_FLAG_CTA_PAIRS;

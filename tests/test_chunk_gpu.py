@@ -59,8 +59,10 @@ def _chunk(M, N, K, seed, rows=None, flags=0):
 
 
 @pytest.mark.parametrize("flags", [0, q.QLIN_FLAG_CTA_PAIRS])
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (70, 300, 272), (200, 512, 1024)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (70, 300, 272), (200, 512, 1024), (64, 264, 768)])
 def test_chunk_gemm_small(M, N, K, flags):
+    # Few output tiles (all but the first shape): each tile's k-groups run as two halves that add
+    # into y; K = 768 splits its three k-groups 2 + 1, K = 272 ends in a partial k-group.
     y, yq, Aq, _, _, _ = _chunk(M, N, K, 10 * M + N, flags=flags)
     err = np.abs(y - yq)
     assert (err <= 2e-6 * Aq).all(), float(np.max(err / np.maximum(Aq, 1e-300)))

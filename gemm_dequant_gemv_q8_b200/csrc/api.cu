@@ -16,6 +16,7 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
                                        int xdt, int M, float* y, float* h, int flags, void* ws, cudaStream_t s);
 extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K);
 extern "C" int64_t qlin_bf16_cache_cols(int64_t K);
+extern "C" int64_t qlin_bf16_cache_bytes(int64_t N, int64_t K);
 extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
                                               int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
                                               cudaStream_t s);
@@ -102,7 +103,7 @@ size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags
     if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
     if (pack_flags == QLIN_PACK_MMA) {
         if (fmt != QLIN_NVFP4)  // the bf16 copy of the dequantized weights, rows of K rounded up to 64
-            return (size_t)qlin::kHdrBytes + (size_t)N * (size_t)qlin_bf16_cache_cols(K) * 2u;
+            return (size_t)qlin::kHdrBytes + (size_t)qlin_bf16_cache_bytes(N, K);
         return (size_t)qlin::kHdrBytes + (size_t)((N + 255) / 256) * (size_t)((K + 255) / 256) * 36864u;
     }
     if (pack_flags & ~QLIN_PACK_GATE_UP) return 0;

@@ -86,6 +86,26 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// The weight copy is blocked (256 rows x 64 values contiguous, 32 KB): a 4-D tensor map {value,
+// row in block, k-block, row block}; one box is this CTA's rows of one block.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map, int c1, int c2, int c3,
+                                                 uint64_t* bar) {
+    asm volatile(
+        "{\n .reg .b32 rb;\n mapa.shared::cluster.u32 rb, %6, 0;\n"
+        " cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [rb];\n}\n" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ uint32_t cta_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -230,7 +250,7 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
             int it = 0;
             for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
                 const int tn = tile / a.TM, tm = tile % a.TM;  // groups at work together share weight tiles
-                const int xrow = (tm * CG + (int)rank) * kRows, wrow = tn * kCols + (int)rank * C::kBRows;
+                const int xrow = (tm * CG + (int)rank) * kRows;
                 for (int ks = 0; ks < a.KS; ++ks, ++it) {
                     const int s = it % S;
                     if (it >= S && !mbar_wait_bounded(&empty[s], ((it / S) - 1) & 1)) {
@@ -242,11 +262,11 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
                     if constexpr (CG == 1) {
                         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
                         tma_load_2d(st, &xmap, ks * kKStage, xrow, &full[s]);
-                        tma_load_2d(st + kABytes, &wmap, ks * kKStage, wrow, &full[s]);
+                        tma_load_4d(st + kABytes, &wmap, 0, ks, tn, &full[s]);
                     } else {
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
                         tma_load_2d_pair(st, &xmap, ks * kKStage, xrow, &full[s]);
-                        tma_load_2d_pair(st + kABytes, &wmap, ks * kKStage, wrow, &full[s]);
+                        tma_load_4d_pair(st + kABytes, &wmap, (int)rank * C::kBRows, ks, tn, &full[s]);
                     }
                     *issued = it + 1;
                 }
@@ -419,6 +439,26 @@ static bool make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int6
 
 // Columns of the bf16 weight copy: K rounded up to whole 64-value stages (zero-filled).
 extern "C" int64_t qlin_bf16_cache_cols(int64_t K) { return (K + cb::kKStage - 1) / cb::kKStage * cb::kKStage; }
+// Bytes of the bf16 weight copy: blocks of 256 rows x 64 values, N rounded up to 256 (zero rows).
+extern "C" int64_t qlin_bf16_cache_bytes(int64_t N, int64_t K) {
+    return (N + cb::kCols - 1) / cb::kCols * cb::kCols * qlin_bf16_cache_cols(K) * 2;
+}
+
+// The blocked weight copy as a 4-D bf16 tensor {64 values, 256 rows, Kc / 64 k-blocks, Np / 256 row
+// blocks}, read in boxes of 64 values x box_rows rows with the 128-byte swizzle.
+static bool make_wblock_map(CUtensorMap* map, const void* base, int64_t N, int64_t K, int box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = bf16_map_encoder();
+    if (!enc) return false;
+    const int64_t kb = qlin_bf16_cache_cols(K) / cb::kKStage, nb = (N + cb::kCols - 1) / cb::kCols;
+    const cuuint64_t dims[4] = {(cuuint64_t)cb::kKStage, (cuuint64_t)cb::kCols, (cuuint64_t)kb, (cuuint64_t)nb};
+    const cuuint64_t strides[3] = {(cuuint64_t)cb::kKStage * 2, (cuuint64_t)cb::kCols * cb::kKStage * 2,
+                                   (cuuint64_t)kb * cb::kCols * cb::kKStage * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)cb::kKStage, (cuuint32_t)box_rows, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 template <int CG>
 static cudaError_t launch_bf16_cg(const cb::Args& a, const CUtensorMap& xmap, const CUtensorMap& wmap, int flags,
@@ -474,7 +514,8 @@ static cudaError_t launch_bf16_cg(const cb::Args& a, const CUtensorMap& xmap, co
     return cudaLaunchKernelEx(&cfg, chunk_bf16_kernel<CG>, a, xmap, wmap);
 }
 
-// wb: the bf16 weights [N][qlin_bf16_cache_cols(K)] (after the 256-byte header of the packed buffer);
+// wb: the blocked bf16 weights (after the 256-byte header of the packed buffer): for row block nb
+// and k-block kb, 256 rows x 64 values at element ((nb * Kc / 64 + kb) * 256 + row) * 64;
 // x: bf16 [M][K] with row pitch ldx (16-byte aligned base, ldx % 8 == 0, checked by the caller).
 // QLIN_FLAG_CTA_PAIRS with M > 128: 256 x 256 tiles on pairs of CTAs.
 extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
@@ -495,7 +536,6 @@ extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t
     memset(&xmap, 0, sizeof(xmap));
     memset(&wmap, 0, sizeof(wmap));
     if (!make_bf16_map(&xmap, x, M, K, ldx, cb::kRows)) return cudaErrorInvalidValue;
-    if (!make_bf16_map(&wmap, wb, N, qlin_bf16_cache_cols(K), qlin_bf16_cache_cols(K), cb::kCols / cg))
-        return cudaErrorInvalidValue;
+    if (!make_wblock_map(&wmap, wb, N, K, cb::kCols / cg)) return cudaErrorInvalidValue;
     return cg == 2 ? launch_bf16_cg<2>(a, xmap, wmap, flags, s) : launch_bf16_cg<1>(a, xmap, wmap, flags, s);
 }

@@ -258,14 +258,14 @@ template <int FMT>
 __global__ void __launch_bounds__(256) pack_bf16_kernel(const uint8_t* __restrict__ blocks,
                                                         const uint8_t* __restrict__ scales, int64_t N, int64_t K,
                                                         int64_t Kc, __nv_bfloat16* __restrict__ out) {
-    const int64_t nb = Kc / 32;
+    const int64_t nb = Kc / 32, Np = (N + 255) / 256 * 256;
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= N * nb) return;
+    if (idx >= Np * nb) return;
     const int64_t n = idx / nb, b = idx - n * nb, k0 = b * 32;
     float w[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) w[j] = 0.f;
-    if (k0 < K) {
+    if (n < N && k0 < K) {
         if (FMT == QLIN_Q8_0 || FMT == QLIN_Q4_0) {
             const int bsz = FMT == QLIN_Q8_0 ? 34 : 18;
             const uint8_t* blk = blocks + n * (K / 32) * bsz + b * bsz;
@@ -315,7 +315,9 @@ __global__ void __launch_bounds__(256) pack_bf16_kernel(const uint8_t* __restric
         const __nv_bfloat162 h = __floats2bfloat162_rn(w[2 * j], w[2 * j + 1]);
         pk[j] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    uint4* dst = reinterpret_cast<uint4*>(out + n * Kc + k0);
+    // blocked: 256 rows x 64 values per (row block, k-block), 32 KB contiguous
+    const int64_t blk = (n / 256) * (Kc / 64) + k0 / 64;
+    uint4* dst = reinterpret_cast<uint4*>(out + (blk * 256 + n % 256) * 64 + k0 % 64);
 #pragma unroll
     for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
 }
@@ -337,7 +339,7 @@ extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void*
                                              (int32_t)((N + 255) / 256), (int32_t)((K + 255) / 256));
         if (fmt == QLIN_NVFP4) return qlin_launch_pack_mma(blocks, scales, N, K, gs, packed, s);
         const int64_t Kc = qlin_bf16_cache_cols(K);
-        const int64_t threads = N * (Kc / 32);
+        const int64_t threads = (N + 255) / 256 * 256 * (Kc / 32);
         const dim3 grid((unsigned)((threads + 255) / 256));
         const uint8_t* bl = (const uint8_t*)blocks;
         const uint8_t* sc = (const uint8_t*)scales;

@@ -77,10 +77,13 @@ enum {
                              (tiles of 256 rows x 256 values, 128-byte-swizzled K-major codes, scale
                              factors in 512-byte atoms), 0.5625 B/weight plus padding to 256 x 256.
                              Q8_0 / Q4_0 / MXFP4 / Q4_K / Q6_K: a bf16 copy of the dequantized
-                             weights, row-major N x roundup(K, 64) after the 256-byte header, each
-                             weight the fp32 value of qlin_dequant_debug rounded to nearest-even
-                             bf16, the tail columns zero (2 B/weight: the full-precision prefill
-                             copy; imp README "Why this exists": prefill via source dequant) */
+                             weights after the 256-byte header, in blocks of 256 rows x 64 values
+                             (32 KB contiguous, rows of 128 bytes): with Kc = roundup(K, 64), row n
+                             and column k at element ((n / 256 * Kc / 64 + k / 64) * 256 + n % 256)
+                             * 64 + k % 64; each weight the fp32 value of qlin_dequant_debug rounded
+                             to nearest-even bf16, columns >= K and rows >= N (to a multiple of
+                             256) zero (2 B/weight: the full-precision prefill copy; imp README
+                             "Why this exists": prefill via source dequant) */
 };
 
 /* qlin_workspace_bytes ops */

@@ -53,9 +53,11 @@ def test_packed_bytes_sizes(lib):
     # MXFP4: codes as NVFP4, one scale byte per 32 values: 4096 + 256 bytes per 32 x 256 unit
     assert q.qlin_packed_bytes(q.QLIN_MXFP4, 4096, 2560) == 256 + 4096 * 2560 * 17 // 32
     assert q.qlin_packed_bytes(q.QLIN_MXFP4, 64, 272) == 0  # K % 32
-    # QLIN_PACK_MMA for the GGUF / MXFP4 formats: the bf16 copy, rows of K rounded up to 64
-    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 100, 96, q.QLIN_PACK_MMA) == 256 + 100 * 128 * 2
-    assert q.qlin_packed_bytes(q.QLIN_Q6_K, 64, 512, q.QLIN_PACK_MMA) == 256 + 64 * 512 * 2
+    # QLIN_PACK_MMA for the GGUF / MXFP4 formats: the bf16 copy in blocks of 256 rows x 64 values,
+    # K rounded up to 64 and N to 256
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 100, 96, q.QLIN_PACK_MMA) == 256 + 256 * 128 * 2
+    assert q.qlin_packed_bytes(q.QLIN_Q6_K, 64, 512, q.QLIN_PACK_MMA) == 256 + 256 * 512 * 2
+    assert q.qlin_packed_bytes(q.QLIN_Q4_0, 17408, 5120, q.QLIN_PACK_MMA) == 256 + 17408 * 5120 * 2
     # Q4_K: 4096 B of codes + 512 B of sub-block scale/min slots + 128 B of per-row d/dmin per unit
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 4096, 2560) == 256 + (4096 // 32) * (2560 // 256) * 4736
     assert q.qlin_packed_bytes(q.QLIN_Q4_K, 33, 512) == 256 + 2 * 2 * 4736

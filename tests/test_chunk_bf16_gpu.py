@@ -34,8 +34,11 @@ def make(fmt, N, K, seed):
 
 
 def cache(packed, N, K):
+    # blocks of 256 rows x 64 values: block (nb, kb) holds rows 256 nb.. and columns 64 kb..
     kc = (K + 63) // 64 * 64
-    return packed[256:256 + N * kc * 2].view(torch.bfloat16).view(N, kc), kc
+    npad = (N + 255) // 256 * 256
+    blocks = packed[256:256 + npad * kc * 2].view(torch.bfloat16).view(npad // 256, kc // 64, 256, 64)
+    return blocks.permute(0, 2, 1, 3).reshape(npad, kc), kc
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -47,9 +50,9 @@ def test_bf16_cache_bit_exact(fmt, N, K):
     assert packed.numel() == q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA)
     wb, kc = cache(packed, N, K)
     ref = torch.from_numpy(w32).to(torch.bfloat16)
-    got = wb[:, :K].cpu()
+    got = wb[:N, :K].cpu()
     assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
-    assert (wb[:, K:].cpu().float() == 0).all()
+    assert (wb[:, K:].cpu().float() == 0).all() and (wb[N:].cpu().float() == 0).all()
 
 
 def check(y, x, w32, tol_exact=1e-2):

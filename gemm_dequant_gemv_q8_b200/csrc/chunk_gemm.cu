@@ -45,6 +45,8 @@ template <int CG>
 struct ChunkCfg {
     static constexpr int kWCodes = 32768 / CG;                      // weight code bytes per CTA per k-group
     static constexpr int kStageBytes = kMmaAUnit + kWCodes + 4096;  // + all 256 weight rows' scales
+    static constexpr int kScaleBytes = (kMmaAUnit - kMmaARows * 128) + 4096;  // completes on the scale barrier
+    static constexpr int kCodeBytes = kStageBytes - kScaleBytes;
     static constexpr int kStages = CG == 1 ? 4 : 5;
     static constexpr int kRingBytes = kStages * kStageBytes;
 };
@@ -62,7 +64,7 @@ struct EpiCfg {
     static constexpr int kBytes = kWarps * kBuf;
 };
 template <int CG>
-constexpr int chunk_smem() { return 1024 + ChunkCfg<CG>::kRingBytes + EpiCfg<CG>::kBytes + 256; }
+constexpr int chunk_smem() { return 1024 + ChunkCfg<CG>::kRingBytes + EpiCfg<CG>::kBytes + 512; }
 constexpr int kChunkThreads = 320;
 constexpr int kTmemCols = 512;
 constexpr int kSfCols = 48;  // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
@@ -305,7 +307,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     uint64_t* empty = full + S;
     uint64_t* sfready = empty + S;  // this CTA's scale writers are done with the stage
     uint64_t* pfull = sfready + S;  // CG = 2, rank 0: the other CTA's stage is ready
-    uint64_t* acc_full = pfull + S;
+    uint64_t* sfull = pfull + S;    // the stage's scale bytes have landed (the codes: full)
+    uint64_t* acc_full = sfull + S;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* mma_done = acc_empty + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -322,6 +325,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             mbar_init(&empty[s], 1);
             mbar_init(&sfready[s], 4);
             mbar_init(&pfull[s], 1);
+            mbar_init(&sfull[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, Epi::kWarps * CG);  // the epilogue warps of every CTA of the group
@@ -352,6 +356,20 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     // The weights do not depend on x: the producer starts the first stages' weight copies now, so
     // they land during phase Q (the stage barriers also expect the activation bytes, copied once
     // quantized).
+    // A stage's copies: the scale bytes (2 KB of the activation unit, 4 KB of the weight unit)
+    // complete on sfull, so the scale writers start before the 48 KB (or 32 KB) of codes land.
+    auto expect_stage = [&](int s) {
+        mbar_arrive_expect_tx(&full[s], Cfg::kCodeBytes);
+        mbar_arrive_expect_tx(&sfull[s], Cfg::kScaleBytes);
+    };
+    auto copy_w = [&](uint8_t* st, const uint8_t* wu, int s) {
+        bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &sfull[s]);
+        bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[s]);
+    };
+    auto copy_a = [&](uint8_t* st, const uint8_t* au, int s) {
+        bulk_g2s(st + kMmaARows * 128, au + kMmaARows * 128, kMmaAUnit - kMmaARows * 128, &sfull[s]);
+        bulk_g2s(st, au, kMmaARows * 128, &full[s]);
+    };
     int npre = 0;  // stages of the first tile whose weight part is already in flight (thread 0)
     if (threadIdx.x == 0 && tile0 < ntiles) {
         int t2, tm, g0, g1;
@@ -360,9 +378,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         for (int it = 0; it < npre; ++it) {
             uint8_t* st = smem + it * Cfg::kStageBytes;
             const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g0 + it) * kMmaWUnit;
-            mbar_arrive_expect_tx(&full[it], Cfg::kStageBytes);
-            bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[it]);
-            bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[it]);
+            expect_stage(it);
+            copy_w(st, wu, it);
         }
         *issued = npre;  // in flight (the abort path waits for them, bounded)
     }
@@ -518,11 +535,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     uint8_t* st = smem + s * Cfg::kStageBytes;
                     const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g) * kMmaWUnit;
                     if (it >= npre) {  // (the first stages' weights were started before phase Q)
-                        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
-                        bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[s]);
-                        bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &full[s]);
+                        expect_stage(s);
+                        copy_w(st, wu, s);
                     }
-                    bulk_g2s(st, a.aq + ((int64_t)tm * a.G + g) * kMmaAUnit, kMmaAUnit, &full[s]);
+                    copy_a(st, a.aq + ((int64_t)tm * a.G + g) * kMmaAUnit, s);
                     *issued = it + 1 > npre ? it + 1 : npre;
                 }
             }
@@ -610,7 +626,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     ok = false;
                     break;
                 }
-                if (!mbar_wait_bounded(&full[s], (it / S) & 1)) {
+                if (!mbar_wait_bounded(&sfull[s], (it / S) & 1)) {
                     ok = false;
                     break;
                 }
@@ -752,8 +768,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     if (warp == 0 && lane == 0 && *abort_flag) {
         // wait (bounded) for the last bulk copies issued to land before shared memory is released
         const int n_it = *issued;
-        for (int j = n_it > S ? n_it - S : 0; j < n_it; ++j)
+        for (int j = n_it > S ? n_it - S : 0; j < n_it; ++j) {
             mbar_wait_bounded(&full[j % S], (j / S) & 1, 50000000ull);
+            mbar_wait_bounded(&sfull[j % S], (j / S) & 1, 50000000ull);
+        }
     }
     // CG = 2: the pair's MMAs read both CTAs' shared memory and write both CTAs' tensor memory;
     // neither CTA frees either before the issuing CTA has seen them complete (mma_done above).

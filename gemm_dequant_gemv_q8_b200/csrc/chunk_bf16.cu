@@ -244,6 +244,9 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
     const int ntiles = a.TM * a.TN;  // TM: tiles of 128 * CG activation rows
     const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
     griddep_wait();  // x comes from the previous kernels
+    // No CTA of this grid waits for another: a dependent launch may take SMs as CTAs leave them (it
+    // reads nothing of ours before its own wait).
+    griddep_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {

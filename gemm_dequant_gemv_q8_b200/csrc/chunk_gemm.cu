@@ -452,6 +452,9 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             *ag_sm = ag;
         }
         __syncthreads();
+        // Every CTA of this grid is resident (all passed the barrier): a dependent launch may now
+        // take SMs as this grid's CTAs leave them; it reads nothing of ours before its own wait.
+        griddep_launch_dependents();
         if (!*abort_flag) {
             const float ag = *ag_sm;
             if (resident) {

@@ -131,3 +131,18 @@ def test_chunk_bf16_argument_checks():
     st = lib.qlin_gemm_chunk(fmt, q._dev(packed, "p"), N, K, q._dev(xb, "x"), M, K, q._dev(y, "y"), N, 0,
                              q._dev(ws, "ws"), 255, q._stream(None))
     assert st == 4  # QLIN_ERR_WORKSPACE
+
+
+def test_chunk_bf16_back_to_back_pdl():
+    # calls enqueued back to back with QLIN_FLAG_PDL (each may start while the previous drains)
+    fmt, N, K = q.QLIN_Q4_0, 520, 1024
+    packed, w32 = make(fmt, N, K, 61)
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, 512, N, K))
+    runs = []
+    for M, fl in ((512, 0), (64, 0), (300, q.QLIN_FLAG_CTA_PAIRS), (5, 0)):
+        x = synth.activations(M, K, synth.gen(62 + M), dtype=torch.bfloat16).cuda()
+        runs.append((x, q.qlin_gemm_chunk(fmt, packed, N, K, x, ws=ws, flags=fl | q.QLIN_FLAG_PDL)))
+    torch.cuda.synchronize()
+    assert q.qlin_ws_status(ws) == 0
+    for x, y in runs:
+        check(y, x, w32)

@@ -141,3 +141,25 @@ def test_chunk_gemm_alternating_shapes_one_workspace():
         xq = oracle.dequant(q.QLIN_NVFP4, M, K, ac, asc, ag)
         yq, Aq = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xq, scales=scales.numpy(), g=g)
         assert (np.abs(y.cpu().double().numpy() - yq) <= 2e-6 * Aq).all()
+
+
+def test_chunk_gemm_back_to_back_pdl_one_workspace():
+    """Calls enqueued back to back with QLIN_FLAG_PDL on one workspace (no host synchronisation
+    between them): each may start while the previous drains, yet every result and the status
+    stay as if they ran one after another."""
+    N, K = 1024, 768
+    codes, scales, g = synth.nvfp4(N, K, synth.gen(51))
+    packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA)
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, q.QLIN_NVFP4, 512, N, K))
+    runs = []
+    for M, fl in ((512, 0), (64, 0), (300, q.QLIN_FLAG_CTA_PAIRS), (7, 0), (512, 0), (129, 0)):
+        x = synth.activations(M, K, synth.gen(52 + M), dtype=torch.bfloat16)
+        y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda(), ws=ws, flags=fl | q.QLIN_FLAG_PDL)
+        runs.append((x, y))
+    torch.cuda.synchronize()
+    assert q.qlin_ws_status(ws) == 0
+    for x, y in runs:
+        ac, asc, ag = oracle.act_quant(x.float().numpy())
+        xq = oracle.dequant(q.QLIN_NVFP4, x.shape[0], K, ac, asc, ag)
+        yq, Aq = oracle.gemv(q.QLIN_NVFP4, N, K, codes.numpy(), xq, scales=scales.numpy(), g=g)
+        assert (np.abs(y.cpu().double().numpy() - yq) <= 2e-6 * Aq).all()

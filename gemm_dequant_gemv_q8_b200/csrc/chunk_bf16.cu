@@ -13,7 +13,8 @@
 // stage instead of 48 KB):
 //   warp 0   : producer -- two TMA tensor loads per stage (x rows and weight rows, 64 values each,
 //              128-byte swizzled by the tensor maps) into the ring; rows and columns outside the
-//              tensors read as zero.  With CG = 2 both CTAs' loads complete on the first CTA's
+//              tensors read as zero.  The weight copy is stored in blocks of 256 rows x 64 values,
+//              so a stage's weight tile is one contiguous 32 KB block (a 4-D tensor map).  With CG = 2 both CTAs' loads complete on the first CTA's
 //              stage barrier (the .cta_group::2 form), which alone tracks a stage's bytes;
 //   warp 1   : one thread (of the first CTA) issues the stage's four M128/M256 N256 K16 MMAs,
 //              commits the stage back to the producers (both CTAs) and, after the tile's last

@@ -24,10 +24,15 @@ inline int ring_ctas_per_sm(int fmt) { return (fmt == QLIN_Q8_0 || fmt == QLIN_Q
 // exactly P * 2^-149 (patterns below 2^23 are denormals, 2^23 .. 2^24-1 continue seamlessly as
 // the first binade).  So a nibble or byte masked in place at bit 4j (8j), with nothing else set,
 // IS the float n * 2^(4j) * 2^-149: one AND per weight, no shift, no subtraction.  Codes are
-// unsigned (Q4_0 nibble n = q + 8, Q8_0 byte = q + 128); the offset is removed once per block
-// from a sum of the activations taken in the same order (see prep_x_q4 / prep_x_q8).  Q4_K
-// codes (0..15, placed as Q4_0's) go through the same decoder; their sub-block min multiplies
-// that activation sum instead of an offset.
+// unsigned (Q4_0 nibble n = q + 8, Q8_0 byte = q + 128, Q6_K byte = q + 32).  The offset is
+// removed from each decoded value before it is multiplied: adding -offset * 2^(position - 149)
+// to n * 2^(position - 149) is exact (both are multiples of 2^-149 below 2^-125), one packed add
+// per two values, so every product and partial sum is of the signed weight q.  (Removing the
+// offset once per block instead, from a sum of the activations, leaves rounding errors of the
+// size of offset * sum|x| in the block sum: for blocks of small codes that is far above
+// 2e-6 * sum|q x|.)  Q4_K codes (0..15, placed as Q4_0's) go through the same decoder without an
+// offset; their sub-block min multiplies a sum of the activations (prep_x_q4), as the format
+// defines w = d * scale * code - dmin * min.
 // Activations are pre-scaled by 2^(kXExp - 4j) (2^(kXExp - 8j) for Q8_0), so every product is
 // the exact n * x * 2^(kXExp - 149) computed inside an fp32 FMA; block sums carry 2^(kXExp - 149)
 // and the tile output multiplies by kDenormUnscale = 2^(149 - kXExp).  Products stay normal and
@@ -49,7 +54,9 @@ __device__ __forceinline__ float format_out_scale(const uint8_t* packed) {
 // Elements 0..5 of each word are masked in place (position j = i).  The top bytes of the two
 // words (elements 6 and 7 of each) are gathered by one byte permute into bits 0..15 of a third
 // word, where they sit at positions 0, 1 (word w0) and 2, 3 (word w1).  Pairs per word: (0,1)
-// (2,3) (4,5) (6,7).
+// (2,3) (4,5) (6,7).  SIGNED (Q4_0): the offset 8 is removed from each value (positions 4j:
+// -8 * 2^(4j - 149) = -2^(4j - 146)).
+template <bool SIGNED>
 __device__ __forceinline__ void dec_q4_pair(uint32_t w0, uint32_t w1, float2 (&p0)[4], float2 (&p1)[4]) {
     const uint32_t top = __byte_perm(w0, w1, 0x0073u);  // byte 0 = w0 byte 3, byte 1 = w1 byte 3
     p0[0] = make_float2(__uint_as_float(w0 & 0xfu), __uint_as_float(w0 & 0xf0u));
@@ -60,22 +67,28 @@ __device__ __forceinline__ void dec_q4_pair(uint32_t w0, uint32_t w1, float2 (&p
     p1[1] = make_float2(__uint_as_float(w1 & 0xf00u), __uint_as_float(w1 & 0xf000u));
     p1[2] = make_float2(__uint_as_float(w1 & 0xf0000u), __uint_as_float(w1 & 0xf00000u));
     p1[3] = make_float2(__uint_as_float(top & 0xf00u), __uint_as_float(top & 0xf000u));
+    if (SIGNED) {
+        const float2 b01 = make_float2(-0x1p-146f, -0x1p-142f), b23 = make_float2(-0x1p-138f, -0x1p-134f);
+        const float2 b45 = make_float2(-0x1p-130f, -0x1p-126f);
+        p0[0] = __fadd2_rn(p0[0], b01), p0[1] = __fadd2_rn(p0[1], b23), p0[2] = __fadd2_rn(p0[2], b45);
+        p0[3] = __fadd2_rn(p0[3], b01);  // positions 0, 1
+        p1[0] = __fadd2_rn(p1[0], b01), p1[1] = __fadd2_rn(p1[1], b23), p1[2] = __fadd2_rn(p1[2], b45);
+        p1[3] = __fadd2_rn(p1[3], b23);  // positions 2, 3
+    }
 }
 
-// Q8_0 word: elements 4k..4k+3 stored as q + 128 in bytes 0..3.  Bytes 0..2 are masked in
-// place (positions 0, 1, 2); byte 3 is w >> 24 (position 0).  Pairs: (0,1) (2,3).
+// Q8_0 word: elements 4k..4k+3 stored as q + 128 in bytes 0..3 (Q6_K: q + 32).  Bytes 0..2 are
+// masked in place (positions 0, 1, 2); byte 3 is w >> 24 (position 0).  Pairs: (0,1) (2,3).  The
+// offset OFF is removed from each value: -OFF * 2^(8j - 149) at position j.
+template <int OFF>
 __device__ __forceinline__ void dec_q8(uint32_t w, float2 (&p)[2]) {
-    p[0] = make_float2(__uint_as_float(w & 0xffu), __uint_as_float(w & 0xff00u));
-    p[1] = make_float2(__uint_as_float(w & 0xff0000u), __uint_as_float(w >> 24));
+    constexpr float b0 = -(float)OFF * 0x1p-149f, b1 = -(float)OFF * 0x1p-141f, b2 = -(float)OFF * 0x1p-133f;
+    p[0] = __fadd2_rn(make_float2(__uint_as_float(w & 0xffu), __uint_as_float(w & 0xff00u)), make_float2(b0, b1));
+    p[1] = __fadd2_rn(make_float2(__uint_as_float(w & 0xff0000u), __uint_as_float(w >> 24)), make_float2(b2, b0));
 }
 
-// Offset sum of one lane's part: the products of code == offset (8 for Q4_0, 128 for Q8_0) are
-// offset * x * 2^(kXExp - 149), a power of two times x, and a power-of-two factor commutes with
-// fp32 rounding.  So adding the raw activations in exactly the order unit_dot adds its products
-// (two interleaved pair chains, then the pairs combined lane-wise, then the two halves), times
-// offset * 2^(kXExp - 149), reproduces bit for bit what a block of offset codes sums to: a block
-// of zero weights gives exactly 0.  Both decoders feed even pairs to chain 0 and odd pairs to
-// chain 1, in increasing pair order.
+// Sum of one lane's 32 activations (the Q4_K min term), in the order unit_dot adds its products:
+// two interleaved pair chains, then the pairs combined lane-wise, then the two halves.
 __device__ __forceinline__ float offset_sum(const float2 (&x)[16]) {
     float2 t0 = x[0], t1 = x[1];
 #pragma unroll
@@ -87,49 +100,32 @@ __device__ __forceinline__ float offset_sum(const float2 (&x)[16]) {
     return u.x + u.y;
 }
 
-// Prepare a lane's 32 activations for the Q4_0 decoder: the offset term 8 * sum (scaled), then
-// element e (pair e/2) times 2^(kXExp - 4 j) with j the decoder's position of element e mod 8.
-// Q4_K (same code positions, no offset): xb = sum * 2^(kXExp - 149), the min term's factor.
+// Prepare a lane's 32 activations for the Q4_0 / Q4_K decoder: element e (pair e/2) times
+// 2^(kXExp - 4 j) with j the decoder's position of element e mod 8.  Q4_K also takes
+// xb = sum * 2^(kXExp - 149), the factor of its min term; Q4_0 needs none (xb = 0).
 template <int MP, bool K4 = false>
 __device__ __forceinline__ void prep_x_q4(float2 (&xv)[MP][16], float2 (&xb)[MP]) {
-    constexpr float c = K4 ? 0x1p-86f : 0x1p-83f;  // (1 or 8) * 2^(kXExp - 149)
+    constexpr float c = 0x1p-86f;  // 2^(kXExp - 149)
     const float2 s0 = make_float2(0x1p63f, 0x1p59f), s1 = make_float2(0x1p55f, 0x1p51f);
     const float2 s2 = make_float2(0x1p47f, 0x1p43f);
 #pragma unroll
     for (int mm = 0; mm < MP; ++mm) {
-        xb[mm].x = c * offset_sum(xv[mm]);
+        xb[mm] = make_float2(K4 ? c * offset_sum(xv[mm]) : 0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < 16; ++q)  // pair q = 4k + (q & 3); pair 4k+3 sits at positions 0,1 (k even) or 2,3
             xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 3) == 0 ? s0 : (q & 3) == 1 ? s1 : (q & 3) == 2 ? s2 : ((q >> 2) & 1) ? s1 : s0);
     }
 }
 
-// Prepare a lane's 32 activations for the Q8_0 decoder: offset 128 * sum (scaled), pairs
-// (4k, 4k+1) times (2^63, 2^55) and (4k+2, 4k+3) times (2^47, 2^63).
-// Q6_K (codes 0..63 in the same byte positions, offset 32, a scale per 16 values): the offset
-// sums of elements 0..15 and 16..31 separately, each times 32 * 2^(kXExp - 149).
-template <int MP, bool K6 = false>
+// Prepare a lane's 32 activations for the Q8_0 / Q6_K decoder (codes in the same byte positions;
+// the decoder removes their offsets): pairs (4k, 4k+1) times (2^63, 2^55) and (4k+2, 4k+3) times
+// (2^47, 2^63).  No activation sum is needed (xb = 0).
+template <int MP>
 __device__ __forceinline__ void prep_x_q8(float2 (&xv)[MP][16], float2 (&xb)[MP]) {
-    constexpr float c = K6 ? 0x1p-81f : 0x1p-79f;  // (32 or 128) * 2^(kXExp - 149)
     const float2 s0 = make_float2(0x1p63f, 0x1p55f), s1 = make_float2(0x1p47f, 0x1p63f);
 #pragma unroll
     for (int mm = 0; mm < MP; ++mm) {
-        if (K6) {
-            float2 h[2];
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {  // pairs 8b .. 8b+7: words 4b .. 4b+3 of the decoder
-                float2 t0 = xv[mm][8 * b], t1 = xv[mm][8 * b + 1];
-#pragma unroll
-                for (int q = 2; q < 8; q += 2) {
-                    t0 = __fadd2_rn(t0, xv[mm][8 * b + q]);
-                    t1 = __fadd2_rn(t1, xv[mm][8 * b + q + 1]);
-                }
-                h[b] = __fadd2_rn(t0, t1);
-            }
-            xb[mm] = make_float2(c * (h[0].x + h[0].y), c * (h[1].x + h[1].y));
-        } else {
-            xb[mm].x = c * offset_sum(xv[mm]);
-        }
+        xb[mm] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int q = 0; q < 16; ++q) xv[mm][q] = __fmul2_rn(xv[mm][q], (q & 1) ? s1 : s0);
     }
@@ -141,7 +137,7 @@ __device__ __forceinline__ void prep_x(float2 (&xv)[MP][16], float2 (&xb)[MP]) {
     if (FMT == QLIN_Q4_0) prep_x_q4<MP>(xv, xb);
     else if (FMT == QLIN_Q4_K) prep_x_q4<MP, true>(xv, xb);
     else if (FMT == QLIN_Q8_0) prep_x_q8<MP>(xv, xb);
-    else if (FMT == QLIN_Q6_K) prep_x_q8<MP, true>(xv, xb);
+    else if (FMT == QLIN_Q6_K) prep_x_q8<MP>(xv, xb);
     else {
 #pragma unroll
         for (int mm = 0; mm < MP; ++mm) xb[mm] = make_float2(0.f, 0.f);
@@ -457,7 +453,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int kp = 0; kp < 2; ++kp) {
                 float2 p[2][4];
-                dec_q4_pair(cw[2 * kp], cw[2 * kp + 1], p[0], p[1]);
+                dec_q4_pair<FMT == QLIN_Q4_0>(cw[2 * kp], cw[2 * kp + 1], p[0], p[1]);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int k = 2 * kp + h;
@@ -484,7 +480,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
                 for (int mm = 0; mm < MP; ++mm) {
                     const float2 u = __fadd2_rn(s0[mm], s1[mm]);
-                    const float bsum = (u.x + u.y) - xb[mm].x;
+                    const float bsum = u.x + u.y;
                     res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
                 }
             }
@@ -498,7 +494,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 float2 p[2];
-                dec_q8(cw[k], p);
+                dec_q8<128>(cw[k], p);
 #pragma unroll
                 for (int mm = 0; mm < MP; ++mm) {
                     s0[mm] = __ffma2_rn(p[0], xv[mm][2 * k + 0], s0[mm]);
@@ -509,7 +505,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) {
                 const float2 u = __fadd2_rn(s0[mm], s1[mm]);
-                const float bsum = (u.x + u.y) - xb[mm].x;
+                const float bsum = u.x + u.y;
                 res[i][mm] = ACC ? fmaf(d, bsum, res[i][mm]) : d * bsum;
             }
         } else if (FMT == QLIN_Q6_K) {  // Q8_0's byte planes holding 6-bit codes; a scale per 16 values
@@ -524,7 +520,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 float2 p[2];
-                dec_q8(cw[k], p);
+                dec_q8<32>(cw[k], p);
 #pragma unroll
                 for (int mm = 0; mm < MP; ++mm) {
                     s0[k >> 2][mm] = __ffma2_rn(p[0], xv[mm][2 * k + 0], s0[k >> 2][mm]);
@@ -536,7 +532,7 @@ __device__ __forceinline__ void unit_dot(const uint8_t* ub, int lane, const floa
 #pragma unroll
             for (int mm = 0; mm < MP; ++mm) {
                 const float2 u0 = __fadd2_rn(s0[0][mm], s1[0][mm]), u1 = __fadd2_rn(s0[1][mm], s1[1][mm]);
-                const float b0 = (u0.x + u0.y) - xb[mm].x, b1 = (u1.x + u1.y) - xb[mm].y;
+                const float b0 = u0.x + u0.y, b1 = u1.x + u1.y;
                 res[i][mm] = fmaf(e1, b1, ACC ? fmaf(e0, b0, res[i][mm]) : e0 * b0);
             }
         } else if (FMT == QLIN_MXFP4) {  // one 32-element block per part, one UE8M0 scale

@@ -38,6 +38,7 @@ SIGNATURES = {
     "qlin_workspace_bytes": (_SZ, [_I, _I, _I, _I64, _I64, _I, _I]),
     "qlin_gemv": (_I, [_I, _P, _I64, _I64, _P, _I, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "qlin_gemv_noalloc": (_I, [_I, _P, _I64, _I64, _P, _I, _I, _I64, _P, _I64, _I, _P]),
+    "qlin_gemv_noalloc_status": (_I, [_P]),
     "qlin_moe_experts": (_I, [_I, _P, _P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P, _I, _P, _SZ, _P]),
     "qlin_gemm_chunk": (_I, [_I, _P, _I64, _I64, _P, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "qlin_act_quant_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
@@ -46,6 +47,7 @@ SIGNATURES = {
     "qlin_chain_workspace_bytes": (_SZ, [_I, _I, _P, _I]),
     "qlin_gemv_chain": (_I, [_I, _I, _I, _P, _I, _I, _P, _SZ, _P]),
     "qlin_ws_status": (_I, [_P, _P]),
+    "qlin_ws_set_wait_budget": (_I, [_P, ctypes.c_uint32, _P]),
     "qlin_status_string": (ctypes.c_char_p, [_I]),
 }
 
@@ -235,6 +237,11 @@ def qlin_dequant_debug(fmt, packed, N, K, pack_flags=QLIN_PACK_DEFAULT, stream=N
 def qlin_ws_status(ws, stream=None):
     """Read and clear the workspace's sticky device status word (synchronises the stream)."""
     return lib().qlin_ws_status(_dev(ws, "ws"), _stream(stream))
+
+
+def qlin_ws_set_wait_budget(ws, ns, stream=None):
+    """Budget (ns) of the bounded inter-CTA waits of calls using ws; 0 = the default (~2 s)."""
+    _check("qlin_ws_set_wait_budget", lib().qlin_ws_set_wait_budget(_dev(ws, "ws"), int(ns), _stream(stream)))
 
 
 def qlin_status_string(status):

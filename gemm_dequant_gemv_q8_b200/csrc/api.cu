@@ -249,6 +249,15 @@ qlin_status_t qlin_ws_status(void* ws, qlin_stream_t stream) {
     return (word & 1u) ? QLIN_ERR_TIMEOUT : QLIN_ERR_INVALID_ARG;  /* bit 1: bad expert id */
 }
 
+qlin_status_t qlin_ws_set_wait_budget(void* ws, uint32_t ns, qlin_stream_t stream) {
+    if (!ws) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+    cudaError_t e = cudaMemcpyAsync((uint8_t*)ws + qlin::kWsWaitBudgetOff, &ns, sizeof(ns), cudaMemcpyHostToDevice,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);  // ns lives on this stack
+    return cuda_status(e);
+}
+
 const char* qlin_status_string(qlin_status_t s) {
     switch (s) {
         case QLIN_OK: return "QLIN_OK";

@@ -226,7 +226,8 @@ __device__ __forceinline__ void chain_publish(const ChainArgs& a, int j, int t, 
 }
 
 // Finish split tile t of op j: add its n_t published pieces in range order (re-reading, bounded,
-// any word not yet tagged with this launch), then write it.  False if a piece never arrived (~2 s).
+// any word not yet tagged with this launch), then write it.  False if a piece never arrived (~2 s, or the workspace's
+// wait budget).
 template <int MAXM>
 __device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int lane, float gs, uint32_t tag) {
     const ChainOp& o = a.op[j];
@@ -252,7 +253,7 @@ __device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int l
 #pragma unroll
             for (int m = 0; m < MAXM; ++m) ready &= (uint32_t)(w[c][m] >> 32) == tag;
         if (!__all_sync(0xffffffffu, ready)) {  // a piece is not visible yet: re-read (bounded)
-            const uint64_t t0 = globaltimer_ns();
+            const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(a.ws);
             for (uint32_t it = 1;; ++it) {
                 __nanosleep(100);
                 ready = true;
@@ -265,7 +266,7 @@ __device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int l
                             ready &= (uint32_t)(w[c][m] >> 32) == tag;
                         }
                 if (__all_sync(0xffffffffu, ready)) break;
-                if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
+                if (globaltimer_ns() - t0 > budget) return false;
             }
         }
 #pragma unroll
@@ -278,16 +279,17 @@ __device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int l
     return true;
 }
 
-// Bounded wait until every tile of op j is written (2 s); false on timeout.
+// Bounded wait until every tile of op j is written (~2 s, or the workspace's wait budget); false
+// on timeout.
 __device__ __forceinline__ bool chain_wait_op(const ChainArgs& a, int j) {
     const unsigned int* done = reinterpret_cast<const unsigned int*>(a.ws + kChainDoneOff) + j;
     const uint32_t target = (uint32_t)a.op[j].T;
     if (__all_sync(0xffffffffu, ld_acquire_u32(done) >= target)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(a.ws);
     for (uint32_t it = 1;; ++it) {
         __nanosleep(64);
         if (__all_sync(0xffffffffu, ld_acquire_u32(done) >= target)) return true;
-        if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
+        if (globaltimer_ns() - t0 > budget) return false;
     }
 }
 

@@ -186,15 +186,16 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 
 // Grid-wide barrier on a counter that only grows within one launch (reset by the last CTA out).
-// Called by one thread per CTA; false after ~2 s without all CTAs arriving.
-__device__ __forceinline__ bool grid_arrive_wait(unsigned* counter, unsigned target) {
+// Called by one thread per CTA; false after ~2 s (or the workspace's wait budget) without all
+// CTAs arriving.
+__device__ __forceinline__ bool grid_arrive_wait(unsigned* counter, unsigned target, const void* ws) {
     __threadfence();
     atomicAdd(counter, 1u);
     if (ld_acquire_gpu(counter) >= target) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(ws);
     for (uint32_t it = 1;; ++it) {
         if (ld_acquire_gpu(counter) >= target) return true;
-        if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
+        if (globaltimer_ns() - t0 > budget) return false;
         __nanosleep(64);
     }
 }
@@ -442,7 +443,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             for (int w = 0; w < kChunkThreads / 32; ++w) b = fmaxf(b, red[w]);
             atomicMax(&a.words[kWAmax], __float_as_uint(b));  // non-negative floats order as their bits
             float ag = 0.f;
-            if (grid_arrive_wait(&a.words[kWArrive1], gridDim.x)) {
+            if (grid_arrive_wait(&a.words[kWArrive1], gridDim.x, a.status)) {
                 ag = act_global_scale(__uint_as_float(ld_acquire_gpu(&a.words[kWAmax])));
                 if (blockIdx.x == 0) a.words[kWAg] = __float_as_uint(ag);
             } else {
@@ -510,13 +511,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 tile_of(tile, t2, tm, g0, g1);
                 {  // every unit of this tile's activation rows and k-groups quantized (bounded wait)
                     const unsigned* rd = a.ready + (int64_t)tm * a.G;
-                    const uint64_t t0 = globaltimer_ns();
+                    const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(a.status);
                     bool ready = false;
                     while (!ready) {
                         ready = true;
                         for (int g = g0; g < g1; ++g) ready &= ld_relaxed_gpu(rd + g) >= (unsigned)kUnitItems;
                         if (!ready) {
-                            if (globaltimer_ns() - t0 > 2000000000ull) break;
+                            if (globaltimer_ns() - t0 > budget) break;
                             __nanosleep(64);
                         }
                     }

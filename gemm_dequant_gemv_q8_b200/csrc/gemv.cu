@@ -477,12 +477,21 @@ extern "C" qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed
     if (p.ws_bytes > kNoAllocScratchBytes) return QLIN_ERR_WORKSPACE;  // beyond the fixed maximum
     void* scratch = nullptr;
     if (noalloc_scratch(&scratch) != cudaSuccess) return QLIN_ERR_CUDA;
-    // The array keeps the previous call's contents: the status word and the tile tickets must
-    // start at zero (the partial sums are always written before they are read).
-    if (cudaMemsetAsync(scratch, 0, (size_t)ws_partials_off(p.T), (cudaStream_t)stream) != cudaSuccess)
+    // The array keeps the previous call's contents.  The tile tickets must start at zero (a call
+    // that gave up on a wait can leave them set); the partial sums are always written before they
+    // are read.  The status word at offset 0 is left alone: it is sticky, like a workspace's, until
+    // qlin_gemv_noalloc_status reads and clears it (the array starts zeroed when the library loads).
+    if (cudaMemsetAsync((uint8_t*)scratch + ws_counters_off(), 0,
+                        (size_t)(ws_partials_off(p.T) - ws_counters_off()), (cudaStream_t)stream) != cudaSuccess)
         return QLIN_ERR_CUDA;
     return qlin_launch_gemv(fmt, packed, N, K, x, xdt, M, ldx, y, ldy, flags, scratch, (cudaStream_t)stream) ==
                    cudaSuccess
                ? QLIN_OK
                : QLIN_ERR_CUDA;
+}
+
+extern "C" qlin_status_t qlin_gemv_noalloc_status(qlin_stream_t stream) {
+    void* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return QLIN_ERR_CUDA;
+    return qlin_ws_status(scratch, stream);
 }

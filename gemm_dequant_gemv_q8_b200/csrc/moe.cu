@@ -44,8 +44,9 @@ struct MoeArgs {
 };
 
 // Workspace: [0,4) status word (bit 0 timeout, bit 1 bad expert id); [64,68) exit counter;
-// [256, ...) per-work-entry gate_up tile counts; per-(token, down tile) combine tickets (both
-// reset by the last CTA to leave); then the down outputs o and the SiLU-gate outputs h.
+// [256, ...) per-work-entry gate_up tile counts (reset by the last CTA to leave); per-(token, down
+// tile) combine tickets (reset by the combine that uses them, or, after a failed wait, by the
+// last CTA to leave); then the down outputs o and the SiLU-gate outputs h.
 constexpr int64_t kMoeExitOff = 64;
 constexpr int64_t kMoeDoneOff = 256;
 constexpr int kMoeMaxT1 = 1024;  // down tiles per expert (H <= 32768)
@@ -332,19 +333,19 @@ __device__ __forceinline__ void moe_write_tile(const MoeArgs& a, const RouteSmem
     }
 }
 
-// Bounded wait until *p >= target (2 s); false on timeout.
-__device__ __forceinline__ bool moe_wait_count(const unsigned int* p, uint32_t target) {
+// Bounded wait until *p >= target (~2 s, or the workspace's wait budget); false on timeout.
+__device__ __forceinline__ bool moe_wait_count(const unsigned int* p, uint32_t target, const void* ws) {
     auto ld = [&]() {
         uint32_t v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
         return v;
     };
     if (__all_sync(0xffffffffu, ld() >= target)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(ws);
     for (uint32_t it = 1;; ++it) {
         __nanosleep(64);
         if (__all_sync(0xffffffffu, ld() >= target)) return true;
-        if ((it & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) return false;
+        if (globaltimer_ns() - t0 > budget) return false;
     }
 }
 
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
             // down units read h: wait (bounded) for this entry's gate_up tiles
             if (s == 1 && act != waited && !failed) {
                 waited = act;
-                if (!moe_wait_count(done + act, (uint32_t)a.T0)) failed = true;
+                if (!moe_wait_count(done + act, (uint32_t)a.T0, a.ws)) failed = true;
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -590,7 +591,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
         }
     }
     __syncwarp();
-    // The last CTA to leave resets the tile counts.
+    // The last CTA to leave resets the tile counts, and after a failed wait also the combine
+    // tickets (a unit that gave up took none, so some tokens' tickets stopped short of zero).
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -599,6 +601,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm) moe
             __threadfence();
             unsigned int* dn = reinterpret_cast<unsigned int*>(a.ws + kMoeDoneOff);
             for (int j = 0; j < kMoeMaxAct; ++j) dn[j] = 0u;
+            if (__ldcg(reinterpret_cast<const unsigned int*>(a.ws)) & 1u) {
+                unsigned int* comb = reinterpret_cast<unsigned int*>(a.ws + moe_comb_off());
+                for (int j = 0; j < a.M * a.T1; ++j) comb[j] = 0u;
+            }
             *ex = 0u;
         }
     }

@@ -124,6 +124,16 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Budget of the bounded waits between CTAs (dependency counts, grid barriers, partial sums of
+// other CTAs): the uint32 at byte kWsWaitBudgetOff of a workspace, in nanoseconds, or ~2 s when it
+// is 0 (a zero-filled workspace).  Set with qlin_ws_set_wait_budget; read once per launch.
+constexpr int64_t kWsWaitBudgetOff = 32;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+__device__ __forceinline__ uint64_t ws_wait_budget_ns(const void* ws) {
+    const unsigned v = __ldcg(reinterpret_cast<const unsigned*>(reinterpret_cast<const uint8_t*>(ws) + kWsWaitBudgetOff));
+    return v ? (uint64_t)v : kDefaultWaitNs;
+}
+
 // Bounded wait on an mbarrier phase: gives up after ~timeout_ns and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t timeout_ns = 2000000000ull) {

@@ -15,8 +15,10 @@
  * Conventions for every entry point
  *   - W is N x K (output x input), row-major along K; y[m][n] = sum_k x[m][k] * W[n][k].
  *   - Every pointer argument is a caller-owned DEVICE pointer unless stated otherwise.  The
- *     library allocates nothing and keeps no global state (apart from a per-device SM-count
- *     cache); all work is enqueued asynchronously on `stream` (NULL = the legacy default stream).
+ *     library allocates nothing and keeps no global state, with two exceptions: a per-device
+ *     SM-count cache, and qlin_gemv_noalloc's fixed 8 MiB __device__ scratch array (held by every
+ *     GPU that loads the library) with its per-device address cache and the mutex guarding it.
+ *     All work is enqueued asynchronously on `stream` (NULL = the legacy default stream).
  *   - Arguments are validated on the host before anything is launched; a failed check returns
  *     its status code and enqueues nothing.  A launch failure returns QLIN_ERR_CUDA.
  *   - No C++ exception crosses this boundary.
@@ -146,7 +148,9 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
  * Weights stream from HBM once; dequantization happens in registers; products and sums are fp32
  * (activations are never quantized).  Results are deterministic for a given device and shape.
  * Q8_0 / Q4_0 / Q4_K / Q6_K products are exact in fp32 for activations with 2^-40 <= |x| < 2^65; below that
- * range a product is exact to 2^-63 in absolute terms, at or above it the result overflows.
+ * range a product is exact to 2^-63 in absolute terms, at or above it the result overflows.  A 32-value
+ * block whose scaled sum |d * sum q x| falls below 2^-40 (a tiny scale times tiny activations) is exact
+ * to about 2^-64 in absolute terms.
  * The dequantize-and-multiply of quantized weight blocks against activations is the "NVFP4
  * block-scaled GEMM/GEMV" and "dp4a Q8_0 decode" of the imp pages (README "Features"; release
  * notes v0.4.1), re-designed here for sm_100a. */
@@ -166,12 +170,19 @@ qlin_status_t qlin_gemv(qlin_format_t fmt, const void* packed, int64_t N, int64_
  *     with QLIN_ERR_WORKSPACE before anything is enqueued.
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
  *     with that device current); make that first call before any stream capture.
- *   - Every call clears the array's status word and tickets on `stream` (cudaMemsetAsync), then
- *     launches the kernel.  All calls share the one array: calls that can overlap on the GPU
- *     (different streams without ordering between them) race and must not be issued. */
+ *   - Every call clears the array's tile tickets on `stream` (cudaMemsetAsync), then launches the
+ *     kernel.  All calls share the one array: calls that can overlap on the GPU (different
+ *     streams without ordering between them) race and must not be issued.
+ *   - The array's status word is sticky across calls, as a workspace's is: a bounded device wait
+ *     that gave up sets it, and qlin_gemv_noalloc_status reads and clears it. */
 qlin_status_t qlin_gemv_noalloc(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,
                                 const void* x, qlin_dtype_t xdt, int M, int64_t ldx, float* y,
                                 int64_t ldy, int flags, qlin_stream_t stream);
+
+/* Read and clear the status word of qlin_gemv_noalloc's scratch array on the current device, as
+ * qlin_ws_status does for a workspace (synchronises `stream`): QLIN_OK, or QLIN_ERR_TIMEOUT if a
+ * bounded device wait of some qlin_gemv_noalloc call on this device gave up since the last check. */
+qlin_status_t qlin_gemv_noalloc_status(qlin_stream_t stream);
 
 /* ------------------------------------------------------------------------- GEMV chains */
 
@@ -300,6 +311,18 @@ qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t 
  * Returns QLIN_OK, QLIN_ERR_TIMEOUT if a bounded device wait gave up since the last check, or
  * QLIN_ERR_INVALID_ARG if qlin_moe_experts met an invalid or repeated expert id. */
 qlin_status_t qlin_ws_status(void* ws, qlin_stream_t stream);
+
+/* Test and fault-injection aid: set the budget, in nanoseconds, of the bounded device waits between
+ * CTAs in the calls that use workspace `ws` -- qlin_gemv_chain's dependency and partial-sum waits,
+ * qlin_moe_experts' waits for an expert's gate_up tiles, qlin_gemm_chunk's (NVFP4) grid barrier and
+ * activation-ready waits.  0 restores the default of about 2 s.  The value is kept in the workspace
+ * (the uint32 at byte 32, which a zero-filled workspace has at 0) until it is set again.  A wait
+ * that runs out sets the status word (qlin_ws_status then reports QLIN_ERR_TIMEOUT), its warp
+ * abandons the rest of its work and waits (bounded) for its own copies in flight, and the launch
+ * finishes; that call's outputs are unspecified, and the workspace is usable again by the next
+ * call.  Waits for this CTA's own bulk copies are not affected.  Synchronises `stream`.  The pages
+ * have no counterpart (the Imparo README, "Why Imparo", reports failures rather than hiding them). */
+qlin_status_t qlin_ws_set_wait_budget(void* ws, uint32_t ns, qlin_stream_t stream);
 
 const char* qlin_status_string(qlin_status_t status);
 

@@ -4,21 +4,25 @@
 Default workload: a synthetic Q4_0 dense decode layer stack shaped like a 4B model at M = 1:
 36 layers of hidden 2560, each with the projections q/k/v (2560 -> 4096/1024/1024, packed and
 launched as one fused 6144-row GEMV), o (4096 -> 2560), gate_up (2560 -> 2 x 9728, fused SiLU gate)
-and down (9728 -> 2560).  One step = one decode token through all 36 layers = 144 GEMV launches,
-captured once in a CUDA graph (with programmatic dependent launch between the kernels) and
-replayed.  Attention, norms, embeddings and the LM head are not part of the path and are not run.
+and down (9728 -> 2560).  One step = one decode token through all 36 layers: the 144 GEMVs run as
+one persistent qlin_gemv_chain launch, captured in a CUDA graph and replayed.  Attention, norms,
+embeddings and the LM head are not part of the path and are not run.
 
 Metric: quantized GEMV weight-stream GB/s (algorithmic bytes: packed codes + scales + activations
-+ outputs, each once) and the equivalent decode tokens/s; JSON line on stdout (rank 0).
++ outputs, each once) and the equivalent decode tokens/s; one JSON line on stdout (rank 0).  With
+one GPU the line also carries a "configs" object: the other workloads (the Q8_0 GEMV, the NVFP4
+27B-shaped MLP at M = 1 and 4, the Q4_0 8B-A1B-shaped MoE layer at M = 1 and 8, the NVFP4 prefill
+chunk at M = 512 and 64 plus an M sweep), each with its value, roofline, clocks and CPU baseline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qlin|reference] [--config NAME]
 
 --impl reference times the fp64 CPU oracle (the test reference) on a bounded sample of the same
-workload; the oracle is used nowhere else in this file except the cpu_baseline leg.
+workload; the oracle is used nowhere else in this file except the cpu_baseline legs.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -26,6 +30,7 @@ import subprocess
 import sys
 import threading
 import time
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -49,6 +54,49 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def fp4_peaks():
+    """FP4 dense tensor denominators (TFLOP/s): the measured cuBLAS bf16 burst x 4 (NVIDIA's nominal
+    fp4/bf16 ratio) as the roofline peak, and the 9 PFLOP/s dense spec beside it."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        return 4 * bf16, "measured bf16 burst (cuBLAS) x 4, the nominal fp4/bf16 ratio", 9000.0
+    except Exception:
+        return 4 * 1590.0, "fallback bf16 x 4", 9000.0
+
+
+def bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured bf16 burst (cuBLAS)"
+    except Exception:
+        return 1590.0, "fallback bf16"
+
+
+def sources_sha(names):
+    """Short hash of library sources, so a recorded ncu traffic figure is used only for the
+    kernel it was captured from."""
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "gemm_dequant_gemv_q8_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(key):
+    """dram read + write bytes per launch from profiles/traffic.json, or None when the capture is
+    of other sources than the current ones (the figure is then stale)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t.get(key)
+        if not e or e.get("sources_sha") != sources_sha(e["sources"]):
+            return None
+        return e["bytes_per_launch"]
+    except Exception:
+        return None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -310,50 +358,34 @@ def time_graph(graph, steps, warmup):
     return a.elapsed_time(b) / steps
 
 
-def time_chain_kernel(stack, reps=3):
-    """Average duration of one chain launch, timed with CUDA events on the launching stream
-    (eager launches, no graph); algorithmic bytes of the ops that launch covers."""
+def time_chain_kernel(stack, reps=4):
+    """Average duration of one chain launch: `reps` steps' chain launches (no PDL, so launches do
+    not overlap) captured in one CUDA graph, timed with CUDA events on the stream that replays it.
+    Returns (ms per launch, algorithmic bytes per launch)."""
     q = stack.q
-    st = torch.cuda.current_stream()
 
     def run():
-        for ops, ws in stack.chains:
-            q.qlin_gemv_chain(stack.fmt, q.QLIN_F32, stack.M, ops, ws=ws)
+        for _ in range(reps):
+            for ops, ws in stack.chains:
+                q.qlin_gemv_chain(stack.fmt, q.QLIN_F32, stack.M, ops, ws=ws)
 
-    run()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(st)
-    for _ in range(reps):
-        run()
-    b.record(st)
-    b.synchronize()
-    ms = a.elapsed_time(b) / (reps * len(stack.chains))
+    ms = _time_graph_of(run, 3, 2) / (reps * len(stack.chains))
     return ms, stack.step_bytes / len(stack.chains)
 
 
 def time_dominant_kernel(stack, reps=3):
-    """Average duration of the gate_up + SiLU GEMV launch (the largest per-launch share),
-    timed with CUDA events on the launching stream, rotating over the layers' matrices
-    (1 GB of weights at 36 layers, so every launch streams from HBM)."""
+    """Average duration of the gate_up + SiLU GEMV launch (the largest per-launch share): a graph of
+    every layer's gate_up launch (1 GB of weights at 36 layers, so every launch streams from HBM),
+    timed with CUDA events."""
     q = stack.q
     name, N, K, epi = STACK[2]
-    st = torch.cuda.current_stream()
 
     def run():
         for l in range(stack.layers):
             q.qlin_gemv(stack.fmt, stack.packed[l][2], N, K, stack.x[(l, 2)], y=stack.y[(l, 2)],
                         ws=stack.ws[l][2], flags=q.QLIN_EPI_SILU_GATE)
 
-    run()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(st)
-    for _ in range(reps):
-        run()
-    b.record(st)
-    b.synchronize()
-    ms = a.elapsed_time(b) / (reps * stack.layers)
+    ms = _time_graph_of(run, reps, 2) / stack.layers
     bytes_ = (q.qlin_packed_bytes(stack.fmt, N, K, q.QLIN_PACK_GATE_UP) - 256) + 4 * stack.M * (K + N // 2)
     return ms, bytes_
 
@@ -361,7 +393,7 @@ def time_dominant_kernel(stack, reps=3):
 def e2e_stack(stack, steps, warmup, pdl=True):
     """Same metric through the public API with host buffers: every step copies its inputs from
     pinned host memory, runs the stack, and reads its outputs back, all inside the timed region
-    (one graph: H2D copy, 144 GEMV launches, D2H copy)."""
+    (one graph: H2D copy, the chain launch, D2H copy)."""
     hx = stack.xbuf.cpu().pin_memory()
     hy = torch.empty(stack.ybuf.shape, dtype=torch.float32).pin_memory()
     g = stack.capture(pdl, host_io=(hx, hy))
@@ -370,37 +402,76 @@ def e2e_stack(stack, steps, warmup, pdl=True):
     return ms, hx.numel() * 4, hy.numel() * 4
 
 
-def cpu_baseline_stack(fmt, budget_s=12.0, seed=7):
-    """The fp64 oracle on a bounded sample of the stack: rows of every projection shape, timed
-    on the host; scaled to GB/s of weights processed.  Returns (GB/s, cores, description)."""
-    import oracle
-    rng = np.random.default_rng(seed)
-    per_shape = []
-    for (name, N, K, epi) in STACK:
-        b, s, gs = synth.weights(fmt, 64, K, synth.gen(seed + N))
-        x = synth.activations(1, K, synth.gen(seed + K)).double().numpy()
-        per_shape.append((N, K, b.numpy(), None if s is None else s.numpy(), gs, x))
-    # probe, then size the sample to the budget
-    done_bytes, t_used, rows = 0, 0.0, 0
-    t0 = time.perf_counter()
-    while t_used < budget_s:
-        for (N, K, b, s, gs, x) in per_shape:
-            r = rng.integers(0, 64, 16)
-            oracle.gemv(fmt, 64, K, b, x, scales=s, g=gs, rows=r)
-            rowb = oracle.row_bytes(fmt, K)
-            done_bytes += 16 * rowb
-            rows += 16
-        t_used = time.perf_counter() - t0
-    gbs = done_bytes / t_used / 1e9
-    desc = (f"{rows} weight rows of the four stack projection shapes (K = 2560/4096/2560/9728), "
-            f"single-threaded fp64 oracle, {t_used:.1f} s")
-    return gbs, 1, desc
+# ----------------------------------------------------------------------------- CPU baseline
+def cpu_info():
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    return model, n
 
+
+def oracle_rate(fmt, shapes, M, budget_s, threads, seed=7, xdt=torch.float32):
+    """The fp64 oracle (as it stands) on a bounded sample: the 64 rows of a 64-row block of each
+    (N, K) projection shape, in a random order, against M activation rows, repeated for budget_s seconds
+    on `threads` host threads (the oracle's C calls release the GIL, so the threads run on separate
+    cores).  Its cost per row depends on K only, so a 64-row block stands for all N rows.
+    Returns (weight GB/s, GFLOP/s, rows, seconds)."""
+    import oracle
+    data = []
+    for (N, K) in shapes:
+        b, s, gs = synth.weights(fmt, 64, K, synth.gen(seed + K))
+        x = synth.activations(M, K, synth.gen(seed + 1 + K), dtype=xdt).double().numpy()
+        data.append((K, b.numpy(), None if s is None else s.numpy(), gs, x, oracle.row_bytes(fmt, K)))
+
+    def work(tid):
+        rng = np.random.default_rng(seed + tid)
+        nb = fl = rows = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget_s:
+            for (K, b, s, gs, x, rb) in data:
+                oracle.gemv(fmt, 64, K, b, x, scales=s, g=gs, rows=rng.permutation(64))
+                nb += 64 * rb
+                fl += 2 * M * K * 64
+                rows += 64
+        return nb, fl, rows, time.perf_counter() - t0
+
+    if threads == 1:
+        res = [work(0)]
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            res = list(ex.map(work, range(threads)))
+    t = max(r[3] for r in res)
+    return sum(r[0] for r in res) / t / 1e9, sum(r[1] for r in res) / t / 1e9, sum(r[2] for r in res), t
+
+
+def cpu_baseline(fmt, shapes, M, unit="GB/s", budget_s=2.5, xdt=torch.float32, what=""):
+    """cpu_baseline object: the oracle timed on all host cores and on one core."""
+    model, ncores = cpu_info()
+    g_all, f_all, rows_all, t_all = oracle_rate(fmt, shapes, M, budget_s, ncores, xdt=xdt)
+    g_one, f_one, rows_one, t_one = oracle_rate(fmt, shapes, M, budget_s, 1, xdt=xdt)
+    pick = (lambda g, f: g) if unit == "GB/s" else (lambda g, f: f / 1e3)  # TFLOP/s
+    ks = "/".join(str(K) for _, K in shapes)
+    return {"value": pick(g_all, f_all), "unit": unit, "cores": ncores, "kind": "oracle",
+            "sample": (f"{rows_all} weight rows of the {what or 'workload'} projection shapes (K = {ks}) x M = {M} "
+                       f"activation rows, fp64 oracle on {ncores} host threads for {t_all:.1f} s"),
+            "single_thread": {"value": pick(g_one, f_one), "unit": unit, "cores": 1,
+                              "sample": f"{rows_one} rows, one thread, {t_one:.1f} s"},
+            "cpu_model": model}
 
 
 # ----------------------------------------------------------------------------- other configs
-def _time_graph_of(fn, steps, warmup):
-    """Capture fn() (a sequence of launches) in one CUDA graph and time replays with events."""
+def _graph_of(fn):
+    """fn() (a sequence of launches) captured in one CUDA graph, after one eager warm-up run."""
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
@@ -410,126 +481,260 @@ def _time_graph_of(fn, steps, warmup):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def _time_graph_of(fn, steps, warmup):
+    """Capture fn() in one CUDA graph and time replays with events (ms per replay)."""
+    g = _graph_of(fn)
     ms = time_graph(g, steps, warmup)
     del g
     return ms
 
 
+def timed(fn, steps, warmup, min_s=0.3):
+    """ms per replay of fn's graph and the clocks sampled meanwhile: `steps` replays between two
+    events, repeated until at least min_s of device time has passed (so the clock sampler sees the
+    region), after `warmup` untimed replays."""
+    g = _graph_of(fn)
+    for _ in range(max(warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total_ms, n = 0.0, 0
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        while total_ms < 1e3 * min_s:
+            a.record()
+            for _ in range(steps):
+                g.replay()
+            b.record()
+            b.synchronize()
+            total_ms += a.elapsed_time(b)
+            n += steps
+    del g
+    return total_ms / n, clk.summary()
+
+
+def roofline_hbm(kernel, bytes_per_launch, us_per_launch, traffic=None):
+    peak, src = peaks()
+    gbs = bytes_per_launch / (us_per_launch * 1e-6) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peak, "peak_source": f"{src} hbm_gbs (copy)",
+            "unit": "GB/s", "frac": gbs / peak, "traffic": traffic,
+            "algorithmic_bytes_per_launch": bytes_per_launch, "avg_launch_us": us_per_launch}
+
+
+def roofline_fp4(kernel, flop_per_launch, us_per_launch):
+    peak, src, spec = fp4_peaks()
+    tf = flop_per_launch / (us_per_launch * 1e-6) / 1e12
+    return {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peak, "peak_source": src,
+            "unit": "TFLOP/s", "frac": tf / peak, "traffic": None, "spec_peak": spec, "frac_of_spec": tf / spec,
+            "algorithmic_flop_per_launch": flop_per_launch, "avg_launch_us": us_per_launch}
+
+
+def cfg_q8_small(args, cpu=True):
+    """Q8_0 GEMV, M = 1, K = 1024, N = 256: launch-latency bound; a graph of 1000 launches over
+    distinct weight copies (278 MB, more than twice L2)."""
+    import gemm_dequant_gemv_q8_b200 as q
+    fmt, N, K, M, copies = q.QLIN_Q8_0, 256, 1024, 1, 1000
+    packs = []
+    for c in range(copies):
+        b, s_, g = synth.weights(fmt, N, K, synth.gen(1000 + c, device="cuda"), device="cuda")
+        packs.append(q.qlin_pack_weights(fmt, N, K, b, s_, g))
+    x = synth.activations(M, K, synth.gen(1, device="cuda"), device="cuda")
+    y = torch.empty(M, N, device="cuda")
+    ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, N, K)) for _ in range(copies)]
+    fn = lambda: [q.qlin_gemv(fmt, packs[c], N, K, x, y=y, ws=ws[c], flags=q.QLIN_FLAG_PDL) for c in range(copies)]
+    ms, clk = timed(fn, 3, args.warmup)
+    us = ms * 1e3 / copies
+    bytes_ = (q.qlin_packed_bytes(fmt, N, K) - 256) + 4 * M * (K + N)
+    e = {"workload": "Q8_0 GEMV M=1 K=1024 N=256 (launch-latency bound; graph of 1000 launches over distinct "
+                     "weight copies, PDL)", "M": M, "value": bytes_ / (us * 1e-6) / 1e9, "unit": "GB/s",
+         "us_per_launch": us, "gpu_launches_per_replay": copies,
+         "roofline": roofline_hbm("gemv_kernel<Q8_0, M=1>", bytes_, us), "clocks": clk,
+         "l2": "1000 distinct weight copies (278 MB) per replay, more than twice L2"}
+    if cpu:
+        e["cpu_baseline"] = cpu_baseline(fmt, [(N, K)], M, what="Q8_0 GEMV")
+    return {"q8_0_gemv_m1": e}
+
+
+def cfg_mlp(args, fmt_name="nvfp4", cpu=True):
+    """27B-shaped MLP (gate_up 5120 -> 2 x 17408 + SiLU, down 17408 -> 5120), bf16 activations,
+    M = 1 and 4.  Two layers with distinct weights (300 MB) per replay; the step is both layers as
+    one GEMV chain with h in bf16 (the headline value), and also one qlin_gemv per projection."""
+    import gemm_dequant_gemv_q8_b200 as q
+    fmt = q.QLIN_NVFP4 if fmt_name == "nvfp4" else q.QLIN_MXFP4
+    H, I, L = 5120, 17408, 2
+    gu, dn = [], []
+    for l in range(L):
+        b, s_, g = synth.weights(fmt, 2 * I, H, synth.gen(3000 + l, device="cuda"), device="cuda")
+        gu.append(q.qlin_pack_weights(fmt, 2 * I, H, b, s_, g, q.QLIN_PACK_GATE_UP))
+        b, s_, g = synth.weights(fmt, H, I, synth.gen(3100 + l, device="cuda"), device="cuda")
+        dn.append(q.qlin_pack_weights(fmt, H, I, b, s_, g))
+        del b, s_
+    wb = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
+    out = {}
+    for M in (1, 4):
+        x = synth.activations(M, H, synth.gen(3200, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        h = torch.empty(M, I, device="cuda")
+        y = torch.empty(M, H, device="cuda")
+        wsg = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, 2 * I, H)) for _ in range(L)]
+        wsd = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, H, I)) for _ in range(L)]
+
+        def fn():
+            for l in range(L):
+                q.qlin_gemv(fmt, gu[l], 2 * I, H, x, y=h, ws=wsg[l], flags=q.QLIN_EPI_SILU_GATE | q.QLIN_FLAG_PDL)
+                q.qlin_gemv(fmt, dn[l], H, I, h, y=y, ws=wsd[l], flags=q.QLIN_FLAG_PDL)
+        ms1 = _time_graph_of(fn, args.steps, args.warmup) / L
+        bytes1 = wb + M * (2 * H + 4 * I + 4 * I + 4 * H)
+        hb = [torch.empty(M, I, device="cuda", dtype=torch.bfloat16) for _ in range(L)]
+        ops = []
+        for l in range(L):
+            ops.append(q.gemv_op(gu[l], 2 * I, H, x, hb[l], q.QLIN_EPI_SILU_GATE | q.QLIN_OUT_BF16))
+            ops.append(q.gemv_op(dn[l], H, I, hb[l], y, q.QLIN_EPI_NONE, len(ops) - 1))
+        cws = q.workspace(q.qlin_chain_workspace_bytes(fmt, M, ops))
+        fn2 = lambda: q.qlin_gemv_chain(fmt, q.QLIN_BF16, M, ops, flags=q.QLIN_FLAG_PDL, ws=cws)
+        ms, clk = timed(fn2, args.steps, args.warmup)
+        bytes2 = wb + M * (2 * H + 2 * I + 2 * I + 4 * H)  # per layer; h in bf16
+        gbs = bytes2 / (ms / L * 1e-3) / 1e9
+        e = {"workload": f"{fmt_name.upper()} MLP shaped like a 27B model: gate_up 5120->2x17408 + SiLU, down "
+                         f"17408->5120, bf16 x, M={M}; both of two layers' projections as one GEMV chain "
+                         "(h in bf16), two layers with distinct weights per replay (300 MB)",
+             "M": M, "value": gbs, "unit": "GB/s", "us_per_layer": ms / L * 1e3, "tokens_per_s": M / (ms / L * 1e-3),
+             "launches_per_layer": {"us_per_layer": ms1 * 1e3, "gbs": bytes1 / (ms1 * 1e-3) / 1e9,
+                                    "note": "one qlin_gemv per projection, fp32 h"},
+             "roofline": roofline_hbm(f"chain_kernel<{fmt_name.upper()}, bf16 x, M={M}> (4 GEMVs: 2 layers)",
+                                      L * bytes2, ms * 1e3),
+             "clocks": clk}
+        if cpu:
+            e["cpu_baseline"] = cpu_baseline(fmt, [(2 * I, H), (H, I)], M, xdt=torch.bfloat16,
+                                             what=f"{fmt_name.upper()} MLP")
+        out[f"{fmt_name}_mlp_m{M}"] = e
+    return out
+
+
+def cfg_moe(args, cpu=True):
+    """Q4_0 MoE expert layer shaped like an 8B-A1B model (hidden 2048, 32 experts of gate_up
+    2048 -> 2 x 1792 and down 1792 -> 2048, top-4), M = 1 and 8 tokens with independent routing; a
+    graph of 8 layers with distinct weights (1.6 GB), so one replay's selected experts exceed L2."""
+    import gemm_dequant_gemv_q8_b200 as q
+    fmt, E, H, I, k, L = q.QLIN_Q4_0, 32, 2048, 1792, 4, 8
+    gu, dn = [], []
+    for l in range(L):
+        c = [synth.weights(fmt, 2 * I, H, synth.gen(4000 + 100 * l + e, device="cuda"), device="cuda") for e in range(E)]
+        gu.append(q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_GATE_UP))
+        c = [synth.weights(fmt, H, I, synth.gen(5000 + 100 * l + e, device="cuda"), device="cuda") for e in range(E)]
+        dn.append(q.pack_experts(fmt, E, H, I, c))
+        del c
+    per_expert = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
+    out = {}
+    for M in (1, 8):
+        logits = [synth.router_logits(M, E, synth.gen(6000 + l, device="cuda"), device="cuda") for l in range(L)]
+        x = synth.activations(M, H, synth.gen(6100, device="cuda"), device="cuda")
+        ids = torch.empty(M, k, dtype=torch.int32, device="cuda")
+        w = torch.empty(M, k, device="cuda")
+        y = torch.empty(M, H, device="cuda")
+        ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE, fmt, M, H, I, E, k)) for _ in range(L)]
+
+        def fn():
+            for l in range(L):
+                q.qlin_moe_experts(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
+                                   topk_w=w, y=y, ws=ws[l], flags=q.QLIN_FLAG_PDL)
+        ms, clk = timed(fn, args.steps, args.warmup)
+        distinct = []
+        for l in range(L):  # actual distinct experts per layer for these seeds
+            q.qlin_moe_experts(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
+                               topk_w=w, y=y, ws=ws[l])
+            distinct.append(len(set(ids.cpu().flatten().tolist())))
+        nd = sum(distinct) / L
+        bytes_ = nd * per_expert + M * (4 * H + 4 * H + 4 * E)
+        us = ms / L * 1e3
+        e = {"workload": "Q4_0 MoE expert layer shaped like an 8B-A1B model: hidden 2048, 32 experts gate_up "
+                         f"2048->2x1792, down 1792->2048, top-4, M={M} tokens; a graph of 8 layers' launches "
+                         "(distinct weights, 1.6 GB)", "M": M, "distinct_experts": nd,
+             "value": bytes_ / (us * 1e-6) / 1e9, "unit": "GB/s", "us_per_layer": us,
+             "roofline": roofline_hbm(f"moe_kernel<Q4_0, M={M}> (route + gate_up + SiLU + down + combine)", bytes_, us),
+             "clocks": clk,
+             "bytes": "selected experts' packed weights (the actual distinct count per layer) + x, y, logits"}
+        if cpu:
+            e["cpu_baseline"] = cpu_baseline(fmt, [(2 * I, H), (H, I)], M, what="MoE expert")
+        out[f"q4_0_moe_m{M}"] = e
+    del gu, dn
+    return out
+
+
+def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
+    """NVFP4 prefill-chunk GEMM, K = 5120, N = 17408: M = 512 (tensor-bound) and 64 (HBM-bound),
+    and an M sweep on the same matrix; two weight copies alternate so that consecutive calls do not
+    find the weights in L2."""
+    import gemm_dequant_gemv_q8_b200 as q
+    fmt, N, K = q.QLIN_NVFP4, 17408, 5120
+    packs = []
+    for c in range(2):
+        b, s_, g = synth.weights(fmt, N, K, synth.gen(7000 + c, device="cuda"), device="cuda")
+        packs.append(q.qlin_pack_weights(fmt, N, K, b, s_, g, q.QLIN_PACK_MMA))
+        del b, s_
+    wbytes = q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA) - 256
+    out, sw = {}, {}
+    for M in (512, 64) + tuple(sweep):
+        x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(M, N, device="cuda")
+        ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+        fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL) for c in range(2)]
+        ms, clk = timed(fn, args.steps, args.warmup)
+        us = ms / 2 * 1e3
+        flop = 2.0 * M * N * K
+        bytes_ = wbytes + 2 * M * K + 4 * M * N
+        tf, gbs = flop / (us * 1e-6) / 1e12, bytes_ / (us * 1e-6) / 1e9
+        if M in (512, 64):
+            kern = f"chunk_gemm_kernel<1> (activation quantization + tcgen05 mxf4nvf4 GEMM), M={M}"
+            e = {"workload": f"NVFP4 prefill-chunk GEMM M={M} K=5120 N=17408, bf16 x, fp32 accumulate; one persistent "
+                             "launch; two weight copies alternate", "M": M, "us_per_call": us,
+                 "tflops": tf, "gbs": gbs, "clocks": clk}
+            if M == 512:
+                e.update(value=tf, unit="TFLOP/s", roofline=roofline_fp4(kern, flop, us))
+                if cpu:
+                    e["cpu_baseline"] = cpu_baseline(fmt, [(N, K)], M, unit="TFLOP/s", xdt=torch.bfloat16,
+                                                     what="NVFP4 chunk")
+            else:
+                e.update(value=gbs, unit="GB/s", roofline=roofline_hbm(kern, bytes_, us))
+                if cpu:
+                    e["cpu_baseline"] = cpu_baseline(fmt, [(N, K)], M, xdt=torch.bfloat16, what="NVFP4 chunk")
+            out[f"nvfp4_chunk_m{M}"] = e
+        else:
+            sw[str(M)] = {"us_per_call": us, "tflops": tf, "gbs": gbs, "hbm_frac": gbs / peaks()[0]}
+    if sw:
+        out["nvfp4_chunk_m_sweep"] = {"workload": "the same GEMM at small M (the GEMV regime on the chunk path)",
+                                      "by_M": sw}
+    return out
+
+
+CONFIGS = {"q8_small": cfg_q8_small, "nvfp4_mlp": cfg_mlp, "moe": cfg_moe, "chunk": cfg_chunk,
+           "mxfp4_mlp": lambda a, cpu=True: cfg_mlp(a, "mxfp4", cpu)}
+
+
 def run_config(name, args):
-    """Measure one of the non-default workloads; one JSON line per (config, M)."""
+    """Measure one workload other than the default stack; one JSON line per entry."""
     import gemm_dequant_gemv_q8_b200 as q
     torch.cuda.set_device(0)
-    peak, peak_src = peaks()
-    lines = []
-    if name in ("q4_k_stack", "q6_k_stack"):
+    entries = {}
+    if name in CONFIGS:
+        entries = CONFIGS[name](args, cpu=not args.no_cpu_baseline)
+    elif name in ("q4_k_stack", "q6_k_stack"):
         # the default stack's shapes (every K a multiple of 256) in a GGUF K-quant, one chain per step
         fmt, fname, per256 = (q.QLIN_Q4_K, "Q4_K", 144) if name == "q4_k_stack" else (q.QLIN_Q6_K, "Q6_K", 210)
         stack = DenseStack(fmt, args.layers, mode="chain")
-        graph = stack.capture(pdl=True)
-        ms = time_graph(graph, args.steps, max(args.warmup, 3))
-        del graph
+        ms, clk = timed(lambda: stack.step(True), args.steps, args.warmup)
         canon = sum(N * K * per256 // 256 for (_, N, K, _) in STACK) * args.layers
-        lines.append(dict(workload=f"{fname} dense decode layer stack, the Q4_0 stack's shapes ({args.layers} layers "
-                          "of hidden 2560: qkv 2560->6144, o 4096->2560, gate_up 2560->2x9728 + SiLU, "
-                          "down 9728->2560), one GEMV chain per step", M=1, ms_per_step=ms,
-                          packed_weight_bytes=stack.weight_bytes, canonical_weight_bytes=canon,
-                          gbs=stack.step_bytes / (ms * 1e-3) / 1e9, decode_tok_s=1e3 / ms,
-                          l2="inputs larger than L2: %.2f GB of packed weights per step" % (stack.weight_bytes / 1e9)))
-    if name == "q8_small":
-        fmt, N, K, M, copies = q.QLIN_Q8_0, 256, 1024, 1, 1000  # 278 MB of rotating copies > 2x L2
-        packs = []
-        for c in range(copies):
-            b, s_, g = synth.weights(fmt, N, K, synth.gen(1000 + c, device="cuda"), device="cuda")
-            packs.append(q.qlin_pack_weights(fmt, N, K, b, s_, g))
-        x = synth.activations(M, K, synth.gen(1, device="cuda"), device="cuda")
-        y = torch.empty(M, N, device="cuda")
-        ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, N, K)) for _ in range(copies)]
-        fn = lambda: [q.qlin_gemv(fmt, packs[c], N, K, x, y=y, ws=ws[c], flags=q.QLIN_FLAG_PDL) for c in range(copies)]
-        ms = _time_graph_of(fn, max(3, args.steps // 4), args.warmup) / copies
-        wb = q.qlin_packed_bytes(fmt, N, K) - 256
-        bytes_ = wb + 4 * M * (K + N)
-        lines.append(dict(workload="Q8_0 GEMV M=1 K=1024 N=256 (launch-latency bound; graph of 1000 "
-                          "launches over distinct weight copies, PDL)", M=M, us_per_launch=ms * 1e3,
-                          gbs=bytes_ / (ms * 1e-3) / 1e9))
-    elif name in ("nvfp4_mlp", "mxfp4_mlp"):
-        fmt, H, I = (q.QLIN_NVFP4 if name == "nvfp4_mlp" else q.QLIN_MXFP4), 5120, 17408
-        fname = "NVFP4" if fmt == q.QLIN_NVFP4 else "MXFP4"
-        for M in (1, 4):
-            L = 2
-            gu, dn, wsg, wsd = [], [], [], []
-            for l in range(L):
-                b, s_, g = synth.weights(fmt, 2 * I, H, synth.gen(3000 + l, device="cuda"), device="cuda")
-                gu.append(q.qlin_pack_weights(fmt, 2 * I, H, b, s_, g, q.QLIN_PACK_GATE_UP))
-                b, s_, g = synth.weights(fmt, H, I, synth.gen(3100 + l, device="cuda"), device="cuda")
-                dn.append(q.qlin_pack_weights(fmt, H, I, b, s_, g))
-                wsg.append(q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, 2 * I, H)))
-                wsd.append(q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_GEMV, fmt, M, H, I)))
-            x = synth.activations(M, H, synth.gen(3200, device="cuda"), dtype=torch.bfloat16, device="cuda")
-            h = torch.empty(M, I, device="cuda")
-            y = torch.empty(M, H, device="cuda")
-
-            def fn():
-                for l in range(L):
-                    q.qlin_gemv(fmt, gu[l], 2 * I, H, x, y=h, ws=wsg[l], flags=q.QLIN_EPI_SILU_GATE | q.QLIN_FLAG_PDL)
-                    q.qlin_gemv(fmt, dn[l], H, I, h, y=y, ws=wsd[l], flags=q.QLIN_FLAG_PDL)
-            ms = _time_graph_of(fn, args.steps, args.warmup) / L
-            wb = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
-            bytes_ = wb + M * (2 * H + 4 * I + 4 * I + 4 * H)
-            lines.append(dict(workload=f"{fname} MLP shaped like a 27B model: gate_up 5120->2x17408 + SiLU, "
-                              "down 17408->5120, bf16 activations; one qlin_gemv per projection (fp32 h)",
-                              M=M, us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9,
-                              tokens_per_s=M / (ms * 1e-3)))
-            # The same layers as one GEMV chain per step, h kept in bf16 (QLIN_OUT_BF16).
-            hb = [torch.empty(M, I, device="cuda", dtype=torch.bfloat16) for _ in range(L)]
-            ops = []
-            for l in range(L):
-                ops.append(q.gemv_op(gu[l], 2 * I, H, x, hb[l], q.QLIN_EPI_SILU_GATE | q.QLIN_OUT_BF16))
-                ops.append(q.gemv_op(dn[l], H, I, hb[l], y, q.QLIN_EPI_NONE, len(ops) - 1))
-            cws = q.workspace(q.qlin_chain_workspace_bytes(fmt, M, ops))
-            fn2 = lambda: q.qlin_gemv_chain(fmt, q.QLIN_BF16, M, ops, flags=q.QLIN_FLAG_PDL, ws=cws)
-            ms2 = _time_graph_of(fn2, args.steps, args.warmup) / L
-            bytes2 = wb + M * (2 * H + 2 * I + 2 * I + 4 * H)
-            lines.append(dict(workload=f"{fname} MLP shaped like a 27B model, as above; both layers as one "
-                              "GEMV chain, h in bf16", M=M, us_per_layer=ms2 * 1e3,
-                              gbs=bytes2 / (ms2 * 1e-3) / 1e9, tokens_per_s=M / (ms2 * 1e-3)))
-            del gu, dn
-    elif name == "moe":
-        fmt, E, H, I, k = q.QLIN_Q4_0, 32, 2048, 1792, 4
-        L = 8  # 8 layers (1.6 GB): one replay's selected experts (>= 8 x 25 MB) exceed L2
-        canon_gu = [[synth.weights(fmt, 2 * I, H, synth.gen(4000 + 100 * l + e, device="cuda"), device="cuda")
-                     for e in range(E)] for l in range(L)]
-        gu = [q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_GATE_UP) for c in canon_gu]
-        del canon_gu
-        canon_dn = [[synth.weights(fmt, H, I, synth.gen(5000 + 100 * l + e, device="cuda"), device="cuda")
-                     for e in range(E)] for l in range(L)]
-        dn = [q.pack_experts(fmt, E, H, I, c) for c in canon_dn]
-        del canon_dn
-        per_expert = (q.qlin_packed_bytes(fmt, 2 * I, H, 1) - 256) + (q.qlin_packed_bytes(fmt, H, I) - 256)
-        for M in (1, 8):
-            logits = [synth.router_logits(M, E, synth.gen(6000 + l, device="cuda"), device="cuda") for l in range(L)]
-            x = synth.activations(M, H, synth.gen(6100, device="cuda"), device="cuda")
-            ids = torch.empty(M, k, dtype=torch.int32, device="cuda")
-            w = torch.empty(M, k, device="cuda")
-            y = torch.empty(M, H, device="cuda")
-            ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE, fmt, M, H, I, E, k)) for _ in range(L)]
-            distinct = []
-
-            def fn():
-                for l in range(L):
-                    q.qlin_moe_experts(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
-                                       topk_w=w, y=y, ws=ws[l], flags=q.QLIN_FLAG_PDL)
-            ms = _time_graph_of(fn, args.steps, args.warmup) / L
-            for l in range(L):  # actual distinct experts per layer for these seeds
-                q.qlin_moe_experts(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
-                                   topk_w=w, y=y, ws=ws[l])
-                distinct.append(len(set(ids.cpu().flatten().tolist())))
-            nd = sum(distinct) / L
-            bytes_ = nd * per_expert + M * (4 * H + 4 * H + 4 * E)
-            lines.append(dict(workload="Q4_0 MoE expert layer shaped like an 8B-A1B model: hidden 2048, 32 experts "
-                              "gate_up 2048->2x1792, down 1792->2048, top-4; a graph of 8 layers' launches "
-                              "(distinct weights)", M=M, distinct_experts=nd,
-                              us_per_layer=ms * 1e3, gbs=bytes_ / (ms * 1e-3) / 1e9))
-    if name == "gguf_chunk":
+        entries[name] = dict(workload=f"{fname} dense decode layer stack, the Q4_0 stack's shapes ({args.layers} layers "
+                             "of hidden 2560: qkv 2560->6144, o 4096->2560, gate_up 2560->2x9728 + SiLU, "
+                             "down 9728->2560), one GEMV chain per step", M=1, ms_per_step=ms,
+                             packed_weight_bytes=stack.weight_bytes, canonical_weight_bytes=canon,
+                             value=stack.step_bytes / (ms * 1e-3) / 1e9, unit="GB/s", decode_tok_s=1e3 / ms,
+                             roofline=roofline_hbm(f"chain_kernel<{fname}, M=1>", stack.step_bytes, ms * 1e3),
+                             clocks=clk,
+                             l2="inputs larger than L2: %.2f GB of packed weights per step" % (stack.weight_bytes / 1e9))
+    elif name == "gguf_chunk":
         # GGUF prefill chunk: the bf16 copy of dequantized Q4_0 weights (QLIN_PACK_MMA) times bf16 x on
         # the tensor cores (kind::f16), at the NVFP4 chunk workload's shape
         fmt, N, K = q.QLIN_Q4_0, 17408, 5120
@@ -538,55 +743,82 @@ def run_config(name, args):
             b, _, _ = synth.weights(fmt, N, K, synth.gen(7100 + c, device="cuda"), device="cuda")
             packs.append(q.qlin_pack_weights(fmt, N, K, b, None, 1.0, q.QLIN_PACK_MMA))
             del b
-        try:
-            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-                bf16_peak, bf16_src = float(json.load(f)["bf16_tflops"]), "measured bf16 burst (cuBLAS)"
-        except Exception:
-            bf16_peak, bf16_src = 1590.0, "fallback bf16"
+        bpk, bsrc = bf16_peak()
         for M, pairs in ((512, True), (512, False), (64, False)):
             x = synth.activations(M, K, synth.gen(7200 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
             y = torch.empty(M, N, device="cuda")
             ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
             fl = q.QLIN_FLAG_PDL | (q.QLIN_FLAG_CTA_PAIRS if pairs else 0)
             fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=fl) for c in range(2)]
-            ms = _time_graph_of(fn, args.steps, args.warmup) / 2
+            ms, clk = timed(fn, args.steps, args.warmup)
+            us = ms / 2 * 1e3
             flop = 2.0 * M * N * K
+            tf = flop / (us * 1e-6) / 1e12
             bytes_ = N * K * 2 + 2 * M * K + 4 * M * N
             tiling = "256 x 256 tiles on CTA pairs" if pairs else "128 x 256 tiles on single CTAs"
-            lines.append(dict(workload=f"Q4_0 prefill-chunk GEMM M={M} K=5120 N=17408 (bf16 copy of the dequantized "
-                              f"weights x bf16 activations, tcgen05 kind::f16, one launch, {tiling})", M=M,
-                              cta_pairs=pairs, us_per_call=ms * 1e3,
-                              tflops=flop / (ms * 1e-3) / 1e12, bf16_peak_tflops=bf16_peak, bf16_peak_source=bf16_src,
-                              bf16_frac=flop / (ms * 1e-3) / 1e12 / bf16_peak, gbs=bytes_ / (ms * 1e-3) / 1e9))
-    if name == "chunk":
-        fmt, N, K = q.QLIN_NVFP4, 17408, 5120
-        b, s_, g = synth.weights(fmt, N, K, synth.gen(7000, device="cuda"), device="cuda")
-        packs = [q.qlin_pack_weights(fmt, N, K, b, s_, g, q.QLIN_PACK_MMA)]
-        b2, s2, g2 = synth.weights(fmt, N, K, synth.gen(7001, device="cuda"), device="cuda")
-        packs.append(q.qlin_pack_weights(fmt, N, K, b2, s2, g2, q.QLIN_PACK_MMA))  # 2 copies > L2 with y
-        del b, s_, b2, s2
-        try:
-            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-                bf16 = float(json.load(f)["bf16_tflops"])
-            fp4_peak, fp4_src = 4 * bf16, "measured bf16 burst x 4 (nominal fp4/bf16 ratio)"
-        except Exception:
-            fp4_peak, fp4_src = 4 * 1590.0, "fallback bf16 x 4"
-        for M in (512, 64, 16, 8, 4, 2, 1):
-            x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
-            y = torch.empty(M, N, device="cuda")
-            ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
-            fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL) for c in range(2)]
-            ms = _time_graph_of(fn, args.steps, args.warmup) / 2
-            flop = 2.0 * M * N * K
-            bytes_ = (q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA) - 256) + 2 * M * K + 4 * M * N
-            lines.append(dict(workload=f"NVFP4 prefill-chunk GEMM M={M} K=5120 N=17408 (activation quantization "
-                              "+ tcgen05 block-scaled GEMM in one persistent launch)", M=M, us_per_call=ms * 1e3,
-                              tflops=flop / (ms * 1e-3) / 1e12, fp4_peak_tflops=fp4_peak, fp4_peak_source=fp4_src,
-                              fp4_frac=flop / (ms * 1e-3) / 1e12 / fp4_peak, gbs=bytes_ / (ms * 1e-3) / 1e9))
-    for ln in lines:
-        ln.update(metric=METRIC, unit="GB/s", value=ln["gbs"], hbm_frac=ln["gbs"] / peak,
-                  peak=peak, peak_source=peak_src, config=name, impl="qlin", n_gpus=1)
-        print(json.dumps(ln), flush=True)
+            entries[f"gguf_chunk_m{M}{'_pairs' if pairs else ''}"] = dict(
+                workload=f"Q4_0 prefill-chunk GEMM M={M} K=5120 N=17408 (bf16 copy of the dequantized weights x bf16 "
+                         f"activations, tcgen05 kind::f16, one launch, {tiling})", M=M, cta_pairs=pairs,
+                us_per_call=us, value=tf, unit="TFLOP/s", gbs=bytes_ / (us * 1e-6) / 1e9,
+                roofline={"bound": "tensor", "kernel": "chunk_bf16_kernel", "achieved": tf, "peak": bpk,
+                          "peak_source": bsrc, "unit": "TFLOP/s", "frac": tf / bpk, "traffic": None,
+                          "avg_launch_us": us},
+                clocks=clk)
+    for key, e in entries.items():
+        e.update(metric=METRIC, config=name, entry=key, impl="qlin", n_gpus=1)
+        print(json.dumps(e), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+def reference_arm(args, workload, world):
+    """The fp64 oracle as it stands on the host's cores: each step runs, on every host thread, 512
+    random rows of each of the four projection shapes of the stack (row cost depends on K only)
+    against one activation row.  The step time is measured (not extrapolated); value is weight
+    GB/s, the unit of the GPU arm's value."""
+    import oracle
+    fmt = synth.Q4_0
+    model, ncores = cpu_info()
+    data = []
+    for (name, N, K, epi) in STACK:
+        b, s, gs = synth.weights(fmt, 64, K, synth.gen(11 + N))
+        x = synth.activations(1, K, synth.gen(12 + K)).double().numpy()
+        data.append((K, b.numpy(), gs, x, oracle.row_bytes(fmt, K)))
+    rows_per_shape = 512
+
+    def work(tid, step):
+        rng = np.random.default_rng(1000 * step + tid)
+        nb = 0
+        for (K, b, gs, x, rb) in data:
+            for _ in range(rows_per_shape // 64):
+                oracle.gemv(fmt, 64, K, b, x, g=gs, rows=rng.permutation(64))
+                nb += 64 * rb
+        return nb
+
+    with ThreadPoolExecutor(ncores) as ex:
+        def step(i):
+            return sum(ex.map(lambda t: work(t, i), range(ncores)))
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        nbytes = 0
+        for i in range(args.steps):
+            nbytes += step(args.warmup + i)
+        dt = time.perf_counter() - t0
+    gbs = nbytes / dt / 1e9
+    ms = dt * 1e3 / args.steps
+    stack_w = sum((N * K * 9 // 16) for (_, N, K, _) in STACK) * args.layers
+    desc = (f"each step: {rows_per_shape} random weight rows of each of the four stack projection shapes "
+            f"(K = 2560/4096/2560/9728) on each of {ncores} host threads, fp64 oracle ({nbytes // args.steps} "
+            f"weight bytes per step; a full 36-layer token would be {stack_w} bytes)")
+    return {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "decode_tok_s_equivalent": gbs * 1e9 / stack_w,
+            "config": {"workload": workload, "format": "q4_0", "M": 1, "layers": args.layers},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": ncores, "kind": "oracle", "sample": desc,
+                             "cpu_model": model},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
 
 # ----------------------------------------------------------------------------- main
 def main():
@@ -598,6 +830,7 @@ def main():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' entries")
     ap.add_argument("--mode", default="chain", choices=list(DenseStack.MODES),
                     help="how the stack step is launched (default: one persistent GEMV chain)")
     ap.add_argument("--dataflow", default="stated", choices=list(DenseStack.DATAFLOWS),
@@ -606,12 +839,13 @@ def main():
     ap.add_argument("--config", default="stack",
                     choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "chunk", "q4_k_stack",
                              "q6_k_stack", "gguf_chunk"],
-                    help="stack (default): the Q4_0 36-layer decode stack; the others print extra lines")
+                    help="stack (default): the Q4_0 36-layer decode stack line; the others print their "
+                         "entries alone")
     args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
     if args.config != "stack":
         run_config(args.config, args)
         return
-    args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -622,19 +856,8 @@ def main():
                 "down 9728->2560")
 
     if args.impl == "reference":
-        if rank != 0:
-            return
-        gbs, cores, desc = cpu_baseline_stack(fmt, budget_s=max(5.0, 2.0 * args.steps))
-        stack_w = sum((N * K * 9 // 16) for (_, N, K, _) in STACK) * args.layers
-        tok_s = gbs * 1e9 / stack_w
-        line = {"metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": 1e3 / tok_s, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "impl": "reference", "decode_tok_s": tok_s,
-                "config": {"workload": workload, "format": "q4_0", "M": 1, "layers": args.layers},
-                "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc},
-                "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        if rank == 0:
+            print(json.dumps(reference_arm(args, workload, world)), flush=True)
         return
 
     if world > 1:
@@ -678,26 +901,21 @@ def main():
     if stack.chains:
         dom_ms, dom_bytes = time_chain_kernel(stack)
         dom_name = (f"chain_kernel<Q4_0, M=1> ({len(stack.chains[0][0])} GEMVs per launch, "
-                    f"{len(stack.chains)} launches per step)")
+                    f"{len(stack.chains)} launches per step; timed in a graph without PDL)")
+        traffic = recorded_traffic("chain_q4_0_m1") if (args.layers == LAYERS and args.mode == "chain") else None
     else:
         dom_ms, dom_bytes = time_dominant_kernel(stack)
         dom_name = "gemv_kernel<Q4_0, M=1, SiLU-gate> (gate_up 2560->19456)"
+        traffic = None
     e2e_ms, h2d, d2h = e2e_stack(stack, args.steps, args.warmup, pdl=not args.no_pdl)
     e2e_ms = max_over_ranks(e2e_ms, world)
     del graph
 
+    line = None
     if rank == 0:
         peak, peak_src = peaks()
         gbs = whole_job_gbs(stack.step_bytes, world, ms_max)
-        dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
-        traffic = None  # the committed capture's estimate holds for the default 36-layer launch only
-        try:
-            if args.layers == LAYERS:
-                with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-                    key = f"{args.mode}_q4_0_m1_bytes_per_launch" if stack.chains else "gate_up_q4_0_m1_bytes_per_launch"
-                    traffic = json.load(f).get(key)
-        except Exception:
-            pass
+        rf = roofline_hbm(dom_name, dom_bytes, dom_ms * 1e3, traffic)
         line = {
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
@@ -712,21 +930,32 @@ def main():
                        "l2": "inputs larger than L2: %.2f GB of packed weights streamed per step (L2 126 MB)"
                              % (stack.weight_bytes / 1e9),
                        "parallelism": f"replicas{world}"},
-            "roofline": {"bound": "hbm", "kernel": dom_name,
-                         "achieved": dom_gbs, "peak": peak, "peak_source": f"{peak_src} hbm_gbs (copy)",
-                         "unit": "GB/s", "frac": dom_gbs / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": dom_bytes, "avg_launch_us": dom_ms * 1e3},
+            "roofline": rf,
             "e2e": {"value": whole_job_gbs(stack.step_bytes, world, e2e_ms), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             f"{other_df}_dataflow": {"value": whole_job_gbs(other.step_bytes, world, other_ms), "unit": "GB/s",
                                      "ms_per_step": other_ms, "mode": args.mode,
-                                     "launches_per_step": other.launches_per_step},
+                                     "launches_per_step": other.launches_per_step,
+                                     "decode_tok_s": 1e3 / other_ms},
             "gpu_launches": stack.launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline and world == 1:
-            cg, cores, desc = cpu_baseline_stack(fmt)
-            line["cpu_baseline"] = {"value": cg, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+            line["cpu_baseline"] = cpu_baseline(fmt, [(N, K) for (_, N, K, _) in STACK], 1, budget_s=4.0,
+                                                what="stack")
+    del stack, other
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_configs:
+        # The other workloads, each with its own value, roofline, clocks and CPU baseline.
+        cfgs = {}
+        for fn in (cfg_q8_small, cfg_mlp, cfg_moe, cfg_chunk):
+            try:
+                cfgs.update(fn(args, cpu=not args.no_cpu_baseline))
+            except Exception as ex:  # keep the headline line; record what failed
+                cfgs[fn.__name__] = {"error": repr(ex)}
+            torch.cuda.empty_cache()
+        line["configs"] = cfgs
+    if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -189,9 +189,10 @@ __device__ __forceinline__ void chain_write_tile(const ChainOp& o, int M, int t,
     }
 }
 
-// Count n written tiles of op j for the ops waiting for it (one release per batch of tiles).
+// Count n written tiles of op j for the ops waiting for it (one release per batch of tiles).  The
+// warp barrier orders every lane's tile stores before lane 0's release, which is cumulative over
+// them.
 __device__ __forceinline__ void chain_signal(const ChainArgs& a, int j, uint32_t n, int lane) {
-    __threadfence();
     __syncwarp();
     if (lane == 0) red_release_add(reinterpret_cast<unsigned int*>(a.ws + kChainDoneOff) + j, n);
 }
@@ -279,16 +280,45 @@ __device__ __noinline__ bool chain_flush(const ChainArgs& a, int j, int t, int l
     return true;
 }
 
+// Which ops this CTA has seen complete (set by the warp that saw it; zeroed at kernel start), and
+// whether one of its warps is polling the global counts right now.
+__shared__ unsigned int s_chain_seen[kMaxChainOps];
+__shared__ unsigned int s_chain_poll;
+
 // Bounded wait until every tile of op j is written (~2 s, or the workspace's wait budget); false
-// on timeout.
+// on timeout.  One warp of the CTA at a time reads the global count (with a pause between reads);
+// the others wait for the shared-memory flag the reading warp sets when the count is complete.
+// Thousands of warps polling one L2 line slow every other load of the grid.
 __device__ __forceinline__ bool chain_wait_op(const ChainArgs& a, int j) {
     const unsigned int* done = reinterpret_cast<const unsigned int*>(a.ws + kChainDoneOff) + j;
     const uint32_t target = (uint32_t)a.op[j].T;
-    if (__all_sync(0xffffffffu, ld_acquire_u32(done) >= target)) return true;
+    const int lane = threadIdx.x & 31;
+    uint32_t seen = 0;
+    if (lane == 0) {
+        asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(seen) : "r"(smem_u32(&s_chain_seen[j])) : "memory");
+        if (!seen && ld_acquire_u32(done) >= target) seen = 1;
+    }
+    if (__shfl_sync(0xffffffffu, seen, 0)) {
+        __syncwarp();
+        return true;
+    }
     const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(a.ws);
-    for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
-        if (__all_sync(0xffffffffu, ld_acquire_u32(done) >= target)) return true;
+    for (;;) {
+        __nanosleep(256);
+        if (lane == 0) {
+            asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(seen) : "r"(smem_u32(&s_chain_seen[j])) : "memory");
+            if (!seen && atomicExch(&s_chain_poll, 1u) == 0u) {
+                if (ld_acquire_u32(done) >= target) {
+                    asm volatile("st.release.cta.shared.u32 [%0], 1;" ::"r"(smem_u32(&s_chain_seen[j])) : "memory");
+                    seen = 1;
+                }
+                atomicExch(&s_chain_poll, 0u);
+            }
+        }
+        if (__shfl_sync(0xffffffffu, seen, 0)) {
+            __syncwarp();  // the other lanes read after lane 0's acquire
+            return true;
+        }
         if (globaltimer_ns() - t0 > budget) return false;
     }
 }
@@ -318,6 +348,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32, RingCfg<FMT>::kCtasPerSm)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemvWarps * C::D * C::UB) + warp * C::D;
 
     griddep_launch_dependents();
+    for (int i = threadIdx.x; i < kMaxChainOps; i += blockDim.x) s_chain_seen[i] = 0u;
+    if (threadIdx.x == 0) s_chain_poll = 0u;
+    __syncthreads();
     ChainCursor c;
     chain_seek(a, gw, c, 0);
     ChainCursor p = c;  // producer cursor, C::D units ahead once primed

@@ -706,6 +706,30 @@ def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
     if sw:
         out["nvfp4_chunk_m_sweep"] = {"workload": "the same GEMM at small M (the GEMV regime on the chunk path)",
                                       "by_M": sw}
+    # The bf16-operand path for the same NVFP4 weights (QLIN_PACK_MMA_BF16: exact e2m1 * e4m3 products
+    # in bf16, x not quantized), tcgen05 kind::f16 on CTA pairs.
+    del packs
+    bpacks = []
+    for c in range(2):
+        b, s_, g = synth.weights(fmt, N, K, synth.gen(7000 + c, device="cuda"), device="cuda")
+        bpacks.append(q.qlin_pack_weights(fmt, N, K, b, s_, g, q.QLIN_PACK_MMA_BF16))
+        del b, s_
+    bpk, bsrc = bf16_peak()
+    bp = {}
+    for M in (512, 64):
+        x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(M, N, device="cuda")
+        ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+        fl = q.QLIN_FLAG_PDL | q.QLIN_FLAG_BF16_COPY | q.QLIN_FLAG_CTA_PAIRS
+        fn = lambda: [q.qlin_gemm_chunk(fmt, bpacks[c], N, K, x, y=y, ws=ws, flags=fl) for c in range(2)]
+        ms = _time_graph_of(fn, args.steps, args.warmup) / 2
+        us = ms * 1e3
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        bp[str(M)] = {"us_per_call": us, "tflops": tf, "bf16_frac": tf / bpk, "bf16_peak": bpk,
+                      "gbs": (N * K * 2 + 2 * M * K + 4 * M * N) / (us * 1e-6) / 1e9}
+    out["nvfp4_chunk_bf16_path"] = {"workload": "the same NVFP4 weights through the bf16-operand path "
+                                                "(QLIN_PACK_MMA_BF16 + QLIN_FLAG_BF16_COPY, CTA pairs): bf16 x not "
+                                                "quantized, 2 B/weight", "by_M": bp, "bf16_peak_source": bsrc}
     return out
 
 

@@ -19,7 +19,8 @@ import torch
 QLIN_Q8_0, QLIN_Q4_0, QLIN_NVFP4, QLIN_MXFP4, QLIN_Q4_K, QLIN_Q6_K = 1, 2, 3, 4, 5, 6
 QLIN_F32, QLIN_BF16 = 0, 1
 QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_OUT_BF16, QLIN_FLAG_PDL, QLIN_FLAG_CTA_PAIRS = 0, 1, 0x10, 0x100, 0x200
-QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA = 0, 1, 2
+QLIN_FLAG_BF16_COPY = 0x400
+QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA, QLIN_PACK_MMA_BF16 = 0, 1, 2, 4
 QLIN_OP_GEMV, QLIN_OP_MOE, QLIN_OP_CHUNK = 1, 2, 3
 STATUS = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED",
           3: "QLIN_ERR_ALIGNMENT", 4: "QLIN_ERR_WORKSPACE", 5: "QLIN_ERR_CUDA",

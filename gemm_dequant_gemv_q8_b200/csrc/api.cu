@@ -17,7 +17,7 @@ extern "C" cudaError_t qlin_launch_moe(int fmt, const void* gu, const void* dn, 
 extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K);
 extern "C" int64_t qlin_bf16_cache_cols(int64_t K);
 extern "C" int64_t qlin_bf16_cache_bytes(int64_t N, int64_t K);
-extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
+extern "C" cudaError_t qlin_launch_chunk_bf16(const void* packed, int64_t N, int64_t K, const void* x, int M,
                                               int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
                                               cudaStream_t s);
 extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
@@ -101,6 +101,8 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
 
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags) {
     if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
+    if (pack_flags == QLIN_PACK_MMA_BF16)  // the bf16 copy, every format
+        return (size_t)qlin::kHdrBytes + (size_t)qlin_bf16_cache_bytes(N, K);
     if (pack_flags == QLIN_PACK_MMA) {
         if (fmt != QLIN_NVFP4)  // the bf16 copy of the dequantized weights, rows of K rounded up to 64
             return (size_t)qlin::kHdrBytes + (size_t)qlin_bf16_cache_bytes(N, K);
@@ -117,7 +119,8 @@ qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const v
                                 void* packed, size_t packed_bytes, qlin_stream_t stream) {
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
-    if (pack_flags != QLIN_PACK_MMA && (pack_flags & ~QLIN_PACK_GATE_UP)) return QLIN_ERR_INVALID_ARG;
+    if (pack_flags != QLIN_PACK_MMA && pack_flags != QLIN_PACK_MMA_BF16 && (pack_flags & ~QLIN_PACK_GATE_UP))
+        return QLIN_ERR_INVALID_ARG;
     if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
     if (!blocks || !packed) return QLIN_ERR_INVALID_ARG;
     if ((fmt == QLIN_NVFP4 || fmt == QLIN_MXFP4) && !scales) return QLIN_ERR_INVALID_ARG;
@@ -202,16 +205,17 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
                               size_t ws_bytes, qlin_stream_t stream) {
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, N, K) || M < 1 || M > (1 << 20)) return QLIN_ERR_INVALID_ARG;
-    if (flags & ~(QLIN_FLAG_PDL | QLIN_FLAG_CTA_PAIRS)) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~(QLIN_FLAG_PDL | QLIN_FLAG_CTA_PAIRS | QLIN_FLAG_BF16_COPY)) return QLIN_ERR_INVALID_ARG;
     if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
     if (ldx < K || ldy < N) return QLIN_ERR_INVALID_ARG;
     if (!aligned(packed, 256) || !aligned(x, 2) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
-    if (fmt != QLIN_NVFP4) {  // bf16 path: x is read by tensor-map loads (16-byte aligned rows)
+    if (fmt != QLIN_NVFP4 || (flags & QLIN_FLAG_BF16_COPY)) {
+        // bf16 path: x is read by tensor-map loads (16-byte aligned rows)
         if (!aligned(x, 16) || ldx % 8) return QLIN_ERR_ALIGNMENT;
         if (!ws || ws_bytes < 256) return QLIN_ERR_WORKSPACE;
         if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
-        return cuda_status(qlin_launch_chunk_bf16((const uint8_t*)packed + qlin::kHdrBytes, N, K, x, M, ldx, y, ldy,
-                                                  ws, flags, (cudaStream_t)stream));
+        return cuda_status(qlin_launch_chunk_bf16(packed, N, K, x, M, ldx, y, ldy, ws, flags & ~QLIN_FLAG_BF16_COPY,
+                                                  (cudaStream_t)stream));
     }
     if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, N, K)) return QLIN_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;

@@ -1,7 +1,9 @@
 // chunk_bf16.cu -- prefill-chunk GEMM for the GGUF / MXFP4 weight formats on the 5th-generation
-// tensor cores (sm_100a): y[m][n] = sum_k x[m][k] * Wb[n][k], x bf16 as given, Wb the bf16 copy of
-// the dequantized weights that qlin_pack_weights(QLIN_PACK_MMA) builds once (each weight the fp32
-// dequantized value rounded to nearest-even bf16), fp32 accumulation in tensor memory.
+// tensor cores (sm_100a): y[m][n] = g * sum_k x[m][k] * Wb[n][k], x bf16 as given, Wb the bf16 copy
+// of the dequantized weights that qlin_pack_weights(QLIN_PACK_MMA / QLIN_PACK_MMA_BF16) builds once
+// (each weight the fp32 dequantized value rounded to nearest-even bf16; for NVFP4 the exact product
+// of code and block scale), fp32 accumulation in tensor memory, g the per-tensor scale of the
+// packed header (1 for every format but NVFP4) applied once per output.
 //
 // The pages' counterpart: imp keeps "full-precision prefill via source dequant" for GGUF models
 // (README "Why this exists") and runs its prefill GEMMs on the tensor cores; here the dequantized
@@ -52,6 +54,7 @@ struct Cfg {
 static_assert(Cfg<1>::kSmem <= 232448 && Cfg<2>::kSmem <= 232448, "shared memory budget");
 
 struct Args {
+    const float* gscale;  // the per-tensor scale in the packed header
     float* y;
     int64_t ldy;
     int M;
@@ -322,6 +325,7 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         uint8_t* tb = epi + (warp - kFirstEpi) * kEpiBuf;
+        const float gs = *a.gscale;  // written by the packing kernel, before this launch
         int tcount = 0;
         for (int tile = tile0; tile < ntiles; tile += tstep, ++tcount) {
             const int ab = tcount & 1;
@@ -356,8 +360,8 @@ __global__ void __launch_bounds__(cb::kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         *reinterpret_cast<float4*>(tb + lane * 64 + ((j ^ (lane & 3)) << 4)) =
-                            make_float4(v[16 * h + 4 * j], v[16 * h + 4 * j + 1], v[16 * h + 4 * j + 2],
-                                        v[16 * h + 4 * j + 3]);
+                            make_float4(v[16 * h + 4 * j] * gs, v[16 * h + 4 * j + 1] * gs,
+                                        v[16 * h + 4 * j + 2] * gs, v[16 * h + 4 * j + 3] * gs);
                     __syncwarp();
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -518,15 +522,18 @@ static cudaError_t launch_bf16_cg(const cb::Args& a, const CUtensorMap& xmap, co
     return cudaLaunchKernelEx(&cfg, chunk_bf16_kernel<CG>, a, xmap, wmap);
 }
 
-// wb: the blocked bf16 weights (after the 256-byte header of the packed buffer): for row block nb
-// and k-block kb, 256 rows x 64 values at element ((nb * Kc / 64 + kb) * 256 + row) * 64;
+// packed: the 256-byte header (its per-tensor scale multiplies every output), then the blocked bf16
+// weights: for row block nb and k-block kb, 256 rows x 64 values at element
+// ((nb * Kc / 64 + kb) * 256 + row) * 64;
 // x: bf16 [M][K] with row pitch ldx (16-byte aligned base, ldx % 8 == 0, checked by the caller).
 // QLIN_FLAG_CTA_PAIRS with M > 128: 256 x 256 tiles on pairs of CTAs.
-extern "C" cudaError_t qlin_launch_chunk_bf16(const void* wb, int64_t N, int64_t K, const void* x, int M,
+extern "C" cudaError_t qlin_launch_chunk_bf16(const void* packed, int64_t N, int64_t K, const void* x, int M,
                                               int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
                                               cudaStream_t s) {
     const int cg = (flags & QLIN_FLAG_CTA_PAIRS) && M > cb::kRows ? 2 : 1;
+    const void* wb = reinterpret_cast<const uint8_t*>(packed) + kHdrBytes;
     cb::Args a;
+    a.gscale = &reinterpret_cast<const PackedHeader*>(packed)->global_scale;
     a.y = y;
     a.ldy = ldy;
     a.M = M;

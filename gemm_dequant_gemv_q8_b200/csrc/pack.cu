@@ -251,9 +251,11 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t* __restrict__
     }
 }
 
-// QLIN_PACK_MMA for the formats other than NVFP4: the dequantized weights as bf16 rows of Kc
-// values (K rounded up to 64, the tail zero), each the fp32 value qlin_dequant_debug gives rounded
-// to nearest-even bf16 -- the operand of the bf16 prefill-chunk GEMM.  Thread = (row, 32 values).
+// QLIN_PACK_MMA for the formats other than NVFP4, and QLIN_PACK_MMA_BF16: the dequantized weights
+// as bf16 rows of Kc values (K rounded up to 64, the tail zero), each the fp32 value
+// qlin_dequant_debug gives rounded to nearest-even bf16 -- the operand of the bf16 prefill-chunk
+// GEMM.  NVFP4: e2m1 * e4m3 without the per-tensor scale (exact in bf16; the GEMM applies the scale
+// from the header).  Thread = (row, 32 values).
 template <int FMT>
 __global__ void __launch_bounds__(256) pack_bf16_kernel(const uint8_t* __restrict__ blocks,
                                                         const uint8_t* __restrict__ scales, int64_t N, int64_t K,
@@ -274,6 +276,13 @@ __global__ void __launch_bounds__(256) pack_bf16_kernel(const uint8_t* __restric
                 const int q = FMT == QLIN_Q8_0 ? (int)(int8_t)blk[2 + j]
                                                : (j < 16 ? (blk[2 + j] & 0xf) : (blk[2 + j - 16] >> 4)) - 8;
                 w[j] = d * (float)q;  // exact
+            }
+        } else if (FMT == QLIN_NVFP4) {  // K % 16 == 0: the last 32-value part may be half valid
+            const uint8_t* row = blocks + n * (K / 2) + k0 / 2;
+            for (int j = 0; j < 32 && k0 + j < K; ++j) {
+                const uint32_t h2 = e2m1x2_to_f16x2(row[j / 2]);
+                const float v = __half2float(__ushort_as_half((unsigned short)((j & 1) ? (h2 >> 16) : (h2 & 0xffff))));
+                w[j] = __fmul_rn(v, e4m3_to_f32(scales[n * (K / 16) + (k0 + j) / 16]));  // exact
             }
         } else if (FMT == QLIN_MXFP4) {
             const uint8_t* row = blocks + n * (K / 2) + k0 / 2;
@@ -334,10 +343,10 @@ extern "C" cudaError_t qlin_launch_pack_mma(const void* codes, const void* scale
 extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void* scales, int64_t N,
                                         int64_t K, int pack_flags, float gs, void* packed,
                                         cudaStream_t s) {
-    if (pack_flags == QLIN_PACK_MMA) {
+    if (pack_flags == QLIN_PACK_MMA || pack_flags == QLIN_PACK_MMA_BF16) {
         write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags, gs,
                                              (int32_t)((N + 255) / 256), (int32_t)((K + 255) / 256));
-        if (fmt == QLIN_NVFP4) return qlin_launch_pack_mma(blocks, scales, N, K, gs, packed, s);
+        if (fmt == QLIN_NVFP4 && pack_flags == QLIN_PACK_MMA) return qlin_launch_pack_mma(blocks, scales, N, K, gs, packed, s);
         const int64_t Kc = qlin_bf16_cache_cols(K);
         const int64_t threads = (N + 255) / 256 * 256 * (Kc / 32);
         const dim3 grid((unsigned)((threads + 255) / 256));
@@ -348,7 +357,8 @@ extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void*
         else if (fmt == QLIN_Q4_0) pack_bf16_kernel<QLIN_Q4_0><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
         else if (fmt == QLIN_MXFP4) pack_bf16_kernel<QLIN_MXFP4><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
         else if (fmt == QLIN_Q4_K) pack_bf16_kernel<QLIN_Q4_K><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
-        else pack_bf16_kernel<QLIN_Q6_K><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        else if (fmt == QLIN_Q6_K) pack_bf16_kernel<QLIN_Q6_K><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
+        else pack_bf16_kernel<QLIN_NVFP4><<<grid, 256, 0, s>>>(bl, sc, N, K, Kc, out);
         return cudaGetLastError();
     }
     Geometry geo = geometry(fmt, N, K, pack_flags);

@@ -64,10 +64,14 @@ enum {
                                still running, and waits for it before touching x or y.  Only
                                valid when the packed weights were written before the previous
                                kernel on the stream started.                                      */
-    QLIN_FLAG_CTA_PAIRS = 0x200  /* qlin_gemm_chunk only, M > 128: tile with pairs of CTAs
+    QLIN_FLAG_CTA_PAIRS = 0x200, /* qlin_gemm_chunk only, M > 128: tile with pairs of CTAs
                                (tcgen05 cta_group::2, 256 activation rows per tile; each SM streams
                                half of every weight tile).  Same results; the default single-CTA
                                tiling is faster on the sizes measured so far. */
+    QLIN_FLAG_BF16_COPY = 0x400  /* qlin_gemm_chunk only: `packed` is a QLIN_PACK_MMA_BF16 buffer, so
+                               the bf16-operand path runs (for NVFP4 weights too: bf16 x, no
+                               activation quantization).  Optional for the formats other than
+                               NVFP4, whose chunk path is always the bf16 one. */
 };
 
 /* qlin_pack_weights flags */
@@ -75,7 +79,7 @@ enum {
     QLIN_PACK_DEFAULT = 0,
     QLIN_PACK_GATE_UP = 1, /* the N rows are [gate ; up] halves (N even): each packed tile pairs
                              16 gate rows with their 16 up rows so the SiLU-gate epilogue fuses */
-    QLIN_PACK_MMA = 2      /* the weight operand of qlin_gemm_chunk.  NVFP4: the tensor-core layout
+    QLIN_PACK_MMA = 2,     /* the weight operand of qlin_gemm_chunk.  NVFP4: the tensor-core layout
                              (tiles of 256 rows x 256 values, 128-byte-swizzled K-major codes, scale
                              factors in 512-byte atoms), 0.5625 B/weight plus padding to 256 x 256.
                              Q8_0 / Q4_0 / MXFP4 / Q4_K / Q6_K: a bf16 copy of the dequantized
@@ -86,6 +90,12 @@ enum {
                              to nearest-even bf16, columns >= K and rows >= N (to a multiple of
                              256) zero (2 B/weight: the full-precision prefill copy; imp README
                              "Why this exists": prefill via source dequant) */
+    QLIN_PACK_MMA_BF16 = 4  /* the bf16 copy, for every format (the same buffer as QLIN_PACK_MMA for the
+                             formats other than NVFP4).  NVFP4: each element is the product of its
+                             E2M1 code and its E4M3 block scale (at most 2 + 4 significant bits,
+                             2^-10 <= |v| <= 2688: exact in bf16); the per-tensor scale stays in the
+                             header and qlin_gemm_chunk applies it to each output once.  Layout and
+                             size as the QLIN_PACK_MMA bf16 copy. */
 };
 
 /* qlin_workspace_bytes ops */
@@ -288,6 +298,13 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
  * tiles on pairs of CTAs (cta_group::2), each staging its 128 activation rows and 128 weight rows;
  * ws: qlin_workspace_bytes(QLIN_OP_CHUNK, fmt, M, N, K, 0, 0) bytes (256: the status word).
  * Bounded device waits: a timeout sets the workspace status word (qlin_ws_status). */
+/* bf16-operand path for NVFP4 weights (QLIN_FLAG_BF16_COPY with a QLIN_PACK_MMA_BF16 buffer):
+ * y[m][n] = fl(g * sum_k x[m][k] * (e2m1 * e4m3)[n][k]): the bf16 x as given against the exact block
+ * products, fp32 accumulation in tensor memory, the per-tensor scale g applied once per output.  The
+ * activations are not quantized, so this path meets the bf16-operand chunk bound |y - y_ref| <=
+ * 1e-2 * sum|w x| against the unquantized product, which the FP4-activation path above does not
+ * guarantee (its per-output error against y_ref is that of NVFP4-quantized activations, up to about
+ * 1e-2 * sum|w x| on random data).  It streams 2 bytes per weight instead of 0.5625. */
 qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,
                               int M, int64_t ldx, float* y, int64_t ldy, int flags, void* ws,
                               size_t ws_bytes, qlin_stream_t stream);

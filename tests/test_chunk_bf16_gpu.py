@@ -146,3 +146,46 @@ def test_chunk_bf16_back_to_back_pdl():
     assert q.qlin_ws_status(ws) == 0
     for x, y in runs:
         check(y, x, w32)
+
+
+# ------------------------------------------------------------------ NVFP4 weights on the bf16 path
+def make_nvfp4_bf16(N, K, seed):
+    codes, scales, g = synth.weights(q.QLIN_NVFP4, N, K, synth.gen(seed))
+    packed = q.qlin_pack_weights(q.QLIN_NVFP4, N, K, codes.cuda(), scales.cuda(), g, q.QLIN_PACK_MMA_BF16)
+    return codes.numpy(), scales.numpy(), g, packed
+
+
+def test_nvfp4_bf16_copy_holds_exact_block_products():
+    """QLIN_PACK_MMA_BF16 for NVFP4: every element is e2m1 * e4m3 (the oracle's dequant with a
+    per-tensor scale of 1, exact in bf16), the per-tensor scale kept in the header."""
+    N, K = 300, 272  # ragged rows and a K that ends in the middle of a 64-value stage
+    codes, scales, g, packed = make_nvfp4_bf16(N, K, 77)
+    assert packed.numel() == q.qlin_packed_bytes(q.QLIN_NVFP4, N, K, q.QLIN_PACK_MMA_BF16)
+    wb, kc = cache(packed, N, K)
+    prod = oracle.dequant(q.QLIN_NVFP4, N, K, codes, scales, 1.0)
+    ref = torch.from_numpy(prod).to(torch.bfloat16)
+    assert np.array_equal(ref.double().numpy(), prod)  # the products are bf16 numbers
+    assert torch.equal(wb[:N, :K].cpu().view(torch.int16), ref.view(torch.int16))
+    assert (wb[:, K:].cpu().float() == 0).all() and (wb[N:].cpu().float() == 0).all()
+    hdr_g = packed[:256].cpu().view(torch.float32)[7].item()  # PackedHeader.global_scale (byte 28)
+    assert hdr_g == g
+
+
+@pytest.mark.parametrize("flags", [q.QLIN_FLAG_BF16_COPY, q.QLIN_FLAG_BF16_COPY | q.QLIN_FLAG_CTA_PAIRS])
+@pytest.mark.parametrize("M,N,K", [(64, 300, 512), (200, 520, 2560), (513, 1000, 1024), (37, 70, 272)])
+def test_nvfp4_bf16_path_meets_the_bf16_operand_bound(M, N, K, flags):
+    """y = g * sum x * (e2m1 * e4m3): exact products in the tensor core, fp32 accumulation, one
+    rounding for g.  Against the fp64 product of the bf16 x as given and the exact NVFP4 weights
+    (no activation quantization): |y - y_ref| <= (2K + 1) 2^-24 sum|w x| (the fp32 summation bound of
+    the other bf16-path tests plus the scale's rounding), which implies the bf16-operand chunk bound
+    of 1e-2 sum|w x| by a wide margin."""
+    codes, scales, g, packed = make_nvfp4_bf16(N, K, 3000 + M)
+    x = synth.activations(M, K, synth.gen(3100 + M), dtype=torch.bfloat16)
+    y = q.qlin_gemm_chunk(q.QLIN_NVFP4, packed, N, K, x.cuda(), flags=flags)
+    torch.cuda.synchronize()
+    rows = np.unique(np.linspace(0, N - 1, min(N, 64)).astype(np.int64))
+    yref, A = oracle.gemv(q.QLIN_NVFP4, N, K, codes, x.double().numpy(), scales=scales, g=g, rows=rows)
+    err = np.abs(y[:, rows].double().cpu().numpy() - yref)
+    bound = (2 * K + 1) * 2.0 ** -24 * A + 1e-30
+    assert (err <= bound).all(), float(np.max(err / bound))
+    assert (err <= 1e-2 * A + 1e-30).all()

@@ -793,6 +793,48 @@ def run_config(name, args):
         print(json.dumps(e), flush=True)
 
 
+# ----------------------------------------------------------------------------- small cases for ncu
+def small_case(name, reps=3):
+    """A few launches of one kernel on one layer, for ncu captures that end in seconds (the
+    profiles under profiles/ name these commands): moe1 / moe8 = one Q4_0 MoE layer of the 8B-A1B
+    shape at M = 1 / 8; mlp1 / mlp4 = one NVFP4 27B-shaped MLP as a two-op GEMV chain (h in bf16)
+    at M = 1 / 4."""
+    import gemm_dequant_gemv_q8_b200 as q
+    torch.cuda.set_device(0)
+    if name.startswith("moe"):
+        M = int(name[3:])
+        fmt, E, H, I, k = q.QLIN_Q4_0, 32, 2048, 1792, 4
+        c = [synth.weights(fmt, 2 * I, H, synth.gen(4000 + e, device="cuda"), device="cuda") for e in range(E)]
+        gu = q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_GATE_UP)
+        c = [synth.weights(fmt, H, I, synth.gen(5000 + e, device="cuda"), device="cuda") for e in range(E)]
+        dn = q.pack_experts(fmt, E, H, I, c)
+        del c
+        logits = synth.router_logits(M, E, synth.gen(6000, device="cuda"), device="cuda")
+        x = synth.activations(M, H, synth.gen(6100, device="cuda"), device="cuda")
+        ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE, fmt, M, H, I, E, k))
+        for _ in range(reps):
+            q.qlin_moe_experts(fmt, gu, dn, E, H, I, k, x, router_logits=logits, ws=ws)
+    elif name.startswith("mlp"):
+        M = int(name[3:])
+        fmt, H, I = q.QLIN_NVFP4, 5120, 17408
+        b, s_, g = synth.weights(fmt, 2 * I, H, synth.gen(3000, device="cuda"), device="cuda")
+        gu = q.qlin_pack_weights(fmt, 2 * I, H, b, s_, g, q.QLIN_PACK_GATE_UP)
+        b, s_, g = synth.weights(fmt, H, I, synth.gen(3100, device="cuda"), device="cuda")
+        dn = q.qlin_pack_weights(fmt, H, I, b, s_, g)
+        del b, s_
+        x = synth.activations(M, H, synth.gen(3200, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        hb = torch.empty(M, I, device="cuda", dtype=torch.bfloat16)
+        y = torch.empty(M, H, device="cuda")
+        ops = [q.gemv_op(gu, 2 * I, H, x, hb, q.QLIN_EPI_SILU_GATE | q.QLIN_OUT_BF16), q.gemv_op(dn, H, I, hb, y, 0, 0)]
+        ws = q.workspace(q.qlin_chain_workspace_bytes(fmt, M, ops))
+        for _ in range(reps):
+            q.qlin_gemv_chain(fmt, q.QLIN_BF16, M, ops, ws=ws)
+    else:
+        raise ValueError(name)
+    torch.cuda.synchronize()
+    print(json.dumps({"small_case": name, "launches": reps}), flush=True)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def reference_arm(args, workload, world):
     """The fp64 oracle as it stands on the host's cores: each step runs, on every host thread, 512
@@ -865,8 +907,13 @@ def main():
                              "q6_k_stack", "gguf_chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack line; the others print their "
                          "entries alone")
+    ap.add_argument("--small-case", choices=["moe1", "moe8", "mlp1", "mlp4"],
+                    help="three launches of one layer's kernel (for ncu captures); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.small_case:
+        small_case(args.small_case)
+        return
     if args.config != "stack":
         run_config(args.config, args)
         return

@@ -63,6 +63,7 @@ def _l():
             lib.qo_round_e2m1_satfinite.restype = ctypes.c_uint8
             lib.qo_round_e2m1_satfinite.argtypes = [F]
             lib.qo_act_quant.restype = I; lib.qo_act_quant.argtypes = [I, I64, P, P, P, P]
+            lib.qo_act_quant_mx.restype = I; lib.qo_act_quant_mx.argtypes = [I, I64, P, P, P]
             _lib = lib
     return _lib
 
@@ -215,3 +216,24 @@ def gemm_same_quant(w_codes, w_scales, w_g, a_codes, a_scales, a_g, N, K):
     Returns (y, A) as gemv does."""
     Aq = dequant(NVFP4, a_codes.shape[0], K, a_codes, a_scales, a_g)
     return gemv(NVFP4, N, K, w_codes, Aq, scales=w_scales, g=w_g)
+
+
+def act_quant_mx(X):
+    """MXFP4 activation quantizer of the MXFP4 chunk path (OCP MX rule: one UE8M0 scale
+    2^(floor(log2 amax) - 2) per 32 values, E2M1 codes rounded to nearest even, saturating).
+    X: (M, K) fp32 values that are exact bf16 numbers.  Returns (codes [M][K/2], scales [M][K/32])."""
+    X = np.ascontiguousarray(np.asarray(X, np.float32))
+    M, K = X.shape
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    rc = _l().qo_act_quant_mx(M, K, _p(X), _p(codes), _p(scales))
+    assert rc == 0, "bad arguments"
+    return codes, scales
+
+
+def gemm_same_quant_mx(w_codes, w_scales, a_codes, a_scales, N, K):
+    """y_q[m][n] = sum_k A_q[m][k] * W[n][k] with both operands the exact MXFP4 values, fp64.
+
+    Returns (y, A) as gemv does."""
+    Aq = dequant(MXFP4, a_codes.shape[0], K, a_codes, a_scales)
+    return gemv(MXFP4, N, K, w_codes, Aq, scales=w_scales)

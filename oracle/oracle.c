@@ -428,3 +428,53 @@ int qo_act_quant(int M, int64_t K, const float* X, uint8_t* codes, uint8_t* scal
         }
     return 0;
 }
+
+/* ---------------------------------------------------------------- MXFP4 activation quantizer */
+
+/* MXFP4 quantization of a bf16 activation matrix X (M x K, fp32 values that are exact bf16
+ * numbers), the A operand of the MXFP4 chunk GEMM.  The pages give MXFP4 as "E2M1 + UE8M0 block
+ * scales, 4.25 bits per weight" (imp release notes v0.6) and nothing on quantizing activations;
+ * the rule below is the OCP MX v1.0 conversion, the plainest reading for an MX operand.  For each
+ * block of 32 consecutive k of a row, with amax_b its largest magnitude:
+ *   e     = floor(log2(amax_b)) - 2        (2: the exponent of E2M1's largest value, 6 = 1.5 * 2^2)
+ *   byte  = e + 127, clamped to [0, 254]  (the UE8M0 scale X = 2^(byte - 127))
+ *   code  = E2M1_rne_satfinite( x / X )    (x / X is exact: a power-of-two scaling)
+ * A block whose amax is 0 (or below 2^-125) gets byte 0.  A block holding an Inf or NaN gets the
+ * UE8M0 NaN byte 0xFF and all-zero codes (finite activations are the case the chunk path serves).
+ * Output: codes [M][K/2] (element 2i in the low nibble), scales [M][K/32]. */
+int qo_act_quant_mx(int M, int64_t K, const float* X, uint8_t* codes, uint8_t* scales) {
+    if (K % 32) return -1;
+    for (int m = 0; m < M; ++m)
+        for (int64_t b = 0; b < K / 32; ++b) {
+            const float* xb = X + (int64_t)m * K + b * 32;
+            double amax = 0.0;
+            int special = 0;
+            for (int j = 0; j < 32; ++j) {
+                if (!isfinite(xb[j])) special = 1;
+                double a = fabs((double)xb[j]);
+                if (a > amax) amax = a;
+            }
+            uint8_t byte = 0;
+            if (special) {
+                byte = 0xFF;
+            } else if (amax > 0.0) {
+                int E;
+                frexp(amax, &E); /* amax = f * 2^E, f in [0.5, 1): floor(log2(amax)) = E - 1 */
+                int e = (E - 1) - 2;
+                int bi = e + 127;
+                byte = (uint8_t)(bi < 0 ? 0 : (bi > 254 ? 254 : bi));
+            }
+            scales[(int64_t)m * (K / 32) + b] = byte;
+            for (int j = 0; j < 32; j += 2) {
+                uint8_t c0 = 0, c1 = 0;
+                if (!special) {
+                    double inv = ldexp(1.0, 127 - (int)byte); /* 1 / X */
+                    float v0 = (float)((double)xb[j] * inv), v1 = (float)((double)xb[j + 1] * inv);
+                    c0 = qo_round_e2m1_satfinite(v0);
+                    c1 = qo_round_e2m1_satfinite(v1);
+                }
+                codes[(int64_t)m * (K / 2) + b * 16 + j / 2] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    return 0;
+}

@@ -562,3 +562,82 @@ def test_act_quant_error_bound_and_zero_tensor():
             assert np.all(np.abs(blk - Aq[m, 16 * b:16 * b + 16]) <= 1.0 * s * (1 + 1e-6))
     z_codes, z_scales, z_ag = oracle.act_quant(np.zeros((2, 32), np.float32))
     assert z_ag == 0.0 and not z_codes.any() and not z_scales.any()
+
+
+# ----------------------------------------------------------------------------- MXFP4 act quant
+E2M1_MAG = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2), Fraction(3), Fraction(4),
+            Fraction(6)]
+
+
+def _mx_decode(codes, scales, m, j):
+    c = (int(codes[m, j // 2]) >> (4 * (j & 1))) & 0xF
+    return c, int(scales[m, j // 32])
+
+
+def test_act_quant_mx_scale_puts_the_block_max_in_the_top_binade():
+    """OCP MX: X = 2^(floor(log2 amax) - emax_elem) with emax_elem = 2 for E2M1, so amax / X lies
+    in [4, 8) -- the binade of E2M1's 4 and 6 -- for every block not clamped at the UE8M0 range."""
+    rng = np.random.default_rng(11)
+    X = (rng.standard_normal((4, 256)) * np.exp2(rng.integers(-30, 30, (4, 1)))).astype(np.float32)
+    X = torch.tensor(X).to(torch.bfloat16).float().numpy()
+    codes, scales = oracle.act_quant_mx(X)
+    for m in range(4):
+        for b in range(8):
+            amax = Fraction(float(np.max(np.abs(X[m, 32 * b:32 * b + 32].astype(np.float64)))))
+            Xs = Fraction(2) ** (int(scales[m, b]) - 127)
+            assert 4 <= amax / Xs < 8, (m, b, scales[m, b])
+
+
+def test_act_quant_mx_codes_are_nearest_ties_even_saturating():
+    """Every code is the E2M1 value nearest to x / X in exact arithmetic (ties to the even code),
+    with magnitudes from 6 up to 8 saturating to 6 and the sign kept."""
+    rng = np.random.default_rng(12)
+    X = (rng.standard_normal((3, 128)) * 3).astype(np.float32)
+    X[0, :32] = np.linspace(-8, 8, 32)  # block max 8: scale 2^1, every grid point and midpoint region
+    # block max 6 (scale 2^0) holding every midpoint between E2M1 magnitudes: exact ties
+    X[1, :32] = [6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5, -5.0,
+                 7.0, -7.5] + [0.0] * 15
+    X = torch.tensor(X).to(torch.bfloat16).float().numpy()
+    codes, scales = oracle.act_quant_mx(X)
+    for m in range(3):
+        for j in range(128):
+            c, byte = _mx_decode(codes, scales, m, j)
+            q = Fraction(float(X[m, j])) / Fraction(2) ** (byte - 127)
+            a = abs(q)
+            dists = [abs(a - v) for v in E2M1_MAG]
+            best = min(range(8), key=lambda i: (dists[i], i % 2))  # nearest, then even code
+            if a >= 6:
+                best = 7
+            assert (c & 7) == best, (m, j, float(q), c)
+            assert (c >> 3) == (1 if math.copysign(1.0, float(X[m, j])) < 0 else 0)
+
+
+def test_act_quant_mx_grid_round_trip_and_special_blocks():
+    grid = [0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -6.0] * 4  # block max 6: scale 2^0 (byte 127)
+    X = np.array([grid + [v * 2.0 ** -20 for v in grid]], np.float32)
+    codes, scales = oracle.act_quant_mx(X)
+    assert list(scales[0]) == [127, 107]
+    for j in range(64):
+        c, byte = _mx_decode(codes, scales, 0, j)
+        val = float(E2M1_MAG[c & 7]) * (-1 if c & 8 else 1) * 2.0 ** (byte - 127)
+        assert val == X[0, j], j
+    # an all-zero block: byte 0 and zero codes; negative zero keeps its sign (code 8)
+    Z = np.zeros((1, 32), np.float32)
+    Z[0, 3] = -0.0
+    zc, zs = oracle.act_quant_mx(Z)
+    assert zs[0, 0] == 0 and (int(zc[0, 1]) >> 4) == 8 and int(zc[0, 0]) == 0
+    # a block below 2^-125 clamps to byte 0 (X = 2^-127): 2^-130 * 4.5 -> x / X = 0.5625 -> code 1
+    T = np.zeros((1, 32), np.float32)
+    T[0, 0] = np.float32(4.5 * 2.0 ** -130)
+    tc, ts = oracle.act_quant_mx(T)
+    assert ts[0, 0] == 0 and (int(tc[0, 0]) & 0xF) == 1
+    # the largest finite bf16 block: floor(log2(3.39e38)) - 2 = 125 -> byte 252
+    B = np.zeros((1, 32), np.float32)
+    B[0, 5] = torch.tensor(3.3895314e38).to(torch.bfloat16).float().item()
+    bc, bs = oracle.act_quant_mx(B)
+    assert bs[0, 0] == 252
+    # a block holding an infinity: the UE8M0 NaN byte and zero codes
+    I = np.ones((1, 32), np.float32)
+    I[0, 7] = np.inf
+    ic, isc = oracle.act_quant_mx(I)
+    assert isc[0, 0] == 0xFF and not ic.any()

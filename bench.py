@@ -706,9 +706,30 @@ def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
     if sw:
         out["nvfp4_chunk_m_sweep"] = {"workload": "the same GEMM at small M (the GEMV regime on the chunk path)",
                                       "by_M": sw}
+    # MXFP4 weights of the same shape on their own chunk path (MX-quantized activations, kind::mxf4).
+    del packs
+    mpacks = []
+    for c in range(2):
+        b, s_, _ = synth.weights(q.QLIN_MXFP4, N, K, synth.gen(7300 + c, device="cuda"), device="cuda")
+        mpacks.append(q.qlin_pack_weights(q.QLIN_MXFP4, N, K, b, s_, 1.0, q.QLIN_PACK_MMA))
+        del b, s_
+    mx = {}
+    for M in (512, 64):
+        x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(M, N, device="cuda")
+        ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, q.QLIN_MXFP4, M, N, K))
+        fn = lambda: [q.qlin_gemm_chunk(q.QLIN_MXFP4, mpacks[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL)
+                      for c in range(2)]
+        ms = _time_graph_of(fn, args.steps, args.warmup) / 2
+        us = ms * 1e3
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        mx[str(M)] = {"us_per_call": us, "tflops": tf, "fp4_frac": tf / fp4_peaks()[0],
+                      "gbs": (wbytes + 2 * M * K + 4 * M * N) / (us * 1e-6) / 1e9}
+    out["mxfp4_chunk"] = {"workload": "MXFP4 weights of the same shape (UE8M0 scales per 32): MX-quantized "
+                                      "activations + tcgen05 kind::mxf4 GEMM in one launch", "by_M": mx}
+    del mpacks
     # The bf16-operand path for the same NVFP4 weights (QLIN_PACK_MMA_BF16: exact e2m1 * e4m3 products
     # in bf16, x not quantized), tcgen05 kind::f16 on CTA pairs.
-    del packs
     bpacks = []
     for c in range(2):
         b, s_, g = synth.weights(fmt, N, K, synth.gen(7000 + c, device="cuda"), device="cuda")

@@ -43,6 +43,7 @@ SIGNATURES = {
     "qlin_moe_experts": (_I, [_I, _P, _P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P, _I, _P, _SZ, _P]),
     "qlin_gemm_chunk": (_I, [_I, _P, _I64, _I64, _P, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
     "qlin_act_quant_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "qlin_act_quant_mx_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "qlin_dequant_debug": (_I, [_I, _P, _I64, _I64, _I, _P, _P]),
     "qlin_chain_max_ops": (_I, []),
     "qlin_chain_workspace_bytes": (_SZ, [_I, _I, _P, _I]),
@@ -225,6 +226,21 @@ def qlin_act_quant_debug(x, ws=None, stream=None):
                                     _dev(ag, "a_g"), _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
     _check("qlin_act_quant_debug", st)
     return codes, scales, ag
+
+
+def qlin_act_quant_mx_debug(x, ws=None, stream=None):
+    """The MXFP4 chunk path's quantized activations: (codes [M][K/2], UE8M0 scales [M][K/32])."""
+    if x.dtype != torch.bfloat16 or x.stride(1) != 1:
+        raise TypeError("x must be bfloat16 with contiguous rows")
+    M, K = x.shape
+    codes = torch.empty(M, K // 2, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(M, K // 32, dtype=torch.uint8, device=x.device)
+    if ws is None:
+        ws = workspace(qlin_workspace_bytes(QLIN_OP_CHUNK, QLIN_MXFP4, M, 256, K), x.device)
+    st = lib().qlin_act_quant_mx_debug(_dev(x, "x"), M, K, x.stride(0), _dev(codes, "codes"), _dev(scales, "scales"),
+                                       _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    _check("qlin_act_quant_mx_debug", st)
+    return codes, scales
 
 
 def qlin_dequant_debug(fmt, packed, N, K, pack_flags=QLIN_PACK_DEFAULT, stream=None):

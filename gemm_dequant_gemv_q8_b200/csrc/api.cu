@@ -20,8 +20,10 @@ extern "C" int64_t qlin_bf16_cache_bytes(int64_t N, int64_t K);
 extern "C" cudaError_t qlin_launch_chunk_bf16(const void* packed, int64_t N, int64_t K, const void* x, int M,
                                               int64_t ldx, float* y, int64_t ldy, void* ws, int flags,
                                               cudaStream_t s);
-extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
-                                         float* y, int64_t ldy, void* ws, int flags, cudaStream_t s);
+extern "C" cudaError_t qlin_launch_chunk(int fmt, const void* packed, int64_t N, int64_t K, const void* x, int M,
+                                         int64_t ldx, float* y, int64_t ldy, void* ws, int flags, cudaStream_t s);
+extern "C" cudaError_t qlin_launch_act_quant_mx(const void* x, int M, int64_t K, int64_t ldx, void* aq,
+                                                void* canon_codes, void* canon_scales, cudaStream_t s);
 extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* ws,
                                                    void* codes, void* scales, float* ag, cudaStream_t s);
 extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, int64_t K,
@@ -104,7 +106,7 @@ size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags
     if (pack_flags == QLIN_PACK_MMA_BF16)  // the bf16 copy, every format
         return (size_t)qlin::kHdrBytes + (size_t)qlin_bf16_cache_bytes(N, K);
     if (pack_flags == QLIN_PACK_MMA) {
-        if (fmt != QLIN_NVFP4)  // the bf16 copy of the dequantized weights, rows of K rounded up to 64
+        if (fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4)  // the bf16 copy of the dequantized weights, rows of K rounded up to 64
             return (size_t)qlin::kHdrBytes + (size_t)qlin_bf16_cache_bytes(N, K);
         return (size_t)qlin::kHdrBytes + (size_t)((N + 255) / 256) * (size_t)((K + 255) / 256) * 36864u;
     }
@@ -142,7 +144,7 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
     }
     if (op == QLIN_OP_CHUNK) {
         if (M < 1 || M > (1 << 20)) return 0;
-        return fmt == QLIN_NVFP4 ? qlin_chunk_ws_bytes(M, N, K) : 256;  // bf16 path: the status word
+        return (fmt == QLIN_NVFP4 || fmt == QLIN_MXFP4) ? qlin_chunk_ws_bytes(M, N, K) : 256;  // bf16 path: the status word
     }
     if (op == QLIN_OP_GEMV) {
         if (M < 1 || M > 8) return 0;
@@ -209,7 +211,7 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
     if (!packed || !x || !y) return QLIN_ERR_INVALID_ARG;
     if (ldx < K || ldy < N) return QLIN_ERR_INVALID_ARG;
     if (!aligned(packed, 256) || !aligned(x, 2) || !aligned(y, 4)) return QLIN_ERR_ALIGNMENT;
-    if (fmt != QLIN_NVFP4 || (flags & QLIN_FLAG_BF16_COPY)) {
+    if ((fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4) || (flags & QLIN_FLAG_BF16_COPY)) {
         // bf16 path: x is read by tensor-map loads (16-byte aligned rows)
         if (!aligned(x, 16) || ldx % 8) return QLIN_ERR_ALIGNMENT;
         if (!ws || ws_bytes < 256) return QLIN_ERR_WORKSPACE;
@@ -219,7 +221,7 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
     }
     if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, N, K)) return QLIN_ERR_WORKSPACE;
     if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
-    return cuda_status(qlin_launch_chunk(packed, N, K, x, M, ldx, y, ldy, ws, flags, (cudaStream_t)stream));
+    return cuda_status(qlin_launch_chunk(fmt, packed, N, K, x, M, ldx, y, ldy, ws, flags, (cudaStream_t)stream));
 }
 
 qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* codes, void* scales,
@@ -228,6 +230,14 @@ qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx,
     if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, 256, K)) return QLIN_ERR_WORKSPACE;
     if (!aligned(ws, 256) || !aligned(codes, 8) || !aligned(a_g, 4)) return QLIN_ERR_ALIGNMENT;
     return cuda_status(qlin_launch_act_quant_debug(x, M, K, ldx, ws, codes, scales, a_g, (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_act_quant_mx_debug(const void* x, int M, int64_t K, int64_t ldx, void* codes, void* scales,
+                                      void* ws, size_t ws_bytes, qlin_stream_t stream) {
+    if (!x || !codes || !scales || M < 1 || K < 32 || K % 32 || ldx < K) return QLIN_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < qlin_chunk_ws_bytes(M, 256, K)) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256) || !aligned(codes, 8)) return QLIN_ERR_ALIGNMENT;
+    return cuda_status(qlin_launch_act_quant_mx(x, M, K, ldx, (uint8_t*)ws + 256, codes, scales, (cudaStream_t)stream));
 }
 
 qlin_status_t qlin_dequant_debug(qlin_format_t fmt, const void* packed, int64_t N, int64_t K,

@@ -1,17 +1,21 @@
-// chunk_common.cuh -- operand layouts of the NVFP4 prefill-chunk GEMM (tcgen05 block-scaled MMA).
+// chunk_common.cuh -- operand layouts of the NVFP4 / MXFP4 prefill-chunk GEMM (tcgen05 block-scaled
+// MMA).
 //
 // Both operands are stored in global memory exactly as the tensor core reads them from shared
 // memory, so each pipeline stage is filled by plain bulk copies:
 //   codes : rows of 128 bytes (256 E2M1 values of one k-group), 16-byte chunk c of row r stored at
 //           chunk position c ^ (r % 8) -- the 128-byte-swizzled K-major canonical layout; 8-row
 //           groups are 1024 bytes apart.
-//   scales: per 64-value k-block and per 128 rows, a 512-byte atom; the E4M3 scale of row r
-//           (0..127) and 16-value block j (0..3) is at byte (r % 32) * 16 + (r / 32) * 4 + j, the
-//           layout the 32x128b scale-factor copy into tensor memory expects.
+//   scales: per 128 rows and per 4 scale blocks along k, a 512-byte atom; the scale of row r
+//           (0..127) and block j (0..3) is at byte (r % 32) * 16 + (r / 32) * 4 + j, the layout the
+//           32x128b scale-factor copy into tensor memory expects.  NVFP4: E4M3 scales of 16 values,
+//           an atom per 64-value k-block (4 per k-group); MXFP4: UE8M0 scales of 32 values, an atom
+//           per 128-value span (2 per k-group; the two MMAs of a span take bytes 0-1 and 2-3).
 // Weights (QLIN_PACK_MMA): units of 256 rows x 256 values = 32768 B codes + 8 atoms (4 k-blocks x
-// 2 row halves) = 36864 B, in [row tile][k-group] order after the 256-byte header.
+// 2 row halves) = 36864 B, in [row tile][k-group] order after the 256-byte header (MXFP4: 4 atoms,
+// the unit keeps the NVFP4 size).
 // Activations (quantized by the chunk path): units of 128 rows x 256 values = 16384 B codes +
-// 4 atoms = 18432 B, in [row tile][k-group] order.
+// 4 atoms = 18432 B (MXFP4: 2 atoms), in [row tile][k-group] order.
 #pragma once
 #include "qlin_common.cuh"
 
@@ -181,6 +185,66 @@ __device__ __forceinline__ void act_quant_item(const __nv_bfloat16* __restrict__
     act_load_item(x, M, K, ldx, vec, m, b, w);
     const uint8_t s = act_quant_block(w, act_item_amax(w), ag, c8);
     act_store_item(M, K, G, m, b, s, c8, aq, canon_codes, canon_scales);
+}
+
+// ------------------------------------------------------------------ MXFP4 activation quantization
+// The OCP MX conversion, per 32 consecutive values of a row: scale byte = floor(log2 amax) - 2 + 127
+// clamped to [0, 254] (0xFF when the block holds an Inf or NaN), X = 2^(byte - 127), code =
+// E2M1_rne_satfinite(x / X), the division exact (a power of two).  A 32-value block is two 16-value
+// items, 2c and 2c + 1, which the quantizers place in adjacent lanes: one shuffle gives each the
+// block's amax.  For a normal amax with biased exponent be, floor(log2 amax) = be - 127, so the
+// byte is be - 2; amax below 2^-125 (be < 2, zero and subnormals included) clamps to 0.
+__device__ __forceinline__ uint8_t mx_scale_byte(float amax, bool special) {
+    if (special) return 0xFF;
+    const uint32_t be = (__float_as_uint(amax) >> 23) & 0xffu;
+    return (uint8_t)(be >= 2u ? be - 2u : 0u);
+}
+
+__device__ __forceinline__ bool act_item_special(const uint32_t (&w)[8]) {
+    uint32_t sp = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sp |= (uint32_t)((w[j] & 0x7f80u) == 0x7f80u) | (uint32_t)((w[j] & 0x7f800000u) == 0x7f800000u);
+    return sp != 0u;
+}
+
+// Codes of one 16-value item under the scale byte of its 32-value block.
+__device__ __forceinline__ void act_quant_item_mx_codes(const uint32_t (&w)[8], uint8_t byte, uint32_t (&c8)[2]) {
+    c8[0] = c8[1] = 0u;
+    if (byte == 0xFF) return;
+    const float inv = __uint_as_float((254u - byte) << 23);  // 2^(127 - byte), a normal number
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        c8[j >> 2] |= e2m1x2_rne_sat(__fmul_rn(__uint_as_float(w[j] << 16), inv),
+                                     __fmul_rn(__uint_as_float(w[j] & 0xffff0000u), inv))
+                      << (8 * (j & 3));
+}
+
+// Block scale byte of the 32-value block of an item whose partner item sits in lane ^ 1 (every
+// lane of the warp calls this).
+__device__ __forceinline__ uint8_t act_mx_pair_byte(float bmax, bool special) {
+    const float pm = __shfl_xor_sync(0xffffffffu, bmax, 1);
+    const int ps = __shfl_xor_sync(0xffffffffu, special ? 1 : 0, 1);
+    return mx_scale_byte(fmaxf(bmax, pm), special || ps != 0);
+}
+
+// Store item (m, b) of the padded MXFP4 operand: codes as act_store_item; the block's scale byte
+// is written by the even item of the pair (atom layout: 4 scales of 32 values per 128-value span).
+__device__ __forceinline__ void act_store_item_mx(int M, int64_t K, int64_t G, int m, int64_t b, uint8_t byte,
+                                                  const uint32_t (&c8)[2], uint8_t* __restrict__ aq,
+                                                  uint8_t* __restrict__ canon_codes,
+                                                  uint8_t* __restrict__ canon_scales) {
+    const int64_t k = b * 16;
+    const int tm = m / kMmaARows, r = m % kMmaARows;
+    const int64_t g = k / kGroupK;
+    const int kin = (int)(k % kGroupK);
+    uint8_t* ub = aq + ((int64_t)tm * G + g) * kMmaAUnit;
+    const int chunk = kin / 32, within = (kin % 32) / 2;
+    *reinterpret_cast<uint2*>(ub + mma_code_off(r, chunk) + within) = make_uint2(c8[0], c8[1]);
+    if ((b & 1) == 0) ub[kMmaARows * 128 + mma_scale_off(kin / 128, r, (kin % 128) / 32, 1)] = byte;
+    if (canon_codes && m < M && k < K) {
+        memcpy(canon_codes + (int64_t)m * (K / 2) + k / 2, c8, 8);
+        if ((b & 1) == 0) canon_scales[(int64_t)m * (K / 32) + k / 32] = byte;
+    }
 }
 
 }  // namespace qlin

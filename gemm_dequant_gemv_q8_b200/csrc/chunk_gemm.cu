@@ -41,14 +41,19 @@ constexpr int kAccCols = 256;
 // CG = 2: a cluster of two CTAs per 256 x 256 tile (cta_group::2, M = 256): each CTA holds its
 //         128 activation rows and half of the 256 weight rows; the tensor cores of the pair
 //         exchange the halves, so each SM streams 38 KB per k-group instead of 54 KB.
-template <int CG>
+// MX = false: NVFP4 operands (E4M3 scales of 16 values); MX = true: MXFP4 operands (UE8M0 scales of
+// 32 values, half the scale bytes).  The stage layout is the same; MXFP4 copies fewer scale bytes.
+template <int CG, bool MX = false>
 struct ChunkCfg {
     static constexpr int kWCodes = 32768 / CG;                      // weight code bytes per CTA per k-group
     static constexpr int kStageBytes = kMmaAUnit + kWCodes + 4096;  // + all 256 weight rows' scales
-    static constexpr int kScaleBytes = (kMmaAUnit - kMmaARows * 128) + 4096;  // completes on the scale barrier
-    static constexpr int kCodeBytes = kStageBytes - kScaleBytes;
+    static constexpr int kAScale = MX ? 1024 : 2048;                 // activation scale bytes per k-group
+    static constexpr int kWScale = MX ? 2048 : 4096;                 // weight scale bytes (256 rows)
+    static constexpr int kScaleBytes = kAScale + kWScale;            // completes on the scale barrier
+    static constexpr int kCodeBytes = kMmaARows * 128 + kWCodes;
     static constexpr int kStages = CG == 1 ? 4 : 5;
     static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kSfCols = MX ? 24 : 48;  // TMEM columns of one stage's scale factors
 };
 static_assert(ChunkCfg<1>::kStageBytes % 1024 == 0 && ChunkCfg<2>::kStageBytes % 1024 == 0, "stage alignment");
 // Epilogue warps 6-9, each with a staging box of kBoxRows rows x 32 fp32 columns (128-byte rows,
@@ -67,7 +72,7 @@ template <int CG>
 constexpr int chunk_smem() { return 1024 + ChunkCfg<CG>::kRingBytes + EpiCfg<CG>::kBytes + 512; }
 constexpr int kChunkThreads = 320;
 constexpr int kTmemCols = 512;
-constexpr int kSfCols = 48;  // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
+constexpr int kSfCols = 48;  // per stage, NVFP4: 4 k-blocks x (4 SFA + 8 SFB) columns (MXFP4: 2 spans, 24)
 constexpr int kQItems = 8;   // activation items held in registers per thread in phase Q
 static_assert(kAccCols + ChunkCfg<1>::kStages * kSfCols <= kTmemCols, "TMEM budget");
 static_assert(kAccCols + ChunkCfg<2>::kStages * kSfCols <= kTmemCols, "TMEM budget");
@@ -136,8 +141,8 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 // 16 consecutive 32-bit TMEM columns of this warp's lane quarter from r[O .. O+15] of each thread.
-template <int O>
-__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&r)[48]) {
+template <int O, int R>
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&r)[R]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
             taddr),
@@ -239,6 +244,34 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
     }
 }
 
+// MXFP4 x MXFP4 with UE8M0 scales of 32 values (kind::mxf4, scale_vec::2X); the scale byte pair of
+// this K = 64 step is selected by the scale-factor ids of idesc and the top two bits of sfa / sfb.
+template <int CG>
+__device__ __forceinline__ void tc_mma_mx_cg(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    if constexpr (CG == 1)
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+    else
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+            : "memory");
+}
+
+// 8 consecutive 32-bit TMEM columns of this warp's lane quarter from r[O .. O+7] of each thread.
+template <int O, int R>
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t (&r)[R]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[O + 0]),
+                 "r"(r[O + 1]), "r"(r[O + 2]), "r"(r[O + 3]), "r"(r[O + 4]), "r"(r[O + 5]), "r"(r[O + 6]),
+                 "r"(r[O + 7])
+                 : "memory");
+}
+
 template <int CG>
 __device__ __forceinline__ void tc_mma_cg(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
@@ -295,10 +328,10 @@ __device__ __forceinline__ void tmem_free(uint32_t tmem) {
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-template <int CG>
+template <int CG, bool MX>
 __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const ChunkArgs a,
                                                                        const __grid_constant__ CUtensorMap ymap) {
-    using Cfg = ChunkCfg<CG>;
+    using Cfg = ChunkCfg<CG, MX>;
     using Epi = EpiCfg<CG>;
     constexpr int S = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -364,11 +397,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         mbar_arrive_expect_tx(&sfull[s], Cfg::kScaleBytes);
     };
     auto copy_w = [&](uint8_t* st, const uint8_t* wu, int s) {
-        bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, 4096, &sfull[s]);
+        bulk_g2s(st + kMmaAUnit + Cfg::kWCodes, wu + kMmaWRows * 128, Cfg::kWScale, &sfull[s]);
         bulk_g2s(st + kMmaAUnit, wu + rank * Cfg::kWCodes, Cfg::kWCodes, &full[s]);
     };
     auto copy_a = [&](uint8_t* st, const uint8_t* au, int s) {
-        bulk_g2s(st + kMmaARows * 128, au + kMmaARows * 128, kMmaAUnit - kMmaARows * 128, &sfull[s]);
+        bulk_g2s(st + kMmaARows * 128, au + kMmaARows * 128, Cfg::kAScale, &sfull[s]);
         bulk_g2s(st, au, kMmaARows * 128, &full[s]);
     };
     int npre = 0;  // stages of the first tile whose weight part is already in flight (thread 0)
@@ -450,7 +483,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 atomicOr(a.status, 1u);
                 *abort_flag = 1;
             }
-            *ag_sm = ag;
+            *ag_sm = MX ? 1.0f : ag;  // MXFP4 activations carry no per-tensor scale
         }
         __syncthreads();
         // Every CTA of this grid is resident (all passed the barrier): a dependent launch may now
@@ -458,11 +491,23 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         griddep_launch_dependents();
         if (!*abort_flag) {
             const float ag = *ag_sm;
+            // (the items of one warp are 32 consecutive indices and `items` is a multiple of 32, so
+            // the MXFP4 pair shuffles below run with every lane of the warp)
             if (resident) {
 #pragma unroll
                 for (int j = 0; j < kQItems; ++j) {
                     const int64_t i = gtid + j * gthreads;
-                    if (i < items) {
+                    if constexpr (MX) {
+                        const uint8_t byte = act_mx_pair_byte(bmax[j], act_item_special(xw[j]));
+                        if (i < items) {
+                            int mj;
+                            int64_t bj;
+                            item_mb(i, mj, bj);
+                            uint32_t c8[2];
+                            act_quant_item_mx_codes(xw[j], byte, c8);
+                            act_store_item_mx(a.M, a.K, a.G, mj, bj, byte, c8, a.aq, nullptr, nullptr);
+                        }
+                    } else if (i < items) {
                         int mj;
                         int64_t bj;
                         item_mb(i, mj, bj);
@@ -476,7 +521,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     int mi;
                     int64_t bi;
                     item_mb(i, mi, bi);
-                    act_quant_item(a.x, a.M, a.K, a.ldx, a.G, ag, vec, mi, bi, a.aq, nullptr, nullptr);
+                    if constexpr (MX) {
+                        uint32_t w[8], c8[2];
+                        act_load_item(a.x, a.M, a.K, a.ldx, vec, mi, bi, w);
+                        const uint8_t byte = act_mx_pair_byte(act_item_amax(w), act_item_special(w));
+                        act_quant_item_mx_codes(w, byte, c8);
+                        act_store_item_mx(a.M, a.K, a.G, mi, bi, byte, c8, a.aq, nullptr, nullptr);
+                    } else {
+                        act_quant_item(a.x, a.M, a.K, a.ldx, a.G, ag, vec, mi, bi, a.aq, nullptr, nullptr);
+                    }
                 }
             }
             fence_proxy_async_global();  // the operand is read back by bulk copies (async proxy)
@@ -549,9 +602,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
-            // Instruction descriptor: E2M1 x E2M1, E4M3 scales, K-major A and B, M = 128 * CG, N = 256.
-            const uint32_t idesc =
-                (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)((128 * CG) >> 4) << 24);
+            // Instruction descriptor: E2M1 x E2M1, E4M3 scales (MXFP4: UE8M0, bit 23), K-major A and B,
+            // M = 128 * CG, N = 256.
+            const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                   ((uint32_t)((128 * CG) >> 4) << 24) | (MX ? (1u << 23) : 0u);
             int it = 0, tcount = 0;
             for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep, ++tcount) {
                 if (tcount > 0) {
@@ -578,9 +632,18 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     const uint32_t sb = sa + kMmaAUnit;
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
-                        const uint32_t col = tmem + kAccCols + (uint32_t)(s * kSfCols + kb * 12);  // SFA 4, SFB 8
-                        tc_mma_cg<CG>(tmem, sdesc_sw128(sa + kb * 32), sdesc_sw128(sb + kb * 32), idesc, col, col + 4,
-                                      (g > 0 || kb > 0) ? 1u : 0u);
+                        if constexpr (MX) {
+                            // span kb / 2 of the stage's scale columns (SFA 4, SFB 8); bytes 0-1 or 2-3
+                            const uint32_t col = tmem + kAccCols + (uint32_t)(s * Cfg::kSfCols + (kb >> 1) * 12);
+                            const uint32_t sid = (uint32_t)(kb & 1) * 2u;
+                            tc_mma_mx_cg<CG>(tmem, sdesc_sw128(sa + kb * 32), sdesc_sw128(sb + kb * 32),
+                                             idesc | (sid << 29) | (sid << 4), col | (sid << 30), (col + 4) | (sid << 30),
+                                             (g > 0 || kb > 0) ? 1u : 0u);
+                        } else {
+                            const uint32_t col = tmem + kAccCols + (uint32_t)(s * kSfCols + kb * 12);  // SFA 4, SFB 8
+                            tc_mma_cg<CG>(tmem, sdesc_sw128(sa + kb * 32), sdesc_sw128(sb + kb * 32), idesc, col,
+                                          col + 4, (g > 0 || kb > 0) ? 1u : 0u);
+                        }
                     }
                     tc_commit_cg<CG>(&empty[s]);  // frees the stage (smem and its scale columns) in every CTA
                 }
@@ -639,12 +702,14 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 // word r / 32 of 16-byte row r % 32.  Every lane quarter of TMEM gets the whole atom:
                 // lane 32q + i, columns c..c+3 = the atom's 16-byte row i.  Each CTA holds the
                 // scales of its own activation rows and of all 256 weight rows.
+                // (MXFP4: the same, per 128-value span: 2 atoms of activation scales, 4 of weight scales)
                 const uint8_t* st = smem + s * Cfg::kStageBytes;
                 const uint8_t* sfa = st + kMmaARows * 128 + lane * 16;
                 const uint8_t* sfb = st + kMmaAUnit + Cfg::kWCodes + lane * 16;
-                uint32_t r[48];
+                constexpr int NB = MX ? 2 : 4;  // atoms of activation scales per stage
+                uint32_t r[NB * 12];
 #pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
+                for (int kb = 0; kb < NB; ++kb) {
                     const uint4 va = lds128(sfa + kb * 512);
                     const uint4 vb0 = lds128(sfb + (kb * 2 + 0) * 512);
                     const uint4 vb1 = lds128(sfb + (kb * 2 + 1) * 512);
@@ -652,10 +717,15 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                     r[kb * 12 + 4] = vb0.x, r[kb * 12 + 5] = vb0.y, r[kb * 12 + 6] = vb0.z, r[kb * 12 + 7] = vb0.w;
                     r[kb * 12 + 8] = vb1.x, r[kb * 12 + 9] = vb1.y, r[kb * 12 + 10] = vb1.z, r[kb * 12 + 11] = vb1.w;
                 }
-                const uint32_t cbase = tmem + lane_base + kAccCols + (uint32_t)(s * kSfCols);
-                tc_st16<0>(cbase, r);
-                tc_st16<16>(cbase + 16, r);
-                tc_st16<32>(cbase + 32, r);
+                const uint32_t cbase = tmem + lane_base + kAccCols + (uint32_t)(s * Cfg::kSfCols);
+                if constexpr (MX) {
+                    tc_st16<0>(cbase, r);
+                    tc_st8<16>(cbase + 16, r);
+                } else {
+                    tc_st16<0>(cbase, r);
+                    tc_st16<16>(cbase + 16, r);
+                    tc_st16<32>(cbase + 32, r);
+                }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 tc_fence_before();
                 __syncwarp();
@@ -857,12 +927,12 @@ static bool make_y_map(CUtensorMap* map, float* y, int M, int64_t N, int64_t ldy
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int CG>
+template <int CG, bool MX>
 static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     static bool attr_set = false;
     cudaError_t e;
     if (!attr_set) {
-        e = cudaFuncSetAttribute(chunk_gemm_kernel<CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk_smem<CG>());
+        e = cudaFuncSetAttribute(chunk_gemm_kernel<CG, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk_smem<CG>());
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -892,7 +962,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gemm_kernel<CG>, kChunkThreads,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gemm_kernel<CG, MX>, kChunkThreads,
                                                           chunk_smem<CG>());
         if (e != cudaSuccess) return e;
         if (per_sm < 1) return cudaErrorInvalidConfiguration;
@@ -901,7 +971,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
             cfg.gridDim = dim3((unsigned)(sms & ~1));
             cfg.numAttrs = na;
             int clusters = 0;
-            e = cudaOccupancyMaxActiveClusters(&clusters, chunk_gemm_kernel<CG>, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&clusters, chunk_gemm_kernel<CG, MX>, &cfg);
             if (e != cudaSuccess) return e;
             if (clusters < 1) return cudaErrorInvalidConfiguration;
             units = clusters;
@@ -925,11 +995,11 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     CUtensorMap ymap;
     memset(&ymap, 0, sizeof(ymap));
     a.tma_store = make_y_map(&ymap, a.y, a.M, a.N, a.ldy, EpiCfg<CG>::kBoxRows) ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel<CG>, a, ymap);
+    return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel<CG, MX>, a, ymap);
 }
 
-extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t K, const void* x, int M, int64_t ldx,
-                                         float* y, int64_t ldy, void* ws, int flags, cudaStream_t s) {
+extern "C" cudaError_t qlin_launch_chunk(int fmt, const void* packed, int64_t N, int64_t K, const void* x, int M,
+                                         int64_t ldx, float* y, int64_t ldy, void* ws, int flags, cudaStream_t s) {
     uint8_t* w8 = (uint8_t*)ws;
     ChunkArgs a;
     a.w = (const uint8_t*)packed;
@@ -952,7 +1022,9 @@ extern "C" cudaError_t qlin_launch_chunk(const void* packed, int64_t N, int64_t 
     a.KS = 1;
     a.GS = a.G;
     a.status = (unsigned*)ws;
-    return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2>(a, flags, s) : launch_chunk_cg<1>(a, flags, s);
+    if (fmt == QLIN_MXFP4)
+        return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, true>(a, flags, s) : launch_chunk_cg<1, true>(a, flags, s);
+    return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, false>(a, flags, s) : launch_chunk_cg<1, false>(a, flags, s);
 }
 
 extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* ws,

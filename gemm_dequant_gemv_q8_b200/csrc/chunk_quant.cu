@@ -1,6 +1,7 @@
 // chunk_quant.cu -- the chunk path's operand preparation (sm_100a):
-//   * QLIN_PACK_MMA weight packing: canonical NVFP4 -> the tensor-core operand layout;
-//   * NVFP4 quantization of bf16 activations (the A operand).
+//   * QLIN_PACK_MMA weight packing: canonical NVFP4 / MXFP4 -> the tensor-core operand layout;
+//   * NVFP4 / MXFP4 quantization of bf16 activations (the A operand; MXFP4 by the OCP MX rule,
+//     see chunk_common.cuh).
 //
 // Activation quantization rule (the pages name NVFP4 activations only through the block-scaled
 // "mxf4nvf4" MMA -- imp README, "Features", row "sm_120a kernels"; the rule is the adopted reading,
@@ -13,7 +14,9 @@
 namespace qlin {
 
 // ------------------------------------------------------------------ weight packing
-// One CTA per unit (256-row tile, k-group); thread r writes row r.
+// One CTA per unit (256-row tile, k-group); thread r writes row r.  MX: UE8M0 scales of 32 values
+// (canonical [N][K/32]) instead of E4M3 scales of 16 ([N][K/16]).
+template <bool MX>
 __global__ void __launch_bounds__(256) pack_mma_kernel(const uint8_t* __restrict__ codes,
                                                        const uint8_t* __restrict__ scales, int64_t N,
                                                        int64_t K, int64_t G, uint8_t* __restrict__ packed) {
@@ -37,10 +40,18 @@ __global__ void __launch_bounds__(256) pack_mma_kernel(const uint8_t* __restrict
         *reinterpret_cast<uint4*>(ub + mma_code_off(r, c)) = v;
     }
     uint8_t* sc = ub + kMmaWRows * 128;
-    for (int b = 0; b < 16; ++b) {  // 16-value block b of the k-group
-        const int64_t kb16 = k0 + 16 * b;
-        const uint8_t s = (n < N && kb16 < K) ? scales[n * (K / 16) + kb16 / 16] : 0;
-        sc[mma_scale_off(b >> 2, r, b & 3, 2)] = s;
+    if (MX) {
+        for (int b = 0; b < 8; ++b) {  // 32-value block b of the k-group
+            const int64_t kb32 = k0 + 32 * b;
+            const uint8_t s = (n < N && kb32 < K) ? scales[n * (K / 32) + kb32 / 32] : 0;
+            sc[mma_scale_off(b >> 2, r, b & 3, 2)] = s;
+        }
+    } else {
+        for (int b = 0; b < 16; ++b) {  // 16-value block b of the k-group
+            const int64_t kb16 = k0 + 16 * b;
+            const uint8_t s = (n < N && kb16 < K) ? scales[n * (K / 16) + kb16 / 16] : 0;
+            sc[mma_scale_off(b >> 2, r, b & 3, 2)] = s;
+        }
     }
 }
 
@@ -88,16 +99,50 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const __nv_bfloat16* __r
                    canon_scales);
 }
 
+// MXFP4: one thread per (row, 16-value item) of the padded operand; the two items of a 32-value
+// block are adjacent threads of one warp (no global scale, no max pass).
+__global__ void __launch_bounds__(256) act_quant_mx_kernel(const __nv_bfloat16* __restrict__ x, int M, int64_t K,
+                                                           int64_t ldx, int64_t G, int TM, bool vec,
+                                                           uint8_t* __restrict__ aq, uint8_t* __restrict__ canon_codes,
+                                                           uint8_t* __restrict__ canon_scales) {
+    const int64_t nblk16 = G * 16;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool live = idx < (int64_t)TM * kMmaARows * nblk16;  // a multiple of 32: whole warps
+    const int m = live ? (int)(idx / nblk16) : 0;
+    const int64_t b = live ? idx - (int64_t)m * nblk16 : 0;
+    uint32_t w[8], c8[2];
+    act_load_item(x, live ? M : 0, K, ldx, vec, m, b, w);
+    const uint8_t byte = act_mx_pair_byte(act_item_amax(w), act_item_special(w));
+    if (!live) return;
+    act_quant_item_mx_codes(w, byte, c8);
+    act_store_item_mx(M, K, G, m, b, byte, c8, aq, canon_codes, canon_scales);
+}
+
 }  // namespace qlin
 
 using namespace qlin;
 
-extern "C" cudaError_t qlin_launch_pack_mma(const void* codes, const void* scales, int64_t N, int64_t K, float gs,
+extern "C" cudaError_t qlin_launch_pack_mma(int fmt, const void* codes, const void* scales, int64_t N, int64_t K,
                                             void* packed, cudaStream_t s) {
     const int64_t T = (N + kMmaWRows - 1) / kMmaWRows, G = (K + kGroupK - 1) / kGroupK;
-    (void)gs;  // the header (with the per-tensor scale) is written by qlin_launch_pack
-    pack_mma_kernel<<<(unsigned)(T * G), 256, 0, s>>>((const uint8_t*)codes, (const uint8_t*)scales, N, K, G,
-                                                       (uint8_t*)packed);
+    // (the header, with the per-tensor scale, is written by qlin_launch_pack)
+    if (fmt == QLIN_MXFP4)
+        pack_mma_kernel<true><<<(unsigned)(T * G), 256, 0, s>>>((const uint8_t*)codes, (const uint8_t*)scales, N, K, G,
+                                                                 (uint8_t*)packed);
+    else
+        pack_mma_kernel<false><<<(unsigned)(T * G), 256, 0, s>>>((const uint8_t*)codes, (const uint8_t*)scales, N, K,
+                                                                  G, (uint8_t*)packed);
+    return cudaGetLastError();
+}
+
+extern "C" cudaError_t qlin_launch_act_quant_mx(const void* x, int M, int64_t K, int64_t ldx, void* aq,
+                                                void* canon_codes, void* canon_scales, cudaStream_t s) {
+    const int64_t G = (K + kGroupK - 1) / kGroupK;
+    const int TM = (M + kMmaARows - 1) / kMmaARows;
+    const bool vec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0) && (ldx % 8 == 0);
+    const int64_t threads = (int64_t)TM * kMmaARows * G * 16;
+    act_quant_mx_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+        (const __nv_bfloat16*)x, M, K, ldx, G, TM, vec, (uint8_t*)aq, (uint8_t*)canon_codes, (uint8_t*)canon_scales);
     return cudaGetLastError();
 }
 

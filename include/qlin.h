@@ -69,9 +69,9 @@ enum {
                                half of every weight tile).  Same results; the default single-CTA
                                tiling is faster on the sizes measured so far. */
     QLIN_FLAG_BF16_COPY = 0x400  /* qlin_gemm_chunk only: `packed` is a QLIN_PACK_MMA_BF16 buffer, so
-                               the bf16-operand path runs (for NVFP4 weights too: bf16 x, no
-                               activation quantization).  Optional for the formats other than
-                               NVFP4, whose chunk path is always the bf16 one. */
+                               the bf16-operand path runs (for NVFP4 and MXFP4 weights too: bf16 x,
+                               no activation quantization).  Optional for the GGUF formats, whose
+                               chunk path is always the bf16 one. */
 };
 
 /* qlin_pack_weights flags */
@@ -79,10 +79,11 @@ enum {
     QLIN_PACK_DEFAULT = 0,
     QLIN_PACK_GATE_UP = 1, /* the N rows are [gate ; up] halves (N even): each packed tile pairs
                              16 gate rows with their 16 up rows so the SiLU-gate epilogue fuses */
-    QLIN_PACK_MMA = 2,     /* the weight operand of qlin_gemm_chunk.  NVFP4: the tensor-core layout
-                             (tiles of 256 rows x 256 values, 128-byte-swizzled K-major codes, scale
-                             factors in 512-byte atoms), 0.5625 B/weight plus padding to 256 x 256.
-                             Q8_0 / Q4_0 / MXFP4 / Q4_K / Q6_K: a bf16 copy of the dequantized
+    QLIN_PACK_MMA = 2,     /* the weight operand of qlin_gemm_chunk.  NVFP4 / MXFP4: the tensor-core
+                             layout (tiles of 256 rows x 256 values, 128-byte-swizzled K-major codes,
+                             scale factors in 512-byte atoms: E4M3 per 16 values, or UE8M0 per 32),
+                             36864 B per tile (0.5625 B/weight) plus padding to 256 x 256.
+                             Q8_0 / Q4_0 / Q4_K / Q6_K: a bf16 copy of the dequantized
                              weights after the 256-byte header, in blocks of 256 rows x 64 values
                              (32 KB contiguous, rows of 128 bytes): with Kc = roundup(K, 64), row n
                              and column k at element ((n / 256 * Kc / 64 + k / 64) * 256 + n % 256)
@@ -91,7 +92,7 @@ enum {
                              256) zero (2 B/weight: the full-precision prefill copy; imp README
                              "Why this exists": prefill via source dequant) */
     QLIN_PACK_MMA_BF16 = 4  /* the bf16 copy, for every format (the same buffer as QLIN_PACK_MMA for the
-                             formats other than NVFP4).  NVFP4: each element is the product of its
+                             GGUF formats; MXFP4: e2m1 * 2^(scale - 127), exact in bf16).  NVFP4: each element is the product of its
                              E2M1 code and its E4M3 block scale (at most 2 + 4 significant bits,
                              2^-10 <= |v| <= 2688: exact in bf16); the per-tensor scale stays in the
                              header and qlin_gemm_chunk applies it to each output once.  Layout and
@@ -309,11 +310,25 @@ qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, 
                               int M, int64_t ldx, float* y, int64_t ldy, int flags, void* ws,
                               size_t ws_bytes, qlin_stream_t stream);
 
+/* MXFP4 weights (QLIN_PACK_MMA) take the same one-launch form with MXFP4 activations and the
+ * kind::mxf4 MMA (UE8M0 scales of 32 values, the scale byte pair of each K = 64 step selected in the
+ * instruction descriptor): step 1 quantizes x by the OCP MX rule -- per 32 consecutive values of a
+ * row, scale byte = floor(log2 amax) - 2 + 127 clamped to [0, 254] (0xFF for a block holding an Inf
+ * or NaN), code = E2M1_rne_satfinite(x / 2^(byte - 127)) -- with no per-tensor scale, and step 2 is
+ * y[m][n] = sum_k A_q[m][k] * W_q[n][k].  The pages give MXFP4 as E2M1 codes with UE8M0 block scales
+ * (imp release notes v0.6, "Native MXFP4 GGUF weight format"); the activation rule is the OCP MX
+ * conversion. */
+
 /* Test and inspection aid: run step 1 of qlin_gemm_chunk alone and also write the quantized
  * activations in the canonical NVFP4 layout: codes [M][K/2] (element 2i in the low nibble), E4M3
  * scales [M][K/16], and a_g (one float, device memory).  ws as for qlin_gemm_chunk. */
 qlin_status_t qlin_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* codes, void* scales,
                                    float* a_g, void* ws, size_t ws_bytes, qlin_stream_t stream);
+
+/* The same for the MXFP4 chunk path: the MX-quantized activations in canonical layout, codes
+ * [M][K/2] and UE8M0 scale bytes [M][K/32] (K % 32 == 0).  ws as for qlin_gemm_chunk. */
+qlin_status_t qlin_act_quant_mx_debug(const void* x, int M, int64_t K, int64_t ldx, void* codes, void* scales,
+                                      void* ws, size_t ws_bytes, qlin_stream_t stream);
 
 /* Dequantize a packed buffer back to fp32 W[N][K] (row-major, canonical row order, also for
  * QLIN_PACK_GATE_UP buffers; pass the pack_flags the buffer was packed with).  The value of every

@@ -1,6 +1,6 @@
 """GPU parity of the prefill-chunk GEMM for the GGUF and MXFP4 formats (the bf16 path).
 
-qlin_pack_weights(QLIN_PACK_MMA) builds a bf16 copy of the dequantized weights: every weight is the
+qlin_pack_weights(QLIN_PACK_MMA_BF16) builds a bf16 copy of the dequantized weights: every weight is the
 fp32 value the oracle's dequant gives, rounded to nearest-even bf16 (torch's conversion is the
 reference rounding) -- checked bit for bit, tail columns zero.  qlin_gemm_chunk then multiplies bf16
 x by that copy on the tensor cores with fp32 accumulation: checked against the fp64 product with
@@ -28,7 +28,7 @@ def kquant(fmt):
 def make(fmt, N, K, seed):
     blocks, scales, g = synth.weights(fmt, N, K, synth.gen(seed))
     packed = q.qlin_pack_weights(fmt, N, K, blocks.cuda(), None if scales is None else scales.cuda(), g,
-                                 q.QLIN_PACK_MMA)
+                                 q.QLIN_PACK_MMA_BF16)
     w32 = oracle.dequant_f32(fmt, N, K, blocks.numpy(), None if scales is None else scales.numpy(), g)
     return packed, w32
 
@@ -47,7 +47,7 @@ def test_bf16_cache_bit_exact(fmt, N, K):
     if kquant(fmt) and K % 256:
         pytest.skip("K-quants need K % 256 == 0")
     packed, w32 = make(fmt, N, K, 900 + N)
-    assert packed.numel() == q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA)
+    assert packed.numel() == q.qlin_packed_bytes(fmt, N, K, q.QLIN_PACK_MMA_BF16)
     wb, kc = cache(packed, N, K)
     ref = torch.from_numpy(w32).to(torch.bfloat16)
     got = wb[:N, :K].cpu()
@@ -78,6 +78,8 @@ def test_chunk_bf16_parity(fmt, M, N, K, flags):
     if kquant(fmt) and K % 256:
         pytest.skip("K-quants need K % 256 == 0")
     packed, w32 = make(fmt, N, K, 1000 + M)
+    if fmt == q.QLIN_MXFP4:  # MXFP4's own chunk path is the FP4 one; the bf16 copy asks for this flag
+        flags |= q.QLIN_FLAG_BF16_COPY
     x = synth.activations(M, K, synth.gen(1100 + M), dtype=torch.bfloat16).cuda()
     ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
     y = q.qlin_gemm_chunk(fmt, packed, N, K, x, ws=ws, flags=flags)

@@ -21,7 +21,7 @@ QLIN_F32, QLIN_BF16 = 0, 1
 QLIN_EPI_NONE, QLIN_EPI_SILU_GATE, QLIN_OUT_BF16, QLIN_FLAG_PDL, QLIN_FLAG_CTA_PAIRS = 0, 1, 0x10, 0x100, 0x200
 QLIN_FLAG_BF16_COPY = 0x400
 QLIN_PACK_DEFAULT, QLIN_PACK_GATE_UP, QLIN_PACK_MMA, QLIN_PACK_MMA_BF16 = 0, 1, 2, 4
-QLIN_OP_GEMV, QLIN_OP_MOE, QLIN_OP_CHUNK = 1, 2, 3
+QLIN_OP_GEMV, QLIN_OP_MOE, QLIN_OP_CHUNK, QLIN_OP_MOE_PREFILL = 1, 2, 3, 4
 STATUS = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED",
           3: "QLIN_ERR_ALIGNMENT", 4: "QLIN_ERR_WORKSPACE", 5: "QLIN_ERR_CUDA",
           6: "QLIN_ERR_TIMEOUT"}
@@ -42,6 +42,7 @@ SIGNATURES = {
     "qlin_gemv_noalloc_status": (_I, [_P]),
     "qlin_moe_experts": (_I, [_I, _P, _P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P, _I, _P, _SZ, _P]),
     "qlin_gemm_chunk": (_I, [_I, _P, _I64, _I64, _P, _I, _I64, _P, _I64, _I, _P, _SZ, _P]),
+    "qlin_moe_prefill": (_I, [_I, _P, _P, _I, _I64, _I64, _I, _P, _P, _P, _P, _I, _P, _P, _I, _P, _SZ, _P]),
     "qlin_act_quant_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
     "qlin_act_quant_mx_debug": (_I, [_P, _I, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "qlin_dequant_debug": (_I, [_I, _P, _I64, _I64, _I, _P, _P]),
@@ -185,6 +186,31 @@ def qlin_moe_experts(fmt, gate_up_packed, down_packed, E, H, I, top_k, x, router
                                 _dev(h, "h", torch.float32), flags, _dev(ws, "ws"),
                                 ws.numel() * ws.element_size(), _stream(stream))
     _check("qlin_moe_experts", st)
+    return y, topk_ids, topk_w, h
+
+
+def qlin_moe_prefill(fmt, gate_up_packed, down_packed, E, H, I, top_k, x, router_logits=None, topk_ids=None,
+                     topk_w=None, y=None, h=None, ws=None, stream=None):
+    """Routed MoE layer for a prefill chunk of M = x.shape[0] bf16 tokens on the tensor cores
+    (NVFP4 / MXFP4 experts packed with pack_experts(..., QLIN_PACK_MMA[ | QLIN_PACK_GATE_UP])).
+    Returns (y, topk_ids, topk_w, h)."""
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous bfloat16 tensor")
+    M, dev = x.shape[0], x.device
+    if topk_ids is None:
+        topk_ids = torch.empty(M, top_k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(M, top_k, dtype=torch.float32, device=dev)
+    if y is None:
+        y = torch.empty(M, H, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(qlin_workspace_bytes(QLIN_OP_MOE_PREFILL, fmt, M, H, I, E, top_k), dev)
+    st = lib().qlin_moe_prefill(fmt, _dev(gate_up_packed, "gate_up_packed"), _dev(down_packed, "down_packed"), E, H,
+                                I, top_k, _dev(router_logits, "router_logits", torch.float32),
+                                _dev(topk_ids, "topk_ids", torch.int32), _dev(topk_w, "topk_w", torch.float32),
+                                _dev(x, "x"), M, _dev(y, "y", torch.float32), _dev(h, "h", torch.float32), 0,
+                                _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    _check("qlin_moe_prefill", st)
     return y, topk_ids, topk_w, h
 
 

@@ -30,6 +30,12 @@ extern "C" cudaError_t qlin_launch_gemv(int fmt, const void* packed, int64_t N, 
                                         const void* x, int xdt, int M, int64_t ldx, float* y,
                                         int64_t ldy, int flags, void* ws, cudaStream_t s);
 
+extern "C" size_t qlin_moe_prefill_ws_bytes(int M, int64_t H, int64_t I, int E, int top_k);
+extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const void* dn, int E, int64_t H, int64_t I,
+                                               int top_k, const float* logits, int32_t* ids, float* wts,
+                                               const void* x, int M, float* y, float* h, void* ws, size_t gu_stride,
+                                               size_t dn_stride, cudaStream_t s);
+
 extern "C" int qlin_chain_max_ops();
 extern "C" size_t qlin_chain_ws_bytes(int fmt, int M, const qlin_gemv_op* ops, int n_ops);
 extern "C" cudaError_t qlin_launch_chain(int fmt, int xdt, int M, const qlin_gemv_op* ops, int n_ops, int flags,
@@ -103,6 +109,10 @@ qlin_status_t qlin_gemv_chain(qlin_format_t fmt, qlin_dtype_t xdt, int M, const 
 
 size_t qlin_packed_bytes(qlin_format_t fmt, int64_t N, int64_t K, int pack_flags) {
     if (!valid_fmt(fmt) || !valid_shape(fmt, N, K)) return 0;
+    if (pack_flags == (QLIN_PACK_MMA | QLIN_PACK_GATE_UP)) {  // NVFP4 / MXFP4: gate and up rows interleaved
+        if ((fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4) || N % 2) return 0;
+        return (size_t)qlin::kHdrBytes + (size_t)((N / 2 + 127) / 128) * (size_t)((K + 255) / 256) * 36864u;
+    }
     if (pack_flags == QLIN_PACK_MMA_BF16)  // the bf16 copy, every format
         return (size_t)qlin::kHdrBytes + (size_t)qlin_bf16_cache_bytes(N, K);
     if (pack_flags == QLIN_PACK_MMA) {
@@ -121,8 +131,11 @@ qlin_status_t qlin_pack_weights(qlin_format_t fmt, int64_t N, int64_t K, const v
                                 void* packed, size_t packed_bytes, qlin_stream_t stream) {
     if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
     if (!valid_shape(fmt, N, K)) return QLIN_ERR_INVALID_ARG;
-    if (pack_flags != QLIN_PACK_MMA && pack_flags != QLIN_PACK_MMA_BF16 && (pack_flags & ~QLIN_PACK_GATE_UP))
+    if (pack_flags != QLIN_PACK_MMA && pack_flags != QLIN_PACK_MMA_BF16 && (pack_flags & ~QLIN_PACK_GATE_UP) &&
+        pack_flags != (QLIN_PACK_MMA | QLIN_PACK_GATE_UP))
         return QLIN_ERR_INVALID_ARG;
+    if (pack_flags == (QLIN_PACK_MMA | QLIN_PACK_GATE_UP) && fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4)
+        return QLIN_ERR_UNSUPPORTED;
     if ((pack_flags & QLIN_PACK_GATE_UP) && (N % 2)) return QLIN_ERR_INVALID_ARG;
     if (!blocks || !packed) return QLIN_ERR_INVALID_ARG;
     if ((fmt == QLIN_NVFP4 || fmt == QLIN_MXFP4) && !scales) return QLIN_ERR_INVALID_ARG;
@@ -141,6 +154,12 @@ size_t qlin_workspace_bytes(int op, qlin_format_t fmt, int M, int64_t N, int64_t
         if (M < 1 || M > 8 || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return 0;
         if (!valid_shape(fmt, 2 * K, N) || !valid_shape(fmt, N, K)) return 0;
         return qlin_moe_ws_bytes(fmt, M, N, K, E, top_k);
+    }
+    if (op == QLIN_OP_MOE_PREFILL) {  /* N = H, K = I */
+        if ((fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4) || M < 1 || M > (1 << 20) || E < 1 || E > 256 || top_k < 1 ||
+            top_k > 8 || top_k > E || N % 32 || K % 32)
+            return 0;
+        return qlin_moe_prefill_ws_bytes(M, N, K, E, top_k);
     }
     if (op == QLIN_OP_CHUNK) {
         if (M < 1 || M > (1 << 20)) return 0;
@@ -200,6 +219,30 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
     if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
     return cuda_status(qlin_launch_moe(fmt, gate_up_packed, down_packed, E, H, I, top_k, router_logits, topk_ids,
                                        topk_w, x, xdt, M, y, h, flags, ws, (cudaStream_t)stream));
+}
+
+qlin_status_t qlin_moe_prefill(qlin_format_t fmt, const void* gate_up_packed, const void* down_packed, int E,
+                               int64_t H, int64_t I, int top_k, const float* router_logits, int32_t* topk_ids,
+                               float* topk_w, const void* x, int M, float* y, float* h, int flags, void* ws,
+                               size_t ws_bytes, qlin_stream_t stream) {
+    if (!valid_fmt(fmt)) return QLIN_ERR_INVALID_ARG;
+    if (fmt != QLIN_NVFP4 && fmt != QLIN_MXFP4) return QLIN_ERR_UNSUPPORTED;
+    if (M < 1 || M > (1 << 20) || E < 1 || E > 256 || top_k < 1 || top_k > 8 || top_k > E) return QLIN_ERR_INVALID_ARG;
+    if (H < 32 || I < 32 || H % 32 || I % 32 || H > kMaxDim || I > kMaxDim) return QLIN_ERR_INVALID_ARG;
+    if (flags != 0) return QLIN_ERR_INVALID_ARG;
+    if (!gate_up_packed || !down_packed || !topk_ids || !topk_w || !x || !y) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(gate_up_packed, 256) || !aligned(down_packed, 256) || !aligned(x, 16) || !aligned(y, 4) ||
+        !aligned(topk_ids, 4) || !aligned(topk_w, 4) || (router_logits && !aligned(router_logits, 4)) ||
+        (h && !aligned(h, 4)))
+        return QLIN_ERR_ALIGNMENT;
+    const size_t need = qlin_moe_prefill_ws_bytes(M, H, I, E, top_k);
+    if (!ws || ws_bytes < need) return QLIN_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return QLIN_ERR_ALIGNMENT;
+    const size_t gu_stride = qlin_packed_bytes(fmt, 2 * I, H, QLIN_PACK_MMA | QLIN_PACK_GATE_UP);
+    const size_t dn_stride = qlin_packed_bytes(fmt, H, I, QLIN_PACK_MMA);
+    return cuda_status(qlin_launch_moe_prefill(fmt, gate_up_packed, down_packed, E, H, I, top_k, router_logits,
+                                               topk_ids, topk_w, x, M, y, h, ws, gu_stride, dn_stride,
+                                               (cudaStream_t)stream));
 }
 
 qlin_status_t qlin_gemm_chunk(qlin_format_t fmt, const void* packed, int64_t N, int64_t K, const void* x,

@@ -97,7 +97,26 @@ struct ChunkArgs {
     int KS, GS;     // k-splits per output tile (1 or 2) and k-groups per split
     int xvec, yvec, tma_store;  // yvec: y 16-byte aligned with a row pitch of a multiple of 4 floats
     unsigned* status;
+    // Grouped mode (the MoE prefill), tile_expert != nullptr, single CTAs, no k-split: the rows of x
+    // are sorted by expert, each expert's rows padded to whole 128-row tiles; row tile tm belongs to
+    // expert tile_expert[tm], the first *used_tm row tiles are in use (written by an earlier kernel
+    // of the stream), and expert e's packed weights (header included) start at w + e * w_stride.
+    const int* tile_expert;
+    const int* used_tm;
+    int64_t w_stride;
+    // SiLU-gate epilogue (h != nullptr; weights packed with QLIN_PACK_GATE_UP, so accumulator columns
+    // 0..127 are the gate and 128..255 the up rows of outputs 128 t2 .. 128 t2 + 127): h[m][i] =
+    // bf16(silu(g) * u) for i < h_cols, row pitch ldh; y is not written.
+    __nv_bfloat16* h;
+    int64_t ldh, h_cols;
 };
+
+// silu(z) = z * sigmoid(z), the exponential taken of -|z| only.
+__device__ __forceinline__ float chunk_silu(float z) {
+    const float e = expf(-fabsf(z));
+    const float sig = z >= 0.f ? 1.0f / (1.0f + e) : e / (1.0f + e);
+    return z * sig;
+}
 
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     uint64_t d = (uint64_t)((saddr >> 4) & 0x3fffu);
@@ -374,7 +393,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     if constexpr (CG == 2) cluster_sync_all();  // the pair's barriers exist before either CTA signals the other
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int TMP = a.TM / CG;  // activation tiles of 128 * CG rows
+    const int TMA = a.tile_expert ? *a.used_tm : a.TM;  // activation row tiles in use
+    const int TMP = TMA / CG;  // activation tiles of 128 * CG rows
     const int ntiles = a.T2 * TMP * a.KS;
     const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
     // Work item `tile`: weight tile t2, activation tile tm (this CTA's 128 rows of it) and the
@@ -386,6 +406,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         tm = (rest % TMP) * CG + (int)rank;
         g0 = ks * a.GS;
         g1 = g0 + a.GS < a.G ? g0 + a.GS : a.G;
+    };
+    // Packed weights of the expert of row tile tm (grouped mode), else of the one matrix.
+    auto wbase = [&](int tm) -> const uint8_t* {
+        return a.tile_expert ? a.w + (int64_t)a.tile_expert[tm] * a.w_stride : a.w;
     };
     // The weights do not depend on x: the producer starts the first stages' weight copies now, so
     // they land during phase Q (the stage barriers also expect the activation bytes, copied once
@@ -411,7 +435,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         npre = g1 - g0 < S ? g1 - g0 : S;
         for (int it = 0; it < npre; ++it) {
             uint8_t* st = smem + it * Cfg::kStageBytes;
-            const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g0 + it) * kMmaWUnit;
+            const uint8_t* wu = wbase(tm) + kHdrBytes + ((int64_t)t2 * a.G + g0 + it) * kMmaWUnit;
             expect_stage(it);
             copy_w(st, wu, it);
         }
@@ -427,7 +451,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     {
         const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
         const int64_t gthreads = (int64_t)gridDim.x * blockDim.x;
-        const int64_t items = (int64_t)a.TM * a.G * kUnitItems;
+        const int64_t items = (int64_t)TMA * a.G * kUnitItems;
         const bool resident = items <= gthreads * kQItems;
         const bool vec = a.xvec != 0;
         auto item_mb = [&](int64_t i, int& m, int64_t& b) {
@@ -455,7 +479,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 m = fmaxf(m, bmax[j]);
             }
         } else {
-            m = act_amax_partial(a.x, a.M, a.K, a.ldx, vec, gtid, gthreads);
+            // (grouped: only the row tiles in use; the rows past them hold no data of this call)
+            m = act_amax_partial(a.x, a.tile_expert ? TMA * kMmaARows : a.M, a.K, a.ldx, vec, gtid, gthreads);
         }
         if (a.KS > 1) {  // the k-split halves add into y: zero it (ordered before them by the barrier)
             const int64_t nq = (a.N + 3) / 4;
@@ -590,7 +615,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                         break;
                     }
                     uint8_t* st = smem + s * Cfg::kStageBytes;
-                    const uint8_t* wu = a.w + kHdrBytes + ((int64_t)t2 * a.G + g) * kMmaWUnit;
+                    const uint8_t* wu = wbase(tm) + kHdrBytes + ((int64_t)t2 * a.G + g) * kMmaWUnit;
                     if (it >= npre) {  // (the first stages' weights were started before phase Q)
                         expect_stage(s);
                         copy_w(st, wu, s);
@@ -741,7 +766,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         const int q = warp & 3;
         const int c_lo = ((warp - Epi::kFirstWarp) >> 2) * Epi::kCols;  // this warp's first column
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float gw_ag = __fmul_rn(reinterpret_cast<const PackedHeader*>(a.w)->global_scale, *ag_sm);
+        float gw_ag = __fmul_rn(reinterpret_cast<const PackedHeader*>(a.w)->global_scale, *ag_sm);
         uint8_t* tb = epi + (warp - Epi::kFirstWarp) * Epi::kBuf;
         constexpr int R = Epi::kBoxRows;
         const bool tma = a.tma_store != 0;
@@ -759,6 +784,44 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             tile_of(tile, t2, tm, g0, g1);
             const int m0 = tm * kMmaARows + q * 32;  // this warp's first row
             const int64_t n0 = (int64_t)t2 * kMmaWRows;
+            if (a.tile_expert)  // this tile's expert's per-tensor scale
+                gw_ag = __fmul_rn(reinterpret_cast<const PackedHeader*>(wbase(tm))->global_scale, *ag_sm);
+            if (a.h) {
+                // SiLU-gate epilogue: columns c (gate) and c + 128 (up) of output 128 t2 + c; this
+                // thread's row m0 + lane; 32 outputs of one row per step, stored as bf16.
+                const int row = m0 + lane;
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 32) {
+                    float g[32], u[32];
+                    tc_ld32(tmem + lane_base + (uint32_t)c, g);
+                    tc_ld32(tmem + lane_base + (uint32_t)(128 + c), u);
+                    if (c == 96) {  // every column of this warp's rows is read: release them
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acc_empty);
+                    }
+                    const int64_t i0 = (int64_t)t2 * 128 + c;
+                    if (row >= a.M || i0 >= a.h_cols) continue;
+                    __nv_bfloat16* dst = a.h + (int64_t)row * a.ldh + i0;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float h0 = chunk_silu(g[2 * j] * gw_ag) * (u[2 * j] * gw_ag);
+                        const float h1 = chunk_silu(g[2 * j + 1] * gw_ag) * (u[2 * j + 1] * gw_ag);
+                        const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
+                        pk[j] = *reinterpret_cast<const uint32_t*>(&hb);
+                    }
+                    if (i0 + 32 <= a.h_cols && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            reinterpret_cast<uint4*>(dst)[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    } else {
+                        for (int j = 0; j < 32 && i0 + j < a.h_cols; ++j)
+                            dst[j] = __ushort_as_bfloat16((unsigned short)(pk[j >> 1] >> (16 * (j & 1))));
+                    }
+                }
+                continue;
+            }
 #pragma unroll 1
             for (int c = c_lo; c < c_lo + Epi::kCols; c += 32) {
                 float v[32];
@@ -981,7 +1044,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     }
     // Too few output tiles to give every CTA one: split each tile's k-groups in two halves.
     const int base_tiles = a.T2 * (a.TM / CG);
-    a.KS = (CG == 1 && a.G >= 2 && 2 * base_tiles <= max_units) ? 2 : 1;
+    a.KS = (CG == 1 && !a.tile_expert && a.G >= 2 && 2 * base_tiles <= max_units) ? 2 : 1;
     a.GS = (a.G + a.KS - 1) / a.KS;
     const int ntiles = base_tiles * a.KS;
     const int units = ntiles < max_units ? ntiles : max_units;
@@ -994,7 +1057,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     cfg.numAttrs = na;
     CUtensorMap ymap;
     memset(&ymap, 0, sizeof(ymap));
-    a.tma_store = make_y_map(&ymap, a.y, a.M, a.N, a.ldy, EpiCfg<CG>::kBoxRows) ? 1 : 0;
+    a.tma_store = (!a.h && a.y && make_y_map(&ymap, a.y, a.M, a.N, a.ldy, EpiCfg<CG>::kBoxRows)) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel<CG, MX>, a, ymap);
 }
 
@@ -1022,6 +1085,11 @@ extern "C" cudaError_t qlin_launch_chunk(int fmt, const void* packed, int64_t N,
     a.KS = 1;
     a.GS = a.G;
     a.status = (unsigned*)ws;
+    a.tile_expert = nullptr;
+    a.used_tm = nullptr;
+    a.w_stride = 0;
+    a.h = nullptr;
+    a.ldh = a.h_cols = 0;
     if (fmt == QLIN_MXFP4)
         return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, true>(a, flags, s) : launch_chunk_cg<1, true>(a, flags, s);
     return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, false>(a, flags, s) : launch_chunk_cg<1, false>(a, flags, s);
@@ -1034,4 +1102,46 @@ extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t
     cudaError_t e = qlin_launch_act_quant(x, M, K, ldx, words, w8 + 256, codes, scales, s);
     if (e != cudaSuccess) return e;
     return cudaMemcpyAsync(ag, words + 2, 4, cudaMemcpyDeviceToDevice, s);
+}
+
+// Grouped launch (the MoE prefill): x = the expert-sorted bf16 activations (rows_max rows with
+// K % 8 == 0 values each, the first *used_tm * 128 rows in use), w = E packed weight buffers
+// w_stride bytes apart, T2 weight tiles per expert.  h != nullptr: the SiLU-gate epilogue (weights
+// packed QLIN_PACK_MMA | QLIN_PACK_GATE_UP) writing h_cols bf16 outputs per row; else y (fp32, N
+// columns).  Single CTAs, no k-split, no programmatic dependent launch (the routing kernel before it
+// writes the tile table this launch reads at its start).
+extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t w_stride, int T2, int64_t N,
+                                                 int64_t K, const void* x, int rows_max, float* y, int64_t ldy,
+                                                 void* h, int64_t ldh, int64_t h_cols, const int* tile_expert,
+                                                 const int* used_tm, void* ws, cudaStream_t s) {
+    uint8_t* w8 = (uint8_t*)ws;
+    ChunkArgs a;
+    memset(&a, 0, sizeof(a));
+    a.w = (const uint8_t*)w;
+    a.x = (const __nv_bfloat16*)x;
+    a.ldx = K;
+    a.aq = w8 + 256;
+    a.words = (unsigned*)(w8 + 64);
+    a.ready = (unsigned*)(w8 + 256 +
+                          chunk_units_m(rows_max, QLIN_FLAG_CTA_PAIRS) * ((K + kGroupK - 1) / kGroupK) * kMmaAUnit);
+    a.y = y;
+    a.ldy = ldy;
+    a.M = rows_max;
+    a.N = N;
+    a.K = K;
+    a.T2 = T2;
+    a.G = (int)((K + kGroupK - 1) / kGroupK);
+    a.TM = (int)chunk_units_m(rows_max, 0);
+    a.xvec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && K % 8 == 0) ? 1 : 0;
+    a.yvec = (y && (reinterpret_cast<uintptr_t>(y) & 15) == 0 && ldy % 4 == 0) ? 1 : 0;
+    a.KS = 1;
+    a.GS = a.G;
+    a.status = (unsigned*)ws;
+    a.tile_expert = tile_expert;
+    a.used_tm = used_tm;
+    a.w_stride = w_stride;
+    a.h = (__nv_bfloat16*)h;
+    a.ldh = ldh;
+    a.h_cols = h_cols;
+    return fmt == QLIN_MXFP4 ? launch_chunk_cg<1, true>(a, 0, s) : launch_chunk_cg<1, false>(a, 0, s);
 }

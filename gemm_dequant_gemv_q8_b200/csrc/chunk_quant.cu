@@ -15,15 +15,23 @@ namespace qlin {
 
 // ------------------------------------------------------------------ weight packing
 // One CTA per unit (256-row tile, k-group); thread r writes row r.  MX: UE8M0 scales of 32 values
-// (canonical [N][K/32]) instead of E4M3 scales of 16 ([N][K/16]).
+// (canonical [N][K/32]) instead of E4M3 scales of 16 ([N][K/16]).  gate_half > 0 (QLIN_PACK_GATE_UP,
+// the N = 2 * gate_half rows being [gate ; up]): tile t holds gate rows 128t .. 128t + 127 in its
+// rows 0..127 and the matching up rows in rows 128..255, so an output tile holds g and u of the same
+// 128 outputs (rows past gate_half are zero).
 template <bool MX>
 __global__ void __launch_bounds__(256) pack_mma_kernel(const uint8_t* __restrict__ codes,
                                                        const uint8_t* __restrict__ scales, int64_t N,
-                                                       int64_t K, int64_t G, uint8_t* __restrict__ packed) {
+                                                       int64_t K, int64_t G, int64_t gate_half,
+                                                       uint8_t* __restrict__ packed) {
     const int64_t unit = blockIdx.x;
     const int64_t t = unit / G, g = unit % G;
     const int r = threadIdx.x;
-    const int64_t n = t * kMmaWRows + r;
+    int64_t n = t * kMmaWRows + r;
+    if (gate_half > 0) {
+        const int64_t i = t * 128 + (r & 127);
+        n = i < gate_half ? (r < 128 ? i : gate_half + i) : N;  // N: a zero row
+    }
     uint8_t* ub = packed + kHdrBytes + unit * (int64_t)kMmaWUnit;
     const int64_t k0 = g * kGroupK;
 #pragma unroll 1
@@ -122,16 +130,22 @@ __global__ void __launch_bounds__(256) act_quant_mx_kernel(const __nv_bfloat16* 
 
 using namespace qlin;
 
+// Weight tiles of the MMA layout: 256 rows each, or (gate_up) one per 128 gate rows.
+extern "C" int64_t qlin_mma_tiles(int64_t N, int gate_up) {
+    return gate_up ? (N / 2 + 127) / 128 : (N + kMmaWRows - 1) / kMmaWRows;
+}
+
 extern "C" cudaError_t qlin_launch_pack_mma(int fmt, const void* codes, const void* scales, int64_t N, int64_t K,
-                                            void* packed, cudaStream_t s) {
-    const int64_t T = (N + kMmaWRows - 1) / kMmaWRows, G = (K + kGroupK - 1) / kGroupK;
+                                            int gate_up, void* packed, cudaStream_t s) {
+    const int64_t T = qlin_mma_tiles(N, gate_up), G = (K + kGroupK - 1) / kGroupK;
+    const int64_t half = gate_up ? N / 2 : 0;
     // (the header, with the per-tensor scale, is written by qlin_launch_pack)
     if (fmt == QLIN_MXFP4)
         pack_mma_kernel<true><<<(unsigned)(T * G), 256, 0, s>>>((const uint8_t*)codes, (const uint8_t*)scales, N, K, G,
-                                                                 (uint8_t*)packed);
+                                                                 half, (uint8_t*)packed);
     else
         pack_mma_kernel<false><<<(unsigned)(T * G), 256, 0, s>>>((const uint8_t*)codes, (const uint8_t*)scales, N, K,
-                                                                  G, (uint8_t*)packed);
+                                                                  G, half, (uint8_t*)packed);
     return cudaGetLastError();
 }
 

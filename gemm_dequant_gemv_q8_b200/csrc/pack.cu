@@ -338,16 +338,21 @@ using namespace qlin;
 extern "C" int64_t qlin_bf16_cache_cols(int64_t K);
 
 extern "C" cudaError_t qlin_launch_pack_mma(int fmt, const void* codes, const void* scales, int64_t N, int64_t K,
-                                            void* packed, cudaStream_t s);
+                                            int gate_up, void* packed, cudaStream_t s);
 
 extern "C" cudaError_t qlin_launch_pack(int fmt, const void* blocks, const void* scales, int64_t N,
                                         int64_t K, int pack_flags, float gs, void* packed,
                                         cudaStream_t s) {
+    if ((pack_flags & ~QLIN_PACK_GATE_UP) == QLIN_PACK_MMA && (fmt == QLIN_NVFP4 || fmt == QLIN_MXFP4)) {
+        const int gu = (pack_flags & QLIN_PACK_GATE_UP) ? 1 : 0;
+        write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags, gs,
+                                             (int32_t)(gu ? (N / 2 + 127) / 128 : (N + 255) / 256),
+                                             (int32_t)((K + 255) / 256));
+        return qlin_launch_pack_mma(fmt, blocks, scales, N, K, gu, packed, s);
+    }
     if (pack_flags == QLIN_PACK_MMA || pack_flags == QLIN_PACK_MMA_BF16) {
         write_header_kernel<<<1, 64, 0, s>>>((uint8_t*)packed, (uint32_t)fmt, N, K, (uint32_t)pack_flags, gs,
                                              (int32_t)((N + 255) / 256), (int32_t)((K + 255) / 256));
-        if ((fmt == QLIN_NVFP4 || fmt == QLIN_MXFP4) && pack_flags == QLIN_PACK_MMA)
-            return qlin_launch_pack_mma(fmt, blocks, scales, N, K, packed, s);
         const int64_t Kc = qlin_bf16_cache_cols(K);
         const int64_t threads = (N + 255) / 256 * 256 * (Kc / 32);
         const dim3 grid((unsigned)((threads + 255) / 256));

@@ -100,7 +100,7 @@ enum {
 };
 
 /* qlin_workspace_bytes ops */
-enum { QLIN_OP_GEMV = 1, QLIN_OP_MOE = 2, QLIN_OP_CHUNK = 3 };
+enum { QLIN_OP_GEMV = 1, QLIN_OP_MOE = 2, QLIN_OP_CHUNK = 3, QLIN_OP_MOE_PREFILL = 4 };
 
 /* ------------------------------------------------------------------------- weight repacking */
 
@@ -270,6 +270,35 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
                                int32_t* topk_ids, float* topk_w, const void* x, qlin_dtype_t xdt, int M,
                                float* y, float* h, int flags, void* ws, size_t ws_bytes,
                                qlin_stream_t stream);
+
+/* Top-k routed MoE expert projections for a prefill chunk of M tokens (M >= 1; built for M >= 64) on
+ * the tcgen05 tensor cores: what qlin_moe_experts computes -- the same routing (top_k by logit, ties
+ * to the lower expert index, a NaN logit ranks as -inf, weights renormalised over the selected
+ * experts), h = silu(W_gate[e] x) * (W_up[e] x), o = W_down[e] h, y[m] = sum over slots in slot
+ * order of weight * o -- with NVFP4 or MXFP4 expert weights and the chunk path's quantization of the
+ * activations: the (token, slot) rows are sorted by expert (tokens ascending, each expert's rows
+ * padded to whole 128-row tiles) and quantized as qlin_gemm_chunk quantizes x (NVFP4: one
+ * per-tensor scale over all sorted rows; MXFP4: the OCP MX rule), each 128-row tile multiplied by
+ * its expert's weights with the SiLU-gate fused in the epilogue; h is kept as bf16 and quantized
+ * the same way for the down projection (NVFP4: with its own per-tensor scale).  The pages'
+ * counterpart is imp's MoE top-k grouped GEMM, an NVFP4 grouped GEMM on sm_120a (imp README,
+ * "Features" table, row "Architectures"; release notes v0.7.0).  Five launches on `stream`
+ * (route + sort, gather, two grouped GEMMs, combine), no host synchronisation.
+ *   gate_up_packed: E consecutive buffers, each qlin_packed_bytes(fmt, 2I, H, QLIN_PACK_MMA |
+ *                   QLIN_PACK_GATE_UP) bytes, expert e packed from its [gate ; up] rows (2I x H)
+ *   down_packed   : E consecutive buffers, each qlin_packed_bytes(fmt, H, I, QLIN_PACK_MMA) bytes
+ *   router_logits : M x E fp32, or NULL -- then topk_ids / topk_w are inputs (a bad or repeated id is
+ *                   skipped and qlin_ws_status() reports QLIN_ERR_INVALID_ARG)
+ *   topk_ids, topk_w: M x top_k int32 / fp32, written when router_logits is given
+ *   x : M x H bf16, contiguous, 16-byte aligned;  y : M x H fp32, contiguous
+ *   h : optional M x top_k x I fp32: the bf16 h of each (token, slot), as fp32 (NULL: not written)
+ *   flags: 0;  ws: qlin_workspace_bytes(QLIN_OP_MOE_PREFILL, fmt, M, H, I, E, top_k) bytes
+ * fmt NVFP4 or MXFP4 (else QLIN_ERR_UNSUPPORTED); E <= 256, top_k <= min(8, E); H % 32 == 0 and
+ * I % 32 == 0 (QLIN_ERR_INVALID_ARG otherwise).  Bounded device waits as qlin_gemm_chunk. */
+qlin_status_t qlin_moe_prefill(qlin_format_t fmt, const void* gate_up_packed, const void* down_packed, int E,
+                               int64_t H, int64_t I, int top_k, const float* router_logits, int32_t* topk_ids,
+                               float* topk_w, const void* x, int M, float* y, float* h, int flags, void* ws,
+                               size_t ws_bytes, qlin_stream_t stream);
 
 /* ------------------------------------------------------------------------- prefill-chunk GEMM */
 

@@ -98,7 +98,8 @@ def test_pack_argument_checks(lib):
     assert f(2, 64, 256, P(0), None, 1.0, 0, P(0x1000), 1 << 30, None) == 1
     assert f(3, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # NVFP4 needs scales
     assert f(4, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 1 << 30, None) == 1  # MXFP4 needs scales
-    assert f(4, 64, 256, P(0x1000), P(0x2000), 1.0, 3, P(0x10000), 1 << 30, None) == 1  # no gate_up MMA form
+    assert f(2, 64, 256, P(0x1000), None, 1.0, 3, P(0x10000), 1 << 30, None) == 2  # gate_up MMA form: FP4 only
+    assert f(4, 63, 256, P(0x1000), P(0x2000), 1.0, 3, P(0x10000), 1 << 30, None) == 1  # ... with N even
     assert f(2, 64, 256, P(0x1000), None, 1.0, 2, P(0x10000), 256 + 64 * 256, None) == 1  # bf16 copy needs 2 B/w
     assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10010), 1 << 30, None) == 3
     assert f(2, 64, 256, P(0x1000), None, 1.0, 0, P(0x10000), 10, None) == 1

@@ -663,6 +663,73 @@ def cfg_moe(args, cpu=True):
     return out
 
 
+def cfg_moe_prefill(args, cpu=True):
+    """NVFP4 / MXFP4 MoE expert layer of the 8B-A1B shape (hidden 2048, 32 experts of gate_up
+    2048 -> 2 x 1792 and down 1792 -> 2048, top-4) over a prefill chunk of M = 512 (and 2048) bf16
+    tokens on the tensor cores: route + sort, gather, two grouped GEMMs, combine.  Two layers with
+    distinct weights alternate (each 198 MB of packed experts, above L2).  At 64 routed rows per
+    expert on average the layer sits below the FP4 ridge point, so its roofline is HBM: every
+    expert's packed weights once per layer, plus x, y and the logits."""
+    import gemm_dequant_gemv_q8_b200 as q
+    E, H, I, k, L = 32, 2048, 1792, 4, 2
+    out = {}
+    for fmt, fname in ((q.QLIN_NVFP4, "NVFP4"), (q.QLIN_MXFP4, "MXFP4")):
+        gu, dn = [], []
+        for l in range(L):
+            c = [synth.weights(fmt, 2 * I, H, synth.gen(8000 + 100 * l + e, device="cuda"), device="cuda")
+                 for e in range(E)]
+            gu.append(q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_MMA | q.QLIN_PACK_GATE_UP))
+            c = [synth.weights(fmt, H, I, synth.gen(8500 + 100 * l + e, device="cuda"), device="cuda")
+                 for e in range(E)]
+            dn.append(q.pack_experts(fmt, E, H, I, c, q.QLIN_PACK_MMA))
+            del c
+        per_expert = (q.qlin_packed_bytes(fmt, 2 * I, H, q.QLIN_PACK_MMA | q.QLIN_PACK_GATE_UP) - 256 +
+                      q.qlin_packed_bytes(fmt, H, I, q.QLIN_PACK_MMA) - 256)
+        for M in ((512, 2048) if fmt == q.QLIN_NVFP4 else (512,)):
+            logits = [synth.router_logits(M, E, synth.gen(8900 + l, device="cuda"), device="cuda") for l in range(L)]
+            x = synth.activations(M, H, synth.gen(8950, device="cuda"), dtype=torch.bfloat16, device="cuda")
+            ids = torch.empty(M, k, dtype=torch.int32, device="cuda")
+            w = torch.empty(M, k, device="cuda")
+            y = torch.empty(M, H, device="cuda")
+            ws = [q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, fmt, M, H, I, E, k)) for _ in range(L)]
+
+            def fn():
+                for l in range(L):
+                    q.qlin_moe_prefill(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
+                                       topk_w=w, y=y, ws=ws[l])
+            ms, clk = timed(fn, args.steps, args.warmup)
+            distinct, rows_padded = [], []
+            for l in range(L):  # the routing these seeds give: experts in use, padded sorted rows
+                q.qlin_moe_prefill(fmt, gu[l], dn[l], E, H, I, k, x, router_logits=logits[l], topk_ids=ids,
+                                   topk_w=w, y=y, ws=ws[l])
+                cnt = torch.bincount(ids.flatten().long(), minlength=E).cpu()
+                distinct.append(int((cnt > 0).sum()))
+                rows_padded.append(int(((cnt + 127) // 128 * 128).sum()))
+            nd = sum(distinct) / L
+            us = ms / L * 1e3
+            flop = 2.0 * M * k * (2 * I * H + H * I)
+            bytes_ = nd * per_expert + M * (2 * H + 4 * H + 4 * E)
+            tf = flop / (us * 1e-6) / 1e12
+            rl = roofline_hbm(f"moe prefill layer ({fname}: route, gather, grouped gate_up + SiLU, grouped down, "
+                              "combine; 5 launches)", bytes_, us)
+            rl["tensor_frac"] = tf / fp4_peaks()[0]
+            e = {"workload": f"{fname} MoE expert layer of the 8B-A1B shape over a prefill chunk: hidden 2048, 32 "
+                             f"experts gate_up 2048->2x1792, down 1792->2048, top-4, M={M} bf16 tokens; two layers' "
+                             "weights alternate (198 MB each)", "M": M, "distinct_experts": nd,
+                 "sorted_rows_padded": sum(rows_padded) / L, "us_per_layer": us, "tflops": tf,
+                 "value": bytes_ / (us * 1e-6) / 1e9, "unit": "GB/s", "roofline": rl, "clocks": clk,
+                 "bytes": "every routed expert's packed weights + x (bf16), y (fp32), logits",
+                 "flop": "2 * M * top_k * (2I * H + H * I), padding rows excluded"}
+            if cpu and M == 512:
+                e["cpu_baseline"] = cpu_baseline(fmt, [(2 * I, H), (H, I)], M * k // E, xdt=torch.bfloat16,
+                                                 what="MoE expert (the mean routed rows per expert)")
+            out[f"{fname.lower()}_moe_prefill_m{M}"] = e
+            del ws
+        del gu, dn
+        torch.cuda.empty_cache()
+    return out
+
+
 def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
     """NVFP4 prefill-chunk GEMM, K = 5120, N = 17408: M = 512 (tensor-bound) and 64 (HBM-bound),
     and an M sweep on the same matrix; two weight copies alternate so that consecutive calls do not
@@ -755,7 +822,7 @@ def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
 
 
 CONFIGS = {"q8_small": cfg_q8_small, "nvfp4_mlp": cfg_mlp, "moe": cfg_moe, "chunk": cfg_chunk,
-           "mxfp4_mlp": lambda a, cpu=True: cfg_mlp(a, "mxfp4", cpu)}
+           "moe_prefill": cfg_moe_prefill, "mxfp4_mlp": lambda a, cpu=True: cfg_mlp(a, "mxfp4", cpu)}
 
 
 def run_config(name, args):
@@ -818,11 +885,12 @@ def run_config(name, args):
 def small_case(name, reps=3):
     """A few launches of one kernel on one layer, for ncu captures that end in seconds (the
     profiles under profiles/ name these commands): moe1 / moe8 = one Q4_0 MoE layer of the 8B-A1B
-    shape at M = 1 / 8; mlp1 / mlp4 = one NVFP4 27B-shaped MLP as a two-op GEMV chain (h in bf16)
+    shape at M = 1 / 8; moepf512 = one NVFP4 MoE prefill layer of that shape at M = 512 (five
+    launches per call); mlp1 / mlp4 = one NVFP4 27B-shaped MLP as a two-op GEMV chain (h in bf16)
     at M = 1 / 4."""
     import gemm_dequant_gemv_q8_b200 as q
     torch.cuda.set_device(0)
-    if name.startswith("moe"):
+    if name.startswith("moe") and not name.startswith("moepf"):
         M = int(name[3:])
         fmt, E, H, I, k = q.QLIN_Q4_0, 32, 2048, 1792, 4
         c = [synth.weights(fmt, 2 * I, H, synth.gen(4000 + e, device="cuda"), device="cuda") for e in range(E)]
@@ -835,6 +903,19 @@ def small_case(name, reps=3):
         ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE, fmt, M, H, I, E, k))
         for _ in range(reps):
             q.qlin_moe_experts(fmt, gu, dn, E, H, I, k, x, router_logits=logits, ws=ws)
+    elif name.startswith("moepf"):
+        M = int(name[5:])
+        fmt, E, H, I, k = q.QLIN_NVFP4, 32, 2048, 1792, 4
+        c = [synth.weights(fmt, 2 * I, H, synth.gen(8000 + e, device="cuda"), device="cuda") for e in range(E)]
+        gu = q.pack_experts(fmt, E, 2 * I, H, c, q.QLIN_PACK_MMA | q.QLIN_PACK_GATE_UP)
+        c = [synth.weights(fmt, H, I, synth.gen(8500 + e, device="cuda"), device="cuda") for e in range(E)]
+        dn = q.pack_experts(fmt, E, H, I, c, q.QLIN_PACK_MMA)
+        del c
+        logits = synth.router_logits(M, E, synth.gen(8900, device="cuda"), device="cuda")
+        x = synth.activations(M, H, synth.gen(8950, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, fmt, M, H, I, E, k))
+        for _ in range(reps):
+            q.qlin_moe_prefill(fmt, gu, dn, E, H, I, k, x, router_logits=logits, ws=ws)
     elif name.startswith("mlp"):
         M = int(name[3:])
         fmt, H, I = q.QLIN_NVFP4, 5120, 17408
@@ -924,11 +1005,11 @@ def main():
                     help="stated: independent inputs, down reads h; serial: every projection reads the "
                          "previous one's output (reported as an extra field either way)")
     ap.add_argument("--config", default="stack",
-                    choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "chunk", "q4_k_stack",
+                    choices=["stack", "q8_small", "nvfp4_mlp", "mxfp4_mlp", "moe", "moe_prefill", "chunk", "q4_k_stack",
                              "q6_k_stack", "gguf_chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack line; the others print their "
                          "entries alone")
-    ap.add_argument("--small-case", choices=["moe1", "moe8", "mlp1", "mlp4"],
+    ap.add_argument("--small-case", choices=["moe1", "moe8", "mlp1", "mlp4", "moepf512"],
                     help="three launches of one layer's kernel (for ncu captures); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -1040,7 +1121,7 @@ def main():
     if world == 1 and not args.no_configs:
         # The other workloads, each with its own value, roofline, clocks and CPU baseline.
         cfgs = {}
-        for fn in (cfg_q8_small, cfg_mlp, cfg_moe, cfg_chunk):
+        for fn in (cfg_q8_small, cfg_mlp, cfg_moe, cfg_moe_prefill, cfg_chunk):
             try:
                 cfgs.update(fn(args, cpu=not args.no_cpu_baseline))
             except Exception as ex:  # keep the headline line; record what failed

@@ -102,6 +102,7 @@ struct ChunkArgs {
     // expert tile_expert[tm], the first *used_tm row tiles are in use (written by an earlier kernel
     // of the stream), and expert e's packed weights (header included) start at w + e * w_stride.
     const int* tile_expert;
+    const int* tile_rows;  // rows of tile tm that hold data (the epilogue stores no others)
     const int* used_tm;
     int64_t w_stride;
     // SiLU-gate epilogue (h != nullptr; weights packed with QLIN_PACK_GATE_UP, so accumulator columns
@@ -109,13 +110,24 @@ struct ChunkArgs {
     // bf16(silu(g) * u) for i < h_cols, row pitch ldh; y is not written.
     __nv_bfloat16* h;
     int64_t ldh, h_cols;
+    // Grouped mode: aq already holds the quantized operand (written by an earlier kernel of the
+    // stream); amax_in: the max |x| it was quantized with (the bits of a non-negative float; NVFP4's
+    // a_g follows from it).  amax_out != nullptr (SiLU-gate epilogue): max |h| over the stored bf16
+    // values is folded in with atomicMax.
+    const unsigned* amax_in;
+    unsigned* amax_out;
 };
 
-// silu(z) = z * sigmoid(z), the exponential taken of -|z| only.
+// silu(z) = z * sigmoid(z) with e = exp(-|z|) = 2^(-|z| log2 e) from the MUFU ex2 unit and the
+// reciprocal from the MUFU rcp unit (each within about 2^-22 relative; the rounding of the argument
+// adds |z| 2^-23 relative to e; subnormal e flushes to 0).  The result is rounded to bf16 (2^-9
+// relative) right after, so the approximations cost nothing visible while taking the epilogue from
+// ~25 instructions per output (IEEE exp and division) to ~6.
 __device__ __forceinline__ float chunk_silu(float z) {
-    const float e = expf(-fabsf(z));
-    const float sig = z >= 0.f ? 1.0f / (1.0f + e) : e / (1.0f + e);
-    return z * sig;
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-fabsf(z) * 1.44269504088896341f));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+    return z * (z >= 0.f ? r : e * r);
 }
 
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
@@ -347,7 +359,9 @@ __device__ __forceinline__ void tmem_free(uint32_t tmem) {
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-template <int CG, bool MX>
+// GR: grouped mode (the MoE prefill; CG = 1): pre-quantized activations, per-tile expert weights,
+// the optional SiLU-gate epilogue.  The plain chunk GEMM (GR = false) carries none of that code.
+template <int CG, bool MX, bool GR>
 __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const ChunkArgs a,
                                                                        const __grid_constant__ CUtensorMap ymap) {
     using Cfg = ChunkCfg<CG, MX>;
@@ -393,7 +407,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     if constexpr (CG == 2) cluster_sync_all();  // the pair's barriers exist before either CTA signals the other
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int TMA = a.tile_expert ? *a.used_tm : a.TM;  // activation row tiles in use
+    const int TMA = GR ? *a.used_tm : a.TM;  // activation row tiles in use
     const int TMP = TMA / CG;  // activation tiles of 128 * CG rows
     const int ntiles = a.T2 * TMP * a.KS;
     const int tile0 = blockIdx.x / CG, tstep = gridDim.x / CG;
@@ -409,7 +423,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     };
     // Packed weights of the expert of row tile tm (grouped mode), else of the one matrix.
     auto wbase = [&](int tm) -> const uint8_t* {
-        return a.tile_expert ? a.w + (int64_t)a.tile_expert[tm] * a.w_stride : a.w;
+        if constexpr (GR)
+            return a.w + (int64_t)a.tile_expert[tm] * a.w_stride;
+        else
+            return a.w;
     };
     // The weights do not depend on x: the producer starts the first stages' weight copies now, so
     // they land during phase Q (the stage barriers also expect the activation bytes, copied once
@@ -448,7 +465,12 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
     // (i % kUnitItems) / 16 of the unit's 128 and 16-value block i % 16 of its k-group.  When every
     // thread has at most kQItems items, they stay in registers between the max pass and the
     // quantization (x is read once, all loads in flight together); otherwise x is read twice.
-    {
+    // Grouped mode: the operand was quantized by an earlier kernel; only a_g is taken here.
+    if constexpr (GR) {
+        if (threadIdx.x == 0) *ag_sm = MX ? 1.0f : act_global_scale(__uint_as_float(__ldcg(a.amax_in)));
+        __syncthreads();
+        griddep_launch_dependents();
+    } else {
         const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
         const int64_t gthreads = (int64_t)gridDim.x * blockDim.x;
         const int64_t items = (int64_t)TMA * a.G * kUnitItems;
@@ -479,8 +501,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                 m = fmaxf(m, bmax[j]);
             }
         } else {
-            // (grouped: only the row tiles in use; the rows past them hold no data of this call)
-            m = act_amax_partial(a.x, a.tile_expert ? TMA * kMmaARows : a.M, a.K, a.ldx, vec, gtid, gthreads);
+            m = act_amax_partial(a.x, a.M, a.K, a.ldx, vec, gtid, gthreads);
         }
         if (a.KS > 1) {  // the k-split halves add into y: zero it (ordered before them by the barrier)
             const int64_t nq = (a.N + 3) / 4;
@@ -587,7 +608,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             for (int tile = tile0; tile < ntiles && !*abort_flag; tile += tstep) {
                 int t2, tm, g0, g1;
                 tile_of(tile, t2, tm, g0, g1);
-                {  // every unit of this tile's activation rows and k-groups quantized (bounded wait)
+                if constexpr (!GR) {  // every unit of this tile's activation rows and k-groups quantized (bounded wait)
                     const unsigned* rd = a.ready + (int64_t)tm * a.G;
                     const uint64_t t0 = globaltimer_ns(), budget = ws_wait_budget_ns(a.status);
                     bool ready = false;
@@ -773,20 +794,24 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         const bool add = a.KS > 1;  // k-split: add this half into y (zeroed in phase Q)
         if (add && lane == 0) fence_proxy_async_global();  // the zeroing stores before the TMA adds
         int tcount = 0, nstore = 0;
+        float hmax = 0.f;  // max |h| over this thread's stored values (amax_out)
         for (int tile = tile0; tile < ntiles; tile += tstep, ++tcount) {
+            int t2, tm, g0, g1;
+            tile_of(tile, t2, tm, g0, g1);
+            // grouped: this tile's expert's per-tensor scale and its rows holding data, loaded while
+            // its MMAs run
+            const float ws_g = GR ? reinterpret_cast<const PackedHeader*>(wbase(tm))->global_scale : 0.f;
+            const int mlim = GR ? tm * kMmaARows + a.tile_rows[tm] : a.M;  // rows past it: not stored
             if (*abort_flag || !mbar_wait_bounded(acc_full, tcount & 1)) {
                 if (lane == 0) atomicOr(a.status, 1u);
                 *abort_flag = 1;
                 break;
             }
             tc_fence_after();
-            int t2, tm, g0, g1;
-            tile_of(tile, t2, tm, g0, g1);
             const int m0 = tm * kMmaARows + q * 32;  // this warp's first row
             const int64_t n0 = (int64_t)t2 * kMmaWRows;
-            if (a.tile_expert)  // this tile's expert's per-tensor scale
-                gw_ag = __fmul_rn(reinterpret_cast<const PackedHeader*>(wbase(tm))->global_scale, *ag_sm);
-            if (a.h) {
+            if (GR) gw_ag = __fmul_rn(ws_g, *ag_sm);
+            if (GR && a.h) {
                 // SiLU-gate epilogue: columns c (gate) and c + 128 (up) of output 128 t2 + c; this
                 // thread's row m0 + lane; 32 outputs of one row per step, stored as bf16.
                 const int row = m0 + lane;
@@ -801,7 +826,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                         if (lane == 0) mbar_arrive(acc_empty);
                     }
                     const int64_t i0 = (int64_t)t2 * 128 + c;
-                    if (row >= a.M || i0 >= a.h_cols) continue;
+                    if (row >= mlim || i0 >= a.h_cols) continue;
                     __nv_bfloat16* dst = a.h + (int64_t)row * a.ldh + i0;
                     uint32_t pk[16];
 #pragma unroll
@@ -810,6 +835,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                         const float h1 = chunk_silu(g[2 * j + 1] * gw_ag) * (u[2 * j + 1] * gw_ag);
                         const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
                         pk[j] = *reinterpret_cast<const uint32_t*>(&hb);
+                        hmax = fmaxf(hmax, fmaxf(fabsf(__uint_as_float(pk[j] << 16)),
+                                                 fabsf(__uint_as_float(pk[j] & 0xffff0000u))));
                     }
                     if (i0 + 32 <= a.h_cols && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
 #pragma unroll
@@ -836,13 +863,13 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                             mbar_arrive_cluster(acc_empty, 0);
                     }
                 }
-                if (m0 >= a.M || n0 + c >= a.N) continue;
+                if (m0 >= mlim || n0 + c >= a.N) continue;
                 if (tma) {
                     // rows hh*R .. hh*R+R-1 of the warp's 32 as one R x 32 box; row r's 16-byte chunk j
                     // at position j ^ (r % 8) (the 128B swizzle of the tensor map)
 #pragma unroll
                     for (int hh = 0; hh < 32 / R; ++hh) {
-                        if (m0 + hh * R >= a.M) break;
+                        if (m0 + hh * R >= mlim) break;
                         if (lane == 0 && nstore > 0) bulk_wait_read_all();  // the previous store has read the box
                         __syncwarp();
                         if (lane / R == hh) {
@@ -881,7 +908,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
                         const float4 val = *reinterpret_cast<const float4*>(tb + r * 64 + ((ch ^ (r & 3)) << 4));
                         const int mrow = m0 + r;
                         const int64_t ncol = n0 + c + 16 * h + 4 * ch;
-                        if (mrow < a.M && ncol < a.N) {
+                        if (mrow < mlim && ncol < a.N) {
                             float* dst = a.y + (int64_t)mrow * a.ldy + ncol;
                             if (add) {
                                 const float e[4] = {val.x, val.y, val.z, val.w};
@@ -899,6 +926,10 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
             }
         }
         if (tma && lane == 0) bulk_wait_all();
+        if (GR && a.amax_out) {  // (fmaxf skips a NaN, as the quantizer's own max pass does)
+            for (int o = 16; o; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+            if (lane == 0) atomicMax(a.amax_out, __float_as_uint(hmax));
+        }
         __syncwarp();
     }
     __syncthreads();
@@ -990,12 +1021,13 @@ static bool make_y_map(CUtensorMap* map, float* y, int M, int64_t N, int64_t ldy
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int CG, bool MX>
+template <int CG, bool MX, bool GR>
 static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     static bool attr_set = false;
     cudaError_t e;
     if (!attr_set) {
-        e = cudaFuncSetAttribute(chunk_gemm_kernel<CG, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, chunk_smem<CG>());
+        e = cudaFuncSetAttribute(chunk_gemm_kernel<CG, MX, GR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 chunk_smem<CG>());
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -1025,7 +1057,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gemm_kernel<CG, MX>, kChunkThreads,
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gemm_kernel<CG, MX, GR>, kChunkThreads,
                                                           chunk_smem<CG>());
         if (e != cudaSuccess) return e;
         if (per_sm < 1) return cudaErrorInvalidConfiguration;
@@ -1034,7 +1066,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
             cfg.gridDim = dim3((unsigned)(sms & ~1));
             cfg.numAttrs = na;
             int clusters = 0;
-            e = cudaOccupancyMaxActiveClusters(&clusters, chunk_gemm_kernel<CG, MX>, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&clusters, chunk_gemm_kernel<CG, MX, GR>, &cfg);
             if (e != cudaSuccess) return e;
             if (clusters < 1) return cudaErrorInvalidConfiguration;
             units = clusters;
@@ -1044,7 +1076,7 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     }
     // Too few output tiles to give every CTA one: split each tile's k-groups in two halves.
     const int base_tiles = a.T2 * (a.TM / CG);
-    a.KS = (CG == 1 && !a.tile_expert && a.G >= 2 && 2 * base_tiles <= max_units) ? 2 : 1;
+    a.KS = (CG == 1 && !GR && a.G >= 2 && 2 * base_tiles <= max_units) ? 2 : 1;
     a.GS = (a.G + a.KS - 1) / a.KS;
     const int ntiles = base_tiles * a.KS;
     const int units = ntiles < max_units ? ntiles : max_units;
@@ -1058,13 +1090,14 @@ static cudaError_t launch_chunk_cg(ChunkArgs a, int flags, cudaStream_t s) {
     CUtensorMap ymap;
     memset(&ymap, 0, sizeof(ymap));
     a.tma_store = (!a.h && a.y && make_y_map(&ymap, a.y, a.M, a.N, a.ldy, EpiCfg<CG>::kBoxRows)) ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel<CG, MX>, a, ymap);
+    return cudaLaunchKernelEx(&cfg, chunk_gemm_kernel<CG, MX, GR>, a, ymap);
 }
 
 extern "C" cudaError_t qlin_launch_chunk(int fmt, const void* packed, int64_t N, int64_t K, const void* x, int M,
                                          int64_t ldx, float* y, int64_t ldy, void* ws, int flags, cudaStream_t s) {
     uint8_t* w8 = (uint8_t*)ws;
     ChunkArgs a;
+    memset(&a, 0, sizeof(a));  // (grouped-mode fields off)
     a.w = (const uint8_t*)packed;
     a.x = (const __nv_bfloat16*)x;
     a.ldx = ldx;
@@ -1091,8 +1124,10 @@ extern "C" cudaError_t qlin_launch_chunk(int fmt, const void* packed, int64_t N,
     a.h = nullptr;
     a.ldh = a.h_cols = 0;
     if (fmt == QLIN_MXFP4)
-        return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, true>(a, flags, s) : launch_chunk_cg<1, true>(a, flags, s);
-    return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, false>(a, flags, s) : launch_chunk_cg<1, false>(a, flags, s);
+        return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, true, false>(a, flags, s)
+                                       : launch_chunk_cg<1, true, false>(a, flags, s);
+    return chunk_cg(M, flags) == 2 ? launch_chunk_cg<2, false, false>(a, flags, s)
+                                   : launch_chunk_cg<1, false, false>(a, flags, s);
 }
 
 extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t K, int64_t ldx, void* ws,
@@ -1104,21 +1139,23 @@ extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t
     return cudaMemcpyAsync(ag, words + 2, 4, cudaMemcpyDeviceToDevice, s);
 }
 
-// Grouped launch (the MoE prefill): x = the expert-sorted bf16 activations (rows_max rows with
-// K % 8 == 0 values each, the first *used_tm * 128 rows in use), w = E packed weight buffers
-// w_stride bytes apart, T2 weight tiles per expert.  h != nullptr: the SiLU-gate epilogue (weights
-// packed QLIN_PACK_MMA | QLIN_PACK_GATE_UP) writing h_cols bf16 outputs per row; else y (fp32, N
-// columns).  Single CTAs, no k-split, no programmatic dependent launch (the routing kernel before it
-// writes the tile table this launch reads at its start).
+// Grouped launch (the MoE prefill): the activations are expert-sorted rows (rows_max at most, the
+// first *used_tm * 128 in use, each expert's rows padded to whole 128-row tiles), already quantized
+// into the workspace's operand units by an earlier kernel of the stream, with max |x| = *amax_in;
+// w = E packed weight buffers w_stride bytes apart, T2 weight tiles per expert, row tile tm against
+// expert tile_expert[tm].  h != nullptr: the SiLU-gate epilogue (weights packed QLIN_PACK_MMA |
+// QLIN_PACK_GATE_UP) writing h_cols bf16 outputs per row and folding max |h| into *amax_out; else
+// y (fp32, N columns).  Either way rows past tile_rows[tm] of tile tm are not stored.  Single CTAs,
+// no k-split, no programmatic dependent launch.
 extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t w_stride, int T2, int64_t N,
-                                                 int64_t K, const void* x, int rows_max, float* y, int64_t ldy,
-                                                 void* h, int64_t ldh, int64_t h_cols, const int* tile_expert,
-                                                 const int* used_tm, void* ws, cudaStream_t s) {
+                                                 int64_t K, int rows_max, float* y, int64_t ldy, void* h,
+                                                 int64_t ldh, int64_t h_cols, const int* tile_expert,
+                                                 const int* tile_rows, const int* used_tm, const unsigned* amax_in,
+                                                 unsigned* amax_out, void* ws, cudaStream_t s) {
     uint8_t* w8 = (uint8_t*)ws;
     ChunkArgs a;
     memset(&a, 0, sizeof(a));
     a.w = (const uint8_t*)w;
-    a.x = (const __nv_bfloat16*)x;
     a.ldx = K;
     a.aq = w8 + 256;
     a.words = (unsigned*)(w8 + 64);
@@ -1132,16 +1169,18 @@ extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t
     a.T2 = T2;
     a.G = (int)((K + kGroupK - 1) / kGroupK);
     a.TM = (int)chunk_units_m(rows_max, 0);
-    a.xvec = ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && K % 8 == 0) ? 1 : 0;
     a.yvec = (y && (reinterpret_cast<uintptr_t>(y) & 15) == 0 && ldy % 4 == 0) ? 1 : 0;
     a.KS = 1;
     a.GS = a.G;
     a.status = (unsigned*)ws;
     a.tile_expert = tile_expert;
+    a.tile_rows = tile_rows;
     a.used_tm = used_tm;
     a.w_stride = w_stride;
     a.h = (__nv_bfloat16*)h;
     a.ldh = ldh;
     a.h_cols = h_cols;
-    return fmt == QLIN_MXFP4 ? launch_chunk_cg<1, true>(a, 0, s) : launch_chunk_cg<1, false>(a, 0, s);
+    a.amax_in = amax_in;
+    a.amax_out = amax_out;
+    return fmt == QLIN_MXFP4 ? launch_chunk_cg<1, true, true>(a, 0, s) : launch_chunk_cg<1, false, true>(a, 0, s);
 }

@@ -5,27 +5,37 @@
 // o = W_down[e] h; y[m] = sum over slots, in slot order, of weight * o), with NVFP4 / MXFP4 expert
 // weights and the chunk path's activation quantization.  The pages' counterpart: imp's MoE "top-k
 // grouped GEMM" and its NVFP4 grouped GEMM for MoE prefill (imp README, "Features" table, row
-// "Architectures"; release notes v0.7.0), there on sm_120a.  Five launches on one stream, no host
+// "Architectures"; release notes v0.7.0), there on sm_120a.  Six launches on one stream, no host
 // synchronisation (the counts and the tile table live on the device, so the sequence can be
 // captured in a CUDA graph):
-//   1. route + counting sort (one CTA): top_k per token (ties to the lower expert index, a NaN logit
-//      ranks as -inf), renormalised weights, then the (token, slot) entries sorted by expert --
-//      tokens ascending within an expert, each expert's rows padded to whole 128-row tiles -- and
-//      the table row tile -> expert;
-//   2. gather: x rows into the sorted bf16 matrix (padding rows zero);
-//   3. grouped chunk GEMM, gate_up: the sorted rows quantized as the chunk path quantizes (NVFP4:
-//      one per-tensor scale over them; MXFP4: the OCP MX rule), each 128-row tile against its
-//      expert's gate/up-interleaved weights, the SiLU-gate fused in the epilogue, h stored as bf16;
-//   4. grouped chunk GEMM, down: h quantized the same way (NVFP4: its own per-tensor scale), each
-//      tile against its expert's down weights, o (fp32) per sorted row;
-//   5. combine: y[m] = sum over slots, in slot order, of weight * o[row of (m, slot)] (deterministic),
-//      the optional h output, and the two GEMMs' status words folded into the caller's.
+//   1. route (a warp per token): top_k (ties to the lower expert index, a NaN logit ranks as
+//      -inf), renormalised weights, max |x| of the token folded into one word, and for each valid
+//      slot its index among the expert's entries (an atomic counter per expert); the last CTA to
+//      finish turns the counts into each expert's first sorted row (rows padded to whole 128-row
+//      tiles) and the table row tile -> expert;
+//   2. gather-quantize (a CTA per token): the token's row quantized once as the chunk path
+//      quantizes (NVFP4: one per-tensor scale from max |x| over the chunk; MXFP4: the OCP MX rule)
+//      and stored, in the tensor-core operand layout, at each of its sorted rows; extra CTAs zero
+//      each expert's padding rows;
+//   3. grouped chunk GEMM, gate_up: each 128-row tile against its expert's gate/up-interleaved
+//      weights, the SiLU-gate fused in the epilogue, h stored as bf16 (padding rows not stored) and
+//      max |h| folded into a word;
+//   4. h quantized the same way (NVFP4: its own per-tensor scale, from that word), a thread per
+//      16-value item;
+//   5. grouped chunk GEMM, down: each tile against its expert's down weights, o (fp32) per sorted row
+//      (padding rows not stored);
+//   6. combine: y[m] = sum over slots, in slot order, of weight * o[row of (m, slot)] (deterministic),
+//      the optional h output, the two GEMMs' status words folded into the caller's.
+// Which sorted row an entry takes depends on the order of the atomic counter, but every row is
+// computed on its own (the MMA rows are independent and the per-tensor scales are maxima), so the
+// results do not: y, h, ids and weights are the same from run to run.
 #include "chunk_common.cuh"
 
 extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t w_stride, int T2, int64_t N,
-                                                 int64_t K, const void* x, int rows_max, float* y, int64_t ldy,
-                                                 void* h, int64_t ldh, int64_t h_cols, const int* tile_expert,
-                                                 const int* used_tm, void* ws, cudaStream_t s);
+                                                 int64_t K, int rows_max, float* y, int64_t ldy, void* h,
+                                                 int64_t ldh, int64_t h_cols, const int* tile_expert,
+                                                 const int* tile_rows, const int* used_tm, const unsigned* amax_in,
+                                                 unsigned* amax_out, void* ws, cudaStream_t s);
 extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K);
 extern "C" int64_t qlin_mma_tiles(int64_t N, int gate_up);
 
@@ -33,7 +43,9 @@ namespace qlin {
 
 constexpr int kPfMaxTopK = 8;
 constexpr int kPfMaxE = 256;
-constexpr int kPfThreads = 1024;
+constexpr int kPfRouteWarps = 8;  // tokens per route CTA
+constexpr int kPfGatherThreads = 128;
+constexpr int kPfPadCtas = 4;  // CTAs zeroing one expert's padding rows
 
 static inline int64_t pf_al256(int64_t v) { return (v + 255) / 256 * 256; }
 
@@ -43,9 +55,11 @@ static inline int pf_rows_max(int M, int E, int top_k) {
     return (int)((r + 127) / 128 * 128);
 }
 
-// Workspace layout (offsets in bytes).
+// Workspace layout (offsets in bytes).  [0, 256): the status word (and the wait budget word).
+// rt: cnt[256] at 0, fill[256] at 1024, off[257] at 2048, words at 3328: [0] ticket, [1] max |x|,
+// [2] max |h|, [3] row tiles in use.
 struct PfLayout {
-    int64_t pos, tile_expert, used_tm, row_token, xs, ws_a, hs, ws_b, os, total;
+    int64_t lpos, pos, rt, tile_expert, ws_a, hs, ws_b, os, total;
     int rows_max;
 };
 
@@ -53,17 +67,15 @@ static PfLayout pf_layout(int M, int64_t H, int64_t I, int E, int top_k) {
     PfLayout L;
     L.rows_max = pf_rows_max(M, E, top_k);
     const int64_t R = L.rows_max, TMx = R / 128;
-    int64_t o = 256;  // [0, 256): the status word
+    int64_t o = 256;
+    L.lpos = o;
+    o += pf_al256(4 * (int64_t)M * top_k);
     L.pos = o;
     o += pf_al256(4 * (int64_t)M * top_k);
-    L.tile_expert = o;
-    o += pf_al256(4 * TMx);
-    L.used_tm = o;
-    o += 256;
-    L.row_token = o;
-    o += pf_al256(4 * R);
-    L.xs = o;
-    o += pf_al256(2 * R * H);
+    L.rt = o;
+    o += 4096;
+    L.tile_expert = o;  // then tile_rows
+    o += pf_al256(8 * TMx);
     L.ws_a = o;
     o += pf_al256((int64_t)qlin_chunk_ws_bytes((int)R, 2 * I, H));
     L.hs = o;
@@ -80,11 +92,17 @@ struct PfArgs {
     const float* logits;  // M x E, or nullptr (ids / weights given)
     int32_t* ids;         // M x top_k
     float* wts;           // M x top_k
+    const __nv_bfloat16* x;  // M x H
+    int64_t H;
     int M, E, top_k, TMx;
+    int* lpos;            // M x top_k: index of (token, slot) among its expert's entries, -1 skipped
     int* pos;             // M x top_k: sorted row of (token, slot), -1 for a skipped slot
+    int* cnt;             // E: entries per expert (counted in step 1, cleared by its last CTA)
+    int* fill;            // E: the counts, kept for steps 2 and 5
+    int* off;             // E + 1: first sorted row of each expert
+    unsigned* words;      // [0] ticket, [1] max |x|, [2] max |h|, [3] row tiles in use
     int* tile_expert;     // TMx
-    int* used_tm;
-    int* row_token;       // rows_max: token of a sorted row, -1 for padding
+    int* tile_rows;       // TMx: rows of the tile that hold entries (the rest is padding)
     unsigned* status;     // bit 1: an invalid or repeated given expert id (the slot is skipped)
 };
 
@@ -94,140 +112,288 @@ __device__ __forceinline__ bool pf_before(float a, int ia, float b, int ib) {
     return fa > fb || (fa == fb && ia < ib);
 }
 
-__global__ void __launch_bounds__(kPfThreads) moe_prefill_route_kernel(const PfArgs a) {
-    __shared__ int cnt[kPfMaxE];
-    __shared__ int off[kPfMaxE + 1];
-    __shared__ int warp_sum[kPfThreads / 32];
-    __shared__ int chunk_base;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int k = a.top_k;
-    for (int e = tid; e < a.E; e += blockDim.x) cnt[e] = 0;
-    __syncthreads();
-    // 1. routing (or validation of the given ids), and the per-expert counts
-    for (int m = tid; m < a.M; m += blockDim.x) {
+__global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(const PfArgs a) {
+    __shared__ int s_off[kPfMaxE + 1];
+    __shared__ int s_last;
+    const int lane = threadIdx.x & 31, k = a.top_k;
+    const int m = blockIdx.x * kPfRouteWarps + (threadIdx.x >> 5);
+    if (m < a.M) {
+        // max |x| of the token (fmaxf skips a NaN, as the chunk quantizer's max pass does)
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.H);
+        float mx = 0.f;
+#pragma unroll 8
+        for (int64_t v = lane; v < a.H / 8; v += 32) {
+            const uint4 q = __ldg(xr + v);
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[j] << 16)), fabsf(__uint_as_float(w[j] & 0xffff0000u))));
+        }
+        for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) atomicMax(&a.words[1], __float_as_uint(mx));  // non-negative floats order as their bits
+
         int32_t* id = a.ids + (int64_t)m * k;
+        int sel[kPfMaxTopK];
+#pragma unroll
+        for (int r = 0; r < kPfMaxTopK; ++r) sel[r] = -1;
         if (a.logits) {
+            // top_k rounds of a warp-wide argmax under pf_before; lane l holds experts l, l + 32, ...
             const float* l = a.logits + (int64_t)m * a.E;
-            int sel[kPfMaxTopK];
-            for (int e = 0; e < a.E; ++e) {
-                int r = 0;
-                const float le = l[e];
-                for (int e2 = 0; e2 < a.E && r < k; ++e2) r += pf_before(l[e2], e2, le, e) ? 1 : 0;
-                if (r < k) sel[r] = e;
+            float v[kPfMaxE / 32];
+#pragma unroll
+            for (int j = 0; j < kPfMaxE / 32; ++j) {
+                const int e = lane + 32 * j;
+                v[j] = e < a.E ? l[e] : -INFINITY;
             }
-            const float lmax = l[sel[0]] != l[sel[0]] ? 0.f : l[sel[0]];
+            unsigned taken = 0u;
+#pragma unroll
+            for (int r = 0; r < kPfMaxTopK; ++r) {
+                if (r >= k) break;
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+#pragma unroll
+                for (int j = 0; j < kPfMaxE / 32; ++j) {
+                    const int e = lane + 32 * j;
+                    if (e < a.E && !((taken >> j) & 1u) && pf_before(v[j], e, bv, bi)) {
+                        bv = v[j];
+                        bi = e;
+                    }
+                }
+                for (int o = 16; o; o >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                    if (pf_before(ov, oi, bv, bi)) {
+                        bv = ov;
+                        bi = oi;
+                    }
+                }
+                sel[r] = bi;
+                if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            }
+            // weights: softmax over the selected logits (the largest first), fp32
+            const float l0 = l[sel[0]];
+            const float lmax = l0 != l0 ? 0.f : l0;
             float ex[kPfMaxTopK], sum = 0.f;
-            for (int r = 0; r < k; ++r) {
+#pragma unroll
+            for (int r = 0; r < kPfMaxTopK; ++r) {
+                if (r >= k) break;
                 ex[r] = expf(l[sel[r]] - lmax);
                 sum += ex[r];
             }
-            for (int r = 0; r < k; ++r) {
-                id[r] = sel[r];
-                a.wts[(int64_t)m * k + r] = ex[r] / sum;
-            }
-        }
-        for (int r = 0; r < k; ++r) {
-            const int e = id[r];
-            bool ok = e >= 0 && e < a.E;
-            for (int r2 = 0; r2 < r && ok; ++r2) ok = id[r2] != e;
-            if (ok) atomicAdd(&cnt[e], 1);
-            else atomicOr(a.status, 2u);
-        }
-    }
-    __syncthreads();
-    // 2. offsets: each expert's rows padded to whole 128-row tiles; the tile table
-    if (tid == 0) {
-        int run = 0;
-        for (int e = 0; e < a.E; ++e) {
-            off[e] = run;
-            run += (cnt[e] + 127) / 128 * 128;
-        }
-        off[a.E] = run;
-        *a.used_tm = run / 128;
-    }
-    __syncthreads();
-    for (int e = 0; e < a.E; ++e)
-        for (int t = off[e] / 128 + tid; t < off[e + 1] / 128; t += blockDim.x) a.tile_expert[t] = e;
-    for (int t = off[a.E] / 128 + tid; t < a.TMx; t += blockDim.x) a.tile_expert[t] = -1;
-    for (int r = tid; r < a.TMx * 128; r += blockDim.x) a.row_token[r] = -1;
-    for (int i = tid; i < a.M * k; i += blockDim.x) a.pos[i] = -1;
-    __syncthreads();
-    // 3. sorted rows: the entry (m, slot) of expert e goes to off[e] + #{m' < m routed to e}
-    for (int e = 0; e < a.E; ++e) {
-        if (cnt[e] == 0) continue;  // (uniform: every thread reads the same shared count)
-        if (tid == 0) chunk_base = 0;
-        __syncthreads();
-        for (int m0 = 0; m0 < a.M; m0 += blockDim.x) {
-            const int m = m0 + tid;
-            int slot = -1;
-            if (m < a.M) {
-                const int32_t* id = a.ids + (int64_t)m * k;
-                for (int r = 0; r < k; ++r) {
-                    bool ok = id[r] == e;
-                    for (int r2 = 0; r2 < r && ok; ++r2) ok = id[r2] != e;  // a repeated id counts once
-                    if (ok) slot = r;
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < kPfMaxTopK; ++r) {
+                    if (r >= k) break;
+                    id[r] = sel[r];
+                    a.wts[(int64_t)m * k + r] = ex[r] / sum;
                 }
             }
-            const unsigned bal = __ballot_sync(0xffffffffu, slot >= 0);
-            if (lane == 0) warp_sum[wid] = __popc(bal);
-            __syncthreads();
-            int before = chunk_base;
-            for (int w = 0; w < wid; ++w) before += warp_sum[w];
-            before += __popc(bal & ((1u << lane) - 1u));
-            if (slot >= 0) {
-                const int row = off[e] + before;
-                a.pos[(int64_t)m * k + slot] = row;
-                a.row_token[row] = m;
+        } else {
+#pragma unroll
+            for (int r = 0; r < kPfMaxTopK; ++r)
+                if (r < k) sel[r] = id[r];
+        }
+        // each valid slot's index among its expert's entries (lane r takes slot r)
+        if (lane < k) {
+            int e = sel[0];
+            bool ok = true;
+#pragma unroll
+            for (int r = 1; r < kPfMaxTopK; ++r)
+                if (r == lane) e = sel[r];
+#pragma unroll
+            for (int r2 = 0; r2 < kPfMaxTopK; ++r2)
+                if (r2 < lane && sel[r2] == e) ok = false;  // a repeated id counts once
+            ok = ok && e >= 0 && e < a.E;
+            if (ok) {
+                a.lpos[(int64_t)m * k + lane] = atomicAdd(&a.cnt[e], 1);
+            } else {
+                a.lpos[(int64_t)m * k + lane] = -1;
+                atomicOr(a.status, 2u);
             }
-            __syncthreads();
-            if (tid == 0) {
-                int tot = 0;
-                for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += warp_sum[w];
-                chunk_base += tot;
+        }
+    }
+    // The last CTA to finish: first sorted row of each expert, the tile table, and the counters
+    // cleared for the next call.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(&a.words[0], 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {  // the counts, read once and cleared
+        const int c = __ldcg(&a.cnt[e]);
+        s_off[e] = c;
+        a.fill[e] = c;
+        a.cnt[e] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int e = 0; e < a.E; ++e) {
+            const int c = s_off[e];
+            s_off[e] = run;
+            run += (c + 127) / 128 * 128;
+        }
+        s_off[a.E] = run;
+        a.words[3] = (unsigned)(run / 128);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.off[e] = s_off[e];
+    for (int t = threadIdx.x; t < a.TMx; t += blockDim.x) {
+        int ex = -1;
+        for (int e = 0; e < a.E && ex < 0; ++e)
+            if (s_off[e] <= 128 * t && 128 * t < s_off[e + 1]) ex = e;
+        a.tile_expert[t] = ex;
+        const int live = ex < 0 ? 0 : s_off[ex] + a.fill[ex] - 128 * t;
+        a.tile_rows[t] = live < 0 ? 0 : (live > 128 ? 128 : live);
+    }
+    if (threadIdx.x == 0) {
+        a.words[0] = 0u;  // the ticket
+        a.words[2] = 0u;  // max |h|, accumulated by the gate_up GEMM that follows
+    }
+}
+
+// Blocks [0, M): token m's row quantized once (item = 16 values; NVFP4 with a_g from max |x|, MXFP4
+// by the pair rule) and stored at each of its sorted rows, in the operand units of the gate_up
+// GEMM's workspace (G k-groups of 256 values per 128-row tile; values past H are zeros); the
+// sorted row of each (m, slot) recorded.  Blocks [M, M + kPfPadCtas E): expert e's padding rows
+// zeroed, per row and k-group its 8 16-byte code chunks and its 4 (MXFP4: 2) scale words.
+template <bool MX>
+__global__ void __launch_bounds__(kPfGatherThreads) moe_prefill_gather_quant_kernel(const PfArgs a, int64_t G,
+                                                                                  uint8_t* __restrict__ aq) {
+    const int b = blockIdx.x, k = a.top_k;
+    const int64_t nitems = G * 16;
+    if (b < a.M) {
+        const int m = b;
+        int rows[kPfMaxTopK];
+#pragma unroll
+        for (int r = 0; r < kPfMaxTopK; ++r) {
+            rows[r] = -1;
+            if (r < k) {
+                const int li = a.lpos[(int64_t)m * k + r];
+                if (li >= 0) rows[r] = a.off[a.ids[(int64_t)m * k + r]] + li;
+                if (threadIdx.x == 0) a.pos[(int64_t)m * k + r] = rows[r];
             }
-            __syncthreads();
+        }
+        const float ag = MX ? 1.0f : act_global_scale(__uint_as_float(__ldcg(&a.words[1])));
+        // (nitems is even, so the two items of a 32-value block are both live or both not, and the
+        // loop bounds are the same for every lane: the MXFP4 pair shuffles run with the whole warp)
+        for (int64_t i0 = 0; i0 < nitems; i0 += kPfGatherThreads) {
+            const int64_t it = i0 + threadIdx.x;
+            const bool live = it < nitems;
+            uint32_t w[8], c8[2];
+            act_load_item(a.x, live ? a.M : 0, a.H, a.H, true, m, live ? it : 0, w);
+            uint8_t sc;
+            if constexpr (MX) {
+                sc = act_mx_pair_byte(act_item_amax(w), act_item_special(w));
+                act_quant_item_mx_codes(w, sc, c8);
+            } else {
+                sc = act_quant_block(w, act_item_amax(w), ag, c8);
+            }
+            if (!live) continue;
+#pragma unroll
+            for (int r = 0; r < kPfMaxTopK; ++r) {
+                if (r >= k || rows[r] < 0) continue;
+                if constexpr (MX)
+                    act_store_item_mx(0, a.H, G, rows[r], it, sc, c8, aq, nullptr, nullptr);
+                else
+                    act_store_item(0, a.H, G, rows[r], it, sc, c8, aq, nullptr, nullptr);
+            }
+        }
+    } else {
+        const int e = (b - a.M) / kPfPadCtas, part = (b - a.M) % kPfPadCtas;
+        const int r0 = a.off[e] + a.fill[e], npad = a.off[e + 1] - r0;  // < 128 rows, one tile
+        const int per_row = (int)G * 12;
+        for (int i = part * kPfGatherThreads + threadIdx.x; i < npad * per_row; i += kPfPadCtas * kPfGatherThreads) {
+            const int rr = i / per_row, rem = i - rr * per_row;
+            const int g = rem / 12, piece = rem - g * 12;
+            const int row = r0 + rr, r = row & (kMmaARows - 1);
+            uint8_t* ub = aq + ((int64_t)(row / kMmaARows) * G + g) * kMmaAUnit;
+            if (piece < 8)
+                *reinterpret_cast<uint4*>(ub + mma_code_off(r, piece)) = make_uint4(0u, 0u, 0u, 0u);
+            else if (!MX || piece < 10)
+                *reinterpret_cast<uint32_t*>(ub + kMmaARows * 128 + mma_scale_off(piece - 8, r, 0, 1)) = 0u;
         }
     }
 }
 
-// One CTA per sorted row in use: the token's bf16 activations, or zeros for a padding row.
-__global__ void __launch_bounds__(128) moe_prefill_gather_kernel(const __nv_bfloat16* __restrict__ x, int64_t H,
-                                                                 const int* __restrict__ row_token,
-                                                                 const int* __restrict__ used_tm,
-                                                                 __nv_bfloat16* __restrict__ xs) {
-    const int r = blockIdx.x;
-    if (r >= *used_tm * 128) return;
-    const int t = row_token[r];
-    uint4* dst = reinterpret_cast<uint4*>(xs + (int64_t)r * H);
-    const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(t < 0 ? 0 : t) * H);
-    for (int64_t v = threadIdx.x; v < H / 8; v += blockDim.x) dst[v] = t < 0 ? make_uint4(0, 0, 0, 0) : src[v];
+// h (the sorted rows in use, bf16) quantized for the down GEMM, one thread per 16-value item:
+// NVFP4 with a_g from max |h| (word [2], folded in by the gate_up epilogue), MXFP4 by the pair rule;
+// stored in the down GEMM's operand units (G k-groups per 128-row tile; values past I are zeros).
+// Padding rows (not written by the gate_up epilogue) are not read: their operand rows are zeros.
+// The grid covers every row the workspace can hold; CTAs past the rows in use return at once.
+template <bool MX>
+__global__ void __launch_bounds__(256) moe_prefill_quant_h_kernel(const __nv_bfloat16* __restrict__ hs, int64_t I,
+                                                                  int64_t G, const unsigned* __restrict__ words,
+                                                                  const int* __restrict__ tile_rows,
+                                                                  uint8_t* __restrict__ aq) {
+    const int64_t nitems = G * 16;
+    const int rows = (int)words[3] * kMmaARows;
+    const int64_t used = (int64_t)rows * nitems;
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x;
+    if (first >= used) return;  // (the whole CTA: the pair shuffles below run with every lane)
+    const int64_t i = first + threadIdx.x;
+    const bool live = i < used;
+    const int row = live ? (int)(i / nitems) : 0;
+    const int64_t it = live ? i - (int64_t)row * nitems : 0;
+    const bool data = live && (row % kMmaARows) < tile_rows[row / kMmaARows];
+    uint32_t w[8], c8[2];
+    act_load_item(hs, data ? rows : 0, I, I, true, row, it, w);
+    uint8_t sc;
+    if constexpr (MX) {
+        sc = act_mx_pair_byte(act_item_amax(w), act_item_special(w));
+        act_quant_item_mx_codes(w, sc, c8);
+        if (live) act_store_item_mx(0, I, G, row, it, sc, c8, aq, nullptr, nullptr);
+    } else {
+        sc = act_quant_block(w, act_item_amax(w), act_global_scale(__uint_as_float(__ldcg(&words[2]))), c8);
+        if (live) act_store_item(0, I, G, row, it, sc, c8, aq, nullptr, nullptr);
+    }
 }
 
 // One CTA per token: y[m] = sum over slots in slot order of w * o[row]; the optional h output
-// (fp32 values of the bf16 h of each (token, slot)); the GEMMs' status words folded in.
-__global__ void __launch_bounds__(256) moe_prefill_combine_kernel(const int* __restrict__ pos,
-                                                                  const float* __restrict__ wts, int top_k,
-                                                                  const float* __restrict__ os, int64_t H,
+// (fp32 values of the bf16 h of each (token, slot)); the GEMMs' status words folded in; max |x|
+// cleared for the next call.
+__global__ void __launch_bounds__(256) moe_prefill_combine_kernel(const PfArgs a, const float* __restrict__ os,
                                                                   const __nv_bfloat16* __restrict__ hs, int64_t I,
                                                                   float* __restrict__ y, float* __restrict__ h,
-                                                                  unsigned* status, const unsigned* st_a,
-                                                                  const unsigned* st_b) {
-    const int m = blockIdx.x;
+                                                                  const unsigned* st_a, const unsigned* st_b) {
+    const int m = blockIdx.x, top_k = a.top_k;
+    const int64_t H = a.H;
     if (m == 0 && threadIdx.x == 0) {
         const unsigned s = *st_a | *st_b;
-        if (s) atomicOr(status, s & 1u);
+        if (s) atomicOr(a.status, s & 1u);
+        a.words[1] = 0u;
     }
     int rows[kPfMaxTopK];
     float w[kPfMaxTopK];
-    for (int r = 0; r < top_k; ++r) {
-        rows[r] = pos[(int64_t)m * top_k + r];
-        w[r] = wts[(int64_t)m * top_k + r];
+#pragma unroll
+    for (int r = 0; r < kPfMaxTopK; ++r) {
+        rows[r] = r < top_k ? a.pos[(int64_t)m * top_k + r] : -1;
+        w[r] = r < top_k ? a.wts[(int64_t)m * top_k + r] : 0.f;
     }
-    for (int64_t n = threadIdx.x; n < H; n += blockDim.x) {
-        float sum = 0.f;
-        for (int r = 0; r < top_k; ++r)
-            if (rows[r] >= 0) sum += w[r] * os[(int64_t)rows[r] * H + n];
-        y[(int64_t)m * H + n] = sum;
+    // four columns per thread (H % 32 == 0; the o rows are 16-byte aligned), one fused multiply-add
+    // per slot and column
+    const bool yvec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+    for (int64_t n4 = threadIdx.x; n4 < H / 4; n4 += blockDim.x) {
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kPfMaxTopK; ++r) {
+            if (r < top_k && rows[r] >= 0) {
+                const float4 o = *reinterpret_cast<const float4*>(os + (int64_t)rows[r] * H + 4 * n4);
+                sum.x = __fmaf_rn(w[r], o.x, sum.x);
+                sum.y = __fmaf_rn(w[r], o.y, sum.y);
+                sum.z = __fmaf_rn(w[r], o.z, sum.z);
+                sum.w = __fmaf_rn(w[r], o.w, sum.w);
+            }
+        }
+        float* dst = y + (int64_t)m * H + 4 * n4;
+        if (yvec) {
+            *reinterpret_cast<float4*>(dst) = sum;
+        } else {
+            dst[0] = sum.x, dst[1] = sum.y, dst[2] = sum.z, dst[3] = sum.w;
+        }
     }
     if (h) {
         for (int r = 0; r < top_k; ++r)
@@ -253,34 +419,58 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
                                                size_t dn_stride, cudaStream_t s) {
     const PfLayout L = pf_layout(M, H, I, E, top_k);
     uint8_t* w8 = (uint8_t*)ws;
+    uint8_t* rt = w8 + L.rt;
     PfArgs pa;
     pa.logits = logits;
     pa.ids = ids;
     pa.wts = wts;
+    pa.x = (const __nv_bfloat16*)x;
+    pa.H = H;
     pa.M = M;
     pa.E = E;
     pa.top_k = top_k;
     pa.TMx = L.rows_max / 128;
+    pa.lpos = (int*)(w8 + L.lpos);
     pa.pos = (int*)(w8 + L.pos);
+    pa.cnt = (int*)rt;
+    pa.fill = (int*)(rt + 1024);
+    pa.off = (int*)(rt + 2048);
+    pa.words = (unsigned*)(rt + 3328);
     pa.tile_expert = (int*)(w8 + L.tile_expert);
-    pa.used_tm = (int*)(w8 + L.used_tm);
-    pa.row_token = (int*)(w8 + L.row_token);
+    pa.tile_rows = pa.tile_expert + pa.TMx;
     pa.status = (unsigned*)ws;
-    moe_prefill_route_kernel<<<1, kPfThreads, 0, s>>>(pa);
+    const int* used_tm = (const int*)(pa.words + 3);
+    moe_prefill_route_kernel<<<(M + kPfRouteWarps - 1) / kPfRouteWarps, kPfRouteWarps * 32, 0, s>>>(pa);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    __nv_bfloat16* xs = (__nv_bfloat16*)(w8 + L.xs);
+    const int64_t Gh = (H + kGroupK - 1) / kGroupK;
+    uint8_t* aq = w8 + L.ws_a + 256;  // the gate_up GEMM's operand units (its workspace layout)
+    if (fmt == QLIN_MXFP4)
+        moe_prefill_gather_quant_kernel<true><<<M + kPfPadCtas * E, kPfGatherThreads, 0, s>>>(pa, Gh, aq);
+    else
+        moe_prefill_gather_quant_kernel<false><<<M + kPfPadCtas * E, kPfGatherThreads, 0, s>>>(pa, Gh, aq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     __nv_bfloat16* hs = (__nv_bfloat16*)(w8 + L.hs);
     float* os = (float*)(w8 + L.os);
-    moe_prefill_gather_kernel<<<L.rows_max, 128, 0, s>>>((const __nv_bfloat16*)x, H, pa.row_token, pa.used_tm, xs);
+    e = qlin_launch_chunk_grouped(fmt, gu, (int64_t)gu_stride, (int)qlin_mma_tiles(2 * I, 1), 2 * I, H, L.rows_max,
+                                  nullptr, 0, hs, I, I, pa.tile_expert, pa.tile_rows, used_tm, pa.words + 1,
+                                  pa.words + 2, w8 + L.ws_a, s);
+    if (e != cudaSuccess) return e;
+    const int64_t Gi = (I + kGroupK - 1) / kGroupK;
+    const int64_t hitems = (int64_t)L.rows_max * Gi * 16;
+    uint8_t* aq_b = w8 + L.ws_b + 256;  // the down GEMM's operand units
+    if (fmt == QLIN_MXFP4)
+        moe_prefill_quant_h_kernel<true><<<(unsigned)((hitems + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
+                                                                                          pa.tile_rows, aq_b);
+    else
+        moe_prefill_quant_h_kernel<false><<<(unsigned)((hitems + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
+                                                                                           pa.tile_rows, aq_b);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = qlin_launch_chunk_grouped(fmt, gu, (int64_t)gu_stride, (int)qlin_mma_tiles(2 * I, 1), 2 * I, H, xs,
-                                  L.rows_max, nullptr, 0, hs, I, I, pa.tile_expert, pa.used_tm, w8 + L.ws_a, s);
+    e = qlin_launch_chunk_grouped(fmt, dn, (int64_t)dn_stride, (int)qlin_mma_tiles(H, 0), H, I, L.rows_max, os, H,
+                                  nullptr, 0, 0, pa.tile_expert, pa.tile_rows, used_tm, pa.words + 2, nullptr,
+                                  w8 + L.ws_b, s);
     if (e != cudaSuccess) return e;
-    e = qlin_launch_chunk_grouped(fmt, dn, (int64_t)dn_stride, (int)qlin_mma_tiles(H, 0), H, I, hs, L.rows_max, os, H,
-                                  nullptr, 0, 0, pa.tile_expert, pa.used_tm, w8 + L.ws_b, s);
-    if (e != cudaSuccess) return e;
-    moe_prefill_combine_kernel<<<M, 256, 0, s>>>(pa.pos, wts, top_k, os, H, hs, I, y, h, pa.status,
-                                                 (const unsigned*)(w8 + L.ws_a), (const unsigned*)(w8 + L.ws_b));
+    moe_prefill_combine_kernel<<<M, 256, 0, s>>>(pa, os, hs, I, y, h, (const unsigned*)(w8 + L.ws_a),
+                                                 (const unsigned*)(w8 + L.ws_b));
     return cudaGetLastError();
 }

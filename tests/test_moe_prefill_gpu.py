@@ -4,10 +4,10 @@ Checked stage by stage against the fp64 oracle, with every bound derived from th
   routing   ids equal to the oracle's (the decision is taken on the fp32 logits on both sides),
             weights within 1e-6 relative (fp32 softmax over the selected experts);
   gate_up   h of each (token, slot) against silu(g) * u of the oracle's product of the same
-            quantized activations (NVFP4: one per-tensor scale over all routed rows, which is
-            amax|x| since every token is routed; MXFP4: the OCP MX rule, row-local) with the
-            expert's weights: the GEMM bound 2e-6 sum|a_q w| carried through silu(g) * u, the
-            epilogue's fp32 roundings, and h's rounding to bf16 (half an ulp, 2^-8 relative);
+            quantized activations (NVFP4: one per-tensor scale from max |x| over the chunk; MXFP4:
+            the OCP MX rule, row-local) with the expert's weights: the GEMM bound 2e-6 sum|a_q w|
+            carried through silu(g) * u, the epilogue's error (silu_tol below), and h's rounding
+            to bf16 (half an ulp, at most 2^-8 relative);
   down      y against the slot-ordered sum of the oracle's down projections of the kernel's own
             h quantized the same way (NVFP4: a per-tensor scale over all h): 2e-6 sum|h_q w| per
             slot and gamma(top_k) for the fp32 combine, as for the decode MoE.
@@ -28,8 +28,16 @@ def gamma(n):
     return n * U32 / (1 - n * U32)
 
 
-def silu_tol(href, Ah, u):
-    return 2e-6 * Ah + 8 * U32 * np.abs(href) + 4 * 2.0 ** -126 * (1 + np.abs(u))
+def silu_tol(href, Ah, g, u):
+    """The epilogue forms z = g s, e = exp(-|z|) with the MUFU ex2 unit (argument -|z| log2 e
+    rounded: |z| 2^-23 relative on e; the unit itself taken as 2^-21 relative) and 1 / (1 + e)
+    with the MUFU rcp unit (2^-21); sigmoid is r (z >= 0) or e r (z < 0), so within
+    2 (2^-21 + |z| 2^-23) + 2^-21 + 2^-23 relative; four fp32 roundings (z, u s, z sig, times u)
+    add 2^-22.  Together under (2^-19 + |g| 2^-22) |h|, plus the GEMM bound carried through
+    silu(g) u (2e-6 Ah), plus (|g| + 4) 2^-126 (1 + |u|) for e flushed to zero below 2^-126
+    (|h| <= |z| e^-|z| |u| there)."""
+    return (2e-6 * Ah + (2.0 ** -19 + np.abs(g) * 2.0 ** -22) * np.abs(href) +
+            (np.abs(g) + 4) * 2.0 ** -126 * (1 + np.abs(u)))
 
 
 class Experts:
@@ -71,7 +79,9 @@ def run_and_check(ex, M, top_k, seed, tokens=None, logits=None, given=None):
                                           topk_ids=torch.as_tensor(given[0], dtype=torch.int32).cuda(),
                                           topk_w=torch.as_tensor(given[1], dtype=torch.float32).cuda(), h=h, ws=ws)
     torch.cuda.synchronize()
-    assert q.qlin_ws_status(ws) == 0
+    bad = given is not None and any(not (0 <= int(e) < E) or int(e) in [int(v) for v in r[:i]]
+                                    for r in given[0] for i, e in enumerate(r))
+    assert q.qlin_ws_status(ws) == (1 if bad else 0)  # QLIN_ERR_INVALID_ARG: a bad expert id
     ids, w = ids.cpu().numpy(), w.cpu().double().numpy()
     h, y = h.cpu().double().numpy(), y.cpu().double().numpy()
     if given is None:
@@ -85,10 +95,13 @@ def run_and_check(ex, M, top_k, seed, tokens=None, logits=None, given=None):
         A = np.zeros(H)
         for s in range(top_k):
             e = int(ids[m, s])
+            if not (0 <= e < E) or e in [int(v) for v in ids[m, :s]]:  # a skipped slot
+                assert (h[m, s] == 0).all()
+                continue
             gb, gs, gg = ex.w(ex.gu[e])
             gu, Agu = oracle.gemv(fmt, 2 * I, H, gb, xq[m:m + 1], scales=gs, g=gg)
             href, Ah = oracle.silu_gate(gu, Agu)
-            tol = silu_tol(href[0], Ah[0], gu[0, I:])
+            tol = silu_tol(href[0], Ah[0], gu[0, :I], gu[0, I:])
             tol = tol + 2.0 ** -8 * (np.abs(href[0]) + tol)
             err = np.abs(h[m, s] - href[0])
             assert (err <= tol).all(), (m, s, float(np.max(err / tol)))
@@ -127,6 +140,20 @@ def test_moe_prefill_given_ids_uneven_load():
     w = rng.uniform(0.1, 1.0, (M, k)).astype(np.float32)
     out_ids, _, _ = run_and_check(ex, M, k, 7401, given=(ids, w))
     assert np.array_equal(out_ids, ids)
+
+
+@pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_MXFP4])
+def test_moe_prefill_bad_ids_reported_and_skipped(fmt):
+    # given ids with an out-of-range id and a repeated one: status bit 1 set, those slots skipped
+    E, H, I, M, k = 6, 256, 160, 40, 3
+    ex = Experts(fmt, E, H, I, 7450)
+    rng = np.random.default_rng(5)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(M)]).astype(np.int32)
+    ids[3, 1] = E + 2
+    ids[7, 2] = ids[7, 0]
+    ids[9, 0] = -1
+    w = rng.uniform(0.1, 1.0, (M, k)).astype(np.float32)
+    run_and_check(ex, M, k, 7451, given=(ids, w))
 
 
 def test_moe_prefill_deterministic_and_graph_capturable():

@@ -9,8 +9,9 @@
 // synchronisation (the counts and the tile table live on the device, so the sequence can be
 // captured in a CUDA graph):
 //   1. route (a warp per token): top_k (ties to the lower expert index, a NaN logit ranks as
-//      -inf), renormalised weights, max |x| of the token folded into one word, and for each valid
-//      slot its index among the expert's entries (an atomic counter per expert); the last CTA to
+//      -inf), renormalised weights, max |x| folded into one word, and for each valid slot its
+//      index among the expert's entries (a shared-memory count per CTA, then one atomic per expert
+//      and CTA on the global count); the last CTA to
 //      finish turns the counts into each expert's first sorted row (rows padded to whole 128-row
 //      tiles) and the table row tile -> expert;
 //   2. gather-quantize (a CTA per token): the token's row quantized once as the chunk path
@@ -43,7 +44,7 @@ namespace qlin {
 
 constexpr int kPfMaxTopK = 8;
 constexpr int kPfMaxE = 256;
-constexpr int kPfRouteWarps = 8;  // tokens per route CTA
+constexpr int kPfRouteWarps = 16;  // tokens per route CTA
 constexpr int kPfGatherThreads = 128;
 constexpr int kPfPadCtas = 4;  // CTAs zeroing one expert's padding rows
 
@@ -113,14 +114,19 @@ __device__ __forceinline__ bool pf_before(float a, int ia, float b, int ib) {
 }
 
 __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(const PfArgs a) {
+    __shared__ int s_cnt[kPfMaxE];  // this CTA's entries per expert, then their first index
     __shared__ int s_off[kPfMaxE + 1];
+    __shared__ float s_max[kPfRouteWarps];
     __shared__ int s_last;
-    const int lane = threadIdx.x & 31, k = a.top_k;
-    const int m = blockIdx.x * kPfRouteWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, k = a.top_k;
+    const int m = blockIdx.x * kPfRouteWarps + warp;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) s_cnt[e] = 0;
+    __syncthreads();
+    int my_e = -1, my_li = 0;  // lane r < top_k: slot r's expert and its index among this CTA's
+    float mx = 0.f;
     if (m < a.M) {
         // max |x| of the token (fmaxf skips a NaN, as the chunk quantizer's max pass does)
         const uint4* xr = reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.H);
-        float mx = 0.f;
 #pragma unroll 8
         for (int64_t v = lane; v < a.H / 8; v += 32) {
             const uint4 q = __ldg(xr + v);
@@ -130,7 +136,6 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
                 mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[j] << 16)), fabsf(__uint_as_float(w[j] & 0xffff0000u))));
         }
         for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) atomicMax(&a.words[1], __float_as_uint(mx));  // non-negative floats order as their bits
 
         int32_t* id = a.ids + (int64_t)m * k;
         int sel[kPfMaxTopK];
@@ -146,6 +151,7 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
                 v[j] = e < a.E ? l[e] : -INFINITY;
             }
             unsigned taken = 0u;
+            float selv[kPfMaxTopK];  // the selected logits (as given)
 #pragma unroll
             for (int r = 0; r < kPfMaxTopK; ++r) {
                 if (r >= k) break;
@@ -168,16 +174,16 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
                     }
                 }
                 sel[r] = bi;
+                selv[r] = bv;
                 if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
             }
             // weights: softmax over the selected logits (the largest first), fp32
-            const float l0 = l[sel[0]];
-            const float lmax = l0 != l0 ? 0.f : l0;
+            const float lmax = selv[0] != selv[0] ? 0.f : selv[0];
             float ex[kPfMaxTopK], sum = 0.f;
 #pragma unroll
             for (int r = 0; r < kPfMaxTopK; ++r) {
                 if (r >= k) break;
-                ex[r] = expf(l[sel[r]] - lmax);
+                ex[r] = expf(selv[r] - lmax);
                 sum += ex[r];
             }
             if (lane == 0) {
@@ -205,16 +211,31 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
                 if (r2 < lane && sel[r2] == e) ok = false;  // a repeated id counts once
             ok = ok && e >= 0 && e < a.E;
             if (ok) {
-                a.lpos[(int64_t)m * k + lane] = atomicAdd(&a.cnt[e], 1);
+                my_e = e;
+                my_li = atomicAdd(&s_cnt[e], 1);
             } else {
                 a.lpos[(int64_t)m * k + lane] = -1;
                 atomicOr(a.status, 2u);
             }
         }
     }
+    // One global atomic per expert present in this CTA gives its entries' first index; one per CTA
+    // folds max |x| in (non-negative floats order as their bits).
+    if (lane == 0) s_max[warp] = mx;
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        const int c = s_cnt[e];
+        if (c) s_cnt[e] = atomicAdd(&a.cnt[e], c);
+    }
+    if (threadIdx.x == 0) {
+        float b = 0.f;
+        for (int w = 0; w < kPfRouteWarps; ++w) b = fmaxf(b, s_max[w]);
+        atomicMax(&a.words[1], __float_as_uint(b));
+    }
+    __syncthreads();
+    if (my_e >= 0) a.lpos[(int64_t)m * k + lane] = s_cnt[my_e] + my_li;
     // The last CTA to finish: first sorted row of each expert, the tile table, and the counters
     // cleared for the next call.
-    __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
         s_last = atomicAdd(&a.words[0], 1u) == gridDim.x - 1;
@@ -224,29 +245,53 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
     __threadfence();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {  // the counts, read once and cleared
         const int c = __ldcg(&a.cnt[e]);
-        s_off[e] = c;
+        s_cnt[e] = c;
         a.fill[e] = c;
         a.cnt[e] = 0;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < a.E; ++e) {
-            const int c = s_off[e];
-            s_off[e] = run;
-            run += (c + 127) / 128 * 128;
+    if (warp == 0) {  // exclusive scan of the padded counts: lane l takes experts 8l .. 8l + 7
+        int c[kPfMaxE / 32], sum = 0;
+#pragma unroll
+        for (int j = 0; j < kPfMaxE / 32; ++j) {
+            const int e = lane * (kPfMaxE / 32) + j;
+            c[j] = e < a.E ? (s_cnt[e] + 127) / 128 * 128 : 0;
+            sum += c[j];
         }
-        s_off[a.E] = run;
-        a.words[3] = (unsigned)(run / 128);
+        int incl = sum;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int j = 0; j < kPfMaxE / 32; ++j) {
+            const int e = lane * (kPfMaxE / 32) + j;
+            if (e < a.E) s_off[e] = run;
+            run += c[j];
+        }
+        if (lane == 31) {
+            s_off[a.E] = incl;
+            a.words[3] = (unsigned)(incl / 128);
+        }
     }
     __syncthreads();
     for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.off[e] = s_off[e];
     for (int t = threadIdx.x; t < a.TMx; t += blockDim.x) {
+        // the expert whose rows hold tile t: the last e with s_off[e] <= 128 t (an expert without
+        // entries holds no rows), -1 past the rows in use
         int ex = -1;
-        for (int e = 0; e < a.E && ex < 0; ++e)
-            if (s_off[e] <= 128 * t && 128 * t < s_off[e + 1]) ex = e;
+        if (128 * t < s_off[a.E]) {
+            int lo = 0, hi = a.E - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_off[mid] <= 128 * t) lo = mid;
+                else hi = mid - 1;
+            }
+            ex = lo;
+        }
         a.tile_expert[t] = ex;
-        const int live = ex < 0 ? 0 : s_off[ex] + a.fill[ex] - 128 * t;
+        const int live = ex < 0 ? 0 : s_off[ex] + s_cnt[ex] - 128 * t;
         a.tile_rows[t] = live < 0 ? 0 : (live > 128 ? 128 : live);
     }
     if (threadIdx.x == 0) {
@@ -267,6 +312,9 @@ __global__ void __launch_bounds__(kPfGatherThreads) moe_prefill_gather_quant_ker
     const int64_t nitems = G * 16;
     if (b < a.M) {
         const int m = b;
+        // the token's first item in flight before the routing reads
+        uint32_t w[8], c8[2];
+        act_load_item(a.x, threadIdx.x < nitems ? a.M : 0, a.H, a.H, true, m, threadIdx.x < nitems ? threadIdx.x : 0, w);
         int rows[kPfMaxTopK];
 #pragma unroll
         for (int r = 0; r < kPfMaxTopK; ++r) {
@@ -283,8 +331,7 @@ __global__ void __launch_bounds__(kPfGatherThreads) moe_prefill_gather_quant_ker
         for (int64_t i0 = 0; i0 < nitems; i0 += kPfGatherThreads) {
             const int64_t it = i0 + threadIdx.x;
             const bool live = it < nitems;
-            uint32_t w[8], c8[2];
-            act_load_item(a.x, live ? a.M : 0, a.H, a.H, true, m, live ? it : 0, w);
+            if (i0 > 0) act_load_item(a.x, live ? a.M : 0, a.H, a.H, true, m, live ? it : 0, w);
             uint8_t sc;
             if constexpr (MX) {
                 sc = act_mx_pair_byte(act_item_amax(w), act_item_special(w));
@@ -319,37 +366,58 @@ __global__ void __launch_bounds__(kPfGatherThreads) moe_prefill_gather_quant_ker
     }
 }
 
-// h (the sorted rows in use, bf16) quantized for the down GEMM, one thread per 16-value item:
-// NVFP4 with a_g from max |h| (word [2], folded in by the gate_up epilogue), MXFP4 by the pair rule;
-// stored in the down GEMM's operand units (G k-groups per 128-row tile; values past I are zeros).
-// Padding rows (not written by the gate_up epilogue) are not read: their operand rows are zeros.
-// The grid covers every row the workspace can hold; CTAs past the rows in use return at once.
+// h (the sorted rows in use, bf16) quantized for the down GEMM: one thread per 64 consecutive
+// values of a row (four 16-value items; NVFP4 with a_g from max |h|, word [2], folded in by the
+// gate_up epilogue; MXFP4 by the OCP MX rule, the two 32-value blocks within the thread), stored
+// in the down GEMM's operand units (G k-groups per 128-row tile; values past I are zeros) as two
+// 16-byte code chunks and one scale word.  Padding rows (not written by the gate_up epilogue) are
+// not read: their operand rows are zeros.  The grid covers every row the workspace can hold;
+// threads past the rows in use return at once.
 template <bool MX>
 __global__ void __launch_bounds__(256) moe_prefill_quant_h_kernel(const __nv_bfloat16* __restrict__ hs, int64_t I,
                                                                   int64_t G, const unsigned* __restrict__ words,
                                                                   const int* __restrict__ tile_rows,
                                                                   uint8_t* __restrict__ aq) {
-    const int64_t nitems = G * 16;
+    const int64_t nq = G * 4;  // 64-value quads per (padded) row
+    const int64_t qd = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int rows = (int)words[3] * kMmaARows;
-    const int64_t used = (int64_t)rows * nitems;
-    const int64_t first = (int64_t)blockIdx.x * blockDim.x;
-    if (first >= used) return;  // (the whole CTA: the pair shuffles below run with every lane)
-    const int64_t i = first + threadIdx.x;
-    const bool live = i < used;
-    const int row = live ? (int)(i / nitems) : 0;
-    const int64_t it = live ? i - (int64_t)row * nitems : 0;
-    const bool data = live && (row % kMmaARows) < tile_rows[row / kMmaARows];
-    uint32_t w[8], c8[2];
-    act_load_item(hs, data ? rows : 0, I, I, true, row, it, w);
-    uint8_t sc;
+    if (qd >= (int64_t)rows * nq) return;
+    const int row = (int)(qd / nq);
+    const int64_t qi = qd - (int64_t)row * nq;
+    const int tm = row / kMmaARows, r = row % kMmaARows;
+    const int lim = r < tile_rows[tm] ? rows : 0;  // a padding row reads as zeros
+    uint32_t w[4][8], c8[4][2];
+    uint8_t sc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) act_load_item(hs, lim, I, I, true, row, 4 * qi + j, w[j]);
     if constexpr (MX) {
-        sc = act_mx_pair_byte(act_item_amax(w), act_item_special(w));
-        act_quant_item_mx_codes(w, sc, c8);
-        if (live) act_store_item_mx(0, I, G, row, it, sc, c8, aq, nullptr, nullptr);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint8_t byte = mx_scale_byte(fmaxf(act_item_amax(w[2 * h]), act_item_amax(w[2 * h + 1])),
+                                               act_item_special(w[2 * h]) || act_item_special(w[2 * h + 1]));
+            sc[2 * h] = sc[2 * h + 1] = byte;
+            act_quant_item_mx_codes(w[2 * h], byte, c8[2 * h]);
+            act_quant_item_mx_codes(w[2 * h + 1], byte, c8[2 * h + 1]);
+        }
     } else {
-        sc = act_quant_block(w, act_item_amax(w), act_global_scale(__uint_as_float(__ldcg(&words[2]))), c8);
-        if (live) act_store_item(0, I, G, row, it, sc, c8, aq, nullptr, nullptr);
+        const float ag = act_global_scale(__uint_as_float(__ldcg(&words[2])));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc[j] = act_quant_block(w[j], act_item_amax(w[j]), ag, c8[j]);
     }
+    const int64_t k0 = 64 * qi;
+    const int kin = (int)(k0 % kGroupK);
+    uint8_t* ub = aq + ((int64_t)tm * G + k0 / kGroupK) * kMmaAUnit;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)  // 16-byte chunk kin / 32 + h: items 2h and 2h + 1
+        *reinterpret_cast<uint4*>(ub + mma_code_off(r, kin / 32 + h)) =
+            make_uint4(c8[2 * h][0], c8[2 * h][1], c8[2 * h + 1][0], c8[2 * h + 1][1]);
+    uint8_t* sb = ub + kMmaARows * 128;
+    if constexpr (MX)  // the two block scales of this half span: bytes j, j + 1 of the row's word
+        *reinterpret_cast<uint16_t*>(sb + mma_scale_off(kin / 128, r, (kin % 128) / 32, 1)) =
+            (uint16_t)(sc[0] | (sc[2] << 8));
+    else  // the four 16-value scales of this 64-value block: the row's word of atom kin / 64
+        *reinterpret_cast<uint32_t*>(sb + mma_scale_off(kin / 64, r, 0, 1)) =
+            (uint32_t)sc[0] | ((uint32_t)sc[1] << 8) | ((uint32_t)sc[2] << 16) | ((uint32_t)sc[3] << 24);
 }
 
 // One CTA per token: y[m] = sum over slots in slot order of w * o[row]; the optional h output
@@ -457,13 +525,13 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
                                   pa.words + 2, w8 + L.ws_a, s);
     if (e != cudaSuccess) return e;
     const int64_t Gi = (I + kGroupK - 1) / kGroupK;
-    const int64_t hitems = (int64_t)L.rows_max * Gi * 16;
+    const int64_t hquads = (int64_t)L.rows_max * Gi * 4;
     uint8_t* aq_b = w8 + L.ws_b + 256;  // the down GEMM's operand units
     if (fmt == QLIN_MXFP4)
-        moe_prefill_quant_h_kernel<true><<<(unsigned)((hitems + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
+        moe_prefill_quant_h_kernel<true><<<(unsigned)((hquads + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
                                                                                           pa.tile_rows, aq_b);
     else
-        moe_prefill_quant_h_kernel<false><<<(unsigned)((hitems + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
+        moe_prefill_quant_h_kernel<false><<<(unsigned)((hquads + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
                                                                                            pa.tile_rows, aq_b);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = qlin_launch_chunk_grouped(fmt, dn, (int64_t)dn_stride, (int)qlin_mma_tiles(H, 0), H, I, L.rows_max, os, H,

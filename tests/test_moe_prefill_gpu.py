@@ -122,6 +122,18 @@ def test_moe_prefill_small(fmt, M):
     run_and_check(ex, M, 2, 7100 + M)
 
 
+@pytest.mark.parametrize("fmt,E,H,I,M,k", [
+    (q.QLIN_NVFP4, 256, 64, 64, 5, 8),     # the largest expert count and top_k the entry point takes
+    (q.QLIN_MXFP4, 1, 96, 160, 70, 1),     # one expert: every token on it
+    (q.QLIN_NVFP4, 4, 32, 32, 9, 4),       # the smallest H and I, top_k = E
+    (q.QLIN_MXFP4, 16, 64, 96, 4096, 2),   # many tokens: 256 routing CTAs, 64 tiles per expert on average
+])
+def test_moe_prefill_edge_shapes(fmt, E, H, I, M, k):
+    ex = Experts(fmt, E, H, I, 7600 + E)
+    tokens = None if M <= 128 else [0, 1, 2047, 2048, 4095]
+    run_and_check(ex, M, k, 7700 + M, tokens=tokens)
+
+
 @pytest.mark.parametrize("fmt", [q.QLIN_NVFP4, q.QLIN_MXFP4])
 def test_moe_prefill_lfm2_shape_sampled(fmt):
     # the 8B-A1B MoE layer (H 2048, 32 experts of gate_up 2048 -> 2 x 1792, down 1792 -> 2048, top-4)

@@ -271,28 +271,37 @@ qlin_status_t qlin_moe_experts(qlin_format_t fmt, const void* gate_up_packed, co
                                float* y, float* h, int flags, void* ws, size_t ws_bytes,
                                qlin_stream_t stream);
 
-/* Top-k routed MoE expert projections for a prefill chunk of M tokens (M >= 1; built for M >= 64) on
- * the tcgen05 tensor cores: what qlin_moe_experts computes -- the same routing (top_k by logit, ties
- * to the lower expert index, a NaN logit ranks as -inf, weights renormalised over the selected
+/* Top-k routed MoE expert projections for a prefill chunk of M tokens (M >= 1; built for M >= 64)
+ * on the tcgen05 tensor cores: what qlin_moe_experts computes -- the same routing (top_k by logit,
+ * ties to the lower expert index, a NaN logit ranks as -inf, weights renormalised over the selected
  * experts), h = silu(W_gate[e] x) * (W_up[e] x), o = W_down[e] h, y[m] = sum over slots in slot
- * order of weight * o -- with NVFP4 or MXFP4 expert weights and the chunk path's quantization of the
- * activations: the (token, slot) rows are sorted by expert (tokens ascending, each expert's rows
- * padded to whole 128-row tiles) and quantized as qlin_gemm_chunk quantizes x (NVFP4: one
- * per-tensor scale over all sorted rows; MXFP4: the OCP MX rule), each 128-row tile multiplied by
- * its expert's weights with the SiLU-gate fused in the epilogue; h is kept as bf16 and quantized
- * the same way for the down projection (NVFP4: with its own per-tensor scale).  The pages'
- * counterpart is imp's MoE top-k grouped GEMM, an NVFP4 grouped GEMM on sm_120a (imp README,
- * "Features" table, row "Architectures"; release notes v0.7.0).  Five launches on `stream`
- * (route + sort, gather, two grouped GEMMs, combine), no host synchronisation.
+ * order of weight * o -- with NVFP4 or MXFP4 expert weights and the chunk path's quantization of
+ * the activations:
+ *   - x is quantized once per token as qlin_gemm_chunk quantizes it (NVFP4: one per-tensor scale
+ *     from max |x| over all M tokens; MXFP4: the OCP MX rule) and copied to the token's sorted rows
+ *     (the routed (token, slot) entries grouped by expert, each expert padded to whole 128-row
+ *     tiles);
+ *   - each 128-row tile is multiplied by its expert's gate/up weights with the SiLU-gate fused in
+ *     the epilogue (silu from the MUFU ex2 / rcp units: within (2^-19 + |g| 2^-22) |h| of the fp32
+ *     expression before h is rounded to bf16);
+ *   - h (bf16) is quantized the same way for the down projection (NVFP4: its own per-tensor scale
+ *     from max |h| over every routed row).
+ * Which sorted row an entry takes depends on the order of device atomics, but every row is computed
+ * on its own, so y, h, ids and weights are the same from run to run (and under graph replay).  The
+ * pages' counterpart is imp's MoE top-k grouped GEMM, an NVFP4 grouped GEMM on sm_120a (imp README,
+ * "Features" table, row "Architectures"; release notes v0.7.0).  Six launches on `stream` (route,
+ * gather-quantize, grouped gate_up GEMM, h quantization, grouped down GEMM, combine), no host
+ * synchronisation.
  *   gate_up_packed: E consecutive buffers, each qlin_packed_bytes(fmt, 2I, H, QLIN_PACK_MMA |
  *                   QLIN_PACK_GATE_UP) bytes, expert e packed from its [gate ; up] rows (2I x H)
  *   down_packed   : E consecutive buffers, each qlin_packed_bytes(fmt, H, I, QLIN_PACK_MMA) bytes
  *   router_logits : M x E fp32, or NULL -- then topk_ids / topk_w are inputs (a bad or repeated id is
- *                   skipped and qlin_ws_status() reports QLIN_ERR_INVALID_ARG)
+ *                   skipped, its h row is zero, and qlin_ws_status() reports QLIN_ERR_INVALID_ARG)
  *   topk_ids, topk_w: M x top_k int32 / fp32, written when router_logits is given
  *   x : M x H bf16, contiguous, 16-byte aligned;  y : M x H fp32, contiguous
  *   h : optional M x top_k x I fp32: the bf16 h of each (token, slot), as fp32 (NULL: not written)
- *   flags: 0;  ws: qlin_workspace_bytes(QLIN_OP_MOE_PREFILL, fmt, M, H, I, E, top_k) bytes
+ *   flags: 0;  ws: qlin_workspace_bytes(QLIN_OP_MOE_PREFILL, fmt, M, H, I, E, top_k) bytes, zero-filled
+ *       before its first use like every workspace
  * fmt NVFP4 or MXFP4 (else QLIN_ERR_UNSUPPORTED); E <= 256, top_k <= min(8, E); H % 32 == 0 and
  * I % 32 == 0 (QLIN_ERR_INVALID_ARG otherwise).  Bounded device waits as qlin_gemm_chunk. */
 qlin_status_t qlin_moe_prefill(qlin_format_t fmt, const void* gate_up_packed, const void* down_packed, int E,

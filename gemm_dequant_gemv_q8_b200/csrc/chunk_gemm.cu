@@ -1146,7 +1146,7 @@ extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t
 // expert tile_expert[tm].  h != nullptr: the SiLU-gate epilogue (weights packed QLIN_PACK_MMA |
 // QLIN_PACK_GATE_UP) writing h_cols bf16 outputs per row and folding max |h| into *amax_out; else
 // y (fp32, N columns).  Either way rows past tile_rows[tm] of tile tm are not stored.  Single CTAs,
-// no k-split, no programmatic dependent launch.
+// no k-split, launched as a programmatic dependent of the kernel before it.
 extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t w_stride, int T2, int64_t N,
                                                  int64_t K, int rows_max, float* y, int64_t ldy, void* h,
                                                  int64_t ldh, int64_t h_cols, const int* tile_expert,
@@ -1182,5 +1182,8 @@ extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t
     a.h_cols = h_cols;
     a.amax_in = amax_in;
     a.amax_out = amax_out;
-    return fmt == QLIN_MXFP4 ? launch_chunk_cg<1, true, true>(a, 0, s) : launch_chunk_cg<1, false, true>(a, 0, s);
+    // programmatic dependent launch: the tile table, the row counts and the weights read before
+    // the kernel's wait come from kernels that finished before the previous one passed its own wait
+    return fmt == QLIN_MXFP4 ? launch_chunk_cg<1, true, true>(a, QLIN_FLAG_PDL, s)
+                             : launch_chunk_cg<1, false, true>(a, QLIN_FLAG_PDL, s);
 }

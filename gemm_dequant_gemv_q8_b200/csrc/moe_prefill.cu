@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
     __shared__ int s_last;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, k = a.top_k;
     const int m = blockIdx.x * kPfRouteWarps + warp;
+    griddep_launch_dependents();  // (the gather reads nothing of this grid before its own wait)
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) s_cnt[e] = 0;
     __syncthreads();
     int my_e = -1, my_li = 0;  // lane r < top_k: slot r's expert and its index among this CTA's
@@ -312,9 +313,11 @@ __global__ void __launch_bounds__(kPfGatherThreads) moe_prefill_gather_quant_ker
     const int64_t nitems = G * 16;
     if (b < a.M) {
         const int m = b;
-        // the token's first item in flight before the routing reads
+        // the token's first item (the caller's x) in flight before the wait for the routing
         uint32_t w[8], c8[2];
         act_load_item(a.x, threadIdx.x < nitems ? a.M : 0, a.H, a.H, true, m, threadIdx.x < nitems ? threadIdx.x : 0, w);
+        griddep_wait();
+        griddep_launch_dependents();  // after the wait: the next grid's early reads see the routing
         int rows[kPfMaxTopK];
 #pragma unroll
         for (int r = 0; r < kPfMaxTopK; ++r) {
@@ -350,6 +353,8 @@ __global__ void __launch_bounds__(kPfGatherThreads) moe_prefill_gather_quant_ker
             }
         }
     } else {
+        griddep_wait();
+        griddep_launch_dependents();
         const int e = (b - a.M) / kPfPadCtas, part = (b - a.M) % kPfPadCtas;
         const int r0 = a.off[e] + a.fill[e], npad = a.off[e + 1] - r0;  // < 128 rows, one tile
         const int per_row = (int)G * 12;
@@ -378,6 +383,8 @@ __global__ void __launch_bounds__(256) moe_prefill_quant_h_kernel(const __nv_bfl
                                                                   int64_t G, const unsigned* __restrict__ words,
                                                                   const int* __restrict__ tile_rows,
                                                                   uint8_t* __restrict__ aq) {
+    griddep_wait();  // h and max |h| come from the gate_up GEMM
+    griddep_launch_dependents();
     const int64_t nq = G * 4;  // 64-value quads per (padded) row
     const int64_t qd = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int rows = (int)words[3] * kMmaARows;
@@ -429,6 +436,7 @@ __global__ void __launch_bounds__(256) moe_prefill_combine_kernel(const PfArgs a
                                                                   const unsigned* st_a, const unsigned* st_b) {
     const int m = blockIdx.x, top_k = a.top_k;
     const int64_t H = a.H;
+    griddep_wait();  // o comes from the down GEMM
     if (m == 0 && threadIdx.x == 0) {
         const unsigned s = *st_a | *st_b;
         if (s) atomicOr(a.status, s & 1u);
@@ -475,6 +483,24 @@ __global__ void __launch_bounds__(256) moe_prefill_combine_kernel(const PfArgs a
 
 using namespace qlin;
 
+// A launch that may begin while the previous kernel of the stream finishes (programmatic dependent
+// launch); the kernel waits (griddepcontrol.wait) before it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+static cudaError_t pf_launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
+                                 Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 extern "C" size_t qlin_moe_prefill_ws_bytes(int M, int64_t H, int64_t I, int E, int top_k) {
     return (size_t)pf_layout(M, H, I, E, top_k).total;
 }
@@ -513,11 +539,10 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
     if (e != cudaSuccess) return e;
     const int64_t Gh = (H + kGroupK - 1) / kGroupK;
     uint8_t* aq = w8 + L.ws_a + 256;  // the gate_up GEMM's operand units (its workspace layout)
-    if (fmt == QLIN_MXFP4)
-        moe_prefill_gather_quant_kernel<true><<<M + kPfPadCtas * E, kPfGatherThreads, 0, s>>>(pa, Gh, aq);
-    else
-        moe_prefill_gather_quant_kernel<false><<<M + kPfPadCtas * E, kPfGatherThreads, 0, s>>>(pa, Gh, aq);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = fmt == QLIN_MXFP4
+            ? pf_launch_pdl(moe_prefill_gather_quant_kernel<true>, M + kPfPadCtas * E, kPfGatherThreads, s, pa, Gh, aq)
+            : pf_launch_pdl(moe_prefill_gather_quant_kernel<false>, M + kPfPadCtas * E, kPfGatherThreads, s, pa, Gh, aq);
+    if (e != cudaSuccess) return e;
     __nv_bfloat16* hs = (__nv_bfloat16*)(w8 + L.hs);
     float* os = (float*)(w8 + L.os);
     e = qlin_launch_chunk_grouped(fmt, gu, (int64_t)gu_stride, (int)qlin_mma_tiles(2 * I, 1), 2 * I, H, L.rows_max,
@@ -527,18 +552,17 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
     const int64_t Gi = (I + kGroupK - 1) / kGroupK;
     const int64_t hquads = (int64_t)L.rows_max * Gi * 4;
     uint8_t* aq_b = w8 + L.ws_b + 256;  // the down GEMM's operand units
-    if (fmt == QLIN_MXFP4)
-        moe_prefill_quant_h_kernel<true><<<(unsigned)((hquads + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
-                                                                                          pa.tile_rows, aq_b);
-    else
-        moe_prefill_quant_h_kernel<false><<<(unsigned)((hquads + 255) / 256), 256, 0, s>>>(hs, I, Gi, pa.words,
-                                                                                           pa.tile_rows, aq_b);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const unsigned hgrid = (unsigned)((hquads + 255) / 256);
+    e = fmt == QLIN_MXFP4 ? pf_launch_pdl(moe_prefill_quant_h_kernel<true>, hgrid, 256, s, hs, I, Gi,
+                                          (const unsigned*)pa.words, (const int*)pa.tile_rows, aq_b)
+                          : pf_launch_pdl(moe_prefill_quant_h_kernel<false>, hgrid, 256, s, hs, I, Gi,
+                                          (const unsigned*)pa.words, (const int*)pa.tile_rows, aq_b);
+    if (e != cudaSuccess) return e;
     e = qlin_launch_chunk_grouped(fmt, dn, (int64_t)dn_stride, (int)qlin_mma_tiles(H, 0), H, I, L.rows_max, os, H,
                                   nullptr, 0, 0, pa.tile_expert, pa.tile_rows, used_tm, pa.words + 2, nullptr,
                                   w8 + L.ws_b, s);
     if (e != cudaSuccess) return e;
-    moe_prefill_combine_kernel<<<M, 256, 0, s>>>(pa, os, hs, I, y, h, (const unsigned*)(w8 + L.ws_a),
-                                                 (const unsigned*)(w8 + L.ws_b));
-    return cudaGetLastError();
+    return pf_launch_pdl(moe_prefill_combine_kernel, (unsigned)M, 256, s, pa, (const float*)os,
+                         (const __nv_bfloat16*)hs, I, y, h, (const unsigned*)(w8 + L.ws_a),
+                         (const unsigned*)(w8 + L.ws_b));
 }

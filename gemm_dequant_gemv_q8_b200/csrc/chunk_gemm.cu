@@ -503,6 +503,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         } else {
             m = act_amax_partial(a.x, a.M, a.K, a.ldx, vec, gtid, gthreads);
         }
+        // The per-unit ready counters start from zero: cleared here, before the grid barrier that
+        // orders every CTA's increments after them.  (Their place in the workspace depends on the
+        // shape, so what a call with other shapes left there is not zero.)
+        for (int64_t u = gtid; u < (int64_t)a.TM * a.G; u += gthreads) a.ready[u] = 0u;
+        __threadfence();
         if (a.KS > 1) {  // the k-split halves add into y: zero it (ordered before them by the barrier)
             const int64_t nq = (a.N + 3) / 4;
             for (int64_t i = gtid; i < (int64_t)a.M * nq; i += gthreads) {
@@ -949,20 +954,19 @@ __global__ void __launch_bounds__(kChunkThreads, 1) chunk_gemm_kernel(const Chun
         tc_fence_after();
         tmem_free<CG>(tmem);
     }
-    // The last CTA out clears the counters for the next call.
-    if (threadIdx.x == 0) {
-        __threadfence();
-        *issued = atomicAdd(&a.words[kWExit], 1u) == gridDim.x - 1 ? -1 : 0;
-    }
-    __syncthreads();
-    if (*issued == -1) {
-        for (int64_t u = threadIdx.x; u < (int64_t)a.TM * a.G; u += blockDim.x) a.ready[u] = 0u;
+    // The last CTA out clears the words of phase Q for the next call (grouped mode uses none).
+    if constexpr (!GR) {
         if (threadIdx.x == 0) {
+            __threadfence();
+            *issued = atomicAdd(&a.words[kWExit], 1u) == gridDim.x - 1 ? -1 : 0;
+        }
+        __syncthreads();
+        if (*issued == -1 && threadIdx.x == 0) {
             a.words[kWAmax] = 0u;
             a.words[kWArrive1] = 0u;
             a.words[kWExit] = 0u;
+            __threadfence();
         }
-        __threadfence();
     }
 }
 
@@ -1145,13 +1149,14 @@ extern "C" cudaError_t qlin_launch_act_quant_debug(const void* x, int M, int64_t
 // w = E packed weight buffers w_stride bytes apart, T2 weight tiles per expert, row tile tm against
 // expert tile_expert[tm].  h != nullptr: the SiLU-gate epilogue (weights packed QLIN_PACK_MMA |
 // QLIN_PACK_GATE_UP) writing h_cols bf16 outputs per row and folding max |h| into *amax_out; else
-// y (fp32, N columns).  Either way rows past tile_rows[tm] of tile tm are not stored.  Single CTAs,
+// y (fp32, N columns).  Either way rows past tile_rows[tm] of tile tm are not stored.  Errors go to
+// *status (the first word of the caller's workspace, whose wait budget word the waits read).  Single CTAs,
 // no k-split, launched as a programmatic dependent of the kernel before it.
 extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t w_stride, int T2, int64_t N,
                                                  int64_t K, int rows_max, float* y, int64_t ldy, void* h,
                                                  int64_t ldh, int64_t h_cols, const int* tile_expert,
                                                  const int* tile_rows, const int* used_tm, const unsigned* amax_in,
-                                                 unsigned* amax_out, void* ws, cudaStream_t s) {
+                                                 unsigned* amax_out, unsigned* status, void* ws, cudaStream_t s) {
     uint8_t* w8 = (uint8_t*)ws;
     ChunkArgs a;
     memset(&a, 0, sizeof(a));
@@ -1172,7 +1177,7 @@ extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t
     a.yvec = (y && (reinterpret_cast<uintptr_t>(y) & 15) == 0 && ldy % 4 == 0) ? 1 : 0;
     a.KS = 1;
     a.GS = a.G;
-    a.status = (unsigned*)ws;
+    a.status = status;  // the caller's status word (its wait budget word 32 bytes on)
     a.tile_expert = tile_expert;
     a.tile_rows = tile_rows;
     a.used_tm = used_tm;

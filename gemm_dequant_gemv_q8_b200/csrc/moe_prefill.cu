@@ -26,7 +26,7 @@
 //   5. grouped chunk GEMM, down: each tile against its expert's down weights, o (fp32) per sorted row
 //      (padding rows not stored);
 //   6. combine: y[m] = sum over slots, in slot order, of weight * o[row of (m, slot)] (deterministic),
-//      the optional h output, the two GEMMs' status words folded into the caller's.
+//      and the optional h output.  The GEMMs report their errors in the caller's status word.
 // Which sorted row an entry takes depends on the order of the atomic counter, but every row is
 // computed on its own (the MMA rows are independent and the per-tensor scales are maxima), so the
 // results do not: y, h, ids and weights are the same from run to run.
@@ -36,7 +36,7 @@ extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t
                                                  int64_t K, int rows_max, float* y, int64_t ldy, void* h,
                                                  int64_t ldh, int64_t h_cols, const int* tile_expert,
                                                  const int* tile_rows, const int* used_tm, const unsigned* amax_in,
-                                                 unsigned* amax_out, void* ws, cudaStream_t s);
+                                                 unsigned* amax_out, unsigned* status, void* ws, cudaStream_t s);
 extern "C" size_t qlin_chunk_ws_bytes(int M, int64_t N, int64_t K);
 extern "C" int64_t qlin_mma_tiles(int64_t N, int gate_up);
 
@@ -57,7 +57,8 @@ static inline int pf_rows_max(int M, int E, int top_k) {
 }
 
 // Workspace layout (offsets in bytes).  [0, 256): the status word (and the wait budget word).
-// rt: cnt[256] at 0, fill[256] at 1024, off[257] at 2048, words at 3328: [0] ticket, [1] max |x|,
+// rt, at a fixed offset (its counters start each call at zero, whatever the shapes of the call
+// before): cnt[256] at 0, fill[256] at 1024, off[257] at 2048, words at 3328: [0] ticket, [1] max |x|,
 // [2] max |h|, [3] row tiles in use.
 struct PfLayout {
     int64_t lpos, pos, rt, tile_expert, ws_a, hs, ws_b, os, total;
@@ -69,12 +70,12 @@ static PfLayout pf_layout(int M, int64_t H, int64_t I, int E, int top_k) {
     L.rows_max = pf_rows_max(M, E, top_k);
     const int64_t R = L.rows_max, TMx = R / 128;
     int64_t o = 256;
+    L.rt = o;
+    o += 4096;
     L.lpos = o;
     o += pf_al256(4 * (int64_t)M * top_k);
     L.pos = o;
     o += pf_al256(4 * (int64_t)M * top_k);
-    L.rt = o;
-    o += 4096;
     L.tile_expert = o;  // then tile_rows
     o += pf_al256(8 * TMx);
     L.ws_a = o;
@@ -428,20 +429,14 @@ __global__ void __launch_bounds__(256) moe_prefill_quant_h_kernel(const __nv_bfl
 }
 
 // One CTA per token: y[m] = sum over slots in slot order of w * o[row]; the optional h output
-// (fp32 values of the bf16 h of each (token, slot)); the GEMMs' status words folded in; max |x|
-// cleared for the next call.
+// (fp32 values of the bf16 h of each (token, slot)); max |x| cleared for the next call.
 __global__ void __launch_bounds__(256) moe_prefill_combine_kernel(const PfArgs a, const float* __restrict__ os,
                                                                   const __nv_bfloat16* __restrict__ hs, int64_t I,
-                                                                  float* __restrict__ y, float* __restrict__ h,
-                                                                  const unsigned* st_a, const unsigned* st_b) {
+                                                                  float* __restrict__ y, float* __restrict__ h) {
     const int m = blockIdx.x, top_k = a.top_k;
     const int64_t H = a.H;
     griddep_wait();  // o comes from the down GEMM
-    if (m == 0 && threadIdx.x == 0) {
-        const unsigned s = *st_a | *st_b;
-        if (s) atomicOr(a.status, s & 1u);
-        a.words[1] = 0u;
-    }
+    if (m == 0 && threadIdx.x == 0) a.words[1] = 0u;
     int rows[kPfMaxTopK];
     float w[kPfMaxTopK];
 #pragma unroll
@@ -547,7 +542,7 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
     float* os = (float*)(w8 + L.os);
     e = qlin_launch_chunk_grouped(fmt, gu, (int64_t)gu_stride, (int)qlin_mma_tiles(2 * I, 1), 2 * I, H, L.rows_max,
                                   nullptr, 0, hs, I, I, pa.tile_expert, pa.tile_rows, used_tm, pa.words + 1,
-                                  pa.words + 2, w8 + L.ws_a, s);
+                                  pa.words + 2, pa.status, w8 + L.ws_a, s);
     if (e != cudaSuccess) return e;
     const int64_t Gi = (I + kGroupK - 1) / kGroupK;
     const int64_t hquads = (int64_t)L.rows_max * Gi * 4;
@@ -560,9 +555,8 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
     if (e != cudaSuccess) return e;
     e = qlin_launch_chunk_grouped(fmt, dn, (int64_t)dn_stride, (int)qlin_mma_tiles(H, 0), H, I, L.rows_max, os, H,
                                   nullptr, 0, 0, pa.tile_expert, pa.tile_rows, used_tm, pa.words + 2, nullptr,
-                                  w8 + L.ws_b, s);
+                                  pa.status, w8 + L.ws_b, s);
     if (e != cudaSuccess) return e;
     return pf_launch_pdl(moe_prefill_combine_kernel, (unsigned)M, 256, s, pa, (const float*)os,
-                         (const __nv_bfloat16*)hs, I, y, h, (const unsigned*)(w8 + L.ws_a),
-                         (const unsigned*)(w8 + L.ws_b));
+                         (const __nv_bfloat16*)hs, I, y, h);
 }

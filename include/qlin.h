@@ -26,6 +26,10 @@
  *     bytes, 256-byte aligned, ZERO-FILLED before their first use.  Every call leaves the
  *     workspace's counters zero again when it completes, so a workspace can be reused by calls
  *     that run one after another on one stream; calls that overlap on the GPU must not share one.
+ *     Where the counters sit depends on the call's shapes for qlin_gemv, qlin_gemv_chain and
+ *     qlin_moe_experts: reuse their workspace only for calls with the same op and shapes (or zero
+ *     it again).  qlin_gemm_chunk and qlin_moe_prefill keep theirs at fixed places or clear them
+ *     themselves, so any later call may reuse their workspace.
  */
 #ifndef QLIN_H
 #define QLIN_H

@@ -195,6 +195,22 @@ def test_moe_prefill_deterministic_and_graph_capturable():
     assert q.qlin_ws_status(ws) == 0
 
 
+def test_moe_prefill_workspace_reused_across_shapes():
+    """One workspace (sized for the largest call) through calls of different M: each result equals
+    the same call on a fresh workspace, bit for bit, and the status stays clean."""
+    fmt, E, H, I, k = q.QLIN_NVFP4, 8, 256, 160, 2
+    ex = Experts(fmt, E, H, I, 7800)
+    ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, fmt, 300, H, I, E, k))
+    for M in (300, 17, 129, 300, 1):
+        x = synth.activations(M, H, synth.gen(7801 + M), dtype=torch.bfloat16).cuda()
+        logits = synth.router_logits(M, E, synth.gen(7901 + M)).cuda()
+        y = q.qlin_moe_prefill(fmt, ex.gu_p, ex.dn_p, E, H, I, k, x, router_logits=logits, ws=ws)[0]
+        ref = q.qlin_moe_prefill(fmt, ex.gu_p, ex.dn_p, E, H, I, k, x, router_logits=logits)[0]
+        torch.cuda.synchronize()
+        assert q.qlin_ws_status(ws) == 0
+        assert torch.equal(y, ref), M
+
+
 def test_moe_prefill_argument_checks():
     lib, P = q.lib(), q._dev
     x = torch.zeros(4, 256, dtype=torch.bfloat16, device="cuda")

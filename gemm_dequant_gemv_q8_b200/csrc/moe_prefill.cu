@@ -7,13 +7,14 @@
 // grouped GEMM" and its NVFP4 grouped GEMM for MoE prefill (imp README, "Features" table, row
 // "Architectures"; release notes v0.7.0), there on sm_120a.  Six launches on one stream, no host
 // synchronisation (the counts and the tile table live on the device, so the sequence can be
-// captured in a CUDA graph):
+// captured in a CUDA graph); every launch after the first is a programmatic dependent of the one
+// before it and reads that one's results only after griddepcontrol.wait:
 //   1. route (a warp per token): top_k (ties to the lower expert index, a NaN logit ranks as
 //      -inf), renormalised weights, max |x| folded into one word, and for each valid slot its
 //      index among the expert's entries (a shared-memory count per CTA, then one atomic per expert
-//      and CTA on the global count); the last CTA to
-//      finish turns the counts into each expert's first sorted row (rows padded to whole 128-row
-//      tiles) and the table row tile -> expert;
+//      and CTA on the global count); the last CTA to finish turns the counts into each expert's
+//      first sorted row (rows padded to whole 128-row tiles), the table row tile -> expert and
+//      each tile's count of rows holding entries;
 //   2. gather-quantize (a CTA per token): the token's row quantized once as the chunk path
 //      quantizes (NVFP4: one per-tensor scale from max |x| over the chunk; MXFP4: the OCP MX rule)
 //      and stored, in the tensor-core operand layout, at each of its sorted rows; extra CTAs zero
@@ -22,7 +23,7 @@
 //      weights, the SiLU-gate fused in the epilogue, h stored as bf16 (padding rows not stored) and
 //      max |h| folded into a word;
 //   4. h quantized the same way (NVFP4: its own per-tensor scale, from that word), a thread per
-//      16-value item;
+//      64 values of a row;
 //   5. grouped chunk GEMM, down: each tile against its expert's down weights, o (fp32) per sorted row
 //      (padding rows not stored);
 //   6. combine: y[m] = sum over slots, in slot order, of weight * o[row of (m, slot)] (deterministic),

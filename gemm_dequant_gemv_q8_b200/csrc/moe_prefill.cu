@@ -128,6 +128,14 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
     int my_e = -1, my_li = 0;  // lane r < top_k: slot r's expert and its index among this CTA's
     float mx = 0.f;
     if (m < a.M) {
+        // the token's logits (lane l holds experts l, l + 32, ...), in flight with the x loads below
+        float v[kPfMaxE / 32];
+        const float* l = a.logits ? a.logits + (int64_t)m * a.E : nullptr;
+#pragma unroll
+        for (int j = 0; j < kPfMaxE / 32; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = (l && e < a.E) ? l[e] : -INFINITY;
+        }
         // max |x| of the token (fmaxf skips a NaN, as the chunk quantizer's max pass does)
         const uint4* xr = reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.H);
 #pragma unroll 8
@@ -144,15 +152,8 @@ __global__ void __launch_bounds__(kPfRouteWarps * 32) moe_prefill_route_kernel(c
         int sel[kPfMaxTopK];
 #pragma unroll
         for (int r = 0; r < kPfMaxTopK; ++r) sel[r] = -1;
-        if (a.logits) {
-            // top_k rounds of a warp-wide argmax under pf_before; lane l holds experts l, l + 32, ...
-            const float* l = a.logits + (int64_t)m * a.E;
-            float v[kPfMaxE / 32];
-#pragma unroll
-            for (int j = 0; j < kPfMaxE / 32; ++j) {
-                const int e = lane + 32 * j;
-                v[j] = e < a.E ? l[e] : -INFINITY;
-            }
+        if (l) {
+            // top_k rounds of a warp-wide argmax under pf_before
             unsigned taken = 0u;
             float selv[kPfMaxTopK];  // the selected logits (as given)
 #pragma unroll

@@ -213,6 +213,7 @@ def test_moe_deterministic_and_graph_capturable():
     ref = q.qlin_moe_experts(fmt, ex.gu_p, ex.dn_p, E, H, I, k, x, router_logits=logits, ws=ws)[0].clone()
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())  # calls sharing a workspace must not overlap
     with torch.cuda.stream(s):
         q.qlin_moe_experts(fmt, ex.gu_p, ex.dn_p, E, H, I, k, x, router_logits=logits, topk_ids=ids, topk_w=w,
                            y=y, ws=ws, flags=q.QLIN_FLAG_PDL)

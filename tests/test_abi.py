@@ -156,3 +156,42 @@ def test_moe_rejects_oversized_hidden_before_launch(lib):
                               P(0x400000), P(0x500000), P(0x600000), 1, 1, P(0x700000), None, 0,
                               P(0x800000), 1 << 30, None)
     assert st == 2  # QLIN_ERR_UNSUPPORTED: down tiles per expert are tracked for H <= 32768
+
+
+def test_moe_prefill_argument_checks_return_before_launch(lib):
+    """Every bad argument of qlin_moe_prefill is reported before anything is enqueued (the device
+    pointers below are never dereferenced: the checks run on the host)."""
+    P = ctypes.c_void_p
+    N4, MX = q.QLIN_NVFP4, q.QLIN_MXFP4
+    ok = dict(fmt=N4, gu=P(0x100000), dn=P(0x200000), E=32, H=2048, I=1792, k=4, logits=P(0x300000),
+              ids=P(0x400000), w=P(0x500000), x=P(0x600000), M=64, y=P(0x700000), h=None, flags=0,
+              ws=P(0x800000), wsb=1 << 34)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.qlin_moe_prefill(a["fmt"], a["gu"], a["dn"], a["E"], a["H"], a["I"], a["k"], a["logits"], a["ids"],
+                                    a["w"], a["x"], a["M"], a["y"], a["h"], a["flags"], a["ws"], a["wsb"], None)
+
+    assert call(fmt=q.QLIN_Q4_0) == 2       # GGUF experts: not on this path
+    assert call(fmt=q.QLIN_Q8_0) == 2
+    assert call(fmt=99) == 1                # unknown format
+    assert call(E=0) == 1 and call(E=257) == 1
+    assert call(k=0) == 1 and call(k=9) == 1 and call(E=2, k=3) == 1
+    assert call(H=2047) == 1 and call(I=1800) == 1 and call(H=16) == 1
+    assert call(M=0) == 1
+    assert call(flags=1) == 1
+    assert call(gu=None) == 1 and call(y=None) == 1 and call(ids=None) == 1
+    assert call(x=P(0x600008)) == 3         # x not 16-byte aligned
+    assert call(gu=P(0x100010)) == 3        # packed buffers 256-byte aligned
+    assert call(wsb=16) == 4 and call(ws=None) == 4
+    assert call(fmt=MX, wsb=16) == 4
+
+
+def test_moe_prefill_workspace_bytes(lib):
+    N4 = q.QLIN_NVFP4
+    assert q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, q.QLIN_Q4_0, 64, 2048, 1792, 32, 4) == 0
+    assert q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, N4, 64, 2048, 1800, 32, 4) == 0
+    sizes = [q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, N4, M, 2048, 1792, 32, 4) for M in (1, 64, 512, 4096)]
+    assert all(s > 0 for s in sizes) and sizes == sorted(sizes)
+    # the same for MXFP4 experts (the operand units keep the NVFP4 size)
+    assert q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, q.QLIN_MXFP4, 512, 2048, 1792, 32, 4) == sizes[2]

@@ -887,7 +887,7 @@ def small_case(name, reps=3):
     profiles under profiles/ name these commands): moe1 / moe8 = one Q4_0 MoE layer of the 8B-A1B
     shape at M = 1 / 8; moepf512 = one NVFP4 MoE prefill layer of that shape at M = 512 (five
     launches per call); mlp1 / mlp4 = one NVFP4 27B-shaped MLP as a two-op GEMV chain (h in bf16)
-    at M = 1 / 4."""
+    at M = 1 / 4; chunk512 = the NVFP4 prefill-chunk GEMM (K 5120, N 17408) at M = 512."""
     import gemm_dequant_gemv_q8_b200 as q
     torch.cuda.set_device(0)
     if name.startswith("moe") and not name.startswith("moepf"):
@@ -903,6 +903,16 @@ def small_case(name, reps=3):
         ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_MOE, fmt, M, H, I, E, k))
         for _ in range(reps):
             q.qlin_moe_experts(fmt, gu, dn, E, H, I, k, x, router_logits=logits, ws=ws)
+    elif name == "chunk512":
+        fmt, N, K, M = q.QLIN_NVFP4, 17408, 5120, 512
+        b, s_, g = synth.weights(fmt, N, K, synth.gen(7000, device="cuda"), device="cuda")
+        pk = q.qlin_pack_weights(fmt, N, K, b, s_, g, q.QLIN_PACK_MMA)
+        del b, s_
+        x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
+        y = torch.empty(M, N, device="cuda")
+        ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
+        for _ in range(reps):
+            q.qlin_gemm_chunk(fmt, pk, N, K, x, y=y, ws=ws)
     elif name.startswith("moepf"):
         M = int(name[5:])
         fmt, E, H, I, k = q.QLIN_NVFP4, 32, 2048, 1792, 4
@@ -1009,7 +1019,7 @@ def main():
                              "q6_k_stack", "gguf_chunk"],
                     help="stack (default): the Q4_0 36-layer decode stack line; the others print their "
                          "entries alone")
-    ap.add_argument("--small-case", choices=["moe1", "moe8", "mlp1", "mlp4", "moepf512"],
+    ap.add_argument("--small-case", choices=["moe1", "moe8", "mlp1", "mlp4", "moepf512", "chunk512"],
                     help="three launches of one layer's kernel (for ncu captures); prints no bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

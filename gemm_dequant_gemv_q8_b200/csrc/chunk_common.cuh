@@ -128,6 +128,19 @@ __device__ __forceinline__ float div_by_recip(float x, float d, float y) {
     return copysignf(__fmaf_rn(r1, y, q1), x);
 }
 
+// Two quotients at once: the same steps on a pair of values with the packed fp32 operations, each
+// lane rounded as the scalar operation rounds it (so the results are div_by_recip's, bit for bit);
+// -q * d + x is taken as fma(q, -d, x), the same value.
+__device__ __forceinline__ float2 div_by_recip2(float2 x, float d, float y) {
+    const float2 yy = make_float2(y, y), nd = make_float2(-d, -d);
+    const float2 q0 = __fmul2_rn(x, yy);
+    const float2 r0 = __ffma2_rn(q0, nd, x);
+    const float2 q1 = __ffma2_rn(r0, yy, q0);
+    const float2 r1 = __ffma2_rn(q1, nd, x);
+    const float2 q = __ffma2_rn(r1, yy, q1);
+    return make_float2(copysignf(q.x, x.x), copysignf(q.y, x.y));
+}
+
 // Scale byte and 8 code bytes (element 2j in the low nibble of byte j) of one 16-value block.
 __device__ __forceinline__ uint8_t act_quant_block(const uint32_t (&w)[8], float bmax, float ag, uint32_t (&c8)[2]) {
     c8[0] = c8[1] = 0u;
@@ -142,10 +155,11 @@ __device__ __forceinline__ uint8_t act_quant_block(const uint32_t (&w)[8], float
         if (special == 0u && div >= 0x1p-96f && div <= 0x1p100f) {
             const float y = __frcp_rn(div);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                c8[j >> 2] |= e2m1x2_rne_sat(div_by_recip(__uint_as_float(w[j] << 16), div, y),
-                                             div_by_recip(__uint_as_float(w[j] & 0xffff0000u), div, y))
-                              << (8 * (j & 3));
+            for (int j = 0; j < 8; ++j) {
+                const float2 qv =
+                    div_by_recip2(make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u)), div, y);
+                c8[j >> 2] |= e2m1x2_rne_sat(qv.x, qv.y) << (8 * (j & 3));
+            }
         } else {
 #pragma unroll
             for (int j = 0; j < 8; ++j)

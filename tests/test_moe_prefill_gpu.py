@@ -196,6 +196,18 @@ def test_moe_prefill_deterministic_and_graph_capturable():
     assert q.qlin_ws_status(ws) == 0
 
 
+def test_moe_prefill_tied_logits():
+    """Equal logits go to the lower expert index: the routing equals the oracle's on rows built
+    with ties, and the layer matches as in the other tests."""
+    fmt, E, H, I, M, k = q.QLIN_NVFP4, 8, 128, 96, 6, 3
+    ex = Experts(fmt, E, H, I, 7950)
+    logits = synth.router_logits(M, E, synth.gen(7951)).clone()
+    logits[1, :] = 0.25                       # all tied: experts 0, 1, 2
+    logits[2, [1, 5, 6]] = 8.0                # a three-way tie at the top
+    logits[4, [0, 3]] = -8.0                  # a tie at the bottom, never selected
+    run_and_check(ex, M, k, 7952, logits=logits)
+
+
 def test_moe_prefill_workspace_reused_across_shapes():
     """One workspace (sized for the largest call) through calls of different M: each result equals
     the same call on a fresh workspace, bit for bit, and the status stays clean."""

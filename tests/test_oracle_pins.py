@@ -641,3 +641,47 @@ def test_act_quant_mx_grid_round_trip_and_special_blocks():
     I[0, 7] = np.inf
     ic, isc = oracle.act_quant_mx(I)
     assert isc[0, 0] == 0xFF and not ic.any()
+
+
+# ----------------------------------------------------------------------------- same-quant products
+def _fp4_value(codes, r, j):
+    c = (int(codes[r, j // 2]) >> (4 * (j & 1))) & 0xF
+    return -E2M1_MAG[c & 7] if c & 8 else E2M1_MAG[c & 7]
+
+
+def _e4m3_fraction(b):
+    return Fraction(torch.tensor([b], dtype=torch.uint8).view(torch.float8_e4m3fn).double().item())
+
+
+@pytest.mark.parametrize("mx", [False, True])
+def test_gemm_same_quant_is_the_exact_product_of_the_decoded_operands(mx):
+    """y[m][n] = sum_k a[m][k] w[n][k], both operands decoded here from their codes by the format
+    definitions (E2M1 table, E4M3 through torch's float8, UE8M0 as a power of two), in exact
+    arithmetic.  M, N and K differ, so a transposed operand, a scale applied to the wrong row or a
+    block index off by one fails."""
+    M, N, K = 3, 5, 96
+    rng = np.random.default_rng(21 + mx)
+    bs = 32 if mx else 16
+    a_codes = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    w_codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    if mx:
+        a_sc = rng.integers(118, 136, (M, K // bs), dtype=np.uint8)
+        w_sc = rng.integers(118, 136, (N, K // bs), dtype=np.uint8)
+        y, A = oracle.gemm_same_quant_mx(w_codes, w_sc, a_codes, a_sc, N, K)
+        scale = lambda b: Fraction(2) ** (int(b) - 127)
+        a_g = w_g = Fraction(1)
+    else:
+        a_sc = rng.integers(0x08, 0x7F, (M, K // bs), dtype=np.uint8)   # finite E4M3, no NaN
+        w_sc = rng.integers(0x08, 0x7F, (N, K // bs), dtype=np.uint8)
+        ag, wg = float(np.float32(1 / 448)), float(np.float32(3 / 1000))
+        y, A = oracle.gemm_same_quant(w_codes, w_sc, wg, a_codes, a_sc, ag, N, K)
+        scale = _e4m3_fraction
+        a_g, w_g = Fraction(ag), Fraction(wg)
+    assert y.shape == (M, N) and A.shape == (M, N)
+    for m in range(M):
+        for n in range(N):
+            terms = [_fp4_value(a_codes, m, k) * scale(a_sc[m, k // bs]) * a_g *
+                     _fp4_value(w_codes, n, k) * scale(w_sc[n, k // bs]) * w_g for k in range(K)]
+            exact, absum = sum(terms), sum(abs(t) for t in terms)
+            assert abs(Fraction(float(y[m, n])) - exact) <= Fraction(K * 2.0 ** -52) * absum, (m, n)
+            assert abs(Fraction(float(A[m, n])) - absum) <= Fraction(K * 2.0 ** -52) * absum, (m, n)

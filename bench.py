@@ -524,11 +524,41 @@ def roofline_hbm(kernel, bytes_per_launch, us_per_launch, traffic=None):
             "algorithmic_bytes_per_launch": bytes_per_launch, "avg_launch_us": us_per_launch}
 
 
+_PROBE = {}
+
+
+def fp4_mma_probe(iters=8192):
+    """The FP4 tensor path's MMA-only rate on this device, measured once per process outside every
+    timed region: qlin_probe_fp4_mma (one CTA per SM, `iters` back-to-back M128 N256 K64
+    mxf4nvf4 MMAs on fixed shared-memory operands), two warm-up launches, then one launch timed
+    with CUDA events."""
+    if not _PROBE:
+        import gemm_dequant_gemv_q8_b200 as q
+        cycles = torch.zeros(1024, dtype=torch.int64, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for _ in range(2):
+            q.qlin_probe_fp4_mma(iters, cycles, status)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        ctas = q.qlin_probe_fp4_mma(iters, cycles, status)
+        b.record()
+        b.synchronize()
+        ms = a.elapsed_time(b)
+        _PROBE.update(tflops=2.0 * 128 * 256 * 64 * iters * ctas / (ms * 1e-3) / 1e12,
+                      cycles_per_mma=float(cycles[:ctas].max()) / iters, ctas=ctas, iters=iters,
+                      status=int(status.item()))
+    return _PROBE
+
+
 def roofline_fp4(kernel, flop_per_launch, us_per_launch):
     peak, src, spec = fp4_peaks()
     tf = flop_per_launch / (us_per_launch * 1e-6) / 1e12
+    pr = fp4_mma_probe()
     return {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peak, "peak_source": src,
             "unit": "TFLOP/s", "frac": tf / peak, "traffic": None, "spec_peak": spec, "frac_of_spec": tf / spec,
+            "probe_peak": pr["tflops"], "frac_of_probe": tf / pr["tflops"],
+            "probe": {"what": "qlin_probe_fp4_mma: M128 N256 K64 mxf4nvf4 MMAs back to back, one CTA per SM, "
+                              "fixed shared-memory operands", **pr},
             "algorithmic_flop_per_launch": flop_per_launch, "avg_launch_us": us_per_launch}
 
 

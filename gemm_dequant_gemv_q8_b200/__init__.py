@@ -51,6 +51,7 @@ SIGNATURES = {
     "qlin_gemv_chain": (_I, [_I, _I, _I, _P, _I, _I, _P, _SZ, _P]),
     "qlin_ws_status": (_I, [_P, _P]),
     "qlin_ws_set_wait_budget": (_I, [_P, ctypes.c_uint32, _P]),
+    "qlin_probe_fp4_mma": (_I, [_I, _P, _I, _P, ctypes.POINTER(_I), _P]),
     "qlin_status_string": (ctypes.c_char_p, [_I]),
 }
 
@@ -285,6 +286,20 @@ def qlin_ws_status(ws, stream=None):
 def qlin_ws_set_wait_budget(ws, ns, stream=None):
     """Budget (ns) of the bounded inter-CTA waits of calls using ws; 0 = the default (~2 s)."""
     _check("qlin_ws_set_wait_budget", lib().qlin_ws_set_wait_budget(_dev(ws, "ws"), int(ns), _stream(stream)))
+
+
+def qlin_probe_fp4_mma(iters, cycles, status, stream=None):
+    """Launch the MMA-only FP4 rate probe: `iters` M128 N256 K64 mxf4nvf4 MMAs per SM.  cycles:
+    an int64 CUDA tensor with one entry per possible CTA (its length is max_ctas); status: an
+    int32 CUDA word that bit 0 is or-ed into if a wait gave up.  Returns the number of CTAs
+    launched.  The caller times the launch."""
+    if cycles.dtype != torch.int64 or status.dtype != torch.int32:
+        raise TypeError("cycles must be int64 and status int32")
+    ctas = _I(0)
+    _check("qlin_probe_fp4_mma", lib().qlin_probe_fp4_mma(int(iters), _dev(cycles, "cycles"), cycles.numel(),
+                                                          _dev(status, "status"), ctypes.byref(ctas),
+                                                          _stream(stream)))
+    return ctas.value
 
 
 def qlin_status_string(status):

@@ -36,6 +36,8 @@ extern "C" cudaError_t qlin_launch_moe_prefill(int fmt, const void* gu, const vo
                                                const void* x, int M, float* y, float* h, void* ws, size_t gu_stride,
                                                size_t dn_stride, cudaStream_t s);
 
+extern "C" cudaError_t qlin_launch_fp4_mma_rate(int iters, unsigned long long* cycles, int max_ctas,
+                                                unsigned* status, int* ctas, cudaStream_t s);
 extern "C" int qlin_chain_max_ops();
 extern "C" size_t qlin_chain_ws_bytes(int fmt, int M, const qlin_gemv_op* ops, int n_ops);
 extern "C" cudaError_t qlin_launch_chain(int fmt, int xdt, int M, const qlin_gemv_op* ops, int n_ops, int flags,
@@ -312,6 +314,16 @@ qlin_status_t qlin_ws_set_wait_budget(void* ws, uint32_t ns, qlin_stream_t strea
     cudaError_t e = cudaMemcpyAsync((uint8_t*)ws + qlin::kWsWaitBudgetOff, &ns, sizeof(ns), cudaMemcpyHostToDevice,
                                     (cudaStream_t)stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);  // ns lives on this stack
+    return cuda_status(e);
+}
+
+qlin_status_t qlin_probe_fp4_mma(int iters, unsigned long long* cycles, int max_ctas, unsigned int* status,
+                                 int* ctas, qlin_stream_t stream) {
+    if (iters < 1 || iters > (1 << 20) || max_ctas < 1 || !cycles || !status || !ctas) return QLIN_ERR_INVALID_ARG;
+    if (!aligned(cycles, 8) || !aligned(status, 4)) return QLIN_ERR_ALIGNMENT;
+    *ctas = 0;
+    const cudaError_t e = qlin_launch_fp4_mma_rate(iters, cycles, max_ctas, status, ctas, (cudaStream_t)stream);
+    if (e == cudaErrorInvalidValue && *ctas > max_ctas) return QLIN_ERR_INVALID_ARG;  // nothing launched
     return cuda_status(e);
 }
 

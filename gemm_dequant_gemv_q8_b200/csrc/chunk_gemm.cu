@@ -1192,3 +1192,86 @@ extern "C" cudaError_t qlin_launch_chunk_grouped(int fmt, const void* w, int64_t
     return fmt == QLIN_MXFP4 ? launch_chunk_cg<1, true, true>(a, QLIN_FLAG_PDL, s)
                              : launch_chunk_cg<1, false, true>(a, QLIN_FLAG_PDL, s);
 }
+
+// ---------------------------------------------------------------------------------------------
+// MMA-only rate of the FP4 tensor path on this device (a measurement aid, not on the hot path).
+// One CTA per SM; one thread issues `iters` back-to-back kind::mxf4nvf4 block16 MMAs of M 128,
+// N 256, K 64 into one TMEM accumulator. These use the chunk GEMM's own instruction, shared-memory
+// descriptors and instruction word, on fixed operands: arbitrary E2M1 bytes (every 4-bit pattern
+// is a finite value) and E4M3 1.0 in every scale factor. No operand moves while the MMAs run, so
+// the rate is the tensor pipe's own. Each CTA records its clock64 span from the first issue to the
+// commit's arrival; the caller times the launch with events.
+constexpr int kProbeABytes = kMmaARows * 128;  // 128 rows x 256 E2M1 values: four K = 64 steps
+constexpr int kProbeBBytes = kMmaWRows * 128;  // 256 rows x 256 values
+constexpr int kProbePad = 128 * 1024;          // keeps one CTA, and one TMEM allocation, per SM
+constexpr int kProbeSmem = 1024 + kProbeABytes + kProbeBBytes + 64 + kProbePad;
+static_assert(kProbeSmem <= 232448 && 2 * kProbeSmem > 233472, "one probe CTA per SM");
+
+__global__ void __launch_bounds__(128, 1) fp4_mma_rate_kernel(int iters, unsigned long long* cycles,
+                                                              unsigned* status) {
+    extern __shared__ uint8_t probe_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)probe_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* bar = (uint64_t*)(sm + kProbeABytes + kProbeBBytes);
+    uint32_t* holder = (uint32_t*)(bar + 1);
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < (kProbeABytes + kProbeBBytes) / 4; i += blockDim.x) {
+        uint32_t v = (uint32_t)i * 2654435761u ^ (blockIdx.x * 40503u);
+        v ^= v >> 15;
+        v *= 0x2c1b3c6du;
+        v ^= v >> 12;
+        ((uint32_t*)sm)[i] = v;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    fence_proxy_async_smem();  // the operands were written through the generic proxy
+    if (warp == 0) tmem_alloc<1>(holder);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *holder;
+    {  // scale-factor columns kAccCols .. kAccCols + 15 of this warp's lane quarter: E4M3 1.0
+        uint32_t r[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) r[j] = 0x38383838u;
+        tc_st16<0, 16>(tmem + ((uint32_t)(warp * 32) << 16) + kAccCols, r);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+        const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(kMmaWRows >> 3) << 17) |
+                               ((uint32_t)(kMmaARows >> 4) << 24);
+        const uint32_t sa = smem_u32(sm), sb = sa + kProbeABytes, sf = tmem + kAccCols;
+        const unsigned long long t0 = clock64();
+        for (int i = 0; i < iters; ++i) {
+            const uint32_t kb = (uint32_t)(i & 3) * 32;  // the K = 64 step inside the 128-byte swizzle row
+            tc_mma(tmem, sdesc_sw128(sa + kb), sdesc_sw128(sb + kb), idesc, sf, sf + 4, i > 0 ? 1u : 0u);
+        }
+        tc_commit(bar);
+        if (!mbar_wait_bounded(bar, 0)) atomicOr(status, 1u);
+        cycles[blockIdx.x] = clock64() - t0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_free<1>(tmem);
+    }
+}
+
+extern "C" cudaError_t qlin_launch_fp4_mma_rate(int iters, unsigned long long* cycles, int max_ctas,
+                                                unsigned* status, int* ctas, cudaStream_t s) {
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    *ctas = sms;
+    if (sms > max_ctas) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(fp4_mma_rate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);
+    if (e != cudaSuccess) return e;
+    fp4_mma_rate_kernel<<<sms, 128, kProbeSmem, s>>>(iters, cycles, status);
+    return cudaGetLastError();
+}

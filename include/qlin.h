@@ -398,6 +398,24 @@ qlin_status_t qlin_ws_status(void* ws, qlin_stream_t stream);
  * have no counterpart (the Imparo README, "Why Imparo", reports failures rather than hiding them). */
 qlin_status_t qlin_ws_set_wait_budget(void* ws, uint32_t ns, qlin_stream_t stream);
 
+/* Measurement aid, not on the hot path: the MMA-only rate of the FP4 tensor path on this device,
+ * the denominator beside the 9 PFLOP/s dense FP4 figure of the datacenter part (imp README, "Why
+ * this exists": tcgen05 and TMEM are the datacenter path). Launches one CTA per SM on `stream`.
+ * One thread of each CTA issues `iters` (1 .. 2^20) dependent tcgen05.mma kind::mxf4nvf4
+ * block16 MMAs of M 128, N 256, K 64 (4,194,304 flops each). They use the instruction,
+ * descriptors and instruction word of qlin_gemm_chunk's NVFP4 path, on fixed shared-memory
+ * operands into one TMEM accumulator; the operands hold arbitrary E2M1 codes and E4M3 1.0 scales,
+ * and nothing is written back.
+ * cycles: device array of max_ctas uint64 (8-byte aligned). CTA i writes its clock64 span from
+ *   the first issue to the MMAs' completion into cycles[i].
+ * status: a device uint32 word; bit 0 is or-ed in if a CTA's bounded wait for its MMAs gave up
+ *   (after about 2 s).
+ * *ctas (host) receives the number of CTAs, the SM count. If that exceeds max_ctas, the call
+ *   returns QLIN_ERR_INVALID_ARG and launches nothing.
+ * The caller times the launch (CUDA events on `stream`): flops = 4,194,304 * iters * *ctas. */
+qlin_status_t qlin_probe_fp4_mma(int iters, unsigned long long* cycles, int max_ctas, unsigned int* status,
+                                 int* ctas, qlin_stream_t stream);
+
 const char* qlin_status_string(qlin_status_t status);
 
 #ifdef __cplusplus

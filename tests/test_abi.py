@@ -208,3 +208,17 @@ def test_moe_prefill_workspace_bytes(lib):
     assert all(s > 0 for s in sizes) and sizes == sorted(sizes)
     # the same for MXFP4 experts (the operand units keep the NVFP4 size)
     assert q.qlin_workspace_bytes(q.QLIN_OP_MOE_PREFILL, q.QLIN_MXFP4, 512, 2048, 1792, 32, 4) == sizes[2]
+
+
+@made_up_addresses
+def test_probe_fp4_mma_argument_checks(lib):
+    P = ctypes.c_void_p
+    ctas = ctypes.c_int(-1)
+
+    def call(iters=64, cycles=0x100000, max_ctas=1024, status=0x200000):
+        return lib.qlin_probe_fp4_mma(iters, P(cycles), max_ctas, P(status), ctypes.byref(ctas), None)
+
+    assert call(iters=0) == 1 and call(iters=(1 << 20) + 1) == 1
+    assert call(max_ctas=0) == 1
+    assert call(cycles=0) == 1 and call(status=0) == 1
+    assert call(cycles=0x100004) == 3 and call(status=0x200002) == 3

@@ -226,7 +226,10 @@ def pack_experts(fmt, E, N, K, canon, pack_flags=QLIN_PACK_DEFAULT, stream=None)
 
 
 def qlin_gemm_chunk(fmt, packed, N, K, x, y=None, flags=0, ws=None, stream=None):
-    """NVFP4 prefill-chunk GEMM: y (M, N) fp32 = quantized x (M, K) bf16 times W^T."""
+    """Prefill-chunk GEMM: y (M, N) fp32 = x (M, K) bf16 times W^T.  NVFP4 / MXFP4 weights packed
+    with QLIN_PACK_MMA: x quantized in the same launch.  GGUF weights packed with QLIN_PACK_MMA,
+    or any format packed with QLIN_PACK_MMA_BF16 and called with QLIN_FLAG_BF16_COPY: bf16 x
+    times the bf16 copy of the weights."""
     if x.dtype != torch.bfloat16 or x.stride(1) != 1:
         raise TypeError("x must be bfloat16 with contiguous rows")
     M = x.shape[0]

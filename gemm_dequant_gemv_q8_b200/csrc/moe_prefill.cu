@@ -101,7 +101,7 @@ struct PfArgs {
     int* lpos;            // M x top_k: index of (token, slot) among its expert's entries, -1 skipped
     int* pos;             // M x top_k: sorted row of (token, slot), -1 for a skipped slot
     int* cnt;             // E: entries per expert (counted in step 1, cleared by its last CTA)
-    int* fill;            // E: the counts, kept for steps 2 and 5
+    int* fill;            // E: the counts, kept for step 2 (an expert's padding rows start at off + fill)
     int* off;             // E + 1: first sorted row of each expert
     unsigned* words;      // [0] ticket, [1] max |x|, [2] max |h|, [3] row tiles in use
     int* tile_expert;     // TMx

@@ -553,10 +553,14 @@ def fp4_mma_probe(iters=8192):
 def roofline_fp4(kernel, flop_per_launch, us_per_launch):
     peak, src, spec = fp4_peaks()
     tf = flop_per_launch / (us_per_launch * 1e-6) / 1e12
-    pr = fp4_mma_probe()
+    try:
+        pr = fp4_mma_probe()
+    except Exception as e:  # the roofline line stands without the probe
+        pr = {"error": f"{type(e).__name__}: {e}"}
+    ok = pr.get("status") == 0 and bool(pr.get("tflops"))
     return {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peak, "peak_source": src,
             "unit": "TFLOP/s", "frac": tf / peak, "traffic": None, "spec_peak": spec, "frac_of_spec": tf / spec,
-            "probe_peak": pr["tflops"], "frac_of_probe": tf / pr["tflops"],
+            "probe_peak": pr["tflops"] if ok else None, "frac_of_probe": tf / pr["tflops"] if ok else None,
             "probe": {"what": "qlin_probe_fp4_mma: M128 N256 K64 mxf4nvf4 MMAs back to back, one CTA per SM, "
                               "fixed shared-memory operands", **pr},
             "algorithmic_flop_per_launch": flop_per_launch, "avg_launch_us": us_per_launch}

@@ -106,3 +106,20 @@ def test_sources_sha_depends_on_every_listed_file():
 def test_cpu_info_reports_usable_cores():
     model, n = bench.cpu_info()
     assert n >= 1 and (model is None or isinstance(model, str))
+
+
+def test_fp4_roofline_carries_the_probe_or_nulls(monkeypatch):
+    monkeypatch.setattr(bench, "fp4_peaks", lambda: (6500.0, "test", 9000.0))
+    monkeypatch.setattr(bench, "fp4_mma_probe", lambda: {"tflops": 8000.0, "status": 0})
+    r = bench.roofline_fp4("k", 2e12, 1000.0)  # 2 TFLOP in 1 ms
+    assert r["achieved"] == pytest.approx(2000.0) and r["frac"] == pytest.approx(2000 / 6500)
+    assert r["probe_peak"] == 8000.0 and r["frac_of_probe"] == pytest.approx(0.25)
+    monkeypatch.setattr(bench, "fp4_mma_probe", lambda: {"tflops": 8000.0, "status": 1})  # a wait gave up
+    r = bench.roofline_fp4("k", 2e12, 1000.0)
+    assert r["probe_peak"] is None and r["frac_of_probe"] is None and r["frac"] == pytest.approx(2000 / 6500)
+
+    def boom():
+        raise RuntimeError("no device")
+    monkeypatch.setattr(bench, "fp4_mma_probe", boom)
+    r = bench.roofline_fp4("k", 2e12, 1000.0)
+    assert r["probe_peak"] is None and "no device" in r["probe"]["error"]

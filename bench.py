@@ -516,11 +516,15 @@ def timed(fn, steps, warmup, min_s=0.3):
     return total_ms / n, clk.summary()
 
 
+HBM_SPEC_GBS = 8000.0  # B200 HBM3e, NVIDIA's 8 TB/s figure (printed beside the measured copy peak)
+
+
 def roofline_hbm(kernel, bytes_per_launch, us_per_launch, traffic=None):
     peak, src = peaks()
     gbs = bytes_per_launch / (us_per_launch * 1e-6) / 1e9
     return {"bound": "hbm", "kernel": kernel, "achieved": gbs, "peak": peak, "peak_source": f"{src} hbm_gbs (copy)",
-            "unit": "GB/s", "frac": gbs / peak, "traffic": traffic,
+            "unit": "GB/s", "frac": gbs / peak, "traffic": traffic, "spec_peak": HBM_SPEC_GBS,
+            "frac_of_spec": gbs / HBM_SPEC_GBS,
             "algorithmic_bytes_per_launch": bytes_per_launch, "avg_launch_us": us_per_launch}
 
 

@@ -123,3 +123,11 @@ def test_fp4_roofline_carries_the_probe_or_nulls(monkeypatch):
     monkeypatch.setattr(bench, "fp4_mma_probe", boom)
     r = bench.roofline_fp4("k", 2e12, 1000.0)
     assert r["probe_peak"] is None and "no device" in r["probe"]["error"]
+
+
+def test_hbm_roofline_prints_the_measured_and_the_spec_peak(monkeypatch):
+    monkeypatch.setattr(bench, "peaks", lambda: (6558.1, "measured"))
+    r = bench.roofline_hbm("k", 6.5581e9, 1000.0, traffic=123)  # 6.5581 GB in 1 ms
+    assert r["achieved"] == pytest.approx(6558.1) and r["frac"] == pytest.approx(1.0)
+    assert r["spec_peak"] == 8000.0 and r["frac_of_spec"] == pytest.approx(6558.1 / 8000.0)
+    assert r["traffic"] == 123 and r["bound"] == "hbm" and r["unit"] == "GB/s"

@@ -768,14 +768,17 @@ def cfg_moe_prefill(args, cpu=True):
     return out
 
 
+FP4_COPIES = 6  # packed FP4 copies of the K = 5120, N = 17408 matrix rotated by the chunk configs
+
+
 def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
     """NVFP4 prefill-chunk GEMM, K = 5120, N = 17408: M = 512 (tensor-bound) and 64 (HBM-bound),
-    and an M sweep on the same matrix; two weight copies alternate so that consecutive calls do not
-    find the weights in L2."""
+    and an M sweep on the same matrix.  FP4_COPIES copies of the 50 MB packed matrix rotate, so one
+    graph replay streams 300 MB, more than twice the 126 MB L2: no call finds its weights there."""
     import gemm_dequant_gemv_q8_b200 as q
     fmt, N, K = q.QLIN_NVFP4, 17408, 5120
     packs = []
-    for c in range(2):
+    for c in range(FP4_COPIES):
         b, s_, g = synth.weights(fmt, N, K, synth.gen(7000 + c, device="cuda"), device="cuda")
         packs.append(q.qlin_pack_weights(fmt, N, K, b, s_, g, q.QLIN_PACK_MMA))
         del b, s_
@@ -785,16 +788,18 @@ def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
         x = synth.activations(M, K, synth.gen(7100 + M, device="cuda"), dtype=torch.bfloat16, device="cuda")
         y = torch.empty(M, N, device="cuda")
         ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, fmt, M, N, K))
-        fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL) for c in range(2)]
+        fn = lambda: [q.qlin_gemm_chunk(fmt, packs[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL)
+                      for c in range(FP4_COPIES)]
         ms, clk = timed(fn, args.steps, args.warmup)
-        us = ms / 2 * 1e3
+        us = ms / FP4_COPIES * 1e3
         flop = 2.0 * M * N * K
         bytes_ = wbytes + 2 * M * K + 4 * M * N
         tf, gbs = flop / (us * 1e-6) / 1e12, bytes_ / (us * 1e-6) / 1e9
         if M in (512, 64):
             kern = f"chunk_gemm_kernel<1> (activation quantization + tcgen05 mxf4nvf4 GEMM), M={M}"
             e = {"workload": f"NVFP4 prefill-chunk GEMM M={M} K=5120 N=17408, bf16 x, fp32 accumulate; one persistent "
-                             "launch; two weight copies alternate", "M": M, "us_per_call": us,
+                             f"launch; {FP4_COPIES} weight copies rotate (300 MB per replay, above twice L2)",
+                 "M": M, "us_per_call": us,
                  "tflops": tf, "gbs": gbs, "clocks": clk}
             if M == 512:
                 e.update(value=tf, unit="TFLOP/s", roofline=roofline_fp4(kern, flop, us))
@@ -814,7 +819,7 @@ def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
     # MXFP4 weights of the same shape on their own chunk path (MX-quantized activations, kind::mxf4).
     del packs
     mpacks = []
-    for c in range(2):
+    for c in range(FP4_COPIES):
         b, s_, _ = synth.weights(q.QLIN_MXFP4, N, K, synth.gen(7300 + c, device="cuda"), device="cuda")
         mpacks.append(q.qlin_pack_weights(q.QLIN_MXFP4, N, K, b, s_, 1.0, q.QLIN_PACK_MMA))
         del b, s_
@@ -824,8 +829,8 @@ def cfg_chunk(args, cpu=True, sweep=(1, 2, 4, 8, 16)):
         y = torch.empty(M, N, device="cuda")
         ws = q.workspace(q.qlin_workspace_bytes(q.QLIN_OP_CHUNK, q.QLIN_MXFP4, M, N, K))
         fn = lambda: [q.qlin_gemm_chunk(q.QLIN_MXFP4, mpacks[c], N, K, x, y=y, ws=ws, flags=q.QLIN_FLAG_PDL)
-                      for c in range(2)]
-        ms = _time_graph_of(fn, args.steps, args.warmup) / 2
+                      for c in range(FP4_COPIES)]
+        ms = _time_graph_of(fn, args.steps, args.warmup) / FP4_COPIES
         us = ms * 1e3
         tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
         mx[str(M)] = {"us_per_call": us, "tflops": tf, "fp4_frac": tf / fp4_peaks()[0],
